@@ -1,0 +1,176 @@
+"""Decoder forward, denoise step, causal encode and the block-autoregressive decode loop.
+
+The loop is the one the pages describe ([canvas] steps 1-4, [arch]): encode the
+prompt causally into a KV cache; for each 256-token block fill a canvas with
+uniform-random ids, run denoise steps (a full bidirectional forward over the
+canvas against the cache, then the sampler and stop test), commit the argmax
+block by encoding it causally into the cache like the prompt, and start the next
+canvas conditioned on the longer history.
+
+Model structure (the pages give only "Gemma 4 26B-A4B backbone, MoE, diffusion
+head"; the plainest decoder reading is used):
+
+    x      = E[ids]                                   tied embedding, no scale
+    per layer:
+      xn   = rnd(rmsnorm(x, w_attn))                  pre-norm, eps 1e-6
+      q,k,v= xn Wqkv^T ; q,k = rope(q,k; absolute pos); rnd(q), rnd(k), rnd(v)
+      o    = rnd(attention(q, [K_cache | k], [V_cache | v]))  no mask / causal
+      x    = f32(x + o Wo^T)
+      xn2  = rnd(rmsnorm(x, w_ffn))
+      x    = f32(x + moe_ffn(xn2))
+    logits = f32(rnd(rmsnorm(x, w_final)) E^T)        the LM ("diffusion") head
+
+rnd() is the path's storage rounding (bf16 RNE, or fp32 for the all-fp32
+configuration); f32() is rounding to binary32 for the fp32 residual stream and
+logits.  RoPE is rotate-half: for i < hd/2, angle = pos * theta^(-2i/hd),
+out_i = x_i cos - x_{i+hd/2} sin, out_{i+hd/2} = x_{i+hd/2} cos + x_i sin.
+"""
+from dataclasses import dataclass, field
+
+import numpy as np
+
+from . import sampler as smp
+from .attention import attention
+from .moe import moe_ffn
+from .numerics import round_f32, round_storage
+
+
+@dataclass
+class ModelConfig:
+    n_layers: int
+    d_model: int
+    n_heads: int
+    n_kv_heads: int
+    head_dim: int
+    n_experts: int
+    top_k: int
+    expert_hidden: int
+    shared_hidden: int
+    vocab: int
+    canvas: int = 256
+    storage: str = "bf16"
+    eps: float = 1e-6
+    rope_theta: float = 10000.0
+    tau: float = smp.TAU
+    h_bound: float = smp.H_BOUND
+    max_steps: int = smp.MAX_STEPS
+
+
+def rmsnorm(x, w, eps):
+    x = np.asarray(x, dtype=np.float64)
+    return x / np.sqrt((x * x).mean(axis=-1, keepdims=True) + eps) * np.asarray(w, dtype=np.float64)
+
+
+def rope(x, positions, theta):
+    """x [H, T, hd] rotated at absolute positions [T] (rotate-half)."""
+    x = np.asarray(x, dtype=np.float64)
+    hd = x.shape[-1]
+    half = hd // 2
+    inv = theta ** (-2.0 * np.arange(half, dtype=np.float64) / hd)
+    ang = np.asarray(positions, dtype=np.float64)[:, None] * inv[None, :]
+    c, s = np.cos(ang)[None], np.sin(ang)[None]
+    x1, x2 = x[..., :half], x[..., half:]
+    return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)
+
+
+@dataclass
+class KVCache:
+    """Per-layer committed keys/values [Hkv, P, hd] (float64 holding stored values)."""
+    k: list = field(default_factory=list)
+    v: list = field(default_factory=list)
+
+    @property
+    def length(self):
+        return 0 if not self.k else self.k[0].shape[1]
+
+
+def layer_forward(cfg, lw, x, positions, cache_k, cache_v, causal):
+    """One decoder layer over new tokens x [T, d] (fp32 values).
+
+    cache_k/v: [Hkv, P, hd] committed history.  Returns (x_out, k_new, v_new, info).
+    """
+    st = cfg.storage
+    t = x.shape[0]
+    hq, hkv, hd = cfg.n_heads, cfg.n_kv_heads, cfg.head_dim
+    xn = round_storage(rmsnorm(x, lw["attn_norm"], cfg.eps), st)
+    qkv = xn @ np.asarray(lw["wqkv"], dtype=np.float64).T
+    q = qkv[:, :hq * hd].reshape(t, hq, hd).transpose(1, 0, 2)
+    k = qkv[:, hq * hd:(hq + hkv) * hd].reshape(t, hkv, hd).transpose(1, 0, 2)
+    v = qkv[:, (hq + hkv) * hd:].reshape(t, hkv, hd).transpose(1, 0, 2)
+    q = round_storage(rope(q, positions, cfg.rope_theta), st)
+    k = round_storage(rope(k, positions, cfg.rope_theta), st)
+    v = round_storage(v, st)
+    keys = np.concatenate([cache_k, k], axis=1)
+    vals = np.concatenate([cache_v, v], axis=1)
+    p = cache_k.shape[1]
+    o = attention(q, keys, vals, 1.0 / np.sqrt(hd), causal_prefix=p if causal else None)
+    o = round_storage(o.transpose(1, 0, 2).reshape(t, hq * hd), st)
+    x1 = round_f32(x + o @ np.asarray(lw["wo"], dtype=np.float64).T)
+    xn2 = round_storage(rmsnorm(x1, lw["ffn_norm"], cfg.eps), st)
+    shared = (lw["ws_gu"], lw["ws_d"]) if lw.get("ws_gu") is not None else None
+    y, minfo = moe_ffn(xn2, lw["wr"], lw["w_gu"], lw["w_d"], cfg.top_k, st, shared)
+    x2 = round_f32(x1 + y)
+    info = dict(xn=xn, q=q, k=k, v=v, o=o, x_attn=x1, xn2=xn2, moe=minfo)
+    return x2, k, v, info
+
+
+def forward_tokens(cfg, weights, ids, positions, cache, causal, keep_info=False):
+    """Run all layers over new tokens; returns (final hidden x [T, d], per-layer (k, v), infos)."""
+    x = round_f32(np.asarray(weights["embed"], dtype=np.float64)[np.asarray(ids)])
+    kv_new, infos = [], []
+    for l, lw in enumerate(weights["layers"]):
+        if cache.length:
+            ck, cv = cache.k[l], cache.v[l]
+        else:
+            ck = np.zeros((cfg.n_kv_heads, 0, cfg.head_dim))
+            cv = np.zeros((cfg.n_kv_heads, 0, cfg.head_dim))
+        x, k, v, info = layer_forward(cfg, lw, x, positions, ck, cv, causal)
+        kv_new.append((k, v))
+        if keep_info:
+            infos.append(info)
+    return x, kv_new, infos
+
+
+def lm_head(cfg, weights, x):
+    """Final norm then the tied LM head; logits rounded to fp32 like the GPU's accumulators."""
+    xf = round_storage(rmsnorm(x, weights["final_norm"], cfg.eps), cfg.storage)
+    return round_f32(xf @ np.asarray(weights["embed"], dtype=np.float64).T)
+
+
+def denoise_logits(cfg, weights, canvas, cache, keep_info=False):
+    """One denoise forward: canvas [T] ids at positions P..P+T-1, no mask, cache untouched."""
+    p = cache.length
+    pos = p + np.arange(len(canvas))
+    x, _, infos = forward_tokens(cfg, weights, canvas, pos, cache, causal=False, keep_info=keep_info)
+    logits = lm_head(cfg, weights, x)
+    return (logits, infos) if keep_info else logits
+
+
+def causal_encode(cfg, weights, ids, cache):
+    """Prefill / commit: encode ids causally at positions P.. and append their K/V."""
+    p = cache.length
+    pos = p + np.arange(len(ids))
+    _, kv_new, _ = forward_tokens(cfg, weights, ids, pos, cache, causal=True)
+    for l, (k, v) in enumerate(kv_new):
+        if len(cache.k) <= l:
+            cache.k.append(k)
+            cache.v.append(v)
+        else:
+            cache.k[l] = np.concatenate([cache.k[l], k], axis=1)
+            cache.v[l] = np.concatenate([cache.v[l], v], axis=1)
+    return cache
+
+
+def decode(cfg, weights, prompt_ids, n_blocks, seed, fixed_steps=None):
+    """Block-autoregressive diffusion decode; returns committed ids and per-block records."""
+    cache = KVCache()
+    causal_encode(cfg, weights, prompt_ids, cache)
+    blocks = []
+    for b in range(n_blocks):
+        res = smp.run_block(lambda t, canvas: denoise_logits(cfg, weights, canvas, cache),
+                            seed, b, cfg.vocab, cfg.canvas, max_steps=cfg.max_steps,
+                            fixed_steps=fixed_steps, tau=cfg.tau, h_bound=cfg.h_bound)
+        causal_encode(cfg, weights, res["committed"], cache)
+        blocks.append(res)
+    out = np.concatenate([b["committed"] for b in blocks]) if blocks else np.zeros(0, np.int64)
+    return out, blocks, cache
