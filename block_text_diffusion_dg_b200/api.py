@@ -1,0 +1,258 @@
+"""Python binding of libdg: the same entry points as include/dg.h, taking torch CUDA tensors.
+
+PyTorch provides device memory and streams only; every step of the denoise path runs in
+libdg's kernels.  Each wrapper checks the library's status and raises on failure.
+"""
+import ctypes as C
+
+import torch
+
+from . import _lib as L
+from ._lib import check, lib
+
+
+def _ptr(t):
+    return C.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return C.c_void_p(s.cuda_stream)
+
+
+def _need_cuda(t, name, dtype=None):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def make_config(shape, *, kv_capacity, fixed_steps=16, max_steps=48, tau=0.9, h_bound=0.005,
+                eps=1e-6, rope_theta=10000.0):
+    s = shape
+    return L.Config(
+        n_layers=s["n_layers"], d_model=s["d_model"], n_heads=s["n_heads"],
+        n_kv_heads=s["n_kv_heads"], head_dim=s["head_dim"], n_experts=s["n_experts"],
+        top_k=s["top_k"], expert_hidden=s["expert_hidden"], shared_hidden=s["shared_hidden"],
+        vocab=s["vocab"], canvas=s["canvas"], kv_capacity=kv_capacity,
+        dtype=L.DTYPE_FP32 if s["storage"] == "fp32" else L.DTYPE_BF16, eps=eps,
+        rope_theta=rope_theta, tau=tau, h_bound=h_bound, max_steps=max_steps,
+        fixed_steps=fixed_steps)
+
+
+def workspace_bytes(cfg):
+    kv, scratch = C.c_size_t(), C.c_size_t()
+    check(lib().dg_workspace_bytes(C.byref(cfg), C.byref(kv), C.byref(scratch)),
+          "dg_workspace_bytes")
+    return kv.value, scratch.value
+
+
+class DiffusionModel:
+    """A bound model context (dg_ctx): weights, KV cache and scratch owned by torch tensors."""
+
+    def __init__(self, cfg, weights, device="cuda", stream=None):
+        self.cfg = cfg
+        self.weights = weights  # keep the tensors alive
+        self.device = torch.device(device)
+        kv_b, sc_b = workspace_bytes(cfg)
+        self.kv = torch.empty(kv_b, dtype=torch.uint8, device=self.device)
+        self.scratch = torch.empty(sc_b, dtype=torch.uint8, device=self.device)
+        layers = (L.LayerWeights * cfg.n_layers)()
+        for i, lw in enumerate(weights["layers"]):
+            for name in ("attn_norm", "wqkv", "wo", "ffn_norm", "wr", "w_gu", "w_d", "ws_gu", "ws_d"):
+                t = lw.get(name)
+                _need_cuda(t, name)
+                setattr(layers[i], name, None if t is None else t.data_ptr())
+        _need_cuda(weights["embed"], "embed")
+        _need_cuda(weights["final_norm"], "final_norm")
+        self._layers = layers
+        w = L.Weights(embed=weights["embed"].data_ptr(), final_norm=weights["final_norm"].data_ptr(),
+                      layers=layers)
+        h = C.c_void_p()
+        check(lib().dg_create(C.byref(cfg), C.byref(w), _ptr(self.kv), _ptr(self.scratch),
+                              _stream(stream), C.byref(h)), "dg_create")
+        self.handle = h
+        bufs = [C.c_void_p() for _ in range(5)]
+        check(lib().dg_get_buffers(h, *[C.byref(b) for b in bufs]), "dg_get_buffers")
+        self._bufs = [b.value for b in bufs]
+        self.out_ids = torch.empty(cfg.canvas, dtype=torch.int32, device=self.device)
+        self.out_state = torch.empty(L.STATE_WORDS, dtype=torch.int32, device=self.device)
+
+    def close(self):
+        if getattr(self, "handle", None):
+            lib().dg_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # --- the five entry points of the decode loop ---
+    def kv_append(self, ids, stream=None):
+        _need_cuda(ids, "ids", torch.int32)
+        check(lib().dg_kv_append(self.handle, _ptr(ids), ids.numel(), _stream(stream)),
+              "dg_kv_append")
+
+    def canvas_init(self, seed, block, stream=None):
+        check(lib().dg_canvas_init(self.handle, C.c_uint64(seed), block, _stream(stream)),
+              "dg_canvas_init")
+
+    def denoise_step(self, step, stream=None):
+        check(lib().dg_denoise_step(self.handle, step, _stream(stream)), "dg_denoise_step")
+
+    def sample_update(self, step, stream=None):
+        check(lib().dg_sample_update(self.handle, step, _stream(stream)), "dg_sample_update")
+
+    def commit_block(self, out_ids=None, out_state=None, stream=None):
+        out_ids = self.out_ids if out_ids is None else out_ids
+        out_state = self.out_state if out_state is None else out_state
+        check(lib().dg_commit_block(self.handle, _ptr(out_ids), _ptr(out_state), _stream(stream)),
+              "dg_commit_block")
+        return out_ids, out_state
+
+    # --- inspection ---
+    @property
+    def kv_length(self):
+        return lib().dg_kv_length(self.handle)
+
+    def kv_truncate(self, n):
+        check(lib().dg_kv_truncate(self.handle, n), "dg_kv_truncate")
+
+    def _view(self, ptr, n, dtype):
+        # a non-owning view of a scratch buffer (offset into self.scratch)
+        off = ptr - self.scratch.data_ptr()
+        nbytes = n * torch.empty((), dtype=dtype).element_size()
+        return self.scratch[off:off + nbytes].view(dtype)
+
+    def buffers(self):
+        t = self.cfg.canvas
+        return dict(canvas=self._view(self._bufs[0], t, torch.int32),
+                    argmax=self._view(self._bufs[1], t, torch.int32),
+                    entropy=self._view(self._bufs[2], t, torch.float32),
+                    conf=self._view(self._bufs[3], t, torch.float32),
+                    state=self._view(self._bufs[4], L.STATE_WORDS, torch.int32))
+
+    def check_device_status(self, stream=None):
+        check(lib().dg_check_device_status(self.handle, _stream(stream)), "dg_check_device_status")
+
+    def debug_logits(self, stream=None):
+        out = torch.empty(self.cfg.canvas, self.cfg.vocab, dtype=torch.float32, device=self.device)
+        check(lib().dg_debug_logits(self.handle, _ptr(out), _stream(stream)), "dg_debug_logits")
+        return out
+
+    def debug_hidden(self):
+        p = C.c_void_p()
+        check(lib().dg_debug_hidden(self.handle, C.byref(p)), "dg_debug_hidden")
+        return self._view(p.value, self.cfg.canvas * self.cfg.d_model, torch.float32).view(
+            self.cfg.canvas, self.cfg.d_model)
+
+    def debug_layer(self, layer, x_in, causal, stream=None):
+        _need_cuda(x_in, "x_in", torch.float32)
+        out = torch.empty_like(x_in)
+        check(lib().dg_debug_layer(self.handle, layer, _ptr(x_in), _ptr(out), x_in.shape[0],
+                                   int(bool(causal)), _stream(stream)), "dg_debug_layer")
+        return out
+
+
+def generate(model, prompt_ids, n_blocks, seed, stream=None):
+    """Block-autoregressive decode through the C ABI; returns (ids [n_blocks*T], states)."""
+    cfg = model.cfg
+    if prompt_ids is not None and prompt_ids.numel():
+        model.kv_append(prompt_ids, stream)
+    steps = cfg.fixed_steps if cfg.fixed_steps > 0 else cfg.max_steps
+    out = torch.empty(n_blocks * cfg.canvas, dtype=torch.int32, device=model.device)
+    states = torch.empty(n_blocks, L.STATE_WORDS, dtype=torch.int32, device=model.device)
+    for b in range(n_blocks):
+        model.canvas_init(seed, b, stream)
+        for t in range(1, steps + 1):
+            model.denoise_step(t, stream)
+            model.sample_update(t, stream)
+        model.commit_block(out[b * cfg.canvas:(b + 1) * cfg.canvas], states[b], stream)
+    return out, states
+
+
+# ---------------------------------------------------------------------------------------
+# standalone operators
+class Sampler:
+    """The canvas sampler over caller-provided logits [rows, V] (bf16 or fp32)."""
+
+    def __init__(self, rows, vocab, device="cuda"):
+        self.rows, self.vocab = rows, vocab
+        n = C.c_size_t()
+        check(lib().dg_sampler_workspace_bytes(rows, vocab, C.byref(n)), "dg_sampler_workspace_bytes")
+        self.ws = torch.empty(n.value, dtype=torch.uint8, device=device)
+        self.state = torch.zeros(L.STATE_WORDS, dtype=torch.int32, device=device)
+        self.canvas = torch.empty(rows, dtype=torch.int32, device=device)
+        self.argmax = torch.empty(rows, dtype=torch.int32, device=device)
+        self.entropy = torch.empty(rows, dtype=torch.float32, device=device)
+        self.conf = torch.empty(rows, dtype=torch.float32, device=device)
+
+    def reset(self, stream=None):
+        check(lib().dg_sampler_reset(self.rows, self.vocab, _ptr(self.ws), _ptr(self.state),
+                                     _stream(stream)), "dg_sampler_reset")
+
+    def step(self, logits, seed, block, step, tau=0.9, h_bound=0.005, max_steps=48,
+             fixed_steps=0, stream=None):
+        _need_cuda(logits, "logits")
+        if tuple(logits.shape) != (self.rows, self.vocab):
+            raise ValueError("logits shape mismatch")
+        dt = {torch.bfloat16: L.DTYPE_BF16, torch.float32: L.DTYPE_FP32}[logits.dtype]
+        check(lib().dg_sampler_step(_ptr(logits), dt, self.rows, self.vocab, C.c_uint64(seed),
+                                    block, step, tau, h_bound, max_steps, fixed_steps, _ptr(self.ws),
+                                    _ptr(self.canvas), _ptr(self.argmax), _ptr(self.entropy),
+                                    _ptr(self.conf), _ptr(self.state), _stream(stream)),
+              "dg_sampler_step")
+
+
+def canvas_attention(q, k, vt, n_keys, causal_prefix=-1, scale=None, n_queries=None, out=None,
+                     workspace=None, stream=None):
+    """q [Hq, Tq, 128] bf16, k [Hkv, ldk, 128] bf16, vt [Hkv, 128, ldk] bf16 -> o [T, Hq*128]."""
+    for t, n in ((q, "q"), (k, "k"), (vt, "vt")):
+        _need_cuda(t, n, torch.bfloat16)
+    hq, tq, hd = q.shape
+    hkv, ldk, _ = k.shape
+    t = tq if n_queries is None else n_queries
+    scale = hd ** -0.5 if scale is None else scale
+    if out is None:
+        out = torch.empty(t, hq * hd, dtype=torch.bfloat16, device=q.device)
+    if workspace is None:
+        n = C.c_size_t()
+        check(lib().dg_attention_workspace_bytes(hq, hkv, tq, n_keys, C.byref(n)),
+              "dg_attention_workspace_bytes")
+        workspace = torch.empty(n.value, dtype=torch.uint8, device=q.device)
+    check(lib().dg_canvas_attention(_ptr(q), _ptr(k), _ptr(vt), _ptr(out), hq, hkv, t, tq, n_keys,
+                                    ldk, causal_prefix, scale, _ptr(workspace), workspace.numel(),
+                                    _stream(stream)), "dg_canvas_attention")
+    return out
+
+
+def moe_workspace(t, d, e, k, h, hs, device="cuda"):
+    n = C.c_size_t()
+    check(lib().dg_moe_workspace_bytes(t, d, e, k, h, hs, C.byref(n)), "dg_moe_workspace_bytes")
+    return torch.empty(n.value, dtype=torch.uint8, device=device)
+
+
+def moe_ffn(x, wr, w_gu, w_d, top_k, ws_gu=None, ws_d=None, residual=None, workspace=None,
+            out=None, ids=None, weights=None, router_logits=None, stream=None):
+    """Top-k MoE over x [T, d] bf16 -> y [T, d] fp32 (= residual + MoE(x))."""
+    for t, n in ((x, "x"), (wr, "wr"), (w_gu, "w_gu"), (w_d, "w_d"), (ws_gu, "ws_gu"), (ws_d, "ws_d")):
+        _need_cuda(t, n, torch.bfloat16)
+    t, d = x.shape
+    e, two_h, _ = w_gu.shape
+    h = two_h // 2
+    hs = 0 if ws_gu is None else ws_gu.shape[0] // 2
+    if workspace is None:
+        workspace = moe_workspace(t, d, e, top_k, h, hs, x.device)
+    if out is None:
+        out = torch.empty(t, d, dtype=torch.float32, device=x.device)
+    check(lib().dg_moe_ffn(_ptr(x), _ptr(residual), _ptr(wr), _ptr(w_gu), _ptr(w_d), _ptr(ws_gu),
+                           _ptr(ws_d), _ptr(out), _ptr(ids), _ptr(weights), _ptr(router_logits), t,
+                           d, e, top_k, h, hs, _ptr(workspace), workspace.numel(), _stream(stream)),
+          "dg_moe_ffn")
+    return out

@@ -1,0 +1,1259 @@
+// dg_api.cu -- the C ABI of libdg: argument checks, workspace planning, TMA descriptors and
+// the launch sequences of the denoise step, the sampler, prefill/commit and the standalone
+// operators.  Kernels live in the *.cuh files included below; nothing here computes.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "../../include/dg.h"
+#include "attention.cuh"
+#include "dg_common.cuh"
+#include "fp32_path.cuh"
+#include "gemm.cuh"
+#include "layer.cuh"
+#include "sampler.cuh"
+
+using namespace dg;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+#define DG_CUDA(call)                                                                        \
+  do {                                                                                       \
+    cudaError_t e_ = (call);                                                                 \
+    if (e_ != cudaSuccess)                                                                   \
+      return fail(DG_ERR_CUDA, "%s failed: %s (%s:%d)", #call, cudaGetErrorString(e_),       \
+                  __FILE__, __LINE__);                                                       \
+  } while (0)
+
+#define DG_LAUNCHED()                                                                        \
+  do {                                                                                       \
+    cudaError_t e_ = cudaGetLastError();                                                     \
+    if (e_ != cudaSuccess)                                                                   \
+      return fail(DG_ERR_CUDA, "launch failed: %s (%s:%d)", cudaGetErrorString(e_), __FILE__, \
+                  __LINE__);                                                                 \
+  } while (0)
+
+#define DG_TRY(expr)        \
+  do {                      \
+    int rc_ = (expr);       \
+    if (rc_ != DG_OK) return rc_; \
+  } while (0)
+
+inline cudaStream_t S(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+inline int cdiv(long long a, long long b) { return static_cast<int>((a + b - 1) / b); }
+
+// ---- TMA descriptor encoding through the driver entry point ---------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// bf16 matrix [rows, cols] with row pitch `pitch` elements; box = 64 columns x box_rows,
+// 128-byte swizzle (the layout the UMMA descriptors expect).
+int make_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint64_t pitch,
+              uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  if (reinterpret_cast<uintptr_t>(base) % 16 != 0 || (pitch * 2) % 16 != 0)
+    return fail(DG_ERR_INVALID_ARG, "TMA operand not 16-byte aligned (base %p, pitch %llu)", base,
+                (unsigned long long)pitch);
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {pitch * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) rows=%llu cols=%llu box=%u",
+                static_cast<int>(r), (unsigned long long)rows, (unsigned long long)cols, box_rows);
+  return DG_OK;
+}
+
+int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
+
+template <typename K>
+int set_smem(K kernel, int bytes) {
+  DG_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  return DG_OK;
+}
+
+// ---- GEMM launch helpers -----------------------------------------------------------------
+constexpr int kDenseN = 256, kDenseStages = 4;
+constexpr int kGroupN = 64, kGroupStages = 8;
+
+template <int MAXN, int STAGES, int EPI>
+int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, int grid,
+                cudaStream_t st) {
+  auto k = gemm_swapab_kernel<MAXN, STAGES, EPI>;
+  constexpr int smem = GemmCfg<MAXN, STAGES>::kSmemBytes;
+  DG_TRY(set_smem(k, smem));
+  k<<<grid, 192, smem, st>>>(ta, tb, p);
+  DG_LAUNCHED();
+  return DG_OK;
+}
+
+GemmParams dense_params(int m_rows, int n_tokens, int k_dim, int k_splits, int* err,
+                        const int* done) {
+  GemmParams p{};
+  p.m_tiles = cdiv(m_rows, 128);
+  p.k_splits = k_splits;
+  p.n_chunk = kDenseN;
+  p.n_total = n_tokens;
+  p.n_chunks = cdiv(n_tokens, kDenseN);
+  p.kb_total = k_dim / 64;
+  p.m_valid = m_rows;
+  p.err = err;
+  p.done = done;
+  return p;
+}
+
+int pick_splits(int m_tiles, int kb_total, int sms) {
+  int s = std::max(1, sms / std::max(1, m_tiles));
+  s = std::min(s, std::max(1, kb_total / 2));
+  return std::min(s, 16);
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------------------
+struct dg_ctx {
+  dg_config cfg;
+  std::vector<dg_layer_weights> layers;
+  const void* embed;
+  const float* final_norm;
+  uint8_t* kv;
+  uint8_t* scratch;
+  int32_t kv_len;
+  int sms;
+  bool bf16;
+  int esz;          // bytes per stored element (2 or 4)
+  int tq;           // query rows per head in the Q buffer
+  int qkv_rows;
+  int split_qkv, split_o, split_r;
+  int att_splits_max;
+  size_t part_elems;
+  // scratch views
+  int32_t *canvas, *argmax, *prev_argmax, *locked, *state, *ticket, *err;
+  float *entropy, *conf;
+  double* row_h;
+  float* x;
+  void* xn;
+  float* part;
+  void* q;
+  float* o_part;
+  float2* ml_part;
+  void* o;
+  float* router_logits;
+  int32_t *topk_ids, *offsets, *perm, *item_counts;
+  float* topk_w;
+  int4 *items_gu, *items_d;
+  void *x_perm, *h, *hs;
+  float *y_slot, *y_shared;
+  StatPartial* lm_part;
+  float* logits;  // fp32 path
+  float2* rope_tab;
+  void *kc, *vtc;
+  // tensor maps (bf16)
+  CUtensorMap tm_xn32, tm_xn128, tm_o32, tm_xperm, tm_h, tm_hs, tm_q, tm_k, tm_vt, tm_embed;
+  std::vector<CUtensorMap> tm_wqkv, tm_wo, tm_wr, tm_wgu, tm_wd, tm_wsgu, tm_wsd;
+  uint64_t seed;
+  uint32_t block;
+};
+
+namespace {
+
+int check_config(const dg_config* c) {
+  if (!c) return fail(DG_ERR_INVALID_ARG, "null config");
+  if (c->n_layers < 1 || c->d_model < 1 || c->n_heads < 1 || c->n_kv_heads < 1 ||
+      c->head_dim < 2 || c->n_experts < 1 || c->top_k < 1 || c->expert_hidden < 1 ||
+      c->shared_hidden < 0 || c->vocab < 2 || c->canvas < 1 || c->kv_capacity < 1)
+    return fail(DG_ERR_INVALID_ARG, "config has a non-positive size");
+  if (c->n_heads % c->n_kv_heads != 0)
+    return fail(DG_ERR_INVALID_ARG, "n_heads must be a multiple of n_kv_heads");
+  if (c->top_k > 8 || c->top_k > c->n_experts || c->n_experts > 256)
+    return fail(DG_ERR_UNSUPPORTED, "need top_k <= min(8, E) and E <= 256");
+  if (c->canvas > 256) return fail(DG_ERR_UNSUPPORTED, "canvas must be <= 256");
+  if (c->kv_capacity % 8 != 0 || c->kv_capacity < c->canvas)
+    return fail(DG_ERR_INVALID_ARG, "kv_capacity must be a multiple of 8 and >= canvas");
+  if (c->head_dim % 2 != 0) return fail(DG_ERR_INVALID_ARG, "head_dim must be even");
+  if (c->vocab % 8 != 0) return fail(DG_ERR_UNSUPPORTED, "vocab must be a multiple of 8");
+  if (c->max_steps < 1 || c->fixed_steps < 0)
+    return fail(DG_ERR_INVALID_ARG, "max_steps must be >= 1 and fixed_steps >= 0");
+  if (c->dtype == DG_DTYPE_BF16) {
+    if (c->head_dim != 128) return fail(DG_ERR_UNSUPPORTED, "bf16 path needs head_dim 128");
+    if (c->d_model % 64 || c->expert_hidden % 64 || c->shared_hidden % 64)
+      return fail(DG_ERR_UNSUPPORTED, "bf16 path needs d, h, hs multiples of 64");
+    if (c->vocab % 256) return fail(DG_ERR_UNSUPPORTED, "bf16 path needs vocab % 256 == 0");
+  } else if (c->dtype == DG_DTYPE_FP32) {
+    if (c->head_dim > 128) return fail(DG_ERR_UNSUPPORTED, "fp32 path needs head_dim <= 128");
+    if (c->vocab % 4) return fail(DG_ERR_UNSUPPORTED, "fp32 path needs vocab % 4 == 0");
+  } else {
+    return fail(DG_ERR_INVALID_ARG, "unknown dtype %d", c->dtype);
+  }
+  return DG_OK;
+}
+
+// Workspace plan: every buffer at a 256-byte boundary, in this order.
+struct Plan {
+  size_t off[40];
+  size_t total;
+  size_t kv;
+};
+
+enum Buf {
+  B_CANVAS, B_ARGMAX, B_PREV, B_LOCKED, B_STATE, B_TICKET, B_ERR, B_ENT, B_CONF, B_ROWH, B_X,
+  B_XN, B_PART, B_Q, B_OPART, B_ML, B_O, B_RLOG, B_IDS, B_W, B_OFF, B_PERM, B_ITEMS_GU,
+  B_ITEMS_D, B_ICNT, B_XPERM, B_H, B_HS, B_YSLOT, B_YSH, B_LMPART, B_LOGITS, B_ROPE, B_END
+};
+
+struct Derived {
+  int tq, qkv_rows, split_qkv, split_o, split_r, att_splits, esz;
+  size_t part_elems;
+  long long max_items_gu, max_items_d;
+};
+
+Derived derive(const dg_config& c, int sms) {
+  Derived d{};
+  const bool bf16 = c.dtype == DG_DTYPE_BF16;
+  d.esz = bf16 ? 2 : 4;
+  d.tq = bf16 ? 256 : c.canvas;
+  d.qkv_rows = (c.n_heads + 2 * c.n_kv_heads) * c.head_dim;
+  if (bf16) {
+    d.split_qkv = pick_splits(cdiv(d.qkv_rows, 128), c.d_model / 64, sms);
+    d.split_o = pick_splits(cdiv(c.d_model, 128), c.n_heads * c.head_dim / 64, sms);
+    d.split_r = std::min(16, std::max(1, c.d_model / 64 / 4));
+  } else {
+    d.split_qkv = d.split_o = d.split_r = 1;
+  }
+  const long long T = c.canvas;
+  size_t pe = std::max({static_cast<size_t>(d.split_qkv) * T * d.qkv_rows,
+                        static_cast<size_t>(d.split_o) * T * c.d_model,
+                        static_cast<size_t>(d.split_r) * T * c.n_experts});
+  d.part_elems = pe;
+  const int group = c.n_heads / c.n_kv_heads;
+  const int m_tiles = group * d.tq / 128;
+  d.att_splits = std::max(1, std::min(16, sms / std::max(1, m_tiles * c.n_kv_heads)));
+  const long long chunks = c.n_experts + (T * c.top_k + kGroupN - 1) / kGroupN;
+  d.max_items_gu = chunks * cdiv(2 * c.expert_hidden, 128);
+  d.max_items_d = chunks * cdiv(c.d_model, 128);
+  return d;
+}
+
+Plan plan(const dg_config& c, int sms) {
+  Plan p{};
+  const Derived dv = derive(c, sms);
+  const bool bf16 = c.dtype == DG_DTYPE_BF16;
+  const size_t T = c.canvas, d = c.d_model, E = c.n_experts, k = c.top_k, es = dv.esz;
+  const size_t hd = c.head_dim, Hq = c.n_heads;
+  const size_t nv = bf16 ? c.vocab / 256 : cdiv(c.vocab, 4096);
+  size_t sz[B_END];
+  sz[B_CANVAS] = sz[B_ARGMAX] = sz[B_PREV] = sz[B_LOCKED] = T * 4;
+  sz[B_STATE] = kStWords * 4;
+  sz[B_TICKET] = sz[B_ERR] = 4;
+  sz[B_ENT] = sz[B_CONF] = T * 4;
+  sz[B_ROWH] = T * 8;
+  sz[B_X] = T * d * 4;
+  sz[B_XN] = T * d * es;
+  sz[B_PART] = dv.part_elems * 4;
+  sz[B_Q] = Hq * dv.tq * hd * es;
+  sz[B_OPART] = bf16 ? static_cast<size_t>(dv.att_splits) * Hq * dv.tq * 128 * 4 : 0;
+  sz[B_ML] = bf16 ? static_cast<size_t>(dv.att_splits) * Hq * dv.tq * 8 : 0;
+  sz[B_O] = T * Hq * hd * es;
+  sz[B_RLOG] = T * E * 4;
+  sz[B_IDS] = sz[B_W] = T * k * 4;
+  sz[B_OFF] = (E + 1) * 4;
+  sz[B_PERM] = T * k * 4;
+  sz[B_ITEMS_GU] = bf16 ? dv.max_items_gu * 16 : 0;
+  sz[B_ITEMS_D] = bf16 ? dv.max_items_d * 16 : 0;
+  sz[B_ICNT] = 8;
+  sz[B_XPERM] = bf16 ? T * k * d * es : 0;
+  sz[B_H] = bf16 ? T * k * c.expert_hidden * es : 0;
+  sz[B_HS] = bf16 ? T * std::max<size_t>(1, c.shared_hidden) * es : 0;
+  sz[B_YSLOT] = T * k * d * 4;
+  sz[B_YSH] = T * d * 4;
+  sz[B_LMPART] = T * nv * sizeof(StatPartial);
+  sz[B_LOGITS] = bf16 ? 0 : T * c.vocab * 4;
+  sz[B_ROPE] = static_cast<size_t>(c.kv_capacity) * (hd / 2) * 8;
+  size_t o = 0;
+  for (int b = 0; b < B_END; ++b) {
+    p.off[b] = o;
+    o += align256(std::max<size_t>(sz[b], 1));
+  }
+  p.total = o;
+  p.kv = 2 * static_cast<size_t>(c.n_layers) * c.n_kv_heads * c.kv_capacity * hd * es;
+  return p;
+}
+
+// ---- the layer pipeline -----------------------------------------------------------------
+// Runs every layer over n tokens at positions pos0.. (canvas buffer or caller ids), writes their
+// K/V into cache slots pos0..pos0+n-1 and leaves the final-normed hidden state in xn.
+int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_norm,
+              const int* done, cudaStream_t st);
+
+int run_forward(dg_ctx* c, const int32_t* ids, int n, int pos0, int causal, const int* done,
+                cudaStream_t st) {
+  const dg_config& g = c->cfg;
+  if (c->bf16)
+    embed_norm_kernel<__nv_bfloat16, __nv_bfloat16><<<n, 256, 0, st>>>(
+        ids, static_cast<const __nv_bfloat16*>(c->embed), g.d_model, c->layers[0].attn_norm, g.eps,
+        c->x, static_cast<__nv_bfloat16*>(c->xn), done);
+  else
+    embed_norm_kernel<float, float><<<n, 256, 0, st>>>(ids, static_cast<const float*>(c->embed),
+                                                       g.d_model, c->layers[0].attn_norm, g.eps,
+                                                       c->x, static_cast<float*>(c->xn), done);
+  DG_LAUNCHED();
+  for (int l = 0; l < g.n_layers; ++l) {
+    const float* nn = (l + 1 < g.n_layers) ? c->layers[l + 1].attn_norm : c->final_norm;
+    DG_TRY(run_layer(c, l, n, pos0, causal, nn, done, st));
+  }
+  return DG_OK;
+}
+
+template <typename TA>
+int layer_tail_common(dg_ctx* c, int l, int n, int pos0, const int* done, cudaStream_t st,
+                      long long qkv_ss, int splits_qkv) {
+  const dg_config& g = c->cfg;
+  const int hd = g.head_dim;
+  const size_t kv_head_elems = static_cast<size_t>(g.kv_capacity) * hd;
+  TA* kc = static_cast<TA*>(c->kc) + static_cast<size_t>(l) * g.n_kv_heads * kv_head_elems;
+  TA* vtc = static_cast<TA*>(c->vtc) + static_cast<size_t>(l) * g.n_kv_heads * kv_head_elems;
+  rope_qk_kernel<TA><<<dim3(n, g.n_heads + g.n_kv_heads), hd / 2, 0, st>>>(
+      c->part, splits_qkv, qkv_ss, c->qkv_rows, hd, g.n_heads, c->rope_tab, pos0,
+      static_cast<TA*>(c->q), c->tq, kc, g.kv_capacity, done);
+  DG_LAUNCHED();
+  v_store_kernel<TA><<<dim3(cdiv(n, 32), g.n_kv_heads), dim3(32, 8), 0, st>>>(
+      c->part, splits_qkv, qkv_ss, c->qkv_rows, hd, (g.n_heads + g.n_kv_heads) * hd, n, pos0, vtc,
+      g.kv_capacity, done);
+  DG_LAUNCHED();
+  return DG_OK;
+}
+
+int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_norm,
+              const int* done, cudaStream_t st) {
+  const dg_config& g = c->cfg;
+  const dg_layer_weights& w = c->layers[l];
+  const int d = g.d_model, hd = g.head_dim, k = g.top_k, E = g.n_experts;
+  const int n_keys = pos0 + n;
+  const int n_slots = n * k;
+  if (!c->bf16) {
+    // ---------------- all-fp32 path ----------------
+    const float* xn = static_cast<const float*>(c->xn);
+    gemm_f32_nt_kernel<<<dim3(cdiv(c->qkv_rows, 64), cdiv(n, 64)), 256, 0, st>>>(
+        xn, static_cast<const float*>(w.wqkv), n, c->qkv_rows, d, c->part, c->qkv_rows, done);
+    DG_LAUNCHED();
+    DG_TRY(layer_tail_common<float>(c, l, n, pos0, done, st, 0, 1));
+    const size_t kv_head_elems = static_cast<size_t>(g.kv_capacity) * hd;
+    const float* kc = static_cast<const float*>(c->kc) + static_cast<size_t>(l) * g.n_kv_heads * kv_head_elems;
+    const float* vtc = static_cast<const float*>(c->vtc) + static_cast<size_t>(l) * g.n_kv_heads * kv_head_elems;
+    const int smem = (n_keys + hd) * 4;
+    if (smem > 200 * 1024) return fail(DG_ERR_UNSUPPORTED, "fp32 attention: too many keys");
+    DG_TRY(set_smem(attention_f32_kernel, smem));
+    attention_f32_kernel<<<dim3(n, g.n_heads), 128, smem, st>>>(
+        static_cast<const float*>(c->q), kc, vtc, static_cast<float*>(c->o), g.n_heads,
+        g.n_heads / g.n_kv_heads, c->tq, hd, g.kv_capacity, n_keys, causal ? pos0 : -1,
+        1.0f / sqrtf(static_cast<float>(hd)), done);
+    DG_LAUNCHED();
+    gemm_f32_nt_kernel<<<dim3(cdiv(d, 64), cdiv(n, 64)), 256, 0, st>>>(
+        static_cast<const float*>(c->o), static_cast<const float*>(w.wo), n, d, g.n_heads * hd,
+        c->part, d, done);
+    DG_LAUNCHED();
+    residual_norm_kernel<float><<<n, 256, 0, st>>>(c->x, c->part, 1, 0, d, w.ffn_norm, g.eps,
+                                                   static_cast<float*>(c->xn), done);
+    DG_LAUNCHED();
+    gemm_f32_nt_kernel<<<dim3(cdiv(E, 64), cdiv(n, 64)), 256, 0, st>>>(
+        xn, static_cast<const float*>(w.wr), n, E, d, c->part, E, done);
+    DG_LAUNCHED();
+    router_topk_kernel<<<cdiv(n, 4), 128, 0, st>>>(c->part, 1, 0, n, E, k, c->router_logits,
+                                                   c->topk_ids, c->topk_w, done);
+    DG_LAUNCHED();
+    const int smem_e = (d + g.expert_hidden) * 4;
+    DG_TRY(set_smem(moe_expert_f32_kernel, smem_e));
+    moe_expert_f32_kernel<<<n_slots, 256, smem_e, st>>>(
+        xn, c->topk_ids, c->topk_w, k, static_cast<const float*>(w.w_gu),
+        static_cast<const float*>(w.w_d), d, g.expert_hidden, c->y_slot, done);
+    DG_LAUNCHED();
+    const float* ysh = nullptr;
+    if (g.shared_hidden > 0) {
+      const int smem_s = (d + g.shared_hidden) * 4;
+      DG_TRY(set_smem(moe_expert_f32_kernel, std::max(smem_s, smem_e)));
+      moe_expert_f32_kernel<<<n, 256, smem_s, st>>>(
+          xn, nullptr, nullptr, 1, static_cast<const float*>(w.ws_gu),
+          static_cast<const float*>(w.ws_d), d, g.shared_hidden, c->y_shared, done);
+      DG_LAUNCHED();
+      ysh = c->y_shared;
+    }
+    moe_combine_norm_kernel<float><<<n, 256, 0, st>>>(c->x, c->y_slot, k, ysh, d, next_norm,
+                                                      g.eps, static_cast<float*>(c->xn), done);
+    DG_LAUNCHED();
+    return DG_OK;
+  }
+  // ---------------- bf16 tcgen05 path ----------------
+  // QKV projection, split-K partials [split][token][row]
+  {
+    GemmParams p = dense_params(c->qkv_rows, n, d, c->split_qkv, c->err, done);
+    p.out_f32 = c->part;
+    p.ld_out = c->qkv_rows;
+    p.split_stride = static_cast<long long>(n) * c->qkv_rows;
+    const int items = p.m_tiles * p.k_splits * p.n_chunks;
+    DG_TRY((launch_gemm<kDenseN, kDenseStages, kEpiPartialF32>(c->tm_wqkv[l], c->tm_xn32, p,
+                                                                 std::min(items, c->sms), st)));
+    DG_TRY(layer_tail_common<__nv_bfloat16>(c, l, n, pos0, done, st, p.split_stride,
+                                            c->split_qkv));
+  }
+  // attention over [cache 0..pos0 | new tokens], split over keys
+  {
+    const int group = g.n_heads / g.n_kv_heads;
+    const int m_tiles = group * c->tq / 128;
+    const int n_kv_tiles = cdiv(n_keys, 128);
+    int splits = std::max(1, std::min(c->att_splits_max, c->sms / (m_tiles * g.n_kv_heads)));
+    splits = std::min(splits, n_kv_tiles);
+    const int tps = cdiv(n_kv_tiles, splits);
+    splits = cdiv(n_kv_tiles, tps);
+    AttnParams a{};
+    a.group = group;
+    a.tq = c->tq;
+    a.n_queries = n;
+    a.n_keys = n_keys;
+    a.causal_prefix = causal ? pos0 : -1;
+    a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(hd)));
+    a.tiles_per_split = tps;
+    a.q_row_base = 0;
+    a.k_row_base = static_cast<long long>(l) * g.n_kv_heads * g.kv_capacity;
+    a.ldk = g.kv_capacity;
+    a.vt_row_base = l * g.n_kv_heads * hd;
+    a.n_heads = g.n_heads;
+    a.o_part = c->o_part;
+    a.ml_part = c->ml_part;
+    a.err = c->err;
+    a.done = done;
+    DG_TRY(set_smem(attention_kernel, kAttnSmemBytes));
+    attention_kernel<<<dim3(m_tiles, g.n_kv_heads, splits), 192, kAttnSmemBytes, st>>>(
+        c->tm_q, c->tm_k, c->tm_vt, a);
+    DG_LAUNCHED();
+    attn_combine_kernel<__nv_bfloat16><<<dim3(n, g.n_heads), 128, 0, st>>>(
+        c->o_part, c->ml_part, splits, g.n_heads, c->tq, n, static_cast<__nv_bfloat16*>(c->o),
+        done);
+    DG_LAUNCHED();
+  }
+  // O projection + residual + ffn norm
+  {
+    GemmParams p = dense_params(d, n, g.n_heads * hd, c->split_o, c->err, done);
+    p.out_f32 = c->part;
+    p.ld_out = d;
+    p.split_stride = static_cast<long long>(n) * d;
+    const int items = p.m_tiles * p.k_splits * p.n_chunks;
+    DG_TRY((launch_gemm<kDenseN, kDenseStages, kEpiPartialF32>(c->tm_wo[l], c->tm_o32, p,
+                                                                 std::min(items, c->sms), st)));
+    residual_norm_kernel<__nv_bfloat16><<<n, 256, 0, st>>>(
+        c->x, c->part, c->split_o, p.split_stride, d, w.ffn_norm, g.eps,
+        static_cast<__nv_bfloat16*>(c->xn), done);
+    DG_LAUNCHED();
+  }
+  // router + top-k
+  {
+    GemmParams p = dense_params(E, n, d, c->split_r, c->err, done);
+    p.out_f32 = c->part;
+    p.ld_out = E;
+    p.split_stride = static_cast<long long>(n) * E;
+    const int items = p.m_tiles * p.k_splits * p.n_chunks;
+    DG_TRY((launch_gemm<kDenseN, kDenseStages, kEpiPartialF32>(c->tm_wr[l], c->tm_xn32, p,
+                                                                 std::min(items, c->sms), st)));
+    router_topk_kernel<<<cdiv(n, 4), 128, 0, st>>>(c->part, c->split_r, p.split_stride, n, E, k,
+                                                   c->router_logits, c->topk_ids, c->topk_w, done);
+    DG_LAUNCHED();
+  }
+  // permutation and grouped expert GEMMs
+  {
+    RouteArgs ra{};
+    ra.ids = c->topk_ids;
+    ra.n_slots = n_slots;
+    ra.n_experts = E;
+    ra.offsets = c->offsets;
+    ra.perm = c->perm;
+    ra.items_gu = c->items_gu;
+    ra.items_d = c->items_d;
+    ra.counts = c->item_counts;
+    ra.m_tiles_gu = cdiv(2 * g.expert_hidden, 128);
+    ra.m_tiles_d = cdiv(d, 128);
+    ra.n_chunk = kGroupN;
+    ra.done = done;
+    moe_route_kernel<<<1, 1024, 0, st>>>(ra);
+    DG_LAUNCHED();
+    gather_rows_kernel<<<n_slots, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(c->xn), c->perm,
+                                                k, d, static_cast<__nv_bfloat16*>(c->x_perm),
+                                                done);
+    DG_LAUNCHED();
+    GemmParams p{};
+    p.items = c->items_gu;
+    p.item_count = c->item_counts;
+    p.a_rows_per_group = 2 * g.expert_hidden;
+    p.kb_total = d / 64;
+    p.m_valid = 2 * g.expert_hidden;
+    p.out_bf16 = static_cast<__nv_bfloat16*>(c->h);
+    p.ld_out = g.expert_hidden;
+    p.err = c->err;
+    p.done = done;
+    DG_TRY((launch_gemm<kGroupN, kGroupStages, kEpiGluBf16>(c->tm_wgu[l], c->tm_xperm, p, c->sms,
+                                                             st)));
+    GemmParams q{};
+    q.items = c->items_d;
+    q.item_count = c->item_counts + 1;
+    q.a_rows_per_group = d;
+    q.kb_total = g.expert_hidden / 64;
+    q.m_valid = d;
+    q.out_f32 = c->y_slot;
+    q.ld_out = d;
+    q.perm = c->perm;
+    q.scale = c->topk_w;
+    q.err = c->err;
+    q.done = done;
+    DG_TRY((launch_gemm<kGroupN, kGroupStages, kEpiScatterF32>(c->tm_wd[l], c->tm_h, q, c->sms,
+                                                                st)));
+  }
+  const float* ysh = nullptr;
+  if (g.shared_hidden > 0) {
+    GemmParams p = dense_params(2 * g.shared_hidden, n, d, 1, c->err, done);
+    p.out_bf16 = static_cast<__nv_bfloat16*>(c->hs);
+    p.ld_out = g.shared_hidden;
+    int items = p.m_tiles * p.n_chunks;
+    DG_TRY((launch_gemm<kDenseN, kDenseStages, kEpiGluBf16>(c->tm_wsgu[l], c->tm_xn32, p,
+                                                              std::min(items, c->sms), st)));
+    GemmParams q = dense_params(d, n, g.shared_hidden, 1, c->err, done);
+    q.out_f32 = c->y_shared;
+    q.ld_out = d;
+    items = q.m_tiles * q.n_chunks;
+    DG_TRY((launch_gemm<kDenseN, kDenseStages, kEpiScatterF32>(c->tm_wsd[l], c->tm_hs, q,
+                                                                 std::min(items, c->sms), st)));
+    ysh = c->y_shared;
+  }
+  moe_combine_norm_kernel<__nv_bfloat16><<<n, 256, 0, st>>>(
+      c->x, c->y_slot, k, ysh, d, next_norm, g.eps, static_cast<__nv_bfloat16*>(c->xn), done);
+  DG_LAUNCHED();
+  return DG_OK;
+}
+
+int run_lm_head(dg_ctx* c, float* logits_out, const int* done, cudaStream_t st) {
+  const dg_config& g = c->cfg;
+  const int T = g.canvas;
+  if (c->bf16) {
+    LmHeadParams p{};
+    p.n_tokens = T;
+    p.n_vtiles = g.vocab / 256;
+    p.kb_total = g.d_model / 64;
+    p.partials = c->lm_part;
+    p.logits = logits_out;
+    p.vocab = g.vocab;
+    p.err = c->err;
+    p.done = done;
+    const int grid = std::min(p.n_vtiles, c->sms);
+    if (logits_out) {
+      DG_TRY(set_smem(lmhead_kernel<false>, kLmSmemBytes));
+      lmhead_kernel<false><<<grid, 192, kLmSmemBytes, st>>>(c->tm_xn128, c->tm_embed, p);
+    } else {
+      DG_TRY(set_smem(lmhead_kernel<true>, kLmSmemBytes));
+      lmhead_kernel<true><<<grid, 192, kLmSmemBytes, st>>>(c->tm_xn128, c->tm_embed, p);
+    }
+    DG_LAUNCHED();
+    return DG_OK;
+  }
+  float* dst = logits_out ? logits_out : c->logits;
+  gemm_f32_nt_kernel<<<dim3(cdiv(g.vocab, 64), cdiv(T, 64)), 256, 0, st>>>(
+      static_cast<const float*>(c->xn), static_cast<const float*>(c->embed), T, g.vocab, g.d_model,
+      dst, g.vocab, done);
+  DG_LAUNCHED();
+  if (!logits_out) {
+    logits_stats_kernel<float, 16><<<dim3(cdiv(g.vocab, 4096), T), 256, 0, st>>>(
+        c->logits, g.vocab, 4096, c->lm_part, done);
+    DG_LAUNCHED();
+  }
+  return DG_OK;
+}
+
+int bind_tmaps(dg_ctx* c) {
+  const dg_config& g = c->cfg;
+  const uint64_t T = g.canvas, d = g.d_model, hd = g.head_dim, k = g.top_k;
+  DG_TRY(make_tmap(&c->tm_xn32, c->xn, T, d, d, 32));
+  DG_TRY(make_tmap(&c->tm_xn128, c->xn, T, d, d, 128));
+  DG_TRY(make_tmap(&c->tm_o32, c->o, T, g.n_heads * hd, g.n_heads * hd, 32));
+  DG_TRY(make_tmap(&c->tm_xperm, c->x_perm, T * k, d, d, 32));
+  DG_TRY(make_tmap(&c->tm_h, c->h, T * k, g.expert_hidden, g.expert_hidden, 32));
+  if (g.shared_hidden > 0)
+    DG_TRY(make_tmap(&c->tm_hs, c->hs, T, g.shared_hidden, g.shared_hidden, 32));
+  DG_TRY(make_tmap(&c->tm_q, c->q, static_cast<uint64_t>(g.n_heads) * c->tq, hd, hd, 128));
+  const uint64_t kv_rows = static_cast<uint64_t>(g.n_layers) * g.n_kv_heads * g.kv_capacity;
+  DG_TRY(make_tmap(&c->tm_k, c->kc, kv_rows, hd, hd, 128));
+  const uint64_t vt_rows = static_cast<uint64_t>(g.n_layers) * g.n_kv_heads * hd;
+  DG_TRY(make_tmap(&c->tm_vt, c->vtc, vt_rows, g.kv_capacity, g.kv_capacity, 128));
+  DG_TRY(make_tmap(&c->tm_embed, c->embed, g.vocab, d, d, 256));
+  const int L = g.n_layers;
+  c->tm_wqkv.resize(L);
+  c->tm_wo.resize(L);
+  c->tm_wr.resize(L);
+  c->tm_wgu.resize(L);
+  c->tm_wd.resize(L);
+  c->tm_wsgu.resize(L);
+  c->tm_wsd.resize(L);
+  for (int l = 0; l < L; ++l) {
+    const dg_layer_weights& w = c->layers[l];
+    DG_TRY(make_tmap(&c->tm_wqkv[l], w.wqkv, c->qkv_rows, d, d, 128));
+    DG_TRY(make_tmap(&c->tm_wo[l], w.wo, d, g.n_heads * hd, g.n_heads * hd, 128));
+    DG_TRY(make_tmap(&c->tm_wr[l], w.wr, g.n_experts, d, d, 128));
+    DG_TRY(make_tmap(&c->tm_wgu[l], w.w_gu, static_cast<uint64_t>(g.n_experts) * 2 * g.expert_hidden,
+                     d, d, 128));
+    DG_TRY(make_tmap(&c->tm_wd[l], w.w_d, static_cast<uint64_t>(g.n_experts) * d, g.expert_hidden,
+                     g.expert_hidden, 128));
+    if (g.shared_hidden > 0) {
+      DG_TRY(make_tmap(&c->tm_wsgu[l], w.ws_gu, 2ull * g.shared_hidden, d, d, 128));
+      DG_TRY(make_tmap(&c->tm_wsd[l], w.ws_d, d, g.shared_hidden, g.shared_hidden, 128));
+    }
+  }
+  return DG_OK;
+}
+
+int check_ctx(const dg_ctx* c) {
+  if (!c) return fail(DG_ERR_INVALID_ARG, "null context");
+  return DG_OK;
+}
+
+}  // namespace
+
+// =======================================================================================
+extern "C" {
+
+const char* dg_last_error(void) { return g_last_error.c_str(); }
+const char* dg_version(void) { return "libdg 0.1 sm_100a"; }
+
+int dg_workspace_bytes(const dg_config* cfg, size_t* kv_bytes, size_t* scratch_bytes) {
+  DG_TRY(check_config(cfg));
+  if (!kv_bytes || !scratch_bytes) return fail(DG_ERR_INVALID_ARG, "null output pointer");
+  const Plan p = plan(*cfg, num_sms());
+  *kv_bytes = p.kv;
+  *scratch_bytes = p.total;
+  return DG_OK;
+}
+
+int dg_create(const dg_config* cfg, const dg_weights* w, void* d_kv, void* d_scratch, void* stream,
+              dg_ctx** out) {
+  DG_TRY(check_config(cfg));
+  if (!w || !w->embed || !w->final_norm || !w->layers || !d_kv || !d_scratch || !out)
+    return fail(DG_ERR_INVALID_ARG, "null weights or buffers");
+  if (reinterpret_cast<uintptr_t>(d_kv) % 256 || reinterpret_cast<uintptr_t>(d_scratch) % 256)
+    return fail(DG_ERR_INVALID_ARG, "kv and scratch must be 256-byte aligned");
+  for (int l = 0; l < cfg->n_layers; ++l) {
+    const dg_layer_weights& lw = w->layers[l];
+    if (!lw.attn_norm || !lw.wqkv || !lw.wo || !lw.ffn_norm || !lw.wr || !lw.w_gu || !lw.w_d)
+      return fail(DG_ERR_INVALID_ARG, "layer %d has a null weight", l);
+    if (cfg->shared_hidden > 0 && (!lw.ws_gu || !lw.ws_d))
+      return fail(DG_ERR_INVALID_ARG, "layer %d lacks shared expert weights", l);
+  }
+  dg_ctx* c = new dg_ctx();
+  c->cfg = *cfg;
+  c->layers.assign(w->layers, w->layers + cfg->n_layers);
+  c->embed = w->embed;
+  c->final_norm = w->final_norm;
+  c->kv = static_cast<uint8_t*>(d_kv);
+  c->scratch = static_cast<uint8_t*>(d_scratch);
+  c->kv_len = 0;
+  c->sms = num_sms();
+  c->bf16 = cfg->dtype == DG_DTYPE_BF16;
+  const Derived dv = derive(*cfg, c->sms);
+  c->esz = dv.esz;
+  c->tq = dv.tq;
+  c->qkv_rows = dv.qkv_rows;
+  c->split_qkv = dv.split_qkv;
+  c->split_o = dv.split_o;
+  c->split_r = dv.split_r;
+  c->att_splits_max = dv.att_splits;
+  c->part_elems = dv.part_elems;
+  const Plan p = plan(*cfg, c->sms);
+  uint8_t* s = c->scratch;
+  c->canvas = reinterpret_cast<int32_t*>(s + p.off[B_CANVAS]);
+  c->argmax = reinterpret_cast<int32_t*>(s + p.off[B_ARGMAX]);
+  c->prev_argmax = reinterpret_cast<int32_t*>(s + p.off[B_PREV]);
+  c->locked = reinterpret_cast<int32_t*>(s + p.off[B_LOCKED]);
+  c->state = reinterpret_cast<int32_t*>(s + p.off[B_STATE]);
+  c->ticket = reinterpret_cast<int32_t*>(s + p.off[B_TICKET]);
+  c->err = reinterpret_cast<int32_t*>(s + p.off[B_ERR]);
+  c->entropy = reinterpret_cast<float*>(s + p.off[B_ENT]);
+  c->conf = reinterpret_cast<float*>(s + p.off[B_CONF]);
+  c->row_h = reinterpret_cast<double*>(s + p.off[B_ROWH]);
+  c->x = reinterpret_cast<float*>(s + p.off[B_X]);
+  c->xn = s + p.off[B_XN];
+  c->part = reinterpret_cast<float*>(s + p.off[B_PART]);
+  c->q = s + p.off[B_Q];
+  c->o_part = reinterpret_cast<float*>(s + p.off[B_OPART]);
+  c->ml_part = reinterpret_cast<float2*>(s + p.off[B_ML]);
+  c->o = s + p.off[B_O];
+  c->router_logits = reinterpret_cast<float*>(s + p.off[B_RLOG]);
+  c->topk_ids = reinterpret_cast<int32_t*>(s + p.off[B_IDS]);
+  c->topk_w = reinterpret_cast<float*>(s + p.off[B_W]);
+  c->offsets = reinterpret_cast<int32_t*>(s + p.off[B_OFF]);
+  c->perm = reinterpret_cast<int32_t*>(s + p.off[B_PERM]);
+  c->items_gu = reinterpret_cast<int4*>(s + p.off[B_ITEMS_GU]);
+  c->items_d = reinterpret_cast<int4*>(s + p.off[B_ITEMS_D]);
+  c->item_counts = reinterpret_cast<int32_t*>(s + p.off[B_ICNT]);
+  c->x_perm = s + p.off[B_XPERM];
+  c->h = s + p.off[B_H];
+  c->hs = s + p.off[B_HS];
+  c->y_slot = reinterpret_cast<float*>(s + p.off[B_YSLOT]);
+  c->y_shared = reinterpret_cast<float*>(s + p.off[B_YSH]);
+  c->lm_part = reinterpret_cast<StatPartial*>(s + p.off[B_LMPART]);
+  c->logits = reinterpret_cast<float*>(s + p.off[B_LOGITS]);
+  c->rope_tab = reinterpret_cast<float2*>(s + p.off[B_ROPE]);
+  const size_t kv_half = p.kv / 2;
+  c->kc = c->kv;
+  c->vtc = c->kv + kv_half;
+  if (c->bf16) {
+    const int rc = bind_tmaps(c);
+    if (rc != DG_OK) {
+      delete c;
+      return rc;
+    }
+  }
+  cudaStream_t st = S(stream);
+  cudaError_t e = cudaMemsetAsync(c->kv, 0, p.kv, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(c->scratch, 0, p.total, st);
+  if (e != cudaSuccess) {
+    delete c;
+    return fail(DG_ERR_CUDA, "memset failed: %s", cudaGetErrorString(e));
+  }
+  const int half = cfg->head_dim / 2;
+  const long long n_tab = static_cast<long long>(cfg->kv_capacity) * half;
+  rope_table_kernel<<<cdiv(n_tab, 256), 256, 0, st>>>(c->rope_tab, cfg->kv_capacity, half,
+                                                       static_cast<double>(cfg->rope_theta));
+  e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    delete c;
+    return fail(DG_ERR_CUDA, "rope table launch failed: %s", cudaGetErrorString(e));
+  }
+  *out = c;
+  return DG_OK;
+}
+
+void dg_destroy(dg_ctx* ctx) { delete ctx; }
+
+int32_t dg_kv_length(const dg_ctx* ctx) { return ctx ? ctx->kv_len : -1; }
+
+int dg_kv_truncate(dg_ctx* ctx, int32_t length) {
+  DG_TRY(check_ctx(ctx));
+  if (length < 0 || length > ctx->kv_len)
+    return fail(DG_ERR_INVALID_ARG, "truncate length %d outside [0, %d]", length, ctx->kv_len);
+  ctx->kv_len = length;
+  return DG_OK;
+}
+
+int dg_kv_append(dg_ctx* ctx, const int32_t* d_ids, int32_t n, void* stream) {
+  DG_TRY(check_ctx(ctx));
+  if (!d_ids || n <= 0) return fail(DG_ERR_INVALID_ARG, "need ids and n > 0");
+  if (static_cast<long long>(ctx->kv_len) + n + ctx->cfg.canvas > ctx->cfg.kv_capacity)
+    return fail(DG_ERR_CAPACITY, "cache of %d positions cannot take %d more plus a canvas of %d",
+                ctx->cfg.kv_capacity, ctx->kv_len + n, ctx->cfg.canvas);
+  cudaStream_t st = S(stream);
+  for (int off = 0; off < n; off += ctx->cfg.canvas) {
+    const int m = std::min(ctx->cfg.canvas, n - off);
+    DG_TRY(run_forward(ctx, d_ids + off, m, ctx->kv_len, 1, nullptr, st));
+    ctx->kv_len += m;
+  }
+  return DG_OK;
+}
+
+int dg_canvas_init(dg_ctx* ctx, uint64_t seed, uint32_t block, void* stream) {
+  DG_TRY(check_ctx(ctx));
+  if (ctx->kv_len + ctx->cfg.canvas > ctx->cfg.kv_capacity)
+    return fail(DG_ERR_CAPACITY, "no room for a canvas after %d committed positions", ctx->kv_len);
+  ctx->seed = seed;
+  ctx->block = block;
+  canvas_init_kernel<<<cdiv(ctx->cfg.canvas, 256), 256, 0, S(stream)>>>(
+      ctx->canvas, ctx->cfg.canvas, ctx->cfg.vocab, seed, block, ctx->state, ctx->ticket);
+  DG_LAUNCHED();
+  return DG_OK;
+}
+
+int dg_denoise_step(dg_ctx* ctx, uint32_t step, void* stream) {
+  DG_TRY(check_ctx(ctx));
+  if (step < 1) return fail(DG_ERR_INVALID_ARG, "steps are numbered from 1");
+  if (ctx->kv_len + ctx->cfg.canvas > ctx->cfg.kv_capacity)
+    return fail(DG_ERR_CAPACITY, "no room for the canvas");
+  cudaStream_t st = S(stream);
+  const int* done = ctx->state + kStDone;
+  DG_TRY(run_forward(ctx, ctx->canvas, ctx->cfg.canvas, ctx->kv_len, 0, done, st));
+  DG_TRY(run_lm_head(ctx, nullptr, done, st));
+  return DG_OK;
+}
+
+int dg_sample_update(dg_ctx* ctx, uint32_t step, void* stream) {
+  DG_TRY(check_ctx(ctx));
+  if (step < 1) return fail(DG_ERR_INVALID_ARG, "steps are numbered from 1");
+  const dg_config& g = ctx->cfg;
+  SamplerArgs a{};
+  a.partials = ctx->lm_part;
+  a.nsplit = ctx->bf16 ? g.vocab / 256 : cdiv(g.vocab, 4096);
+  a.rows = g.canvas;
+  a.vocab = g.vocab;
+  a.seed = ctx->seed;
+  a.block = ctx->block;
+  a.step = step;
+  a.tau = g.tau;
+  a.h_bound = g.h_bound;
+  a.max_steps = g.max_steps;
+  a.fixed_steps = g.fixed_steps;
+  a.canvas = ctx->canvas;
+  a.argmax = ctx->argmax;
+  a.prev_argmax = ctx->prev_argmax;
+  a.entropy = ctx->entropy;
+  a.conf = ctx->conf;
+  a.row_h = ctx->row_h;
+  a.locked = ctx->locked;
+  a.state = ctx->state;
+  a.ticket = ctx->ticket;
+  sampler_merge_kernel<<<g.canvas, 256, 0, S(stream)>>>(a);
+  DG_LAUNCHED();
+  return DG_OK;
+}
+
+int dg_commit_block(dg_ctx* ctx, int32_t* d_out_ids, int32_t* d_state, void* stream) {
+  DG_TRY(check_ctx(ctx));
+  const dg_config& g = ctx->cfg;
+  if (ctx->kv_len + g.canvas > g.kv_capacity) return fail(DG_ERR_CAPACITY, "cache full");
+  cudaStream_t st = S(stream);
+  if (d_out_ids)
+    DG_CUDA(cudaMemcpyAsync(d_out_ids, ctx->argmax, g.canvas * 4, cudaMemcpyDeviceToDevice, st));
+  if (d_state)
+    DG_CUDA(cudaMemcpyAsync(d_state, ctx->state, kStWords * 4, cudaMemcpyDeviceToDevice, st));
+  DG_TRY(run_forward(ctx, ctx->argmax, g.canvas, ctx->kv_len, 1, nullptr, st));
+  ctx->kv_len += g.canvas;
+  return DG_OK;
+}
+
+int dg_get_buffers(const dg_ctx* ctx, int32_t** canvas, int32_t** argmax, float** entropy,
+                   float** conf, int32_t** state) {
+  DG_TRY(check_ctx(ctx));
+  if (canvas) *canvas = ctx->canvas;
+  if (argmax) *argmax = ctx->argmax;
+  if (entropy) *entropy = ctx->entropy;
+  if (conf) *conf = ctx->conf;
+  if (state) *state = ctx->state;
+  return DG_OK;
+}
+
+int dg_check_device_status(dg_ctx* ctx, void* stream) {
+  DG_TRY(check_ctx(ctx));
+  DG_CUDA(cudaStreamSynchronize(S(stream)));
+  int err = 0;
+  DG_CUDA(cudaMemcpy(&err, ctx->err, 4, cudaMemcpyDeviceToHost));
+  if (err != 0) return fail(DG_ERR_TIMEOUT, "a device wait gave up (code %d)", err);
+  return DG_OK;
+}
+
+int dg_debug_logits(dg_ctx* ctx, float* d_logits, void* stream) {
+  DG_TRY(check_ctx(ctx));
+  if (!d_logits) return fail(DG_ERR_INVALID_ARG, "null logits");
+  return run_lm_head(ctx, d_logits, nullptr, S(stream));
+}
+
+int dg_debug_hidden(const dg_ctx* ctx, float** d_x) {
+  DG_TRY(check_ctx(ctx));
+  if (!d_x) return fail(DG_ERR_INVALID_ARG, "null output");
+  *d_x = ctx->x;
+  return DG_OK;
+}
+
+int dg_debug_layer(dg_ctx* ctx, int32_t layer, const float* d_x_in, float* d_x_out, int32_t n,
+                   int32_t causal, void* stream) {
+  DG_TRY(check_ctx(ctx));
+  const dg_config& g = ctx->cfg;
+  if (layer < 0 || layer >= g.n_layers) return fail(DG_ERR_INVALID_ARG, "bad layer %d", layer);
+  if (!d_x_in || !d_x_out || n < 1 || n > g.canvas)
+    return fail(DG_ERR_INVALID_ARG, "need x_in, x_out and 1 <= n <= canvas");
+  if (ctx->kv_len + n > g.kv_capacity) return fail(DG_ERR_CAPACITY, "cache full");
+  cudaStream_t st = S(stream);
+  DG_CUDA(cudaMemcpyAsync(ctx->x, d_x_in, static_cast<size_t>(n) * g.d_model * 4,
+                          cudaMemcpyDeviceToDevice, st));
+  const float* w = ctx->layers[layer].attn_norm;
+  if (ctx->bf16)
+    residual_norm_kernel<__nv_bfloat16><<<n, 256, 0, st>>>(
+        ctx->x, ctx->part, 0, 0, g.d_model, w, g.eps, static_cast<__nv_bfloat16*>(ctx->xn), nullptr);
+  else
+    residual_norm_kernel<float><<<n, 256, 0, st>>>(ctx->x, ctx->part, 0, 0, g.d_model, w, g.eps,
+                                                   static_cast<float*>(ctx->xn), nullptr);
+  DG_LAUNCHED();
+  const float* nn = (layer + 1 < g.n_layers) ? ctx->layers[layer + 1].attn_norm : ctx->final_norm;
+  DG_TRY(run_layer(ctx, layer, n, ctx->kv_len, causal, nn, nullptr, st));
+  DG_CUDA(cudaMemcpyAsync(d_x_out, ctx->x, static_cast<size_t>(n) * g.d_model * 4,
+                          cudaMemcpyDeviceToDevice, st));
+  return DG_OK;
+}
+
+// ---- standalone sampler ----------------------------------------------------------------
+static int sampler_chunk(int32_t dtype) { return dtype == DG_DTYPE_BF16 ? 8192 : 4096; }
+
+int dg_sampler_workspace_bytes(int32_t rows, int32_t vocab, size_t* bytes) {
+  if (rows < 1 || rows > 1024 || vocab < 2 || vocab % 8 || !bytes)
+    return fail(DG_ERR_INVALID_ARG, "need 1 <= rows <= 1024, vocab % 8 == 0");
+  const size_t nchunk = cdiv(vocab, 4096);  // upper bound over both dtypes
+  *bytes = align256(rows * nchunk * sizeof(StatPartial)) + 3 * align256(rows * 8) + 256;
+  return DG_OK;
+}
+
+static void sampler_views(void* ws, int rows, int vocab, StatPartial** part, int32_t** prev,
+                          double** row_h, int32_t** locked, int32_t** ticket) {
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  const size_t nchunk = cdiv(vocab, 4096);
+  *part = reinterpret_cast<StatPartial*>(b);
+  b += align256(rows * nchunk * sizeof(StatPartial));
+  *prev = reinterpret_cast<int32_t*>(b);
+  b += align256(rows * 8);
+  *row_h = reinterpret_cast<double*>(b);
+  b += align256(rows * 8);
+  *locked = reinterpret_cast<int32_t*>(b);
+  b += align256(rows * 8);
+  *ticket = reinterpret_cast<int32_t*>(b);
+}
+
+int dg_sampler_reset(int32_t rows, int32_t vocab, void* d_workspace, int32_t* d_state,
+                     void* stream) {
+  size_t bytes = 0;
+  DG_TRY(dg_sampler_workspace_bytes(rows, vocab, &bytes));
+  if (!d_workspace || !d_state) return fail(DG_ERR_INVALID_ARG, "null workspace or state");
+  DG_CUDA(cudaMemsetAsync(d_workspace, 0, bytes, S(stream)));
+  DG_CUDA(cudaMemsetAsync(d_state, 0, kStWords * 4, S(stream)));
+  return DG_OK;
+}
+
+int dg_sampler_step(const void* d_logits, int32_t dtype, int32_t rows, int32_t vocab, uint64_t seed,
+                    uint32_t block, uint32_t step, double tau, double h_bound, int32_t max_steps,
+                    int32_t fixed_steps, void* d_workspace, int32_t* d_canvas, int32_t* d_argmax,
+                    float* d_entropy, float* d_conf, int32_t* d_state, void* stream) {
+  size_t bytes = 0;
+  DG_TRY(dg_sampler_workspace_bytes(rows, vocab, &bytes));
+  if (!d_logits || !d_workspace || !d_canvas || !d_argmax || !d_entropy || !d_conf || !d_state)
+    return fail(DG_ERR_INVALID_ARG, "null pointer argument");
+  if (reinterpret_cast<uintptr_t>(d_logits) % 16)
+    return fail(DG_ERR_INVALID_ARG, "logits must be 16-byte aligned");
+  if (step < 1 || max_steps < 1 || fixed_steps < 0)
+    return fail(DG_ERR_INVALID_ARG, "bad step / max_steps / fixed_steps");
+  if (dtype != DG_DTYPE_BF16 && dtype != DG_DTYPE_FP32)
+    return fail(DG_ERR_INVALID_ARG, "dtype must be bf16 or fp32");
+  StatPartial* part;
+  int32_t *prev, *locked, *ticket;
+  double* row_h;
+  sampler_views(d_workspace, rows, vocab, &part, &prev, &row_h, &locked, &ticket);
+  cudaStream_t st = S(stream);
+  const int chunk = sampler_chunk(dtype);
+  const int nchunk = cdiv(vocab, chunk);
+  const int* done = d_state + kStDone;
+  if (dtype == DG_DTYPE_BF16)
+    logits_stats_kernel<__nv_bfloat16, 32><<<dim3(nchunk, rows), 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(d_logits), vocab, chunk, part, done);
+  else
+    logits_stats_kernel<float, 16><<<dim3(nchunk, rows), 256, 0, st>>>(
+        static_cast<const float*>(d_logits), vocab, chunk, part, done);
+  DG_LAUNCHED();
+  SamplerArgs a{};
+  a.partials = part;
+  a.nsplit = nchunk;
+  a.rows = rows;
+  a.vocab = vocab;
+  a.seed = seed;
+  a.block = block;
+  a.step = step;
+  a.tau = tau;
+  a.h_bound = h_bound;
+  a.max_steps = max_steps;
+  a.fixed_steps = fixed_steps;
+  a.canvas = d_canvas;
+  a.argmax = d_argmax;
+  a.prev_argmax = prev;
+  a.entropy = d_entropy;
+  a.conf = d_conf;
+  a.row_h = row_h;
+  a.locked = locked;
+  a.state = d_state;
+  a.ticket = ticket;
+  sampler_merge_kernel<<<rows, 256, 0, st>>>(a);
+  DG_LAUNCHED();
+  return DG_OK;
+}
+
+// ---- standalone attention --------------------------------------------------------------
+int dg_attention_workspace_bytes(int32_t n_heads, int32_t n_kv_heads, int32_t tq, int32_t n_keys,
+                                 size_t* bytes) {
+  if (n_heads < 1 || n_kv_heads < 1 || tq < 128 || tq % 128 || n_keys < 1 || !bytes)
+    return fail(DG_ERR_INVALID_ARG, "bad attention shape");
+  const int splits = std::max(1, cdiv(n_keys, 128));
+  *bytes = align256(static_cast<size_t>(splits) * n_heads * tq * 128 * 4) +
+           align256(static_cast<size_t>(splits) * n_heads * tq * 8) + 4 * 256;
+  return DG_OK;
+}
+
+int dg_canvas_attention(const void* d_q, const void* d_k, const void* d_vt, void* d_o,
+                        int32_t n_heads, int32_t n_kv_heads, int32_t t, int32_t tq, int32_t n_keys,
+                        int32_t ldk, int32_t causal_prefix, float scale, void* d_workspace,
+                        size_t workspace_bytes, void* stream) {
+  if (!d_q || !d_k || !d_vt || !d_o || !d_workspace) return fail(DG_ERR_INVALID_ARG, "null pointer");
+  if (n_heads < 1 || n_kv_heads < 1 || n_heads % n_kv_heads || t < 1 || tq < t || tq % 128 ||
+      n_keys < 1 || ldk < n_keys || ldk % 8)
+    return fail(DG_ERR_INVALID_ARG, "bad attention shape");
+  if (causal_prefix >= 0 && causal_prefix + t > n_keys)
+    return fail(DG_ERR_INVALID_ARG, "causal prefix + queries exceeds keys");
+  const int sms = num_sms();
+  const int group = n_heads / n_kv_heads;
+  const int m_tiles = group * tq / 128;
+  const int n_kv_tiles = cdiv(n_keys, 128);
+  int splits = std::max(1, std::min(16, sms / (m_tiles * n_kv_heads)));
+  splits = std::min(splits, n_kv_tiles);
+  const int tps = cdiv(n_kv_tiles, splits);
+  splits = cdiv(n_kv_tiles, tps);
+  const size_t o_bytes = align256(static_cast<size_t>(splits) * n_heads * tq * 128 * 4);
+  const size_t need = o_bytes + align256(static_cast<size_t>(splits) * n_heads * tq * 8) + 256;
+  if (workspace_bytes < need) return fail(DG_ERR_CAPACITY, "attention workspace too small");
+  uint8_t* ws = static_cast<uint8_t*>(d_workspace);
+  CUtensorMap tq_m, tk_m, tv_m;
+  DG_TRY(make_tmap(&tq_m, d_q, static_cast<uint64_t>(n_heads) * tq, 128, 128, 128));
+  DG_TRY(make_tmap(&tk_m, d_k, static_cast<uint64_t>(n_kv_heads) * ldk, 128, 128, 128));
+  DG_TRY(make_tmap(&tv_m, d_vt, static_cast<uint64_t>(n_kv_heads) * 128, ldk, ldk, 128));
+  AttnParams a{};
+  a.group = group;
+  a.tq = tq;
+  a.n_queries = t;
+  a.n_keys = n_keys;
+  a.causal_prefix = causal_prefix;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.tiles_per_split = tps;
+  a.q_row_base = 0;
+  a.k_row_base = 0;
+  a.ldk = ldk;
+  a.vt_row_base = 0;
+  a.n_heads = n_heads;
+  a.o_part = reinterpret_cast<float*>(ws);
+  a.ml_part = reinterpret_cast<float2*>(ws + o_bytes);
+  a.err = reinterpret_cast<int*>(ws + need - 256);
+  a.done = nullptr;
+  cudaStream_t st = S(stream);
+  DG_CUDA(cudaMemsetAsync(a.err, 0, 4, st));
+  DG_TRY(set_smem(attention_kernel, kAttnSmemBytes));
+  attention_kernel<<<dim3(m_tiles, n_kv_heads, splits), 192, kAttnSmemBytes, st>>>(tq_m, tk_m, tv_m,
+                                                                                  a);
+  DG_LAUNCHED();
+  attn_combine_kernel<__nv_bfloat16><<<dim3(t, n_heads), 128, 0, st>>>(
+      a.o_part, a.ml_part, splits, n_heads, tq, t, static_cast<__nv_bfloat16*>(d_o), nullptr);
+  DG_LAUNCHED();
+  return DG_OK;
+}
+
+// ---- standalone MoE --------------------------------------------------------------------
+namespace {
+struct MoePlan {
+  size_t off[12];
+  size_t total;
+  int split_r;
+  long long items_gu, items_d;
+};
+MoePlan moe_plan(int t, int d, int E, int k, int hid, int hs) {
+  MoePlan m{};
+  m.split_r = std::min(16, std::max(1, d / 64 / 4));
+  const long long chunks = E + (static_cast<long long>(t) * k + kGroupN - 1) / kGroupN;
+  m.items_gu = chunks * cdiv(2 * hid, 128);
+  m.items_d = chunks * cdiv(d, 128);
+  size_t sz[12];
+  sz[0] = static_cast<size_t>(m.split_r) * t * E * 4;  // router partials
+  sz[1] = static_cast<size_t>(t) * k * 4;              // ids (internal)
+  sz[2] = static_cast<size_t>(t) * k * 4;              // weights (internal)
+  sz[3] = (E + 1) * 4;                                 // offsets
+  sz[4] = static_cast<size_t>(t) * k * 4;              // perm
+  sz[5] = m.items_gu * 16;
+  sz[6] = m.items_d * 16;
+  sz[7] = 16;                                          // item counts + error word
+  sz[8] = static_cast<size_t>(t) * k * d * 2;          // x_perm
+  sz[9] = static_cast<size_t>(t) * k * hid * 2;        // h
+  sz[10] = align256(static_cast<size_t>(t) * std::max(hs, 1) * 2) +
+           static_cast<size_t>(t) * d * 4;  // hs, then y_shared at the next 256-byte boundary
+  sz[11] = static_cast<size_t>(t) * k * d * 4;         // y_slot
+  size_t o = 0;
+  for (int i = 0; i < 12; ++i) {
+    m.off[i] = o;
+    o += align256(std::max<size_t>(sz[i], 1));
+  }
+  m.total = o;
+  return m;
+}
+}  // namespace
+
+int dg_moe_workspace_bytes(int32_t t, int32_t d, int32_t n_experts, int32_t top_k, int32_t hidden,
+                           int32_t shared_hidden, size_t* bytes) {
+  if (t < 1 || d < 64 || d % 64 || n_experts < 1 || n_experts > 256 || top_k < 1 || top_k > 8 ||
+      top_k > n_experts || hidden < 64 || hidden % 64 || shared_hidden < 0 || shared_hidden % 64 ||
+      !bytes)
+    return fail(DG_ERR_INVALID_ARG, "bad MoE shape");
+  *bytes = moe_plan(t, d, n_experts, top_k, hidden, shared_hidden).total;
+  return DG_OK;
+}
+
+int dg_moe_ffn(const void* d_x, const float* d_residual, const void* d_wr, const void* d_w_gu,
+               const void* d_w_d, const void* d_ws_gu, const void* d_ws_d, float* d_y,
+               int32_t* d_ids, float* d_weights, float* d_router_logits, int32_t t, int32_t d,
+               int32_t n_experts, int32_t top_k, int32_t hidden, int32_t shared_hidden,
+               void* d_workspace, size_t workspace_bytes, void* stream) {
+  size_t need = 0;
+  DG_TRY(dg_moe_workspace_bytes(t, d, n_experts, top_k, hidden, shared_hidden, &need));
+  if (!d_x || !d_wr || !d_w_gu || !d_w_d || !d_y || !d_workspace)
+    return fail(DG_ERR_INVALID_ARG, "null pointer argument");
+  if (shared_hidden > 0 && (!d_ws_gu || !d_ws_d))
+    return fail(DG_ERR_INVALID_ARG, "shared expert weights missing");
+  if (workspace_bytes < need) return fail(DG_ERR_CAPACITY, "MoE workspace too small");
+  if (t > 4096) return fail(DG_ERR_UNSUPPORTED, "at most 4096 tokens per call");
+  const MoePlan m = moe_plan(t, d, n_experts, top_k, hidden, shared_hidden);
+  uint8_t* ws = static_cast<uint8_t*>(d_workspace);
+  float* rpart = reinterpret_cast<float*>(ws + m.off[0]);
+  int32_t* ids = reinterpret_cast<int32_t*>(ws + m.off[1]);
+  float* wts = reinterpret_cast<float*>(ws + m.off[2]);
+  int32_t* offs = reinterpret_cast<int32_t*>(ws + m.off[3]);
+  int32_t* perm = reinterpret_cast<int32_t*>(ws + m.off[4]);
+  int4* items_gu = reinterpret_cast<int4*>(ws + m.off[5]);
+  int4* items_d = reinterpret_cast<int4*>(ws + m.off[6]);
+  int32_t* icnt = reinterpret_cast<int32_t*>(ws + m.off[7]);
+  int* err = icnt + 2;
+  __nv_bfloat16* x_perm = reinterpret_cast<__nv_bfloat16*>(ws + m.off[8]);
+  __nv_bfloat16* hbuf = reinterpret_cast<__nv_bfloat16*>(ws + m.off[9]);
+  __nv_bfloat16* hsbuf = reinterpret_cast<__nv_bfloat16*>(ws + m.off[10]);
+  float* ysh = reinterpret_cast<float*>(ws + m.off[10] + align256(static_cast<size_t>(t) * std::max(shared_hidden, 1) * 2));
+  float* y_slot = reinterpret_cast<float*>(ws + m.off[11]);
+  const int sms = num_sms();
+  cudaStream_t st = S(stream);
+  DG_CUDA(cudaMemsetAsync(err, 0, 4, st));
+  CUtensorMap t_x32, t_wr, t_xp, t_wgu, t_h, t_wd, t_wsgu, t_hs, t_wsd;
+  DG_TRY(make_tmap(&t_x32, d_x, t, d, d, 32));
+  DG_TRY(make_tmap(&t_wr, d_wr, n_experts, d, d, 128));
+  DG_TRY(make_tmap(&t_xp, x_perm, static_cast<uint64_t>(t) * top_k, d, d, 32));
+  DG_TRY(make_tmap(&t_wgu, d_w_gu, static_cast<uint64_t>(n_experts) * 2 * hidden, d, d, 128));
+  DG_TRY(make_tmap(&t_h, hbuf, static_cast<uint64_t>(t) * top_k, hidden, hidden, 32));
+  DG_TRY(make_tmap(&t_wd, d_w_d, static_cast<uint64_t>(n_experts) * d, hidden, hidden, 128));
+  if (shared_hidden > 0) {
+    DG_TRY(make_tmap(&t_wsgu, d_ws_gu, 2ull * shared_hidden, d, d, 128));
+    DG_TRY(make_tmap(&t_hs, hsbuf, t, shared_hidden, shared_hidden, 32));
+    DG_TRY(make_tmap(&t_wsd, d_ws_d, d, shared_hidden, shared_hidden, 128));
+  }
+  // router
+  GemmParams pr = dense_params(n_experts, t, d, m.split_r, err, nullptr);
+  pr.out_f32 = rpart;
+  pr.ld_out = n_experts;
+  pr.split_stride = static_cast<long long>(t) * n_experts;
+  DG_TRY((launch_gemm<kDenseN, kDenseStages, kEpiPartialF32>(
+      t_wr, t_x32, pr, std::min(pr.m_tiles * pr.k_splits * pr.n_chunks, sms), st)));
+  router_topk_kernel<<<cdiv(t, 4), 128, 0, st>>>(rpart, m.split_r, pr.split_stride, t, n_experts,
+                                                 top_k, d_router_logits, ids, wts, nullptr);
+  DG_LAUNCHED();
+  RouteArgs ra{};
+  ra.ids = ids;
+  ra.n_slots = t * top_k;
+  ra.n_experts = n_experts;
+  ra.offsets = offs;
+  ra.perm = perm;
+  ra.items_gu = items_gu;
+  ra.items_d = items_d;
+  ra.counts = icnt;
+  ra.m_tiles_gu = cdiv(2 * hidden, 128);
+  ra.m_tiles_d = cdiv(d, 128);
+  ra.n_chunk = kGroupN;
+  ra.done = nullptr;
+  moe_route_kernel<<<1, 1024, 0, st>>>(ra);
+  DG_LAUNCHED();
+  gather_rows_kernel<<<t * top_k, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(d_x), perm, top_k,
+                                                d, x_perm, nullptr);
+  DG_LAUNCHED();
+  GemmParams pg{};
+  pg.items = items_gu;
+  pg.item_count = icnt;
+  pg.a_rows_per_group = 2 * hidden;
+  pg.kb_total = d / 64;
+  pg.m_valid = 2 * hidden;
+  pg.out_bf16 = hbuf;
+  pg.ld_out = hidden;
+  pg.err = err;
+  DG_TRY((launch_gemm<kGroupN, kGroupStages, kEpiGluBf16>(t_wgu, t_xp, pg, sms, st)));
+  GemmParams pd{};
+  pd.items = items_d;
+  pd.item_count = icnt + 1;
+  pd.a_rows_per_group = d;
+  pd.kb_total = hidden / 64;
+  pd.m_valid = d;
+  pd.out_f32 = y_slot;
+  pd.ld_out = d;
+  pd.perm = perm;
+  pd.scale = wts;
+  pd.err = err;
+  DG_TRY((launch_gemm<kGroupN, kGroupStages, kEpiScatterF32>(t_wd, t_h, pd, sms, st)));
+  const float* ysh_ptr = nullptr;
+  if (shared_hidden > 0) {
+    GemmParams p = dense_params(2 * shared_hidden, t, d, 1, err, nullptr);
+    p.out_bf16 = hsbuf;
+    p.ld_out = shared_hidden;
+    DG_TRY((launch_gemm<kDenseN, kDenseStages, kEpiGluBf16>(
+        t_wsgu, t_x32, p, std::min(p.m_tiles * p.n_chunks, sms), st)));
+    GemmParams q = dense_params(d, t, shared_hidden, 1, err, nullptr);
+    q.out_f32 = ysh;
+    q.ld_out = d;
+    DG_TRY((launch_gemm<kDenseN, kDenseStages, kEpiScatterF32>(
+        t_wsd, t_hs, q, std::min(q.m_tiles * q.n_chunks, sms), st)));
+    ysh_ptr = ysh;
+  }
+  if (d_residual)
+    DG_CUDA(cudaMemcpyAsync(d_y, d_residual, static_cast<size_t>(t) * d * 4,
+                            cudaMemcpyDeviceToDevice, st));
+  else
+    DG_CUDA(cudaMemsetAsync(d_y, 0, static_cast<size_t>(t) * d * 4, st));
+  moe_combine_norm_kernel<__nv_bfloat16><<<t, 256, 0, st>>>(d_y, y_slot, top_k, ysh_ptr, d, nullptr,
+                                                            0.f, nullptr, nullptr);
+  DG_LAUNCHED();
+  if (d_ids)
+    DG_CUDA(cudaMemcpyAsync(d_ids, ids, static_cast<size_t>(t) * top_k * 4,
+                            cudaMemcpyDeviceToDevice, st));
+  if (d_weights)
+    DG_CUDA(cudaMemcpyAsync(d_weights, wts, static_cast<size_t>(t) * top_k * 4,
+                            cudaMemcpyDeviceToDevice, st));
+  return DG_OK;
+}
+
+}  // extern "C"

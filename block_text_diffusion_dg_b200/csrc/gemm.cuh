@@ -1,0 +1,442 @@
+// gemm.cuh -- tcgen05 GEMMs of the denoise step.
+//
+// gemm_swapab_kernel: D[r, j] = sum_k W[a_row + r, k] * X[b_row + j, k] with the weight tile
+// as the UMMA "A" operand (M = 128 rows) and the token tile as "B" (N = n tokens, 16..MAXN).
+// Weights stream through shared memory exactly once per tile; the few tokens (256 on a
+// canvas, ~16 per expert) ride along as the narrow N side.  One CTA per SM, three roles:
+//   warp 0  : TMA producer (one elected thread) filling a STAGES-deep ring of 64-wide K slabs
+//   warp 1  : UMMA issuer (one elected thread), fp32 accumulators double-buffered in TMEM
+//   warps 2-5: epilogue, TMEM lane quarter (warp % 4), one accumulator row per thread.
+// Work items are either arithmetic (dense layers, optional split-K) or a device-built list
+// (grouped experts, one item per (expert, 128-row tile, token chunk)).
+//
+// lmhead_kernel: logits tile = X[256 tokens] * E[256 vocab rows]^T (two M=128 token tiles,
+// N = 256 vocab) with the epilogue reducing every row of the tile straight from TMEM to the
+// softmax statistics (max, argmax, sum e^(x-m), sum e^(x-m)(x-m)); logits never reach HBM.
+#pragma once
+#include "dg_common.cuh"
+#include "sampler.cuh"
+
+namespace dg {
+
+enum EpiMode : int { kEpiPartialF32 = 0, kEpiGluBf16 = 1, kEpiScatterF32 = 2 };
+
+struct GemmParams {
+  // dense items: it -> (m tile, k split, n chunk)
+  int m_tiles, k_splits, n_chunks, n_total, n_chunk, a_row_base, b_row_base;
+  // grouped items: device list of (group, m tile, first token row, n tokens)
+  const int4* items;
+  const int* item_count;
+  int a_rows_per_group;
+  int kb_total;  // K / 64
+  int m_valid;   // rows of A per group that are real (epilogue guard)
+  // epilogue
+  float* out_f32;
+  __nv_bfloat16* out_bf16;
+  long long ld_out;
+  long long split_stride;
+  const int* perm;
+  const float* scale;
+  int* err;
+  const int* done;
+};
+
+struct GemmItem {
+  int a_row, b_row, n, kb0, kb1, r_base, aux;
+};
+
+DG_DEV GemmItem gemm_item(const GemmParams& p, int it) {
+  GemmItem w;
+  if (p.items == nullptr) {
+    const int mt = it % p.m_tiles;
+    const int rest = it / p.m_tiles;
+    const int split = rest % p.k_splits;
+    const int nc = rest / p.k_splits;
+    w.r_base = mt * 128;
+    w.a_row = p.a_row_base + w.r_base;
+    w.b_row = p.b_row_base + nc * p.n_chunk;
+    w.n = min(p.n_chunk, p.n_total - nc * p.n_chunk);
+    w.kb0 = split * p.kb_total / p.k_splits;
+    w.kb1 = (split + 1) * p.kb_total / p.k_splits;
+    w.aux = split;
+  } else {
+    const int4 e = p.items[it];
+    w.r_base = e.y * 128;
+    w.a_row = e.x * p.a_rows_per_group + w.r_base;
+    w.b_row = e.z;
+    w.n = e.w;
+    w.kb0 = 0;
+    w.kb1 = p.kb_total;
+    w.aux = e.x;
+  }
+  return w;
+}
+
+DG_DEV int gemm_item_count(const GemmParams& p) {
+  return p.items ? *reinterpret_cast<const volatile int*>(p.item_count)
+                 : p.m_tiles * p.k_splits * p.n_chunks;
+}
+
+template <int MAXN, int STAGES>
+struct GemmCfg {
+  static constexpr int kABytes = 128 * 128;   // 128 rows x 64 bf16
+  static constexpr int kBBytes = MAXN * 128;  // MAXN rows x 64 bf16
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kTmemCols = 2 * MAXN;
+  static constexpr int kSmemBytes = STAGES * kStageBytes + 1024 + 256;
+  static_assert(MAXN % 32 == 0 && MAXN >= 32 && MAXN <= 256, "MAXN");
+};
+
+template <int EPI>
+DG_DEV void gemm_epilogue_chunk(const GemmParams& p, const GemmItem& w, const float (&v)[32],
+                                int c, int r) {
+  const int row = w.r_base + r;  // row inside the group (output feature / gate-up row)
+  if constexpr (EPI == kEpiPartialF32) {
+    if (row < p.m_valid) {
+      float* o = p.out_f32 + static_cast<long long>(w.aux) * p.split_stride + row;
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (c + i < w.n) o[static_cast<long long>(w.b_row + c + i) * p.ld_out] = v[i];
+    }
+  } else if constexpr (EPI == kEpiGluBf16) {
+    // rows come in (gate, up) pairs on adjacent lanes: lane 2u has gate unit u, 2u+1 up unit u
+    const bool gate_lane = (lane_id() & 1) == 0;
+    const int unit = row >> 1;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float other = __shfl_xor_sync(0xffffffffu, v[i], 1);
+      if (((i >> 4) & 1) == (gate_lane ? 0 : 1) && c + i < w.n && row < p.m_valid) {
+        const float g = gate_lane ? v[i] : other;
+        const float u = gate_lane ? other : v[i];
+        const float h = g / (1.0f + __expf(-g)) * u;
+        p.out_bf16[static_cast<long long>(w.b_row + c + i) * p.ld_out + unit] =
+            __float2bfloat16_rn(h);
+      }
+    }
+  } else {  // kEpiScatterF32
+    if (row < p.m_valid) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        if (c + i < w.n) {
+          const int src = w.b_row + c + i;
+          const int dst = p.perm ? p.perm[src] : src;
+          const float s = p.scale ? p.scale[dst] : 1.0f;
+          p.out_f32[static_cast<long long>(dst) * p.ld_out + row] = v[i] * s;
+        }
+      }
+    }
+  }
+}
+
+template <int MAXN, int STAGES, int EPI>
+__global__ void __launch_bounds__(192, 1)
+    gemm_swapab_kernel(const __grid_constant__ CUtensorMap tm_a,
+                       const __grid_constant__ CUtensorMap tm_b, const GemmParams p) {
+  using C = GemmCfg<MAXN, STAGES>;
+  if (block_done(p.done)) return;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * C::kStageBytes);
+  uint64_t* empty = full + STAGES;
+  uint64_t* acc_full = empty + STAGES;
+  uint64_t* acc_empty = acc_full + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  const int warp = threadIdx.x >> 5;
+
+  if (warp == 0 && lane_id() == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 128);
+    }
+    fence_barrier_init();
+    tma_prefetch_desc(&tm_a);
+    tma_prefetch_desc(&tm_b);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const int n_items = gemm_item_count(p);
+
+  if (warp == 0) {
+    if (elect_one()) {
+      const uint64_t pol_a = policy_evict_first();
+      const uint64_t pol_b = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+        const GemmItem w = gemm_item(p, it);
+        const int nbox = (w.n + 31) >> 5;
+        const uint32_t bytes = C::kABytes + nbox * 32 * 128;
+        for (int kb = w.kb0; kb < w.kb1; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, p.err)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + stage * C::kStageBytes;
+          uint8_t* sb = sa + C::kABytes;
+          mbar_arrive_expect_tx(&full[stage], bytes);
+          tma_load_2d(&tm_a, &full[stage], sa, kb * 64, w.a_row, pol_a);
+          for (int bx = 0; bx < nbox; ++bx)
+            tma_load_2d(&tm_b, &full[stage], sb + bx * 4096, kb * 64, w.b_row + bx * 32, pol_b);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (elect_one()) {
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+        const GemmItem w = gemm_item(p, it);
+        const uint32_t idesc = idesc_bf16_f32(128, (w.n + 15) & ~15);
+        if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, p.err)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * MAXN;
+        for (int kb = w.kb0; kb < w.kb1; ++kb) {
+          if (!mbar_wait(&full[stage], phase, p.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * C::kStageBytes);
+          const uint64_t da = sdesc_sw128(sa);
+          const uint64_t db = sdesc_sw128(sa + C::kABytes);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            umma_bf16(d_tmem, da + 2 * k, db + 2 * k, idesc, (kb > w.kb0 || k > 0) ? 1u : 0u);
+          umma_commit(&empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        umma_commit(&acc_full[acc]);
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+    }
+  } else {
+    const int q = warp & 3;
+    const int r = q * 32 + lane_id();
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
+      const GemmItem w = gemm_item(p, it);
+      if (!mbar_wait(&acc_full[acc], acc_phase, p.err)) break;
+      tc_fence_after();
+      const uint32_t t_row = tmem_base + acc * MAXN + (static_cast<uint32_t>(q * 32) << 16);
+      for (int c = 0; c < w.n; c += 32) {
+        float v[32];
+        tmem_ld32(t_row + c, v);
+        gemm_epilogue_chunk<EPI>(p, w, v, c, r);
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[acc]);
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+struct LmHeadParams {
+  int n_tokens;   // valid token rows (<= 256)
+  int n_vtiles;   // vocab / 256
+  int kb_total;   // d / 64
+  StatPartial* partials;  // [n_tokens, n_vtiles]
+  float* logits;          // debug: [n_tokens, vocab] when not null (statistics skipped)
+  int vocab;
+  int* err;
+  const int* done;
+};
+
+constexpr int kLmStages = 3;
+constexpr int kLmStageBytes = 2 * 16384 + 32768;  // two token tiles + one 256-row vocab tile
+constexpr int kLmSmemBytes = kLmStages * kLmStageBytes + 1024 + 256;
+
+template <bool kStats>
+__global__ void __launch_bounds__(192, 1)
+    lmhead_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_e,
+                  const LmHeadParams p) {
+  if (block_done(p.done)) return;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kLmStages * kLmStageBytes);
+  uint64_t* empty = full + kLmStages;
+  uint64_t* acc_full = empty + kLmStages;
+  uint64_t* acc_empty = acc_full + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_empty + 1);
+  const int warp = threadIdx.x >> 5;
+  const int n_ttiles = (p.n_tokens + 127) >> 7;
+
+  if (warp == 0 && lane_id() == 0) {
+    for (int s = 0; s < kLmStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 128);
+    fence_barrier_init();
+    tma_prefetch_desc(&tm_x);
+    tma_prefetch_desc(&tm_e);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    if (elect_one()) {
+      const uint64_t pol_x = policy_evict_last();
+      const uint64_t pol_e = policy_evict_first();
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int vt = blockIdx.x; vt < p.n_vtiles && ok; vt += gridDim.x) {
+        for (int kb = 0; kb < p.kb_total; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, p.err)) {
+            ok = false;
+            break;
+          }
+          uint8_t* s0 = smem + stage * kLmStageBytes;
+          mbar_arrive_expect_tx(&full[stage], n_ttiles * 16384 + 32768);
+          for (int tt = 0; tt < n_ttiles; ++tt)
+            tma_load_2d(&tm_x, &full[stage], s0 + tt * 16384, kb * 64, tt * 128, pol_x);
+          tma_load_2d(&tm_e, &full[stage], s0 + 32768, kb * 64, vt * 256, pol_e);
+          if (++stage == kLmStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (elect_one()) {
+      int stage = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      const uint32_t idesc = idesc_bf16_f32(128, 256);
+      bool ok = true;
+      for (int vt = blockIdx.x; vt < p.n_vtiles && ok; vt += gridDim.x) {
+        if (!mbar_wait(acc_empty, acc_phase ^ 1u, p.err)) break;
+        tc_fence_after();
+        for (int kb = 0; kb < p.kb_total; ++kb) {
+          if (!mbar_wait(&full[stage], phase, p.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t s0 = smem_u32(smem + stage * kLmStageBytes);
+          const uint64_t de = sdesc_sw128(s0 + 32768);
+          for (int tt = 0; tt < n_ttiles; ++tt) {
+            const uint64_t dx = sdesc_sw128(s0 + tt * 16384);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              umma_bf16(tmem_base + tt * 256, dx + 2 * k, de + 2 * k, idesc,
+                        (kb > 0 || k > 0) ? 1u : 0u);
+          }
+          umma_commit(&empty[stage]);
+          if (++stage == kLmStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        umma_commit(acc_full);
+        acc_phase ^= 1u;
+      }
+    }
+  } else {
+    const int q = warp & 3;
+    const int r = q * 32 + lane_id();
+    uint32_t acc_phase = 0;
+    for (int vt = blockIdx.x; vt < p.n_vtiles; vt += gridDim.x) {
+      if (!mbar_wait(acc_full, acc_phase, p.err)) break;
+      tc_fence_after();
+      for (int tt = 0; tt < n_ttiles; ++tt) {
+        const int tok = tt * 128 + r;
+        const uint32_t t_row = tmem_base + tt * 256 + (static_cast<uint32_t>(q * 32) << 16);
+        if constexpr (kStats) {
+          float m = -INFINITY;
+          int a = 0;
+          for (int c = 0; c < 256; c += 32) {
+            float v[32];
+            tmem_ld32(t_row + c, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (v[i] > m) {
+                m = v[i];
+                a = c + i;
+              }
+          }
+          float s = 0.f, u = 0.f;
+          for (int c = 0; c < 256; c += 32) {
+            float v[32];
+            tmem_ld32(t_row + c, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float d = v[i] - m;
+              const float e = __expf(d);
+              s += e;
+              u = fmaf(e, d, u);
+            }
+          }
+          if (tok < p.n_tokens)
+            p.partials[static_cast<long long>(tok) * p.n_vtiles + vt] =
+                StatPartial{m, s, u, vt * 256 + a};
+        } else {
+          for (int c = 0; c < 256; c += 32) {
+            float v[32];
+            tmem_ld32(t_row + c, v);
+            if (tok < p.n_tokens) {
+              float4* dst = reinterpret_cast<float4*>(
+                  p.logits + static_cast<long long>(tok) * p.vocab + vt * 256 + c);
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(acc_empty);
+      acc_phase ^= 1u;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+}  // namespace dg

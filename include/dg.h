@@ -1,0 +1,237 @@
+/*
+ * dg.h -- C ABI of libdg, the B200 (sm_100a) denoise path for block text diffusion.
+ *
+ * What the path computes (sources, all prose web pages; no code is printed on them):
+ *  [canvas]  alphalab.site, "DiffusionGemma: 256-token Canvas and a local A/B test",
+ *            section "how the 256-token canvas turns noise into text", steps 1-4:
+ *            causal prompt encode into a reusable KV cache; a canvas of ids drawn
+ *            uniformly from the whole vocabulary; repeated denoising where confident
+ *            tokens stay and uncertain ones are re-randomised, at most 48 steps, stopping
+ *            when mean canvas entropy < 0.005 and the argmax prediction is identical on two
+ *            consecutive steps; commit of the converged block to the KV cache.
+ *  [uniform] k7ail.com (Arabic rendering of the MarkTechPost launch article), section
+ *            "how text diffusion works": uniform-state diffusion, bidirectional attention
+ *            over the whole canvas while denoising, re-noising of tokens whose confidence
+ *            drops.
+ *  [arch]    same article, section "architecture": causal prefill writes the KV cache,
+ *            bidirectional denoise; block-autoregressive diffusion commits each block to the
+ *            KV cache; Gemma 4 26B-A4B mixture-of-experts backbone.
+ *  [course]  ai-directories.com course outline, part 2 tables 2.1 (lock high-confidence
+ *            tokens first) and 2.2 (MoE 26B total, 3.8B active).
+ *  [philox]  Salmon et al., "Parallel random numbers: as easy as 1, 2, 3" (SC'11).
+ *
+ * Conventions for every entry point:
+ *  - All pointers named d_* are DEVICE pointers owned by the caller; the library keeps
+ *    raw copies and never frees them.  Host pointers are only read during the call.
+ *  - `stream` is a cudaStream_t passed as void*; every call only enqueues work on it and
+ *    returns without synchronising.  NULL means the legacy default stream.
+ *  - Return value: DG_OK (0) or a negative DG_ERR_* code.  Argument checks run before any
+ *    launch, so a failed check enqueues nothing.  dg_last_error() gives a text for the
+ *    most recent failure on the calling thread.
+ *  - Tensors are dense row-major; shapes are written [outer, ..., inner].
+ *  - bf16 is IEEE binary32's upper half; "bf16 config" stores weights, Q/K/V, the KV cache
+ *    and activations between kernels in bf16 (round-to-nearest-even), keeps the residual
+ *    stream, router logits and softmax statistics in fp32, and accumulates in fp32.  The
+ *    "fp32 config" stores everything in fp32.
+ */
+#ifndef DG_H_
+#define DG_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DG_API __attribute__((visibility("default")))
+#else
+#define DG_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  DG_OK = 0,
+  DG_ERR_INVALID_ARG = -1, /* null pointer, bad size or shape, misaligned pointer */
+  DG_ERR_CAPACITY = -2,    /* KV cache or workspace too small for the request */
+  DG_ERR_CUDA = -3,        /* a CUDA call or launch failed; text in dg_last_error() */
+  DG_ERR_TIMEOUT = -4,     /* a device wait gave up (read by dg_check_device_status) */
+  DG_ERR_UNSUPPORTED = -5  /* shape outside what the kernels implement */
+};
+
+enum { DG_DTYPE_BF16 = 0, DG_DTYPE_FP32 = 1 };
+
+/* Model and decode configuration.  Shapes follow the pages' model ([course], [arch]). */
+typedef struct dg_config {
+  int32_t n_layers;
+  int32_t d_model;        /* bf16: multiple of 64 */
+  int32_t n_heads;        /* query heads Hq */
+  int32_t n_kv_heads;     /* key/value heads Hkv; Hq % Hkv == 0 (grouped-query attention) */
+  int32_t head_dim;       /* bf16: 128; fp32: even, <= 128 */
+  int32_t n_experts;      /* E */
+  int32_t top_k;          /* k <= min(E, 8) */
+  int32_t expert_hidden;  /* h; bf16: multiple of 64 */
+  int32_t shared_hidden;  /* hs (0 = no shared expert); bf16: multiple of 64 */
+  int32_t vocab;          /* V; bf16: multiple of 256 */
+  int32_t canvas;         /* canvas length T; 256 in the pages ([canvas]); 1..256 */
+  int32_t kv_capacity;    /* positions the caller's KV cache holds (multiple of 8) */
+  int32_t dtype;          /* DG_DTYPE_BF16 or DG_DTYPE_FP32 */
+  float eps;              /* RMSNorm epsilon (1e-6) */
+  float rope_theta;       /* RoPE base (10000) */
+  double tau;             /* lock threshold on max-probability confidence (0.9) */
+  double h_bound;         /* mean-entropy stop bound in nats (0.005, [canvas] step 3) */
+  int32_t max_steps;      /* adaptive step cap (48, [canvas] step 3) */
+  int32_t fixed_steps;    /* > 0: fixed-step mode, exactly this many steps; 0: adaptive */
+} dg_config;
+
+/* Per-layer weights, all device pointers, dtype = config dtype unless noted.
+ * Gate and up projections are stored row-interleaved: row 2j is gate unit j, row 2j+1 is
+ * up unit j. */
+typedef struct dg_layer_weights {
+  const float* attn_norm; /* fp32 [d] */
+  const void* wqkv;       /* [(Hq + 2 Hkv) * hd, d]: q heads, then k heads, then v heads */
+  const void* wo;         /* [d, Hq * hd] */
+  const float* ffn_norm;  /* fp32 [d] */
+  const void* wr;         /* router [E, d] */
+  const void* w_gu;       /* experts gate/up [E, 2h, d] */
+  const void* w_d;        /* experts down [E, d, h] */
+  const void* ws_gu;      /* shared expert gate/up [2hs, d], or NULL */
+  const void* ws_d;       /* shared expert down [d, hs], or NULL */
+} dg_layer_weights;
+
+typedef struct dg_weights {
+  const void* embed;              /* tied embedding / LM head [V, d] */
+  const float* final_norm;        /* fp32 [d] */
+  const dg_layer_weights* layers; /* HOST array of n_layers entries (copied by dg_create) */
+} dg_weights;
+
+/* Device-side decode state words (int32), readable by the caller after a block. */
+enum {
+  DG_STATE_DONE = 0,        /* 1 once the block stopped (adaptive) or ran its fixed steps */
+  DG_STATE_STOP_STEP = 1,   /* step whose argmax is committed */
+  DG_STATE_WOULD_STOP = 2,  /* first step meeting the stop rule, 0 if none yet */
+  DG_STATE_STEPS_RUN = 3,   /* sampler updates applied in this block */
+  DG_STATE_LOCKED = 4,      /* positions locked by the last update */
+  DG_STATE_ERROR = 5,       /* nonzero: a device wait timed out (DG_ERR_TIMEOUT) */
+  DG_STATE_WORDS = 16
+};
+
+typedef struct dg_ctx dg_ctx;
+
+/* ---- model context ---------------------------------------------------------------- */
+
+/* Bytes of the KV cache and of the scratch workspace the caller must allocate for cfg.
+ * KV cache layout: K [L, Hkv, cap, hd] followed by V transposed [L, Hkv, hd, cap]. */
+DG_API int dg_workspace_bytes(const dg_config* cfg, size_t* kv_bytes, size_t* scratch_bytes);
+
+/* Bind weights and caller-allocated buffers (kv: kv_bytes, scratch: scratch_bytes, both
+ * 256-byte aligned).  Builds the TMA descriptors, zero-fills kv and scratch on `stream`,
+ * and sets the cache length to 0.  Allocates no device memory. */
+DG_API int dg_create(const dg_config* cfg, const dg_weights* w, void* d_kv, void* d_scratch,
+              void* stream, dg_ctx** out);
+DG_API void dg_destroy(dg_ctx* ctx);
+
+/* Committed cache length (host-side counter advanced by dg_kv_append / dg_commit_block). */
+DG_API int32_t dg_kv_length(const dg_ctx* ctx);
+/* Forget committed positions >= length (0 <= length <= current length). */
+DG_API int dg_kv_truncate(dg_ctx* ctx, int32_t length);
+
+/* Causal encode ([canvas] step 1, [arch] prefill): run every layer over ids[0..n) at
+ * positions P..P+n-1 with a causal mask and append their K/V to the cache (P += n).
+ * d_ids: int32 [n], each in [0, V).  Processed in chunks of `canvas` tokens.
+ * DG_ERR_CAPACITY if P + n + canvas > kv_capacity (room for the next canvas is kept). */
+DG_API int dg_kv_append(dg_ctx* ctx, const int32_t* d_ids, int32_t n, void* stream);
+
+/* Fill the canvas with ids uniform over [0, V) ([canvas] step 2): Philox4x32-10 with
+ * counter (position, 0, block, 0) and key (seed lo32, seed hi32); id = floor(r0 V / 2^32).
+ * Resets the decode state words (done, steps, stop step). */
+DG_API int dg_canvas_init(dg_ctx* ctx, uint64_t seed, uint32_t block, void* stream);
+
+/* One denoise forward ([uniform], [canvas] step 3): embed the canvas, run every layer with
+ * bidirectional attention over [committed cache | canvas] (canvas K/V are written to the
+ * cache slots P..P+T-1 but P does not advance), final RMSNorm, and the LM head fused with
+ * per-row vocab-tile softmax statistics (logits are not written to memory).
+ * A no-op on the device once the block is done.  step is 1-based. */
+DG_API int dg_denoise_step(dg_ctx* ctx, uint32_t step, void* stream);
+
+/* Sampler and stop test for step `step` ([canvas] step 3, [uniform], [course] 2.1):
+ * merge the statistics to conf (max probability), entropy (nats) and argmax (lowest
+ * index on ties); next canvas id = argmax if conf >= tau else Philox draw with counter
+ * (position, step, block, 1); mean entropy and the two-step argmax equality decide the
+ * stop, all on the device.  A no-op once the block is done. */
+DG_API int dg_sample_update(dg_ctx* ctx, uint32_t step, void* stream);
+
+/* Commit ([canvas] step 4, [arch]): copy the stop step's argmax block to d_out_ids (int32
+ * [T], may be NULL), the decode state words to d_state (int32 [DG_STATE_WORDS], may be
+ * NULL), then causally re-encode the block into the cache (P += T). */
+DG_API int dg_commit_block(dg_ctx* ctx, int32_t* d_out_ids, int32_t* d_state, void* stream);
+
+/* Device buffers of the context (for inspection; owned by the caller's scratch):
+ * canvas int32 [T], argmax int32 [T], entropy fp32 [T], conf fp32 [T], state int32 [16]. */
+DG_API int dg_get_buffers(const dg_ctx* ctx, int32_t** canvas, int32_t** argmax, float** entropy,
+                   float** conf, int32_t** state);
+
+/* Blocking: synchronise `stream` and return DG_ERR_TIMEOUT if a device wait gave up. */
+DG_API int dg_check_device_status(dg_ctx* ctx, void* stream);
+
+/* ---- standalone operators (the same kernels the context runs) -------------------- */
+
+/* Sampler over given logits ([canvas] step 3): d_logits [rows, V] (dtype), one call per
+ * step.  d_state int32[DG_STATE_WORDS] and the workspace carry the stop test across
+ * calls; zero both (dg_sampler_reset) before step 1.  Outputs: d_canvas (next ids),
+ * d_argmax, d_entropy, d_conf, each [rows].  Requires V % 8 == 0, rows <= 1024. */
+DG_API int dg_sampler_workspace_bytes(int32_t rows, int32_t vocab, size_t* bytes);
+DG_API int dg_sampler_reset(int32_t rows, int32_t vocab, void* d_workspace, int32_t* d_state,
+                     void* stream);
+DG_API int dg_sampler_step(const void* d_logits, int32_t dtype, int32_t rows, int32_t vocab,
+                    uint64_t seed, uint32_t block, uint32_t step, double tau, double h_bound,
+                    int32_t max_steps, int32_t fixed_steps, void* d_workspace,
+                    int32_t* d_canvas, int32_t* d_argmax, float* d_entropy, float* d_conf,
+                    int32_t* d_state, void* stream);
+
+/* Canvas attention ([uniform], [arch]): bf16 q [Hq, Tq, 128] (head stride Tq), keys
+ * k [Hkv, ldk, 128] and values TRANSPOSED vt [Hkv, 128, ldk], keys 0..n_keys-1 used;
+ * causal_prefix < 0: no mask; >= 0: query t sees keys n <= causal_prefix + t.
+ * Output o bf16 [T, Hq*128].  Requires Tq % 128 == 0, T <= Tq, ldk % 8 == 0, n_keys >= 1. */
+DG_API int dg_attention_workspace_bytes(int32_t n_heads, int32_t n_kv_heads, int32_t tq,
+                                 int32_t n_keys, size_t* bytes);
+DG_API int dg_canvas_attention(const void* d_q, const void* d_k, const void* d_vt, void* d_o,
+                        int32_t n_heads, int32_t n_kv_heads, int32_t t, int32_t tq,
+                        int32_t n_keys, int32_t ldk, int32_t causal_prefix, float scale,
+                        void* d_workspace, size_t workspace_bytes, void* stream);
+
+/* Top-k routed MoE FFN ([course] 2.2, [arch]): x bf16 [T, d] (already normalised),
+ * router wr bf16 [E, d], experts w_gu [E, 2h, d] (row-interleaved gate/up), w_d [E, d, h],
+ * optional shared expert ws_gu [2hs, d], ws_d [d, hs] (NULL, hs = 0 for none).
+ * y fp32 [T, d] = (residual or 0) + sum over slots in order of w * expert(x) + shared(x).
+ * Router: softmax over all E, top-k lowest index on ties, weights renormalised over k.
+ * Optional outputs: ids int32 [T, k], weights fp32 [T, k], router logits fp32 [T, E]. */
+DG_API int dg_moe_workspace_bytes(int32_t t, int32_t d, int32_t n_experts, int32_t top_k,
+                           int32_t hidden, int32_t shared_hidden, size_t* bytes);
+DG_API int dg_moe_ffn(const void* d_x, const float* d_residual, const void* d_wr, const void* d_w_gu,
+               const void* d_w_d, const void* d_ws_gu, const void* d_ws_d, float* d_y,
+               int32_t* d_ids, float* d_weights, float* d_router_logits, int32_t t, int32_t d,
+               int32_t n_experts, int32_t top_k, int32_t hidden, int32_t shared_hidden,
+               void* d_workspace, size_t workspace_bytes, void* stream);
+
+/* ---- test exports ------------------------------------------------------------------ */
+
+/* Unfused LM head of the context on its current final hidden state: logits fp32 [T, V]
+ * from the same MMA core as the fused path (for parity of the statistics). */
+DG_API int dg_debug_logits(dg_ctx* ctx, float* d_logits, void* stream);
+/* Teacher-forced layer: x_out fp32 [n, d] = layer `layer` applied to the residual stream
+ * x_in fp32 [n, d] at positions P..P+n-1 (P = committed length) against that layer's cache.
+ * causal != 0 masks causally over the n tokens, 0 attends bidirectionally.  The n tokens'
+ * K/V are written to cache slots P..P+n-1 like a denoise step; P does not advance. */
+DG_API int dg_debug_layer(dg_ctx* ctx, int32_t layer, const float* d_x_in, float* d_x_out, int32_t n,
+                   int32_t causal, void* stream);
+/* Final hidden state (fp32 [T, d]) of the last denoise step, for LM-head checks. */
+DG_API int dg_debug_hidden(const dg_ctx* ctx, float** d_x);
+
+DG_API const char* dg_last_error(void);
+DG_API const char* dg_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DG_H_ */

@@ -1,0 +1,172 @@
+"""End-to-end parity of the model context: prefill, denoise steps, sampler, commit.
+
+Two models: the all-fp32 two-layer model (1e-4 tolerance, every step compared) and a small
+bf16 model with the production kernels' tile shapes (2e-2 tolerance, teacher-forced layers,
+LM-head statistics on identical logits, ragged prefill chunk, two committed blocks).
+"""
+import numpy as np
+import pytest
+import torch
+
+from dg_synth import SHAPES, model_weights, uniform_ids
+from oracle import model as om
+from oracle import sampler as osmp
+from oracle.numerics import round_bf16
+from tests._helpers import np64, rel_close, weights_to_np
+
+pytestmark = pytest.mark.gpu
+
+
+def _ocfg(shape, **kw):
+    s = SHAPES[shape]
+    return om.ModelConfig(**{k: s[k] for k in ("n_layers", "d_model", "n_heads", "n_kv_heads",
+                                               "head_dim", "n_experts", "top_k", "expert_hidden",
+                                               "shared_hidden", "vocab", "canvas", "storage")}, **kw)
+
+
+def _to_cuda(w):
+    def cv(t):
+        return None if t is None else t.cuda()
+    return dict(embed=cv(w["embed"]), final_norm=cv(w["final_norm"]),
+                layers=[{k: cv(v) for k, v in lw.items()} for lw in w["layers"]])
+
+
+def _kv_views(m, cfg):
+    """K [L, Hkv, cap, hd] and V^T [L, Hkv, hd, cap] views of the context's cache."""
+    dt = torch.float32 if cfg.dtype == 1 else torch.bfloat16
+    kv = m.kv.view(dt)
+    half = kv.numel() // 2
+    shp = (cfg.n_layers, cfg.n_kv_heads, cfg.kv_capacity, cfg.head_dim)
+    return kv[:half].view(shp), kv[half:].view(cfg.n_layers, cfg.n_kv_heads, cfg.head_dim,
+                                               cfg.kv_capacity)
+
+
+def _argmax_guarded(logits_ref, got, margin):
+    srt = -np.sort(-logits_ref, axis=1)[:, :2]
+    clear = (srt[:, 0] - srt[:, 1]) > margin
+    ref = np.argmax(logits_ref, axis=1)
+    return np.array_equal(got[clear], ref[clear]), clear.mean()
+
+
+def test_tiny_fp32_end_to_end():
+    """2-layer fp32 model, 128-token prompt, one canvas, 16 fixed steps, seed 0."""
+    from block_text_diffusion_dg_b200 import DiffusionModel, make_config
+    shape = SHAPES["tiny_fp32"]
+    w = model_weights("tiny_fp32", seed=0)
+    prompt = uniform_ids(shape["prompt"], shape["vocab"], seed=0)
+    cfg = make_config(shape, kv_capacity=1024, fixed_steps=16)
+    m = DiffusionModel(cfg, _to_cuda(w))
+    ocfg, ow = _ocfg("tiny_fp32"), weights_to_np(w)
+    _, blocks, ocache = om.decode(ocfg, ow, prompt.numpy(), 1, seed=0, fixed_steps=16)
+    ref_steps = blocks[0]["steps"]
+    m.kv_append(prompt.cuda())
+    k_gpu, vt_gpu = _kv_views(m, cfg)
+    torch.cuda.synchronize()
+    for l in range(cfg.n_layers):
+        ok, worst, _ = rel_close(np64(k_gpu[l, :, :128]), ocache.k[l][:, :128], 1e-4)
+        assert ok, ("prefill K", l, worst)
+        ok, worst, _ = rel_close(np64(vt_gpu[l, :, :, :128]).transpose(0, 2, 1), ocache.v[l][:, :128], 1e-4)
+        assert ok, ("prefill V", l, worst)
+    m.canvas_init(0, 0)
+    bufs = m.buffers()
+    torch.cuda.synchronize()
+    assert np.array_equal(bufs["canvas"].cpu().numpy(), ref_steps[0]["canvas_in"])
+    for t in range(1, 17):
+        m.denoise_step(t)
+        if t == 16:
+            logits = m.debug_logits()
+        m.sample_update(t)
+        torch.cuda.synchronize()
+        r = ref_steps[t - 1]
+        assert np.array_equal(bufs["canvas"].cpu().numpy(), r["canvas_out"]), t
+        assert np.max(np.abs(bufs["entropy"].cpu().numpy() - r["entropy"])) < 1e-5, t
+        ok, frac = _argmax_guarded(
+            om.denoise_logits(ocfg, ow, r["canvas_in"], _cache_prefix(ocache, 128)),
+            bufs["argmax"].cpu().numpy(), 1e-4) if t in (1, 16) else (True, 1.0)
+        assert ok and frac > 0.9, t
+    ref_logits = om.denoise_logits(ocfg, ow, ref_steps[15]["canvas_in"], _cache_prefix(ocache, 128))
+    ok, worst, _ = rel_close(np64(logits), ref_logits, 1e-4)
+    assert ok, worst
+    ids, st = m.commit_block()
+    torch.cuda.synchronize()
+    assert st.cpu().tolist()[:4] == [1, 16, 0, 16]
+    assert np.array_equal(ids.cpu().numpy(), bufs["argmax"].cpu().numpy())
+    assert m.kv_length == 128 + 256
+
+
+def _cache_prefix(cache, n):
+    c = om.KVCache()
+    c.k = [k[:, :n] for k in cache.k]
+    c.v = [v[:, :n] for v in cache.v]
+    return c
+
+
+def test_small_bf16_prefill_denoise_commit():
+    from block_text_diffusion_dg_b200 import DiffusionModel, make_config
+    shape = SHAPES["small_bf16"]
+    w = model_weights("small_bf16", seed=1, norm_jitter=0.1)
+    prompt = uniform_ids(shape["prompt"], shape["vocab"], seed=2)  # 320 = 256 + ragged 64
+    cfg = make_config(shape, kv_capacity=1024, fixed_steps=3)
+    m = DiffusionModel(cfg, _to_cuda(w))
+    ocfg, ow = _ocfg("small_bf16"), weights_to_np(w)
+    ocache = om.causal_encode(ocfg, ow, prompt.numpy(), om.KVCache())
+    m.kv_append(prompt.cuda())
+    assert m.kv_length == 320
+    k_gpu, vt_gpu = _kv_views(m, cfg)
+    torch.cuda.synchronize()
+    for l in range(cfg.n_layers):
+        ok, worst, nrel = rel_close(np64(k_gpu[l, :, :320]), ocache.k[l], 2e-2)
+        assert ok and nrel < 1e-2, ("prefill K", l, worst, nrel)
+        ok, worst, nrel = rel_close(np64(vt_gpu[l, :, :, :320]).transpose(0, 2, 1), ocache.v[l], 2e-2)
+        assert ok and nrel < 1e-2, ("prefill V", l, worst, nrel)
+    # one denoise step; teacher-force every layer from the oracle's own layer inputs
+    m.canvas_init(11, 0)
+    m.denoise_step(1)
+    logits = m.debug_logits()
+    m.sample_update(1)
+    bufs = m.buffers()
+    torch.cuda.synchronize()
+    canvas0 = osmp.canvas_init(11, 0, 256, shape["vocab"])
+    ref_logits, infos = om.denoise_logits(ocfg, ow, canvas0, ocache, keep_info=True)
+    ok, worst, nrel = rel_close(np64(logits), ref_logits, 3e-2 / 0.5)
+    assert np.max(np.abs(np64(logits) - ref_logits)) < 3e-2, np.max(np.abs(np64(logits) - ref_logits))
+    # statistics and argmax of the fused LM head equal the oracle's on the GPU's own logits
+    conf, ent, amax = osmp.row_stats(np64(logits))
+    assert np.array_equal(bufs["argmax"].cpu().numpy(), amax)
+    assert np.max(np.abs(bufs["entropy"].cpu().numpy() - ent)) < 1e-5
+    nxt, _ = osmp.sample_update(conf, amax, 11, 0, 1, shape["vocab"])
+    assert np.array_equal(bufs["canvas"].cpu().numpy(), nxt)
+    # teacher-forced layers
+    x = np.asarray(ow["embed"], dtype=np.float64)[canvas0].astype(np.float32).astype(np.float64)
+    pos = 320 + np.arange(256)
+    for l in range(cfg.n_layers):
+        x_ref, _, _, _ = om.layer_forward(ocfg, ow["layers"][l], x, pos, ocache.k[l], ocache.v[l],
+                                          causal=False)
+        x_gpu = m.debug_layer(l, torch.from_numpy(x.astype(np.float32)).cuda(), causal=False)
+        torch.cuda.synchronize()
+        ok, worst, nrel = rel_close(np64(x_gpu), x_ref, 2e-2)
+        assert ok and nrel < 5e-3, ("layer", l, worst, nrel)
+        x = x_ref
+    # finish the block, commit it, check the committed K slots against a teacher-forced commit
+    for t in (2, 3):
+        m.denoise_step(t)
+        m.sample_update(t)
+    ids, st = m.commit_block()
+    torch.cuda.synchronize()
+    ids_np = ids.cpu().numpy()
+    assert st.cpu().tolist()[:2] == [1, 3]
+    assert m.kv_length == 320 + 256
+    om.causal_encode(ocfg, ow, ids_np, ocache)
+    k_gpu, vt_gpu = _kv_views(m, cfg)
+    for l in range(cfg.n_layers):
+        ok, worst, nrel = rel_close(np64(k_gpu[l, :, 320:576]), ocache.k[l][:, 320:576], 2e-2)
+        assert ok and nrel < 1e-2, ("commit K", l, worst, nrel)
+    # second block runs against the longer history
+    m.canvas_init(11, 1)
+    for t in (1, 2, 3):
+        m.denoise_step(t)
+        m.sample_update(t)
+    ids2, st2 = m.commit_block()
+    torch.cuda.synchronize()
+    assert st2.cpu().tolist()[:2] == [1, 3] and m.kv_length == 320 + 512
+    m.check_device_status()
