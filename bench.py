@@ -1,0 +1,371 @@
+#!/usr/bin/env python
+"""Committed canvas tokens/s of block text diffusion on B200 (one JSON line on rank 0).
+
+Workload (the full block decode): a random-init 30-layer MoE decoder shaped like Gemma 4
+26B-A4B (d 2816, 16 q / 8 kv heads x 128, 128 experts top-8 SiLU-GLU 704 + shared 2112,
+tied vocab 262144, bf16), a 4,096-token uniform prompt prefilled into the KV cache once, then
+4 canvases of 256 tokens, 16 fixed denoise steps each (1,024 committed tokens).  One bench
+step is that whole 4-block decode (KV cache cut back to the prompt before each step).
+
+  value  : committed tokens / s over K timed steps, device time (CUDA events), max over ranks
+  e2e    : the same through the public API from pinned host buffers: prompt H2D, prefill,
+           4 blocks, committed ids + states D2H, all inside the timed region
+  roofline: the dominant kernel's launches timed with CUDA events on its own stream (a
+           profiled pass after the timed region) against the measured HBM copy bandwidth
+  cpu_baseline: the CPU oracle on one denoise layer + 1/16 of the LM head + the sampler,
+           extrapolated to the decode (rank 0, N = 1)
+
+Multi-GPU: every rank decodes its own sequence with its own weights ("replicas only": the
+one-canvas, batch-1 decode has no data-path exchange); value sums all ranks.
+"""
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+PROMPT, BLOCKS, FIXED_STEPS, CANVAS = 4096, 4, 16, 256
+WORKLOAD = ("full block decode: 30-layer MoE decoder (d 2816, 16/8 heads x 128, 128 experts "
+            "top-8 x 704 + shared 2112, vocab 262144, bf16, random init), 4096-token prompt "
+            "prefilled, 4 canvases x 256 tokens x 16 fixed denoise steps")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--roofline-kernel", default="expert_gate_up")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained"), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ---------------------------------------------------------------------------------------
+class Clocks:
+    """nvidia-smi sampling (200 ms) of this process's GPU during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.uuid = str(torch.cuda.get_device_properties(device).uuid)
+        if not self.uuid.startswith("GPU-"):
+            self.uuid = "GPU-" + self.uuid
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.p = None
+
+    def start(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", "-i", self.uuid, f"--query-gpu={self.Q}",
+                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.p.terminate()
+        self.p.wait()
+        self.f.flush()
+        rows = []
+        for line in open(self.f.name):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.f.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------------------
+def cpu_oracle_sample(seed=0):
+    """Time the CPU oracle on a bounded sample of the decode and extrapolate to tokens/s.
+
+    Sample: one bidirectional denoise layer over the 256-token canvas against a 4,096-token
+    history, the LM head over 1/16 of the vocabulary, and the sampler statistics over the full
+    vocabulary.  Extrapolation: a denoise step = 30 layers + 16 x LM-head slice + sampler; a
+    block = 16 steps + a causal commit (30 layers); 4 blocks = 1,024 tokens.
+    """
+    import numpy as np
+    from dg_synth import SHAPES
+    from oracle import model as om
+    from oracle import sampler as osmp
+    s = SHAPES["a4b"]
+    g = torch.Generator().manual_seed(seed)
+    d, hd, e, h, hs, v = (s["d_model"], s["head_dim"], s["n_experts"], s["expert_hidden"],
+                          s["shared_hidden"], s["vocab"])
+
+    def n(*shape, std=0.02):
+        return (torch.empty(shape).normal_(0, std, generator=g)).to(torch.bfloat16).float().numpy()
+
+    lw = dict(attn_norm=np.ones(d, np.float32), ffn_norm=np.ones(d, np.float32),
+              wqkv=n((s["n_heads"] + 2 * s["n_kv_heads"]) * hd, d), wo=n(d, s["n_heads"] * hd),
+              wr=n(e, d), w_gu=n(e, 2 * h, d), w_d=n(e, d, h), ws_gu=n(2 * hs, d), ws_d=n(d, hs))
+    cfg = om.ModelConfig(**{k: s[k] for k in ("n_layers", "d_model", "n_heads", "n_kv_heads",
+                                              "head_dim", "n_experts", "top_k", "expert_hidden",
+                                              "shared_hidden", "vocab", "canvas", "storage")})
+    x = n(CANVAS, d, std=1.0).astype(np.float64)
+    ck = n(s["n_kv_heads"], PROMPT, hd, std=1.0)
+    cv = n(s["n_kv_heads"], PROMPT, hd, std=1.0)
+    pos = PROMPT + np.arange(CANVAS)
+    t0 = time.perf_counter()
+    om.layer_forward(cfg, lw, x, pos, ck, cv, causal=False)
+    t_layer = time.perf_counter() - t0
+    emb = n(v // 16, d)
+    t0 = time.perf_counter()
+    logits = om.lm_head(cfg, dict(embed=emb, final_norm=np.ones(d)), x)
+    t_head = (time.perf_counter() - t0) * 16
+    full = np.tile(logits, (1, 16))
+    t0 = time.perf_counter()
+    osmp.row_stats(full)
+    t_samp = time.perf_counter() - t0
+    t_step = s["n_layers"] * t_layer + t_head + t_samp
+    t_decode = BLOCKS * (FIXED_STEPS * t_step + s["n_layers"] * t_layer)
+    sample_s = t_layer + t_head / 16 + t_samp
+    return dict(value=BLOCKS * CANVAS / t_decode, unit="tok/s", cores=len(os.sched_getaffinity(0)),
+                kind="oracle",
+                sample=(f"1 denoise layer ({t_layer:.2f} s) + LM head on V/16 ({t_head / 16:.2f} s) "
+                        f"+ sampler over V ({t_samp:.2f} s), extrapolated to 4 blocks x 16 steps "
+                        f"x 30 layers; sample wall {sample_s:.1f} s"),
+                sample_seconds=sample_s)
+
+
+# ---------------------------------------------------------------------------------------
+def run_reference(args, rank):
+    if rank != 0:
+        return
+    steps = []
+    for i in range(args.warmup + args.steps):
+        r = cpu_oracle_sample(seed=i)
+        if i >= args.warmup:
+            steps.append(r)
+    val = statistics.median(r["value"] for r in steps)
+    cb = dict(value=val, unit="tok/s", cores=steps[0]["cores"], kind="oracle",
+              sample=steps[0]["sample"])
+    out = dict(impl="reference", metric="committed canvas tokens/s", value=val, unit="tok/s",
+               n_gpus=args.gpus, steps=args.steps, warmup=args.warmup,
+               ms_per_step=1e3 * BLOCKS * CANVAS / val, higher_is_better=True, scaling="weak",
+               vs_baseline=None, dtype="f64", data="synthetic",
+               config=dict(workload=WORKLOAD, global_batch=1, seq_len=PROMPT + BLOCKS * CANVAS,
+                           parallelism="replicas"),
+               cpu_baseline=cb,
+               e2e=dict(value=val, unit="tok/s", h2d_bytes_per_step=0, d2h_bytes_per_step=0))
+    print(json.dumps(out), flush=True)
+
+
+def max_over_ranks(x, world, device=None):
+    """Max of a per-rank float over all ranks (identity for one rank)."""
+    if world <= 1:
+        return float(x)
+    import torch.distributed as dist
+    on_gpu = dist.get_backend() == "nccl"
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device if on_gpu else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(tokens_per_rank, world, ms_max):
+    """Whole-job tokens/s: every rank decodes its own sequence; time is the slowest rank's."""
+    return world * tokens_per_rank / (ms_max / 1e3)
+
+
+def decode(model, seed, out_ids, out_states, stream):
+    model.kv_truncate(PROMPT)
+    for b in range(BLOCKS):
+        model.canvas_init(seed, b, stream)
+        for t in range(1, FIXED_STEPS + 1):
+            model.denoise_step(t, stream)
+            model.sample_update(t, stream)
+        model.commit_block(out_ids[b * CANVAS:(b + 1) * CANVAS], out_states[b], stream)
+
+
+def run_ours(args, rank, world, local_rank):
+    from block_text_diffusion_dg_b200 import DiffusionModel, generate, make_config
+    from block_text_diffusion_dg_b200 import _lib as L
+    from dg_synth import SHAPES, model_weights, uniform_ids
+    import torch.distributed as dist
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    shape = SHAPES["a4b"]
+    cap = PROMPT + BLOCKS * CANVAS + CANVAS
+    cfg = make_config(shape, kv_capacity=cap, fixed_steps=FIXED_STEPS)
+    weights = model_weights("a4b", seed=1000 + rank, device=dev)
+    model = DiffusionModel(cfg, weights, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    prompt = uniform_ids(PROMPT, shape["vocab"], seed=rank).pin_memory()
+    prompt_dev = prompt.to(dev)
+    out_ids = torch.empty(BLOCKS * CANVAS, dtype=torch.int32, device=dev)
+    out_states = torch.empty(BLOCKS, L.STATE_WORDS, dtype=torch.int32, device=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # prefill once (timed separately)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    model.kv_append(prompt_dev, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    prefill_ms = e0.elapsed_time(e1)
+
+    for i in range(args.warmup):
+        decode(model, 100 + i, out_ids, out_states, stream)
+    model.check_device_status(stream)
+    clocks = Clocks(dev)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    n0 = L.lib().dg_launch_count()
+    e0.record(stream)
+    for i in range(args.steps):
+        decode(model, i, out_ids, out_states, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    n1 = L.lib().dg_launch_count()
+    barrier()
+    ck = clocks.stop()
+    ms_max = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    model.check_device_status(stream)
+    value = replica_throughput(args.steps * BLOCKS * CANVAS, world, ms_max)
+
+    # denoise step time on its own (16 steps of block 0)
+    model.kv_truncate(PROMPT)
+    model.canvas_init(7, 0, stream)
+    e0.record(stream)
+    for tt in range(1, FIXED_STEPS + 1):
+        model.denoise_step(tt, stream)
+        model.sample_update(tt, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    us_step = 1e3 * e0.elapsed_time(e1) / FIXED_STEPS
+
+    # profiled pass: the roofline kernel's launches timed on its stream
+    kind = L.KERNEL_KINDS[args.roofline_kernel]
+    n_pairs = shape["n_layers"] * FIXED_STEPS
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(2 * n_pairs)]
+    import ctypes as C
+    arr = (C.c_void_p * (2 * n_pairs))(*[C.c_void_p(ev.cuda_event) for ev in evs])
+    for ev in evs:
+        ev.record(stream)  # materialise the events before handing them to the library
+    torch.cuda.synchronize()
+    L.check(L.lib().dg_profile_kernel(kind, arr, n_pairs), "dg_profile_kernel")
+    model.kv_truncate(PROMPT)
+    model.canvas_init(8, 0, stream)
+    for tt in range(1, FIXED_STEPS + 1):
+        model.denoise_step(tt, stream)
+        model.sample_update(tt, stream)
+    torch.cuda.synchronize()
+    rec = L.lib().dg_profile_recorded()
+    L.check(L.lib().dg_profile_kernel(0, None, 0), "dg_profile_kernel")
+    durs = [evs[2 * i].elapsed_time(evs[2 * i + 1]) for i in range(rec)]
+    avg_ms = sum(durs) / max(1, len(durs))
+    hbm, tf_burst, tf_sust, src = peaks()
+    d, e, h, k = shape["d_model"], shape["n_experts"], shape["expert_hidden"], shape["top_k"]
+    slots = CANVAS * k
+    algo = {  # algorithmic bytes per launch (all 128 experts are routed at these shapes)
+        "expert_gate_up": e * 2 * h * d * 2 + slots * d * 2 + slots * h * 2,
+        "expert_down": e * d * h * 2 + slots * h * 2 + slots * d * 4,
+        "lm_head": shape["vocab"] * d * 2 + CANVAS * d * 2 + CANVAS * (shape["vocab"] // 256) * 16,
+    }
+    roof = None
+    if args.roofline_kernel in algo and rec:
+        achieved = algo[args.roofline_kernel] / (avg_ms / 1e3) / 1e9
+        roof = dict(kernel=args.roofline_kernel, bound="hbm", achieved=round(achieved, 1),
+                    peak=hbm, unit="GB/s", frac=round(achieved / hbm, 4), traffic=None,
+                    launches_timed=rec, avg_launch_us=round(avg_ms * 1e3, 2),
+                    algorithmic_bytes_per_launch=algo[args.roofline_kernel],
+                    peak_source=f"{src} (MEASURED_PEAKS.json hbm_gbs)")
+
+    # end to end through the public API, pinned host buffers in and out
+    host_ids = torch.empty(BLOCKS * CANVAS, dtype=torch.int32).pin_memory()
+    host_states = torch.empty(BLOCKS, L.STATE_WORDS, dtype=torch.int32).pin_memory()
+    e2e_ms = []
+    for i in range(1 + args.e2e_steps):
+        torch.cuda.synchronize()
+        barrier()
+        e0.record(stream)
+        dev_prompt = prompt.to(dev, non_blocking=True)
+        model.kv_truncate(0)
+        ids, states = generate(model, dev_prompt, BLOCKS, seed=500 + i, stream=stream)
+        host_ids.copy_(ids, non_blocking=True)
+        host_states.copy_(states, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if i > 0:
+            e2e_ms.append(e0.elapsed_time(e1))
+    e2e_val = replica_throughput(BLOCKS * CANVAS, world, max_over_ranks(max(e2e_ms), world, dev))
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        r = cpu_oracle_sample()
+        cpu = dict(value=r["value"], unit="tok/s", cores=r["cores"], kind="oracle", sample=r["sample"])
+    if rank == 0:
+        out = dict(metric="committed canvas tokens/s", value=round(value, 2), unit="tok/s",
+                   n_gpus=world, steps=args.steps, warmup=args.warmup,
+                   ms_per_step=round(ms_max / args.steps, 3), higher_is_better=True,
+                   scaling="weak", vs_baseline=None, dtype="bf16", data="synthetic",
+                   config=dict(workload=WORKLOAD, global_batch=world, seq_len=PROMPT + BLOCKS * CANVAS,
+                               parallelism=f"replicas x{world}",
+                               l2="inputs larger than L2: ~49 GB of weights streamed per denoise step"),
+                   us_per_denoise_step=round(us_step, 1), prefill_ms=round(prefill_ms, 2),
+                   roofline=roof, cpu_baseline=cpu,
+                   e2e=dict(value=round(e2e_val, 2), unit="tok/s",
+                            h2d_bytes_per_step=prompt.numel() * 4,
+                            d2h_bytes_per_step=host_ids.numel() * 4 + host_states.numel() * 4,
+                            includes="prompt H2D, 4096-token prefill, 4 blocks, ids D2H"),
+                   gpu_launches=int((n1 - n0) // args.steps), clocks=ck)
+        print(json.dumps(out), flush=True)
+    model.close()
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -11,6 +11,8 @@ DG_ERR = {-1: "DG_ERR_INVALID_ARG", -2: "DG_ERR_CAPACITY", -3: "DG_ERR_CUDA",
 DTYPE_BF16, DTYPE_FP32 = 0, 1
 STATE_DONE, STATE_STOP_STEP, STATE_WOULD_STOP, STATE_STEPS_RUN, STATE_LOCKED, STATE_ERROR = range(6)
 STATE_WORDS = 16
+KERNEL_KINDS = dict(expert_gate_up=0, expert_down=1, attention=2, lm_head=3, qkv=4,
+                    o_proj=5, sampler=6, shared_expert=7)
 
 
 class Config(C.Structure):
@@ -65,6 +67,10 @@ _PROTOS = {
     "dg_debug_logits": (C.c_int, [_P, _P, _P]),
     "dg_debug_layer": (C.c_int, [_P, _I, _P, _P, _I, _I, _P]),
     "dg_debug_hidden": (C.c_int, [_P, C.POINTER(_P)]),
+    "dg_debug_routing": (C.c_int, [_P, C.POINTER(_P), C.POINTER(_P), C.POINTER(_P)]),
+    "dg_launch_count": (C.c_uint64, []),
+    "dg_profile_kernel": (C.c_int, [_I, C.POINTER(_P), _I]),
+    "dg_profile_recorded": (C.c_int32, []),
     "dg_last_error": (C.c_char_p, []),
     "dg_version": (C.c_char_p, []),
 }

@@ -152,6 +152,16 @@ class DiffusionModel:
         return self._view(p.value, self.cfg.canvas * self.cfg.d_model, torch.float32).view(
             self.cfg.canvas, self.cfg.d_model)
 
+    def debug_routing(self, n=None):
+        """(ids [n, k], weights [n, k], router logits [n, E]) of the last layer run."""
+        n = self.cfg.canvas if n is None else n
+        ps = [C.c_void_p() for _ in range(3)]
+        check(lib().dg_debug_routing(self.handle, *[C.byref(x) for x in ps]), "dg_debug_routing")
+        k, e = self.cfg.top_k, self.cfg.n_experts
+        return (self._view(ps[0].value, n * k, torch.int32).view(n, k),
+                self._view(ps[1].value, n * k, torch.float32).view(n, k),
+                self._view(ps[2].value, n * e, torch.float32).view(n, e))
+
     def debug_layer(self, layer, x_in, causal, stream=None):
         _need_cuda(x_in, "x_in", torch.float32)
         out = torch.empty_like(x_in)

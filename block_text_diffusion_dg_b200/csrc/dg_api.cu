@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -45,12 +46,34 @@ int fail(int code, const char* fmt, ...) {
                   __FILE__, __LINE__);                                                       \
   } while (0)
 
+std::atomic<uint64_t> g_launches{0};
+
+// Optional per-kernel event hook (dg_profile_kernel).
+struct ProfileHook {
+  int kind = -1;
+  std::vector<cudaEvent_t> events;
+  int n_pairs = 0;
+  int recorded = 0;
+} g_prof;
+
+inline void prof_before(int kind, cudaStream_t st) {
+  if (g_prof.kind == kind && g_prof.recorded < g_prof.n_pairs)
+    cudaEventRecord(g_prof.events[2 * g_prof.recorded], st);
+}
+inline void prof_after(int kind, cudaStream_t st) {
+  if (g_prof.kind == kind && g_prof.recorded < g_prof.n_pairs) {
+    cudaEventRecord(g_prof.events[2 * g_prof.recorded + 1], st);
+    ++g_prof.recorded;
+  }
+}
+
 #define DG_LAUNCHED()                                                                        \
   do {                                                                                       \
     cudaError_t e_ = cudaGetLastError();                                                     \
     if (e_ != cudaSuccess)                                                                   \
       return fail(DG_ERR_CUDA, "launch failed: %s (%s:%d)", cudaGetErrorString(e_), __FILE__, \
                   __LINE__);                                                                 \
+    g_launches.fetch_add(1, std::memory_order_relaxed);                                      \
   } while (0)
 
 #define DG_TRY(expr)        \
@@ -125,12 +148,14 @@ constexpr int kGroupN = 64, kGroupStages = 8;
 
 template <int MAXN, int STAGES, int EPI>
 int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, int grid,
-                cudaStream_t st) {
+                cudaStream_t st, int kind = -1) {
   auto k = gemm_swapab_kernel<MAXN, STAGES, EPI>;
   constexpr int smem = GemmCfg<MAXN, STAGES>::kSmemBytes;
   DG_TRY(set_smem(k, smem));
+  prof_before(kind, st);
   k<<<grid, 192, smem, st>>>(ta, tb, p);
   DG_LAUNCHED();
+  prof_after(kind, st);
   return DG_OK;
 }
 
@@ -438,7 +463,8 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     p.split_stride = static_cast<long long>(n) * c->qkv_rows;
     const int items = p.m_tiles * p.k_splits * p.n_chunks;
     DG_TRY((launch_gemm<kDenseN, kDenseStages, kEpiPartialF32>(c->tm_wqkv[l], c->tm_xn32, p,
-                                                                 std::min(items, c->sms), st)));
+                                                                 std::min(items, c->sms), st,
+                                                                 DG_KERNEL_QKV)));
     DG_TRY(layer_tail_common<__nv_bfloat16>(c, l, n, pos0, done, st, p.split_stride,
                                             c->split_qkv));
   }
@@ -469,9 +495,11 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     a.err = c->err;
     a.done = done;
     DG_TRY(set_smem(attention_kernel, kAttnSmemBytes));
+    prof_before(DG_KERNEL_ATTENTION, st);
     attention_kernel<<<dim3(m_tiles, g.n_kv_heads, splits), 192, kAttnSmemBytes, st>>>(
         c->tm_q, c->tm_k, c->tm_vt, a);
     DG_LAUNCHED();
+    prof_after(DG_KERNEL_ATTENTION, st);
     attn_combine_kernel<__nv_bfloat16><<<dim3(n, g.n_heads), 128, 0, st>>>(
         c->o_part, c->ml_part, splits, g.n_heads, c->tq, n, static_cast<__nv_bfloat16*>(c->o),
         done);
@@ -485,7 +513,8 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     p.split_stride = static_cast<long long>(n) * d;
     const int items = p.m_tiles * p.k_splits * p.n_chunks;
     DG_TRY((launch_gemm<kDenseN, kDenseStages, kEpiPartialF32>(c->tm_wo[l], c->tm_o32, p,
-                                                                 std::min(items, c->sms), st)));
+                                                                 std::min(items, c->sms), st,
+                                                                 DG_KERNEL_O_PROJ)));
     residual_norm_kernel<__nv_bfloat16><<<n, 256, 0, st>>>(
         c->x, c->part, c->split_o, p.split_stride, d, w.ffn_norm, g.eps,
         static_cast<__nv_bfloat16*>(c->xn), done);
@@ -536,7 +565,7 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     p.err = c->err;
     p.done = done;
     DG_TRY((launch_gemm<kGroupN, kGroupStages, kEpiGluBf16>(c->tm_wgu[l], c->tm_xperm, p, c->sms,
-                                                             st)));
+                                                             st, DG_KERNEL_EXPERT_GATE_UP)));
     GemmParams q{};
     q.items = c->items_d;
     q.item_count = c->item_counts + 1;
@@ -550,7 +579,7 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     q.err = c->err;
     q.done = done;
     DG_TRY((launch_gemm<kGroupN, kGroupStages, kEpiScatterF32>(c->tm_wd[l], c->tm_h, q, c->sms,
-                                                                st)));
+                                                                st, DG_KERNEL_EXPERT_DOWN)));
   }
   const float* ysh = nullptr;
   if (g.shared_hidden > 0) {
@@ -559,13 +588,15 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     p.ld_out = g.shared_hidden;
     int items = p.m_tiles * p.n_chunks;
     DG_TRY((launch_gemm<kDenseN, kDenseStages, kEpiGluBf16>(c->tm_wsgu[l], c->tm_xn32, p,
-                                                              std::min(items, c->sms), st)));
+                                                              std::min(items, c->sms), st,
+                                                              DG_KERNEL_SHARED_EXPERT)));
     GemmParams q = dense_params(d, n, g.shared_hidden, 1, c->err, done);
     q.out_f32 = c->y_shared;
     q.ld_out = d;
     items = q.m_tiles * q.n_chunks;
     DG_TRY((launch_gemm<kDenseN, kDenseStages, kEpiScatterF32>(c->tm_wsd[l], c->tm_hs, q,
-                                                                 std::min(items, c->sms), st)));
+                                                                 std::min(items, c->sms), st,
+                                                                 DG_KERNEL_SHARED_EXPERT)));
     ysh = c->y_shared;
   }
   moe_combine_norm_kernel<__nv_bfloat16><<<n, 256, 0, st>>>(
@@ -588,6 +619,7 @@ int run_lm_head(dg_ctx* c, float* logits_out, const int* done, cudaStream_t st) 
     p.err = c->err;
     p.done = done;
     const int grid = std::min(p.n_vtiles, c->sms);
+    prof_before(DG_KERNEL_LM_HEAD, st);
     if (logits_out) {
       DG_TRY(set_smem(lmhead_kernel<false>, kLmSmemBytes));
       lmhead_kernel<false><<<grid, 192, kLmSmemBytes, st>>>(c->tm_xn128, c->tm_embed, p);
@@ -596,6 +628,7 @@ int run_lm_head(dg_ctx* c, float* logits_out, const int* done, cudaStream_t st) 
       lmhead_kernel<true><<<grid, 192, kLmSmemBytes, st>>>(c->tm_xn128, c->tm_embed, p);
     }
     DG_LAUNCHED();
+    prof_after(DG_KERNEL_LM_HEAD, st);
     return DG_OK;
   }
   float* dst = logits_out ? logits_out : c->logits;
@@ -664,6 +697,21 @@ extern "C" {
 
 const char* dg_last_error(void) { return g_last_error.c_str(); }
 const char* dg_version(void) { return "libdg 0.1 sm_100a"; }
+
+uint64_t dg_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int dg_profile_kernel(int32_t kernel_kind, void* const* events, int32_t n_pairs) {
+  if (n_pairs < 0 || (n_pairs > 0 && (!events || kernel_kind < 0 || kernel_kind >= DG_KERNEL_KINDS)))
+    return fail(DG_ERR_INVALID_ARG, "bad profile request");
+  g_prof.kind = n_pairs > 0 ? kernel_kind : -1;
+  g_prof.n_pairs = n_pairs;
+  g_prof.recorded = 0;
+  g_prof.events.assign(2 * static_cast<size_t>(n_pairs), nullptr);
+  for (int i = 0; i < 2 * n_pairs; ++i) g_prof.events[i] = static_cast<cudaEvent_t>(events[i]);
+  return DG_OK;
+}
+
+int32_t dg_profile_recorded(void) { return g_prof.recorded; }
 
 int dg_workspace_bytes(const dg_config* cfg, size_t* kv_bytes, size_t* scratch_bytes) {
   DG_TRY(check_config(cfg));
@@ -848,8 +896,10 @@ int dg_sample_update(dg_ctx* ctx, uint32_t step, void* stream) {
   a.locked = ctx->locked;
   a.state = ctx->state;
   a.ticket = ctx->ticket;
+  prof_before(DG_KERNEL_SAMPLER, S(stream));
   sampler_merge_kernel<<<g.canvas, 256, 0, S(stream)>>>(a);
   DG_LAUNCHED();
+  prof_after(DG_KERNEL_SAMPLER, S(stream));
   return DG_OK;
 }
 
@@ -891,6 +941,15 @@ int dg_debug_logits(dg_ctx* ctx, float* d_logits, void* stream) {
   DG_TRY(check_ctx(ctx));
   if (!d_logits) return fail(DG_ERR_INVALID_ARG, "null logits");
   return run_lm_head(ctx, d_logits, nullptr, S(stream));
+}
+
+int dg_debug_routing(const dg_ctx* ctx, int32_t** d_ids, float** d_weights,
+                     float** d_router_logits) {
+  DG_TRY(check_ctx(ctx));
+  if (d_ids) *d_ids = ctx->topk_ids;
+  if (d_weights) *d_weights = ctx->topk_w;
+  if (d_router_logits) *d_router_logits = ctx->router_logits;
+  return DG_OK;
 }
 
 int dg_debug_hidden(const dg_ctx* ctx, float** d_x) {

@@ -214,6 +214,32 @@ DG_API int dg_moe_ffn(const void* d_x, const float* d_residual, const void* d_wr
                int32_t n_experts, int32_t top_k, int32_t hidden, int32_t shared_hidden,
                void* d_workspace, size_t workspace_bytes, void* stream);
 
+/* ---- tracing ------------------------------------------------------------------------- */
+
+/* Kernels that dg_profile_kernel can time. */
+enum {
+  DG_KERNEL_EXPERT_GATE_UP = 0, /* grouped expert gate/up GEMM + SiLU-GLU */
+  DG_KERNEL_EXPERT_DOWN = 1,    /* grouped expert down GEMM + weighted scatter */
+  DG_KERNEL_ATTENTION = 2,      /* canvas attention (before the split combine) */
+  DG_KERNEL_LM_HEAD = 3,        /* LM head fused with vocab-tile statistics */
+  DG_KERNEL_QKV = 4,            /* QKV projection GEMM */
+  DG_KERNEL_O_PROJ = 5,         /* attention output projection GEMM */
+  DG_KERNEL_SAMPLER = 6,        /* sampler merge + stop test */
+  DG_KERNEL_SHARED_EXPERT = 7,  /* shared expert gate/up and down GEMMs */
+  DG_KERNEL_KINDS = 8
+};
+
+/* Number of kernels this library has launched in the calling process (all entry points). */
+DG_API uint64_t dg_launch_count(void);
+
+/* Time launches of one kernel kind: before/after each of its next n_pairs launches (on the
+ * stream the kernel is launched on) the library records events[2i] and events[2i+1]
+ * (cudaEvent_t values created by the caller).  n_pairs = 0 disables the hook.  The number of
+ * pairs recorded so far is returned by dg_profile_recorded.  Host-side only; not thread-safe
+ * across contexts. */
+DG_API int dg_profile_kernel(int32_t kernel_kind, void* const* events, int32_t n_pairs);
+DG_API int32_t dg_profile_recorded(void);
+
 /* ---- test exports ------------------------------------------------------------------ */
 
 /* Unfused LM head of the context on its current final hidden state: logits fp32 [T, V]
@@ -225,6 +251,10 @@ DG_API int dg_debug_logits(dg_ctx* ctx, float* d_logits, void* stream);
  * K/V are written to cache slots P..P+n-1 like a denoise step; P does not advance. */
 DG_API int dg_debug_layer(dg_ctx* ctx, int32_t layer, const float* d_x_in, float* d_x_out, int32_t n,
                    int32_t causal, void* stream);
+/* Routing of the most recent layer the context ran: ids int32 [n, k], weights fp32 [n, k]
+ * (renormalised over the k experts), router logits fp32 [n, E] (device pointers into scratch). */
+DG_API int dg_debug_routing(const dg_ctx* ctx, int32_t** d_ids, float** d_weights,
+                            float** d_router_logits);
 /* Final hidden state (fp32 [T, d]) of the last denoise step, for LM-head checks. */
 DG_API int dg_debug_hidden(const dg_ctx* ctx, float** d_x);
 

@@ -15,8 +15,11 @@ RTOL = 2e-2
 def _case(hq, hkv, t, tq, prefix, causal, seed):
     from block_text_diffusion_dg_b200 import canvas_attention
     q, k, v = attention_inputs(hq, hkv, canvas=tq, prefix=prefix, head_dim=128, seed=seed)
+    pad = (-k.shape[1]) % 8  # key stride must be a multiple of 8 (16-byte TMA rows)
+    if pad:
+        k = torch.cat([k, torch.zeros(hkv, pad, 128, dtype=k.dtype)], dim=1)
+        v = torch.cat([v, torch.zeros(hkv, pad, 128, dtype=v.dtype)], dim=1)
     ldk = k.shape[1]
-    assert ldk % 8 == 0
     n_keys = prefix + t
     vt = v.transpose(1, 2).contiguous()
     o = canvas_attention(q.cuda(), k.cuda(), vt.cuda(), n_keys, causal_prefix=prefix if causal else -1,
