@@ -69,8 +69,8 @@ _PROTOS = {
     "dg_debug_hidden": (C.c_int, [_P, C.POINTER(_P)]),
     "dg_debug_routing": (C.c_int, [_P, C.POINTER(_P), C.POINTER(_P), C.POINTER(_P)]),
     "dg_launch_count": (C.c_uint64, []),
-    "dg_profile_kernel": (C.c_int, [_I, C.POINTER(_P), _I]),
-    "dg_profile_recorded": (C.c_int32, []),
+    "dg_profile_kernel": (C.c_int, [_I, _I]),
+    "dg_profile_read": (C.c_int32, [C.POINTER(C.c_float), _I]),
     "dg_last_error": (C.c_char_p, []),
     "dg_version": (C.c_char_p, []),
 }

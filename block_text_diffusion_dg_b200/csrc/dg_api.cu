@@ -700,18 +700,29 @@ const char* dg_version(void) { return "libdg 0.1 sm_100a"; }
 
 uint64_t dg_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
-int dg_profile_kernel(int32_t kernel_kind, void* const* events, int32_t n_pairs) {
-  if (n_pairs < 0 || (n_pairs > 0 && (!events || kernel_kind < 0 || kernel_kind >= DG_KERNEL_KINDS)))
+int dg_profile_kernel(int32_t kernel_kind, int32_t n_pairs) {
+  if (n_pairs < 0 || n_pairs > (1 << 20) ||
+      (n_pairs > 0 && (kernel_kind < 0 || kernel_kind >= DG_KERNEL_KINDS)))
     return fail(DG_ERR_INVALID_ARG, "bad profile request");
+  for (cudaEvent_t e : g_prof.events)
+    if (e) cudaEventDestroy(e);
+  g_prof.events.assign(2 * static_cast<size_t>(n_pairs), nullptr);
+  for (auto& e : g_prof.events) DG_CUDA(cudaEventCreate(&e));
   g_prof.kind = n_pairs > 0 ? kernel_kind : -1;
   g_prof.n_pairs = n_pairs;
   g_prof.recorded = 0;
-  g_prof.events.assign(2 * static_cast<size_t>(n_pairs), nullptr);
-  for (int i = 0; i < 2 * n_pairs; ++i) g_prof.events[i] = static_cast<cudaEvent_t>(events[i]);
   return DG_OK;
 }
 
-int32_t dg_profile_recorded(void) { return g_prof.recorded; }
+int32_t dg_profile_read(float* durations_ms, int32_t max_pairs) {
+  if (!durations_ms || max_pairs < 0) return fail(DG_ERR_INVALID_ARG, "bad profile read");
+  const int n = std::min(max_pairs, g_prof.recorded);
+  for (int i = 0; i < n; ++i) {
+    DG_CUDA(cudaEventSynchronize(g_prof.events[2 * i + 1]));
+    DG_CUDA(cudaEventElapsedTime(&durations_ms[i], g_prof.events[2 * i], g_prof.events[2 * i + 1]));
+  }
+  return n;
+}
 
 int dg_workspace_bytes(const dg_config* cfg, size_t* kv_bytes, size_t* scratch_bytes) {
   DG_TRY(check_config(cfg));

@@ -232,13 +232,14 @@ enum {
 /* Number of kernels this library has launched in the calling process (all entry points). */
 DG_API uint64_t dg_launch_count(void);
 
-/* Time launches of one kernel kind: before/after each of its next n_pairs launches (on the
- * stream the kernel is launched on) the library records events[2i] and events[2i+1]
- * (cudaEvent_t values created by the caller).  n_pairs = 0 disables the hook.  The number of
- * pairs recorded so far is returned by dg_profile_recorded.  Host-side only; not thread-safe
- * across contexts. */
-DG_API int dg_profile_kernel(int32_t kernel_kind, void* const* events, int32_t n_pairs);
-DG_API int32_t dg_profile_recorded(void);
+/* Time launches of one kernel kind: before/after each of its next n_pairs launches the library
+ * records a pair of CUDA events (created here, timing enabled) on the stream the kernel is
+ * launched on.  n_pairs = 0 disables the hook and releases the events.  Host-side only, one hook
+ * per process. */
+DG_API int dg_profile_kernel(int32_t kernel_kind, int32_t n_pairs);
+/* Blocking: waits for the recorded pairs and writes their durations (milliseconds) to the host
+ * array durations_ms[0..max_pairs).  Returns the number of pairs written (>= 0) or an error. */
+DG_API int32_t dg_profile_read(float* durations_ms, int32_t max_pairs);
 
 /* ---- test exports ------------------------------------------------------------------ */
 
