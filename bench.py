@@ -48,6 +48,9 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--roofline-kernel", default="expert_gate_up")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", choices=["decode_step", "moe", "attention", "sampler"],
+                    help="run one profiled region between cudaProfilerStart/Stop and exit "
+                         "(for ncu --profile-from-start off); prints no JSON")
     return ap.parse_args()
 
 
@@ -345,8 +348,67 @@ def run_ours(args, rank, world, local_rank):
     model.close()
 
 
+def run_profile(args):
+    """One region for ncu: after warm-up, the profiled calls sit between profiler start/stop.
+
+    decode_step: the full decode model, prompt prefilled, then canvas init + one denoise step
+                 + one sampler update (483 launches of libdg).
+    moe:         the MoE operator at 256 tokens, d 2816, 128 experts top-8 + shared (1.5 GB).
+    attention:   canvas attention, 16/8 heads x 128, 4096 + 256 keys.
+    sampler:     the sampler on bf16 logits [256, 262144].
+    """
+    import block_text_diffusion_dg_b200 as dg
+    from dg_synth import SHAPES, attention_inputs, model_weights, moe_inputs, sampler_logits, uniform_ids
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    prof = torch.cuda.profiler
+    if args.profile == "decode_step":
+        shape = SHAPES["a4b"]
+        cfg = dg.make_config(shape, kv_capacity=PROMPT + BLOCKS * CANVAS + CANVAS,
+                             fixed_steps=FIXED_STEPS)
+        model = dg.DiffusionModel(cfg, model_weights("a4b", seed=1000, device=dev), device=dev)
+        model.kv_append(uniform_ids(PROMPT, shape["vocab"], seed=0).to(dev))
+        model.canvas_init(1, 0)
+        model.denoise_step(1)
+        model.sample_update(1)
+        torch.cuda.synchronize()
+        prof.start()
+        model.canvas_init(2, 0)
+        model.denoise_step(1)
+        model.sample_update(1)
+        torch.cuda.synchronize()
+        prof.stop()
+        model.check_device_status()
+        model.close()
+        return
+    if args.profile == "moe":
+        m = {k: (None if v is None else v.to(dev)) for k, v in moe_inputs(seed=0).items()}
+        ws = dg.moe_workspace(256, 2816, 128, 8, 704, 2112, dev)
+        call = lambda: dg.moe_ffn(m["x"], m["wr"], m["w_gu"], m["w_d"], 8, m["ws_gu"], m["ws_d"],
+                                  workspace=ws)
+    elif args.profile == "attention":
+        q, k, v = (t.to(dev) for t in attention_inputs(seed=0))
+        vt = v.transpose(1, 2).contiguous()
+        call = lambda: dg.canvas_attention(q, k, vt, 4096 + 256)
+    else:
+        x = sampler_logits(256, 262144, seed=0).to(dev)
+        s = dg.Sampler(256, 262144)
+        s.reset()
+        call = lambda: s.step(x, seed=0, block=0, step=1)
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    prof.start()
+    call()
+    torch.cuda.synchronize()
+    prof.stop()
+
+
 def main():
     args = parse()
+    if args.profile:
+        run_profile(args)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
