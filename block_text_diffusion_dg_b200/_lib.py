@@ -58,6 +58,8 @@ _PROTOS = {
     "dg_sampler_reset": (C.c_int, [_I, _I, _P, _P, _P]),
     "dg_sampler_step": (C.c_int, [_P, _I, _I, _I, C.c_uint64, C.c_uint32, C.c_uint32, C.c_double,
                                   C.c_double, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
+    "dg_sampler_step_static": (C.c_int, [_P, _I, _I, _I, C.c_uint64, C.c_uint32, C.c_uint32,
+                                         C.c_double, C.c_double, _I, _I, _P, _P, _P, _P, _P, _P]),
     "dg_attention_workspace_bytes": (C.c_int, [_I, _I, _I, _I, C.POINTER(_SZ)]),
     "dg_canvas_attention": (C.c_int, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, C.c_float, _P,
                                       _SZ, _P]),

@@ -1327,3 +1327,112 @@ int dg_moe_ffn(const void* d_x, const float* d_residual, const void* d_wr, const
 }
 
 }  // extern "C"
+
+// ---- sampler without caller-provided workspace -------------------------------------------
+// Some callers cannot allocate device memory: for example a host framework whose own pool owns
+// the whole device budget, or a latency-critical path that may not risk cudaMalloc's implicit
+// device synchronisation.  dg_sampler_step_static keeps the sampler's temporaries and its
+// step-to-step stop-test state in one fixed file-scope device array instead of a workspace.
+namespace {
+constexpr int kStaticRows = 256;
+constexpr int kStaticVocab = 262144;
+constexpr int kStaticChunks = kStaticVocab / 4096;  // fp32 slices are the finer ones
+constexpr size_t kStaticPartBytes = static_cast<size_t>(kStaticRows) * kStaticChunks * sizeof(StatPartial);
+constexpr size_t kStaticPrevOff = kStaticPartBytes;
+constexpr size_t kStaticRowHOff = kStaticPrevOff + 256 * 4;
+constexpr size_t kStaticLockedOff = kStaticRowHOff + 256 * 8;
+constexpr size_t kStaticTicketOff = kStaticLockedOff + 256 * 4;
+constexpr size_t kStaticBytes = kStaticTicketOff + 256;
+}  // namespace
+
+// Held by every GPU that loads this library until the process exits (about 266 KB).
+static __device__ __align__(256) uint8_t g_sampler_scratch[kStaticBytes];
+
+namespace {
+std::mutex g_static_mu;
+void* g_static_ptr[256] = {};  // device address of g_sampler_scratch, per device ordinal
+
+// First call on a device looks up the array's device address with that device current.
+int static_scratch(void** out) {
+  int dev = 0;
+  DG_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 256) return fail(DG_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (!g_static_ptr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_sampler_scratch);
+    if (e != cudaSuccess || !p)
+      return fail(DG_ERR_CUDA, "cudaGetSymbolAddress(sampler scratch) failed: %s",
+                  cudaGetErrorString(e));
+    g_static_ptr[dev] = p;
+  }
+  *out = g_static_ptr[dev];
+  return DG_OK;
+}
+}  // namespace
+
+extern "C" int dg_sampler_step_static(const void* d_logits, int32_t dtype, int32_t rows,
+                                      int32_t vocab, uint64_t seed, uint32_t block, uint32_t step,
+                                      double tau, double h_bound, int32_t max_steps,
+                                      int32_t fixed_steps, int32_t* d_canvas, int32_t* d_argmax,
+                                      float* d_entropy, float* d_conf, int32_t* d_state,
+                                      void* stream) {
+  if (rows < 1 || rows > kStaticRows || vocab < 2 || vocab > kStaticVocab || vocab % 8)
+    return fail(DG_ERR_CAPACITY,
+                "dg_sampler_step_static handles at most %d rows and %d vocabulary entries "
+                "(vocab a multiple of 8); got rows %d, vocab %d",
+                kStaticRows, kStaticVocab, rows, vocab);
+  if (!d_logits || !d_canvas || !d_argmax || !d_entropy || !d_conf || !d_state)
+    return fail(DG_ERR_INVALID_ARG, "null pointer argument");
+  if (reinterpret_cast<uintptr_t>(d_logits) % 16)
+    return fail(DG_ERR_INVALID_ARG, "logits must be 16-byte aligned");
+  if (step < 1 || max_steps < 1 || fixed_steps < 0)
+    return fail(DG_ERR_INVALID_ARG, "bad step / max_steps / fixed_steps");
+  if (dtype != DG_DTYPE_BF16 && dtype != DG_DTYPE_FP32)
+    return fail(DG_ERR_INVALID_ARG, "dtype must be bf16 or fp32");
+  void* base = nullptr;
+  DG_TRY(static_scratch(&base));
+  uint8_t* b = static_cast<uint8_t*>(base);
+  StatPartial* part = reinterpret_cast<StatPartial*>(b);
+  int32_t* prev = reinterpret_cast<int32_t*>(b + kStaticPrevOff);
+  double* row_h = reinterpret_cast<double*>(b + kStaticRowHOff);
+  int32_t* locked = reinterpret_cast<int32_t*>(b + kStaticLockedOff);
+  int32_t* ticket = reinterpret_cast<int32_t*>(b + kStaticTicketOff);
+  cudaStream_t st = S(stream);
+  // the completion ticket must start at zero; the previous argmax is only read from step 2 on
+  DG_CUDA(cudaMemsetAsync(ticket, 0, sizeof(int32_t), st));
+  const int chunk = dtype == DG_DTYPE_BF16 ? 8192 : 4096;
+  const int nchunk = cdiv(vocab, chunk);
+  const int* done = d_state + kStDone;
+  if (dtype == DG_DTYPE_BF16)
+    logits_stats_kernel<__nv_bfloat16, 32><<<dim3(nchunk, rows), 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(d_logits), vocab, chunk, part, done);
+  else
+    logits_stats_kernel<float, 16><<<dim3(nchunk, rows), 256, 0, st>>>(
+        static_cast<const float*>(d_logits), vocab, chunk, part, done);
+  DG_LAUNCHED();
+  SamplerArgs a{};
+  a.partials = part;
+  a.nsplit = nchunk;
+  a.rows = rows;
+  a.vocab = vocab;
+  a.seed = seed;
+  a.block = block;
+  a.step = step;
+  a.tau = tau;
+  a.h_bound = h_bound;
+  a.max_steps = max_steps;
+  a.fixed_steps = fixed_steps;
+  a.canvas = d_canvas;
+  a.argmax = d_argmax;
+  a.prev_argmax = prev;
+  a.entropy = d_entropy;
+  a.conf = d_conf;
+  a.row_h = row_h;
+  a.locked = locked;
+  a.state = d_state;
+  a.ticket = ticket;
+  sampler_merge_kernel<<<rows, 256, 0, st>>>(a);
+  DG_LAUNCHED();
+  return DG_OK;
+}

@@ -189,6 +189,24 @@ DG_API int dg_sampler_step(const void* d_logits, int32_t dtype, int32_t rows, in
                     int32_t* d_canvas, int32_t* d_argmax, float* d_entropy, float* d_conf,
                     int32_t* d_state, void* stream);
 
+/* The sampler step above without a caller-provided workspace (the pages have no
+ * counterpart: this is a deployment variant).  For callers that cannot allocate device memory,
+ * such as a host framework whose memory pool owns the whole device budget, or a latency-critical
+ * path that may not risk cudaMalloc's implicit device synchronisation.  Its temporaries and the
+ * step-to-step stop-test state live in one file-scope device array of about 266 KB, held by every
+ * GPU that loads the library until the process exits.  Limits: rows <= 256, V <= 262144,
+ * V % 8 == 0; larger requests return DG_ERR_CAPACITY.  Arguments and outputs are those of
+ * dg_sampler_step; the caller zeroes d_state before step 1.  The first call on each device looks
+ * up the array's device address (cudaGetSymbolAddress) with that device current, so make that
+ * first call before any stream capture.  Every call on a device shares the one array, which keeps
+ * the previous call's contents: calls that overlap on the GPU (other streams, other threads) race,
+ * so serialise them.  Allocates no memory (no cudaMalloc, cudaFree or allocating library call). */
+DG_API int dg_sampler_step_static(const void* d_logits, int32_t dtype, int32_t rows,
+                                  int32_t vocab, uint64_t seed, uint32_t block, uint32_t step,
+                                  double tau, double h_bound, int32_t max_steps,
+                                  int32_t fixed_steps, int32_t* d_canvas, int32_t* d_argmax,
+                                  float* d_entropy, float* d_conf, int32_t* d_state, void* stream);
+
 /* Canvas attention ([uniform], [arch]): bf16 q [Hq, Tq, 128] (head stride Tq), keys
  * k [Hkv, ldk, 128] and values TRANSPOSED vt [Hkv, 128, ldk], keys 0..n_keys-1 used;
  * causal_prefix < 0: no mask; >= 0: query t sees keys n <= causal_prefix + t.
