@@ -48,7 +48,8 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--roofline-kernel", default="expert_gate_up")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["decode_step", "moe", "attention", "sampler"],
+    ap.add_argument("--profile", choices=["decode_step", "decode_step_small", "moe", "attention",
+                                          "sampler"],
                     help="run one profiled region between cudaProfilerStart/Stop and exit "
                          "(for ncu --profile-from-start off); prints no JSON")
     return ap.parse_args()
@@ -198,6 +199,65 @@ def replica_throughput(tokens_per_rank, world, ms_max):
     return world * tokens_per_rank / (ms_max / 1e3)
 
 
+def _time_op(fn, stream, reps=10, flush=None):
+    """Average device time (ms) of fn() over reps, CUDA events on `stream`, L2 flushed between reps."""
+    for _ in range(3):
+        fn()
+    total = 0.0
+    for _ in range(reps):
+        if flush is not None:
+            flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        total += e0.elapsed_time(e1)
+    return total / reps
+
+
+def run_ops(dev, stream, hbm, tf_burst):
+    """The standalone operators at their full sizes, each against its roofline (kernel timed
+    alone: burst peaks).  sampler: bf16 logits [256, 262144]; attention: 16 q / 8 kv heads x 128,
+    4096 + 256 keys; MoE: 256 tokens, d 2816, 128 experts top-8 x 704 + shared 2112."""
+    import block_text_diffusion_dg_b200 as dg
+    from dg_synth import attention_inputs, moe_inputs, sampler_logits
+    # 1 GB flush (> L2): it also keeps the GPU busy while the host enqueues the timed call, so
+    # the event interval holds device time only
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.float32, device=dev)
+    out = {}
+    x = sampler_logits(256, 262144, seed=0).to(dev)
+    s = dg.Sampler(256, 262144, device=dev)
+    s.reset()
+    ms = _time_op(lambda: s.step(x, seed=0, block=0, step=1, stream=stream), stream, flush=flush)
+    gbs = 256 * 262144 * 2 / (ms / 1e3) / 1e9
+    out["sampler"] = dict(us=round(ms * 1e3, 2), bound="hbm", achieved_gbs=round(gbs, 1),
+                          frac=round(gbs / hbm, 4), bytes=256 * 262144 * 2)
+    del x, s
+    q, k, v = (t.to(dev) for t in attention_inputs(seed=0))
+    vt = v.transpose(1, 2).contiguous()
+    ws = torch.empty(64 << 20, dtype=torch.uint8, device=dev)
+    o = torch.empty(256, 16 * 128, dtype=torch.bfloat16, device=dev)
+    ms = _time_op(lambda: dg.canvas_attention(q, k, vt, 4096 + 256, out=o, workspace=ws,
+                                              stream=stream), stream, flush=flush)
+    flops = 4 * 16 * 256 * 4352 * 128
+    tf = flops / (ms / 1e3) / 1e12
+    out["attention"] = dict(us=round(ms * 1e3, 2), bound="tensor", achieved_tflops=round(tf, 1),
+                            frac=round(tf / tf_burst, 4), flops=flops)
+    del q, k, v, vt, ws, o
+    m = {kk: (None if vv is None else vv.to(dev)) for kk, vv in moe_inputs(seed=0).items()}
+    wsm = dg.moe_workspace(256, 2816, 128, 8, 704, 2112, dev)
+    y = torch.empty(256, 2816, dtype=torch.float32, device=dev)
+    ms = _time_op(lambda: dg.moe_ffn(m["x"], m["wr"], m["w_gu"], m["w_d"], 8, m["ws_gu"], m["ws_d"],
+                                     workspace=wsm, out=y, stream=stream), stream, flush=flush)
+    nbytes = sum(t.numel() * 2 for t in (m["wr"], m["w_gu"], m["w_d"], m["ws_gu"], m["ws_d"]))
+    gbs = nbytes / (ms / 1e3) / 1e9
+    out["moe"] = dict(us=round(ms * 1e3, 2), bound="hbm", achieved_gbs=round(gbs, 1),
+                      frac=round(gbs / hbm, 4), bytes=nbytes)
+    del m, wsm, y, flush
+    return out
+
+
 def decode(model, seed, out_ids, out_states, stream):
     model.kv_truncate(PROMPT)
     for b in range(BLOCKS):
@@ -306,6 +366,28 @@ def run_ours(args, rank, world, local_rank):
                     algorithmic_bytes_per_launch=algo[args.roofline_kernel],
                     peak_source=f"{src} (MEASURED_PEAKS.json hbm_gbs)")
 
+    # live per-kernel table: one profiled denoise step per kernel kind
+    table = {}
+    for kname, kk in L.KERNEL_KINDS.items():
+        L.check(L.lib().dg_profile_kernel(kk, 64), "dg_profile_kernel")
+        model.kv_truncate(PROMPT)
+        model.canvas_init(9, 0, stream)
+        model.denoise_step(1, stream)
+        model.sample_update(1, stream)
+        torch.cuda.synchronize()
+        buf2 = (C.c_float * 64)()
+        nrec = L.lib().dg_profile_read(buf2, 64)
+        L.check(L.lib().dg_profile_kernel(0, 0), "dg_profile_kernel")
+        if nrec > 0:
+            tot = sum(buf2[:nrec]) * 1e3
+            table[kname] = dict(launches=nrec, us_per_launch=round(tot / nrec, 2),
+                                us_per_step=round(tot, 1))
+    step_us = sum(v["us_per_step"] for v in table.values())
+    for v in table.values():
+        v["share"] = round(v["us_per_step"] / step_us, 4)
+
+    ops = run_ops(dev, stream, hbm, tf_burst)
+
     # end to end through the public API, pinned host buffers in and out
     host_ids = torch.empty(BLOCKS * CANVAS, dtype=torch.int32).pin_memory()
     host_states = torch.empty(BLOCKS, L.STATE_WORDS, dtype=torch.int32).pin_memory()
@@ -343,7 +425,8 @@ def run_ours(args, rank, world, local_rank):
                             h2d_bytes_per_step=prompt.numel() * 4,
                             d2h_bytes_per_step=host_ids.numel() * 4 + host_states.numel() * 4,
                             includes="prompt H2D, 4096-token prefill, 4 blocks, ids D2H"),
-                   gpu_launches=int((n1 - n0) // args.steps), clocks=ck)
+                   gpu_launches=int((n1 - n0) // args.steps), clocks=ck,
+                   kernels_live=table, ops=ops)
         print(json.dumps(out), flush=True)
     model.close()
 
@@ -352,7 +435,9 @@ def run_profile(args):
     """One region for ncu: after warm-up, the profiled calls sit between profiler start/stop.
 
     decode_step: the full decode model, prompt prefilled, then canvas init + one denoise step
-                 + one sampler update (483 launches of libdg).
+                 + one sampler update.
+    decode_step_small: the same with 2 layers and a 32768-token vocabulary (a few GB on the
+                 device, for multi-pass captures of single kernels).
     moe:         the MoE operator at 256 tokens, d 2816, 128 experts top-8 + shared (1.5 GB).
     attention:   canvas attention, 16/8 heads x 128, 4096 + 256 keys.
     sampler:     the sampler on bf16 logits [256, 262144].
@@ -362,11 +447,13 @@ def run_profile(args):
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     prof = torch.cuda.profiler
-    if args.profile == "decode_step":
-        shape = SHAPES["a4b"]
+    if args.profile in ("decode_step", "decode_step_small"):
+        shape = dict(SHAPES["a4b"])
+        if args.profile == "decode_step_small":
+            shape.update(n_layers=2, vocab=32768)
         cfg = dg.make_config(shape, kv_capacity=PROMPT + BLOCKS * CANVAS + CANVAS,
                              fixed_steps=FIXED_STEPS)
-        model = dg.DiffusionModel(cfg, model_weights("a4b", seed=1000, device=dev), device=dev)
+        model = dg.DiffusionModel(cfg, model_weights(shape, seed=1000, device=dev), device=dev)
         model.kv_append(uniform_ids(PROMPT, shape["vocab"], seed=0).to(dev))
         model.canvas_init(1, 0)
         model.denoise_step(1)

@@ -12,7 +12,9 @@ DTYPE_BF16, DTYPE_FP32 = 0, 1
 STATE_DONE, STATE_STOP_STEP, STATE_WOULD_STOP, STATE_STEPS_RUN, STATE_LOCKED, STATE_ERROR = range(6)
 STATE_WORDS = 16
 KERNEL_KINDS = dict(expert_gate_up=0, expert_down=1, attention=2, lm_head=3, qkv=4,
-                    o_proj=5, sampler=6, shared_expert=7)
+                    o_proj=5, sampler=6, router=8, qkv_finalize=9, attn_combine=10,
+                    residual_norm=11, router_topk=12, route=13, gather=14, combine_norm=15,
+                    embed=16)
 
 
 class Config(C.Structure):

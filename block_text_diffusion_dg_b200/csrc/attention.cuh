@@ -6,10 +6,13 @@
 //
 // One CTA per (128-row query tile, kv head, key split).  The query tile packs rows of the
 // group's heads (row = head * Tq + token), so every K/V tile is used by all of them.
-// Roles: warp 0 TMA (Q once, then K and V^T tiles of 128 keys through a 2-deep ring),
-// warp 1 UMMA (S = Q K^T into one of two TMEM buffers, then O += P V), warps 2-5 softmax
-// (one query row per thread, exp2 with the scale folded in, P written to shared memory in
-// the UMMA's 128-byte swizzled K-major layout).  O lives in TMEM for the whole key range;
+// Roles: warp 0 TMA (Q once, then K and V^T tiles of 128 keys through separate 2-deep rings:
+// a K slot frees as soon as its S = Q K^T is done, so K runs one tile ahead of V),
+// warp 1 UMMA (S = Q K^T into one of two TMEM buffers, then O += P V), warps 2-9 softmax:
+// two threads per query row, each owning 64 of the tile's 128 keys (the partners sit in
+// different warps of the same TMEM lane quarter and trade their partial row maxima through a
+// spare TMEM column); exp2 with the scale folded in, P written to shared memory in the UMMA's
+// 128-byte swizzled K-major layout.  O lives in TMEM for the whole key range;
 // its running maximum is only moved (and O rescaled) when a new tile raises the row max by
 // more than 2^8, otherwise exponents relative to the stale maximum stay below 256.
 // Each split writes its unnormalised O, its max and its denominator; a combine kernel merges
@@ -43,7 +46,9 @@ constexpr int kAttnTile = 16384;  // one 128-row x 128-byte swizzled slab
 // Q (2 slabs) + K,V^T ring (2 stages x 4 slabs) + P (2 buffers x 2 slabs) + barriers
 constexpr int kAttnSmemBytes = 14 * kAttnTile + 1024 + 256;
 
-__global__ void __launch_bounds__(192, 1)
+constexpr int kAttnThreads = 64 + 32 * 8;
+
+__global__ void __launch_bounds__(kAttnThreads, 1)
     attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_vt, const AttnParams p) {
   if (block_done(p.done)) return;
@@ -51,16 +56,19 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* s_q = smem;                   // slabs: hd 0-63, hd 64-127
-  uint8_t* s_kv = smem + 2 * kAttnTile;  // stage s: K (2 slabs) then V^T (2 slabs)
-  uint8_t* s_p = s_kv + 8 * kAttnTile;   // buffer b: 2 slabs (keys 0-63, 64-127)
+  uint8_t* s_k = smem + 2 * kAttnTile;   // K stage s: 2 slabs (hd 0-63, 64-127)
+  uint8_t* s_v = s_k + 4 * kAttnTile;    // V^T stage s: 2 slabs (keys 0-63, 64-127)
+  uint8_t* s_p = s_v + 4 * kAttnTile;    // P buffer b: 2 slabs (keys 0-63, 64-127)
   uint64_t* bars = reinterpret_cast<uint64_t*>(s_p + 4 * kAttnTile);
   uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;   // [2] per K/V stage
-  uint64_t* kv_empty = bars + 3;  // [2]
-  uint64_t* s_full = bars + 5;    // [2] per S buffer
-  uint64_t* p_full = bars + 7;    // [2] per P buffer
-  uint64_t* pv_done = bars + 9;   // [2] per P buffer (P V of that buffer completed)
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 11);
+  uint64_t* k_full = bars + 1;    // [2] per K stage
+  uint64_t* k_empty = bars + 3;   // [2] (S = Q K^T of that stage completed)
+  uint64_t* v_full = bars + 5;    // [2] per V stage
+  uint64_t* v_empty = bars + 7;   // [2] (P V of that stage completed)
+  uint64_t* s_full = bars + 9;    // [2] per S buffer
+  uint64_t* p_full = bars + 11;   // [2] per P buffer
+  uint64_t* pv_done = bars + 13;  // [2] per P buffer (P V of that buffer completed)
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 15);
 
   const int warp = threadIdx.x >> 5;
   const int mt = blockIdx.x;  // query tile inside the kv group
@@ -77,10 +85,12 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 0 && lane_id() == 0) {
     mbar_init(q_full, 1);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
       mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[s], 128);
+      mbar_init(&p_full[s], 256);
       mbar_init(&pv_done[s], 1);
     }
     fence_barrier_init();
@@ -95,7 +105,8 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem_base = *tmem_holder;  // cols [0,128): O, [128,256) S0, [256,384) S1
+  // TMEM columns: [0,128) O, [128,256) S0, [256,384) S1, [384,390) partner exchange
+  const uint32_t tmem_base = *tmem_holder;
 
   if (warp == 0) {
     if (elect_one() && n_tiles > 0) {
@@ -104,18 +115,33 @@ __global__ void __launch_bounds__(192, 1)
       mbar_arrive_expect_tx(q_full, 2 * kAttnTile);
       tma_load_2d(&tm_q, q_full, s_q, 0, q_row, pol);
       tma_load_2d(&tm_q, q_full, s_q + kAttnTile, 64, q_row, pol);
-      for (int j = 0; j < n_tiles; ++j) {
+      const int vt_row = p.vt_row_base + g * 128;
+      auto load_k = [&](int j) -> bool {
         const int st = j & 1;
-        if (!mbar_wait(&kv_empty[st], ((j >> 1) & 1) ^ 1u, p.err)) break;
-        uint8_t* sk = s_kv + st * 4 * kAttnTile;
+        if (!mbar_wait(&k_empty[st], ((j >> 1) & 1) ^ 1u, p.err)) return false;
         const int key0 = (tile0 + j) * 128;
         const int k_row = static_cast<int>(p.k_row_base + static_cast<long long>(g) * p.ldk + key0);
-        const int vt_row = p.vt_row_base + g * 128;
-        mbar_arrive_expect_tx(&kv_full[st], 4 * kAttnTile);
-        tma_load_2d(&tm_k, &kv_full[st], sk, 0, k_row, pol);
-        tma_load_2d(&tm_k, &kv_full[st], sk + kAttnTile, 64, k_row, pol);
-        tma_load_2d(&tm_vt, &kv_full[st], sk + 2 * kAttnTile, key0, vt_row, pol);
-        tma_load_2d(&tm_vt, &kv_full[st], sk + 3 * kAttnTile, key0 + 64, vt_row, pol);
+        uint8_t* sk = s_k + st * 2 * kAttnTile;
+        mbar_arrive_expect_tx(&k_full[st], 2 * kAttnTile);
+        tma_load_2d(&tm_k, &k_full[st], sk, 0, k_row, pol);
+        tma_load_2d(&tm_k, &k_full[st], sk + kAttnTile, 64, k_row, pol);
+        return true;
+      };
+      auto load_v = [&](int j) -> bool {
+        const int st = j & 1;
+        if (!mbar_wait(&v_empty[st], ((j >> 1) & 1) ^ 1u, p.err)) return false;
+        const int key0 = (tile0 + j) * 128;
+        uint8_t* sv = s_v + st * 2 * kAttnTile;
+        mbar_arrive_expect_tx(&v_full[st], 2 * kAttnTile);
+        tma_load_2d(&tm_vt, &v_full[st], sv, key0, vt_row, pol);
+        tma_load_2d(&tm_vt, &v_full[st], sv + kAttnTile, key0 + 64, vt_row, pol);
+        return true;
+      };
+      // the UMMA needs K of tile j + 1 (for S) before V of tile j (for P V)
+      bool ok = load_k(0);
+      for (int j = 0; j < n_tiles && ok; ++j) {
+        if (j + 1 < n_tiles) ok = load_k(j + 1);
+        if (ok) ok = load_v(j);
       }
     }
   } else if (warp == 1) {
@@ -125,9 +151,9 @@ __global__ void __launch_bounds__(192, 1)
       bool ok = mbar_wait(q_full, 0, p.err);
       auto issue_s = [&](int j) -> bool {
         const int st = j & 1;
-        if (!mbar_wait(&kv_full[st], (j >> 1) & 1, p.err)) return false;
+        if (!mbar_wait(&k_full[st], (j >> 1) & 1, p.err)) return false;
         tc_fence_after();
-        const uint32_t a_k = smem_u32(s_kv + st * 4 * kAttnTile);
+        const uint32_t a_k = smem_u32(s_k + st * 2 * kAttnTile);
         const uint32_t d = tmem_base + 128 + st * 128;
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
@@ -136,6 +162,7 @@ __global__ void __launch_bounds__(192, 1)
                     idesc, k > 0 ? 1u : 0u);
         }
         umma_commit(&s_full[st]);
+        umma_commit(&k_empty[st]);
         return true;
       };
       if (ok) ok = issue_s(0);
@@ -144,9 +171,10 @@ __global__ void __launch_bounds__(192, 1)
         if (j + 1 < n_tiles && !issue_s(j + 1)) break;
         const int b = j & 1;
         if (!mbar_wait(&p_full[b], (j >> 1) & 1, p.err)) break;
+        if (!mbar_wait(&v_full[b], (j >> 1) & 1, p.err)) break;
         tc_fence_after();
         const uint32_t a_p = smem_u32(s_p + b * 2 * kAttnTile);
-        const uint32_t a_v = smem_u32(s_kv + b * 4 * kAttnTile + 2 * kAttnTile);
+        const uint32_t a_v = smem_u32(s_v + b * 2 * kAttnTile);
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const uint32_t off = (k >> 2) * kAttnTile;
@@ -154,112 +182,133 @@ __global__ void __launch_bounds__(192, 1)
                     sdesc_sw128(a_v + off) + 2 * (k & 3), idesc, (j > 0 || k > 0) ? 1u : 0u);
         }
         umma_commit(&pv_done[b]);
-        umma_commit(&kv_empty[b]);
+        umma_commit(&v_empty[b]);
       }
     }
   } else {
-    const int q4 = warp & 3;
-    const int r = q4 * 32 + lane_id();
+    const int q4 = warp & 3;             // TMEM lane quarter
+    const int half = (warp - 2) >> 2;    // keys [64 half, 64 half + 64) of each tile
+    const int r = q4 * 32 + lane_id();   // query row of the tile
     const int tok = tok0 + r;
     const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
+    const uint32_t xchg = tmem_base + 384 + lane_off;  // partner exchange columns
+    const int bar_id = 1 + q4;                         // the two warps of this lane quarter
     const int key_lim =
         p.causal_prefix >= 0 ? min(p.n_keys, p.causal_prefix + tok + 1) : p.n_keys;
+    // Every thread passes the same named barriers whatever happens (one per tile and one at
+    // the end), so a failed wait only turns the remaining work off: `ok` is warp-uniform.
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    for (int j = 0; j < n_tiles && ok; ++j) {
+    for (int j = 0; j < n_tiles; ++j) {
       const int st = j & 1;
-      if (!mbar_wait(&s_full[st], (j >> 1) & 1, p.err)) {
-        ok = false;
-        break;
-      }
+      ok = __all_sync(0xffffffffu, ok && mbar_wait(&s_full[st], (j >> 1) & 1, p.err));
       tc_fence_after();
-      const int key0 = (tile0 + j) * 128;
-      const uint32_t s_addr = tmem_base + 128 + st * 128 + lane_off;
-      // pass 1: row maximum of this tile (scaled, log2 units)
-      float m_tile = -INFINITY;
+      const int key0 = (tile0 + j) * 128 + 64 * half;
+      const bool full_tile = key0 + 64 <= key_lim;  // none of my 64 keys is masked
+      float x[64];
+      tmem_ld64(tmem_base + 128 + st * 128 + 64 * half + lane_off, x);
+      if (!full_tile) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float v[32];
-        tmem_ld32(s_addr + c * 32, v);
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (key0 + c * 32 + i < key_lim) m_tile = fmaxf(m_tile, v[i] * p.scale_log2);
+        for (int i = 0; i < 64; ++i)
+          if (key0 + i >= key_lim) x[i] = -INFINITY;
       }
-      // move the reference maximum only when it grows by more than 8 (factor 256)
+      float mp;
+      {
+        float t[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) t[i] = fmaxf(x[i], x[i + 32]);
+#pragma unroll
+        for (int w = 16; w >= 1; w >>= 1)
+#pragma unroll
+          for (int i = 0; i < w; ++i) t[i] = fmaxf(t[i], t[i + w]);
+        mp = t[0];
+      }
+      // row maximum of the tile: my half and my partner's (raw scores, scale applied after)
+      tmem_st1(xchg + 2 * st + half, mp);
+      tc_fence_before();
+      named_barrier(bar_id, 64);
+      tc_fence_after();
+      const float mo = tmem_ld1(xchg + 2 * st + (1 - half));
+      if (!ok) continue;
+      const float m_tile = fmaxf(mp, mo) * p.scale_log2;  // -inf stays -inf
+      // move the reference maximum only when it grows by more than 8 (factor 256); both
+      // partners take the same decision from the same values
       float alpha = 1.0f;
       bool rescale = false;
       if (m_tile > m_run + 8.0f || (m_run == -INFINITY && m_tile > -INFINITY)) {
         if (m_run != -INFINITY) {
-          alpha = exp2f(m_run - m_tile);
+          alpha = fast_exp2(m_run - m_tile);
           rescale = true;
         }
         m_run = m_tile;
       }
       if (__any_sync(0xffffffffu, rescale)) {
         // O must hold every earlier P V before it is rescaled
-        if (j > 0 && !mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, p.err)) {
-          ok = false;
-          break;
-        }
+        if (j > 0)
+          ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, p.err));
+        if (!ok) continue;
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
           float v[32];
-          tmem_ld32(tmem_base + lane_off + c * 32, v);
+          const uint32_t oa = tmem_base + 64 * half + 32 * c + lane_off;
+          tmem_ld32(oa, v);
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] *= alpha;
-          tmem_st32(tmem_base + lane_off + c * 32, v);
+          tmem_st32(oa, v);
         }
       }
       // the P buffer of this tile was last read by P V of tile j - 2
       const int b = j & 1;
-      if (j >= 2 && !mbar_wait(&pv_done[b], ((j - 2) >> 1) & 1, p.err)) {
-        ok = false;
-        break;
-      }
+      if (j >= 2)
+        ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[b], ((j - 2) >> 1) & 1, p.err));
+      if (!ok) continue;
       tc_fence_after();
-      // pass 2: probabilities (bf16) into the swizzled K-major layout: slab key / 64; the
-      // 16-byte unit u of row r's 128-byte line lands at unit u ^ (r % 8)
-      uint8_t* pb = s_p + b * 2 * kAttnTile + (r >> 3) * 1024 + (r & 7) * 128;
-      float rowsum = 0.f;
+      // probabilities (bf16) of my 64 keys = slab `half` of the P buffer; 16-byte unit u of
+      // row r's 128-byte line lands at unit u ^ (r % 8)
+      uint8_t* pb = s_p + b * 2 * kAttnTile + half * kAttnTile + (r >> 3) * 1024 + (r & 7) * 128;
+      const float mr = (m_run == -INFINITY) ? 0.f : m_run;
+      float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float v[32];
-        tmem_ld32(s_addr + c * 32, v);
-        uint32_t pk[16];
+      for (int i = 0; i < 64; ++i) {
+        float e = fast_exp2(fmaf(x[i], p.scale_log2, -mr));
+        if ((!full_tile && key0 + i >= key_lim) || m_run == -INFINITY) e = 0.f;
+        x[i] = e;
+        part[i & 7] += e;
+      }
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int k0 = key0 + c * 32 + 2 * i;
-          const float e0 = (k0 < key_lim) ? exp2f(v[2 * i] * p.scale_log2 - m_run) : 0.f;
-          const float e1 = (k0 + 1 < key_lim) ? exp2f(v[2 * i + 1] * p.scale_log2 - m_run) : 0.f;
-          const __nv_bfloat162 h2 = __floats2bfloat162_rn(e0, e1);
-          // the denominator sums exactly the probabilities P V uses
-          rowsum += __low2float(h2) + __high2float(h2);
-          pk[i] = *reinterpret_cast<const uint32_t*>(&h2);
-        }
+      for (int u = 0; u < 8; ++u) {
+        uint32_t pk[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const int unit = c * 4 + q;  // 16-byte unit of the 256-byte row (0..15)
-          const int slab = unit >> 3, u = unit & 7;
-          *reinterpret_cast<uint4*>(pb + slab * kAttnTile + ((u ^ (r & 7)) << 4)) =
-              make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+          const __nv_bfloat162 h2 = __floats2bfloat162_rn(x[u * 8 + 2 * q], x[u * 8 + 2 * q + 1]);
+          pk[q] = *reinterpret_cast<const uint32_t*>(&h2);
         }
+        *reinterpret_cast<uint4*>(pb + ((u ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
+      const float rowsum = ((part[0] + part[1]) + (part[2] + part[3])) +
+                           ((part[4] + part[5]) + (part[6] + part[7]));
       l_run = l_run * alpha + rowsum;
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&p_full[b]);
     }
+    // denominators of the two halves
+    tmem_st1(xchg + 4 + half, l_run);
+    tc_fence_before();
+    named_barrier(bar_id, 64);
+    tc_fence_after();
+    const float l_tot = l_run + tmem_ld1(xchg + 4 + (1 - half));
     const long long row = (static_cast<long long>(split) * p.n_heads + head) * p.tq + tok;
-    float4* dst = reinterpret_cast<float4*>(p.o_part + row * 128);
+    float4* dst = reinterpret_cast<float4*>(p.o_part + row * 128 + 64 * half);
     const bool have_o = ok && n_tiles > 0 &&
                         mbar_wait(&pv_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, p.err);
     if (have_o) {
       tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         float v[32];
-        tmem_ld32(tmem_base + lane_off + c * 32, v);
+        tmem_ld32(tmem_base + 64 * half + 32 * c + lane_off, v);
         if (tok < p.n_queries) {
 #pragma unroll
           for (int i = 0; i < 8; ++i)
@@ -267,11 +316,10 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
     } else if (tok < p.n_queries) {
-      for (int i = 0; i < 32; ++i) dst[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-      m_run = -INFINITY;
-      l_run = 0.f;
+      for (int i = 0; i < 16; ++i) dst[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    if (tok < p.n_queries) p.ml_part[row] = make_float2(m_run, l_run);
+    if (tok < p.n_queries && half == 0)
+      p.ml_part[row] = have_o ? make_float2(m_run, l_tot) : make_float2(-INFINITY, 0.f);
   }
   tc_fence_before();
   __syncthreads();
@@ -281,28 +329,48 @@ __global__ void __launch_bounds__(192, 1)
   }
 }
 
-// Merge the key splits: O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s, stored bf16 into
-// o [T, Hq * 128] (token-major, ready to be the O-projection's token operand).
+// Merge the key splits: O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s, stored into
+// o [T, Hq * 128] (token-major, ready to be the O-projection's token operand).  One warp per
+// (token, head), 4 dims per lane; 8 warps per CTA.
 template <typename TA>
-__global__ void attn_combine_kernel(const float* __restrict__ o_part,
-                                    const float2* __restrict__ ml_part, int n_splits, int n_heads,
-                                    int tq, int n_queries, TA* __restrict__ o, const int* done) {
+__global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restrict__ o_part,
+                                                           const float2* __restrict__ ml_part,
+                                                           int n_splits, int n_heads, int tq,
+                                                           int n_queries, TA* __restrict__ o,
+                                                           const int* done) {
   if (block_done(done)) return;
-  const int tok = blockIdx.x, head = blockIdx.y, d = threadIdx.x;
-  if (tok >= n_queries) return;
+  const int pair = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (pair >= n_queries * n_heads) return;
+  const int tok = pair / n_heads, head = pair % n_heads, d4 = lane_id();
+  constexpr int kMax = 16;
+  float2 ml[kMax];
   float mmax = -INFINITY;
-  for (int s = 0; s < n_splits; ++s)
-    mmax = fmaxf(mmax, ml_part[(static_cast<long long>(s) * n_heads + head) * tq + tok].x);
-  float num = 0.f, den = 0.f;
-  for (int s = 0; s < n_splits; ++s) {
-    const long long row = (static_cast<long long>(s) * n_heads + head) * tq + tok;
-    const float2 ml = ml_part[row];
-    if (ml.y == 0.f) continue;
-    const float w = exp2f(ml.x - mmax);
-    num += w * o_part[row * 128 + d];
-    den += w * ml.y;
-  }
-  o[static_cast<long long>(tok) * n_heads * 128 + head * 128 + d] = store_from_f32<TA>(num / den);
+#pragma unroll
+  for (int s = 0; s < kMax; ++s)
+    if (s < n_splits) {
+      ml[s] = ml_part[(static_cast<long long>(s) * n_heads + head) * tq + tok];
+      mmax = fmaxf(mmax, ml[s].x);
+    }
+  float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+  float den = 0.f;
+#pragma unroll
+  for (int s = 0; s < kMax; ++s)
+    if (s < n_splits && ml[s].y != 0.f) {
+      const long long row = (static_cast<long long>(s) * n_heads + head) * tq + tok;
+      const float w = exp2f(ml[s].x - mmax);
+      const float4 v = reinterpret_cast<const float4*>(o_part + row * 128)[d4];
+      num.x += w * v.x;
+      num.y += w * v.y;
+      num.z += w * v.z;
+      num.w += w * v.w;
+      den += w * ml[s].y;
+    }
+  const float inv = 1.0f / den;
+  TA* dst = o + static_cast<long long>(tok) * n_heads * 128 + head * 128 + 4 * d4;
+  dst[0] = store_from_f32<TA>(num.x * inv);
+  dst[1] = store_from_f32<TA>(num.y * inv);
+  dst[2] = store_from_f32<TA>(num.z * inv);
+  dst[3] = store_from_f32<TA>(num.w * inv);
 }
 
 }  // namespace dg

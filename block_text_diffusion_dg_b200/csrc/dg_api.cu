@@ -146,14 +146,18 @@ int set_smem(K kernel, int bytes) {
 constexpr int kDenseN = 256, kDenseStages = 4;
 constexpr int kGroupN = 64, kGroupStages = 8;
 
+// ta2/tb2 are read only by items of the alternate group (p.alt_group >= 0).
 template <int MAXN, int STAGES, int EPI>
 int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, int grid,
-                cudaStream_t st, int kind = -1) {
+                cudaStream_t st, int kind = -1, const CUtensorMap* ta2 = nullptr,
+                const CUtensorMap* tb2 = nullptr) {
   auto k = gemm_swapab_kernel<MAXN, STAGES, EPI>;
   constexpr int smem = GemmCfg<MAXN, STAGES>::kSmemBytes;
+  if (p.alt_group >= 0 && (!ta2 || !tb2))
+    return fail(DG_ERR_INVALID_ARG, "alternate group without its tensor maps");
   DG_TRY(set_smem(k, smem));
   prof_before(kind, st);
-  k<<<grid, 192, smem, st>>>(ta, tb, p);
+  k<<<grid, GemmCfg<MAXN, STAGES>::kThreads, smem, st>>>(ta, tb, ta2 ? *ta2 : ta, tb2 ? *tb2 : tb, p);
   DG_LAUNCHED();
   prof_after(kind, st);
   return DG_OK;
@@ -162,6 +166,7 @@ int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& 
 GemmParams dense_params(int m_rows, int n_tokens, int k_dim, int k_splits, int* err,
                         const int* done) {
   GemmParams p{};
+  p.alt_group = -1;
   p.m_tiles = cdiv(m_rows, 128);
   p.k_splits = k_splits;
   p.n_chunk = kDenseN;
@@ -242,7 +247,11 @@ int check_config(const dg_config* c) {
   if (c->canvas > 256) return fail(DG_ERR_UNSUPPORTED, "canvas must be <= 256");
   if (c->kv_capacity % 8 != 0 || c->kv_capacity < c->canvas)
     return fail(DG_ERR_INVALID_ARG, "kv_capacity must be a multiple of 8 and >= canvas");
-  if (c->head_dim % 2 != 0) return fail(DG_ERR_INVALID_ARG, "head_dim must be even");
+  if (c->head_dim % 4 != 0) return fail(DG_ERR_INVALID_ARG, "head_dim must be a multiple of 4");
+  if (c->d_model % 4 != 0 || c->d_model > 4096)
+    return fail(DG_ERR_UNSUPPORTED, "d_model must be a multiple of 4 and at most 4096");
+  if (c->n_experts % 4 != 0)
+    return fail(DG_ERR_UNSUPPORTED, "n_experts must be a multiple of 4");
   if (c->vocab % 8 != 0) return fail(DG_ERR_UNSUPPORTED, "vocab must be a multiple of 8");
   if (c->max_steps < 1 || c->fixed_steps < 0)
     return fail(DG_ERR_INVALID_ARG, "max_steps must be >= 1 and fixed_steps >= 0");
@@ -301,8 +310,9 @@ Derived derive(const dg_config& c, int sms) {
   const int m_tiles = group * d.tq / 128;
   d.att_splits = std::max(1, std::min(16, sms / std::max(1, m_tiles * c.n_kv_heads)));
   const long long chunks = c.n_experts + (T * c.top_k + kGroupN - 1) / kGroupN;
-  d.max_items_gu = chunks * cdiv(2 * c.expert_hidden, 128);
-  d.max_items_d = chunks * cdiv(c.d_model, 128);
+  const long long sh_chunks = c.shared_hidden > 0 ? (T + kGroupN - 1) / kGroupN : 0;
+  d.max_items_gu = chunks * cdiv(2 * c.expert_hidden, 128) + sh_chunks * cdiv(2 * c.shared_hidden, 128);
+  d.max_items_d = (chunks + sh_chunks) * cdiv(c.d_model, 128);
   return d;
 }
 
@@ -360,6 +370,7 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
 int run_forward(dg_ctx* c, const int32_t* ids, int n, int pos0, int causal, const int* done,
                 cudaStream_t st) {
   const dg_config& g = c->cfg;
+  prof_before(DG_KERNEL_EMBED, st);
   if (c->bf16)
     embed_norm_kernel<__nv_bfloat16, __nv_bfloat16><<<n, 256, 0, st>>>(
         ids, static_cast<const __nv_bfloat16*>(c->embed), g.d_model, c->layers[0].attn_norm, g.eps,
@@ -369,6 +380,7 @@ int run_forward(dg_ctx* c, const int32_t* ids, int n, int pos0, int causal, cons
                                                        g.d_model, c->layers[0].attn_norm, g.eps,
                                                        c->x, static_cast<float*>(c->xn), done);
   DG_LAUNCHED();
+  prof_after(DG_KERNEL_EMBED, st);
   for (int l = 0; l < g.n_layers; ++l) {
     const float* nn = (l + 1 < g.n_layers) ? c->layers[l + 1].attn_norm : c->final_norm;
     DG_TRY(run_layer(c, l, n, pos0, causal, nn, done, st));
@@ -384,14 +396,12 @@ int layer_tail_common(dg_ctx* c, int l, int n, int pos0, const int* done, cudaSt
   const size_t kv_head_elems = static_cast<size_t>(g.kv_capacity) * hd;
   TA* kc = static_cast<TA*>(c->kc) + static_cast<size_t>(l) * g.n_kv_heads * kv_head_elems;
   TA* vtc = static_cast<TA*>(c->vtc) + static_cast<size_t>(l) * g.n_kv_heads * kv_head_elems;
-  rope_qk_kernel<TA><<<dim3(n, g.n_heads + g.n_kv_heads), hd / 2, 0, st>>>(
-      c->part, splits_qkv, qkv_ss, c->qkv_rows, hd, g.n_heads, c->rope_tab, pos0,
-      static_cast<TA*>(c->q), c->tq, kc, g.kv_capacity, done);
+  prof_before(DG_KERNEL_QKV_FINALIZE, st);
+  qkv_finalize_kernel<TA><<<dim3(cdiv(n, kQkvTok), g.n_heads + 2 * g.n_kv_heads), 128, 0, st>>>(
+      c->part, splits_qkv, qkv_ss, c->qkv_rows, hd, g.n_heads, g.n_kv_heads, c->rope_tab, n, pos0,
+      static_cast<TA*>(c->q), c->tq, kc, vtc, g.kv_capacity, done);
   DG_LAUNCHED();
-  v_store_kernel<TA><<<dim3(cdiv(n, 32), g.n_kv_heads), dim3(32, 8), 0, st>>>(
-      c->part, splits_qkv, qkv_ss, c->qkv_rows, hd, (g.n_heads + g.n_kv_heads) * hd, n, pos0, vtc,
-      g.kv_capacity, done);
-  DG_LAUNCHED();
+  prof_after(DG_KERNEL_QKV_FINALIZE, st);
   return DG_OK;
 }
 
@@ -496,14 +506,16 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     a.done = done;
     DG_TRY(set_smem(attention_kernel, kAttnSmemBytes));
     prof_before(DG_KERNEL_ATTENTION, st);
-    attention_kernel<<<dim3(m_tiles, g.n_kv_heads, splits), 192, kAttnSmemBytes, st>>>(
+    attention_kernel<<<dim3(m_tiles, g.n_kv_heads, splits), kAttnThreads, kAttnSmemBytes, st>>>(
         c->tm_q, c->tm_k, c->tm_vt, a);
     DG_LAUNCHED();
     prof_after(DG_KERNEL_ATTENTION, st);
-    attn_combine_kernel<__nv_bfloat16><<<dim3(n, g.n_heads), 128, 0, st>>>(
+    prof_before(DG_KERNEL_ATTN_COMBINE, st);
+    attn_combine_kernel<__nv_bfloat16><<<cdiv(n * g.n_heads, 8), 256, 0, st>>>(
         c->o_part, c->ml_part, splits, g.n_heads, c->tq, n, static_cast<__nv_bfloat16*>(c->o),
         done);
     DG_LAUNCHED();
+    prof_after(DG_KERNEL_ATTN_COMBINE, st);
   }
   // O projection + residual + ffn norm
   {
@@ -515,10 +527,12 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     DG_TRY((launch_gemm<kDenseN, kDenseStages, kEpiPartialF32>(c->tm_wo[l], c->tm_o32, p,
                                                                  std::min(items, c->sms), st,
                                                                  DG_KERNEL_O_PROJ)));
+    prof_before(DG_KERNEL_RESIDUAL_NORM, st);
     residual_norm_kernel<__nv_bfloat16><<<n, 256, 0, st>>>(
         c->x, c->part, c->split_o, p.split_stride, d, w.ffn_norm, g.eps,
         static_cast<__nv_bfloat16*>(c->xn), done);
     DG_LAUNCHED();
+    prof_after(DG_KERNEL_RESIDUAL_NORM, st);
   }
   // router + top-k
   {
@@ -528,12 +542,16 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     p.split_stride = static_cast<long long>(n) * E;
     const int items = p.m_tiles * p.k_splits * p.n_chunks;
     DG_TRY((launch_gemm<kDenseN, kDenseStages, kEpiPartialF32>(c->tm_wr[l], c->tm_xn32, p,
-                                                                 std::min(items, c->sms), st)));
+                                                                 std::min(items, c->sms), st,
+                                                                 DG_KERNEL_ROUTER)));
+    prof_before(DG_KERNEL_ROUTER_TOPK, st);
     router_topk_kernel<<<cdiv(n, 4), 128, 0, st>>>(c->part, c->split_r, p.split_stride, n, E, k,
                                                    c->router_logits, c->topk_ids, c->topk_w, done);
     DG_LAUNCHED();
+    prof_after(DG_KERNEL_ROUTER_TOPK, st);
   }
-  // permutation and grouped expert GEMMs
+  // permutation and grouped expert GEMMs; the shared expert rides along as group E
+  const bool shared = g.shared_hidden > 0;
   {
     RouteArgs ra{};
     ra.ids = c->topk_ids;
@@ -547,13 +565,20 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     ra.m_tiles_gu = cdiv(2 * g.expert_hidden, 128);
     ra.m_tiles_d = cdiv(d, 128);
     ra.n_chunk = kGroupN;
+    ra.n_tokens = n;
+    ra.shared_m_tiles_gu = shared ? cdiv(2 * g.shared_hidden, 128) : 0;
+    ra.shared_m_tiles_d = shared ? cdiv(d, 128) : 0;
     ra.done = done;
+    prof_before(DG_KERNEL_ROUTE, st);
     moe_route_kernel<<<1, 1024, 0, st>>>(ra);
     DG_LAUNCHED();
-    gather_rows_kernel<<<n_slots, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(c->xn), c->perm,
-                                                k, d, static_cast<__nv_bfloat16*>(c->x_perm),
-                                                done);
+    prof_after(DG_KERNEL_ROUTE, st);
+    prof_before(DG_KERNEL_GATHER, st);
+    gather_rows_kernel<<<cdiv(n_slots, 4), 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(c->xn), c->perm, k, d, n_slots,
+        static_cast<__nv_bfloat16*>(c->x_perm), done);
     DG_LAUNCHED();
+    prof_after(DG_KERNEL_GATHER, st);
     GemmParams p{};
     p.items = c->items_gu;
     p.item_count = c->item_counts;
@@ -562,10 +587,16 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     p.m_valid = 2 * g.expert_hidden;
     p.out_bf16 = static_cast<__nv_bfloat16*>(c->h);
     p.ld_out = g.expert_hidden;
+    p.alt_group = shared ? E : -1;
+    p.alt_kb_total = d / 64;
+    p.alt_m_valid = 2 * g.shared_hidden;
+    p.alt_out_bf16 = static_cast<__nv_bfloat16*>(c->hs);
+    p.alt_ld_out = g.shared_hidden;
     p.err = c->err;
     p.done = done;
-    DG_TRY((launch_gemm<kGroupN, kGroupStages, kEpiGluBf16>(c->tm_wgu[l], c->tm_xperm, p, c->sms,
-                                                             st, DG_KERNEL_EXPERT_GATE_UP)));
+    DG_TRY((launch_gemm<kGroupN, kGroupStages, kEpiGluBf16>(
+        c->tm_wgu[l], c->tm_xperm, p, c->sms, st, DG_KERNEL_EXPERT_GATE_UP,
+        shared ? &c->tm_wsgu[l] : nullptr, shared ? &c->tm_xn32 : nullptr)));
     GemmParams q{};
     q.items = c->items_d;
     q.item_count = c->item_counts + 1;
@@ -576,32 +607,23 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     q.ld_out = d;
     q.perm = c->perm;
     q.scale = c->topk_w;
+    q.alt_group = shared ? E : -1;
+    q.alt_kb_total = g.shared_hidden / 64;
+    q.alt_m_valid = d;
+    q.alt_out_f32 = c->y_shared;
+    q.alt_ld_out = d;
     q.err = c->err;
     q.done = done;
-    DG_TRY((launch_gemm<kGroupN, kGroupStages, kEpiScatterF32>(c->tm_wd[l], c->tm_h, q, c->sms,
-                                                                st, DG_KERNEL_EXPERT_DOWN)));
+    DG_TRY((launch_gemm<kGroupN, kGroupStages, kEpiScatterF32>(
+        c->tm_wd[l], c->tm_h, q, c->sms, st, DG_KERNEL_EXPERT_DOWN,
+        shared ? &c->tm_wsd[l] : nullptr, shared ? &c->tm_hs : nullptr)));
   }
-  const float* ysh = nullptr;
-  if (g.shared_hidden > 0) {
-    GemmParams p = dense_params(2 * g.shared_hidden, n, d, 1, c->err, done);
-    p.out_bf16 = static_cast<__nv_bfloat16*>(c->hs);
-    p.ld_out = g.shared_hidden;
-    int items = p.m_tiles * p.n_chunks;
-    DG_TRY((launch_gemm<kDenseN, kDenseStages, kEpiGluBf16>(c->tm_wsgu[l], c->tm_xn32, p,
-                                                              std::min(items, c->sms), st,
-                                                              DG_KERNEL_SHARED_EXPERT)));
-    GemmParams q = dense_params(d, n, g.shared_hidden, 1, c->err, done);
-    q.out_f32 = c->y_shared;
-    q.ld_out = d;
-    items = q.m_tiles * q.n_chunks;
-    DG_TRY((launch_gemm<kDenseN, kDenseStages, kEpiScatterF32>(c->tm_wsd[l], c->tm_hs, q,
-                                                                 std::min(items, c->sms), st,
-                                                                 DG_KERNEL_SHARED_EXPERT)));
-    ysh = c->y_shared;
-  }
+  const float* ysh = shared ? c->y_shared : nullptr;
+  prof_before(DG_KERNEL_COMBINE_NORM, st);
   moe_combine_norm_kernel<__nv_bfloat16><<<n, 256, 0, st>>>(
       c->x, c->y_slot, k, ysh, d, next_norm, g.eps, static_cast<__nv_bfloat16*>(c->xn), done);
   DG_LAUNCHED();
+  prof_after(DG_KERNEL_COMBINE_NORM, st);
   return DG_OK;
 }
 
@@ -622,10 +644,10 @@ int run_lm_head(dg_ctx* c, float* logits_out, const int* done, cudaStream_t st) 
     prof_before(DG_KERNEL_LM_HEAD, st);
     if (logits_out) {
       DG_TRY(set_smem(lmhead_kernel<false>, kLmSmemBytes));
-      lmhead_kernel<false><<<grid, 192, kLmSmemBytes, st>>>(c->tm_xn128, c->tm_embed, p);
+      lmhead_kernel<false><<<grid, kLmThreads, kLmSmemBytes, st>>>(c->tm_xn128, c->tm_embed, p);
     } else {
       DG_TRY(set_smem(lmhead_kernel<true>, kLmSmemBytes));
-      lmhead_kernel<true><<<grid, 192, kLmSmemBytes, st>>>(c->tm_xn128, c->tm_embed, p);
+      lmhead_kernel<true><<<grid, kLmThreads, kLmSmemBytes, st>>>(c->tm_xn128, c->tm_embed, p);
     }
     DG_LAUNCHED();
     prof_after(DG_KERNEL_LM_HEAD, st);
@@ -1144,10 +1166,10 @@ int dg_canvas_attention(const void* d_q, const void* d_k, const void* d_vt, void
   cudaStream_t st = S(stream);
   DG_CUDA(cudaMemsetAsync(a.err, 0, 4, st));
   DG_TRY(set_smem(attention_kernel, kAttnSmemBytes));
-  attention_kernel<<<dim3(m_tiles, n_kv_heads, splits), 192, kAttnSmemBytes, st>>>(tq_m, tk_m, tv_m,
+  attention_kernel<<<dim3(m_tiles, n_kv_heads, splits), kAttnThreads, kAttnSmemBytes, st>>>(tq_m, tk_m, tv_m,
                                                                                   a);
   DG_LAUNCHED();
-  attn_combine_kernel<__nv_bfloat16><<<dim3(t, n_heads), 128, 0, st>>>(
+  attn_combine_kernel<__nv_bfloat16><<<cdiv(t * n_heads, 8), 256, 0, st>>>(
       a.o_part, a.ml_part, splits, n_heads, tq, t, static_cast<__nv_bfloat16*>(d_o), nullptr);
   DG_LAUNCHED();
   return DG_OK;
@@ -1165,8 +1187,9 @@ MoePlan moe_plan(int t, int d, int E, int k, int hid, int hs) {
   MoePlan m{};
   m.split_r = std::min(16, std::max(1, d / 64 / 4));
   const long long chunks = E + (static_cast<long long>(t) * k + kGroupN - 1) / kGroupN;
-  m.items_gu = chunks * cdiv(2 * hid, 128);
-  m.items_d = chunks * cdiv(d, 128);
+  const long long sh_chunks = hs > 0 ? (t + kGroupN - 1) / kGroupN : 0;
+  m.items_gu = chunks * cdiv(2 * hid, 128) + sh_chunks * cdiv(2 * hs, 128);
+  m.items_d = (chunks + sh_chunks) * cdiv(d, 128);
   size_t sz[12];
   sz[0] = static_cast<size_t>(m.split_r) * t * E * 4;  // router partials
   sz[1] = static_cast<size_t>(t) * k * 4;              // ids (internal)
@@ -1193,7 +1216,8 @@ MoePlan moe_plan(int t, int d, int E, int k, int hid, int hs) {
 
 int dg_moe_workspace_bytes(int32_t t, int32_t d, int32_t n_experts, int32_t top_k, int32_t hidden,
                            int32_t shared_hidden, size_t* bytes) {
-  if (t < 1 || d < 64 || d % 64 || n_experts < 1 || n_experts > 256 || top_k < 1 || top_k > 8 ||
+  if (t < 1 || d < 64 || d % 64 || d > 4096 || n_experts < 4 || n_experts % 4 || n_experts > 256 ||
+      top_k < 1 || top_k > 8 ||
       top_k > n_experts || hidden < 64 || hidden % 64 || shared_hidden < 0 || shared_hidden % 64 ||
       !bytes)
     return fail(DG_ERR_INVALID_ARG, "bad MoE shape");
@@ -1255,6 +1279,7 @@ int dg_moe_ffn(const void* d_x, const float* d_residual, const void* d_wr, const
   router_topk_kernel<<<cdiv(t, 4), 128, 0, st>>>(rpart, m.split_r, pr.split_stride, t, n_experts,
                                                  top_k, d_router_logits, ids, wts, nullptr);
   DG_LAUNCHED();
+  const bool shared = shared_hidden > 0;
   RouteArgs ra{};
   ra.ids = ids;
   ra.n_slots = t * top_k;
@@ -1267,11 +1292,14 @@ int dg_moe_ffn(const void* d_x, const float* d_residual, const void* d_wr, const
   ra.m_tiles_gu = cdiv(2 * hidden, 128);
   ra.m_tiles_d = cdiv(d, 128);
   ra.n_chunk = kGroupN;
+  ra.n_tokens = t;
+  ra.shared_m_tiles_gu = shared ? cdiv(2 * shared_hidden, 128) : 0;
+  ra.shared_m_tiles_d = shared ? cdiv(d, 128) : 0;
   ra.done = nullptr;
   moe_route_kernel<<<1, 1024, 0, st>>>(ra);
   DG_LAUNCHED();
-  gather_rows_kernel<<<t * top_k, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(d_x), perm, top_k,
-                                                d, x_perm, nullptr);
+  gather_rows_kernel<<<cdiv(t * top_k, 4), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(d_x),
+                                                         perm, top_k, d, t * top_k, x_perm, nullptr);
   DG_LAUNCHED();
   GemmParams pg{};
   pg.items = items_gu;
@@ -1281,8 +1309,15 @@ int dg_moe_ffn(const void* d_x, const float* d_residual, const void* d_wr, const
   pg.m_valid = 2 * hidden;
   pg.out_bf16 = hbuf;
   pg.ld_out = hidden;
+  pg.alt_group = shared ? n_experts : -1;
+  pg.alt_kb_total = d / 64;
+  pg.alt_m_valid = 2 * shared_hidden;
+  pg.alt_out_bf16 = hsbuf;
+  pg.alt_ld_out = shared_hidden;
   pg.err = err;
-  DG_TRY((launch_gemm<kGroupN, kGroupStages, kEpiGluBf16>(t_wgu, t_xp, pg, sms, st)));
+  DG_TRY((launch_gemm<kGroupN, kGroupStages, kEpiGluBf16>(t_wgu, t_xp, pg, sms, st, -1,
+                                                           shared ? &t_wsgu : nullptr,
+                                                           shared ? &t_x32 : nullptr)));
   GemmParams pd{};
   pd.items = items_d;
   pd.item_count = icnt + 1;
@@ -1293,22 +1328,16 @@ int dg_moe_ffn(const void* d_x, const float* d_residual, const void* d_wr, const
   pd.ld_out = d;
   pd.perm = perm;
   pd.scale = wts;
+  pd.alt_group = shared ? n_experts : -1;
+  pd.alt_kb_total = shared_hidden / 64;
+  pd.alt_m_valid = d;
+  pd.alt_out_f32 = ysh;
+  pd.alt_ld_out = d;
   pd.err = err;
-  DG_TRY((launch_gemm<kGroupN, kGroupStages, kEpiScatterF32>(t_wd, t_h, pd, sms, st)));
-  const float* ysh_ptr = nullptr;
-  if (shared_hidden > 0) {
-    GemmParams p = dense_params(2 * shared_hidden, t, d, 1, err, nullptr);
-    p.out_bf16 = hsbuf;
-    p.ld_out = shared_hidden;
-    DG_TRY((launch_gemm<kDenseN, kDenseStages, kEpiGluBf16>(
-        t_wsgu, t_x32, p, std::min(p.m_tiles * p.n_chunks, sms), st)));
-    GemmParams q = dense_params(d, t, shared_hidden, 1, err, nullptr);
-    q.out_f32 = ysh;
-    q.ld_out = d;
-    DG_TRY((launch_gemm<kDenseN, kDenseStages, kEpiScatterF32>(
-        t_wsd, t_hs, q, std::min(q.m_tiles * q.n_chunks, sms), st)));
-    ysh_ptr = ysh;
-  }
+  DG_TRY((launch_gemm<kGroupN, kGroupStages, kEpiScatterF32>(t_wd, t_h, pd, sms, st, -1,
+                                                              shared ? &t_wsd : nullptr,
+                                                              shared ? &t_hs : nullptr)));
+  const float* ysh_ptr = shared ? ysh : nullptr;
   if (d_residual)
     DG_CUDA(cudaMemcpyAsync(d_y, d_residual, static_cast<size_t>(t) * d * 4,
                             cudaMemcpyDeviceToDevice, st));

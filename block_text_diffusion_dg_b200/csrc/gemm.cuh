@@ -37,16 +37,27 @@ struct GemmParams {
   long long split_stride;
   const int* perm;
   const float* scale;
+  // alternate group (the shared expert folded into a grouped launch): items whose group id is
+  // alt_group read tm_a2 / tm_b2, run alt_kb_total K slabs and write alt_out_* (no permutation,
+  // weight 1)
+  int alt_group;
+  int alt_kb_total;
+  int alt_m_valid;
+  float* alt_out_f32;
+  __nv_bfloat16* alt_out_bf16;
+  long long alt_ld_out;
   int* err;
   const int* done;
 };
 
 struct GemmItem {
   int a_row, b_row, n, kb0, kb1, r_base, aux;
+  bool alt;
 };
 
 DG_DEV GemmItem gemm_item(const GemmParams& p, int it) {
   GemmItem w;
+  w.alt = false;
   if (p.items == nullptr) {
     const int mt = it % p.m_tiles;
     const int rest = it / p.m_tiles;
@@ -61,12 +72,13 @@ DG_DEV GemmItem gemm_item(const GemmParams& p, int it) {
     w.aux = split;
   } else {
     const int4 e = p.items[it];
+    w.alt = e.x == p.alt_group;
     w.r_base = e.y * 128;
-    w.a_row = e.x * p.a_rows_per_group + w.r_base;
+    w.a_row = (w.alt ? 0 : e.x * p.a_rows_per_group) + w.r_base;
     w.b_row = e.z;
     w.n = e.w;
     w.kb0 = 0;
-    w.kb1 = p.kb_total;
+    w.kb1 = w.alt ? p.alt_kb_total : p.kb_total;
     w.aux = e.x;
   }
   return w;
@@ -82,46 +94,68 @@ struct GemmCfg {
   static constexpr int kABytes = 128 * 128;   // 128 rows x 64 bf16
   static constexpr int kBBytes = MAXN * 128;  // MAXN rows x 64 bf16
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kTmemCols = 2 * MAXN;
+  static constexpr int kAccBufs = MAXN <= 128 ? 4 : 2;  // TMEM accumulators in flight
+  static constexpr int kTmemCols = kAccBufs * MAXN;
+  // epilogue warps: two per TMEM lane quarter for wide token tiles (they split the columns)
+  static constexpr int kEpiWarps = MAXN >= 128 ? 8 : 4;
+  static constexpr int kThreads = 64 + 32 * kEpiWarps;
   static constexpr int kSmemBytes = STAGES * kStageBytes + 1024 + 256;
   static_assert(MAXN % 32 == 0 && MAXN >= 32 && MAXN <= 256, "MAXN");
 };
 
 template <int EPI>
 DG_DEV void gemm_epilogue_chunk(const GemmParams& p, const GemmItem& w, const float (&v)[32],
-                                int c, int r) {
+                                int c, int r, int dst_lane = 0, float scale_lane = 1.0f) {
   const int row = w.r_base + r;  // row inside the group (output feature / gate-up row)
+  const int m_valid = w.alt ? p.alt_m_valid : p.m_valid;
   if constexpr (EPI == kEpiPartialF32) {
-    if (row < p.m_valid) {
-      float* o = p.out_f32 + static_cast<long long>(w.aux) * p.split_stride + row;
+    if (row < m_valid) {
+      float* o = p.out_f32 + static_cast<long long>(w.aux) * p.split_stride +
+                 static_cast<long long>(w.b_row + c) * p.ld_out + row;
+      const long long ld = p.ld_out;
+      if (c + 32 <= w.n) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i)
-        if (c + i < w.n) o[static_cast<long long>(w.b_row + c + i) * p.ld_out] = v[i];
+        for (int i = 0; i < 32; ++i, o += ld) *o = v[i];
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i, o += ld)
+          if (c + i < w.n) *o = v[i];
+      }
     }
   } else if constexpr (EPI == kEpiGluBf16) {
     // rows come in (gate, up) pairs on adjacent lanes: lane 2u has gate unit u, 2u+1 up unit u
     const bool gate_lane = (lane_id() & 1) == 0;
     const int unit = row >> 1;
+    const long long ld = w.alt ? p.alt_ld_out : p.ld_out;
+    // gate lanes store tokens c..c+15, up lanes tokens c+16..c+31
+    __nv_bfloat16* out = (w.alt ? p.alt_out_bf16 : p.out_bf16) +
+                         static_cast<long long>(w.b_row + c + (gate_lane ? 0 : 16)) * ld + unit;
+    const bool ok_row = row < m_valid;
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
       const float other = __shfl_xor_sync(0xffffffffu, v[i], 1);
-      if (((i >> 4) & 1) == (gate_lane ? 0 : 1) && c + i < w.n && row < p.m_valid) {
-        const float g = gate_lane ? v[i] : other;
-        const float u = gate_lane ? other : v[i];
-        const float h = g / (1.0f + __expf(-g)) * u;
-        p.out_bf16[static_cast<long long>(w.b_row + c + i) * p.ld_out + unit] =
-            __float2bfloat16_rn(h);
+      if (((i >> 4) & 1) == (gate_lane ? 0 : 1)) {
+        if (ok_row && c + i < w.n) {
+          const float g = gate_lane ? v[i] : other;
+          const float u = gate_lane ? other : v[i];
+          *out = __float2bfloat16_rn(g / (1.0f + __expf(-g)) * u);
+        }
+        out += ld;
       }
     }
   } else {  // kEpiScatterF32
-    if (row < p.m_valid) {
+    if (row < m_valid) {
+      if (w.alt) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        if (c + i < w.n) {
-          const int src = w.b_row + c + i;
-          const int dst = p.perm ? p.perm[src] : src;
-          const float s = p.scale ? p.scale[dst] : 1.0f;
-          p.out_f32[static_cast<long long>(dst) * p.ld_out + row] = v[i] * s;
+        for (int i = 0; i < 32; ++i)
+          if (c + i < w.n) p.alt_out_f32[static_cast<long long>(w.b_row + c + i) * p.alt_ld_out + row] = v[i];
+      } else {
+        // lane i of the warp holds the destination row and weight of token c + i
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int dst = __shfl_sync(0xffffffffu, dst_lane, i);
+          const float s = __shfl_sync(0xffffffffu, scale_lane, i);
+          if (c + i < w.n) p.out_f32[static_cast<long long>(dst) * p.ld_out + row] = v[i] * s;
         }
       }
     }
@@ -129,9 +163,11 @@ DG_DEV void gemm_epilogue_chunk(const GemmParams& p, const GemmItem& w, const fl
 }
 
 template <int MAXN, int STAGES, int EPI>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(GemmCfg<MAXN, STAGES>::kThreads, 1)
     gemm_swapab_kernel(const __grid_constant__ CUtensorMap tm_a,
-                       const __grid_constant__ CUtensorMap tm_b, const GemmParams p) {
+                       const __grid_constant__ CUtensorMap tm_b,
+                       const __grid_constant__ CUtensorMap tm_a2,
+                       const __grid_constant__ CUtensorMap tm_b2, const GemmParams p) {
   using C = GemmCfg<MAXN, STAGES>;
   if (block_done(p.done)) return;
   extern __shared__ uint8_t smem_raw[];
@@ -140,8 +176,8 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * C::kStageBytes);
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;
-  uint64_t* acc_empty = acc_full + 2;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  uint64_t* acc_empty = acc_full + C::kAccBufs;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_empty + C::kAccBufs);
   const int warp = threadIdx.x >> 5;
 
   if (warp == 0 && lane_id() == 0) {
@@ -149,13 +185,17 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < C::kAccBufs; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 128);
+      mbar_init(&acc_empty[b], 32 * C::kEpiWarps);
     }
     fence_barrier_init();
     tma_prefetch_desc(&tm_a);
     tma_prefetch_desc(&tm_b);
+    if (p.alt_group >= 0) {
+      tma_prefetch_desc(&tm_a2);
+      tma_prefetch_desc(&tm_b2);
+    }
   }
   if (warp == 1) {
     tmem_alloc(tmem_holder, C::kTmemCols);
@@ -178,6 +218,8 @@ __global__ void __launch_bounds__(192, 1)
         const GemmItem w = gemm_item(p, it);
         const int nbox = (w.n + 31) >> 5;
         const uint32_t bytes = C::kABytes + nbox * 32 * 128;
+        const CUtensorMap* ta = w.alt ? &tm_a2 : &tm_a;
+        const CUtensorMap* tb = w.alt ? &tm_b2 : &tm_b;
         for (int kb = w.kb0; kb < w.kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, p.err)) {
             ok = false;
@@ -186,9 +228,9 @@ __global__ void __launch_bounds__(192, 1)
           uint8_t* sa = smem + stage * C::kStageBytes;
           uint8_t* sb = sa + C::kABytes;
           mbar_arrive_expect_tx(&full[stage], bytes);
-          tma_load_2d(&tm_a, &full[stage], sa, kb * 64, w.a_row, pol_a);
+          tma_load_2d(ta, &full[stage], sa, kb * 64, w.a_row, pol_a);
           for (int bx = 0; bx < nbox; ++bx)
-            tma_load_2d(&tm_b, &full[stage], sb + bx * 4096, kb * 64, w.b_row + bx * 32, pol_b);
+            tma_load_2d(tb, &full[stage], sb + bx * 4096, kb * 64, w.b_row + bx * 32, pol_b);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
@@ -226,7 +268,7 @@ __global__ void __launch_bounds__(192, 1)
           }
         }
         umma_commit(&acc_full[acc]);
-        if (++acc == 2) {
+        if (++acc == C::kAccBufs) {
           acc = 0;
           acc_phase ^= 1u;
         }
@@ -235,21 +277,46 @@ __global__ void __launch_bounds__(192, 1)
   } else {
     const int q = warp & 3;
     const int r = q * 32 + lane_id();
+    constexpr int kGroups = C::kEpiWarps / 4;  // warps sharing a lane quarter split the chunks
+    const int grp = (warp - 2) >> 2;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
       const GemmItem w = gemm_item(p, it);
+      // scatter: this lane's token of each 32-wide chunk, loaded before the accumulator is ready
+      int dst_lane[MAXN / 32];
+      float scale_lane[MAXN / 32];
+      if constexpr (EPI == kEpiScatterF32) {
+#pragma unroll
+        for (int cc = 0; cc < MAXN / 32; ++cc) {
+          const int j = cc * 32 + lane_id();
+          dst_lane[cc] = 0;
+          scale_lane[cc] = 1.0f;
+          if (!w.alt && j < w.n) {
+            const int dst = p.perm ? p.perm[w.b_row + j] : w.b_row + j;
+            dst_lane[cc] = dst;
+            scale_lane[cc] = p.scale ? p.scale[dst] : 1.0f;
+          }
+        }
+      }
       if (!mbar_wait(&acc_full[acc], acc_phase, p.err)) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + acc * MAXN + (static_cast<uint32_t>(q * 32) << 16);
-      for (int c = 0; c < w.n; c += 32) {
-        float v[32];
-        tmem_ld32(t_row + c, v);
-        gemm_epilogue_chunk<EPI>(p, w, v, c, r);
+#pragma unroll
+      for (int cc = 0; cc < MAXN / 32; ++cc) {
+        const int c = cc * 32;
+        if (cc % kGroups == grp && c < w.n) {
+          float v[32];
+          tmem_ld32(t_row + c, v);
+          if constexpr (EPI == kEpiScatterF32)
+            gemm_epilogue_chunk<EPI>(p, w, v, c, r, dst_lane[cc], scale_lane[cc]);
+          else
+            gemm_epilogue_chunk<EPI>(p, w, v, c, r);
+        }
       }
       tc_fence_before();
       mbar_arrive(&acc_empty[acc]);
-      if (++acc == 2) {
+      if (++acc == C::kAccBufs) {
         acc = 0;
         acc_phase ^= 1u;
       }
@@ -279,8 +346,10 @@ constexpr int kLmStages = 3;
 constexpr int kLmStageBytes = 2 * 16384 + 32768;  // two token tiles + one 256-row vocab tile
 constexpr int kLmSmemBytes = kLmStages * kLmStageBytes + 1024 + 256;
 
+constexpr int kLmThreads = 64 + 32 * 8;  // TMA, MMA, two epilogue warpgroups (one per token tile)
+
 template <bool kStats>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kLmThreads, 1)
     lmhead_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_e,
                   const LmHeadParams p) {
   if (block_done(p.done)) return;
@@ -301,7 +370,7 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&empty[s], 1);
     }
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 128);
+    mbar_init(acc_empty, 256);
     fence_barrier_init();
     tma_prefetch_desc(&tm_x);
     tma_prefetch_desc(&tm_e);
@@ -377,27 +446,40 @@ __global__ void __launch_bounds__(192, 1)
   } else {
     const int q = warp & 3;
     const int r = q * 32 + lane_id();
+    const int tt = (warp - 2) >> 2;  // token tile of this epilogue warpgroup
     uint32_t acc_phase = 0;
     for (int vt = blockIdx.x; vt < p.n_vtiles; vt += gridDim.x) {
       if (!mbar_wait(acc_full, acc_phase, p.err)) break;
       tc_fence_after();
-      for (int tt = 0; tt < n_ttiles; ++tt) {
+      if (tt < n_ttiles) {
         const int tok = tt * 128 + r;
         const uint32_t t_row = tmem_base + tt * 256 + (static_cast<uint32_t>(q * 32) << 16);
         if constexpr (kStats) {
           float m = -INFINITY;
           int a = 0;
+#pragma unroll 1
           for (int c = 0; c < 256; c += 32) {
             float v[32];
             tmem_ld32(t_row + c, v);
+            // tree argmax of the chunk, lowest index on equal values
+            int idx[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (v[i] > m) {
-                m = v[i];
-                a = c + i;
+            for (int i = 0; i < 32; ++i) idx[i] = i;
+#pragma unroll
+            for (int w = 16; w >= 1; w >>= 1)
+#pragma unroll
+              for (int i = 0; i < w; ++i) {
+                const bool take = v[i + w] > v[i] || (v[i + w] == v[i] && idx[i + w] < idx[i]);
+                v[i] = take ? v[i + w] : v[i];
+                idx[i] = take ? idx[i + w] : idx[i];
               }
+            if (v[0] > m) {  // strict: an earlier chunk keeps equal maxima
+              m = v[0];
+              a = c + idx[0];
+            }
           }
-          float s = 0.f, u = 0.f;
+          float s4[4] = {0.f, 0.f, 0.f, 0.f}, u4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
           for (int c = 0; c < 256; c += 32) {
             float v[32];
             tmem_ld32(t_row + c, v);
@@ -405,10 +487,12 @@ __global__ void __launch_bounds__(192, 1)
             for (int i = 0; i < 32; ++i) {
               const float d = v[i] - m;
               const float e = __expf(d);
-              s += e;
-              u = fmaf(e, d, u);
+              s4[i & 3] += e;
+              u4[i & 3] = fmaf(e, d, u4[i & 3]);
             }
           }
+          const float s = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+          const float u = (u4[0] + u4[1]) + (u4[2] + u4[3]);
           if (tok < p.n_tokens)
             p.partials[static_cast<long long>(tok) * p.n_vtiles + vt] =
                 StatPartial{m, s, u, vt * 256 + a};

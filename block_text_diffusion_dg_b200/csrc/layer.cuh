@@ -1,9 +1,9 @@
 // layer.cuh -- the non-GEMM kernels of one decoder layer (bandwidth-bound, one pass each).
 //
 //   embed_norm        x = E[ids] (fp32 residual), xn = rmsnorm(x) * w        (a1, a2)
-//   rope_qk           sum split-K partials, rotate-half RoPE at absolute positions, store
-//                     Q [Hq, Tq, hd] and K into the cache slots P..P+n-1       (a3)
-//   v_store           sum partials, store V transposed into V^T [hd, cap]      (a3)
+//   qkv_finalize      sum split-K partials; rotate-half RoPE at absolute positions for q and
+//                     k heads (Q [Hq, Tq, hd], K cache slots P..P+n-1); V stored transposed
+//                     into V^T [hd, cap]                                       (a3)
 //   residual_norm     x += O-projection partials; xn2 = rmsnorm(x) * w         (a5, a2)
 //   router_topk       router logits -> top-k ids (lowest index on ties) and the softmax of
 //                     the selected logits (= renormalised full-softmax probabilities) (a6)
@@ -52,61 +52,91 @@ __global__ void __launch_bounds__(256) embed_norm_kernel(const int32_t* __restri
         store_from_f32<TA>(x[static_cast<long long>(t) * d + i] * inv * w[i]);
 }
 
-// grid (n tokens, Hq + Hkv); threads = hd / 2; thread i rotates dims (i, i + hd/2).
-template <typename TA>
-__global__ void rope_qk_kernel(const float* __restrict__ part, int splits, long long split_stride,
-                               int ld, int hd, int n_heads, const float2* __restrict__ rope_tab,
-                               int pos0, TA* __restrict__ q, int tq, TA* __restrict__ k_cache,
-                               int ldk, const int* done) {
-  if (block_done(done)) return;
-  const int t = blockIdx.x, h = blockIdx.y, i = threadIdx.x, half = hd >> 1;
-  const int col = h * hd + i;
-  float a = 0.f, b = 0.f;
-  for (int s = 0; s < splits; ++s) {
-    const float* src = part + s * split_stride + static_cast<long long>(t) * ld + col;
-    a += src[0];
-    b += src[half];
-  }
-  const float2 cs = rope_tab[static_cast<long long>(pos0 + t) * half + i];  // (cos, sin)
-  const float ra = a * cs.x - b * cs.y;
-  const float rb = b * cs.x + a * cs.y;
-  TA* dst;
-  if (h < n_heads) {
-    dst = q + (static_cast<long long>(h) * tq + t) * hd;
-  } else {
-    dst = k_cache + (static_cast<long long>(h - n_heads) * ldk + pos0 + t) * hd;
-  }
-  dst[i] = store_from_f32<TA>(ra);
-  dst[i + half] = store_from_f32<TA>(rb);
-}
-
-// V heads: transpose [token, dim] partial sums into V^T [hd, cap] at columns pos0 + t.
-// grid (ceil(n / 32), Hkv); block (32, 8).
-template <typename TA>
-__global__ void v_store_kernel(const float* __restrict__ part, int splits, long long split_stride,
-                               int ld, int hd, int v_col0, int n, int pos0,
-                               TA* __restrict__ vt_cache, int ldk, const int* done) {
-  if (block_done(done)) return;
-  __shared__ float tile[128][33];
-  const int t0 = blockIdx.x * 32, g = blockIdx.y;
-  for (int tt = threadIdx.y; tt < 32; tt += 8) {
-    const int t = t0 + tt;
-    for (int dd = threadIdx.x; dd < hd; dd += 32) {
-      float v = 0.f;
-      if (t < n)
-        for (int s = 0; s < splits; ++s)
-          v += part[s * split_stride + static_cast<long long>(t) * ld + v_col0 + g * hd + dd];
-      tile[dd][tt] = v;
+// Sum of up to kMaxSplits split-K partials of one float4 column block (independent loads).
+constexpr int kMaxSplits = 16;
+DG_DEV float4 sum_splits4(const float* part, int splits, long long split_stride, long long off) {
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int s = 0; s < kMaxSplits; ++s) {
+    if (s < splits) {
+      const float4 v = *reinterpret_cast<const float4*>(part + s * split_stride + off);
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
     }
   }
-  __syncthreads();
-  const int t = t0 + threadIdx.x;
-  if (t < n)
-    for (int dd = threadIdx.y; dd < hd; dd += 8)
-      vt_cache[(static_cast<long long>(g) * hd + dd) * ldk + pos0 + t] =
-          store_from_f32<TA>(tile[dd][threadIdx.x]);
+  return acc;
 }
 
+template <typename TA>
+DG_DEV void store4(TA* dst, float4 v);
+template <>
+DG_DEV void store4<float>(float* dst, float4 v) {
+  *reinterpret_cast<float4*>(dst) = v;
+}
+template <>
+DG_DEV void store4<__nv_bfloat16>(__nv_bfloat16* dst, float4 v) {
+  const __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y);
+  const __nv_bfloat162 b = __floats2bfloat162_rn(v.z, v.w);
+  uint2 u;
+  u.x = *reinterpret_cast<const uint32_t*>(&a);
+  u.y = *reinterpret_cast<const uint32_t*>(&b);
+  *reinterpret_cast<uint2*>(dst) = u;
+}
+
+// QKV finalize: sum the split-K partials of 16 tokens for one head and store them.
+//  q / k heads: rotate-half RoPE at absolute positions pos0 + t (cos/sin table in fp32 computed
+//               in fp64), stored to Q [Hq, tq, hd] or to the K cache slots pos0 + t;
+//  v heads:     stored transposed into V^T [hd, cap] at columns pos0 + t.
+// grid (ceil(n / 16), Hq + 2 Hkv), 128 threads.  Phase 1 sums the [16, hd] block of every split
+// with independent float4 loads into shared memory; phase 2 rotates or transposes from there.
+// hd % 4 == 0, hd <= 128.
+constexpr int kQkvTok = 16;
+template <typename TA>
+__global__ void __launch_bounds__(128) qkv_finalize_kernel(
+    const float* __restrict__ part, int splits, long long split_stride, int ld, int hd,
+    int n_heads, int n_kv_heads, const float2* __restrict__ rope_tab, int n, int pos0,
+    TA* __restrict__ q, int tq, TA* __restrict__ k_cache, TA* __restrict__ vt_cache, int ldk,
+    const int* done) {
+  if (block_done(done)) return;
+  __shared__ float blk[kQkvTok][128 + 4];
+  const int t0 = blockIdx.x * kQkvTok, h = blockIdx.y, tid = threadIdx.x;
+  const int nt = min(kQkvTok, n - t0);
+  const int hv = hd >> 2;  // float4 per token row
+  for (int e = tid; e < kQkvTok * hv; e += 128) {
+    const int tt = e / hv, c4 = e % hv;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (tt < nt)
+      acc = sum_splits4(part, splits, split_stride,
+                        static_cast<long long>(t0 + tt) * ld + h * hd + 4 * c4);
+    *reinterpret_cast<float4*>(&blk[tt][4 * c4]) = acc;
+  }
+  __syncthreads();
+  const int half = hd >> 1;
+  if (h < n_heads + n_kv_heads) {
+    for (int e = tid; e < nt * half; e += 128) {
+      const int tt = e / half, i = e % half;
+      const int t = t0 + tt;
+      const float a = blk[tt][i], b = blk[tt][i + half];
+      const float2 cs = rope_tab[static_cast<long long>(pos0 + t) * half + i];  // (cos, sin)
+      TA* dst = (h < n_heads) ? q + (static_cast<long long>(h) * tq + t) * hd
+                              : k_cache + (static_cast<long long>(h - n_heads) * ldk + pos0 + t) * hd;
+      dst[i] = store_from_f32<TA>(a * cs.x - b * cs.y);
+      dst[i + half] = store_from_f32<TA>(b * cs.x + a * cs.y);
+    }
+  } else {
+    const int g = h - n_heads - n_kv_heads;
+    for (int dd = tid; dd < hd; dd += 128) {
+      TA* dst = vt_cache + (static_cast<long long>(g) * hd + dd) * ldk + pos0 + t0;
+      for (int tt = 0; tt < nt; ++tt) dst[tt] = store_from_f32<TA>(blk[tt][dd]);
+    }
+  }
+}
+
+// x += sum of split partials (0 splits: x unchanged); xn = rmsnorm(x) * w.  One CTA per token,
+// float4 columns, d % 4 == 0 and d <= 4 * 256 * kNormVec.
+constexpr int kNormVec = 4;
 template <typename TA>
 __global__ void __launch_bounds__(256) residual_norm_kernel(float* __restrict__ x,
                                                             const float* __restrict__ part,
@@ -117,22 +147,41 @@ __global__ void __launch_bounds__(256) residual_norm_kernel(float* __restrict__ 
   if (block_done(done)) return;
   __shared__ float sm[8];
   const int t = blockIdx.x;
+  const int nv = d >> 2;
   float* xr = x + static_cast<long long>(t) * d;
+  float4 v[kNormVec];
   float ss = 0.f;
-  for (int i = threadIdx.x; i < d; i += 256) {
-    float v = xr[i];
-    float acc = 0.f;
-    for (int s = 0; s < splits; ++s) acc += part[s * split_stride + static_cast<long long>(t) * d + i];
-    v += acc;
-    xr[i] = v;
-    ss += v * v;
+#pragma unroll
+  for (int j = 0; j < kNormVec; ++j) {
+    const int i = threadIdx.x + j * 256;
+    if (i < nv) {
+      float4 a = reinterpret_cast<const float4*>(xr)[i];
+      const float4 p = sum_splits4(part, splits, split_stride, static_cast<long long>(t) * d + 4 * i);
+      a.x += p.x;
+      a.y += p.y;
+      a.z += p.z;
+      a.w += p.w;
+      v[j] = a;
+      if (splits > 0) reinterpret_cast<float4*>(xr)[i] = a;
+      ss += a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w;
+    }
   }
   const float inv = rsqrtf(block_sum_256(ss, sm) / d + eps);
-  for (int i = threadIdx.x; i < d; i += 256)
-    xn[static_cast<long long>(t) * d + i] = store_from_f32<TA>(xr[i] * inv * w[i]);
+#pragma unroll
+  for (int j = 0; j < kNormVec; ++j) {
+    const int i = threadIdx.x + j * 256;
+    if (i < nv) {
+      const float4 g = reinterpret_cast<const float4*>(w)[i];
+      store4<TA>(xn + static_cast<long long>(t) * d + 4 * i,
+                 make_float4(v[j].x * inv * g.x, v[j].y * inv * g.y, v[j].z * inv * g.z,
+                             v[j].w * inv * g.w));
+    }
+  }
 }
 
-// one warp per token; E <= 256, k <= 8.
+// One warp per token; E <= 256 and E % 4 == 0, k <= 8.  Lane l holds experts 4l..4l+3 and
+// 128+4l..128+4l+3.  Top-k by repeated warp argmax (largest logit, lowest index on ties); the
+// weights are the softmax of the selected logits.
 __global__ void router_topk_kernel(const float* __restrict__ part, int splits,
                                    long long split_stride, int n_tokens, int n_experts, int top_k,
                                    float* __restrict__ logits_out, int32_t* __restrict__ ids,
@@ -143,16 +192,18 @@ __global__ void router_topk_kernel(const float* __restrict__ part, int splits,
   const int lane = lane_id();
   float v[8];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const int e = lane + 32 * j;
-    float acc = -INFINITY;
-    if (e < n_experts) {
-      acc = 0.f;
-      for (int s = 0; s < splits; ++s)
-        acc += part[s * split_stride + static_cast<long long>(t) * n_experts + e];
-      if (logits_out) logits_out[static_cast<long long>(t) * n_experts + e] = acc;
+  for (int h = 0; h < 2; ++h) {
+    const int e0 = 128 * h + 4 * lane;
+    float4 a = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+    if (e0 < n_experts) {
+      a = sum_splits4(part, splits, split_stride, static_cast<long long>(t) * n_experts + e0);
+      if (logits_out)
+        *reinterpret_cast<float4*>(logits_out + static_cast<long long>(t) * n_experts + e0) = a;
     }
-    v[j] = acc;
+    v[4 * h] = a.x;
+    v[4 * h + 1] = a.y;
+    v[4 * h + 2] = a.z;
+    v[4 * h + 3] = a.w;
   }
   float sel_v[8];
   int sel_i[8];
@@ -161,7 +212,7 @@ __global__ void router_topk_kernel(const float* __restrict__ part, int splits,
     int bi = 0x7fffffff;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      const int e = lane + 32 * j;
+      const int e = 128 * (j >> 2) + 4 * lane + (j & 3);
       if (e < n_experts && (v[j] > bv || (v[j] == bv && e < bi))) {
         bv = v[j];
         bi = e;
@@ -180,7 +231,7 @@ __global__ void router_topk_kernel(const float* __restrict__ part, int splits,
     sel_i[kk] = bi;
 #pragma unroll
     for (int j = 0; j < 8; ++j)
-      if (lane + 32 * j == bi) v[j] = -INFINITY;
+      if (128 * (j >> 2) + 4 * lane + (j & 3) == bi) v[j] = -INFINITY;
   }
   if (lane == 0) {
     float den = 0.f;
@@ -201,57 +252,101 @@ struct RouteArgs {
   int4* items_d;     // grouped items for down
   int32_t* counts;   // [2]: item counts (gate/up, down)
   int m_tiles_gu, m_tiles_d, n_chunk;
+  // shared expert folded in as group n_experts: n_tokens in chunks of n_chunk, listed first
+  int n_tokens, shared_m_tiles_gu, shared_m_tiles_d;  // 0 tiles: no shared expert
   const int* done;
 };
 
-// Single CTA of 1024 threads: counts, exclusive scan, stable (slot-order) placement via
-// warp match + per-warp counts, and the grouped item lists.
+// Exclusive scan of up to 256 values by warp 0 (8 per lane); returns the total to all lanes.
+DG_DEV int warp_exclusive_scan_256(const int* in, int* out, int n) {
+  const int lane = lane_id();
+  int v[8], s = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int e = lane * 8 + j;
+    v[j] = e < n ? in[e] : 0;
+    s += v[j];
+  }
+  int incl = s;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  int run = incl - s;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int e = lane * 8 + j;
+    if (e < n) out[e] = run;
+    run += v[j];
+  }
+  return __shfl_sync(0xffffffffu, incl, 31);
+}
+
+// Single CTA of 1024 threads: per-expert counts, exclusive scans (warp 0), the grouped GEMM item
+// lists, and the stable placement (slot order inside each expert) via warp match + per-warp
+// counts.  Items are (expert, 128-row tile, first permuted row, tokens <= n_chunk).
 __global__ void __launch_bounds__(1024) moe_route_kernel(RouteArgs a) {
   if (block_done(a.done)) return;
   __shared__ int cnt[32][257];  // per-warp counts in the current round, per expert
-  __shared__ int off_s[257];
-  __shared__ int base_s[256];
+  __shared__ int count_s[256], off_s[257], chunk_s[256], cbase_s[256], base_s[256];
   const int tid = threadIdx.x, warp = tid >> 5, lane = lane_id();
   const int E = a.n_experts;
-  // counts and offsets
-  for (int e = tid; e < E; e += 1024) base_s[e] = 0;
+  for (int e = tid; e < E; e += 1024) count_s[e] = 0;
   __syncthreads();
-  for (int s = tid; s < a.n_slots; s += 1024) atomicAdd(&base_s[a.ids[s]], 1);
+  for (int s = tid; s < a.n_slots; s += 1024) atomicAdd(&count_s[a.ids[s]], 1);
   __syncthreads();
-  if (tid == 0) {
-    int acc = 0;
-    int n_gu = 0, n_d = 0;
-    for (int e = 0; e < E; ++e) {
-      off_s[e] = acc;
-      const int c = base_s[e];
-      const int chunks = (c + a.n_chunk - 1) / a.n_chunk;
-      // items are written below by one thread per expert; here only the totals
-      n_gu += chunks * a.m_tiles_gu;
-      n_d += chunks * a.m_tiles_d;
-      acc += c;
+  for (int e = tid; e < E; e += 1024) chunk_s[e] = (count_s[e] + a.n_chunk - 1) / a.n_chunk;
+  __syncthreads();
+  const int sh_chunks = (a.shared_m_tiles_gu > 0) ? (a.n_tokens + a.n_chunk - 1) / a.n_chunk : 0;
+  const int sh_gu = sh_chunks * a.shared_m_tiles_gu, sh_d = sh_chunks * a.shared_m_tiles_d;
+  if (warp == 0) {
+    const int total = warp_exclusive_scan_256(count_s, off_s, E);
+    const int chunks = warp_exclusive_scan_256(chunk_s, cbase_s, E);
+    if (lane == 0) {
+      off_s[E] = total;
+      a.counts[0] = sh_gu + chunks * a.m_tiles_gu;
+      a.counts[1] = sh_d + chunks * a.m_tiles_d;
     }
-    off_s[E] = acc;
-    a.counts[0] = n_gu;
-    a.counts[1] = n_d;
   }
   __syncthreads();
+  // shared-expert items first; the token chunks of one weight tile are adjacent so the tile is
+  // re-read from L2
+  for (int w = tid; w < sh_gu; w += 1024) {
+    const int m = w / sh_chunks, ch = w % sh_chunks;
+    a.items_gu[w] = make_int4(E, m, ch * a.n_chunk, min(a.n_chunk, a.n_tokens - ch * a.n_chunk));
+  }
+  for (int w = tid; w < sh_d; w += 1024) {
+    const int m = w / sh_chunks, ch = w % sh_chunks;
+    a.items_d[w] = make_int4(E, m, ch * a.n_chunk, min(a.n_chunk, a.n_tokens - ch * a.n_chunk));
+  }
   for (int e = tid; e <= E; e += 1024) a.offsets[e] = off_s[e];
-  // grouped items: thread e writes its expert's items (expert order, then m tile, then chunk)
-  for (int e = tid; e < E; e += 1024) {
-    const int c = base_s[e];
-    const int chunks = (c + a.n_chunk - 1) / a.n_chunk;
-    int before = 0;  // chunks of experts < e
-    for (int f = 0; f < e; ++f) before += (base_s[f] + a.n_chunk - 1) / a.n_chunk;
-    for (int ch = 0; ch < chunks; ++ch) {
-      const int tok0 = off_s[e] + ch * a.n_chunk;
-      const int n = min(a.n_chunk, c - ch * a.n_chunk);
-      for (int m = 0; m < a.m_tiles_gu; ++m)
-        a.items_gu[(before + ch) * a.m_tiles_gu + m] = make_int4(e, m, tok0, n);
-      for (int m = 0; m < a.m_tiles_d; ++m)
-        a.items_d[(before + ch) * a.m_tiles_d + m] = make_int4(e, m, tok0, n);
+  // items: one (chunk, m tile) pair per thread
+  const int total_chunks = cbase_s[E - 1] + chunk_s[E - 1];
+  for (int w = tid; w < total_chunks * a.m_tiles_gu; w += 1024) {
+    const int ch = w / a.m_tiles_gu, m = w % a.m_tiles_gu;
+    int lo = 0, hi = E - 1;  // expert owning chunk ch: largest e with cbase_s[e] <= ch, chunk_s[e] > 0
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (cbase_s[mid] <= ch) lo = mid; else hi = mid - 1;
     }
+    while (chunk_s[lo] == 0) --lo;
+    const int local = ch - cbase_s[lo];
+    a.items_gu[sh_gu + w] = make_int4(lo, m, off_s[lo] + local * a.n_chunk,
+                                      min(a.n_chunk, count_s[lo] - local * a.n_chunk));
   }
-  __syncthreads();
+  for (int w = tid; w < total_chunks * a.m_tiles_d; w += 1024) {
+    const int ch = w / a.m_tiles_d, m = w % a.m_tiles_d;
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (cbase_s[mid] <= ch) lo = mid; else hi = mid - 1;
+    }
+    while (chunk_s[lo] == 0) --lo;
+    const int local = ch - cbase_s[lo];
+    a.items_d[sh_d + w] = make_int4(lo, m, off_s[lo] + local * a.n_chunk,
+                                    min(a.n_chunk, count_s[lo] - local * a.n_chunk));
+  }
   // stable placement, 1024 slots per round
   for (int e = tid; e < E; e += 1024) base_s[e] = off_s[e];
   for (int r0 = 0; r0 < a.n_slots; r0 += 1024) {
@@ -279,18 +374,23 @@ __global__ void __launch_bounds__(1024) moe_route_kernel(RouteArgs a) {
   }
 }
 
-// x_perm[p] = xn[perm[p] / k]; one CTA per permuted row, 16-byte copies.
-__global__ void gather_rows_kernel(const __nv_bfloat16* __restrict__ xn,
-                                   const int32_t* __restrict__ perm, int top_k, int d,
-                                   __nv_bfloat16* __restrict__ x_perm, const int* done) {
+// x_perm[p] = xn[perm[p] / k]; 64 threads per permuted row, 4 rows per CTA, 16-byte copies.
+__global__ void __launch_bounds__(256) gather_rows_kernel(const __nv_bfloat16* __restrict__ xn,
+                                                          const int32_t* __restrict__ perm,
+                                                          int top_k, int d, int n_rows,
+                                                          __nv_bfloat16* __restrict__ x_perm,
+                                                          const int* done) {
   if (block_done(done)) return;
-  const int p = blockIdx.x;
+  const int p = blockIdx.x * 4 + (threadIdx.x >> 6);
+  if (p >= n_rows) return;
   const int t = perm[p] / top_k;
   const uint4* src = reinterpret_cast<const uint4*>(xn + static_cast<long long>(t) * d);
   uint4* dst = reinterpret_cast<uint4*>(x_perm + static_cast<long long>(p) * d);
-  for (int i = threadIdx.x; i < d / 8; i += blockDim.x) dst[i] = src[i];
+  for (int i = threadIdx.x & 63; i < d / 8; i += 64) dst[i] = src[i];
 }
 
+// x += sum over slots s = 0..k-1 (in order) of y_slot[t*k + s] + y_shared[t]; then, when w is
+// given, xn = rmsnorm(x) * w for the next layer (or the final norm).  One CTA per token.
 template <typename TA>
 __global__ void __launch_bounds__(256) moe_combine_norm_kernel(
     float* __restrict__ x, const float* __restrict__ y_slot, int top_k,
@@ -299,20 +399,58 @@ __global__ void __launch_bounds__(256) moe_combine_norm_kernel(
   if (block_done(done)) return;
   __shared__ float sm[8];
   const int t = blockIdx.x;
+  const int nv = d >> 2;
   float* xr = x + static_cast<long long>(t) * d;
+  float4 v[kNormVec];
   float ss = 0.f;
-  for (int i = threadIdx.x; i < d; i += 256) {
-    float y = 0.f;
-    for (int s = 0; s < top_k; ++s) y += y_slot[(static_cast<long long>(t) * top_k + s) * d + i];
-    if (y_shared) y += y_shared[static_cast<long long>(t) * d + i];
-    const float v = xr[i] + y;
-    xr[i] = v;
-    ss += v * v;
+#pragma unroll
+  for (int j = 0; j < kNormVec; ++j) {
+    const int i = threadIdx.x + j * 256;
+    if (i < nv) {
+      float4 y[8];
+#pragma unroll
+      for (int s = 0; s < 8; ++s)
+        if (s < top_k)
+          y[s] = reinterpret_cast<const float4*>(
+              y_slot + (static_cast<long long>(t) * top_k + s) * d)[i];
+      float4 a = reinterpret_cast<const float4*>(xr)[i];
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int s = 0; s < 8; ++s)
+        if (s < top_k) {
+          acc.x += y[s].x;
+          acc.y += y[s].y;
+          acc.z += y[s].z;
+          acc.w += y[s].w;
+        }
+      if (y_shared) {
+        const float4 b = reinterpret_cast<const float4*>(y_shared + static_cast<long long>(t) * d)[i];
+        acc.x += b.x;
+        acc.y += b.y;
+        acc.z += b.z;
+        acc.w += b.w;
+      }
+      a.x += acc.x;
+      a.y += acc.y;
+      a.z += acc.z;
+      a.w += acc.w;
+      v[j] = a;
+      reinterpret_cast<float4*>(xr)[i] = a;
+      ss += a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w;
+    }
   }
   if (w == nullptr) return;  // standalone MoE: no following norm
   const float inv = rsqrtf(block_sum_256(ss, sm) / d + eps);
-  for (int i = threadIdx.x; i < d; i += 256)
-    xn[static_cast<long long>(t) * d + i] = store_from_f32<TA>(xr[i] * inv * w[i]);
+#pragma unroll
+  for (int j = 0; j < kNormVec; ++j) {
+    const int i = threadIdx.x + j * 256;
+    if (i < nv) {
+      const float4 g = reinterpret_cast<const float4*>(w)[i];
+      store4<TA>(xn + static_cast<long long>(t) * d + 4 * i,
+                 make_float4(v[j].x * inv * g.x, v[j].y * inv * g.y, v[j].z * inv * g.z,
+                             v[j].w * inv * g.w));
+    }
+  }
 }
 
 // RoPE table: (cos, sin) of pos * theta^(-2i/hd) for pos < n_pos, i < hd/2, computed in fp64.

@@ -243,8 +243,17 @@ enum {
   DG_KERNEL_QKV = 4,            /* QKV projection GEMM */
   DG_KERNEL_O_PROJ = 5,         /* attention output projection GEMM */
   DG_KERNEL_SAMPLER = 6,        /* sampler merge + stop test */
-  DG_KERNEL_SHARED_EXPERT = 7,  /* shared expert gate/up and down GEMMs */
-  DG_KERNEL_KINDS = 8
+  DG_KERNEL_SHARED_EXPERT = 7,  /* reserved: the shared expert runs inside kinds 0 and 1 */
+  DG_KERNEL_ROUTER = 8,         /* router logits GEMM */
+  DG_KERNEL_QKV_FINALIZE = 9,   /* RoPE + K/V cache store */
+  DG_KERNEL_ATTN_COMBINE = 10,  /* split-KV merge */
+  DG_KERNEL_RESIDUAL_NORM = 11, /* residual add + RMSNorm */
+  DG_KERNEL_ROUTER_TOPK = 12,   /* top-k selection */
+  DG_KERNEL_ROUTE = 13,         /* expert permutation + item lists */
+  DG_KERNEL_GATHER = 14,        /* permuted token rows */
+  DG_KERNEL_COMBINE_NORM = 15,  /* weighted expert sum + RMSNorm */
+  DG_KERNEL_EMBED = 16,         /* embedding gather + RMSNorm */
+  DG_KERNEL_KINDS = 17
 };
 
 /* Number of kernels this library has launched in the calling process (all entry points). */
