@@ -71,6 +71,8 @@ _PROTOS = {
     "dg_debug_logits": (C.c_int, [_P, _P, _P]),
     "dg_debug_layer": (C.c_int, [_P, _I, _P, _P, _I, _I, _P]),
     "dg_debug_hidden": (C.c_int, [_P, C.POINTER(_P)]),
+    "dg_debug_layer_part": (C.c_int, [_P, _I, _I, _P, _P, _I, _I, _P]),
+    "dg_debug_tensors": (C.c_int, [_P, C.POINTER(_P), C.POINTER(_P), C.POINTER(_P)]),
     "dg_debug_routing": (C.c_int, [_P, C.POINTER(_P), C.POINTER(_P), C.POINTER(_P)]),
     "dg_launch_count": (C.c_uint64, []),
     "dg_profile_kernel": (C.c_int, [_I, _I]),

@@ -162,6 +162,28 @@ class DiffusionModel:
                 self._view(ps[1].value, n * k, torch.float32).view(n, k),
                 self._view(ps[2].value, n * e, torch.float32).view(n, e))
 
+    def debug_tensors(self, n=None):
+        """(q, o, xn) views of the most recent layer's intermediates."""
+        n = self.cfg.canvas if n is None else n
+        c = self.cfg
+        dt = torch.float32 if c.dtype == L.DTYPE_FP32 else torch.bfloat16
+        tq = c.canvas if c.dtype == L.DTYPE_FP32 else 256
+        ps = [C.c_void_p() for _ in range(3)]
+        check(lib().dg_debug_tensors(self.handle, *[C.byref(x) for x in ps]), "dg_debug_tensors")
+        q = self._view(ps[0].value, c.n_heads * tq * c.head_dim, dt).view(c.n_heads, tq, c.head_dim)
+        o = self._view(ps[1].value, n * c.n_heads * c.head_dim, dt).view(n, c.n_heads * c.head_dim)
+        xn = self._view(ps[2].value, n * c.d_model, dt).view(n, c.d_model)
+        return q, o, xn
+
+    def debug_layer_part(self, layer, part, x_in, causal, stream=None):
+        """Half a layer: part 0 attention sub-block, part 1 MoE sub-block (x_out = x_in + ...)."""
+        _need_cuda(x_in, "x_in", torch.float32)
+        out = torch.empty_like(x_in)
+        check(lib().dg_debug_layer_part(self.handle, layer, part, _ptr(x_in), _ptr(out),
+                                        x_in.shape[0], int(bool(causal)), _stream(stream)),
+              "dg_debug_layer_part")
+        return out
+
     def debug_layer(self, layer, x_in, causal, stream=None):
         _need_cuda(x_in, "x_in", torch.float32)
         out = torch.empty_like(x_in)

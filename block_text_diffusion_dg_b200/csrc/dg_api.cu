@@ -364,8 +364,10 @@ Plan plan(const dg_config& c, int sms) {
 // ---- the layer pipeline -----------------------------------------------------------------
 // Runs every layer over n tokens at positions pos0.. (canvas buffer or caller ids), writes their
 // K/V into cache slots pos0..pos0+n-1 and leaves the final-normed hidden state in xn.
+// parts: bit 0 = attention sub-block (QKV .. O projection, residual, ffn norm), bit 1 = MoE
+// sub-block (router .. weighted combine, residual, next norm).
 int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_norm,
-              const int* done, cudaStream_t st);
+              const int* done, cudaStream_t st, int parts = 3);
 
 int run_forward(dg_ctx* c, const int32_t* ids, int n, int pos0, int causal, const int* done,
                 cudaStream_t st) {
@@ -406,7 +408,7 @@ int layer_tail_common(dg_ctx* c, int l, int n, int pos0, const int* done, cudaSt
 }
 
 int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_norm,
-              const int* done, cudaStream_t st) {
+              const int* done, cudaStream_t st, int parts) {
   const dg_config& g = c->cfg;
   const dg_layer_weights& w = c->layers[l];
   const int d = g.d_model, hd = g.head_dim, k = g.top_k, E = g.n_experts;
@@ -415,6 +417,7 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
   if (!c->bf16) {
     // ---------------- all-fp32 path ----------------
     const float* xn = static_cast<const float*>(c->xn);
+    if (parts & 1) {
     gemm_f32_nt_kernel<<<dim3(cdiv(c->qkv_rows, 64), cdiv(n, 64)), 256, 0, st>>>(
         xn, static_cast<const float*>(w.wqkv), n, c->qkv_rows, d, c->part, c->qkv_rows, done);
     DG_LAUNCHED();
@@ -437,6 +440,8 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     residual_norm_kernel<float><<<n, 256, 0, st>>>(c->x, c->part, 1, 0, d, w.ffn_norm, g.eps,
                                                    static_cast<float*>(c->xn), done);
     DG_LAUNCHED();
+    }
+    if (!(parts & 2)) return DG_OK;
     gemm_f32_nt_kernel<<<dim3(cdiv(E, 64), cdiv(n, 64)), 256, 0, st>>>(
         xn, static_cast<const float*>(w.wr), n, E, d, c->part, E, done);
     DG_LAUNCHED();
@@ -465,6 +470,7 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     return DG_OK;
   }
   // ---------------- bf16 tcgen05 path ----------------
+  if (parts & 1) {
   // QKV projection, split-K partials [split][token][row]
   {
     GemmParams p = dense_params(c->qkv_rows, n, d, c->split_qkv, c->err, done);
@@ -534,6 +540,8 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     DG_LAUNCHED();
     prof_after(DG_KERNEL_RESIDUAL_NORM, st);
   }
+  }
+  if (!(parts & 2)) return DG_OK;
   // router + top-k
   {
     GemmParams p = dense_params(E, n, d, c->split_r, c->err, done);
@@ -985,6 +993,41 @@ int dg_debug_routing(const dg_ctx* ctx, int32_t** d_ids, float** d_weights,
   return DG_OK;
 }
 
+int dg_debug_layer_part(dg_ctx* ctx, int32_t layer, int32_t part, const float* d_x_in,
+                        float* d_x_out, int32_t n, int32_t causal, void* stream) {
+  DG_TRY(check_ctx(ctx));
+  const dg_config& g = ctx->cfg;
+  if (layer < 0 || layer >= g.n_layers) return fail(DG_ERR_INVALID_ARG, "bad layer %d", layer);
+  if (part != 0 && part != 1) return fail(DG_ERR_INVALID_ARG, "part must be 0 or 1");
+  if (!d_x_in || !d_x_out || n < 1 || n > g.canvas)
+    return fail(DG_ERR_INVALID_ARG, "need x_in, x_out and 1 <= n <= canvas");
+  if (ctx->kv_len + n > g.kv_capacity) return fail(DG_ERR_CAPACITY, "cache full");
+  cudaStream_t st = S(stream);
+  DG_CUDA(cudaMemcpyAsync(ctx->x, d_x_in, static_cast<size_t>(n) * g.d_model * 4,
+                          cudaMemcpyDeviceToDevice, st));
+  const float* w = part == 0 ? ctx->layers[layer].attn_norm : ctx->layers[layer].ffn_norm;
+  if (ctx->bf16)
+    residual_norm_kernel<__nv_bfloat16><<<n, 256, 0, st>>>(
+        ctx->x, ctx->part, 0, 0, g.d_model, w, g.eps, static_cast<__nv_bfloat16*>(ctx->xn), nullptr);
+  else
+    residual_norm_kernel<float><<<n, 256, 0, st>>>(ctx->x, ctx->part, 0, 0, g.d_model, w, g.eps,
+                                                   static_cast<float*>(ctx->xn), nullptr);
+  DG_LAUNCHED();
+  const float* nn = (layer + 1 < g.n_layers) ? ctx->layers[layer + 1].attn_norm : ctx->final_norm;
+  DG_TRY(run_layer(ctx, layer, n, ctx->kv_len, causal, nn, nullptr, st, part == 0 ? 1 : 2));
+  DG_CUDA(cudaMemcpyAsync(d_x_out, ctx->x, static_cast<size_t>(n) * g.d_model * 4,
+                          cudaMemcpyDeviceToDevice, st));
+  return DG_OK;
+}
+
+int dg_debug_tensors(const dg_ctx* ctx, void** d_q, void** d_o, void** d_xn) {
+  DG_TRY(check_ctx(ctx));
+  if (d_q) *d_q = ctx->q;
+  if (d_o) *d_o = ctx->o;
+  if (d_xn) *d_xn = ctx->xn;
+  return DG_OK;
+}
+
 int dg_debug_hidden(const dg_ctx* ctx, float** d_x) {
   DG_TRY(check_ctx(ctx));
   if (!d_x) return fail(DG_ERR_INVALID_ARG, "null output");
@@ -1025,12 +1068,13 @@ int dg_sampler_workspace_bytes(int32_t rows, int32_t vocab, size_t* bytes) {
   if (rows < 1 || rows > 1024 || vocab < 2 || vocab % 8 || !bytes)
     return fail(DG_ERR_INVALID_ARG, "need 1 <= rows <= 1024, vocab % 8 == 0");
   const size_t nchunk = cdiv(vocab, 4096);  // upper bound over both dtypes
-  *bytes = align256(rows * nchunk * sizeof(StatPartial)) + 3 * align256(rows * 8) + 256;
+  *bytes = align256(rows * nchunk * sizeof(StatPartial)) + 4 * align256(rows * 8) + 256;
   return DG_OK;
 }
 
 static void sampler_views(void* ws, int rows, int vocab, StatPartial** part, int32_t** prev,
-                          double** row_h, int32_t** locked, int32_t** ticket) {
+                          double** row_h, int32_t** locked, int32_t** ticket,
+                          int32_t** row_ticket) {
   uint8_t* b = static_cast<uint8_t*>(ws);
   const size_t nchunk = cdiv(vocab, 4096);
   *part = reinterpret_cast<StatPartial*>(b);
@@ -1040,6 +1084,8 @@ static void sampler_views(void* ws, int rows, int vocab, StatPartial** part, int
   *row_h = reinterpret_cast<double*>(b);
   b += align256(rows * 8);
   *locked = reinterpret_cast<int32_t*>(b);
+  b += align256(rows * 8);
+  *row_ticket = reinterpret_cast<int32_t*>(b);
   b += align256(rows * 8);
   *ticket = reinterpret_cast<int32_t*>(b);
 }
@@ -1069,20 +1115,12 @@ int dg_sampler_step(const void* d_logits, int32_t dtype, int32_t rows, int32_t v
   if (dtype != DG_DTYPE_BF16 && dtype != DG_DTYPE_FP32)
     return fail(DG_ERR_INVALID_ARG, "dtype must be bf16 or fp32");
   StatPartial* part;
-  int32_t *prev, *locked, *ticket;
+  int32_t *prev, *locked, *ticket, *row_ticket;
   double* row_h;
-  sampler_views(d_workspace, rows, vocab, &part, &prev, &row_h, &locked, &ticket);
+  sampler_views(d_workspace, rows, vocab, &part, &prev, &row_h, &locked, &ticket, &row_ticket);
   cudaStream_t st = S(stream);
   const int chunk = sampler_chunk(dtype);
   const int nchunk = cdiv(vocab, chunk);
-  const int* done = d_state + kStDone;
-  if (dtype == DG_DTYPE_BF16)
-    logits_stats_kernel<__nv_bfloat16, 32><<<dim3(nchunk, rows), 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(d_logits), vocab, chunk, part, done);
-  else
-    logits_stats_kernel<float, 16><<<dim3(nchunk, rows), 256, 0, st>>>(
-        static_cast<const float*>(d_logits), vocab, chunk, part, done);
-  DG_LAUNCHED();
   SamplerArgs a{};
   a.partials = part;
   a.nsplit = nchunk;
@@ -1104,8 +1142,15 @@ int dg_sampler_step(const void* d_logits, int32_t dtype, int32_t rows, int32_t v
   a.locked = locked;
   a.state = d_state;
   a.ticket = ticket;
-  sampler_merge_kernel<<<rows, 256, 0, st>>>(a);
+  prof_before(DG_KERNEL_SAMPLER, st);
+  if (dtype == DG_DTYPE_BF16)
+    sampler_fused_kernel<__nv_bfloat16, 32><<<dim3(nchunk, rows), 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(d_logits), chunk, a, row_ticket);
+  else
+    sampler_fused_kernel<float, 16><<<dim3(nchunk, rows), 256, 0, st>>>(
+        static_cast<const float*>(d_logits), chunk, a, row_ticket);
   DG_LAUNCHED();
+  prof_after(DG_KERNEL_SAMPLER, st);
   return DG_OK;
 }
 

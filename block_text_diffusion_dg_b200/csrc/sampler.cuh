@@ -64,96 +64,119 @@ __global__ void canvas_init_kernel(int32_t* canvas, int32_t t, int32_t vocab, ui
   }
 }
 
-// Partial statistics of one row slice.  grid = (chunks, rows), 256 threads; each thread
-// holds up to kPerThread values in registers.  Partial index = row * chunks + chunk.
+// Statistics (m, S, U, argmax) of one row slice held in registers by a 256-thread CTA: pass 1
+// takes the maximum (only threads holding it then look for its lowest column), pass 2
+// accumulates e = 2^((x - m) log2 e), S += e, U += e (x - m).  Value i of a thread sits at column
+// c0 + ((i / kVec) * 256 + tid) * kVec + i % kVec; values past the row end are -inf (`full` = no
+// such padding in this slice, uniform over the CTA).
+template <int kPerThread, int kVec>
+DG_DEV StatPartial slice_stats(const float (&v)[kPerThread], int c0, bool full, float* sm_f,
+                               int* sm_i) {
+  const int warp = threadIdx.x >> 5;
+  float tm = v[0];
+#pragma unroll
+  for (int i = 1; i < kPerThread; ++i) tm = fmaxf(tm, v[i]);
+  float m = tm;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane_id() == 0) sm_f[warp] = m;
+  __syncthreads();
+  float bm = sm_f[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) bm = fmaxf(bm, sm_f[w]);
+  int a = 0x7fffffff;
+  if (tm == bm) {  // rare: this thread holds the slice maximum; values are in column order
+#pragma unroll
+    for (int i = kPerThread - 1; i >= 0; --i)
+      if (v[i] == bm) a = c0 + ((i / kVec) * 256 + static_cast<int>(threadIdx.x)) * kVec + i % kVec;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) a = min(a, __shfl_xor_sync(0xffffffffu, a, o));
+  constexpr float kLog2e = 1.4426950408889634f;
+  float s4[4] = {0.f, 0.f, 0.f, 0.f}, u4[4] = {0.f, 0.f, 0.f, 0.f};
+  if (full) {
+#pragma unroll
+    for (int i = 0; i < kPerThread; ++i) {
+      const float d = v[i] - bm;
+      const float e = fast_exp2(d * kLog2e);
+      s4[i & 3] += e;
+      u4[i & 3] = fmaf(e, d, u4[i & 3]);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < kPerThread; ++i) {
+      if (v[i] != -INFINITY) {
+        const float d = v[i] - bm;
+        const float e = fast_exp2(d * kLog2e);
+        s4[i & 3] += e;
+        u4[i & 3] = fmaf(e, d, u4[i & 3]);
+      }
+    }
+  }
+  float s = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+  float u = (u4[0] + u4[1]) + (u4[2] + u4[3]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    s += __shfl_xor_sync(0xffffffffu, s, o);
+    u += __shfl_xor_sync(0xffffffffu, u, o);
+  }
+  __syncthreads();  // sm_f is reused below
+  if (lane_id() == 0) {
+    sm_f[warp] = s;
+    sm_f[8 + warp] = u;
+    sm_i[warp] = a;
+  }
+  __syncthreads();
+  StatPartial r{bm, 0.f, 0.f, 0x7fffffff};
+  if (threadIdx.x == 0) {
+    for (int w = 0; w < 8; ++w) {
+      r.s += sm_f[w];
+      r.u += sm_f[8 + w];
+      r.a = min(r.a, sm_i[w]);
+    }
+  }
+  return r;  // valid in thread 0
+}
+
+// Load this CTA's slice of one row (layout as above); returns whether it has no padding.
+template <typename T, int kPerThread>
+DG_DEV bool load_slice(const T* base, int c0, int c1, float (&v)[kPerThread]) {
+  constexpr int kVec = 16 / sizeof(T);
+  constexpr int kLoads = kPerThread / kVec;
+  const bool full = c0 + kPerThread * 256 <= c1;
+#pragma unroll
+  for (int l = 0; l < kLoads; ++l) {
+    const int c = c0 + (l * 256 + threadIdx.x) * kVec;
+    if (full || c < c1) {
+      const uint4 raw = __ldcs(reinterpret_cast<const uint4*>(base + c));
+      const T* e = reinterpret_cast<const T*>(&raw);
+#pragma unroll
+      for (int j = 0; j < kVec; ++j) v[l * kVec + j] = load_as_f32<T>(e, j);
+    } else {
+#pragma unroll
+      for (int j = 0; j < kVec; ++j) v[l * kVec + j] = -INFINITY;
+    }
+  }
+  return full;
+}
+
+// Partial statistics of one row slice.  grid = (chunks, rows), 256 threads, chunk =
+// 256 * kPerThread columns.  Partial index = row * chunks + chunk.
 template <typename T, int kPerThread>
 __global__ void __launch_bounds__(256) logits_stats_kernel(const T* __restrict__ logits,
                                                            int32_t vocab, int32_t chunk,
                                                            StatPartial* __restrict__ out,
                                                            const int* done) {
   if (block_done(done)) return;
-  constexpr int kVec = 16 / sizeof(T);
-  constexpr int kLoads = kPerThread / kVec;
+  __shared__ float sm_f[16];
+  __shared__ int sm_i[8];
   const int row = blockIdx.y;
   const int c0 = blockIdx.x * chunk;
-  const int c1 = min(c0 + chunk, vocab);
-  const T* base = logits + static_cast<size_t>(row) * vocab;
   float v[kPerThread];
-  float m = -INFINITY;
-  int a = 0x7fffffff;
-#pragma unroll
-  for (int l = 0; l < kLoads; ++l) {
-    const int col = c0 + (l * blockDim.x + threadIdx.x) * kVec;
-    if (col < c1) {
-      const uint4 raw = __ldcs(reinterpret_cast<const uint4*>(base + col));
-      const T* e = reinterpret_cast<const T*>(&raw);
-#pragma unroll
-      for (int j = 0; j < kVec; ++j) {
-        const float x = load_as_f32<T>(e, j);
-        v[l * kVec + j] = x;
-        if (x > m) {
-          m = x;
-          a = col + j;
-        }
-      }
-    } else {
-#pragma unroll
-      for (int j = 0; j < kVec; ++j) v[l * kVec + j] = -INFINITY;
-    }
-  }
-  // block max with lowest index
-  __shared__ float sm_m[8];
-  __shared__ int sm_a[8];
-  __shared__ float sm_s[8], sm_u[8];
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const float om = __shfl_xor_sync(0xffffffffu, m, o);
-    const int oa = __shfl_xor_sync(0xffffffffu, a, o);
-    if (om > m || (om == m && oa < a)) {
-      m = om;
-      a = oa;
-    }
-  }
-  const int warp = threadIdx.x >> 5;
-  if (lane_id() == 0) {
-    sm_m[warp] = m;
-    sm_a[warp] = a;
-  }
-  __syncthreads();
-  float bm = sm_m[0];
-  int ba = sm_a[0];
-  for (int w = 1; w < 8; ++w) {
-    if (sm_m[w] > bm || (sm_m[w] == bm && sm_a[w] < ba)) {
-      bm = sm_m[w];
-      ba = sm_a[w];
-    }
-  }
-  float s = 0.f, u = 0.f;
-#pragma unroll
-  for (int i = 0; i < kPerThread; ++i) {
-    const float d = v[i] - bm;
-    const float e = __expf(d);  // exp(-inf) = 0 for padding
-    s += e;
-    u += (d > -INFINITY) ? e * d : 0.f;
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    s += __shfl_xor_sync(0xffffffffu, s, o);
-    u += __shfl_xor_sync(0xffffffffu, u, o);
-  }
-  if (lane_id() == 0) {
-    sm_s[warp] = s;
-    sm_u[warp] = u;
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float ts = 0.f, tu = 0.f;
-    for (int w = 0; w < 8; ++w) {
-      ts += sm_s[w];
-      tu += sm_u[w];
-    }
-    out[static_cast<size_t>(row) * gridDim.x + blockIdx.x] = StatPartial{bm, ts, tu, ba};
-  }
+  const bool full = load_slice<T, kPerThread>(logits + static_cast<size_t>(row) * vocab, c0,
+                                              min(c0 + chunk, vocab), v);
+  const StatPartial r = slice_stats<kPerThread, 16 / sizeof(T)>(v, c0, full, sm_f, sm_i);
+  if (threadIdx.x == 0) out[static_cast<size_t>(row) * gridDim.x + blockIdx.x] = r;
 }
 
 struct SamplerArgs {
@@ -179,11 +202,9 @@ struct SamplerArgs {
   int32_t* ticket;
 };
 
-// One CTA per row: merge the row's partials, decide lock / re-noise; the last CTA to finish
-// evaluates the stop rule for the whole canvas (no CTA ever waits on another).
-__global__ void __launch_bounds__(256) sampler_merge_kernel(SamplerArgs p) {
-  if (block_done(p.state + kStDone)) return;
-  const int row = blockIdx.x;
+// Merge one row's partials (block-wide, fp64), decide lock / re-noise and write the row's
+// outputs; returns (in thread 0) whether this CTA is the last row to finish the step.
+DG_DEV bool sampler_row(const SamplerArgs& p, int row) {
   StatD acc{0.0, 0.0, 0.0, 0x7fffffff};
   for (int i = threadIdx.x; i < p.nsplit; i += blockDim.x) {
     const StatPartial q = p.partials[static_cast<size_t>(row) * p.nsplit + i];
@@ -214,9 +235,12 @@ __global__ void __launch_bounds__(256) sampler_merge_kernel(SamplerArgs p) {
     is_last = (atomicAdd(p.ticket, 1) == p.rows - 1);
   }
   __syncthreads();
-  if (!is_last) return;
+  return is_last;
+}
+
+// The stop test over the whole canvas, run by the last row's CTA (after a fence).
+DG_DEV void sampler_stop_test(const SamplerArgs& p) {
   __threadfence();
-  // --- last CTA: stop test over the whole canvas -------------------------------------
   __shared__ int n_diff, n_locked;
   if (threadIdx.x == 0) {
     n_diff = 0;
@@ -253,6 +277,42 @@ __global__ void __launch_bounds__(256) sampler_merge_kernel(SamplerArgs p) {
   __syncthreads();
   for (int i = threadIdx.x; i < p.rows; i += blockDim.x)
     p.prev_argmax[i] = *reinterpret_cast<volatile int32_t*>(p.argmax + i);
+}
+
+// One CTA per row: merge the row's partials, decide lock / re-noise; the last CTA to finish
+// evaluates the stop rule for the whole canvas (no CTA ever waits on another).
+__global__ void __launch_bounds__(256) sampler_merge_kernel(SamplerArgs p) {
+  if (block_done(p.state + kStDone)) return;
+  if (sampler_row(p, blockIdx.x)) sampler_stop_test(p);
+}
+
+// Statistics, merge and stop test in one launch: grid = (chunks, rows).  Each CTA writes its
+// slice's partial; the last CTA of a row (per-row ticket) merges the row; the last row runs the
+// stop test.  row_ticket [rows] must start at zero and is left at zero.
+template <typename T, int kPerThread>
+__global__ void __launch_bounds__(256) sampler_fused_kernel(const T* __restrict__ logits,
+                                                            int32_t chunk, SamplerArgs p,
+                                                            int32_t* __restrict__ row_ticket) {
+  if (block_done(p.state + kStDone)) return;
+  __shared__ float sm_f[16];
+  __shared__ int sm_i[8];
+  __shared__ int last_chunk;
+  const int row = blockIdx.y;
+  const int c0 = blockIdx.x * chunk;
+  float v[kPerThread];
+  const bool full = load_slice<T, kPerThread>(logits + static_cast<size_t>(row) * p.vocab, c0,
+                                              min(c0 + chunk, p.vocab), v);
+  const StatPartial r = slice_stats<kPerThread, 16 / sizeof(T)>(v, c0, full, sm_f, sm_i);
+  if (threadIdx.x == 0) {
+    const_cast<StatPartial*>(p.partials)[static_cast<size_t>(row) * p.nsplit + blockIdx.x] = r;
+    __threadfence();
+    last_chunk = (atomicAdd(row_ticket + row, 1) == p.nsplit - 1);
+  }
+  __syncthreads();
+  if (!last_chunk) return;
+  __threadfence();
+  if (threadIdx.x == 0) row_ticket[row] = 0;
+  if (sampler_row(p, row)) sampler_stop_test(p);
 }
 
 }  // namespace dg

@@ -283,6 +283,15 @@ DG_API int dg_debug_layer(dg_ctx* ctx, int32_t layer, const float* d_x_in, float
  * (renormalised over the k experts), router logits fp32 [n, E] (device pointers into scratch). */
 DG_API int dg_debug_routing(const dg_ctx* ctx, int32_t** d_ids, float** d_weights,
                             float** d_router_logits);
+/* Half of a teacher-forced layer: part 0 = attention sub-block (x_out = x_in + O-projection of
+ * the attention over RMSNorm(x_in), K/V written to slots P..P+n-1), part 1 = MoE sub-block
+ * (x_out = x_in + MoE(RMSNorm(x_in)) with the shared expert).  Shapes as dg_debug_layer. */
+DG_API int dg_debug_layer_part(dg_ctx* ctx, int32_t layer, int32_t part, const float* d_x_in,
+                               float* d_x_out, int32_t n, int32_t causal, void* stream);
+/* Intermediate buffers of the most recent layer the context ran (device pointers into scratch):
+ * q [Hq, 256, hd] (bf16 model; [Hq, T, hd] fp32 model), attention output o [n, Hq*hd] and the
+ * normalised activations xn [n, d] in the storage type. */
+DG_API int dg_debug_tensors(const dg_ctx* ctx, void** d_q, void** d_o, void** d_xn);
 /* Final hidden state (fp32 [T, d]) of the last denoise step, for LM-head checks. */
 DG_API int dg_debug_hidden(const dg_ctx* ctx, float** d_x);
 

@@ -84,10 +84,10 @@ class KVCache:
         return 0 if not self.k else self.k[0].shape[1]
 
 
-def layer_forward(cfg, lw, x, positions, cache_k, cache_v, causal):
-    """One decoder layer over new tokens x [T, d] (fp32 values).
+def attention_block(cfg, lw, x, positions, cache_k, cache_v, causal):
+    """Attention half of a layer over new tokens x [T, d]: returns (x + O-projection, k, v, info).
 
-    cache_k/v: [Hkv, P, hd] committed history.  Returns (x_out, k_new, v_new, info).
+    cache_k/v: [Hkv, P, hd] committed history.
     """
     st = cfg.storage
     t = x.shape[0]
@@ -105,12 +105,28 @@ def layer_forward(cfg, lw, x, positions, cache_k, cache_v, causal):
     p = cache_k.shape[1]
     o = attention(q, keys, vals, 1.0 / np.sqrt(hd), causal_prefix=p if causal else None)
     o = round_storage(o.transpose(1, 0, 2).reshape(t, hq * hd), st)
-    x1 = round_f32(x + o @ np.asarray(lw["wo"], dtype=np.float64).T)
+    x1 = round_f32(np.asarray(x, dtype=np.float64) + o @ np.asarray(lw["wo"], dtype=np.float64).T)
+    return x1, k, v, dict(xn=xn, q=q, k=k, v=v, o=o, x_attn=x1)
+
+
+def moe_block(cfg, lw, x1):
+    """MoE half of a layer: returns (x1 + MoE(rmsnorm(x1)), info)."""
+    st = cfg.storage
     xn2 = round_storage(rmsnorm(x1, lw["ffn_norm"], cfg.eps), st)
     shared = (lw["ws_gu"], lw["ws_d"]) if lw.get("ws_gu") is not None else None
     y, minfo = moe_ffn(xn2, lw["wr"], lw["w_gu"], lw["w_d"], cfg.top_k, st, shared)
-    x2 = round_f32(x1 + y)
-    info = dict(xn=xn, q=q, k=k, v=v, o=o, x_attn=x1, xn2=xn2, moe=minfo)
+    x2 = round_f32(np.asarray(x1, dtype=np.float64) + y)
+    return x2, dict(xn2=xn2, moe=minfo)
+
+
+def layer_forward(cfg, lw, x, positions, cache_k, cache_v, causal):
+    """One decoder layer over new tokens x [T, d] (fp32 values).
+
+    cache_k/v: [Hkv, P, hd] committed history.  Returns (x_out, k_new, v_new, info).
+    """
+    x1, k, v, info = attention_block(cfg, lw, x, positions, cache_k, cache_v, causal)
+    x2, minfo = moe_block(cfg, lw, x1)
+    info.update(minfo)
     return x2, k, v, info
 
 

@@ -32,3 +32,36 @@ def weights_to_np(w):
     for lw in w["layers"]:
         out["layers"].append({k: cv(v) for k, v in lw.items()})
     return out
+
+
+def check_layer_parts(model, ocfg, lw, x_in, positions, cache_k, cache_v, layer, top_k,
+                      causal=False, rtol=2e-2):
+    """Teacher-forced parity of one layer, half by half, from identical inputs.
+
+    Attention half: x_in -> x_attn on both sides.  MoE half: the GPU's own x_attn goes into both
+    the GPU and the oracle, so the router sees (nearly) identical logits: routing must match as a
+    set of experts except where the oracle's k-th and (k+1)-th router logits lie within 1e-3
+    (then either set is valid), and every token with a matching set must match in value.
+    Returns (x_attn parity, x_out parity, fraction of tokens with matching routing).
+    """
+    import torch
+    from oracle import model as om
+    x1_ref, _, _, _ = om.attention_block(ocfg, lw, x_in, positions, cache_k, cache_v, causal)
+    x1_gpu = model.debug_layer_part(layer, 0, torch.from_numpy(np.asarray(x_in, np.float32)).cuda(),
+                                    causal)
+    x1 = np64(x1_gpu)
+    att = rel_close(x1, x1_ref, rtol)
+    x2_ref, info = om.moe_block(ocfg, lw, x1)
+    x2_gpu = model.debug_layer_part(layer, 1, x1_gpu.contiguous(), causal)
+    ids_g, _, _ = model.debug_routing(n=x1.shape[0])
+    torch.cuda.synchronize()
+    same = np.array_equal
+    g_set = np.sort(ids_g.cpu().numpy(), axis=1)
+    o_set = np.sort(info["moe"]["ids"], axis=1)
+    match = np.all(g_set == o_set, axis=1)
+    srt = -np.sort(-info["moe"]["router_logits"], axis=1)
+    gap = srt[:, top_k - 1] - srt[:, top_k] if top_k < srt.shape[1] else np.full(len(srt), np.inf)
+    assert np.all(gap[~match] < 1e-3), ("routing set differs away from a near-tie", layer,
+                                        gap[~match])
+    moe = rel_close(np64(x2_gpu)[match], x2_ref[match], rtol)
+    return att, moe, float(match.mean())
