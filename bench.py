@@ -206,7 +206,8 @@ def _time_op(fn, stream, reps=10, flush=None):
     total = 0.0
     for _ in range(reps):
         if flush is not None:
-            flush.fill_(1)
+            # read (not write) the flush buffer: L2 ends up holding clean lines only
+            torch.sum(flush)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         fn()
@@ -224,7 +225,7 @@ def run_ops(dev, stream, hbm, tf_burst):
     from dg_synth import attention_inputs, moe_inputs, sampler_logits
     # 1 GB flush (> L2): it also keeps the GPU busy while the host enqueues the timed call, so
     # the event interval holds device time only
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.float32, device=dev)
+    flush = torch.ones(256 * 1024 * 1024, dtype=torch.float32, device=dev)
     out = {}
     x = sampler_logits(256, 262144, seed=0).to(dev)
     s = dg.Sampler(256, 262144, device=dev)

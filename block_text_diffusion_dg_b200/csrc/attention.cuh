@@ -51,6 +51,7 @@ constexpr int kAttnThreads = 64 + 32 * 8;
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_vt, const AttnParams p) {
+  pdl_enter();
   if (block_done(p.done)) return;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -338,6 +339,7 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restri
                                                            int n_splits, int n_heads, int tq,
                                                            int n_queries, TA* __restrict__ o,
                                                            const int* done) {
+  pdl_enter();
   if (block_done(done)) return;
   const int pair = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (pair >= n_queries * n_heads) return;

@@ -142,6 +142,27 @@ int set_smem(K kernel, int bytes) {
   return DG_OK;
 }
 
+// Every kernel goes through cudaLaunchKernelEx with programmatic stream serialisation: the next
+// kernel in the stream may begin launching while this one drains; each kernel's first act is
+// griddepcontrol.wait, so it still sees all of its predecessor's writes.
+template <typename... KArgs, typename... Args>
+int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+               Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  if (e != cudaSuccess) return fail(DG_ERR_CUDA, "kernel launch failed: %s", cudaGetErrorString(e));
+  return DG_OK;
+}
+
 // ---- GEMM launch helpers -----------------------------------------------------------------
 constexpr int kDenseN = 256, kDenseStages = 4;
 constexpr int kGroupN = 64, kGroupStages = 8;
@@ -157,7 +178,7 @@ int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& 
     return fail(DG_ERR_INVALID_ARG, "alternate group without its tensor maps");
   DG_TRY(set_smem(k, smem));
   prof_before(kind, st);
-  k<<<grid, GemmCfg<MAXN, STAGES>::kThreads, smem, st>>>(ta, tb, ta2 ? *ta2 : ta, tb2 ? *tb2 : tb, p);
+  DG_TRY(launch_pdl(k, dim3(grid), dim3(GemmCfg<MAXN, STAGES>::kThreads), smem, st, ta, tb, ta2 ? *ta2 : ta, tb2 ? *tb2 : tb, p));
   DG_LAUNCHED();
   prof_after(kind, st);
   return DG_OK;
@@ -374,13 +395,13 @@ int run_forward(dg_ctx* c, const int32_t* ids, int n, int pos0, int causal, cons
   const dg_config& g = c->cfg;
   prof_before(DG_KERNEL_EMBED, st);
   if (c->bf16)
-    embed_norm_kernel<__nv_bfloat16, __nv_bfloat16><<<n, 256, 0, st>>>(
+    DG_TRY(launch_pdl(embed_norm_kernel<__nv_bfloat16, __nv_bfloat16>, dim3(n), dim3(256), 0, st, 
         ids, static_cast<const __nv_bfloat16*>(c->embed), g.d_model, c->layers[0].attn_norm, g.eps,
-        c->x, static_cast<__nv_bfloat16*>(c->xn), done);
+        c->x, static_cast<__nv_bfloat16*>(c->xn), done));
   else
-    embed_norm_kernel<float, float><<<n, 256, 0, st>>>(ids, static_cast<const float*>(c->embed),
+    DG_TRY(launch_pdl(embed_norm_kernel<float, float>, dim3(n), dim3(256), 0, st, ids, static_cast<const float*>(c->embed),
                                                        g.d_model, c->layers[0].attn_norm, g.eps,
-                                                       c->x, static_cast<float*>(c->xn), done);
+                                                       c->x, static_cast<float*>(c->xn), done));
   DG_LAUNCHED();
   prof_after(DG_KERNEL_EMBED, st);
   for (int l = 0; l < g.n_layers; ++l) {
@@ -399,9 +420,9 @@ int layer_tail_common(dg_ctx* c, int l, int n, int pos0, const int* done, cudaSt
   TA* kc = static_cast<TA*>(c->kc) + static_cast<size_t>(l) * g.n_kv_heads * kv_head_elems;
   TA* vtc = static_cast<TA*>(c->vtc) + static_cast<size_t>(l) * g.n_kv_heads * kv_head_elems;
   prof_before(DG_KERNEL_QKV_FINALIZE, st);
-  qkv_finalize_kernel<TA><<<dim3(cdiv(n, kQkvTok), g.n_heads + 2 * g.n_kv_heads), 128, 0, st>>>(
+  DG_TRY(launch_pdl(qkv_finalize_kernel<TA>, dim3(cdiv(n, kQkvTok), g.n_heads + 2 * g.n_kv_heads), dim3(128), 0, st, 
       c->part, splits_qkv, qkv_ss, c->qkv_rows, hd, g.n_heads, g.n_kv_heads, c->rope_tab, n, pos0,
-      static_cast<TA*>(c->q), c->tq, kc, vtc, g.kv_capacity, done);
+      static_cast<TA*>(c->q), c->tq, kc, vtc, g.kv_capacity, done));
   DG_LAUNCHED();
   prof_after(DG_KERNEL_QKV_FINALIZE, st);
   return DG_OK;
@@ -418,8 +439,8 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     // ---------------- all-fp32 path ----------------
     const float* xn = static_cast<const float*>(c->xn);
     if (parts & 1) {
-    gemm_f32_nt_kernel<<<dim3(cdiv(c->qkv_rows, 64), cdiv(n, 64)), 256, 0, st>>>(
-        xn, static_cast<const float*>(w.wqkv), n, c->qkv_rows, d, c->part, c->qkv_rows, done);
+    DG_TRY(launch_pdl(gemm_f32_nt_kernel, dim3(cdiv(c->qkv_rows, 64), cdiv(n, 64)), dim3(256), 0, st,
+        xn, static_cast<const float*>(w.wqkv), n, c->qkv_rows, d, c->part, c->qkv_rows, done));
     DG_LAUNCHED();
     DG_TRY(layer_tail_common<float>(c, l, n, pos0, done, st, 0, 1));
     const size_t kv_head_elems = static_cast<size_t>(g.kv_capacity) * hd;
@@ -428,44 +449,44 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     const int smem = (n_keys + hd) * 4;
     if (smem > 200 * 1024) return fail(DG_ERR_UNSUPPORTED, "fp32 attention: too many keys");
     DG_TRY(set_smem(attention_f32_kernel, smem));
-    attention_f32_kernel<<<dim3(n, g.n_heads), 128, smem, st>>>(
+    DG_TRY(launch_pdl(attention_f32_kernel, dim3(n, g.n_heads), dim3(128), smem, st, 
         static_cast<const float*>(c->q), kc, vtc, static_cast<float*>(c->o), g.n_heads,
         g.n_heads / g.n_kv_heads, c->tq, hd, g.kv_capacity, n_keys, causal ? pos0 : -1,
-        1.0f / sqrtf(static_cast<float>(hd)), done);
+        1.0f / sqrtf(static_cast<float>(hd)), done));
     DG_LAUNCHED();
-    gemm_f32_nt_kernel<<<dim3(cdiv(d, 64), cdiv(n, 64)), 256, 0, st>>>(
+    DG_TRY(launch_pdl(gemm_f32_nt_kernel, dim3(cdiv(d, 64), cdiv(n, 64)), dim3(256), 0, st, 
         static_cast<const float*>(c->o), static_cast<const float*>(w.wo), n, d, g.n_heads * hd,
-        c->part, d, done);
+        c->part, d, done));
     DG_LAUNCHED();
-    residual_norm_kernel<float><<<n, 256, 0, st>>>(c->x, c->part, 1, 0, d, w.ffn_norm, g.eps,
-                                                   static_cast<float*>(c->xn), done);
+    DG_TRY(launch_pdl(residual_norm_kernel<float>, dim3(n), dim3(256), 0, st, c->x, c->part, 1, 0, d, w.ffn_norm, g.eps,
+                                                   static_cast<float*>(c->xn), done));
     DG_LAUNCHED();
     }
     if (!(parts & 2)) return DG_OK;
-    gemm_f32_nt_kernel<<<dim3(cdiv(E, 64), cdiv(n, 64)), 256, 0, st>>>(
-        xn, static_cast<const float*>(w.wr), n, E, d, c->part, E, done);
+    DG_TRY(launch_pdl(gemm_f32_nt_kernel, dim3(cdiv(E, 64), cdiv(n, 64)), dim3(256), 0, st, 
+        xn, static_cast<const float*>(w.wr), n, E, d, c->part, E, done));
     DG_LAUNCHED();
-    router_topk_kernel<<<cdiv(n, 4), 128, 0, st>>>(c->part, 1, 0, n, E, k, c->router_logits,
-                                                   c->topk_ids, c->topk_w, done);
+    DG_TRY(launch_pdl(router_topk_kernel, dim3(cdiv(n, 4)), dim3(128), 0, st, c->part, 1, 0, n, E, k, c->router_logits,
+                                                   c->topk_ids, c->topk_w, done));
     DG_LAUNCHED();
     const int smem_e = (d + g.expert_hidden) * 4;
     DG_TRY(set_smem(moe_expert_f32_kernel, smem_e));
-    moe_expert_f32_kernel<<<n_slots, 256, smem_e, st>>>(
+    DG_TRY(launch_pdl(moe_expert_f32_kernel, dim3(n_slots), dim3(256), smem_e, st, 
         xn, c->topk_ids, c->topk_w, k, static_cast<const float*>(w.w_gu),
-        static_cast<const float*>(w.w_d), d, g.expert_hidden, c->y_slot, done);
+        static_cast<const float*>(w.w_d), d, g.expert_hidden, c->y_slot, done));
     DG_LAUNCHED();
     const float* ysh = nullptr;
     if (g.shared_hidden > 0) {
       const int smem_s = (d + g.shared_hidden) * 4;
       DG_TRY(set_smem(moe_expert_f32_kernel, std::max(smem_s, smem_e)));
-      moe_expert_f32_kernel<<<n, 256, smem_s, st>>>(
+      DG_TRY(launch_pdl(moe_expert_f32_kernel, dim3(n), dim3(256), smem_s, st, 
           xn, nullptr, nullptr, 1, static_cast<const float*>(w.ws_gu),
-          static_cast<const float*>(w.ws_d), d, g.shared_hidden, c->y_shared, done);
+          static_cast<const float*>(w.ws_d), d, g.shared_hidden, c->y_shared, done));
       DG_LAUNCHED();
       ysh = c->y_shared;
     }
-    moe_combine_norm_kernel<float><<<n, 256, 0, st>>>(c->x, c->y_slot, k, ysh, d, next_norm,
-                                                      g.eps, static_cast<float*>(c->xn), done);
+    DG_TRY(launch_pdl(moe_combine_norm_kernel<float>, dim3(n), dim3(256), 0, st, c->x, c->y_slot, k, ysh, d, next_norm,
+                                                      g.eps, static_cast<float*>(c->xn), done));
     DG_LAUNCHED();
     return DG_OK;
   }
@@ -512,14 +533,14 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     a.done = done;
     DG_TRY(set_smem(attention_kernel, kAttnSmemBytes));
     prof_before(DG_KERNEL_ATTENTION, st);
-    attention_kernel<<<dim3(m_tiles, g.n_kv_heads, splits), kAttnThreads, kAttnSmemBytes, st>>>(
-        c->tm_q, c->tm_k, c->tm_vt, a);
+    DG_TRY(launch_pdl(attention_kernel, dim3(m_tiles, g.n_kv_heads, splits), dim3(kAttnThreads), kAttnSmemBytes, st, 
+        c->tm_q, c->tm_k, c->tm_vt, a));
     DG_LAUNCHED();
     prof_after(DG_KERNEL_ATTENTION, st);
     prof_before(DG_KERNEL_ATTN_COMBINE, st);
-    attn_combine_kernel<__nv_bfloat16><<<cdiv(n * g.n_heads, 8), 256, 0, st>>>(
-        c->o_part, c->ml_part, splits, g.n_heads, c->tq, n, static_cast<__nv_bfloat16*>(c->o),
-        done);
+    DG_TRY(launch_pdl(attn_combine_kernel<__nv_bfloat16>, dim3(cdiv(n * g.n_heads, 8)), dim3(256), 0,
+                      st, c->o_part, c->ml_part, splits, g.n_heads, c->tq, n,
+                      static_cast<__nv_bfloat16*>(c->o), done));
     DG_LAUNCHED();
     prof_after(DG_KERNEL_ATTN_COMBINE, st);
   }
@@ -534,9 +555,9 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
                                                                  std::min(items, c->sms), st,
                                                                  DG_KERNEL_O_PROJ)));
     prof_before(DG_KERNEL_RESIDUAL_NORM, st);
-    residual_norm_kernel<__nv_bfloat16><<<n, 256, 0, st>>>(
+    DG_TRY(launch_pdl(residual_norm_kernel<__nv_bfloat16>, dim3(n), dim3(256), 0, st, 
         c->x, c->part, c->split_o, p.split_stride, d, w.ffn_norm, g.eps,
-        static_cast<__nv_bfloat16*>(c->xn), done);
+        static_cast<__nv_bfloat16*>(c->xn), done));
     DG_LAUNCHED();
     prof_after(DG_KERNEL_RESIDUAL_NORM, st);
   }
@@ -553,8 +574,8 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
                                                                  std::min(items, c->sms), st,
                                                                  DG_KERNEL_ROUTER)));
     prof_before(DG_KERNEL_ROUTER_TOPK, st);
-    router_topk_kernel<<<cdiv(n, 4), 128, 0, st>>>(c->part, c->split_r, p.split_stride, n, E, k,
-                                                   c->router_logits, c->topk_ids, c->topk_w, done);
+    DG_TRY(launch_pdl(router_topk_kernel, dim3(cdiv(n, 4)), dim3(128), 0, st, c->part, c->split_r, p.split_stride, n, E, k,
+                                                   c->router_logits, c->topk_ids, c->topk_w, done));
     DG_LAUNCHED();
     prof_after(DG_KERNEL_ROUTER_TOPK, st);
   }
@@ -578,13 +599,13 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     ra.shared_m_tiles_d = shared ? cdiv(d, 128) : 0;
     ra.done = done;
     prof_before(DG_KERNEL_ROUTE, st);
-    moe_route_kernel<<<1, 1024, 0, st>>>(ra);
+    DG_TRY(launch_pdl(moe_route_kernel, dim3(1), dim3(1024), 0, st, ra));
     DG_LAUNCHED();
     prof_after(DG_KERNEL_ROUTE, st);
     prof_before(DG_KERNEL_GATHER, st);
-    gather_rows_kernel<<<cdiv(n_slots, 4), 256, 0, st>>>(
+    DG_TRY(launch_pdl(gather_rows_kernel, dim3(cdiv(n_slots, 4)), dim3(256), 0, st, 
         static_cast<const __nv_bfloat16*>(c->xn), c->perm, k, d, n_slots,
-        static_cast<__nv_bfloat16*>(c->x_perm), done);
+        static_cast<__nv_bfloat16*>(c->x_perm), done));
     DG_LAUNCHED();
     prof_after(DG_KERNEL_GATHER, st);
     GemmParams p{};
@@ -628,8 +649,8 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
   }
   const float* ysh = shared ? c->y_shared : nullptr;
   prof_before(DG_KERNEL_COMBINE_NORM, st);
-  moe_combine_norm_kernel<__nv_bfloat16><<<n, 256, 0, st>>>(
-      c->x, c->y_slot, k, ysh, d, next_norm, g.eps, static_cast<__nv_bfloat16*>(c->xn), done);
+  DG_TRY(launch_pdl(moe_combine_norm_kernel<__nv_bfloat16>, dim3(n), dim3(256), 0, st, 
+      c->x, c->y_slot, k, ysh, d, next_norm, g.eps, static_cast<__nv_bfloat16*>(c->xn), done));
   DG_LAUNCHED();
   prof_after(DG_KERNEL_COMBINE_NORM, st);
   return DG_OK;
@@ -652,23 +673,23 @@ int run_lm_head(dg_ctx* c, float* logits_out, const int* done, cudaStream_t st) 
     prof_before(DG_KERNEL_LM_HEAD, st);
     if (logits_out) {
       DG_TRY(set_smem(lmhead_kernel<false>, kLmSmemBytes));
-      lmhead_kernel<false><<<grid, kLmThreads, kLmSmemBytes, st>>>(c->tm_xn128, c->tm_embed, p);
+      DG_TRY(launch_pdl(lmhead_kernel<false>, dim3(grid), dim3(kLmThreads), kLmSmemBytes, st, c->tm_xn128, c->tm_embed, p));
     } else {
       DG_TRY(set_smem(lmhead_kernel<true>, kLmSmemBytes));
-      lmhead_kernel<true><<<grid, kLmThreads, kLmSmemBytes, st>>>(c->tm_xn128, c->tm_embed, p);
+      DG_TRY(launch_pdl(lmhead_kernel<true>, dim3(grid), dim3(kLmThreads), kLmSmemBytes, st, c->tm_xn128, c->tm_embed, p));
     }
     DG_LAUNCHED();
     prof_after(DG_KERNEL_LM_HEAD, st);
     return DG_OK;
   }
   float* dst = logits_out ? logits_out : c->logits;
-  gemm_f32_nt_kernel<<<dim3(cdiv(g.vocab, 64), cdiv(T, 64)), 256, 0, st>>>(
+  DG_TRY(launch_pdl(gemm_f32_nt_kernel, dim3(cdiv(g.vocab, 64), cdiv(T, 64)), dim3(256), 0, st, 
       static_cast<const float*>(c->xn), static_cast<const float*>(c->embed), T, g.vocab, g.d_model,
-      dst, g.vocab, done);
+      dst, g.vocab, done));
   DG_LAUNCHED();
   if (!logits_out) {
-    logits_stats_kernel<float, 16><<<dim3(cdiv(g.vocab, 4096), T), 256, 0, st>>>(
-        c->logits, g.vocab, 4096, c->lm_part, done);
+    DG_TRY(launch_pdl(logits_stats_kernel<float, 16>, dim3(cdiv(g.vocab, 4096), T), dim3(256), 0, st, 
+        c->logits, g.vocab, 4096, c->lm_part, done));
     DG_LAUNCHED();
   }
   return DG_OK;
@@ -850,8 +871,8 @@ int dg_create(const dg_config* cfg, const dg_weights* w, void* d_kv, void* d_scr
   }
   const int half = cfg->head_dim / 2;
   const long long n_tab = static_cast<long long>(cfg->kv_capacity) * half;
-  rope_table_kernel<<<cdiv(n_tab, 256), 256, 0, st>>>(c->rope_tab, cfg->kv_capacity, half,
-                                                       static_cast<double>(cfg->rope_theta));
+  DG_TRY(launch_pdl(rope_table_kernel, dim3(cdiv(n_tab, 256)), dim3(256), 0, st, c->rope_tab, cfg->kv_capacity, half,
+                                                       static_cast<double>(cfg->rope_theta)));
   e = cudaGetLastError();
   if (e != cudaSuccess) {
     delete c;
@@ -894,8 +915,8 @@ int dg_canvas_init(dg_ctx* ctx, uint64_t seed, uint32_t block, void* stream) {
     return fail(DG_ERR_CAPACITY, "no room for a canvas after %d committed positions", ctx->kv_len);
   ctx->seed = seed;
   ctx->block = block;
-  canvas_init_kernel<<<cdiv(ctx->cfg.canvas, 256), 256, 0, S(stream)>>>(
-      ctx->canvas, ctx->cfg.canvas, ctx->cfg.vocab, seed, block, ctx->state, ctx->ticket);
+  DG_TRY(launch_pdl(canvas_init_kernel, dim3(cdiv(ctx->cfg.canvas, 256)), dim3(256), 0, S(stream),
+      ctx->canvas, ctx->cfg.canvas, ctx->cfg.vocab, seed, block, ctx->state, ctx->ticket));
   DG_LAUNCHED();
   return DG_OK;
 }
@@ -938,7 +959,7 @@ int dg_sample_update(dg_ctx* ctx, uint32_t step, void* stream) {
   a.state = ctx->state;
   a.ticket = ctx->ticket;
   prof_before(DG_KERNEL_SAMPLER, S(stream));
-  sampler_merge_kernel<<<g.canvas, 256, 0, S(stream)>>>(a);
+  DG_TRY(launch_pdl(sampler_merge_kernel, dim3(g.canvas), dim3(256), 0, S(stream), a));
   DG_LAUNCHED();
   prof_after(DG_KERNEL_SAMPLER, S(stream));
   return DG_OK;
@@ -1007,11 +1028,11 @@ int dg_debug_layer_part(dg_ctx* ctx, int32_t layer, int32_t part, const float* d
                           cudaMemcpyDeviceToDevice, st));
   const float* w = part == 0 ? ctx->layers[layer].attn_norm : ctx->layers[layer].ffn_norm;
   if (ctx->bf16)
-    residual_norm_kernel<__nv_bfloat16><<<n, 256, 0, st>>>(
-        ctx->x, ctx->part, 0, 0, g.d_model, w, g.eps, static_cast<__nv_bfloat16*>(ctx->xn), nullptr);
+    DG_TRY(launch_pdl(residual_norm_kernel<__nv_bfloat16>, dim3(n), dim3(256), 0, st, 
+        ctx->x, ctx->part, 0, 0, g.d_model, w, g.eps, static_cast<__nv_bfloat16*>(ctx->xn), nullptr));
   else
-    residual_norm_kernel<float><<<n, 256, 0, st>>>(ctx->x, ctx->part, 0, 0, g.d_model, w, g.eps,
-                                                   static_cast<float*>(ctx->xn), nullptr);
+    DG_TRY(launch_pdl(residual_norm_kernel<float>, dim3(n), dim3(256), 0, st, ctx->x, ctx->part, 0, 0, g.d_model, w, g.eps,
+                                                   static_cast<float*>(ctx->xn), nullptr));
   DG_LAUNCHED();
   const float* nn = (layer + 1 < g.n_layers) ? ctx->layers[layer + 1].attn_norm : ctx->final_norm;
   DG_TRY(run_layer(ctx, layer, n, ctx->kv_len, causal, nn, nullptr, st, part == 0 ? 1 : 2));
@@ -1048,11 +1069,11 @@ int dg_debug_layer(dg_ctx* ctx, int32_t layer, const float* d_x_in, float* d_x_o
                           cudaMemcpyDeviceToDevice, st));
   const float* w = ctx->layers[layer].attn_norm;
   if (ctx->bf16)
-    residual_norm_kernel<__nv_bfloat16><<<n, 256, 0, st>>>(
-        ctx->x, ctx->part, 0, 0, g.d_model, w, g.eps, static_cast<__nv_bfloat16*>(ctx->xn), nullptr);
+    DG_TRY(launch_pdl(residual_norm_kernel<__nv_bfloat16>, dim3(n), dim3(256), 0, st, 
+        ctx->x, ctx->part, 0, 0, g.d_model, w, g.eps, static_cast<__nv_bfloat16*>(ctx->xn), nullptr));
   else
-    residual_norm_kernel<float><<<n, 256, 0, st>>>(ctx->x, ctx->part, 0, 0, g.d_model, w, g.eps,
-                                                   static_cast<float*>(ctx->xn), nullptr);
+    DG_TRY(launch_pdl(residual_norm_kernel<float>, dim3(n), dim3(256), 0, st, ctx->x, ctx->part, 0, 0, g.d_model, w, g.eps,
+                                                   static_cast<float*>(ctx->xn), nullptr));
   DG_LAUNCHED();
   const float* nn = (layer + 1 < g.n_layers) ? ctx->layers[layer + 1].attn_norm : ctx->final_norm;
   DG_TRY(run_layer(ctx, layer, n, ctx->kv_len, causal, nn, nullptr, st));
@@ -1062,7 +1083,6 @@ int dg_debug_layer(dg_ctx* ctx, int32_t layer, const float* d_x_in, float* d_x_o
 }
 
 // ---- standalone sampler ----------------------------------------------------------------
-static int sampler_chunk(int32_t dtype) { return dtype == DG_DTYPE_BF16 ? 8192 : 4096; }
 
 int dg_sampler_workspace_bytes(int32_t rows, int32_t vocab, size_t* bytes) {
   if (rows < 1 || rows > 1024 || vocab < 2 || vocab % 8 || !bytes)
@@ -1119,7 +1139,8 @@ int dg_sampler_step(const void* d_logits, int32_t dtype, int32_t rows, int32_t v
   double* row_h;
   sampler_views(d_workspace, rows, vocab, &part, &prev, &row_h, &locked, &ticket, &row_ticket);
   cudaStream_t st = S(stream);
-  const int chunk = sampler_chunk(dtype);
+  // row slices of 65536 columns (eight 32-value groups per thread)
+  const int chunk = 65536;
   const int nchunk = cdiv(vocab, chunk);
   SamplerArgs a{};
   a.partials = part;
@@ -1144,11 +1165,11 @@ int dg_sampler_step(const void* d_logits, int32_t dtype, int32_t rows, int32_t v
   a.ticket = ticket;
   prof_before(DG_KERNEL_SAMPLER, st);
   if (dtype == DG_DTYPE_BF16)
-    sampler_fused_kernel<__nv_bfloat16, 32><<<dim3(nchunk, rows), 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(d_logits), chunk, a, row_ticket);
+    DG_TRY(launch_pdl(sampler_fused_kernel<__nv_bfloat16, 4>, dim3(nchunk, rows), dim3(256), 0, st, 
+        static_cast<const __nv_bfloat16*>(d_logits), chunk, a, row_ticket));
   else
-    sampler_fused_kernel<float, 16><<<dim3(nchunk, rows), 256, 0, st>>>(
-        static_cast<const float*>(d_logits), chunk, a, row_ticket);
+    DG_TRY(launch_pdl(sampler_fused_kernel<float, 8>, dim3(nchunk, rows), dim3(256), 0, st, 
+        static_cast<const float*>(d_logits), chunk, a, row_ticket));
   DG_LAUNCHED();
   prof_after(DG_KERNEL_SAMPLER, st);
   return DG_OK;
@@ -1161,7 +1182,8 @@ int dg_attention_workspace_bytes(int32_t n_heads, int32_t n_kv_heads, int32_t tq
     return fail(DG_ERR_INVALID_ARG, "bad attention shape");
   const int splits = std::max(1, cdiv(n_keys, 128));
   *bytes = align256(static_cast<size_t>(splits) * n_heads * tq * 128 * 4) +
-           align256(static_cast<size_t>(splits) * n_heads * tq * 8) + 4 * 256;
+           align256(static_cast<size_t>(splits) * n_heads * tq * 8) +
+           align256(static_cast<size_t>(n_heads) * tq / 128 * 4) + 4 * 256;
   return DG_OK;
 }
 
@@ -1184,7 +1206,9 @@ int dg_canvas_attention(const void* d_q, const void* d_k, const void* d_vt, void
   const int tps = cdiv(n_kv_tiles, splits);
   splits = cdiv(n_kv_tiles, tps);
   const size_t o_bytes = align256(static_cast<size_t>(splits) * n_heads * tq * 128 * 4);
-  const size_t need = o_bytes + align256(static_cast<size_t>(splits) * n_heads * tq * 8) + 256;
+  const size_t ml_bytes = align256(static_cast<size_t>(splits) * n_heads * tq * 8);
+  const size_t tk_bytes = align256(static_cast<size_t>(n_kv_heads) * m_tiles * 4);
+  const size_t need = o_bytes + ml_bytes + tk_bytes + 256;
   if (workspace_bytes < need) return fail(DG_ERR_CAPACITY, "attention workspace too small");
   uint8_t* ws = static_cast<uint8_t*>(d_workspace);
   CUtensorMap tq_m, tk_m, tv_m;
@@ -1211,11 +1235,12 @@ int dg_canvas_attention(const void* d_q, const void* d_k, const void* d_vt, void
   cudaStream_t st = S(stream);
   DG_CUDA(cudaMemsetAsync(a.err, 0, 4, st));
   DG_TRY(set_smem(attention_kernel, kAttnSmemBytes));
-  attention_kernel<<<dim3(m_tiles, n_kv_heads, splits), kAttnThreads, kAttnSmemBytes, st>>>(tq_m, tk_m, tv_m,
-                                                                                  a);
+  DG_TRY(launch_pdl(attention_kernel, dim3(m_tiles, n_kv_heads, splits), dim3(kAttnThreads), kAttnSmemBytes, st, tq_m, tk_m, tv_m,
+                                                                                  a));
   DG_LAUNCHED();
-  attn_combine_kernel<__nv_bfloat16><<<cdiv(t * n_heads, 8), 256, 0, st>>>(
-      a.o_part, a.ml_part, splits, n_heads, tq, t, static_cast<__nv_bfloat16*>(d_o), nullptr);
+  DG_TRY(launch_pdl(attn_combine_kernel<__nv_bfloat16>, dim3(cdiv(t * n_heads, 8)), dim3(256), 0, st,
+                    a.o_part, a.ml_part, splits, n_heads, tq, t, static_cast<__nv_bfloat16*>(d_o),
+                    nullptr));
   DG_LAUNCHED();
   return DG_OK;
 }
@@ -1321,8 +1346,8 @@ int dg_moe_ffn(const void* d_x, const float* d_residual, const void* d_wr, const
   pr.split_stride = static_cast<long long>(t) * n_experts;
   DG_TRY((launch_gemm<kDenseN, kDenseStages, kEpiPartialF32>(
       t_wr, t_x32, pr, std::min(pr.m_tiles * pr.k_splits * pr.n_chunks, sms), st)));
-  router_topk_kernel<<<cdiv(t, 4), 128, 0, st>>>(rpart, m.split_r, pr.split_stride, t, n_experts,
-                                                 top_k, d_router_logits, ids, wts, nullptr);
+  DG_TRY(launch_pdl(router_topk_kernel, dim3(cdiv(t, 4)), dim3(128), 0, st, rpart, m.split_r, pr.split_stride, t, n_experts,
+                                                 top_k, d_router_logits, ids, wts, nullptr));
   DG_LAUNCHED();
   const bool shared = shared_hidden > 0;
   RouteArgs ra{};
@@ -1341,10 +1366,10 @@ int dg_moe_ffn(const void* d_x, const float* d_residual, const void* d_wr, const
   ra.shared_m_tiles_gu = shared ? cdiv(2 * shared_hidden, 128) : 0;
   ra.shared_m_tiles_d = shared ? cdiv(d, 128) : 0;
   ra.done = nullptr;
-  moe_route_kernel<<<1, 1024, 0, st>>>(ra);
+  DG_TRY(launch_pdl(moe_route_kernel, dim3(1), dim3(1024), 0, st, ra));
   DG_LAUNCHED();
-  gather_rows_kernel<<<cdiv(t * top_k, 4), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(d_x),
-                                                         perm, top_k, d, t * top_k, x_perm, nullptr);
+  DG_TRY(launch_pdl(gather_rows_kernel, dim3(cdiv(t * top_k, 4)), dim3(256), 0, st, static_cast<const __nv_bfloat16*>(d_x),
+                                                         perm, top_k, d, t * top_k, x_perm, nullptr));
   DG_LAUNCHED();
   GemmParams pg{};
   pg.items = items_gu;
@@ -1388,8 +1413,8 @@ int dg_moe_ffn(const void* d_x, const float* d_residual, const void* d_wr, const
                             cudaMemcpyDeviceToDevice, st));
   else
     DG_CUDA(cudaMemsetAsync(d_y, 0, static_cast<size_t>(t) * d * 4, st));
-  moe_combine_norm_kernel<__nv_bfloat16><<<t, 256, 0, st>>>(d_y, y_slot, top_k, ysh_ptr, d, nullptr,
-                                                            0.f, nullptr, nullptr);
+  DG_TRY(launch_pdl(moe_combine_norm_kernel<__nv_bfloat16>, dim3(t), dim3(256), 0, st, d_y, y_slot, top_k, ysh_ptr, d, nullptr,
+                                                            0.f, nullptr, nullptr));
   DG_LAUNCHED();
   if (d_ids)
     DG_CUDA(cudaMemcpyAsync(d_ids, ids, static_cast<size_t>(t) * top_k * 4,
@@ -1479,11 +1504,11 @@ extern "C" int dg_sampler_step_static(const void* d_logits, int32_t dtype, int32
   const int nchunk = cdiv(vocab, chunk);
   const int* done = d_state + kStDone;
   if (dtype == DG_DTYPE_BF16)
-    logits_stats_kernel<__nv_bfloat16, 32><<<dim3(nchunk, rows), 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(d_logits), vocab, chunk, part, done);
+    DG_TRY(launch_pdl(logits_stats_kernel<__nv_bfloat16, 32>, dim3(nchunk, rows), dim3(256), 0, st, 
+        static_cast<const __nv_bfloat16*>(d_logits), vocab, chunk, part, done));
   else
-    logits_stats_kernel<float, 16><<<dim3(nchunk, rows), 256, 0, st>>>(
-        static_cast<const float*>(d_logits), vocab, chunk, part, done);
+    DG_TRY(launch_pdl(logits_stats_kernel<float, 16>, dim3(nchunk, rows), dim3(256), 0, st, 
+        static_cast<const float*>(d_logits), vocab, chunk, part, done));
   DG_LAUNCHED();
   SamplerArgs a{};
   a.partials = part;
@@ -1506,7 +1531,7 @@ extern "C" int dg_sampler_step_static(const void* d_logits, int32_t dtype, int32
   a.locked = locked;
   a.state = d_state;
   a.ticket = ticket;
-  sampler_merge_kernel<<<rows, 256, 0, st>>>(a);
+  DG_TRY(launch_pdl(sampler_merge_kernel, dim3(rows), dim3(256), 0, st, a));
   DG_LAUNCHED();
   return DG_OK;
 }

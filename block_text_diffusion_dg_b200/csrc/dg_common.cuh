@@ -251,6 +251,30 @@ DG_DEV float tmem_ld1(uint32_t taddr) {
   return __uint_as_float(r);
 }
 
+// Packed fp32 pairs (sm_100 f32x2 arithmetic): a.x/a.y in one 64-bit register.
+DG_DEV float2 ffma2(float2 a, float2 b, float2 c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(r)
+      : "l"(*reinterpret_cast<const uint64_t*>(&a)), "l"(*reinterpret_cast<const uint64_t*>(&b)),
+        "l"(*reinterpret_cast<const uint64_t*>(&c)));
+  return *reinterpret_cast<const float2*>(&r);
+}
+DG_DEV float2 fmul2(float2 a, float2 b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;"
+      : "=l"(r)
+      : "l"(*reinterpret_cast<const uint64_t*>(&a)), "l"(*reinterpret_cast<const uint64_t*>(&b)));
+  return *reinterpret_cast<const float2*>(&r);
+}
+DG_DEV float2 fadd2(float2 a, float2 b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;"
+      : "=l"(r)
+      : "l"(*reinterpret_cast<const uint64_t*>(&a)), "l"(*reinterpret_cast<const uint64_t*>(&b)));
+  return *reinterpret_cast<const float2*>(&r);
+}
+
 // Barrier over `count` threads (whole warps) on hardware barrier `id` (1..15).
 DG_DEV void named_barrier(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
@@ -302,6 +326,15 @@ template <>
 DG_DEV float store_from_f32<float>(float x) { return x; }
 template <>
 DG_DEV __nv_bfloat16 store_from_f32<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+
+// Programmatic dependent launch: wait until the previous grid in the stream has completed and
+// its writes are visible, then let the next grid start launching (it waits the same way).
+DG_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+DG_DEV void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+DG_DEV void pdl_enter() {
+  pdl_wait();
+  pdl_launch_dependents();
+}
 
 // Early-out used by every kernel of a denoise step once the block has stopped.
 DG_DEV bool block_done(const int* done) { return done != nullptr && *reinterpret_cast<const volatile int*>(done) != 0; }

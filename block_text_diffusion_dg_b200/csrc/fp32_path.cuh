@@ -11,6 +11,7 @@ __global__ void __launch_bounds__(256) gemm_f32_nt_kernel(const float* __restric
                                                           const float* __restrict__ W, int M, int N,
                                                           int K, float* __restrict__ out,
                                                           long long ld, const int* done) {
+  pdl_enter();
   if (block_done(done)) return;
   __shared__ float xs[16][65];
   __shared__ float ws[16][65];
@@ -54,6 +55,7 @@ __global__ void __launch_bounds__(128) attention_f32_kernel(
     const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ vt,
     float* __restrict__ o, int n_heads, int group, int tq, int hd, int ldk, int n_keys,
     int causal_prefix, float scale, const int* done) {
+  pdl_enter();
   if (block_done(done)) return;
   extern __shared__ float sc[];  // [n_keys] scores, then [hd] query
   float* qs = sc + n_keys;
@@ -103,6 +105,7 @@ __global__ void __launch_bounds__(256) moe_expert_f32_kernel(
     const float* __restrict__ xn, const int32_t* __restrict__ ids, const float* __restrict__ wts,
     int top_k, const float* __restrict__ w_gu, const float* __restrict__ w_d, int d, int hidden,
     float* __restrict__ y, const int* done) {
+  pdl_enter();
   if (block_done(done)) return;
   extern __shared__ float sm[];  // [d] x, then [hidden] h
   float* xs = sm;

@@ -169,6 +169,7 @@ __global__ void __launch_bounds__(GemmCfg<MAXN, STAGES>::kThreads, 1)
                        const __grid_constant__ CUtensorMap tm_a2,
                        const __grid_constant__ CUtensorMap tm_b2, const GemmParams p) {
   using C = GemmCfg<MAXN, STAGES>;
+  pdl_enter();
   if (block_done(p.done)) return;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -352,6 +353,7 @@ template <bool kStats>
 __global__ void __launch_bounds__(kLmThreads, 1)
     lmhead_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_e,
                   const LmHeadParams p) {
+  pdl_enter();
   if (block_done(p.done)) return;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &

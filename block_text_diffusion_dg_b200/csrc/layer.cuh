@@ -36,6 +36,7 @@ __global__ void __launch_bounds__(256) embed_norm_kernel(const int32_t* __restri
                                                          const float* __restrict__ w, float eps,
                                                          float* __restrict__ x,
                                                          TA* __restrict__ xn, const int* done) {
+  pdl_enter();
   if (block_done(done)) return;
   __shared__ float sm[8];
   const int t = blockIdx.x;
@@ -99,6 +100,7 @@ __global__ void __launch_bounds__(128) qkv_finalize_kernel(
     int n_heads, int n_kv_heads, const float2* __restrict__ rope_tab, int n, int pos0,
     TA* __restrict__ q, int tq, TA* __restrict__ k_cache, TA* __restrict__ vt_cache, int ldk,
     const int* done) {
+  pdl_enter();
   if (block_done(done)) return;
   __shared__ float blk[kQkvTok][128 + 4];
   const int t0 = blockIdx.x * kQkvTok, h = blockIdx.y, tid = threadIdx.x;
@@ -144,6 +146,7 @@ __global__ void __launch_bounds__(256) residual_norm_kernel(float* __restrict__ 
                                                             int d, const float* __restrict__ w,
                                                             float eps, TA* __restrict__ xn,
                                                             const int* done) {
+  pdl_enter();
   if (block_done(done)) return;
   __shared__ float sm[8];
   const int t = blockIdx.x;
@@ -186,6 +189,7 @@ __global__ void router_topk_kernel(const float* __restrict__ part, int splits,
                                    long long split_stride, int n_tokens, int n_experts, int top_k,
                                    float* __restrict__ logits_out, int32_t* __restrict__ ids,
                                    float* __restrict__ wts, const int* done) {
+  pdl_enter();
   if (block_done(done)) return;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= n_tokens) return;
@@ -287,6 +291,7 @@ DG_DEV int warp_exclusive_scan_256(const int* in, int* out, int n) {
 // lists, and the stable placement (slot order inside each expert) via warp match + per-warp
 // counts.  Items are (expert, 128-row tile, first permuted row, tokens <= n_chunk).
 __global__ void __launch_bounds__(1024) moe_route_kernel(RouteArgs a) {
+  pdl_enter();
   if (block_done(a.done)) return;
   __shared__ int cnt[32][257];  // per-warp counts in the current round, per expert
   __shared__ int count_s[256], off_s[257], chunk_s[256], cbase_s[256], base_s[256];
@@ -380,6 +385,7 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const __nv_bfloat16* _
                                                           int top_k, int d, int n_rows,
                                                           __nv_bfloat16* __restrict__ x_perm,
                                                           const int* done) {
+  pdl_enter();
   if (block_done(done)) return;
   const int p = blockIdx.x * 4 + (threadIdx.x >> 6);
   if (p >= n_rows) return;
@@ -396,6 +402,7 @@ __global__ void __launch_bounds__(256) moe_combine_norm_kernel(
     float* __restrict__ x, const float* __restrict__ y_slot, int top_k,
     const float* __restrict__ y_shared, int d, const float* __restrict__ w, float eps,
     TA* __restrict__ xn, const int* done) {
+  pdl_enter();
   if (block_done(done)) return;
   __shared__ float sm[8];
   const int t = blockIdx.x;
@@ -455,6 +462,7 @@ __global__ void __launch_bounds__(256) moe_combine_norm_kernel(
 
 // RoPE table: (cos, sin) of pos * theta^(-2i/hd) for pos < n_pos, i < hd/2, computed in fp64.
 __global__ void rope_table_kernel(float2* tab, int n_pos, int half, double theta) {
+  pdl_enter();
   const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= static_cast<long long>(n_pos) * half) return;
   const int pos = static_cast<int>(idx / half), i = static_cast<int>(idx % half);

@@ -55,6 +55,7 @@ DG_DEV StatD stat_merge(const StatD& x, const StatD& y) {
 
 __global__ void canvas_init_kernel(int32_t* canvas, int32_t t, int32_t vocab, uint64_t seed,
                                    uint32_t block, int32_t* state, int32_t* ticket) {
+  pdl_enter();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < t) canvas[i] = canvas_uniform_id(seed, block, 0u, static_cast<uint32_t>(i), 0u,
                                            static_cast<uint32_t>(vocab));
@@ -167,6 +168,7 @@ __global__ void __launch_bounds__(256) logits_stats_kernel(const T* __restrict__
                                                            int32_t vocab, int32_t chunk,
                                                            StatPartial* __restrict__ out,
                                                            const int* done) {
+  pdl_enter();
   if (block_done(done)) return;
   __shared__ float sm_f[16];
   __shared__ int sm_i[8];
@@ -207,8 +209,9 @@ struct SamplerArgs {
 DG_DEV bool sampler_row(const SamplerArgs& p, int row) {
   StatD acc{0.0, 0.0, 0.0, 0x7fffffff};
   for (int i = threadIdx.x; i < p.nsplit; i += blockDim.x) {
-    const StatPartial q = p.partials[static_cast<size_t>(row) * p.nsplit + i];
-    acc = stat_merge(acc, StatD{q.m, q.s, q.u, q.a});
+    const float4 q4 = __ldcg(reinterpret_cast<const float4*>(p.partials) +
+                             static_cast<size_t>(row) * p.nsplit + i);
+    acc = stat_merge(acc, StatD{q4.x, q4.y, q4.z, __float_as_int(q4.w)});
   }
   __shared__ StatD red[256];
   red[threadIdx.x] = acc;
@@ -238,28 +241,34 @@ DG_DEV bool sampler_row(const SamplerArgs& p, int row) {
   return is_last;
 }
 
-// The stop test over the whole canvas, run by the last row's CTA (after a fence).
+// The stop test over the whole canvas, run by the last row's CTA (after a fence).  Rows written
+// by other CTAs are read through L2 (ld.global.cg); the mean entropy is a fixed-shape fp64 tree
+// over the rows, so it does not depend on timing.  rows <= 1024.
 DG_DEV void sampler_stop_test(const SamplerArgs& p) {
   __threadfence();
+  __shared__ double hs[256];
   __shared__ int n_diff, n_locked;
   if (threadIdx.x == 0) {
     n_diff = 0;
     n_locked = 0;
   }
-  __syncthreads();
+  double h_part = 0.0;
   int my_diff = 0, my_locked = 0;
   for (int i = threadIdx.x; i < p.rows; i += blockDim.x) {
-    my_diff += (*reinterpret_cast<volatile int32_t*>(p.argmax + i) != p.prev_argmax[i]);
-    my_locked += *reinterpret_cast<volatile int32_t*>(p.locked + i);
+    my_diff += (__ldcg(p.argmax + i) != p.prev_argmax[i]);
+    my_locked += __ldcg(p.locked + i);
+    h_part += __ldcg(p.row_h + i);
   }
+  hs[threadIdx.x] = h_part;
+  __syncthreads();
   atomicAdd(&n_diff, my_diff);
   atomicAdd(&n_locked, my_locked);
-  __syncthreads();
+  for (int o = 128; o > 0; o >>= 1) {
+    if (threadIdx.x < o) hs[threadIdx.x] += hs[threadIdx.x + o];
+    __syncthreads();
+  }
   if (threadIdx.x == 0) {
-    double hsum = 0.0;
-    for (int i = 0; i < p.rows; ++i)  // fixed order: deterministic mean
-      hsum += *reinterpret_cast<volatile double*>(p.row_h + i);
-    const double hbar = hsum / p.rows;
+    const double hbar = hs[0] / p.rows;
     const int step = static_cast<int>(p.step);
     const bool stop_now = step >= 2 && hbar < static_cast<double>(p.h_bound) && n_diff == 0;
     int32_t* st = p.state;
@@ -275,34 +284,220 @@ DG_DEV void sampler_stop_test(const SamplerArgs& p) {
     *p.ticket = 0;
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < p.rows; i += blockDim.x)
-    p.prev_argmax[i] = *reinterpret_cast<volatile int32_t*>(p.argmax + i);
+  for (int i = threadIdx.x; i < p.rows; i += blockDim.x) p.prev_argmax[i] = __ldcg(p.argmax + i);
 }
 
 // One CTA per row: merge the row's partials, decide lock / re-noise; the last CTA to finish
 // evaluates the stop rule for the whole canvas (no CTA ever waits on another).
 __global__ void __launch_bounds__(256) sampler_merge_kernel(SamplerArgs p) {
+  pdl_enter();
   if (block_done(p.state + kStDone)) return;
   if (sampler_row(p, blockIdx.x)) sampler_stop_test(p);
 }
 
-// Statistics, merge and stop test in one launch: grid = (chunks, rows).  Each CTA writes its
-// slice's partial; the last CTA of a row (per-row ticket) merges the row; the last row runs the
-// stop test.  row_ticket [rows] must start at zero and is left at zero.
-template <typename T, int kPerThread>
+// (m, S, U, a) <- merge with (m2, S2, U2, a2) in fp32 (2^x on the special-function unit); an
+// empty side (S = 0) is ignored; equal maxima keep the lower argmax.
+DG_DEV void stat_merge_f32(float& m, float& s, float& u, int& a, float m2, float s2, float u2,
+                           int a2) {
+  constexpr float kLog2e = 1.4426950408889634f;
+  if (s2 == 0.f) return;
+  if (s == 0.f) {
+    m = m2;
+    s = s2;
+    u = u2;
+    a = a2;
+    return;
+  }
+  const float mm = fmaxf(m, m2);
+  const int aa = (m > m2 || (m == m2 && a < a2)) ? a : a2;
+  const float d1 = m - mm, d2 = m2 - mm;
+  const float e1 = fast_exp2(d1 * kLog2e), e2 = fast_exp2(d2 * kLog2e);
+  u = e1 * (u + d1 * s) + e2 * (u2 + d2 * s2);
+  s = e1 * s + e2 * s2;
+  m = mm;
+  a = aa;
+}
+
+// Streaming statistics of one row slice for a 256-thread CTA.  Every thread walks its columns in
+// groups of kLoads 16-byte vectors (column c0 + ((g * kLoads + l) * 256 + tid) * kVec + j,
+// increasing in (g, l, j)) keeping running (m, S, T) with T = sum e t, t = (x - m) log2 e and
+// e = 2^t, so U = T / log2 e; S and T are rescaled only when a group raises the maximum.  The
+// argmax is resolved at the end: threads holding the CTA maximum re-read the one group where
+// they last raised it and take its first matching column.  Thread 0 returns the result.
+template <typename T> DG_DEV void to_f32x8(const uint4& raw, float (&v)[16 / sizeof(T)]);
+template <> DG_DEV void to_f32x8<__nv_bfloat16>(const uint4& raw, float (&v)[8]) {
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    v[2 * q] = __uint_as_float(w[q] << 16);
+    v[2 * q + 1] = __uint_as_float(w[q] & 0xffff0000u);
+  }
+}
+template <> DG_DEV void to_f32x8<float>(const uint4& raw, float (&v)[4]) {
+  v[0] = __uint_as_float(raw.x);
+  v[1] = __uint_as_float(raw.y);
+  v[2] = __uint_as_float(raw.z);
+  v[3] = __uint_as_float(raw.w);
+}
+
+template <typename T, int kLoads>
+DG_DEV StatPartial stream_slice_stats(const T* base, int c0, int c1, StatD* red) {
+  constexpr int kVec = 16 / sizeof(T);
+  constexpr int kSpan = kLoads * 256 * kVec;  // columns per group over the CTA
+  constexpr float kLog2e = 1.4426950408889634f;
+  const int tid = threadIdx.x;
+  float m = -INFINITY;
+  float2 s2 = make_float2(0.f, 0.f), t2 = make_float2(0.f, 0.f);
+  int g_best = -1;  // group (its first column) where m was last raised
+  // one group of loads in flight ahead of the arithmetic (register double buffer)
+  auto load_group = [&](int g0, uint4 (&dst)[kLoads]) {
+    const bool full = g0 + kSpan <= c1;
+#pragma unroll
+    for (int l = 0; l < kLoads; ++l) {
+      const int c = g0 + (l * 256 + tid) * kVec;
+      if (full || c < c1) {
+        dst[l] = __ldcs(reinterpret_cast<const uint4*>(base + c));
+      } else if constexpr (sizeof(T) == 2) {
+        dst[l] = make_uint4(0xff80ff80u, 0xff80ff80u, 0xff80ff80u, 0xff80ff80u);  // bf16 -inf
+      } else {
+        dst[l] = make_uint4(0xff800000u, 0xff800000u, 0xff800000u, 0xff800000u);  // fp32 -inf
+      }
+    }
+  };
+  uint4 next[kLoads];
+  if (c0 < c1) load_group(c0, next);
+  for (int g0 = c0; g0 < c1; g0 += kSpan) {
+    const bool full = g0 + kSpan <= c1;
+    uint4 raw[kLoads];
+#pragma unroll
+    for (int l = 0; l < kLoads; ++l) raw[l] = next[l];
+    if (g0 + kSpan < c1) load_group(g0 + kSpan, next);
+    // group maximum (packed bf16 pairs for bf16 input); -inf padding never wins
+    float gm;
+    if constexpr (sizeof(T) == 2) {
+      __nv_bfloat162 mx = *reinterpret_cast<const __nv_bfloat162*>(&raw[0].x);
+#pragma unroll
+      for (int l = 0; l < kLoads; ++l) {
+        const uint32_t w[4] = {raw[l].x, raw[l].y, raw[l].z, raw[l].w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) mx = __hmax2(mx, *reinterpret_cast<const __nv_bfloat162*>(&w[q]));
+      }
+      gm = fmaxf(__low2float(mx), __high2float(mx));
+    } else {
+      gm = -INFINITY;
+#pragma unroll
+      for (int l = 0; l < kLoads; ++l)
+        gm = fmaxf(fmaxf(__uint_as_float(raw[l].x), __uint_as_float(raw[l].y)),
+                   fmaxf(fmaxf(__uint_as_float(raw[l].z), __uint_as_float(raw[l].w)), gm));
+    }
+    if (gm > m) {  // strict: an earlier group keeps an equal maximum
+      if (m != -INFINITY) {
+        const float sc = fast_exp2((m - gm) * kLog2e);
+        const float dt = (m - gm) * kLog2e;  // t shifts by dt for every earlier term
+        t2 = make_float2(sc * (t2.x + dt * s2.x), sc * (t2.y + dt * s2.y));
+        s2 = make_float2(sc * s2.x, sc * s2.y);
+      }
+      m = gm;
+      g_best = g0;
+    }
+    // t = (x - m) log2 e with the subtraction first, so the maximum's own term is exactly 2^0
+    const float2 l2 = make_float2(kLog2e, kLog2e);
+    const float2 nm2 = make_float2(-m, -m);
+    if (full) {
+#pragma unroll
+      for (int l = 0; l < kLoads; ++l) {
+        float v[kVec];
+        to_f32x8<T>(raw[l], v);
+#pragma unroll
+        for (int j = 0; j < kVec; j += 2) {
+          const float2 t = fmul2(fadd2(make_float2(v[j], v[j + 1]), nm2), l2);
+          const float2 e = make_float2(fast_exp2(t.x), fast_exp2(t.y));
+          s2 = fadd2(s2, e);
+          t2 = ffma2(e, t, t2);
+        }
+      }
+    } else {  // ragged end of the row: -inf padding contributes nothing (and no 0 * -inf)
+#pragma unroll
+      for (int l = 0; l < kLoads; ++l) {
+        float v[kVec];
+        to_f32x8<T>(raw[l], v);
+#pragma unroll
+        for (int j = 0; j < kVec; ++j)
+          if (v[j] != -INFINITY) {
+            const float t = (v[j] - m) * kLog2e;
+            const float e = fast_exp2(t);
+            s2.x += e;
+            t2.x = fmaf(e, t, t2.x);
+          }
+      }
+    }
+  }
+  float s = s2.x + s2.y, u = (t2.x + t2.y) * (1.0f / kLog2e);
+  // CTA maximum, then the first column holding it (re-read the recorded group)
+  float bm = m;
+  for (int o = 16; o > 0; o >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
+  const int warp = tid >> 5;
+  __shared__ float wmax[8];
+  if (lane_id() == 0) wmax[warp] = bm;
+  __syncthreads();
+  bm = wmax[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) bm = fmaxf(bm, wmax[w]);
+  int a = 0x7fffffff;
+  if (m == bm && g_best >= 0) {
+#pragma unroll
+    for (int l = kLoads - 1; l >= 0; --l) {
+      const int c = g_best + (l * 256 + tid) * kVec;
+      if (c < c1) {
+        const uint4 raw = __ldcg(reinterpret_cast<const uint4*>(base + c));
+        float v[kVec];
+        to_f32x8<T>(raw, v);
+#pragma unroll
+        for (int j = kVec - 1; j >= 0; --j)
+          if (v[j] == bm) a = c + j;
+      }
+    }
+  }
+  // merge (m, S, U) over the CTA: warp shuffles, then the 8 warp results
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+    const float ss = __shfl_xor_sync(0xffffffffu, s, o);
+    const float uu = __shfl_xor_sync(0xffffffffu, u, o);
+    const int a2 = __shfl_xor_sync(0xffffffffu, a, o);
+    stat_merge_f32(m, s, u, a, m2, ss, uu, a2);
+  }
+  if (lane_id() == 0) red[warp] = StatD{m, s, u, a};
+  __syncthreads();
+  StatPartial r{-INFINITY, 0.f, 0.f, 0x7fffffff};
+  if (tid == 0) {
+    float rm = static_cast<float>(red[0].m), rs = static_cast<float>(red[0].s);
+    float ru = static_cast<float>(red[0].u);
+    int ra = red[0].a;
+    for (int w = 1; w < 8; ++w)
+      stat_merge_f32(rm, rs, ru, ra, static_cast<float>(red[w].m), static_cast<float>(red[w].s),
+                     static_cast<float>(red[w].u), red[w].a);
+    r = StatPartial{rm, rs, ru, ra};
+  }
+  __syncthreads();  // red is reused by the caller
+  return r;
+}
+
+// Statistics, merge and stop test in one launch: grid = (chunks, rows), chunk columns per CTA
+// streamed in groups.  Each CTA writes its slice's partial; the last CTA of a row (per-row ticket)
+// merges the row; the last row runs the stop test.  row_ticket [rows] starts and ends at zero.
+template <typename T, int kLoads>
 __global__ void __launch_bounds__(256) sampler_fused_kernel(const T* __restrict__ logits,
                                                             int32_t chunk, SamplerArgs p,
                                                             int32_t* __restrict__ row_ticket) {
+  pdl_enter();
   if (block_done(p.state + kStDone)) return;
-  __shared__ float sm_f[16];
-  __shared__ int sm_i[8];
+  __shared__ StatD red[256];
   __shared__ int last_chunk;
   const int row = blockIdx.y;
   const int c0 = blockIdx.x * chunk;
-  float v[kPerThread];
-  const bool full = load_slice<T, kPerThread>(logits + static_cast<size_t>(row) * p.vocab, c0,
-                                              min(c0 + chunk, p.vocab), v);
-  const StatPartial r = slice_stats<kPerThread, 16 / sizeof(T)>(v, c0, full, sm_f, sm_i);
+  const StatPartial r = stream_slice_stats<T, kLoads>(
+      logits + static_cast<size_t>(row) * p.vocab, c0, min(c0 + chunk, p.vocab), red);
   if (threadIdx.x == 0) {
     const_cast<StatPartial*>(p.partials)[static_cast<size_t>(row) * p.nsplit + blockIdx.x] = r;
     __threadfence();
