@@ -19,6 +19,7 @@
 #include "dg_common.cuh"
 #include "fp32_path.cuh"
 #include "gemm.cuh"
+#include "gemm_cluster.cuh"
 #include "layer.cuh"
 #include "sampler.cuh"
 
@@ -136,6 +137,16 @@ int num_sms() {
   return n;
 }
 
+// Resident 256-thread CTAs of a kernel on the whole GPU (its persistent grid size).
+template <typename K>
+int resident_ctas(K kernel) {
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, 256, 0) != cudaSuccess ||
+      per_sm < 1)
+    per_sm = 1;
+  return per_sm * num_sms();
+}
+
 template <typename K>
 int set_smem(K kernel, int bytes) {
   DG_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
@@ -164,7 +175,6 @@ int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cud
 }
 
 // ---- GEMM launch helpers -----------------------------------------------------------------
-constexpr int kDenseN = 256, kDenseStages = 4;
 constexpr int kGroupN = 64, kGroupStages = 8;
 
 // ta2/tb2 are read only by items of the alternate group (p.alt_group >= 0).
@@ -184,26 +194,52 @@ int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& 
   return DG_OK;
 }
 
-GemmParams dense_params(int m_rows, int n_tokens, int k_dim, int k_splits, int* err,
-                        const int* done) {
-  GemmParams p{};
-  p.alt_group = -1;
+// Split-K projection with the K splits of each tile in one cluster: grid m_tiles x n_chunks x S.
+template <int EPI>
+int launch_cluster(const CUtensorMap& ta, const CUtensorMap& tb, const CluParams& p,
+                   cudaStream_t st, int kind) {
+  auto k = gemm_cluster_kernel<EPI>;
+  DG_TRY(set_smem(k, kCluSmemBytes));
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(p.m_tiles * p.n_chunks * p.splits);
+  cfg.blockDim = dim3(kCluThreads);
+  cfg.dynamicSmemBytes = kCluSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = p.splits;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  prof_before(kind, st);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, k, ta, tb, p);
+  if (e != cudaSuccess) return fail(DG_ERR_CUDA, "cluster launch failed: %s", cudaGetErrorString(e));
+  DG_LAUNCHED();
+  prof_after(kind, st);
+  return DG_OK;
+}
+
+// Shape part of the cluster projection parameters: `m_rows` weight rows, `n` tokens, K = 64 kb.
+CluParams clu_params(int m_rows, int n, int kb, int splits, int* err, const int* done) {
+  CluParams p{};
+  p.n_tokens = n;
+  p.n_chunks = cdiv(n, 256);
   p.m_tiles = cdiv(m_rows, 128);
-  p.k_splits = k_splits;
-  p.n_chunk = kDenseN;
-  p.n_total = n_tokens;
-  p.n_chunks = cdiv(n_tokens, kDenseN);
-  p.kb_total = k_dim / 64;
-  p.m_valid = m_rows;
+  p.m_rows = m_rows;
+  p.kb_total = kb;
+  p.splits = std::max(1, std::min(splits, kb));
   p.err = err;
   p.done = done;
   return p;
 }
 
-int pick_splits(int m_tiles, int kb_total, int sms) {
-  int s = std::max(1, sms / std::max(1, m_tiles));
-  s = std::min(s, std::max(1, kb_total / 2));
-  return std::min(s, 16);
+// Cluster size (K splits) of a split-K projection with `tiles` weight x token tiles: enough CTAs
+// to cover the SMs, at most kCluMaxSplits and at most one 64-wide K slab per split.
+int clu_splits(int tiles, int kb_total, int sms) {
+  return std::max(1, std::min({kCluMaxSplits, kb_total, sms / std::max(1, tiles)}));
 }
 
 }  // namespace
@@ -237,9 +273,9 @@ struct dg_ctx {
   float2* ml_part;
   void* o;
   float* router_logits;
-  int32_t *topk_ids, *offsets, *perm, *item_counts;
+  int32_t *topk_ids, *offsets, *perm, *n_chunks, *route_ticket;
   float* topk_w;
-  int4 *items_gu, *items_d;
+  int4* chunks;  // routed token chunks of the grouped GEMMs
   void *x_perm, *h, *hs;
   float *y_slot, *y_shared;
   StatPartial* lm_part;
@@ -280,6 +316,8 @@ int check_config(const dg_config* c) {
     if (c->head_dim != 128) return fail(DG_ERR_UNSUPPORTED, "bf16 path needs head_dim 128");
     if (c->d_model % 64 || c->expert_hidden % 64 || c->shared_hidden % 64)
       return fail(DG_ERR_UNSUPPORTED, "bf16 path needs d, h, hs multiples of 64");
+    if (c->n_experts > 128 || c->d_model < 128)
+      return fail(DG_ERR_UNSUPPORTED, "bf16 path needs E <= 128 and d >= 128 (one router tile)");
     if (c->vocab % 256) return fail(DG_ERR_UNSUPPORTED, "bf16 path needs vocab % 256 == 0");
   } else if (c->dtype == DG_DTYPE_FP32) {
     if (c->head_dim > 128) return fail(DG_ERR_UNSUPPORTED, "fp32 path needs head_dim <= 128");
@@ -299,14 +337,14 @@ struct Plan {
 
 enum Buf {
   B_CANVAS, B_ARGMAX, B_PREV, B_LOCKED, B_STATE, B_TICKET, B_ERR, B_ENT, B_CONF, B_ROWH, B_X,
-  B_XN, B_PART, B_Q, B_OPART, B_ML, B_O, B_RLOG, B_IDS, B_W, B_OFF, B_PERM, B_ITEMS_GU,
-  B_ITEMS_D, B_ICNT, B_XPERM, B_H, B_HS, B_YSLOT, B_YSH, B_LMPART, B_LOGITS, B_ROPE, B_END
+  B_XN, B_PART, B_Q, B_OPART, B_ML, B_O, B_RLOG, B_IDS, B_W, B_OFF, B_PERM, B_CHUNKS,
+  B_NCHUNKS, B_RTICKET, B_XPERM, B_H, B_HS, B_YSLOT, B_YSH, B_LMPART, B_LOGITS, B_ROPE, B_END
 };
 
 struct Derived {
   int tq, qkv_rows, split_qkv, split_o, split_r, att_splits, esz;
   size_t part_elems;
-  long long max_items_gu, max_items_d;
+  long long max_chunks;
 };
 
 Derived derive(const dg_config& c, int sms) {
@@ -315,25 +353,23 @@ Derived derive(const dg_config& c, int sms) {
   d.esz = bf16 ? 2 : 4;
   d.tq = bf16 ? 256 : c.canvas;
   d.qkv_rows = (c.n_heads + 2 * c.n_kv_heads) * c.head_dim;
+  const long long T = c.canvas;
   if (bf16) {
-    d.split_qkv = pick_splits(cdiv(d.qkv_rows, 128), c.d_model / 64, sms);
-    d.split_o = pick_splits(cdiv(c.d_model, 128), c.n_heads * c.head_dim / 64, sms);
-    d.split_r = std::min(16, std::max(1, c.d_model / 64 / 4));
+    // cluster sizes of the split-K projections (their partials never leave the cluster)
+    d.split_qkv = clu_splits(cdiv(d.qkv_rows, 128), c.d_model / 64, sms);
+    d.split_o = clu_splits(cdiv(c.d_model, 128), c.n_heads * c.head_dim / 64, sms);
+    d.split_r = std::min(kCluMaxSplits, c.d_model / 64);
+    d.part_elems = 1;
   } else {
     d.split_qkv = d.split_o = d.split_r = 1;
+    d.part_elems = std::max({static_cast<size_t>(T) * d.qkv_rows,
+                             static_cast<size_t>(T) * c.d_model,
+                             static_cast<size_t>(T) * c.n_experts});
   }
-  const long long T = c.canvas;
-  size_t pe = std::max({static_cast<size_t>(d.split_qkv) * T * d.qkv_rows,
-                        static_cast<size_t>(d.split_o) * T * c.d_model,
-                        static_cast<size_t>(d.split_r) * T * c.n_experts});
-  d.part_elems = pe;
   const int group = c.n_heads / c.n_kv_heads;
   const int m_tiles = group * d.tq / 128;
   d.att_splits = std::max(1, std::min(16, sms / std::max(1, m_tiles * c.n_kv_heads)));
-  const long long chunks = c.n_experts + (T * c.top_k + kGroupN - 1) / kGroupN;
-  const long long sh_chunks = c.shared_hidden > 0 ? (T + kGroupN - 1) / kGroupN : 0;
-  d.max_items_gu = chunks * cdiv(2 * c.expert_hidden, 128) + sh_chunks * cdiv(2 * c.shared_hidden, 128);
-  d.max_items_d = (chunks + sh_chunks) * cdiv(c.d_model, 128);
+  d.max_chunks = c.n_experts + (T * c.top_k + kGroupN - 1) / kGroupN;
   return d;
 }
 
@@ -361,9 +397,9 @@ Plan plan(const dg_config& c, int sms) {
   sz[B_IDS] = sz[B_W] = T * k * 4;
   sz[B_OFF] = (E + 1) * 4;
   sz[B_PERM] = T * k * 4;
-  sz[B_ITEMS_GU] = bf16 ? dv.max_items_gu * 16 : 0;
-  sz[B_ITEMS_D] = bf16 ? dv.max_items_d * 16 : 0;
-  sz[B_ICNT] = 8;
+  sz[B_CHUNKS] = bf16 ? dv.max_chunks * 16 : 0;
+  sz[B_NCHUNKS] = 4;
+  sz[B_RTICKET] = 4;
   sz[B_XPERM] = bf16 ? T * k * d * es : 0;
   sz[B_H] = bf16 ? T * k * c.expert_hidden * es : 0;
   sz[B_HS] = bf16 ? T * std::max<size_t>(1, c.shared_hidden) * es : 0;
@@ -492,18 +528,20 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
   }
   // ---------------- bf16 tcgen05 path ----------------
   if (parts & 1) {
-  // QKV projection, split-K partials [split][token][row]
+  // QKV projection (cluster split-K) with RoPE, Q and the K / V^T cache writes in its epilogue
   {
-    GemmParams p = dense_params(c->qkv_rows, n, d, c->split_qkv, c->err, done);
-    p.out_f32 = c->part;
-    p.ld_out = c->qkv_rows;
-    p.split_stride = static_cast<long long>(n) * c->qkv_rows;
-    const int items = p.m_tiles * p.k_splits * p.n_chunks;
-    DG_TRY((launch_gemm<kDenseN, kDenseStages, kEpiPartialF32>(c->tm_wqkv[l], c->tm_xn32, p,
-                                                                 std::min(items, c->sms), st,
-                                                                 DG_KERNEL_QKV)));
-    DG_TRY(layer_tail_common<__nv_bfloat16>(c, l, n, pos0, done, st, p.split_stride,
-                                            c->split_qkv));
+    const size_t kv_head_elems = static_cast<size_t>(g.kv_capacity) * hd;
+    CluParams p = clu_params(c->qkv_rows, n, d / 64, c->split_qkv, c->err, done);
+    p.n_heads = g.n_heads;
+    p.n_kv_heads = g.n_kv_heads;
+    p.tq = c->tq;
+    p.pos0 = pos0;
+    p.ldk = g.kv_capacity;
+    p.rope_tab = c->rope_tab;
+    p.q = static_cast<__nv_bfloat16*>(c->q);
+    p.k_cache = static_cast<__nv_bfloat16*>(c->kc) + static_cast<size_t>(l) * g.n_kv_heads * kv_head_elems;
+    p.vt_cache = static_cast<__nv_bfloat16*>(c->vtc) + static_cast<size_t>(l) * g.n_kv_heads * kv_head_elems;
+    DG_TRY(launch_cluster<kCluQkv>(c->tm_wqkv[l], c->tm_xn32, p, st, DG_KERNEL_QKV));
   }
   // attention over [cache 0..pos0 | new tokens], split over keys
   {
@@ -544,64 +582,34 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     DG_LAUNCHED();
     prof_after(DG_KERNEL_ATTN_COMBINE, st);
   }
-  // O projection + residual + ffn norm
+  // O projection onto the residual stream (cluster split-K), then the ffn norm
   {
-    GemmParams p = dense_params(d, n, g.n_heads * hd, c->split_o, c->err, done);
-    p.out_f32 = c->part;
-    p.ld_out = d;
-    p.split_stride = static_cast<long long>(n) * d;
-    const int items = p.m_tiles * p.k_splits * p.n_chunks;
-    DG_TRY((launch_gemm<kDenseN, kDenseStages, kEpiPartialF32>(c->tm_wo[l], c->tm_o32, p,
-                                                                 std::min(items, c->sms), st,
-                                                                 DG_KERNEL_O_PROJ)));
+    CluParams p = clu_params(d, n, g.n_heads * hd / 64, c->split_o, c->err, done);
+    p.x = c->x;
+    DG_TRY(launch_cluster<kCluResidual>(c->tm_wo[l], c->tm_o32, p, st, DG_KERNEL_O_PROJ));
     prof_before(DG_KERNEL_RESIDUAL_NORM, st);
-    DG_TRY(launch_pdl(residual_norm_kernel<__nv_bfloat16>, dim3(n), dim3(256), 0, st, 
-        c->x, c->part, c->split_o, p.split_stride, d, w.ffn_norm, g.eps,
-        static_cast<__nv_bfloat16*>(c->xn), done));
+    DG_TRY(launch_pdl(residual_norm_kernel<__nv_bfloat16>, dim3(n), dim3(256), 0, st,
+                      c->x, c->part, 0, 0ll, d, w.ffn_norm, g.eps,
+                      static_cast<__nv_bfloat16*>(c->xn), done));
     DG_LAUNCHED();
     prof_after(DG_KERNEL_RESIDUAL_NORM, st);
   }
   }
   if (!(parts & 2)) return DG_OK;
-  // router + top-k
-  {
-    GemmParams p = dense_params(E, n, d, c->split_r, c->err, done);
-    p.out_f32 = c->part;
-    p.ld_out = E;
-    p.split_stride = static_cast<long long>(n) * E;
-    const int items = p.m_tiles * p.k_splits * p.n_chunks;
-    DG_TRY((launch_gemm<kDenseN, kDenseStages, kEpiPartialF32>(c->tm_wr[l], c->tm_xn32, p,
-                                                                 std::min(items, c->sms), st,
-                                                                 DG_KERNEL_ROUTER)));
-    prof_before(DG_KERNEL_ROUTER_TOPK, st);
-    DG_TRY(launch_pdl(router_topk_kernel, dim3(cdiv(n, 4)), dim3(128), 0, st, c->part, c->split_r, p.split_stride, n, E, k,
-                                                   c->router_logits, c->topk_ids, c->topk_w, done));
-    DG_LAUNCHED();
-    prof_after(DG_KERNEL_ROUTER_TOPK, st);
-  }
-  // permutation and grouped expert GEMMs; the shared expert rides along as group E
+  // router (cluster split-K) with top-k in its epilogue; the grid's last CTA routes the canvas
   const bool shared = g.shared_hidden > 0;
   {
-    RouteArgs ra{};
-    ra.ids = c->topk_ids;
-    ra.n_slots = n_slots;
-    ra.n_experts = E;
-    ra.offsets = c->offsets;
-    ra.perm = c->perm;
-    ra.items_gu = c->items_gu;
-    ra.items_d = c->items_d;
-    ra.counts = c->item_counts;
-    ra.m_tiles_gu = cdiv(2 * g.expert_hidden, 128);
-    ra.m_tiles_d = cdiv(d, 128);
-    ra.n_chunk = kGroupN;
-    ra.n_tokens = n;
-    ra.shared_m_tiles_gu = shared ? cdiv(2 * g.shared_hidden, 128) : 0;
-    ra.shared_m_tiles_d = shared ? cdiv(d, 128) : 0;
-    ra.done = done;
-    prof_before(DG_KERNEL_ROUTE, st);
-    DG_TRY(launch_pdl(moe_route_kernel, dim3(1), dim3(1024), 0, st, ra));
-    DG_LAUNCHED();
-    prof_after(DG_KERNEL_ROUTE, st);
+    CluParams p = clu_params(E, n, d / 64, c->split_r, c->err, done);
+    p.router_logits = c->router_logits;
+    p.ids = c->topk_ids;
+    p.wts = c->topk_w;
+    p.top_k = k;
+    p.route = RouteArgs{c->topk_ids, n, k, E, kGroupN, c->offsets, c->perm, c->chunks, c->n_chunks};
+    p.ticket = c->route_ticket;
+    DG_TRY(launch_cluster<kCluRouter>(c->tm_wr[l], c->tm_xn32, p, st, DG_KERNEL_ROUTER));
+  }
+  // permutation gather and grouped expert GEMMs; the shared expert rides along as group E
+  {
     prof_before(DG_KERNEL_GATHER, st);
     DG_TRY(launch_pdl(gather_rows_kernel, dim3(cdiv(n_slots, 4)), dim3(256), 0, st, 
         static_cast<const __nv_bfloat16*>(c->xn), c->perm, k, d, n_slots,
@@ -609,8 +617,13 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     DG_LAUNCHED();
     prof_after(DG_KERNEL_GATHER, st);
     GemmParams p{};
-    p.items = c->items_gu;
-    p.item_count = c->item_counts;
+    p.chunks = c->chunks;
+    p.chunk_count = c->n_chunks;
+    p.m_tiles = cdiv(2 * g.expert_hidden, 128);
+    p.n_chunk = kGroupN;
+    p.alt_m_tiles = cdiv(2 * g.shared_hidden, 128);
+    p.alt_chunks = cdiv(n, kGroupN);
+    p.alt_tokens = n;
     p.a_rows_per_group = 2 * g.expert_hidden;
     p.kb_total = d / 64;
     p.m_valid = 2 * g.expert_hidden;
@@ -627,8 +640,13 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
         c->tm_wgu[l], c->tm_xperm, p, c->sms, st, DG_KERNEL_EXPERT_GATE_UP,
         shared ? &c->tm_wsgu[l] : nullptr, shared ? &c->tm_xn32 : nullptr)));
     GemmParams q{};
-    q.items = c->items_d;
-    q.item_count = c->item_counts + 1;
+    q.chunks = c->chunks;
+    q.chunk_count = c->n_chunks;
+    q.m_tiles = cdiv(d, 128);
+    q.n_chunk = kGroupN;
+    q.alt_m_tiles = cdiv(d, 128);
+    q.alt_chunks = cdiv(n, kGroupN);
+    q.alt_tokens = n;
     q.a_rows_per_group = d;
     q.kb_total = g.expert_hidden / 64;
     q.m_valid = d;
@@ -841,9 +859,9 @@ int dg_create(const dg_config* cfg, const dg_weights* w, void* d_kv, void* d_scr
   c->topk_w = reinterpret_cast<float*>(s + p.off[B_W]);
   c->offsets = reinterpret_cast<int32_t*>(s + p.off[B_OFF]);
   c->perm = reinterpret_cast<int32_t*>(s + p.off[B_PERM]);
-  c->items_gu = reinterpret_cast<int4*>(s + p.off[B_ITEMS_GU]);
-  c->items_d = reinterpret_cast<int4*>(s + p.off[B_ITEMS_D]);
-  c->item_counts = reinterpret_cast<int32_t*>(s + p.off[B_ICNT]);
+  c->chunks = reinterpret_cast<int4*>(s + p.off[B_CHUNKS]);
+  c->n_chunks = reinterpret_cast<int32_t*>(s + p.off[B_NCHUNKS]);
+  c->route_ticket = reinterpret_cast<int32_t*>(s + p.off[B_RTICKET]);
   c->x_perm = s + p.off[B_XPERM];
   c->h = s + p.off[B_H];
   c->hs = s + p.off[B_HS];
@@ -1084,28 +1102,34 @@ int dg_debug_layer(dg_ctx* ctx, int32_t layer, const float* d_x_in, float* d_x_o
 
 // ---- standalone sampler ----------------------------------------------------------------
 
+// The streaming sampler cuts rows into segments of kSamplerSpan columns (both dtypes).
+constexpr int kSamplerSpan = 8192;
+
 int dg_sampler_workspace_bytes(int32_t rows, int32_t vocab, size_t* bytes) {
   if (rows < 1 || rows > 1024 || vocab < 2 || vocab % 8 || !bytes)
     return fail(DG_ERR_INVALID_ARG, "need 1 <= rows <= 1024, vocab % 8 == 0");
-  const size_t nchunk = cdiv(vocab, 4096);  // upper bound over both dtypes
-  *bytes = align256(rows * nchunk * sizeof(StatPartial)) + 4 * align256(rows * 8) + 256;
+  const size_t segs = cdiv(vocab, kSamplerSpan);
+  *bytes = align256(rows * segs * sizeof(StatPartial)) + align256(rows * segs * 4) +
+           4 * align256(rows * 8) + 256;
   return DG_OK;
 }
 
-static void sampler_views(void* ws, int rows, int vocab, StatPartial** part, int32_t** prev,
-                          double** row_h, int32_t** locked, int32_t** ticket,
-                          int32_t** row_ticket) {
+static void sampler_views(void* ws, int rows, int vocab, StatPartial** part, int32_t** piece_len,
+                          int32_t** prev, double** row_h, int32_t** locked, int32_t** ticket,
+                          int32_t** row_units) {
   uint8_t* b = static_cast<uint8_t*>(ws);
-  const size_t nchunk = cdiv(vocab, 4096);
+  const size_t segs = cdiv(vocab, kSamplerSpan);
   *part = reinterpret_cast<StatPartial*>(b);
-  b += align256(rows * nchunk * sizeof(StatPartial));
+  b += align256(rows * segs * sizeof(StatPartial));
+  *piece_len = reinterpret_cast<int32_t*>(b);
+  b += align256(rows * segs * 4);
   *prev = reinterpret_cast<int32_t*>(b);
   b += align256(rows * 8);
   *row_h = reinterpret_cast<double*>(b);
   b += align256(rows * 8);
   *locked = reinterpret_cast<int32_t*>(b);
   b += align256(rows * 8);
-  *row_ticket = reinterpret_cast<int32_t*>(b);
+  *row_units = reinterpret_cast<int32_t*>(b);
   b += align256(rows * 8);
   *ticket = reinterpret_cast<int32_t*>(b);
 }
@@ -1135,16 +1159,15 @@ int dg_sampler_step(const void* d_logits, int32_t dtype, int32_t rows, int32_t v
   if (dtype != DG_DTYPE_BF16 && dtype != DG_DTYPE_FP32)
     return fail(DG_ERR_INVALID_ARG, "dtype must be bf16 or fp32");
   StatPartial* part;
-  int32_t *prev, *locked, *ticket, *row_ticket;
+  int32_t *piece_len, *prev, *locked, *ticket, *row_units;
   double* row_h;
-  sampler_views(d_workspace, rows, vocab, &part, &prev, &row_h, &locked, &ticket, &row_ticket);
+  sampler_views(d_workspace, rows, vocab, &part, &piece_len, &prev, &row_h, &locked, &ticket,
+                &row_units);
   cudaStream_t st = S(stream);
-  // row slices of 65536 columns (eight 32-value groups per thread)
-  const int chunk = 65536;
-  const int nchunk = cdiv(vocab, chunk);
+  const int segs = cdiv(vocab, kSamplerSpan);
   SamplerArgs a{};
   a.partials = part;
-  a.nsplit = nchunk;
+  a.nsplit = segs;
   a.rows = rows;
   a.vocab = vocab;
   a.seed = seed;
@@ -1163,13 +1186,18 @@ int dg_sampler_step(const void* d_logits, int32_t dtype, int32_t rows, int32_t v
   a.locked = locked;
   a.state = d_state;
   a.ticket = ticket;
+  // one wave of resident CTAs, each streaming an equal run of segments
+  static const int grid_bf16 = resident_ctas(sampler_stream_kernel<__nv_bfloat16, 4>);
+  static const int grid_f32 = resident_ctas(sampler_stream_kernel<float, 8>);
+  const long long units = static_cast<long long>(rows) * segs;
+  const int grid = static_cast<int>(std::min<long long>(units, dtype == DG_DTYPE_BF16 ? grid_bf16 : grid_f32));
   prof_before(DG_KERNEL_SAMPLER, st);
   if (dtype == DG_DTYPE_BF16)
-    DG_TRY(launch_pdl(sampler_fused_kernel<__nv_bfloat16, 4>, dim3(nchunk, rows), dim3(256), 0, st, 
-        static_cast<const __nv_bfloat16*>(d_logits), chunk, a, row_ticket));
+    DG_TRY(launch_pdl(sampler_stream_kernel<__nv_bfloat16, 4>, dim3(grid), dim3(256), 0, st,
+                      static_cast<const __nv_bfloat16*>(d_logits), segs, a, row_units, piece_len));
   else
-    DG_TRY(launch_pdl(sampler_fused_kernel<float, 8>, dim3(nchunk, rows), dim3(256), 0, st, 
-        static_cast<const float*>(d_logits), chunk, a, row_ticket));
+    DG_TRY(launch_pdl(sampler_stream_kernel<float, 8>, dim3(grid), dim3(256), 0, st,
+                      static_cast<const float*>(d_logits), segs, a, row_units, piece_len));
   DG_LAUNCHED();
   prof_after(DG_KERNEL_SAMPLER, st);
   return DG_OK;
@@ -1251,24 +1279,21 @@ struct MoePlan {
   size_t off[12];
   size_t total;
   int split_r;
-  long long items_gu, items_d;
+  long long chunks;
 };
 MoePlan moe_plan(int t, int d, int E, int k, int hid, int hs) {
   MoePlan m{};
-  m.split_r = std::min(16, std::max(1, d / 64 / 4));
-  const long long chunks = E + (static_cast<long long>(t) * k + kGroupN - 1) / kGroupN;
-  const long long sh_chunks = hs > 0 ? (t + kGroupN - 1) / kGroupN : 0;
-  m.items_gu = chunks * cdiv(2 * hid, 128) + sh_chunks * cdiv(2 * hs, 128);
-  m.items_d = (chunks + sh_chunks) * cdiv(d, 128);
+  m.split_r = std::min(kCluMaxSplits, d / 64);
+  m.chunks = E + (static_cast<long long>(t) * k + kGroupN - 1) / kGroupN;
   size_t sz[12];
-  sz[0] = static_cast<size_t>(m.split_r) * t * E * 4;  // router partials
+  sz[0] = static_cast<size_t>(t) * E * 4;              // router logits (internal)
   sz[1] = static_cast<size_t>(t) * k * 4;              // ids (internal)
   sz[2] = static_cast<size_t>(t) * k * 4;              // weights (internal)
   sz[3] = (E + 1) * 4;                                 // offsets
   sz[4] = static_cast<size_t>(t) * k * 4;              // perm
-  sz[5] = m.items_gu * 16;
-  sz[6] = m.items_d * 16;
-  sz[7] = 16;                                          // item counts + error word
+  sz[5] = m.chunks * 16;                               // routed token chunks
+  sz[6] = 0;                                           // (unused)
+  sz[7] = 16;                                          // chunk count, -, error word, route ticket
   sz[8] = static_cast<size_t>(t) * k * d * 2;          // x_perm
   sz[9] = static_cast<size_t>(t) * k * hid * 2;        // h
   sz[10] = align256(static_cast<size_t>(t) * std::max(hs, 1) * 2) +
@@ -1286,7 +1311,7 @@ MoePlan moe_plan(int t, int d, int E, int k, int hid, int hs) {
 
 int dg_moe_workspace_bytes(int32_t t, int32_t d, int32_t n_experts, int32_t top_k, int32_t hidden,
                            int32_t shared_hidden, size_t* bytes) {
-  if (t < 1 || d < 64 || d % 64 || d > 4096 || n_experts < 4 || n_experts % 4 || n_experts > 256 ||
+  if (t < 1 || d < 128 || d % 64 || d > 4096 || n_experts < 4 || n_experts % 4 || n_experts > 128 ||
       top_k < 1 || top_k > 8 ||
       top_k > n_experts || hidden < 64 || hidden % 64 || shared_hidden < 0 || shared_hidden % 64 ||
       !bytes)
@@ -1310,15 +1335,15 @@ int dg_moe_ffn(const void* d_x, const float* d_residual, const void* d_wr, const
   if (t > 4096) return fail(DG_ERR_UNSUPPORTED, "at most 4096 tokens per call");
   const MoePlan m = moe_plan(t, d, n_experts, top_k, hidden, shared_hidden);
   uint8_t* ws = static_cast<uint8_t*>(d_workspace);
-  float* rpart = reinterpret_cast<float*>(ws + m.off[0]);
+  float* rlog = reinterpret_cast<float*>(ws + m.off[0]);
   int32_t* ids = reinterpret_cast<int32_t*>(ws + m.off[1]);
   float* wts = reinterpret_cast<float*>(ws + m.off[2]);
   int32_t* offs = reinterpret_cast<int32_t*>(ws + m.off[3]);
   int32_t* perm = reinterpret_cast<int32_t*>(ws + m.off[4]);
-  int4* items_gu = reinterpret_cast<int4*>(ws + m.off[5]);
-  int4* items_d = reinterpret_cast<int4*>(ws + m.off[6]);
+  int4* chunks = reinterpret_cast<int4*>(ws + m.off[5]);
   int32_t* icnt = reinterpret_cast<int32_t*>(ws + m.off[7]);
   int* err = icnt + 2;
+  int32_t* route_ticket = icnt + 3;
   __nv_bfloat16* x_perm = reinterpret_cast<__nv_bfloat16*>(ws + m.off[8]);
   __nv_bfloat16* hbuf = reinterpret_cast<__nv_bfloat16*>(ws + m.off[9]);
   __nv_bfloat16* hsbuf = reinterpret_cast<__nv_bfloat16*>(ws + m.off[10]);
@@ -1326,7 +1351,7 @@ int dg_moe_ffn(const void* d_x, const float* d_residual, const void* d_wr, const
   float* y_slot = reinterpret_cast<float*>(ws + m.off[11]);
   const int sms = num_sms();
   cudaStream_t st = S(stream);
-  DG_CUDA(cudaMemsetAsync(err, 0, 4, st));
+  DG_CUDA(cudaMemsetAsync(err, 0, 8, st));  // error word and route ticket
   CUtensorMap t_x32, t_wr, t_xp, t_wgu, t_h, t_wd, t_wsgu, t_hs, t_wsd;
   DG_TRY(make_tmap(&t_x32, d_x, t, d, d, 32));
   DG_TRY(make_tmap(&t_wr, d_wr, n_experts, d, d, 128));
@@ -1340,40 +1365,26 @@ int dg_moe_ffn(const void* d_x, const float* d_residual, const void* d_wr, const
     DG_TRY(make_tmap(&t_wsd, d_ws_d, d, shared_hidden, shared_hidden, 128));
   }
   // router
-  GemmParams pr = dense_params(n_experts, t, d, m.split_r, err, nullptr);
-  pr.out_f32 = rpart;
-  pr.ld_out = n_experts;
-  pr.split_stride = static_cast<long long>(t) * n_experts;
-  DG_TRY((launch_gemm<kDenseN, kDenseStages, kEpiPartialF32>(
-      t_wr, t_x32, pr, std::min(pr.m_tiles * pr.k_splits * pr.n_chunks, sms), st)));
-  DG_TRY(launch_pdl(router_topk_kernel, dim3(cdiv(t, 4)), dim3(128), 0, st, rpart, m.split_r, pr.split_stride, t, n_experts,
-                                                 top_k, d_router_logits, ids, wts, nullptr));
-  DG_LAUNCHED();
   const bool shared = shared_hidden > 0;
-  RouteArgs ra{};
-  ra.ids = ids;
-  ra.n_slots = t * top_k;
-  ra.n_experts = n_experts;
-  ra.offsets = offs;
-  ra.perm = perm;
-  ra.items_gu = items_gu;
-  ra.items_d = items_d;
-  ra.counts = icnt;
-  ra.m_tiles_gu = cdiv(2 * hidden, 128);
-  ra.m_tiles_d = cdiv(d, 128);
-  ra.n_chunk = kGroupN;
-  ra.n_tokens = t;
-  ra.shared_m_tiles_gu = shared ? cdiv(2 * shared_hidden, 128) : 0;
-  ra.shared_m_tiles_d = shared ? cdiv(d, 128) : 0;
-  ra.done = nullptr;
-  DG_TRY(launch_pdl(moe_route_kernel, dim3(1), dim3(1024), 0, st, ra));
-  DG_LAUNCHED();
+  CluParams pr = clu_params(n_experts, t, d / 64, m.split_r, err, nullptr);
+  pr.router_logits = d_router_logits ? d_router_logits : rlog;
+  pr.ids = ids;
+  pr.wts = wts;
+  pr.top_k = top_k;
+  pr.route = RouteArgs{ids, t, top_k, n_experts, kGroupN, offs, perm, chunks, icnt};
+  pr.ticket = route_ticket;
+  DG_TRY(launch_cluster<kCluRouter>(t_wr, t_x32, pr, st, -1));
   DG_TRY(launch_pdl(gather_rows_kernel, dim3(cdiv(t * top_k, 4)), dim3(256), 0, st, static_cast<const __nv_bfloat16*>(d_x),
                                                          perm, top_k, d, t * top_k, x_perm, nullptr));
   DG_LAUNCHED();
   GemmParams pg{};
-  pg.items = items_gu;
-  pg.item_count = icnt;
+  pg.chunks = chunks;
+  pg.chunk_count = icnt;
+  pg.m_tiles = cdiv(2 * hidden, 128);
+  pg.n_chunk = kGroupN;
+  pg.alt_m_tiles = cdiv(2 * shared_hidden, 128);
+  pg.alt_chunks = cdiv(t, kGroupN);
+  pg.alt_tokens = t;
   pg.a_rows_per_group = 2 * hidden;
   pg.kb_total = d / 64;
   pg.m_valid = 2 * hidden;
@@ -1389,8 +1400,13 @@ int dg_moe_ffn(const void* d_x, const float* d_residual, const void* d_wr, const
                                                            shared ? &t_wsgu : nullptr,
                                                            shared ? &t_x32 : nullptr)));
   GemmParams pd{};
-  pd.items = items_d;
-  pd.item_count = icnt + 1;
+  pd.chunks = chunks;
+  pd.chunk_count = icnt;
+  pd.m_tiles = cdiv(d, 128);
+  pd.n_chunk = kGroupN;
+  pd.alt_m_tiles = cdiv(d, 128);
+  pd.alt_chunks = cdiv(t, kGroupN);
+  pd.alt_tokens = t;
   pd.a_rows_per_group = d;
   pd.kb_total = hidden / 64;
   pd.m_valid = d;

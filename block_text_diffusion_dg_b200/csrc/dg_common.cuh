@@ -327,6 +327,34 @@ DG_DEV float store_from_f32<float>(float x) { return x; }
 template <>
 DG_DEV __nv_bfloat16 store_from_f32<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
 
+// ---------------------------------------------------------------------------------------
+// Thread-block clusters: rank, a full cluster barrier (every thread of every CTA arrives; the
+// release / acquire pair orders shared and global memory across the cluster) and distributed
+// shared memory loads from a peer CTA's shared memory.
+DG_DEV uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+DG_DEV void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
+               ::: "memory");
+}
+// Address of the same shared-memory location in the CTA of the given cluster rank.
+DG_DEV uint32_t dsmem_addr(uint32_t local_addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_addr), "r"(rank));
+  return r;
+}
+DG_DEV float4 dsmem_ld4(uint32_t cluster_addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(cluster_addr)
+               : "memory");
+  return v;
+}
+
 // Programmatic dependent launch: wait until the previous grid in the stream has completed and
 // its writes are visible, then let the next grid start launching (it waits the same way).
 DG_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }

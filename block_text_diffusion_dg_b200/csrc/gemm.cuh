@@ -24,9 +24,11 @@ enum EpiMode : int { kEpiPartialF32 = 0, kEpiGluBf16 = 1, kEpiScatterF32 = 2 };
 struct GemmParams {
   // dense items: it -> (m tile, k split, n chunk)
   int m_tiles, k_splits, n_chunks, n_total, n_chunk, a_row_base, b_row_base;
-  // grouped items: device list of (group, m tile, first token row, n tokens)
-  const int4* items;
-  const int* item_count;
+  // grouped items (chunks != nullptr): the shared expert's (m tile, token chunk) pairs first,
+  // tile-major, then every routed chunk with each of the m_tiles weight tiles, chunk-major.
+  // chunks[c] = (expert, first permuted row, tokens, -), *chunk_count of them (device-built).
+  const int4* chunks;
+  const int* chunk_count;
   int a_rows_per_group;
   int kb_total;  // K / 64
   int m_valid;   // rows of A per group that are real (epilogue guard)
@@ -37,10 +39,13 @@ struct GemmParams {
   long long split_stride;
   const int* perm;
   const float* scale;
-  // alternate group (the shared expert folded into a grouped launch): items whose group id is
-  // alt_group read tm_a2 / tm_b2, run alt_kb_total K slabs and write alt_out_* (no permutation,
-  // weight 1)
+  // the shared expert folded into a grouped launch (alt_group >= 0): its items read tm_a2 /
+  // tm_b2 (rows of the unpermuted tokens), run alt_kb_total K slabs, write alt_out_* with no
+  // permutation and weight 1
   int alt_group;
+  int alt_m_tiles;   // weight tiles of the shared expert
+  int alt_chunks;    // token chunks of the shared expert (n_chunk tokens each)
+  int alt_tokens;
   int alt_kb_total;
   int alt_m_valid;
   float* alt_out_f32;
@@ -58,7 +63,8 @@ struct GemmItem {
 DG_DEV GemmItem gemm_item(const GemmParams& p, int it) {
   GemmItem w;
   w.alt = false;
-  if (p.items == nullptr) {
+  w.kb0 = 0;
+  if (p.chunks == nullptr) {
     const int mt = it % p.m_tiles;
     const int rest = it / p.m_tiles;
     const int split = rest % p.k_splits;
@@ -71,22 +77,35 @@ DG_DEV GemmItem gemm_item(const GemmParams& p, int it) {
     w.kb1 = (split + 1) * p.kb_total / p.k_splits;
     w.aux = split;
   } else {
-    const int4 e = p.items[it];
-    w.alt = e.x == p.alt_group;
-    w.r_base = e.y * 128;
-    w.a_row = (w.alt ? 0 : e.x * p.a_rows_per_group) + w.r_base;
-    w.b_row = e.z;
-    w.n = e.w;
-    w.kb0 = 0;
-    w.kb1 = w.alt ? p.alt_kb_total : p.kb_total;
-    w.aux = e.x;
+    const int sh_items = p.alt_group >= 0 ? p.alt_chunks * p.alt_m_tiles : 0;
+    if (it < sh_items) {  // consecutive items share a weight tile, which L2 then serves
+      const int m = it / p.alt_chunks, ch = it % p.alt_chunks;
+      w.alt = true;
+      w.r_base = m * 128;
+      w.a_row = w.r_base;
+      w.b_row = ch * p.n_chunk;
+      w.n = min(p.n_chunk, p.alt_tokens - ch * p.n_chunk);
+      w.kb1 = p.alt_kb_total;
+      w.aux = p.alt_group;
+    } else {
+      const int r = it - sh_items;
+      const int ch = r / p.m_tiles, m = r % p.m_tiles;
+      const int4 c = p.chunks[ch];
+      w.r_base = m * 128;
+      w.a_row = c.x * p.a_rows_per_group + w.r_base;
+      w.b_row = c.y;
+      w.n = c.z;
+      w.kb1 = p.kb_total;
+      w.aux = c.x;
+    }
   }
   return w;
 }
 
 DG_DEV int gemm_item_count(const GemmParams& p) {
-  return p.items ? *reinterpret_cast<const volatile int*>(p.item_count)
-                 : p.m_tiles * p.k_splits * p.n_chunks;
+  if (p.chunks == nullptr) return p.m_tiles * p.k_splits * p.n_chunks;
+  const int sh_items = p.alt_group >= 0 ? p.alt_chunks * p.alt_m_tiles : 0;
+  return sh_items + *reinterpret_cast<const volatile int*>(p.chunk_count) * p.m_tiles;
 }
 
 template <int MAXN, int STAGES>

@@ -182,33 +182,13 @@ __global__ void __launch_bounds__(256) residual_norm_kernel(float* __restrict__ 
   }
 }
 
-// One warp per token; E <= 256 and E % 4 == 0, k <= 8.  Lane l holds experts 4l..4l+3 and
-// 128+4l..128+4l+3.  Top-k by repeated warp argmax (largest logit, lowest index on ties); the
-// weights are the softmax of the selected logits.
-__global__ void router_topk_kernel(const float* __restrict__ part, int splits,
-                                   long long split_stride, int n_tokens, int n_experts, int top_k,
-                                   float* __restrict__ logits_out, int32_t* __restrict__ ids,
-                                   float* __restrict__ wts, const int* done) {
-  pdl_enter();
-  if (block_done(done)) return;
-  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (t >= n_tokens) return;
+// Top-k of one token's router logits held by one warp; E <= 256 and E % 4 == 0, k <= 8.  Lane
+// l holds experts 4l..4l+3 in v[0..3] and 128+4l..128+4l+3 in v[4..7] (-inf where e >= E).
+// Top-k by repeated warp argmax (largest logit, lowest index on ties); the weights are the
+// softmax of the selected logits.  Lane 0 writes ids_t[0..k) and wts_t[0..k).
+DG_DEV void router_topk_select(float (&v)[8], int n_experts, int top_k, int32_t* ids_t,
+                               float* wts_t) {
   const int lane = lane_id();
-  float v[8];
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int e0 = 128 * h + 4 * lane;
-    float4 a = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-    if (e0 < n_experts) {
-      a = sum_splits4(part, splits, split_stride, static_cast<long long>(t) * n_experts + e0);
-      if (logits_out)
-        *reinterpret_cast<float4*>(logits_out + static_cast<long long>(t) * n_experts + e0) = a;
-    }
-    v[4 * h] = a.x;
-    v[4 * h + 1] = a.y;
-    v[4 * h + 2] = a.z;
-    v[4 * h + 3] = a.w;
-  }
   float sel_v[8];
   int sel_i[8];
   for (int kk = 0; kk < top_k; ++kk) {
@@ -241,27 +221,65 @@ __global__ void router_topk_kernel(const float* __restrict__ part, int splits,
     float den = 0.f;
     for (int kk = 0; kk < top_k; ++kk) den += expf(sel_v[kk] - sel_v[0]);
     for (int kk = 0; kk < top_k; ++kk) {
-      ids[t * top_k + kk] = sel_i[kk];
-      wts[t * top_k + kk] = expf(sel_v[kk] - sel_v[0]) / den;
+      ids_t[kk] = sel_i[kk];
+      wts_t[kk] = expf(sel_v[kk] - sel_v[0]) / den;
     }
   }
 }
 
+// Top-k of token t from split-K partials of its router logits (summed in split order).
+DG_DEV void router_topk_token(const float* __restrict__ part, int splits, long long split_stride,
+                              int t, int n_experts, int top_k, float* __restrict__ logits_out,
+                              int32_t* __restrict__ ids, float* __restrict__ wts) {
+  const int lane = lane_id();
+  float v[8];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int e0 = 128 * h + 4 * lane;
+    float4 a = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+    if (e0 < n_experts) {
+      a = sum_splits4(part, splits, split_stride, static_cast<long long>(t) * n_experts + e0);
+      if (logits_out)
+        *reinterpret_cast<float4*>(logits_out + static_cast<long long>(t) * n_experts + e0) = a;
+    }
+    v[4 * h] = a.x;
+    v[4 * h + 1] = a.y;
+    v[4 * h + 2] = a.z;
+    v[4 * h + 3] = a.w;
+  }
+  router_topk_select(v, n_experts, top_k, ids + static_cast<long long>(t) * top_k,
+                     wts + static_cast<long long>(t) * top_k);
+}
+
+// One warp per token (the all-fp32 path, which needs no permutation).
+__global__ void router_topk_kernel(const float* __restrict__ part, int splits,
+                                   long long split_stride, int n_tokens, int n_experts, int top_k,
+                                   float* __restrict__ logits_out, int32_t* __restrict__ ids,
+                                   float* __restrict__ wts, const int* done) {
+  pdl_enter();
+  if (block_done(done)) return;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= n_tokens) return;
+  router_topk_token(part, splits, split_stride, t, n_experts, top_k, logits_out, ids, wts);
+}
+
 struct RouteArgs {
-  const int32_t* ids;  // [n_slots] expert of slot (token * k + s)
-  int n_slots, n_experts;
-  int32_t* offsets;  // [E + 1]
-  int32_t* perm;     // [n_slots] permuted row -> slot
-  int4* items_gu;    // grouped items for gate/up
-  int4* items_d;     // grouped items for down
-  int32_t* counts;   // [2]: item counts (gate/up, down)
-  int m_tiles_gu, m_tiles_d, n_chunk;
-  // shared expert folded in as group n_experts: n_tokens in chunks of n_chunk, listed first
-  int n_tokens, shared_m_tiles_gu, shared_m_tiles_d;  // 0 tiles: no shared expert
-  const int* done;
+  const int32_t* ids;  // [n_tokens * top_k] expert of slot (token * k + j)
+  int n_tokens, top_k, n_experts;
+  int n_chunk;         // tokens per grouped-GEMM chunk
+  int32_t* offsets;    // [E + 1] first permuted row of each expert
+  int32_t* perm;       // [n_slots] permuted row -> slot
+  int4* chunks;        // [max chunks] (expert, first permuted row, tokens, 0) in expert order
+  int32_t* n_chunks;   // [1] chunks in use
 };
 
-// Exclusive scan of up to 256 values by warp 0 (8 per lane); returns the total to all lanes.
+constexpr int kRouteMaxTokens = 4096;
+// Shared memory the routing needs (ints) for E experts and n tokens.
+__host__ __device__ constexpr int route_smem_ints(int n_experts, int n_tokens) {
+  return 2 * n_experts * ((n_tokens + 31) / 32) + 4 * (n_experts + 1);
+}
+
+// Exclusive scan of up to 256 values by one warp (8 per lane); returns the total to all lanes.
 DG_DEV int warp_exclusive_scan_256(const int* in, int* out, int n) {
   const int lane = lane_id();
   int v[8], s = 0;
@@ -287,96 +305,58 @@ DG_DEV int warp_exclusive_scan_256(const int* in, int* out, int n) {
   return __shfl_sync(0xffffffffu, incl, 31);
 }
 
-// Single CTA of 1024 threads: per-expert counts, exclusive scans (warp 0), the grouped GEMM item
-// lists, and the stable placement (slot order inside each expert) via warp match + per-warp
-// counts.  Items are (expert, 128-row tile, first permuted row, tokens <= n_chunk).
-__global__ void __launch_bounds__(1024) moe_route_kernel(RouteArgs a) {
-  pdl_enter();
-  if (block_done(a.done)) return;
-  __shared__ int cnt[32][257];  // per-warp counts in the current round, per expert
-  __shared__ int count_s[256], off_s[257], chunk_s[256], cbase_s[256], base_s[256];
-  const int tid = threadIdx.x, warp = tid >> 5, lane = lane_id();
-  const int E = a.n_experts;
-  for (int e = tid; e < E; e += 1024) count_s[e] = 0;
+// Expert permutation of the canvas by one CTA (any multiple of 32 threads), from the top-k ids
+// (read through L2: other CTAs wrote them).  A token picks an expert at most once, so with
+// mask[e] the bit set of tokens that picked e, the rank of slot (t, j) inside its expert is the
+// number of earlier tokens in mask[e]: prefix[e][t / 32] + popc(mask[e][t / 32] below bit t % 32).
+// perm[offsets[e] + rank] = slot keeps slot order inside each expert; every expert's rows are
+// then cut into chunks of n_chunk tokens (the grouped GEMMs' token tiles).  sm holds
+// route_smem_ints(E, n_tokens) ints; E <= 256, n_tokens <= kRouteMaxTokens.
+DG_DEV void route_canvas(const RouteArgs& a, int* sm) {
+  const int E = a.n_experts, words = (a.n_tokens + 31) >> 5, n_slots = a.n_tokens * a.top_k;
+  const int tid = threadIdx.x, nth = blockDim.x;
+  uint32_t* mask = reinterpret_cast<uint32_t*>(sm);  // [E][words]
+  int* prefix = sm + E * words;                      // [E][words]
+  int* count_s = prefix + E * words;                 // [E + 1]
+  int* off_s = count_s + (E + 1);
+  int* nch_s = off_s + (E + 1);
+  int* cbase_s = nch_s + (E + 1);
+  for (int i = tid; i < E * words; i += nth) mask[i] = 0u;
   __syncthreads();
-  for (int s = tid; s < a.n_slots; s += 1024) atomicAdd(&count_s[a.ids[s]], 1);
+  for (int s = tid; s < n_slots; s += nth) {
+    const int e = __ldcg(a.ids + s), t = s / a.top_k;
+    atomicOr(&mask[e * words + (t >> 5)], 1u << (t & 31));
+  }
   __syncthreads();
-  for (int e = tid; e < E; e += 1024) chunk_s[e] = (count_s[e] + a.n_chunk - 1) / a.n_chunk;
+  for (int e = tid; e < E; e += nth) {
+    int run = 0;
+    for (int w = 0; w < words; ++w) {
+      prefix[e * words + w] = run;
+      run += __popc(mask[e * words + w]);
+    }
+    count_s[e] = run;
+    nch_s[e] = (run + a.n_chunk - 1) / a.n_chunk;
+  }
   __syncthreads();
-  const int sh_chunks = (a.shared_m_tiles_gu > 0) ? (a.n_tokens + a.n_chunk - 1) / a.n_chunk : 0;
-  const int sh_gu = sh_chunks * a.shared_m_tiles_gu, sh_d = sh_chunks * a.shared_m_tiles_d;
-  if (warp == 0) {
+  if (tid < 32) {
     const int total = warp_exclusive_scan_256(count_s, off_s, E);
-    const int chunks = warp_exclusive_scan_256(chunk_s, cbase_s, E);
-    if (lane == 0) {
+    const int chunks = warp_exclusive_scan_256(nch_s, cbase_s, E);
+    if (tid == 0) {
       off_s[E] = total;
-      a.counts[0] = sh_gu + chunks * a.m_tiles_gu;
-      a.counts[1] = sh_d + chunks * a.m_tiles_d;
+      *a.n_chunks = chunks;
     }
   }
   __syncthreads();
-  // shared-expert items first; the token chunks of one weight tile are adjacent so the tile is
-  // re-read from L2
-  for (int w = tid; w < sh_gu; w += 1024) {
-    const int m = w / sh_chunks, ch = w % sh_chunks;
-    a.items_gu[w] = make_int4(E, m, ch * a.n_chunk, min(a.n_chunk, a.n_tokens - ch * a.n_chunk));
+  for (int e = tid; e <= E; e += nth) a.offsets[e] = off_s[e];
+  for (int s = tid; s < n_slots; s += nth) {
+    const int e = __ldcg(a.ids + s), t = s / a.top_k, w = t >> 5;
+    const int rank = prefix[e * words + w] + __popc(mask[e * words + w] & ((1u << (t & 31)) - 1u));
+    a.perm[off_s[e] + rank] = s;
   }
-  for (int w = tid; w < sh_d; w += 1024) {
-    const int m = w / sh_chunks, ch = w % sh_chunks;
-    a.items_d[w] = make_int4(E, m, ch * a.n_chunk, min(a.n_chunk, a.n_tokens - ch * a.n_chunk));
-  }
-  for (int e = tid; e <= E; e += 1024) a.offsets[e] = off_s[e];
-  // items: one (chunk, m tile) pair per thread
-  const int total_chunks = cbase_s[E - 1] + chunk_s[E - 1];
-  for (int w = tid; w < total_chunks * a.m_tiles_gu; w += 1024) {
-    const int ch = w / a.m_tiles_gu, m = w % a.m_tiles_gu;
-    int lo = 0, hi = E - 1;  // expert owning chunk ch: largest e with cbase_s[e] <= ch, chunk_s[e] > 0
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (cbase_s[mid] <= ch) lo = mid; else hi = mid - 1;
-    }
-    while (chunk_s[lo] == 0) --lo;
-    const int local = ch - cbase_s[lo];
-    a.items_gu[sh_gu + w] = make_int4(lo, m, off_s[lo] + local * a.n_chunk,
-                                      min(a.n_chunk, count_s[lo] - local * a.n_chunk));
-  }
-  for (int w = tid; w < total_chunks * a.m_tiles_d; w += 1024) {
-    const int ch = w / a.m_tiles_d, m = w % a.m_tiles_d;
-    int lo = 0, hi = E - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (cbase_s[mid] <= ch) lo = mid; else hi = mid - 1;
-    }
-    while (chunk_s[lo] == 0) --lo;
-    const int local = ch - cbase_s[lo];
-    a.items_d[sh_d + w] = make_int4(lo, m, off_s[lo] + local * a.n_chunk,
-                                    min(a.n_chunk, count_s[lo] - local * a.n_chunk));
-  }
-  // stable placement, 1024 slots per round
-  for (int e = tid; e < E; e += 1024) base_s[e] = off_s[e];
-  for (int r0 = 0; r0 < a.n_slots; r0 += 1024) {
-    for (int i = tid; i < 32 * 257; i += 1024) (&cnt[0][0])[i] = 0;
-    __syncthreads();
-    const int s = r0 + tid;
-    const bool valid = s < a.n_slots;
-    const int e = valid ? a.ids[s] : -1 - lane;  // distinct dummies never match real experts
-    const unsigned peers = __match_any_sync(0xffffffffu, e);
-    const int rank = __popc(peers & ((1u << lane) - 1u));
-    if (valid && rank == 0) cnt[warp][e] = __popc(peers);
-    __syncthreads();
-    if (valid) {
-      int before = 0;
-      for (int w = 0; w < warp; ++w) before += cnt[w][e];
-      a.perm[base_s[e] + before + rank] = s;
-    }
-    __syncthreads();
-    for (int f = tid; f < E; f += 1024) {
-      int tot = 0;
-      for (int w = 0; w < 32; ++w) tot += cnt[w][f];
-      base_s[f] += tot;
-    }
-    __syncthreads();
-  }
+  for (int e = tid; e < E; e += nth)
+    for (int c = 0; c < nch_s[e]; ++c)
+      a.chunks[cbase_s[e] + c] = make_int4(e, off_s[e] + c * a.n_chunk,
+                                           min(a.n_chunk, count_s[e] - c * a.n_chunk), 0);
 }
 
 // x_perm[p] = xn[perm[p] / k]; 64 threads per permuted row, 4 rows per CTA, 16-byte copies.

@@ -204,25 +204,11 @@ struct SamplerArgs {
   int32_t* ticket;
 };
 
-// Merge one row's partials (block-wide, fp64), decide lock / re-noise and write the row's
-// outputs; returns (in thread 0) whether this CTA is the last row to finish the step.
-DG_DEV bool sampler_row(const SamplerArgs& p, int row) {
-  StatD acc{0.0, 0.0, 0.0, 0x7fffffff};
-  for (int i = threadIdx.x; i < p.nsplit; i += blockDim.x) {
-    const float4 q4 = __ldcg(reinterpret_cast<const float4*>(p.partials) +
-                             static_cast<size_t>(row) * p.nsplit + i);
-    acc = stat_merge(acc, StatD{q4.x, q4.y, q4.z, __float_as_int(q4.w)});
-  }
-  __shared__ StatD red[256];
-  red[threadIdx.x] = acc;
-  __syncthreads();
-  for (int o = blockDim.x / 2; o > 0; o >>= 1) {
-    if (threadIdx.x < o) red[threadIdx.x] = stat_merge(red[threadIdx.x], red[threadIdx.x + o]);
-    __syncthreads();
-  }
+// Decide lock / re-noise for one row from its merged statistics and write the row's outputs;
+// returns (in every thread) whether this CTA is the last row to finish the step.
+DG_DEV bool sampler_row_finish(const SamplerArgs& p, int row, const StatD& r) {
   __shared__ int is_last;
   if (threadIdx.x == 0) {
-    const StatD r = red[0];
     const double conf = 1.0 / r.s;
     const double h = log(r.s) - r.u / r.s;
     p.conf[row] = static_cast<float>(conf);
@@ -239,6 +225,62 @@ DG_DEV bool sampler_row(const SamplerArgs& p, int row) {
   }
   __syncthreads();
   return is_last;
+}
+
+// Merge one row's nsplit partials (block-wide, fp64 tree) and finish the row.
+DG_DEV bool sampler_row(const SamplerArgs& p, int row) {
+  StatD acc{0.0, 0.0, 0.0, 0x7fffffff};
+  for (int i = threadIdx.x; i < p.nsplit; i += blockDim.x) {
+    const float4 q4 = __ldcg(reinterpret_cast<const float4*>(p.partials) +
+                             static_cast<size_t>(row) * p.nsplit + i);
+    acc = stat_merge(acc, StatD{q4.x, q4.y, q4.z, __float_as_int(q4.w)});
+  }
+  __shared__ StatD red[256];
+  red[threadIdx.x] = acc;
+  __syncthreads();
+  for (int o = blockDim.x / 2; o > 0; o >>= 1) {
+    if (threadIdx.x < o) red[threadIdx.x] = stat_merge(red[threadIdx.x], red[threadIdx.x + o]);
+    __syncthreads();
+  }
+  return sampler_row_finish(p, row, red[0]);
+}
+
+// Merge one row's pieces in column order: the piece starting at segment s keeps its partial at
+// slot row * segs + s and its length in segments at the same slot of piece_len.
+DG_DEV bool sampler_row_pieces(const SamplerArgs& p, int row, int segs,
+                               const int32_t* piece_len) {
+  // every slot of the row in one parallel round trip (slots that start no piece hold stale
+  // values and are never visited), then thread 0 follows the chain from segment 0
+  constexpr int kMaxSegs = 256;
+  __shared__ float4 sp[kMaxSegs];
+  __shared__ int sl[kMaxSegs];
+  __shared__ StatD merged;
+  for (int i = threadIdx.x; i < segs && i < kMaxSegs; i += blockDim.x) {
+    const size_t slot = static_cast<size_t>(row) * segs + i;
+    sp[i] = __ldcg(reinterpret_cast<const float4*>(p.partials) + slot);
+    sl[i] = __ldcg(piece_len + slot);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    StatD acc{0.0, 0.0, 0.0, 0x7fffffff};
+    for (int s = 0; s < segs;) {
+      float4 q4;
+      int len;
+      if (s < kMaxSegs) {
+        q4 = sp[s];
+        len = sl[s];
+      } else {
+        const size_t slot = static_cast<size_t>(row) * segs + s;
+        q4 = __ldcg(reinterpret_cast<const float4*>(p.partials) + slot);
+        len = __ldcg(piece_len + slot);
+      }
+      acc = stat_merge(acc, StatD{q4.x, q4.y, q4.z, __float_as_int(q4.w)});
+      s += max(1, len);
+    }
+    merged = acc;
+  }
+  __syncthreads();
+  return sampler_row_finish(p, row, merged);
 }
 
 // The stop test over the whole canvas, run by the last row's CTA (after a fence).  Rows written
@@ -320,10 +362,12 @@ DG_DEV void stat_merge_f32(float& m, float& s, float& u, int& a, float m2, float
 
 // Streaming statistics of one row slice for a 256-thread CTA.  Every thread walks its columns in
 // groups of kLoads 16-byte vectors (column c0 + ((g * kLoads + l) * 256 + tid) * kVec + j,
-// increasing in (g, l, j)) keeping running (m, S, T) with T = sum e t, t = (x - m) log2 e and
-// e = 2^t, so U = T / log2 e; S and T are rescaled only when a group raises the maximum.  The
-// argmax is resolved at the end: threads holding the CTA maximum re-read the one group where
-// they last raised it and take its first matching column.  Thread 0 returns the result.
+// increasing in (g, l, j)) keeping running (m, S, T, a) with T = sum e t, t = (x - m) log2 e,
+// e = 2^t (so U = T / log2 e) and a the first column holding m; S and T are rescaled only when a
+// group raises the maximum, which is also the only time the group is searched for its first
+// maximal column.  The CTA merge rescales every thread's sums once to the CTA maximum and adds
+// them up; the argmax is the lowest column among the threads holding that maximum.  Thread 0
+// returns the result.
 template <typename T> DG_DEV void to_f32x8(const uint4& raw, float (&v)[16 / sizeof(T)]);
 template <> DG_DEV void to_f32x8<__nv_bfloat16>(const uint4& raw, float (&v)[8]) {
   const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
@@ -341,37 +385,28 @@ template <> DG_DEV void to_f32x8<float>(const uint4& raw, float (&v)[4]) {
 }
 
 template <typename T, int kLoads>
-DG_DEV StatPartial stream_slice_stats(const T* base, int c0, int c1, StatD* red) {
+DG_DEV StatPartial stream_slice_stats(const T* base, int c0, int c1) {
   constexpr int kVec = 16 / sizeof(T);
   constexpr int kSpan = kLoads * 256 * kVec;  // columns per group over the CTA
   constexpr float kLog2e = 1.4426950408889634f;
   const int tid = threadIdx.x;
   float m = -INFINITY;
   float2 s2 = make_float2(0.f, 0.f), t2 = make_float2(0.f, 0.f);
-  int g_best = -1;  // group (its first column) where m was last raised
-  // one group of loads in flight ahead of the arithmetic (register double buffer)
-  auto load_group = [&](int g0, uint4 (&dst)[kLoads]) {
-    const bool full = g0 + kSpan <= c1;
-#pragma unroll
-    for (int l = 0; l < kLoads; ++l) {
-      const int c = g0 + (l * 256 + tid) * kVec;
-      if (full || c < c1) {
-        dst[l] = __ldcs(reinterpret_cast<const uint4*>(base + c));
-      } else if constexpr (sizeof(T) == 2) {
-        dst[l] = make_uint4(0xff80ff80u, 0xff80ff80u, 0xff80ff80u, 0xff80ff80u);  // bf16 -inf
-      } else {
-        dst[l] = make_uint4(0xff800000u, 0xff800000u, 0xff800000u, 0xff800000u);  // fp32 -inf
-      }
-    }
-  };
-  uint4 next[kLoads];
-  if (c0 < c1) load_group(c0, next);
+  int a = 0x7fffffff;
   for (int g0 = c0; g0 < c1; g0 += kSpan) {
     const bool full = g0 + kSpan <= c1;
     uint4 raw[kLoads];
 #pragma unroll
-    for (int l = 0; l < kLoads; ++l) raw[l] = next[l];
-    if (g0 + kSpan < c1) load_group(g0 + kSpan, next);
+    for (int l = 0; l < kLoads; ++l) {
+      const int c = g0 + (l * 256 + tid) * kVec;
+      if (full || c < c1) {
+        raw[l] = __ldcs(reinterpret_cast<const uint4*>(base + c));
+      } else if constexpr (sizeof(T) == 2) {
+        raw[l] = make_uint4(0xff80ff80u, 0xff80ff80u, 0xff80ff80u, 0xff80ff80u);  // bf16 -inf
+      } else {
+        raw[l] = make_uint4(0xff800000u, 0xff800000u, 0xff800000u, 0xff800000u);  // fp32 -inf
+      }
+    }
     // group maximum (packed bf16 pairs for bf16 input); -inf padding never wins
     float gm;
     if constexpr (sizeof(T) == 2) {
@@ -392,13 +427,23 @@ DG_DEV StatPartial stream_slice_stats(const T* base, int c0, int c1, StatD* red)
     }
     if (gm > m) {  // strict: an earlier group keeps an equal maximum
       if (m != -INFINITY) {
-        const float sc = fast_exp2((m - gm) * kLog2e);
         const float dt = (m - gm) * kLog2e;  // t shifts by dt for every earlier term
+        const float sc = fast_exp2(dt);
         t2 = make_float2(sc * (t2.x + dt * s2.x), sc * (t2.y + dt * s2.y));
         s2 = make_float2(sc * s2.x, sc * s2.y);
       }
       m = gm;
-      g_best = g0;
+      // first column of this group holding the new maximum (columns increase with l, then j)
+      int found = 0x7fffffff;
+#pragma unroll
+      for (int l = kLoads - 1; l >= 0; --l) {
+        float v[kVec];
+        to_f32x8<T>(raw[l], v);
+#pragma unroll
+        for (int j = kVec - 1; j >= 0; --j)
+          if (v[j] == gm) found = g0 + (l * 256 + tid) * kVec + j;
+      }
+      a = found;
     }
     // t = (x - m) log2 e with the subtraction first, so the maximum's own term is exactly 2^0
     const float2 l2 = make_float2(kLog2e, kLog2e);
@@ -432,82 +477,101 @@ DG_DEV StatPartial stream_slice_stats(const T* base, int c0, int c1, StatD* red)
       }
     }
   }
-  float s = s2.x + s2.y, u = (t2.x + t2.y) * (1.0f / kLog2e);
-  // CTA maximum, then the first column holding it (re-read the recorded group)
-  float bm = m;
-  for (int o = 16; o > 0; o >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
+  float s = s2.x + s2.y, tt = t2.x + t2.y;
+  // CTA maximum
   const int warp = tid >> 5;
   __shared__ float wmax[8];
+  __shared__ float wsum[2][8];
+  __shared__ int warg[8];
+  float bm = m;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
   if (lane_id() == 0) wmax[warp] = bm;
   __syncthreads();
   bm = wmax[0];
 #pragma unroll
   for (int w = 1; w < 8; ++w) bm = fmaxf(bm, wmax[w]);
-  int a = 0x7fffffff;
-  if (m == bm && g_best >= 0) {
-#pragma unroll
-    for (int l = kLoads - 1; l >= 0; --l) {
-      const int c = g_best + (l * 256 + tid) * kVec;
-      if (c < c1) {
-        const uint4 raw = __ldcg(reinterpret_cast<const uint4*>(base + c));
-        float v[kVec];
-        to_f32x8<T>(raw, v);
-#pragma unroll
-        for (int j = kVec - 1; j >= 0; --j)
-          if (v[j] == bm) a = c + j;
-      }
-    }
+  // every thread's sums relative to the CTA maximum, then plain sums; argmax = lowest column
+  // among the threads that hold the maximum
+  if (m == -INFINITY || bm == -INFINITY) {
+    s = 0.f;
+    tt = 0.f;
+  } else if (m != bm) {
+    const float dt = (m - bm) * kLog2e;
+    const float sc = fast_exp2(dt);
+    tt = sc * (tt + dt * s);
+    s *= sc;
   }
-  // merge (m, S, U) over the CTA: warp shuffles, then the 8 warp results
+  int am = (m == bm) ? a : 0x7fffffff;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
-    const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
-    const float ss = __shfl_xor_sync(0xffffffffu, s, o);
-    const float uu = __shfl_xor_sync(0xffffffffu, u, o);
-    const int a2 = __shfl_xor_sync(0xffffffffu, a, o);
-    stat_merge_f32(m, s, u, a, m2, ss, uu, a2);
+    s += __shfl_xor_sync(0xffffffffu, s, o);
+    tt += __shfl_xor_sync(0xffffffffu, tt, o);
+    am = min(am, __shfl_xor_sync(0xffffffffu, am, o));
   }
-  if (lane_id() == 0) red[warp] = StatD{m, s, u, a};
+  if (lane_id() == 0) {
+    wsum[0][warp] = s;
+    wsum[1][warp] = tt;
+    warg[warp] = am;
+  }
   __syncthreads();
   StatPartial r{-INFINITY, 0.f, 0.f, 0x7fffffff};
   if (tid == 0) {
-    float rm = static_cast<float>(red[0].m), rs = static_cast<float>(red[0].s);
-    float ru = static_cast<float>(red[0].u);
-    int ra = red[0].a;
-    for (int w = 1; w < 8; ++w)
-      stat_merge_f32(rm, rs, ru, ra, static_cast<float>(red[w].m), static_cast<float>(red[w].s),
-                     static_cast<float>(red[w].u), red[w].a);
-    r = StatPartial{rm, rs, ru, ra};
+    float rs = 0.f, rt = 0.f;
+    int ra = 0x7fffffff;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      rs += wsum[0][w];
+      rt += wsum[1][w];
+      ra = min(ra, warg[w]);
+    }
+    r = StatPartial{bm, rs, rt * (1.0f / kLog2e), ra};
   }
-  __syncthreads();  // red is reused by the caller
+  __syncthreads();  // the shared arrays are rewritten by the next slice
   return r;
 }
 
-// Statistics, merge and stop test in one launch: grid = (chunks, rows), chunk columns per CTA
-// streamed in groups.  Each CTA writes its slice's partial; the last CTA of a row (per-row ticket)
-// merges the row; the last row runs the stop test.  row_ticket [rows] starts and ends at zero.
+// Statistics, merge and stop test in one launch on a balanced persistent grid.  The rows x segs
+// units (one kSpan-column group each) are cut into gridDim.x contiguous runs of equal length; a
+// CTA streams its run and writes one partial per row piece (a run covers a few rows at most),
+// kept at the piece's first segment together with its length.  A per-row count of finished
+// segments finds the CTA completing the row, which merges the pieces in column order; the last
+// row runs the stop test.  No CTA waits on another; row_units [rows] starts and ends at zero.
 template <typename T, int kLoads>
-__global__ void __launch_bounds__(256) sampler_fused_kernel(const T* __restrict__ logits,
-                                                            int32_t chunk, SamplerArgs p,
-                                                            int32_t* __restrict__ row_ticket) {
+__global__ void __launch_bounds__(256, sizeof(T) == 2 ? 5 : 3)
+    sampler_stream_kernel(const T* __restrict__ logits, int32_t segs, SamplerArgs p,
+                          int32_t* __restrict__ row_units, int32_t* __restrict__ piece_len) {
   pdl_enter();
   if (block_done(p.state + kStDone)) return;
-  __shared__ StatD red[256];
-  __shared__ int last_chunk;
-  const int row = blockIdx.y;
-  const int c0 = blockIdx.x * chunk;
-  const StatPartial r = stream_slice_stats<T, kLoads>(
-      logits + static_cast<size_t>(row) * p.vocab, c0, min(c0 + chunk, p.vocab), red);
-  if (threadIdx.x == 0) {
-    const_cast<StatPartial*>(p.partials)[static_cast<size_t>(row) * p.nsplit + blockIdx.x] = r;
-    __threadfence();
-    last_chunk = (atomicAdd(row_ticket + row, 1) == p.nsplit - 1);
+  constexpr int kSpan = kLoads * 256 * (16 / static_cast<int>(sizeof(T)));
+  __shared__ int last_piece;
+  const long long total = static_cast<long long>(p.rows) * segs;
+  long long u = blockIdx.x * total / gridDim.x;
+  const long long u_end = (blockIdx.x + 1) * total / gridDim.x;
+  while (u < u_end) {
+    const int row = static_cast<int>(u / segs);
+    const int seg0 = static_cast<int>(u % segs);
+    const int len = static_cast<int>(min(u_end, static_cast<long long>(row + 1) * segs) - u);
+    const int c0 = seg0 * kSpan;
+    const int c1 = min(p.vocab, (seg0 + len) * kSpan);
+    const StatPartial r =
+        stream_slice_stats<T, kLoads>(logits + static_cast<size_t>(row) * p.vocab, c0, c1);
+    const size_t slot = static_cast<size_t>(row) * segs + seg0;
+    if (threadIdx.x == 0) {
+      const_cast<StatPartial*>(p.partials)[slot] = r;
+      piece_len[slot] = len;
+      __threadfence();
+      last_piece = (atomicAdd(row_units + row, len) + len == segs);
+    }
+    __syncthreads();
+    if (last_piece) {
+      __threadfence();
+      if (threadIdx.x == 0) row_units[row] = 0;
+      if (sampler_row_pieces(p, row, segs, piece_len)) sampler_stop_test(p);
+    }
+    __syncthreads();  // last_piece is rewritten by the next piece
+    u += len;
   }
-  __syncthreads();
-  if (!last_chunk) return;
-  __threadfence();
-  if (threadIdx.x == 0) row_ticket[row] = 0;
-  if (sampler_row(p, row)) sampler_stop_test(p);
 }
 
 }  // namespace dg
