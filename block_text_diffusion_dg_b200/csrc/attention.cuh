@@ -51,8 +51,6 @@ constexpr int kAttnThreads = 64 + 32 * 8;
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_vt, const AttnParams p) {
-  pdl_enter();
-  if (block_done(p.done)) return;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -108,6 +106,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   // TMEM columns: [0,128) O, [128,256) S0, [256,384) S1, [384,390) partner exchange
   const uint32_t tmem_base = *tmem_holder;
+  // the setup above overlaps the previous kernel; from here on its results are needed
+  pdl_enter();
+  if (block_done(p.done)) {  // uniform over the grid: release TMEM and leave
+    if (warp == 1) tmem_dealloc(tmem_base, 512);
+    return;
+  }
 
   if (warp == 0) {
     if (elect_one() && n_tiles > 0) {

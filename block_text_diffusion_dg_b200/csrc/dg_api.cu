@@ -176,6 +176,7 @@ int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cud
 
 // ---- GEMM launch helpers -----------------------------------------------------------------
 constexpr int kGroupN = 64, kGroupStages = 8;
+constexpr int kRouterChunk = 64;  // tokens per router cluster
 
 // ta2/tb2 are read only by items of the alternate group (p.alt_group >= 0).
 template <int MAXN, int STAGES, int EPI>
@@ -223,10 +224,12 @@ int launch_cluster(const CUtensorMap& ta, const CUtensorMap& tb, const CluParams
 }
 
 // Shape part of the cluster projection parameters: `m_rows` weight rows, `n` tokens, K = 64 kb.
-CluParams clu_params(int m_rows, int n, int kb, int splits, int* err, const int* done) {
+CluParams clu_params(int m_rows, int n, int kb, int splits, int* err, const int* done,
+                     int chunk_n = 256) {
   CluParams p{};
   p.n_tokens = n;
-  p.n_chunks = cdiv(n, 256);
+  p.chunk_n = chunk_n;
+  p.n_chunks = cdiv(n, chunk_n);
   p.m_tiles = cdiv(m_rows, 128);
   p.m_rows = m_rows;
   p.kb_total = kb;
@@ -571,8 +574,8 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     a.done = done;
     DG_TRY(set_smem(attention_kernel, kAttnSmemBytes));
     prof_before(DG_KERNEL_ATTENTION, st);
-    DG_TRY(launch_pdl(attention_kernel, dim3(m_tiles, g.n_kv_heads, splits), dim3(kAttnThreads), kAttnSmemBytes, st, 
-        c->tm_q, c->tm_k, c->tm_vt, a));
+    DG_TRY(launch_pdl(attention_kernel, dim3(m_tiles, g.n_kv_heads, splits), dim3(kAttnThreads),
+                      kAttnSmemBytes, st, c->tm_q, c->tm_k, c->tm_vt, a));
     DG_LAUNCHED();
     prof_after(DG_KERNEL_ATTENTION, st);
     prof_before(DG_KERNEL_ATTN_COMBINE, st);
@@ -599,7 +602,8 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
   // router (cluster split-K) with top-k in its epilogue; the grid's last CTA routes the canvas
   const bool shared = g.shared_hidden > 0;
   {
-    CluParams p = clu_params(E, n, d / 64, c->split_r, c->err, done);
+    // 64-token chunks: the top-k of a chunk is spread over its 8 CTAs
+    CluParams p = clu_params(E, n, d / 64, c->split_r, c->err, done, kRouterChunk);
     p.router_logits = c->router_logits;
     p.ids = c->topk_ids;
     p.wts = c->topk_w;
@@ -1263,8 +1267,8 @@ int dg_canvas_attention(const void* d_q, const void* d_k, const void* d_vt, void
   cudaStream_t st = S(stream);
   DG_CUDA(cudaMemsetAsync(a.err, 0, 4, st));
   DG_TRY(set_smem(attention_kernel, kAttnSmemBytes));
-  DG_TRY(launch_pdl(attention_kernel, dim3(m_tiles, n_kv_heads, splits), dim3(kAttnThreads), kAttnSmemBytes, st, tq_m, tk_m, tv_m,
-                                                                                  a));
+  DG_TRY(launch_pdl(attention_kernel, dim3(m_tiles, n_kv_heads, splits), dim3(kAttnThreads),
+                    kAttnSmemBytes, st, tq_m, tk_m, tv_m, a));
   DG_LAUNCHED();
   DG_TRY(launch_pdl(attn_combine_kernel<__nv_bfloat16>, dim3(cdiv(t * n_heads, 8)), dim3(256), 0, st,
                     a.o_part, a.ml_part, splits, n_heads, tq, t, static_cast<__nv_bfloat16*>(d_o),
@@ -1366,7 +1370,7 @@ int dg_moe_ffn(const void* d_x, const float* d_residual, const void* d_wr, const
   }
   // router
   const bool shared = shared_hidden > 0;
-  CluParams pr = clu_params(n_experts, t, d / 64, m.split_r, err, nullptr);
+  CluParams pr = clu_params(n_experts, t, d / 64, m.split_r, err, nullptr, kRouterChunk);
   pr.router_logits = d_router_logits ? d_router_logits : rlog;
   pr.ids = ids;
   pr.wts = wts;

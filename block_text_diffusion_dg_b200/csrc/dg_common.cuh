@@ -66,8 +66,11 @@ DG_DEV bool mbar_try_wait(uint32_t addr, uint32_t parity) {
   return ok != 0;
 }
 // Wait until the phase with the given parity has completed.  Gives up after kWaitLimitNs
-// (records kDevErrTimeout in *err) or as soon as another thread has recorded an error;
-// returns false in both cases so the caller can unwind to its teardown.
+// (records kDevErrTimeout in *err), or once it has waited kErrPollNs and another thread has
+// recorded an error; returns false in both cases so the caller can unwind to its teardown.  The
+// error word (global memory) is not read during ordinary waits: a phase that completes while
+// such a read is in flight would only be seen after the read returns.
+constexpr uint64_t kErrPollNs = 100000ull;
 DG_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, int* err) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
@@ -76,11 +79,12 @@ DG_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, int* err) {
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(a, parity)) return true;
-    if (*reinterpret_cast<volatile int*>(err) != 0) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    const uint64_t dt = globaltimer_ns() - t0;
+    if (dt > kWaitLimitNs) {
       atomicExch(err, kDevErrTimeout);
       return false;
     }
+    if (dt > kErrPollNs && *reinterpret_cast<volatile int*>(err) != 0) return false;
   }
 }
 

@@ -188,8 +188,6 @@ __global__ void __launch_bounds__(GemmCfg<MAXN, STAGES>::kThreads, 1)
                        const __grid_constant__ CUtensorMap tm_a2,
                        const __grid_constant__ CUtensorMap tm_b2, const GemmParams p) {
   using C = GemmCfg<MAXN, STAGES>;
-  pdl_enter();
-  if (block_done(p.done)) return;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -225,6 +223,12 @@ __global__ void __launch_bounds__(GemmCfg<MAXN, STAGES>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  // the setup above overlaps the previous kernel; from here on its results are needed
+  pdl_enter();
+  if (block_done(p.done)) {  // uniform over the grid: release TMEM and leave
+    if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
+    return;
+  }
   const int n_items = gemm_item_count(p);
 
   if (warp == 0) {
@@ -372,8 +376,6 @@ template <bool kStats>
 __global__ void __launch_bounds__(kLmThreads, 1)
     lmhead_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_e,
                   const LmHeadParams p) {
-  pdl_enter();
-  if (block_done(p.done)) return;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -404,6 +406,12 @@ __global__ void __launch_bounds__(kLmThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  // the setup above overlaps the previous kernel; from here on its results are needed
+  pdl_enter();
+  if (block_done(p.done)) {  // uniform over the grid: release TMEM and leave
+    if (warp == 1) tmem_dealloc(tmem_base, 512);
+    return;
+  }
 
   if (warp == 0) {
     if (elect_one()) {

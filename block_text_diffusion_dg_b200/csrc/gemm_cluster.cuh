@@ -39,8 +39,9 @@ static_assert(kCluDrainBytes + 128 * 256 * 2 <= kCluRingBytes, "V^T scratch");
 static_assert(kCluDrainBytes + 128 * 128 * 4 <= kCluRingBytes, "router scratch");
 
 struct CluParams {
-  int n_tokens;   // tokens of this call (<= 256 per token chunk)
-  int n_chunks;   // token chunks of 256
+  int n_tokens;   // tokens of this call
+  int chunk_n;    // tokens per token chunk (<= 256, a multiple of 32)
+  int n_chunks;   // token chunks
   int m_tiles;    // weight tiles of 128 rows
   int m_rows;     // weight rows in use
   int kb_total;   // K / 64
@@ -69,8 +70,6 @@ template <int EPI>
 __global__ void __launch_bounds__(kCluThreads, 1)
     gemm_cluster_kernel(const __grid_constant__ CUtensorMap tm_a,
                         const __grid_constant__ CUtensorMap tm_b, const CluParams p) {
-  pdl_enter();
-  if (block_done(p.done)) return;  // uniform over the grid
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -83,8 +82,8 @@ __global__ void __launch_bounds__(kCluThreads, 1)
   const int s = static_cast<int>(blockIdx.x) % S;  // == cluster rank (cluster dims (S, 1, 1))
   const int tile = static_cast<int>(blockIdx.x) / S;
   const int mt = tile / p.n_chunks, nc = tile % p.n_chunks;
-  const int t0 = nc * 256;                          // first token of the chunk
-  const int n = min(256, p.n_tokens - t0);          // tokens of the chunk
+  const int t0 = nc * p.chunk_n;                    // first token of the chunk
+  const int n = min(p.chunk_n, p.n_tokens - t0);    // tokens of the chunk
   const int kb0 = s * p.kb_total / S, kb1 = (s + 1) * p.kb_total / S;
 
   if (warp == 0 && lane_id() == 0) {
@@ -105,6 +104,12 @@ __global__ void __launch_bounds__(kCluThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  // the setup above overlaps the previous kernel; from here on its results are needed
+  pdl_enter();
+  if (block_done(p.done)) {  // uniform over the grid: release TMEM and leave
+    if (warp == 1) tmem_dealloc(tmem_base, 256);
+    return;
+  }
   bool ok = true;  // this thread's waits all succeeded
 
   if (warp == 0) {
@@ -182,18 +187,50 @@ __global__ void __launch_bounds__(kCluThreads, 1)
   const int tid = threadIdx.x;
   const int t_lo = n * s / S, t_hi = n * (s + 1) / S, nt = t_hi - t_lo;
   const uint32_t drain_u32 = smem_u32(smem);
-  // sum of the S partials of (token t, rows 4 r4 .. 4 r4 + 3), ranks in order
+  // sum of the S partials of (token t, rows 4 r4 .. 4 r4 + 3), ranks in order; every peer's load
+  // is issued before the first add so the distributed shared memory latencies overlap
   auto reduce4 = [&](int t, int r4) -> float4 {
     const uint32_t off = drain_u32 + static_cast<uint32_t>((t * 128 + 4 * r4) * 4);
+    float4 v[kCluMaxSplits];
+#pragma unroll
+    for (int src = 0; src < kCluMaxSplits; ++src)
+      if (src < S) v[src] = dsmem_ld4(dsmem_addr(off, static_cast<uint32_t>(src)));
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int src = 0; src < S; ++src) {
-      const float4 v = dsmem_ld4(dsmem_addr(off, static_cast<uint32_t>(src)));
-      acc.x += v.x;
-      acc.y += v.y;
-      acc.z += v.z;
-      acc.w += v.w;
-    }
+#pragma unroll
+    for (int src = 0; src < kCluMaxSplits; ++src)
+      if (src < S) {
+        acc.x += v[src].x;
+        acc.y += v[src].y;
+        acc.z += v[src].z;
+        acc.w += v[src].w;
+      }
     return acc;
+  };
+  // the same for two row groups of one token (the rotate-half pair), 2 S loads in flight
+  auto reduce4x2 = [&](int t, int r4a, int r4b, float4& a, float4& b) {
+    const uint32_t oa = drain_u32 + static_cast<uint32_t>((t * 128 + 4 * r4a) * 4);
+    const uint32_t ob = drain_u32 + static_cast<uint32_t>((t * 128 + 4 * r4b) * 4);
+    float4 va[kCluMaxSplits], vb[kCluMaxSplits];
+#pragma unroll
+    for (int src = 0; src < kCluMaxSplits; ++src)
+      if (src < S) {
+        va[src] = dsmem_ld4(dsmem_addr(oa, static_cast<uint32_t>(src)));
+        vb[src] = dsmem_ld4(dsmem_addr(ob, static_cast<uint32_t>(src)));
+      }
+    a = make_float4(0.f, 0.f, 0.f, 0.f);
+    b = a;
+#pragma unroll
+    for (int src = 0; src < kCluMaxSplits; ++src)
+      if (src < S) {
+        a.x += va[src].x;
+        a.y += va[src].y;
+        a.z += va[src].z;
+        a.w += va[src].w;
+        b.x += vb[src].x;
+        b.y += vb[src].y;
+        b.z += vb[src].z;
+        b.w += vb[src].w;
+      }
   };
   const int rows4 = min(32, (p.m_rows - mt * 128 + 3) >> 2);  // valid float4 row groups
   if constexpr (EPI == kCluResidual) {
@@ -220,7 +257,8 @@ __global__ void __launch_bounds__(kCluThreads, 1)
         for (int u = tid; u < nt * 16; u += kCluThreads) {
           const int t = t_lo + u / 16, r4 = u % 16;
           const int tg = t0 + t;
-          const float4 a = reduce4(t, r4), b = reduce4(t, r4 + 16);
+          float4 a, b;
+          reduce4x2(t, r4, r4 + 16, a, b);
           const float2* cs = p.rope_tab + static_cast<long long>(p.pos0 + tg) * 64 + 4 * r4;
           const float2 c0 = cs[0], c1 = cs[1], c2 = cs[2], c3 = cs[3];
           __nv_bfloat16* dst =

@@ -323,9 +323,20 @@ DG_DEV void route_canvas(const RouteArgs& a, int* sm) {
   int* cbase_s = nch_s + (E + 1);
   for (int i = tid; i < E * words; i += nth) mask[i] = 0u;
   __syncthreads();
-  for (int s = tid; s < n_slots; s += nth) {
-    const int e = __ldcg(a.ids + s), t = s / a.top_k;
-    atomicOr(&mask[e * words + (t >> 5)], 1u << (t & 31));
+  // the ids are read in batches of kIdBatch per thread, all loads issued before their use
+  constexpr int kIdBatch = 8;
+  for (int s0 = 0; s0 < n_slots; s0 += nth * kIdBatch) {
+    int e[kIdBatch];
+#pragma unroll
+    for (int b = 0; b < kIdBatch; ++b) {
+      const int s = s0 + b * nth + tid;
+      e[b] = s < n_slots ? __ldcg(a.ids + s) : -1;
+    }
+#pragma unroll
+    for (int b = 0; b < kIdBatch; ++b) {
+      const int t = (s0 + b * nth + tid) / a.top_k;
+      if (e[b] >= 0) atomicOr(&mask[e[b] * words + (t >> 5)], 1u << (t & 31));
+    }
   }
   __syncthreads();
   for (int e = tid; e < E; e += nth) {
@@ -348,10 +359,22 @@ DG_DEV void route_canvas(const RouteArgs& a, int* sm) {
   }
   __syncthreads();
   for (int e = tid; e <= E; e += nth) a.offsets[e] = off_s[e];
-  for (int s = tid; s < n_slots; s += nth) {
-    const int e = __ldcg(a.ids + s), t = s / a.top_k, w = t >> 5;
-    const int rank = prefix[e * words + w] + __popc(mask[e * words + w] & ((1u << (t & 31)) - 1u));
-    a.perm[off_s[e] + rank] = s;
+  for (int s0 = 0; s0 < n_slots; s0 += nth * kIdBatch) {
+    int e[kIdBatch];
+#pragma unroll
+    for (int b = 0; b < kIdBatch; ++b) {
+      const int s = s0 + b * nth + tid;
+      e[b] = s < n_slots ? __ldcg(a.ids + s) : -1;
+    }
+#pragma unroll
+    for (int b = 0; b < kIdBatch; ++b) {
+      const int s = s0 + b * nth + tid, t = s / a.top_k, w = t >> 5;
+      if (e[b] >= 0) {
+        const int rank = prefix[e[b] * words + w] +
+                         __popc(mask[e[b] * words + w] & ((1u << (t & 31)) - 1u));
+        a.perm[off_s[e[b]] + rank] = s;
+      }
+    }
   }
   for (int e = tid; e < E; e += nth)
     for (int c = 0; c < nch_s[e]; ++c)
