@@ -15,8 +15,8 @@
 // 128-byte swizzled K-major layout.  O lives in TMEM for the whole key range;
 // its running maximum is only moved (and O rescaled) when a new tile raises the row max by
 // more than 2^8, otherwise exponents relative to the stale maximum stay below 256.
-// Each split writes its unnormalised O, its max and its denominator; a combine kernel merges
-// splits exactly.  V is read from a transposed copy (V^T [hd, keys]) so that both UMMA
+// Each split writes its unnormalised O, its max and its denominator; the splits of a query tile
+// form a thread-block cluster and merge their rows exactly after a cluster barrier.  V is read from a transposed copy (V^T [hd, keys]) so that both UMMA
 // operands of P V are K-major.
 #pragma once
 #include "dg_common.cuh"
@@ -38,6 +38,7 @@ struct AttnParams {
   int n_heads;
   float* o_part;      // [splits, Hq, tq, 128]
   float2* ml_part;    // [splits, Hq, tq] (max in log2 units, denominator)
+  __nv_bfloat16* o;   // [T, Hq * 128] merged output
   int* err;
   const int* done;
 };
@@ -47,6 +48,50 @@ constexpr int kAttnTile = 16384;  // one 128-row x 128-byte swizzled slab
 constexpr int kAttnSmemBytes = 14 * kAttnTile + 1024 + 256;
 
 constexpr int kAttnThreads = 64 + 32 * 8;
+constexpr int kMaxAttnSplits = 8;  // the key splits of a query tile form one cluster
+
+// Merge of the key splits of one (token, head) by one warp: O = sum_s 2^(m_s - M) O_s /
+// sum_s 2^(m_s - M) l_s, lane d4 owning dims 4 d4 .. 4 d4 + 3, stored as bf16 into o [T, Hq * 128]
+// (token-major, the O projection's token operand).  Lane s < n_splits reads split s's
+// (max, denominator); the partials of other CTAs are read through L2.
+DG_DEV void attn_merge_row(const AttnParams& p, int n_splits, int tok, int head) {
+  const int lane = lane_id();
+  float2 ml = make_float2(-INFINITY, 0.f);
+  if (lane < n_splits)
+    ml = __ldcg(p.ml_part + (static_cast<long long>(lane) * p.n_heads + head) * p.tq + tok);
+  float mmax = ml.x;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mmax = fmaxf(mmax, __shfl_xor_sync(0xffffffffu, mmax, o));
+  const float w_mine = (lane < n_splits && ml.y != 0.f) ? exp2f(ml.x - mmax) : 0.f;
+  float4 v[kMaxAttnSplits];
+#pragma unroll
+  for (int s = 0; s < kMaxAttnSplits; ++s)
+    if (s < n_splits) {
+      const long long row = (static_cast<long long>(s) * p.n_heads + head) * p.tq + tok;
+      v[s] = __ldcg(reinterpret_cast<const float4*>(p.o_part + row * 128) + lane);
+    }
+  float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+  float den = 0.f;
+#pragma unroll
+  for (int s = 0; s < kMaxAttnSplits; ++s)
+    if (s < n_splits) {
+      const float w = __shfl_sync(0xffffffffu, w_mine, s);
+      const float l = __shfl_sync(0xffffffffu, ml.y, s);
+      if (w != 0.f) {
+        num.x += w * v[s].x;
+        num.y += w * v[s].y;
+        num.z += w * v[s].z;
+        num.w += w * v[s].w;
+        den += w * l;
+      }
+    }
+  const float inv = 1.0f / den;
+  const __nv_bfloat162 lo = __floats2bfloat162_rn(num.x * inv, num.y * inv);
+  const __nv_bfloat162 hi = __floats2bfloat162_rn(num.z * inv, num.w * inv);
+  *reinterpret_cast<uint2*>(p.o + static_cast<long long>(tok) * p.n_heads * 128 + head * 128 +
+                            4 * lane) = make_uint2(*reinterpret_cast<const uint32_t*>(&lo),
+                                                   *reinterpret_cast<const uint32_t*>(&hi));
+}
 
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -332,51 +377,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, 512);
   }
-}
-
-// Merge the key splits: O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s, stored into
-// o [T, Hq * 128] (token-major, ready to be the O-projection's token operand).  One warp per
-// (token, head), 4 dims per lane; 8 warps per CTA.
-template <typename TA>
-__global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restrict__ o_part,
-                                                           const float2* __restrict__ ml_part,
-                                                           int n_splits, int n_heads, int tq,
-                                                           int n_queries, TA* __restrict__ o,
-                                                           const int* done) {
-  pdl_enter();
-  if (block_done(done)) return;
-  const int pair = blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (pair >= n_queries * n_heads) return;
-  const int tok = pair / n_heads, head = pair % n_heads, d4 = lane_id();
-  constexpr int kMax = 16;
-  float2 ml[kMax];
-  float mmax = -INFINITY;
-#pragma unroll
-  for (int s = 0; s < kMax; ++s)
-    if (s < n_splits) {
-      ml[s] = ml_part[(static_cast<long long>(s) * n_heads + head) * tq + tok];
-      mmax = fmaxf(mmax, ml[s].x);
-    }
-  float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
-  float den = 0.f;
-#pragma unroll
-  for (int s = 0; s < kMax; ++s)
-    if (s < n_splits && ml[s].y != 0.f) {
-      const long long row = (static_cast<long long>(s) * n_heads + head) * tq + tok;
-      const float w = exp2f(ml[s].x - mmax);
-      const float4 v = reinterpret_cast<const float4*>(o_part + row * 128)[d4];
-      num.x += w * v.x;
-      num.y += w * v.y;
-      num.z += w * v.z;
-      num.w += w * v.w;
-      den += w * ml[s].y;
-    }
-  const float inv = 1.0f / den;
-  TA* dst = o + static_cast<long long>(tok) * n_heads * 128 + head * 128 + 4 * d4;
-  dst[0] = store_from_f32<TA>(num.x * inv);
-  dst[1] = store_from_f32<TA>(num.y * inv);
-  dst[2] = store_from_f32<TA>(num.z * inv);
-  dst[3] = store_from_f32<TA>(num.w * inv);
+  // the key splits of this query tile are one cluster (dims (1, 1, splits)): once every split's
+  // partial rows are written, the CTA of split s merges rows [128 s / S, 128 (s + 1) / S) of
+  // the tile.  Every thread of every CTA reaches the barrier.
+  __threadfence();
+  cluster_sync_all();
+  const int n_splits = gridDim.z;
+  const int r0 = 128 * split / n_splits, r1 = 128 * (split + 1) / n_splits;
+  for (int rr = r0 + warp; rr < r1; rr += kAttnThreads / 32) {
+    const int tok = tok0 + rr;
+    if (tok < p.n_queries) attn_merge_row(p, n_splits, tok, head);
+  }
 }
 
 }  // namespace dg

@@ -174,6 +174,29 @@ int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cud
   return DG_OK;
 }
 
+// launch_pdl with thread-block clusters of the given dimensions.
+template <typename... KArgs, typename... Args>
+int launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, dim3 cluster, Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = cluster.x;
+  attr[1].val.clusterDim.y = cluster.y;
+  attr[1].val.clusterDim.z = cluster.z;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  if (e != cudaSuccess) return fail(DG_ERR_CUDA, "cluster launch failed: %s", cudaGetErrorString(e));
+  return DG_OK;
+}
+
 // ---- GEMM launch helpers -----------------------------------------------------------------
 constexpr int kGroupN = 64, kGroupStages = 8;
 constexpr int kRouterChunk = 64;  // tokens per router cluster
@@ -371,7 +394,7 @@ Derived derive(const dg_config& c, int sms) {
   }
   const int group = c.n_heads / c.n_kv_heads;
   const int m_tiles = group * d.tq / 128;
-  d.att_splits = std::max(1, std::min(16, sms / std::max(1, m_tiles * c.n_kv_heads)));
+  d.att_splits = std::max(1, std::min(kMaxAttnSplits, sms / std::max(1, m_tiles * c.n_kv_heads)));
   d.max_chunks = c.n_experts + (T * c.top_k + kGroupN - 1) / kGroupN;
   return d;
 }
@@ -570,20 +593,16 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     a.n_heads = g.n_heads;
     a.o_part = c->o_part;
     a.ml_part = c->ml_part;
+    a.o = static_cast<__nv_bfloat16*>(c->o);
     a.err = c->err;
     a.done = done;
     DG_TRY(set_smem(attention_kernel, kAttnSmemBytes));
     prof_before(DG_KERNEL_ATTENTION, st);
-    DG_TRY(launch_pdl(attention_kernel, dim3(m_tiles, g.n_kv_heads, splits), dim3(kAttnThreads),
-                      kAttnSmemBytes, st, c->tm_q, c->tm_k, c->tm_vt, a));
+    DG_TRY(launch_pdl_cluster(attention_kernel, dim3(m_tiles, g.n_kv_heads, splits),
+                              dim3(kAttnThreads), kAttnSmemBytes, st, dim3(1, 1, splits), c->tm_q,
+                              c->tm_k, c->tm_vt, a));
     DG_LAUNCHED();
     prof_after(DG_KERNEL_ATTENTION, st);
-    prof_before(DG_KERNEL_ATTN_COMBINE, st);
-    DG_TRY(launch_pdl(attn_combine_kernel<__nv_bfloat16>, dim3(cdiv(n * g.n_heads, 8)), dim3(256), 0,
-                      st, c->o_part, c->ml_part, splits, g.n_heads, c->tq, n,
-                      static_cast<__nv_bfloat16*>(c->o), done));
-    DG_LAUNCHED();
-    prof_after(DG_KERNEL_ATTN_COMBINE, st);
   }
   // O projection onto the residual stream (cluster split-K), then the ffn norm
   {
@@ -1233,7 +1252,7 @@ int dg_canvas_attention(const void* d_q, const void* d_k, const void* d_vt, void
   const int group = n_heads / n_kv_heads;
   const int m_tiles = group * tq / 128;
   const int n_kv_tiles = cdiv(n_keys, 128);
-  int splits = std::max(1, std::min(16, sms / (m_tiles * n_kv_heads)));
+  int splits = std::max(1, std::min(kMaxAttnSplits, sms / (m_tiles * n_kv_heads)));
   splits = std::min(splits, n_kv_tiles);
   const int tps = cdiv(n_kv_tiles, splits);
   splits = cdiv(n_kv_tiles, tps);
@@ -1266,13 +1285,10 @@ int dg_canvas_attention(const void* d_q, const void* d_k, const void* d_vt, void
   a.done = nullptr;
   cudaStream_t st = S(stream);
   DG_CUDA(cudaMemsetAsync(a.err, 0, 4, st));
+  a.o = static_cast<__nv_bfloat16*>(d_o);
   DG_TRY(set_smem(attention_kernel, kAttnSmemBytes));
-  DG_TRY(launch_pdl(attention_kernel, dim3(m_tiles, n_kv_heads, splits), dim3(kAttnThreads),
-                    kAttnSmemBytes, st, tq_m, tk_m, tv_m, a));
-  DG_LAUNCHED();
-  DG_TRY(launch_pdl(attn_combine_kernel<__nv_bfloat16>, dim3(cdiv(t * n_heads, 8)), dim3(256), 0, st,
-                    a.o_part, a.ml_part, splits, n_heads, tq, t, static_cast<__nv_bfloat16*>(d_o),
-                    nullptr));
+  DG_TRY(launch_pdl_cluster(attention_kernel, dim3(m_tiles, n_kv_heads, splits), dim3(kAttnThreads),
+                            kAttnSmemBytes, st, dim3(1, 1, splits), tq_m, tk_m, tv_m, a));
   DG_LAUNCHED();
   return DG_OK;
 }
