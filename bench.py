@@ -34,9 +34,10 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 PROMPT, BLOCKS, FIXED_STEPS, CANVAS = 4096, 4, 16, 256
+PREFILL_CHUNK = 1024  # prompt tokens per causal-encode pass
 WORKLOAD = ("full block decode: 30-layer MoE decoder (d 2816, 16/8 heads x 128, 128 experts "
             "top-8 x 704 + shared 2112, vocab 262144, bf16, random init), 4096-token prompt "
-            "prefilled, 4 canvases x 256 tokens x 16 fixed denoise steps")
+            "prefilled in 1024-token passes, 4 canvases x 256 tokens x 16 fixed denoise steps")
 
 
 def parse():
@@ -279,7 +280,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     shape = SHAPES["a4b"]
     cap = PROMPT + BLOCKS * CANVAS + CANVAS
-    cfg = make_config(shape, kv_capacity=cap, fixed_steps=FIXED_STEPS)
+    cfg = make_config(shape, kv_capacity=cap, fixed_steps=FIXED_STEPS, prefill_chunk=PREFILL_CHUNK)
     weights = model_weights("a4b", seed=1000 + rank, device=dev)
     model = DiffusionModel(cfg, weights, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -352,10 +353,15 @@ def run_ours(args, rank, world, local_rank):
     avg_ms = sum(durs) / max(1, len(durs))
     hbm, tf_burst, tf_sust, src = peaks()
     d, e, h, k = shape["d_model"], shape["n_experts"], shape["expert_hidden"], shape["top_k"]
+    hs = shape["shared_hidden"]
     slots = CANVAS * k
-    algo = {  # algorithmic bytes per launch (all 128 experts are routed at these shapes)
-        "expert_gate_up": e * 2 * h * d * 2 + slots * d * 2 + slots * h * 2,
-        "expert_down": e * d * h * 2 + slots * h * 2 + slots * d * 4,
+    # algorithmic bytes per launch: every routed expert's weights (all 128 are routed at these
+    # shapes) and the shared expert's, which rides in the same launch, plus tokens in and out
+    algo = {
+        "expert_gate_up": (e * 2 * h + 2 * hs) * d * 2 + (slots + CANVAS) * d * 2
+                          + slots * h * 2 + CANVAS * hs * 2,
+        "expert_down": (e * h + hs) * d * 2 + slots * h * 2 + CANVAS * hs * 2
+                       + (slots + CANVAS) * d * 4,
         "lm_head": shape["vocab"] * d * 2 + CANVAS * d * 2 + CANVAS * (shape["vocab"] // 256) * 16,
     }
     roof = None
@@ -453,6 +459,7 @@ def run_profile(args):
         if args.profile == "decode_step_small":
             shape.update(n_layers=2, vocab=32768)
         cfg = dg.make_config(shape, kv_capacity=PROMPT + BLOCKS * CANVAS + CANVAS,
+                             prefill_chunk=PREFILL_CHUNK,
                              fixed_steps=FIXED_STEPS)
         model = dg.DiffusionModel(cfg, model_weights(shape, seed=1000, device=dev), device=dev)
         model.kv_append(uniform_ids(PROMPT, shape["vocab"], seed=0).to(dev))

@@ -25,7 +25,7 @@ class Config(C.Structure):
         ("vocab", C.c_int32), ("canvas", C.c_int32), ("kv_capacity", C.c_int32),
         ("dtype", C.c_int32), ("eps", C.c_float), ("rope_theta", C.c_float),
         ("tau", C.c_double), ("h_bound", C.c_double), ("max_steps", C.c_int32),
-        ("fixed_steps", C.c_int32),
+        ("fixed_steps", C.c_int32), ("prefill_chunk", C.c_int32),
     ]
 
 

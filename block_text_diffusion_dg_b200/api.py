@@ -32,7 +32,7 @@ def _need_cuda(t, name, dtype=None):
 
 
 def make_config(shape, *, kv_capacity, fixed_steps=16, max_steps=48, tau=0.9, h_bound=0.005,
-                eps=1e-6, rope_theta=10000.0):
+                eps=1e-6, rope_theta=10000.0, prefill_chunk=0):
     s = shape
     return L.Config(
         n_layers=s["n_layers"], d_model=s["d_model"], n_heads=s["n_heads"],
@@ -41,7 +41,7 @@ def make_config(shape, *, kv_capacity, fixed_steps=16, max_steps=48, tau=0.9, h_
         vocab=s["vocab"], canvas=s["canvas"], kv_capacity=kv_capacity,
         dtype=L.DTYPE_FP32 if s["storage"] == "fp32" else L.DTYPE_BF16, eps=eps,
         rope_theta=rope_theta, tau=tau, h_bound=h_bound, max_steps=max_steps,
-        fixed_steps=fixed_steps)
+        fixed_steps=fixed_steps, prefill_chunk=prefill_chunk)
 
 
 def workspace_bytes(cfg):

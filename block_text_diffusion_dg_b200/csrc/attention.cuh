@@ -26,6 +26,7 @@ namespace dg {
 struct AttnParams {
   int group;          // Hq / Hkv
   int tq;             // query rows per head in the Q buffer (multiple of 128)
+  int tiles_per_head; // 128-row query tiles per head in use (ceil(n_queries / 128))
   int n_queries;      // valid tokens per head
   int n_keys;         // keys in use
   int causal_prefix;  // < 0: no mask
@@ -118,8 +119,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int mt = blockIdx.x;  // query tile inside the kv group
   const int g = blockIdx.y;   // kv head
   const int split = blockIdx.z;
-  const int head = g * p.group + (mt * 128) / p.tq;
-  const int tok0 = (mt * 128) % p.tq;
+  const int head = g * p.group + mt / p.tiles_per_head;
+  const int tok0 = (mt % p.tiles_per_head) * 128;
   const int n_kv_tiles = (p.n_keys + 127) >> 7;
   int tile_end = n_kv_tiles;
   if (p.causal_prefix >= 0) tile_end = min(tile_end, (p.causal_prefix + tok0 + 127) / 128 + 1);

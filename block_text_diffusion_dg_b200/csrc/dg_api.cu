@@ -284,7 +284,7 @@ struct dg_ctx {
   int esz;          // bytes per stored element (2 or 4)
   int tq;           // query rows per head in the Q buffer
   int qkv_rows;
-  int split_qkv, split_o, split_r;
+  int split_r;  // cluster size of the router projection
   int att_splits_max;
   size_t part_elems;
   // scratch views
@@ -338,6 +338,8 @@ int check_config(const dg_config* c) {
   if (c->vocab % 8 != 0) return fail(DG_ERR_UNSUPPORTED, "vocab must be a multiple of 8");
   if (c->max_steps < 1 || c->fixed_steps < 0)
     return fail(DG_ERR_INVALID_ARG, "max_steps must be >= 1 and fixed_steps >= 0");
+  if (c->prefill_chunk < 0 || c->prefill_chunk % 128 != 0 || c->prefill_chunk > 4096)
+    return fail(DG_ERR_INVALID_ARG, "prefill_chunk must be 0 or a multiple of 128, <= 4096");
   if (c->dtype == DG_DTYPE_BF16) {
     if (c->head_dim != 128) return fail(DG_ERR_UNSUPPORTED, "bf16 path needs head_dim 128");
     if (c->d_model % 64 || c->expert_hidden % 64 || c->shared_hidden % 64)
@@ -368,32 +370,33 @@ enum Buf {
 };
 
 struct Derived {
-  int tq, qkv_rows, split_qkv, split_o, split_r, att_splits, esz;
+  int tq, qkv_rows, split_r, att_splits, esz;
   size_t part_elems;
   long long max_chunks;
 };
+
+// Most tokens one forward pass carries: a canvas, or a prefill chunk of the prompt.
+int tokens_max(const dg_config& c) { return std::max(c.canvas, c.prefill_chunk); }
 
 Derived derive(const dg_config& c, int sms) {
   Derived d{};
   const bool bf16 = c.dtype == DG_DTYPE_BF16;
   d.esz = bf16 ? 2 : 4;
-  d.tq = bf16 ? 256 : c.canvas;
+  const long long T = tokens_max(c);
+  d.tq = bf16 ? std::max(256, cdiv(static_cast<int>(T), 128) * 128) : static_cast<int>(T);
   d.qkv_rows = (c.n_heads + 2 * c.n_kv_heads) * c.head_dim;
-  const long long T = c.canvas;
   if (bf16) {
-    // cluster sizes of the split-K projections (their partials never leave the cluster)
-    d.split_qkv = clu_splits(cdiv(d.qkv_rows, 128), c.d_model / 64, sms);
-    d.split_o = clu_splits(cdiv(c.d_model, 128), c.n_heads * c.head_dim / 64, sms);
+    // cluster size of the router projection (QKV and O pick theirs per call)
     d.split_r = std::min(kCluMaxSplits, c.d_model / 64);
     d.part_elems = 1;
   } else {
-    d.split_qkv = d.split_o = d.split_r = 1;
+    d.split_r = 1;
     d.part_elems = std::max({static_cast<size_t>(T) * d.qkv_rows,
                              static_cast<size_t>(T) * c.d_model,
                              static_cast<size_t>(T) * c.n_experts});
   }
   const int group = c.n_heads / c.n_kv_heads;
-  const int m_tiles = group * d.tq / 128;
+  const int m_tiles = group * cdiv(c.canvas, 128);  // the most splits are taken by a canvas
   d.att_splits = std::max(1, std::min(kMaxAttnSplits, sms / std::max(1, m_tiles * c.n_kv_heads)));
   d.max_chunks = c.n_experts + (T * c.top_k + kGroupN - 1) / kGroupN;
   return d;
@@ -403,15 +406,16 @@ Plan plan(const dg_config& c, int sms) {
   Plan p{};
   const Derived dv = derive(c, sms);
   const bool bf16 = c.dtype == DG_DTYPE_BF16;
-  const size_t T = c.canvas, d = c.d_model, E = c.n_experts, k = c.top_k, es = dv.esz;
+  const size_t Tc = c.canvas, T = tokens_max(c), d = c.d_model, E = c.n_experts, k = c.top_k,
+               es = dv.esz;
   const size_t hd = c.head_dim, Hq = c.n_heads;
   const size_t nv = bf16 ? c.vocab / 256 : cdiv(c.vocab, 4096);
   size_t sz[B_END];
-  sz[B_CANVAS] = sz[B_ARGMAX] = sz[B_PREV] = sz[B_LOCKED] = T * 4;
+  sz[B_CANVAS] = sz[B_ARGMAX] = sz[B_PREV] = sz[B_LOCKED] = Tc * 4;
   sz[B_STATE] = kStWords * 4;
   sz[B_TICKET] = sz[B_ERR] = 4;
-  sz[B_ENT] = sz[B_CONF] = T * 4;
-  sz[B_ROWH] = T * 8;
+  sz[B_ENT] = sz[B_CONF] = Tc * 4;
+  sz[B_ROWH] = Tc * 8;
   sz[B_X] = T * d * 4;
   sz[B_XN] = T * d * es;
   sz[B_PART] = dv.part_elems * 4;
@@ -431,8 +435,8 @@ Plan plan(const dg_config& c, int sms) {
   sz[B_HS] = bf16 ? T * std::max<size_t>(1, c.shared_hidden) * es : 0;
   sz[B_YSLOT] = T * k * d * 4;
   sz[B_YSH] = T * d * 4;
-  sz[B_LMPART] = T * nv * sizeof(StatPartial);
-  sz[B_LOGITS] = bf16 ? 0 : T * c.vocab * 4;
+  sz[B_LMPART] = Tc * nv * sizeof(StatPartial);
+  sz[B_LOGITS] = bf16 ? 0 : Tc * c.vocab * 4;
   sz[B_ROPE] = static_cast<size_t>(c.kv_capacity) * (hd / 2) * 8;
   size_t o = 0;
   for (int b = 0; b < B_END; ++b) {
@@ -557,7 +561,9 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
   // QKV projection (cluster split-K) with RoPE, Q and the K / V^T cache writes in its epilogue
   {
     const size_t kv_head_elems = static_cast<size_t>(g.kv_capacity) * hd;
-    CluParams p = clu_params(c->qkv_rows, n, d / 64, c->split_qkv, c->err, done);
+    CluParams p = clu_params(c->qkv_rows, n, d / 64,
+                             clu_splits(cdiv(c->qkv_rows, 128) * cdiv(n, 256), d / 64, c->sms),
+                             c->err, done);
     p.n_heads = g.n_heads;
     p.n_kv_heads = g.n_kv_heads;
     p.tq = c->tq;
@@ -572,7 +578,8 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
   // attention over [cache 0..pos0 | new tokens], split over keys
   {
     const int group = g.n_heads / g.n_kv_heads;
-    const int m_tiles = group * c->tq / 128;
+    const int tph = cdiv(n, 128);  // query tiles per head in use
+    const int m_tiles = group * tph;
     const int n_kv_tiles = cdiv(n_keys, 128);
     int splits = std::max(1, std::min(c->att_splits_max, c->sms / (m_tiles * g.n_kv_heads)));
     splits = std::min(splits, n_kv_tiles);
@@ -581,6 +588,7 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     AttnParams a{};
     a.group = group;
     a.tq = c->tq;
+    a.tiles_per_head = tph;
     a.n_queries = n;
     a.n_keys = n_keys;
     a.causal_prefix = causal ? pos0 : -1;
@@ -606,7 +614,9 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
   }
   // O projection onto the residual stream (cluster split-K), then the ffn norm
   {
-    CluParams p = clu_params(d, n, g.n_heads * hd / 64, c->split_o, c->err, done);
+    CluParams p = clu_params(d, n, g.n_heads * hd / 64,
+                             clu_splits(cdiv(d, 128) * cdiv(n, 256), g.n_heads * hd / 64, c->sms),
+                             c->err, done);
     p.x = c->x;
     DG_TRY(launch_cluster<kCluResidual>(c->tm_wo[l], c->tm_o32, p, st, DG_KERNEL_O_PROJ));
     prof_before(DG_KERNEL_RESIDUAL_NORM, st);
@@ -738,7 +748,7 @@ int run_lm_head(dg_ctx* c, float* logits_out, const int* done, cudaStream_t st) 
 
 int bind_tmaps(dg_ctx* c) {
   const dg_config& g = c->cfg;
-  const uint64_t T = g.canvas, d = g.d_model, hd = g.head_dim, k = g.top_k;
+  const uint64_t T = tokens_max(g), d = g.d_model, hd = g.head_dim, k = g.top_k;
   DG_TRY(make_tmap(&c->tm_xn32, c->xn, T, d, d, 32));
   DG_TRY(make_tmap(&c->tm_xn128, c->xn, T, d, d, 128));
   DG_TRY(make_tmap(&c->tm_o32, c->o, T, g.n_heads * hd, g.n_heads * hd, 32));
@@ -853,8 +863,6 @@ int dg_create(const dg_config* cfg, const dg_weights* w, void* d_kv, void* d_scr
   c->esz = dv.esz;
   c->tq = dv.tq;
   c->qkv_rows = dv.qkv_rows;
-  c->split_qkv = dv.split_qkv;
-  c->split_o = dv.split_o;
   c->split_r = dv.split_r;
   c->att_splits_max = dv.att_splits;
   c->part_elems = dv.part_elems;
@@ -942,8 +950,9 @@ int dg_kv_append(dg_ctx* ctx, const int32_t* d_ids, int32_t n, void* stream) {
     return fail(DG_ERR_CAPACITY, "cache of %d positions cannot take %d more plus a canvas of %d",
                 ctx->cfg.kv_capacity, ctx->kv_len + n, ctx->cfg.canvas);
   cudaStream_t st = S(stream);
-  for (int off = 0; off < n; off += ctx->cfg.canvas) {
-    const int m = std::min(ctx->cfg.canvas, n - off);
+  const int chunk = ctx->cfg.prefill_chunk > 0 ? ctx->cfg.prefill_chunk : ctx->cfg.canvas;
+  for (int off = 0; off < n; off += chunk) {
+    const int m = std::min(chunk, n - off);
     DG_TRY(run_forward(ctx, d_ids + off, m, ctx->kv_len, 1, nullptr, st));
     ctx->kv_len += m;
   }
@@ -1250,7 +1259,8 @@ int dg_canvas_attention(const void* d_q, const void* d_k, const void* d_vt, void
     return fail(DG_ERR_INVALID_ARG, "causal prefix + queries exceeds keys");
   const int sms = num_sms();
   const int group = n_heads / n_kv_heads;
-  const int m_tiles = group * tq / 128;
+  const int tph = cdiv(t, 128);  // query tiles per head in use
+  const int m_tiles = group * tph;
   const int n_kv_tiles = cdiv(n_keys, 128);
   int splits = std::max(1, std::min(kMaxAttnSplits, sms / (m_tiles * n_kv_heads)));
   splits = std::min(splits, n_kv_tiles);
@@ -1269,6 +1279,7 @@ int dg_canvas_attention(const void* d_q, const void* d_k, const void* d_vt, void
   AttnParams a{};
   a.group = group;
   a.tq = tq;
+  a.tiles_per_head = tph;
   a.n_queries = t;
   a.n_keys = n_keys;
   a.causal_prefix = causal_prefix;

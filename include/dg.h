@@ -82,6 +82,9 @@ typedef struct dg_config {
   double h_bound;         /* mean-entropy stop bound in nats (0.005, [canvas] step 3) */
   int32_t max_steps;      /* adaptive step cap (48, [canvas] step 3) */
   int32_t fixed_steps;    /* > 0: fixed-step mode, exactly this many steps; 0: adaptive */
+  int32_t prefill_chunk;  /* tokens per causal-encode pass of dg_kv_append (0 = canvas); a
+                             multiple of 128, <= 4096; larger chunks stream the weights fewer
+                             times per prompt at the cost of scratch memory */
 } dg_config;
 
 /* Per-layer weights, all device pointers, dtype = config dtype unless noted.

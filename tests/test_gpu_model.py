@@ -185,3 +185,38 @@ def test_small_bf16_prefill_denoise_commit():
     torch.cuda.synchronize()
     assert st2.cpu().tolist()[:2] == [1, 3] and m.kv_length == 320 + 512
     m.check_device_status()
+
+
+def test_small_bf16_prefill_in_large_chunks():
+    """The prompt encoded in 512-token passes (the last one ragged) gives the cache the oracle's
+    chunk-invariant causal encode gives, and a denoise step on top of it (query buffer sized for
+    the larger pass) matches the oracle layer by layer."""
+    from block_text_diffusion_dg_b200 import DiffusionModel, make_config
+    shape = SHAPES["small_bf16"]
+    w = model_weights("small_bf16", seed=3, norm_jitter=0.1)
+    prompt = uniform_ids(640, shape["vocab"], seed=4)  # 512 + ragged 128
+    cfg = make_config(shape, kv_capacity=1024, fixed_steps=2, prefill_chunk=512)
+    m = DiffusionModel(cfg, _to_cuda(w))
+    ocfg, ow = _ocfg("small_bf16"), weights_to_np(w)
+    ocache = om.causal_encode(ocfg, ow, prompt.numpy(), om.KVCache())
+    m.kv_append(prompt.cuda())
+    assert m.kv_length == 640
+    k_gpu, vt_gpu = _kv_views(m, cfg)
+    torch.cuda.synchronize()
+    for l in range(cfg.n_layers):
+        ok, frac = _tokenwise_close(np64(k_gpu[l, :, :640]), ocache.k[l], 2e-2, 0.98 if l else 1.0)
+        assert ok, ("prefill K", l, frac)
+        ok, frac = _tokenwise_close(np64(vt_gpu[l, :, :, :640]).transpose(0, 2, 1), ocache.v[l], 2e-2,
+                                    0.98 if l else 1.0)
+        assert ok, ("prefill V", l, frac)
+    m.canvas_init(5, 0)
+    m.denoise_step(1)
+    m.sample_update(1)
+    torch.cuda.synchronize()
+    canvas0 = osmp.canvas_init(5, 0, 256, shape["vocab"])
+    x = np.asarray(ow["embed"], dtype=np.float64)[canvas0]
+    att, moe, frac = check_layer_parts(m, ocfg, ow["layers"][0], x, 640 + np.arange(256),
+                                       ocache.k[0], ocache.v[0], 0, shape["top_k"])
+    assert att[0] and att[2] < 5e-3, ("attention half", att)
+    assert moe[0] and moe[2] < 5e-3, ("moe half", moe)
+    m.check_device_status()
