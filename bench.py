@@ -34,10 +34,10 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 PROMPT, BLOCKS, FIXED_STEPS, CANVAS = 4096, 4, 16, 256
-PREFILL_CHUNK = 1024  # prompt tokens per causal-encode pass
+PREFILL_CHUNK = 4096  # prompt tokens per causal-encode pass (the whole prompt)
 WORKLOAD = ("full block decode: 30-layer MoE decoder (d 2816, 16/8 heads x 128, 128 experts "
             "top-8 x 704 + shared 2112, vocab 262144, bf16, random init), 4096-token prompt "
-            "prefilled in 1024-token passes, 4 canvases x 256 tokens x 16 fixed denoise steps")
+            "prefilled in one pass, 4 canvases x 256 tokens x 16 fixed denoise steps")
 
 
 def parse():

@@ -351,23 +351,38 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tc_fence_after();
     const float l_tot = l_run + tmem_ld1(xchg + 4 + (1 - half));
     const long long row = (static_cast<long long>(split) * p.n_heads + head) * p.tq + tok;
-    float4* dst = reinterpret_cast<float4*>(p.o_part + row * 128 + 64 * half);
-    const bool have_o = ok && n_tiles > 0 &&
-                        mbar_wait(&pv_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, p.err);
+    const bool have_o =
+        __all_sync(0xffffffffu, ok && n_tiles > 0 &&
+                                    mbar_wait(&pv_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1,
+                                              p.err));
+    // the warp's 32 half rows (256 bytes each) go through shared memory so that every store to
+    // o_part writes whole 256-byte half rows.  Staging: the K ring, idle once the last P V is
+    // done; warp region (warp - 2) * 8 KB, row i at i * 256, 16-byte unit c at (c ^ (i % 16)).
+    uint8_t* stage = s_k + (warp - 2) * 8192;
+    const int lane = lane_id();
     if (have_o) {
       tc_fence_after();
-#pragma unroll
+#pragma unroll 1
       for (int c = 0; c < 2; ++c) {
         float v[32];
         tmem_ld32(tmem_base + 64 * half + 32 * c + lane_off, v);
-        if (tok < p.n_queries) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            dst[c * 8 + i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-        }
+        for (int i = 0; i < 8; ++i)
+          *reinterpret_cast<float4*>(stage + lane * 256 + (((c * 8 + i) ^ (lane & 15)) << 4)) =
+              make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
       }
-    } else if (tok < p.n_queries) {
-      for (int i = 0; i < 16; ++i) dst[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    __syncwarp();
+    const int tok_w = tok - lane;  // token of the warp's row 0
+    const long long row_w = row - lane;
+    for (int i0 = 0; i0 < 32; i0 += 2) {
+      const int i = i0 + (lane >> 4), c = lane & 15;
+      if (tok_w + i < p.n_queries) {
+        const float4 val =
+            have_o ? *reinterpret_cast<const float4*>(stage + i * 256 + ((c ^ (i & 15)) << 4))
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
+        reinterpret_cast<float4*>(p.o_part + (row_w + i) * 128 + 64 * half)[c] = val;
+      }
     }
     if (tok < p.n_queries && half == 0)
       p.ml_part[row] = have_o ? make_float2(m_run, l_tot) : make_float2(-INFINITY, 0.f);

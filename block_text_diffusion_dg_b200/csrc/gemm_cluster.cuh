@@ -30,12 +30,13 @@ constexpr int kCluBBytes = 256 * 128;           // 256 tokens x 64 bf16
 constexpr int kCluStageBytes = kCluABytes + kCluBBytes;
 constexpr int kCluRingBytes = kCluStages * kCluStageBytes;  // 192 KB, reused by the epilogue
 constexpr int kCluDrainBytes = 256 * 128 * 4;   // fp32 [token][row] partial tile
-constexpr int kCluSmemBytes = kCluRingBytes + 1024 + 256;
+// ring, 1 KB that lets the V^T scratch overhang the ring, alignment slack, barriers
+constexpr int kCluSmemBytes = kCluRingBytes + 1024 + 1024 + 256;
 constexpr int kCluThreads = 64 + 32 * 8;
 constexpr int kCluMaxSplits = 8;
 // epilogue scratch after the drained tile: a V^T tile [128][<= 256 tokens] bf16, or the router
 // logits of <= 128 tokens [token][128] fp32
-static_assert(kCluDrainBytes + 128 * 256 * 2 <= kCluRingBytes, "V^T scratch");
+static_assert(kCluDrainBytes + 128 * 257 * 2 <= kCluRingBytes + 1024, "V^T scratch");
 static_assert(kCluDrainBytes + 128 * 128 * 4 <= kCluRingBytes, "router scratch");
 
 struct CluParams {
@@ -66,6 +67,36 @@ struct CluParams {
   const int* done;
 };
 
+// Sums over the S cluster ranks of G row groups (token t[g0 + g], rows 4 r4[g0 + g] ..) of the
+// drained partial tiles, in rank order, with every load issued before the first add.
+template <int G, int SMAX>
+DG_DEV void reduce_groups(uint32_t drain_u32, int S, const int (&t)[4], const int (&r4)[4], int g0,
+                          float4 (&out)[4]) {
+  float4 v[G][SMAX];
+#pragma unroll
+  for (int src = 0; src < SMAX; ++src)
+    if (src < S) {
+#pragma unroll
+      for (int g = 0; g < G; ++g)
+        v[g][src] = dsmem_ld4(dsmem_addr(
+            drain_u32 + static_cast<uint32_t>((t[g0 + g] * 128 + 4 * r4[g0 + g]) * 4),
+            static_cast<uint32_t>(src)));
+    }
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int src = 0; src < SMAX; ++src)
+      if (src < S) {
+        acc.x += v[g][src].x;
+        acc.y += v[g][src].y;
+        acc.z += v[g][src].z;
+        acc.w += v[g][src].w;
+      }
+    out[g0 + g] = acc;
+  }
+}
+
 template <int EPI>
 __global__ void __launch_bounds__(kCluThreads, 1)
     gemm_cluster_kernel(const __grid_constant__ CUtensorMap tm_a,
@@ -73,7 +104,7 @@ __global__ void __launch_bounds__(kCluThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kCluRingBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kCluRingBytes + 1024);
   uint64_t* empty = full + kCluStages;
   uint64_t* acc_full = empty + kCluStages;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_full + 1);
@@ -232,45 +263,90 @@ __global__ void __launch_bounds__(kCluThreads, 1)
         b.w += vb[src].w;
       }
   };
+  // four row groups at once (token, row group) -> sums with all their loads in flight; the
+  // groups go two by two when the cluster is larger than four (register budget)
+  auto reduce4x4 = [&](const int (&t)[4], const int (&r4)[4], float4 (&out)[4]) {
+    if (S <= 4) {
+      reduce_groups<4, 4>(drain_u32, S, t, r4, 0, out);
+    } else {
+      reduce_groups<2, kCluMaxSplits>(drain_u32, S, t, r4, 0, out);
+      reduce_groups<2, kCluMaxSplits>(drain_u32, S, t, r4, 2, out);
+    }
+  };
   const int rows4 = min(32, (p.m_rows - mt * 128 + 3) >> 2);  // valid float4 row groups
   if constexpr (EPI == kCluResidual) {
     if (ok) {
-      for (int u = tid; u < nt * rows4; u += kCluThreads) {
-        const int t = t_lo + u / rows4, r4 = u % rows4;
-        const float4 sum = reduce4(t, r4);
-        float4* xp = reinterpret_cast<float4*>(p.x + static_cast<long long>(t0 + t) * p.m_rows +
-                                               mt * 128 + 4 * r4);
-        float4 a = *xp;
-        a.x += sum.x;
-        a.y += sum.y;
-        a.z += sum.z;
-        a.w += sum.w;
-        *xp = a;
+      // two units per pass: the residual rows and every partial in flight together
+      const int total = nt * rows4;
+      for (int u0 = tid; u0 < total; u0 += 2 * kCluThreads) {
+        int tt[4] = {0, 0, 0, 0}, rr[4] = {0, 0, 0, 0};
+        float4 xv[2];
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int u = min(u0 + k * kCluThreads, total - 1);
+          tt[k] = t_lo + u / rows4;
+          rr[k] = u % rows4;
+          xv[k] = *reinterpret_cast<const float4*>(
+              p.x + static_cast<long long>(t0 + tt[k]) * p.m_rows + mt * 128 + 4 * rr[k]);
+        }
+        float4 sum[4];
+        reduce_groups<2, kCluMaxSplits>(drain_u32, S, tt, rr, 0, sum);
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          if (u0 + k * kCluThreads >= total) break;
+          float4 a = xv[k];
+          a.x += sum[k].x;
+          a.y += sum[k].y;
+          a.z += sum[k].z;
+          a.w += sum[k].w;
+          *reinterpret_cast<float4*>(p.x + static_cast<long long>(t0 + tt[k]) * p.m_rows +
+                                     mt * 128 + 4 * rr[k]) = a;
+        }
       }
     }
   } else if constexpr (EPI == kCluQkv) {
     const int head = mt;  // 128 rows = one head
-    __nv_bfloat16* vt_s = reinterpret_cast<__nv_bfloat16*>(smem + kCluDrainBytes);  // [hd][nt]
+    // [hd][nt + 1]: the odd row pitch spreads a warp's stores (consecutive row groups) over banks
+    __nv_bfloat16* vt_s = reinterpret_cast<__nv_bfloat16*>(smem + kCluDrainBytes);
+    const int vp = nt + 1;
     if (head < p.n_heads + p.n_kv_heads) {
       if (ok) {
-        // rotate-half pairs (i, i + 64): float4 groups r4 and r4 + 16
-        for (int u = tid; u < nt * 16; u += kCluThreads) {
-          const int t = t_lo + u / 16, r4 = u % 16;
-          const int tg = t0 + t;
-          float4 a, b;
-          reduce4x2(t, r4, r4 + 16, a, b);
-          const float2* cs = p.rope_tab + static_cast<long long>(p.pos0 + tg) * 64 + 4 * r4;
-          const float2 c0 = cs[0], c1 = cs[1], c2 = cs[2], c3 = cs[3];
-          __nv_bfloat16* dst =
-              head < p.n_heads
-                  ? p.q + (static_cast<long long>(head) * p.tq + tg) * 128
-                  : p.k_cache + (static_cast<long long>(head - p.n_heads) * p.ldk + p.pos0 + tg) * 128;
-          const float lo[4] = {a.x * c0.x - b.x * c0.y, a.y * c1.x - b.y * c1.y,
-                               a.z * c2.x - b.z * c2.y, a.w * c3.x - b.w * c3.y};
-          const float hi[4] = {b.x * c0.x + a.x * c0.y, b.y * c1.x + a.y * c1.y,
-                               b.z * c2.x + a.z * c2.y, b.w * c3.x + a.w * c3.y};
-          store4<__nv_bfloat16>(dst + 4 * r4, make_float4(lo[0], lo[1], lo[2], lo[3]));
-          store4<__nv_bfloat16>(dst + 64 + 4 * r4, make_float4(hi[0], hi[1], hi[2], hi[3]));
+        // rotate-half pairs (i, i + 64): float4 groups r4 and r4 + 16; two units per pass so
+        // that their table and partial loads are all in flight together
+        for (int u0 = tid; u0 < nt * 16; u0 += 2 * kCluThreads) {
+          int tt[4], rr[4];
+          float2 cs[2][4];
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const int u = min(u0 + k * kCluThreads, nt * 16 - 1);
+            const int t = t_lo + u / 16, r4 = u % 16;
+            tt[2 * k] = tt[2 * k + 1] = t;
+            rr[2 * k] = r4;
+            rr[2 * k + 1] = r4 + 16;
+            const float2* tab = p.rope_tab + static_cast<long long>(p.pos0 + t0 + t) * 64 + 4 * r4;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) cs[k][i] = tab[i];
+          }
+          float4 sum[4];
+          reduce4x4(tt, rr, sum);
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            if (u0 + k * kCluThreads >= nt * 16) break;
+            const int tg = t0 + tt[2 * k], r4 = rr[2 * k];
+            const float4 a = sum[2 * k], b = sum[2 * k + 1];
+            __nv_bfloat16* dst =
+                head < p.n_heads
+                    ? p.q + (static_cast<long long>(head) * p.tq + tg) * 128
+                    : p.k_cache +
+                          (static_cast<long long>(head - p.n_heads) * p.ldk + p.pos0 + tg) * 128;
+            const float2 c0 = cs[k][0], c1 = cs[k][1], c2 = cs[k][2], c3 = cs[k][3];
+            const float lo[4] = {a.x * c0.x - b.x * c0.y, a.y * c1.x - b.y * c1.y,
+                                 a.z * c2.x - b.z * c2.y, a.w * c3.x - b.w * c3.y};
+            const float hi[4] = {b.x * c0.x + a.x * c0.y, b.y * c1.x + a.y * c1.y,
+                                 b.z * c2.x + a.z * c2.y, b.w * c3.x + a.w * c3.y};
+            store4<__nv_bfloat16>(dst + 4 * r4, make_float4(lo[0], lo[1], lo[2], lo[3]));
+            store4<__nv_bfloat16>(dst + 64 + 4 * r4, make_float4(hi[0], hi[1], hi[2], hi[3]));
+          }
         }
       }
     } else {
@@ -279,10 +355,10 @@ __global__ void __launch_bounds__(kCluThreads, 1)
         for (int u = tid; u < nt * 32; u += kCluThreads) {
           const int tl = u / 32, r4 = u % 32;
           const float4 a = reduce4(t_lo + tl, r4);
-          vt_s[(4 * r4 + 0) * nt + tl] = __float2bfloat16_rn(a.x);
-          vt_s[(4 * r4 + 1) * nt + tl] = __float2bfloat16_rn(a.y);
-          vt_s[(4 * r4 + 2) * nt + tl] = __float2bfloat16_rn(a.z);
-          vt_s[(4 * r4 + 3) * nt + tl] = __float2bfloat16_rn(a.w);
+          vt_s[(4 * r4 + 0) * vp + tl] = __float2bfloat16_rn(a.x);
+          vt_s[(4 * r4 + 1) * vp + tl] = __float2bfloat16_rn(a.y);
+          vt_s[(4 * r4 + 2) * vp + tl] = __float2bfloat16_rn(a.z);
+          vt_s[(4 * r4 + 3) * vp + tl] = __float2bfloat16_rn(a.w);
         }
       }
       __syncthreads();
@@ -291,7 +367,7 @@ __global__ void __launch_bounds__(kCluThreads, 1)
         for (int u = tid; u < 128 * nt; u += kCluThreads) {
           const int dd = u / nt, tl = u % nt;
           p.vt_cache[(static_cast<long long>(g) * 128 + dd) * p.ldk + p.pos0 + t0 + t_lo + tl] =
-              vt_s[dd * nt + tl];
+              vt_s[dd * vp + tl];
         }
       }
     }
