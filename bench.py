@@ -364,11 +364,15 @@ def run_ours(args, rank, world, local_rank):
                        + (slots + CANVAS) * d * 4,
         "lm_head": shape["vocab"] * d * 2 + CANVAS * d * 2 + CANVAS * (shape["vocab"] // 256) * 16,
     }
+    # DRAM bytes (read + write) of one launch from the ncu capture summarised in profiles/
+    # (dram__bytes_read.sum + dram__bytes_write.sum); None where no capture of the current kernel
+    traffic = {"expert_gate_up": 1051851000 + 4439808}
     roof = None
     if args.roofline_kernel in algo and rec:
         achieved = algo[args.roofline_kernel] / (avg_ms / 1e3) / 1e9
         roof = dict(kernel=args.roofline_kernel, bound="hbm", achieved=round(achieved, 1),
-                    peak=hbm, unit="GB/s", frac=round(achieved / hbm, 4), traffic=None,
+                    peak=hbm, unit="GB/s", frac=round(achieved / hbm, 4),
+                    traffic=traffic.get(args.roofline_kernel),
                     launches_timed=rec, avg_launch_us=round(avg_ms * 1e3, 2),
                     algorithmic_bytes_per_launch=algo[args.roofline_kernel],
                     peak_source=f"{src} (MEASURED_PEAKS.json hbm_gbs)")

@@ -50,6 +50,9 @@ def _case(t, d, e, k, h, hs, seed):
     (256, 512, 8, 2, 256, 384),      # the small test model's MoE
     (200, 512, 16, 4, 192, 256),     # ragged token count
     (256, 1024, 128, 8, 64, 128),    # many experts, many empty
+    (1100, 512, 16, 4, 128, 256),    # several router chunks; experts with several token chunks
+    (2048, 256, 128, 8, 64, 0),      # a long prompt pass: 16 384 routed slots
+    (4096, 256, 8, 2, 64, 0),        # the largest pass: routing over 4096 tokens
 ])
 def test_moe_small(t, d, e, k, h, hs):
     assert _case(t, d, e, k, h, hs, seed=t + d) > 0.95
