@@ -40,6 +40,12 @@ struct AttnParams {
   float* o_part;      // [splits, Hq, tq, 128]
   float2* ml_part;    // [splits, Hq, tq] (max in log2 units, denominator)
   __nv_bfloat16* o;   // [T, Hq * 128] merged output
+  // weights the next kernels stream (the shared expert's): prefetched into L2 while the
+  // attention, which hardly uses HBM, runs; null for none
+  const void* pf0;
+  long long pf0_bytes;
+  const void* pf1;
+  long long pf1_bytes;
   int* err;
   const int* done;
 };
@@ -194,6 +200,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (j + 1 < n_tiles) ok = load_k(j + 1);
         if (ok) ok = load_v(j);
       }
+      // every K / V load is issued: hint the next kernels' weights into L2 behind them
+      const int cta = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
+      const int n_cta = gridDim.x * gridDim.y * gridDim.z;
+      prefetch_l2_slice(p.pf0, p.pf0_bytes, cta, n_cta);
+      prefetch_l2_slice(p.pf1, p.pf1_bytes, cta, n_cta);
     }
   } else if (warp == 1) {
     if (elect_one() && n_tiles > 0) {

@@ -200,6 +200,7 @@ int launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 // ---- GEMM launch helpers -----------------------------------------------------------------
 constexpr int kGroupN = 64, kGroupStages = 8;
 constexpr int kRouterChunk = 64;  // tokens per router cluster
+constexpr int kPrefetchExperts = 4;  // routed chunks whose expert weights the gather prefetches
 
 // ta2/tb2 are read only by items of the alternate group (p.alt_group >= 0).
 template <int MAXN, int STAGES, int EPI>
@@ -602,6 +603,10 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     a.o_part = c->o_part;
     a.ml_part = c->ml_part;
     a.o = static_cast<__nv_bfloat16*>(c->o);
+    if (parts & 2 && g.shared_hidden > 0) {  // the shared expert's weights of this layer
+      a.pf0 = w.ws_gu;
+      a.pf0_bytes = 2ll * g.shared_hidden * d * 2;
+    }
     a.err = c->err;
     a.done = done;
     DG_TRY(set_smem(attention_kernel, kAttnSmemBytes));
@@ -644,9 +649,11 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
   // permutation gather and grouped expert GEMMs; the shared expert rides along as group E
   {
     prof_before(DG_KERNEL_GATHER, st);
-    DG_TRY(launch_pdl(gather_rows_kernel, dim3(cdiv(n_slots, 4)), dim3(256), 0, st, 
-        static_cast<const __nv_bfloat16*>(c->xn), c->perm, k, d, n_slots,
-        static_cast<__nv_bfloat16*>(c->x_perm), done));
+    const ExpertPrefetch epf{c->chunks, c->n_chunks, kPrefetchExperts, w.w_gu,
+                             2ll * g.expert_hidden * d * 2};
+    DG_TRY(launch_pdl(gather_rows_kernel, dim3(cdiv(n_slots, 4)), dim3(256), 0, st,
+                      static_cast<const __nv_bfloat16*>(c->xn), c->perm, k, d, n_slots,
+                      static_cast<__nv_bfloat16*>(c->x_perm), epf, done));
     DG_LAUNCHED();
     prof_after(DG_KERNEL_GATHER, st);
     GemmParams p{};
@@ -1405,8 +1412,10 @@ int dg_moe_ffn(const void* d_x, const float* d_residual, const void* d_wr, const
   pr.route = RouteArgs{ids, t, top_k, n_experts, kGroupN, offs, perm, chunks, icnt};
   pr.ticket = route_ticket;
   DG_TRY(launch_cluster<kCluRouter>(t_wr, t_x32, pr, st, -1));
-  DG_TRY(launch_pdl(gather_rows_kernel, dim3(cdiv(t * top_k, 4)), dim3(256), 0, st, static_cast<const __nv_bfloat16*>(d_x),
-                                                         perm, top_k, d, t * top_k, x_perm, nullptr));
+  DG_TRY(launch_pdl(gather_rows_kernel, dim3(cdiv(t * top_k, 4)), dim3(256), 0, st,
+                    static_cast<const __nv_bfloat16*>(d_x), perm, top_k, d, t * top_k, x_perm,
+                    ExpertPrefetch{chunks, icnt, kPrefetchExperts, d_w_gu, 2ll * hidden * d * 2},
+                    nullptr));
   DG_LAUNCHED();
   GemmParams pg{};
   pg.chunks = chunks;

@@ -113,6 +113,21 @@ DG_DEV void tma_load_2d(const CUtensorMap* map, uint64_t* bar, void* dst, int32_
       : "memory");
 }
 
+// Hint: bring [p, p + bytes) into L2 (p 16-byte aligned, bytes a multiple of 16).
+DG_DEV void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)),
+               "r"(bytes)
+               : "memory");
+}
+// Part `part` of `parts` equal slices of a region, prefetched into L2 in 64 KB pieces.
+DG_DEV void prefetch_l2_slice(const void* base, long long bytes, int part, int parts) {
+  if (base == nullptr || bytes <= 0) return;
+  const long long lo = (bytes * part / parts) & ~15ll, hi = (bytes * (part + 1) / parts) & ~15ll;
+  const uint8_t* b = static_cast<const uint8_t*>(base);
+  for (long long o = lo; o < hi; o += 65536)
+    prefetch_l2_bulk(b + o, static_cast<uint32_t>(min(65536ll, hi - o)));
+}
+
 // Order generic-proxy shared-memory writes before async-proxy (UMMA/TMA) reads.
 DG_DEV void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

@@ -382,14 +382,33 @@ DG_DEV void route_canvas(const RouteArgs& a, int* sm) {
                                            min(a.n_chunk, count_s[e] - c * a.n_chunk), 0);
 }
 
+// Weights of the first routed chunks' experts, prefetched into L2 by the gather (the grouped
+// GEMM reads them first): chunk c < n_first of the chunk list, `expert_bytes` per expert at w.
+struct ExpertPrefetch {
+  const int4* chunks;
+  const int* n_chunks;
+  int n_first;
+  const void* w;
+  long long expert_bytes;
+};
+
 // x_perm[p] = xn[perm[p] / k]; 64 threads per permuted row, 4 rows per CTA, 16-byte copies.
 __global__ void __launch_bounds__(256) gather_rows_kernel(const __nv_bfloat16* __restrict__ xn,
                                                           const int32_t* __restrict__ perm,
                                                           int top_k, int d, int n_rows,
                                                           __nv_bfloat16* __restrict__ x_perm,
-                                                          const int* done) {
+                                                          ExpertPrefetch pf, const int* done) {
   pdl_enter();
   if (block_done(done)) return;
+  if (threadIdx.x == 0 && pf.w != nullptr && pf.n_first > 0) {
+    const int nf = min(pf.n_first, *pf.n_chunks);
+    if (nf > 0 && static_cast<int>(gridDim.x) >= nf) {
+      const int c = blockIdx.x % nf, parts = gridDim.x / nf, part = blockIdx.x / nf;
+      if (part < parts)
+        prefetch_l2_slice(static_cast<const uint8_t*>(pf.w) + pf.chunks[c].x * pf.expert_bytes,
+                          pf.expert_bytes, part, parts);
+    }
+  }
   const int p = blockIdx.x * 4 + (threadIdx.x >> 6);
   if (p >= n_rows) return;
   const int t = perm[p] / top_k;
