@@ -674,6 +674,10 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     p.alt_m_valid = 2 * g.shared_hidden;
     p.alt_out_bf16 = static_cast<__nv_bfloat16*>(c->hs);
     p.alt_ld_out = g.shared_hidden;
+    if (shared) {  // the down GEMM starts with the shared expert's items
+      p.pf0 = w.ws_d;
+      p.pf0_bytes = static_cast<long long>(d) * g.shared_hidden * 2;
+    }
     p.err = c->err;
     p.done = done;
     DG_TRY((launch_gemm<kGroupN, kGroupStages, kEpiGluBf16>(
@@ -699,6 +703,16 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     q.alt_m_valid = d;
     q.alt_out_f32 = c->y_shared;
     q.alt_ld_out = d;
+    if (l + 1 < g.n_layers) {  // the next layer's QKV and O projections
+      const dg_layer_weights& wn = c->layers[l + 1];
+      q.pf0 = wn.wqkv;
+      q.pf0_bytes = static_cast<long long>(c->qkv_rows) * d * 2;
+      q.pf1 = wn.wo;
+      q.pf1_bytes = static_cast<long long>(d) * g.n_heads * hd * 2;
+    } else {  // the first vocabulary tiles of the LM head
+      q.pf0 = c->embed;
+      q.pf0_bytes = std::min<long long>(64ll << 20, static_cast<long long>(g.vocab) * d * 2);
+    }
     q.err = c->err;
     q.done = done;
     DG_TRY((launch_gemm<kGroupN, kGroupStages, kEpiScatterF32>(

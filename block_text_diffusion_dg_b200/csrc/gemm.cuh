@@ -51,6 +51,12 @@ struct GemmParams {
   float* alt_out_f32;
   __nv_bfloat16* alt_out_bf16;
   long long alt_ld_out;
+  // weights of the kernels that follow, hinted into L2 by each CTA's producer once its items are
+  // all issued (the last wave leaves HBM idle); null for none
+  const void* pf0;
+  long long pf0_bytes;
+  const void* pf1;
+  long long pf1_bytes;
   int* err;
   const int* done;
 };
@@ -261,6 +267,8 @@ __global__ void __launch_bounds__(GemmCfg<MAXN, STAGES>::kThreads, 1)
           }
         }
       }
+      prefetch_l2_slice(p.pf0, p.pf0_bytes, blockIdx.x, gridDim.x);
+      prefetch_l2_slice(p.pf1, p.pf1_bytes, blockIdx.x, gridDim.x);
     }
   } else if (warp == 1) {
     if (elect_one()) {
