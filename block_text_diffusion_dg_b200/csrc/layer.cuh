@@ -1,13 +1,15 @@
 // layer.cuh -- the non-GEMM kernels of one decoder layer (bandwidth-bound, one pass each).
 //
 //   embed_norm        x = E[ids] (fp32 residual), xn = rmsnorm(x) * w        (a1, a2)
-//   qkv_finalize      sum split-K partials; rotate-half RoPE at absolute positions for q and
-//                     k heads (Q [Hq, Tq, hd], K cache slots P..P+n-1); V stored transposed
-//                     into V^T [hd, cap]                                       (a3)
-//   residual_norm     x += O-projection partials; xn2 = rmsnorm(x) * w         (a5, a2)
-//   router_topk       router logits -> top-k ids (lowest index on ties) and the softmax of
+//   qkv_finalize      (all-fp32 path) sum of partials; rotate-half RoPE at absolute positions
+//                     for q and k heads (Q [Hq, Tq, hd], K cache slots P..P+n-1); V stored
+//                     transposed into V^T [hd, cap]                            (a3)
+//   residual_norm     x += partials (none on the bf16 path, whose O projection adds into x
+//                     itself); xn2 = rmsnorm(x) * w                             (a5, a2)
+//   router_topk_*     router logits -> top-k ids (lowest index on ties) and the softmax of
 //                     the selected logits (= renormalised full-softmax probabilities) (a6)
-//   moe_route         per-expert counts, offsets, stable slot order, grouped GEMM item lists (a7)
+//   route_canvas      per-expert token bitmasks -> offsets, stable slot order, the token-chunk
+//                     list of the grouped GEMMs (run by the router kernel's last CTA)  (a7)
 //   gather_rows       x_perm[p] = xn2[token of slot perm[p]]                   (a7)
 //   moe_combine_norm  x += sum over slots in order of y_slot + y_shared; xn = rmsnorm(x) * w
 //                     for the next layer (or the final norm)                  (a9, a2)

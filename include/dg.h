@@ -226,7 +226,10 @@ DG_API int dg_canvas_attention(const void* d_q, const void* d_k, const void* d_v
  * optional shared expert ws_gu [2hs, d], ws_d [d, hs] (NULL, hs = 0 for none).
  * y fp32 [T, d] = (residual or 0) + sum over slots in order of w * expert(x) + shared(x).
  * Router: softmax over all E, top-k lowest index on ties, weights renormalised over k.
- * Optional outputs: ids int32 [T, k], weights fp32 [T, k], router logits fp32 [T, E]. */
+ * Optional outputs: ids int32 [T, k], weights fp32 [T, k], router logits fp32 [T, E].
+ * Shapes: 1 <= T <= 4096; d a multiple of 64 in [128, 4096]; E a multiple of 4, <= 128 (one
+ * router tile); 1 <= k <= min(8, E); h, hs multiples of 64.  Other shapes return
+ * DG_ERR_INVALID_ARG (or DG_ERR_UNSUPPORTED for T > 4096) before any launch. */
 DG_API int dg_moe_workspace_bytes(int32_t t, int32_t d, int32_t n_experts, int32_t top_k,
                            int32_t hidden, int32_t shared_hidden, size_t* bytes);
 DG_API int dg_moe_ffn(const void* d_x, const float* d_residual, const void* d_wr, const void* d_w_gu,
@@ -241,18 +244,18 @@ DG_API int dg_moe_ffn(const void* d_x, const float* d_residual, const void* d_wr
 enum {
   DG_KERNEL_EXPERT_GATE_UP = 0, /* grouped expert gate/up GEMM + SiLU-GLU */
   DG_KERNEL_EXPERT_DOWN = 1,    /* grouped expert down GEMM + weighted scatter */
-  DG_KERNEL_ATTENTION = 2,      /* canvas attention (before the split combine) */
+  DG_KERNEL_ATTENTION = 2,      /* canvas attention, split merge included */
   DG_KERNEL_LM_HEAD = 3,        /* LM head fused with vocab-tile statistics */
-  DG_KERNEL_QKV = 4,            /* QKV projection GEMM */
-  DG_KERNEL_O_PROJ = 5,         /* attention output projection GEMM */
+  DG_KERNEL_QKV = 4,            /* QKV projection (bf16: RoPE and cache writes included) */
+  DG_KERNEL_O_PROJ = 5,         /* attention output projection (bf16: residual add included) */
   DG_KERNEL_SAMPLER = 6,        /* sampler merge + stop test */
   DG_KERNEL_SHARED_EXPERT = 7,  /* reserved: the shared expert runs inside kinds 0 and 1 */
-  DG_KERNEL_ROUTER = 8,         /* router logits GEMM */
-  DG_KERNEL_QKV_FINALIZE = 9,   /* RoPE + K/V cache store */
-  DG_KERNEL_ATTN_COMBINE = 10,  /* split-KV merge */
+  DG_KERNEL_ROUTER = 8,         /* router (bf16: top-k and expert permutation included) */
+  DG_KERNEL_QKV_FINALIZE = 9,   /* reserved: RoPE + K/V cache store (inside kind 4 on bf16) */
+  DG_KERNEL_ATTN_COMBINE = 10,  /* reserved: split-KV merge (inside kind 2) */
   DG_KERNEL_RESIDUAL_NORM = 11, /* residual add + RMSNorm */
-  DG_KERNEL_ROUTER_TOPK = 12,   /* top-k selection */
-  DG_KERNEL_ROUTE = 13,         /* expert permutation + item lists */
+  DG_KERNEL_ROUTER_TOPK = 12,   /* reserved: top-k selection (inside kind 8 on bf16) */
+  DG_KERNEL_ROUTE = 13,         /* reserved: expert permutation (inside kind 8 on bf16) */
   DG_KERNEL_GATHER = 14,        /* permuted token rows */
   DG_KERNEL_COMBINE_NORM = 15,  /* weighted expert sum + RMSNorm */
   DG_KERNEL_EMBED = 16,         /* embedding gather + RMSNorm */
