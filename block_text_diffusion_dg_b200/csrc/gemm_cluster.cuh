@@ -237,32 +237,6 @@ __global__ void __launch_bounds__(kCluThreads, 1)
       }
     return acc;
   };
-  // the same for two row groups of one token (the rotate-half pair), 2 S loads in flight
-  auto reduce4x2 = [&](int t, int r4a, int r4b, float4& a, float4& b) {
-    const uint32_t oa = drain_u32 + static_cast<uint32_t>((t * 128 + 4 * r4a) * 4);
-    const uint32_t ob = drain_u32 + static_cast<uint32_t>((t * 128 + 4 * r4b) * 4);
-    float4 va[kCluMaxSplits], vb[kCluMaxSplits];
-#pragma unroll
-    for (int src = 0; src < kCluMaxSplits; ++src)
-      if (src < S) {
-        va[src] = dsmem_ld4(dsmem_addr(oa, static_cast<uint32_t>(src)));
-        vb[src] = dsmem_ld4(dsmem_addr(ob, static_cast<uint32_t>(src)));
-      }
-    a = make_float4(0.f, 0.f, 0.f, 0.f);
-    b = a;
-#pragma unroll
-    for (int src = 0; src < kCluMaxSplits; ++src)
-      if (src < S) {
-        a.x += va[src].x;
-        a.y += va[src].y;
-        a.z += va[src].z;
-        a.w += va[src].w;
-        b.x += vb[src].x;
-        b.y += vb[src].y;
-        b.z += vb[src].z;
-        b.w += vb[src].w;
-      }
-  };
   // four row groups at once (token, row group) -> sums with all their loads in flight; the
   // groups go two by two when the cluster is larger than four (register budget)
   auto reduce4x4 = [&](const int (&t)[4], const int (&r4)[4], float4 (&out)[4]) {
