@@ -199,6 +199,10 @@ int launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 
 // ---- GEMM launch helpers -----------------------------------------------------------------
 constexpr int kGroupN = 64, kGroupStages = 8;
+// Long passes (a prompt encoded at once) give each expert hundreds of tokens: there the grouped
+// GEMMs take 256-token chunks, so each expert weight tile streams once per 256 tokens, not 64.
+constexpr int kGroupWideN = 256, kGroupWideStages = 4;
+bool group_wide(long long n_slots, int n_experts) { return n_slots > 64ll * n_experts; }
 constexpr int kRouterChunk = 64;  // tokens per router cluster
 constexpr int kPrefetchExperts = 4;  // routed chunks whose expert weights the gather prefetches
 
@@ -642,7 +646,8 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     p.ids = c->topk_ids;
     p.wts = c->topk_w;
     p.top_k = k;
-    p.route = RouteArgs{c->topk_ids, n, k, E, kGroupN, c->offsets, c->perm, c->chunks, c->n_chunks};
+    p.route = RouteArgs{c->topk_ids, n, k, E, group_wide(n_slots, E) ? kGroupWideN : kGroupN,
+                        c->offsets, c->perm, c->chunks, c->n_chunks};
     p.ticket = c->route_ticket;
     DG_TRY(launch_cluster<kCluRouter>(c->tm_wr[l], c->tm_xn32, p, st, DG_KERNEL_ROUTER));
   }
@@ -656,13 +661,15 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
                       static_cast<__nv_bfloat16*>(c->x_perm), epf, done));
     DG_LAUNCHED();
     prof_after(DG_KERNEL_GATHER, st);
+    const bool wide = group_wide(n_slots, E);
+    const int nch = wide ? kGroupWideN : kGroupN;
     GemmParams p{};
     p.chunks = c->chunks;
     p.chunk_count = c->n_chunks;
     p.m_tiles = cdiv(2 * g.expert_hidden, 128);
-    p.n_chunk = kGroupN;
+    p.n_chunk = nch;
     p.alt_m_tiles = cdiv(2 * g.shared_hidden, 128);
-    p.alt_chunks = cdiv(n, kGroupN);
+    p.alt_chunks = cdiv(n, nch);
     p.alt_tokens = n;
     p.a_rows_per_group = 2 * g.expert_hidden;
     p.kb_total = d / 64;
@@ -680,16 +687,21 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     }
     p.err = c->err;
     p.done = done;
-    DG_TRY((launch_gemm<kGroupN, kGroupStages, kEpiGluBf16>(
-        c->tm_wgu[l], c->tm_xperm, p, c->sms, st, DG_KERNEL_EXPERT_GATE_UP,
-        shared ? &c->tm_wsgu[l] : nullptr, shared ? &c->tm_xn32 : nullptr)));
+    if (wide)
+      DG_TRY((launch_gemm<kGroupWideN, kGroupWideStages, kEpiGluBf16>(
+          c->tm_wgu[l], c->tm_xperm, p, c->sms, st, DG_KERNEL_EXPERT_GATE_UP,
+          shared ? &c->tm_wsgu[l] : nullptr, shared ? &c->tm_xn32 : nullptr)));
+    else
+      DG_TRY((launch_gemm<kGroupN, kGroupStages, kEpiGluBf16>(
+          c->tm_wgu[l], c->tm_xperm, p, c->sms, st, DG_KERNEL_EXPERT_GATE_UP,
+          shared ? &c->tm_wsgu[l] : nullptr, shared ? &c->tm_xn32 : nullptr)));
     GemmParams q{};
     q.chunks = c->chunks;
     q.chunk_count = c->n_chunks;
     q.m_tiles = cdiv(d, 128);
-    q.n_chunk = kGroupN;
+    q.n_chunk = nch;
     q.alt_m_tiles = cdiv(d, 128);
-    q.alt_chunks = cdiv(n, kGroupN);
+    q.alt_chunks = cdiv(n, nch);
     q.alt_tokens = n;
     q.a_rows_per_group = d;
     q.kb_total = g.expert_hidden / 64;
@@ -715,9 +727,14 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     }
     q.err = c->err;
     q.done = done;
-    DG_TRY((launch_gemm<kGroupN, kGroupStages, kEpiScatterF32>(
-        c->tm_wd[l], c->tm_h, q, c->sms, st, DG_KERNEL_EXPERT_DOWN,
-        shared ? &c->tm_wsd[l] : nullptr, shared ? &c->tm_hs : nullptr)));
+    if (wide)
+      DG_TRY((launch_gemm<kGroupWideN, kGroupWideStages, kEpiScatterF32>(
+          c->tm_wd[l], c->tm_h, q, c->sms, st, DG_KERNEL_EXPERT_DOWN,
+          shared ? &c->tm_wsd[l] : nullptr, shared ? &c->tm_hs : nullptr)));
+    else
+      DG_TRY((launch_gemm<kGroupN, kGroupStages, kEpiScatterF32>(
+          c->tm_wd[l], c->tm_h, q, c->sms, st, DG_KERNEL_EXPERT_DOWN,
+          shared ? &c->tm_wsd[l] : nullptr, shared ? &c->tm_hs : nullptr)));
   }
   const float* ysh = shared ? c->y_shared : nullptr;
   prof_before(DG_KERNEL_COMBINE_NORM, st);
@@ -1423,7 +1440,9 @@ int dg_moe_ffn(const void* d_x, const float* d_residual, const void* d_wr, const
   pr.ids = ids;
   pr.wts = wts;
   pr.top_k = top_k;
-  pr.route = RouteArgs{ids, t, top_k, n_experts, kGroupN, offs, perm, chunks, icnt};
+  const bool wide = group_wide(static_cast<long long>(t) * top_k, n_experts);
+  const int nch = wide ? kGroupWideN : kGroupN;
+  pr.route = RouteArgs{ids, t, top_k, n_experts, nch, offs, perm, chunks, icnt};
   pr.ticket = route_ticket;
   DG_TRY(launch_cluster<kCluRouter>(t_wr, t_x32, pr, st, -1));
   DG_TRY(launch_pdl(gather_rows_kernel, dim3(cdiv(t * top_k, 4)), dim3(256), 0, st,
@@ -1435,9 +1454,9 @@ int dg_moe_ffn(const void* d_x, const float* d_residual, const void* d_wr, const
   pg.chunks = chunks;
   pg.chunk_count = icnt;
   pg.m_tiles = cdiv(2 * hidden, 128);
-  pg.n_chunk = kGroupN;
+  pg.n_chunk = nch;
   pg.alt_m_tiles = cdiv(2 * shared_hidden, 128);
-  pg.alt_chunks = cdiv(t, kGroupN);
+  pg.alt_chunks = cdiv(t, nch);
   pg.alt_tokens = t;
   pg.a_rows_per_group = 2 * hidden;
   pg.kb_total = d / 64;
@@ -1450,16 +1469,19 @@ int dg_moe_ffn(const void* d_x, const float* d_residual, const void* d_wr, const
   pg.alt_out_bf16 = hsbuf;
   pg.alt_ld_out = shared_hidden;
   pg.err = err;
-  DG_TRY((launch_gemm<kGroupN, kGroupStages, kEpiGluBf16>(t_wgu, t_xp, pg, sms, st, -1,
-                                                           shared ? &t_wsgu : nullptr,
-                                                           shared ? &t_x32 : nullptr)));
+  if (wide)
+    DG_TRY((launch_gemm<kGroupWideN, kGroupWideStages, kEpiGluBf16>(
+        t_wgu, t_xp, pg, sms, st, -1, shared ? &t_wsgu : nullptr, shared ? &t_x32 : nullptr)));
+  else
+    DG_TRY((launch_gemm<kGroupN, kGroupStages, kEpiGluBf16>(
+        t_wgu, t_xp, pg, sms, st, -1, shared ? &t_wsgu : nullptr, shared ? &t_x32 : nullptr)));
   GemmParams pd{};
   pd.chunks = chunks;
   pd.chunk_count = icnt;
   pd.m_tiles = cdiv(d, 128);
-  pd.n_chunk = kGroupN;
+  pd.n_chunk = nch;
   pd.alt_m_tiles = cdiv(d, 128);
-  pd.alt_chunks = cdiv(t, kGroupN);
+  pd.alt_chunks = cdiv(t, nch);
   pd.alt_tokens = t;
   pd.a_rows_per_group = d;
   pd.kb_total = hidden / 64;
@@ -1474,9 +1496,12 @@ int dg_moe_ffn(const void* d_x, const float* d_residual, const void* d_wr, const
   pd.alt_out_f32 = ysh;
   pd.alt_ld_out = d;
   pd.err = err;
-  DG_TRY((launch_gemm<kGroupN, kGroupStages, kEpiScatterF32>(t_wd, t_h, pd, sms, st, -1,
-                                                              shared ? &t_wsd : nullptr,
-                                                              shared ? &t_hs : nullptr)));
+  if (wide)
+    DG_TRY((launch_gemm<kGroupWideN, kGroupWideStages, kEpiScatterF32>(
+        t_wd, t_h, pd, sms, st, -1, shared ? &t_wsd : nullptr, shared ? &t_hs : nullptr)));
+  else
+    DG_TRY((launch_gemm<kGroupN, kGroupStages, kEpiScatterF32>(
+        t_wd, t_h, pd, sms, st, -1, shared ? &t_wsd : nullptr, shared ? &t_hs : nullptr)));
   const float* ysh_ptr = shared ? ysh : nullptr;
   if (d_residual)
     DG_CUDA(cudaMemcpyAsync(d_y, d_residual, static_cast<size_t>(t) * d * 4,
