@@ -40,6 +40,9 @@ Sources (the pages describe the method in prose only; no code, no equations):
           "Cách thức hoạt động của khuếch tán văn bản": canvas of random placeholder
           tokens, iterative refinement that locks correct tokens and uses them as
           context; a new "diffusion head" on the Gemma 4 base.
+[formats] jakiprompt.pl, "Diffusion Gemma – nowy model Google", section "Wymagania
+          sprzętowe" (hardware requirements): the model ships as BF16, FP8 and NVFP4
+          weights (52 / 27 / 18 GB); [course] table 2.2 quotes fp8 on an H100.
 [philox]  Salmon, Moraes, Dror & Shaw, "Parallel random numbers: as easy as 1, 2, 3",
           SC'11: the Philox4x32-10 counter-based generator.
 
@@ -52,7 +55,8 @@ takes a softmax over all experts, keeps the top-k (lowest index on ties) and
 renormalises the k probabilities; a shared expert is added with weight 1;
 RoPE is rotate-half with theta 10000 at absolute positions; RMSNorm is
 pre-norm with eps 1e-6; embeddings are tied with the LM head; commit re-encodes
-the final argmax block causally, exactly like the prompt.
+the final argmax block causally, exactly like the prompt; FP8 experts are e4m3 with
+one scale per weight row and per activation row (quant.py).
 
 Parity status: every function here is pinned by a CPU test against a closed
 form, a brute-force evaluation, a library routine, published known-answer

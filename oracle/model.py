@@ -31,7 +31,7 @@ import numpy as np
 
 from . import sampler as smp
 from .attention import attention
-from .moe import moe_ffn
+from .moe import moe_ffn, moe_ffn_fp8
 from .numerics import round_f32, round_storage
 
 
@@ -49,6 +49,7 @@ class ModelConfig:
     vocab: int
     canvas: int = 256
     storage: str = "bf16"
+    experts: str = "bf16"  # "fp8": e4m3 expert weights and activations (oracle.quant)
     eps: float = 1e-6
     rope_theta: float = 10000.0
     tau: float = smp.TAU
@@ -114,7 +115,10 @@ def moe_block(cfg, lw, x1):
     st = cfg.storage
     xn2 = round_storage(rmsnorm(x1, lw["ffn_norm"], cfg.eps), st)
     shared = (lw["ws_gu"], lw["ws_d"]) if lw.get("ws_gu") is not None else None
-    y, minfo = moe_ffn(xn2, lw["wr"], lw["w_gu"], lw["w_d"], cfg.top_k, st, shared)
+    if cfg.experts == "fp8":
+        y, minfo = moe_ffn_fp8(xn2, lw["wr"], lw["w_gu"], lw["w_d"], cfg.top_k, shared)
+    else:
+        y, minfo = moe_ffn(xn2, lw["wr"], lw["w_gu"], lw["w_d"], cfg.top_k, st, shared)
     x2 = round_f32(np.asarray(x1, dtype=np.float64) + y)
     return x2, dict(xn2=xn2, moe=minfo)
 

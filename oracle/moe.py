@@ -14,6 +14,9 @@ y = h W_d^T, with h stored in the path's storage type.  The token's output is th
 weighted sum over its k slots taken in slot order, plus the shared expert
 (weight 1) when there is one.
 
+With e4m3 experts (moe_ffn_fp8) the router is unchanged and every expert GEMM takes e4m3
+operands with per-row scales, as quant.py states.
+
 Weights of the gate and up projections are stored interleaved by row,
 w_gu[e][2j] = gate row j and w_gu[e][2j+1] = up row j; this is a storage layout
 only and is undone here with strided views.
@@ -21,6 +24,7 @@ only and is undone here with strided views.
 import numpy as np
 
 from .numerics import round_f32, round_storage
+from .quant import quantize_matrix, quantize_rows
 
 
 def silu(x):
@@ -79,3 +83,51 @@ def moe_ffn(xn, w_r, w_gu, w_d, top_k, storage, shared=None):
         ys, _ = expert_glu(xn, shared[0], shared[1], storage)
         y = y + ys
     return y, dict(router_logits=logits, ids=ids, weights=w, y_slot=y_slot, y_shared=ys)
+
+
+# ---- e4m3 experts (the FP8 weight format; scheme and readings in quant.py) -------------------
+
+def gate_up_fp8(xq, xs, gu_q, gu_s):
+    """SiLU-GLU hidden h [n, hid] (bf16-stored) from e4m3 activations and gate/up weights.
+
+    xq [n, d] e4m3 values with row scales xs [n]; gu_q [2hid, d] row-interleaved e4m3 values
+    with row scales gu_s [2hid].  Sums of code products are scaled by (row scale) x (token scale).
+    """
+    acc = np.asarray(xq, dtype=np.float64) @ np.asarray(gu_q, dtype=np.float64).T
+    gu = acc * np.asarray(gu_s, dtype=np.float64)[None, :] * np.asarray(xs, dtype=np.float64)[:, None]
+    return round_storage(silu(gu[:, 0::2]) * gu[:, 1::2], "bf16")
+
+
+def down_fp8(h, d_q, d_s):
+    """Down projection of h [n, hid] (quantised per row here) with e4m3 weights d_q [d, hid]."""
+    hq, hs = quantize_rows(h)
+    acc = hq @ np.asarray(d_q, dtype=np.float64).T
+    return acc * np.asarray(d_s, dtype=np.float64)[None, :] * hs.astype(np.float64)[:, None]
+
+
+def moe_ffn_fp8(xn, w_r, w_gu, w_d, top_k, shared=None):
+    """MoE output with e4m3 experts: the router as in moe_ffn (bf16 weights), then every expert
+    (and the shared one) quantised row by row from the given weights, the token rows quantised
+    once, and each expert's h quantised per token-slot.  Returns (y [T, d], intermediates)."""
+    xn = np.asarray(xn, dtype=np.float64)
+    t, d = xn.shape
+    logits, ids, w = router(xn, w_r, top_k)
+    xq, xs = quantize_rows(xn)
+    y_slot = np.zeros((t, top_k, d), dtype=np.float64)
+    for e in np.unique(ids):
+        rows, slots = np.nonzero(ids == e)
+        gq, gs = quantize_matrix(w_gu[e])
+        dq, ds = quantize_matrix(w_d[e])
+        h = gate_up_fp8(xq[rows], xs[rows], gq, gs)
+        y_slot[rows, slots] = down_fp8(h, dq, ds)
+    y = np.zeros((t, d), dtype=np.float64)
+    for s in range(top_k):  # slot order 0..k-1
+        y = y + w[:, s:s + 1] * y_slot[:, s]
+    ys = None
+    if shared is not None:
+        gq, gs = quantize_matrix(shared[0])
+        dq, ds = quantize_matrix(shared[1])
+        ys = down_fp8(gate_up_fp8(xq, xs, gq, gs), dq, ds)
+        y = y + ys
+    return y, dict(router_logits=logits, ids=ids, weights=w, y_slot=y_slot, y_shared=ys,
+                   x_codes=xq, x_scales=xs)

@@ -1,0 +1,168 @@
+"""Pins of the oracle's e4m3 quantiser and fp8 expert arithmetic (CPU only).
+
+Each check ties the oracle to something other than itself: torch's float8_e4m3fn conversion (a
+library routine) for the code table and for rounding, closed forms for saturation, ties and the
+error bound, and the pinned bf16 MoE oracle for the fp8 expert stages on operands that already
+lie on the e4m3 grid (there quantisation is the identity, so the two must agree).
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import moe as om
+from oracle.quant import (decode_e4m3, e4m3_table, encode_e4m3, quantize_matrix, quantize_rows,
+                          round_e4m3)
+
+
+def _torch_e4m3(x):
+    """torch's RNE conversion of binary32 values to float8_e4m3fn, widened to float64."""
+    t = torch.from_numpy(np.asarray(x, dtype=np.float32))
+    return t.to(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def test_code_table_matches_torch_bit_patterns():
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    tab = e4m3_table()
+    assert np.array_equal(np.isnan(tab), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(tab[ok], ref[ok])
+    assert np.array_equal(np.signbit(tab[ok]), np.signbit(ref[ok]))
+    assert tab[0x7E] == 448.0 and tab[0x01] == 2.0 ** -9 and tab[0x08] == 2.0 ** -6
+
+
+def test_encode_decode_round_trip():
+    tab = e4m3_table()
+    c = np.arange(256, dtype=np.uint8)
+    ok = ~np.isnan(tab)
+    assert np.array_equal(encode_e4m3(tab[ok]), c[ok])
+    assert np.array_equal(decode_e4m3(c[ok]), tab[ok])
+    with pytest.raises(ValueError):
+        encode_e4m3(np.array([1.0625]))  # between 1 and 1.125
+
+
+def test_rounding_matches_torch_everywhere_below_the_clamp():
+    rng = np.random.default_rng(0)
+    # random binary32 values over every binade of the format, plus the subnormal range
+    mags = np.exp2(rng.uniform(-14, 8.85, 200000)).astype(np.float32)
+    x = np.where(rng.random(mags.shape) < 0.5, -mags, mags).astype(np.float32)
+    # every grid point, every midpoint between neighbours, and their binary32 neighbours
+    tab = e4m3_table()[:0x7F]
+    mids = ((tab[1:] + tab[:-1]) / 2).astype(np.float32)
+    pts = np.concatenate([tab.astype(np.float32), mids, [np.float32(456.0)]])
+    near = np.concatenate([pts, np.nextafter(pts, np.float32(np.inf)),
+                           np.nextafter(pts, np.float32(0))])
+    x = np.concatenate([x, near, -near]).astype(np.float32)
+    x = x[np.abs(x) < 464.0]  # torch turns larger values into NaN; the oracle saturates
+    got = round_e4m3(x.astype(np.float64))
+    ref = _torch_e4m3(x)
+    assert np.array_equal(got, ref)
+    assert np.array_equal(np.signbit(got), np.signbit(ref))
+
+
+def test_ties_go_to_the_even_significand():
+    # 1 + 1/16 lies halfway between 1 (mantissa 0) and 1.125 (mantissa 1): even is 1
+    assert round_e4m3(np.array([1.0625]))[0] == 1.0
+    # 1.1875 lies between 1.125 (m 1) and 1.25 (m 2): even is 1.25
+    assert round_e4m3(np.array([1.1875]))[0] == 1.25
+    # halfway between the two smallest subnormals 2^-9 and 2^-8: even is 2^-8 (m 2)
+    assert round_e4m3(np.array([1.5 * 2.0 ** -9]))[0] == 2.0 ** -8
+    # halfway between 0 and 2^-9 goes to zero
+    assert round_e4m3(np.array([2.0 ** -10]))[0] == 0.0
+
+
+def test_saturation_to_448():
+    x = np.array([448.0, 460.0, 464.0, 465.0, 1e6, 3e38, -1e9])
+    assert np.array_equal(round_e4m3(x), [448, 448, 448, 448, 448, 448, -448])
+
+
+def test_row_quantisation_bounds():
+    rng = np.random.default_rng(1)
+    v = (rng.standard_normal((64, 300)) * np.exp2(rng.uniform(-20, 20, (64, 1)))).astype(np.float32)
+    v[3] = 0.0
+    q, s = quantize_rows(v)
+    assert s.dtype == np.float32 and s[3] == 0 and not q[3].any()
+    nz = np.arange(64) != 3
+    amax = np.abs(v[nz]).max(axis=1)
+    assert np.array_equal(s[nz], (amax / np.float32(448)).astype(np.float32))
+    # the largest element of each row lands on +-448
+    assert np.all(np.abs(q[nz]).max(axis=1) == 448.0)
+    # dequantisation error: half a quantum of the element's binade (2^-4 relative for normals,
+    # 2^-10 absolute in scaled units for subnormals), plus the binary32 quotient's rounding
+    deq = q * s[:, None].astype(np.float64)
+    err = np.abs(deq - v)
+    scaled = np.abs(v) / np.where(s > 0, s, 1)[:, None]
+    bound = np.where(scaled >= 2.0 ** -6, 2.0 ** -4 * np.abs(v), 2.0 ** -10 * s[:, None])
+    assert np.all(err[nz] <= bound[nz] * (1 + 2.0 ** -20))
+
+
+def test_rows_already_on_the_grid_are_exact():
+    rng = np.random.default_rng(2)
+    codes = rng.integers(0, 0x7F, (16, 64))
+    codes[:, 5] = 0x7E  # each row's largest magnitude is 448
+    vals = e4m3_table()[codes] * np.where(rng.random((16, 64)) < 0.5, -1, 1)
+    sigma = np.exp2(rng.integers(-12, 4, 16)).astype(np.float64)
+    q, s = quantize_rows(vals * sigma[:, None])
+    assert np.array_equal(q, vals)
+    assert np.array_equal(s.astype(np.float64), sigma)
+
+
+def _on_grid(rng, shape, lo=-15, hi=-10):
+    """Rows of e4m3 values times a power of two per row, each row's max magnitude 448 x 2^j."""
+    rows = int(np.prod(shape[:-1]))
+    codes = rng.integers(0, 0x7F, (rows, shape[-1]))
+    codes[np.arange(rows), rng.integers(0, shape[-1], rows)] = 0x7E
+    sign = np.where(rng.random((rows, shape[-1])) < 0.5, -1.0, 1.0)
+    sigma = np.exp2(rng.integers(lo, hi, rows)).astype(np.float64)
+    return (e4m3_table()[codes] * sign * sigma[:, None]).reshape(shape)
+
+
+def test_fp8_stages_equal_the_bf16_expert_on_grid_operands():
+    rng = np.random.default_rng(3)
+    n, d, hid = 24, 128, 48
+    x = _on_grid(rng, (n, d), -9, -6)
+    w_gu = _on_grid(rng, (2 * hid, d))
+    w_d = _on_grid(rng, (d, hid))
+    xq, xs = quantize_rows(x)
+    gq, gs = quantize_matrix(w_gu)
+    h8 = om.gate_up_fp8(xq, xs, gq, gs)
+    y16, h16 = om.expert_glu(x, w_gu, w_d, "bf16")
+    assert np.array_equal(h8, h16)
+    # the down stage on an h that lies on the grid reproduces the plain product
+    hg = _on_grid(rng, (n, hid), -6, -2)
+    dq, ds = quantize_matrix(w_d)
+    ref = hg @ w_d.T
+    got = om.down_fp8(hg, dq, ds)
+    assert np.allclose(got, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+    # a transposed or per-column scale would break this: check that scales vary along rows
+    assert len(np.unique(gs)) > 1 and len(np.unique(ds)) > 1
+
+
+def test_fp8_moe_within_the_quantisation_bound_of_the_bf16_moe():
+    rng = np.random.default_rng(4)
+    t, d, e, k, hid, hs = 48, 128, 8, 2, 64, 96
+    wr = (rng.standard_normal((e, d)) * 0.02).astype(np.float32)
+    w_gu = _on_grid(rng, (e, 2 * hid, d))
+    w_d = _on_grid(rng, (e, d, hid))
+    s_gu = _on_grid(rng, (2 * hs, d))
+    s_d = _on_grid(rng, (d, hs))
+    xg = _on_grid(rng, (t, d), -9, -6)
+    y8, info8 = om.moe_ffn_fp8(xg, wr, w_gu, w_d, k, (s_gu, s_d))
+    y16, info16 = om.moe_ffn(xg, wr, w_gu, w_d, k, "bf16", (s_gu, s_d))
+    assert np.array_equal(info8["ids"], info16["ids"])
+    # the only difference left is h's quantisation: |dh| <= 2^-4 |h| + 2^-10 s_h elementwise, so
+    # |dy_slot| <= sum_j (2^-4 |h_j| + 2^-10 s_h) |w_d[., j]|
+    bound = np.zeros((t, d))
+    for s in range(k):
+        for tok in range(t):
+            ex = info16["ids"][tok, s]
+            _, h = om.expert_glu(xg[tok:tok + 1], w_gu[ex], w_d[ex], "bf16")
+            sh = np.abs(h).max() / 448
+            bound[tok] += info16["weights"][tok, s] * (
+                (2.0 ** -4 * np.abs(h) + 2.0 ** -10 * sh) @ np.abs(w_d[ex]).T)[0]
+    _, hsh = om.expert_glu(xg, s_gu, s_d, "bf16")
+    sh = np.abs(hsh).max(axis=1, keepdims=True) / 448
+    bound += (2.0 ** -4 * np.abs(hsh) + 2.0 ** -10 * sh) @ np.abs(s_d).T
+    err = np.abs(y8 - y16)
+    assert np.all(err <= bound * 1.001 + 1e-12)
+    assert err.max() > 0  # h quantisation did change something
