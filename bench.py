@@ -15,6 +15,9 @@ step is that whole 4-block decode (KV cache cut back to the prompt before each s
   cpu_baseline: the CPU oracle on one denoise layer + 1/16 of the LM head + the sampler,
            extrapolated to the decode (rank 0, N = 1)
 
+--experts e4m3 runs the same decode with the FP8 expert format (routed and shared expert weights
+e4m3 with per-row scales, expert activations quantised per row; everything else bf16).
+
 Multi-GPU: every rank decodes its own sequence with its own weights ("replicas only": the
 one-canvas, batch-1 decode has no data-path exchange); value sums all ranks.
 """
@@ -38,6 +41,7 @@ PREFILL_CHUNK = 4096  # prompt tokens per causal-encode pass (the whole prompt)
 WORKLOAD = ("full block decode: 30-layer MoE decoder (d 2816, 16/8 heads x 128, 128 experts "
             "top-8 x 704 + shared 2112, vocab 262144, bf16, random init), 4096-token prompt "
             "prefilled in one pass, 4 canvases x 256 tokens x 16 fixed denoise steps")
+WORKLOAD_E4M3 = WORKLOAD.replace("bf16, random init", "bf16 with e4m3 experts, random init")
 
 
 def parse():
@@ -49,8 +53,10 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--roofline-kernel", default="expert_gate_up")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["decode_step", "decode_step_small", "moe", "attention",
-                                          "sampler"],
+    ap.add_argument("--experts", choices=["bf16", "e4m3"], default="bf16",
+                    help="expert weight format of the decode model")
+    ap.add_argument("--profile", choices=["decode_step", "decode_step_small", "decode_step_e4m3",
+                                          "moe", "moe_e4m3", "attention", "sampler"],
                     help="run one profiled region between cudaProfilerStart/Stop and exit "
                          "(for ncu --profile-from-start off); prints no JSON")
     return ap.parse_args()
@@ -256,7 +262,20 @@ def run_ops(dev, stream, hbm, tf_burst):
     gbs = nbytes / (ms / 1e3) / 1e9
     out["moe"] = dict(us=round(ms * 1e3, 2), bound="hbm", achieved_gbs=round(gbs, 1),
                       frac=round(gbs / hbm, 4), bytes=nbytes)
-    del m, wsm, y, flush
+    # the same MoE with e4m3 experts (1 byte per weight + one fp32 scale per row)
+    q = {}
+    for name in ("w_gu", "w_d", "ws_gu", "ws_d"):
+        q[name], q[name + "_scale"] = dg.quantize_e4m3(m[name])
+    ms = _time_op(lambda: dg.moe_ffn_e4m3(m["x"], m["wr"], q["w_gu"], q["w_gu_scale"], q["w_d"],
+                                          q["w_d_scale"], 8, q["ws_gu"], q["ws_gu_scale"],
+                                          q["ws_d"], q["ws_d_scale"], workspace=wsm, out=y,
+                                          stream=stream), stream, flush=flush)
+    nbytes = m["wr"].numel() * 2 + sum(m[n].numel() + q[n + "_scale"].numel() * 4
+                                       for n in ("w_gu", "w_d", "ws_gu", "ws_d"))
+    gbs = nbytes / (ms / 1e3) / 1e9
+    out["moe_e4m3"] = dict(us=round(ms * 1e3, 2), bound="hbm", achieved_gbs=round(gbs, 1),
+                           frac=round(gbs / hbm, 4), bytes=nbytes)
+    del m, q, wsm, y, flush
     return out
 
 
@@ -271,7 +290,7 @@ def decode(model, seed, out_ids, out_states, stream):
 
 
 def run_ours(args, rank, world, local_rank):
-    from block_text_diffusion_dg_b200 import DiffusionModel, generate, make_config
+    from block_text_diffusion_dg_b200 import DiffusionModel, generate, make_config, quantize_experts
     from block_text_diffusion_dg_b200 import _lib as L
     from dg_synth import SHAPES, model_weights, uniform_ids
     import torch.distributed as dist
@@ -280,8 +299,14 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     shape = SHAPES["a4b"]
     cap = PROMPT + BLOCKS * CANVAS + CANVAS
-    cfg = make_config(shape, kv_capacity=cap, fixed_steps=FIXED_STEPS, prefill_chunk=PREFILL_CHUNK)
+    f8 = args.experts == "e4m3"
+    cfg = make_config(shape, kv_capacity=cap, fixed_steps=FIXED_STEPS, prefill_chunk=PREFILL_CHUNK,
+                      experts=args.experts)
     weights = model_weights("a4b", seed=1000 + rank, device=dev)
+    if f8:  # the bf16 expert matrices are dropped once quantised
+        weights = quantize_experts(weights)
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
     model = DiffusionModel(cfg, weights, device=dev)
     stream = torch.cuda.current_stream(dev)
     prompt = uniform_ids(PROMPT, shape["vocab"], seed=rank).pin_memory()
@@ -356,17 +381,20 @@ def run_ours(args, rank, world, local_rank):
     hs = shape["shared_hidden"]
     slots = CANVAS * k
     # algorithmic bytes per launch: every routed expert's weights (all 128 are routed at these
-    # shapes) and the shared expert's, which rides in the same launch, plus tokens in and out
+    # shapes) and the shared expert's, which rides in the same launch, plus tokens in and out;
+    # e4m3: one byte per weight and per quantised activation, plus the fp32 row scales
+    wb = 1 if f8 else 2
     algo = {
-        "expert_gate_up": (e * 2 * h + 2 * hs) * d * 2 + (slots + CANVAS) * d * 2
-                          + slots * h * 2 + CANVAS * hs * 2,
-        "expert_down": (e * h + hs) * d * 2 + slots * h * 2 + CANVAS * hs * 2
-                       + (slots + CANVAS) * d * 4,
+        "expert_gate_up": (e * 2 * h + 2 * hs) * d * wb + (slots + CANVAS) * d * wb
+                          + slots * h * 2 + CANVAS * hs * 2
+                          + (f8 and (e * 2 * h + 2 * hs + slots + CANVAS) * 4),
+        "expert_down": (e * h + hs) * d * wb + slots * h * wb + CANVAS * hs * wb
+                       + (slots + CANVAS) * d * 4 + (f8 and (e * d + d + slots + CANVAS) * 4),
         "lm_head": shape["vocab"] * d * 2 + CANVAS * d * 2 + CANVAS * (shape["vocab"] // 256) * 16,
     }
     # DRAM bytes (read + write) of one launch from the ncu capture summarised in profiles/
     # (dram__bytes_read.sum + dram__bytes_write.sum); None where no capture of the current kernel
-    traffic = {"expert_gate_up": 1051851000 + 4439808}
+    traffic = {} if f8 else {"expert_gate_up": 1051851000 + 4439808}
     roof = None
     if args.roofline_kernel in algo and rec:
         achieved = algo[args.roofline_kernel] / (avg_ms / 1e3) / 1e9
@@ -426,10 +454,13 @@ def run_ours(args, rank, world, local_rank):
         out = dict(metric="committed canvas tokens/s", value=round(value, 2), unit="tok/s",
                    n_gpus=world, steps=args.steps, warmup=args.warmup,
                    ms_per_step=round(ms_max / args.steps, 3), higher_is_better=True,
-                   scaling="weak", vs_baseline=None, dtype="bf16", data="synthetic",
-                   config=dict(workload=WORKLOAD, global_batch=world, seq_len=PROMPT + BLOCKS * CANVAS,
+                   scaling="weak", vs_baseline=None, dtype="bf16+e4m3" if f8 else "bf16",
+                   data="synthetic",
+                   config=dict(workload=WORKLOAD_E4M3 if f8 else WORKLOAD, global_batch=world,
+                               seq_len=PROMPT + BLOCKS * CANVAS,
                                parallelism=f"replicas x{world}",
-                               l2="inputs larger than L2: ~49 GB of weights streamed per denoise step"),
+                               l2="inputs larger than L2: ~%d GB of weights streamed per denoise "
+                                  "step" % (25 if f8 else 49)),
                    us_per_denoise_step=round(us_step, 1), prefill_ms=round(prefill_ms, 2),
                    roofline=roof, cpu_baseline=cpu,
                    e2e=dict(value=round(e2e_val, 2), unit="tok/s",
@@ -449,7 +480,9 @@ def run_profile(args):
                  + one sampler update.
     decode_step_small: the same with 2 layers and a 32768-token vocabulary (a few GB on the
                  device, for multi-pass captures of single kernels).
+    decode_step_e4m3: decode_step with e4m3 experts.
     moe:         the MoE operator at 256 tokens, d 2816, 128 experts top-8 + shared (1.5 GB).
+    moe_e4m3:    the same operator with e4m3 experts (0.8 GB of expert weights).
     attention:   canvas attention, 16/8 heads x 128, 4096 + 256 keys.
     sampler:     the sampler on bf16 logits [256, 262144].
     """
@@ -458,14 +491,20 @@ def run_profile(args):
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     prof = torch.cuda.profiler
-    if args.profile in ("decode_step", "decode_step_small"):
+    if args.profile in ("decode_step", "decode_step_small", "decode_step_e4m3"):
         shape = dict(SHAPES["a4b"])
         if args.profile == "decode_step_small":
             shape.update(n_layers=2, vocab=32768)
+        f8 = args.profile == "decode_step_e4m3"
         cfg = dg.make_config(shape, kv_capacity=PROMPT + BLOCKS * CANVAS + CANVAS,
                              prefill_chunk=PREFILL_CHUNK,
-                             fixed_steps=FIXED_STEPS)
-        model = dg.DiffusionModel(cfg, model_weights(shape, seed=1000, device=dev), device=dev)
+                             fixed_steps=FIXED_STEPS, experts="e4m3" if f8 else "bf16")
+        w = model_weights(shape, seed=1000, device=dev)
+        if f8:
+            w = dg.quantize_experts(w)
+            torch.cuda.synchronize()
+            torch.cuda.empty_cache()
+        model = dg.DiffusionModel(cfg, w, device=dev)
         model.kv_append(uniform_ids(PROMPT, shape["vocab"], seed=0).to(dev))
         model.canvas_init(1, 0)
         model.denoise_step(1)
@@ -485,6 +524,16 @@ def run_profile(args):
         ws = dg.moe_workspace(256, 2816, 128, 8, 704, 2112, dev)
         call = lambda: dg.moe_ffn(m["x"], m["wr"], m["w_gu"], m["w_d"], 8, m["ws_gu"], m["ws_d"],
                                   workspace=ws)
+    elif args.profile == "moe_e4m3":
+        m = {k: (None if v is None else v.to(dev)) for k, v in moe_inputs(seed=0).items()}
+        q = {}
+        for name in ("w_gu", "w_d", "ws_gu", "ws_d"):
+            q[name], q[name + "_scale"] = dg.quantize_e4m3(m[name])
+            m[name] = None
+        ws = dg.moe_workspace(256, 2816, 128, 8, 704, 2112, dev)
+        call = lambda: dg.moe_ffn_e4m3(m["x"], m["wr"], q["w_gu"], q["w_gu_scale"], q["w_d"],
+                                       q["w_d_scale"], 8, q["ws_gu"], q["ws_gu_scale"], q["ws_d"],
+                                       q["ws_d_scale"], workspace=ws)
     elif args.profile == "attention":
         q, k, v = (t.to(dev) for t in attention_inputs(seed=0))
         vt = v.transpose(1, 2).contiguous()

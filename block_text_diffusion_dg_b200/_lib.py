@@ -8,13 +8,13 @@ LIB_PATH = os.path.join(_HERE, "libdg.so")
 DG_OK = 0
 DG_ERR = {-1: "DG_ERR_INVALID_ARG", -2: "DG_ERR_CAPACITY", -3: "DG_ERR_CUDA",
           -4: "DG_ERR_TIMEOUT", -5: "DG_ERR_UNSUPPORTED"}
-DTYPE_BF16, DTYPE_FP32 = 0, 1
+DTYPE_BF16, DTYPE_FP32, DTYPE_BF16_E4M3 = 0, 1, 2
 STATE_DONE, STATE_STOP_STEP, STATE_WOULD_STOP, STATE_STEPS_RUN, STATE_LOCKED, STATE_ERROR = range(6)
 STATE_WORDS = 16
 KERNEL_KINDS = dict(expert_gate_up=0, expert_down=1, attention=2, lm_head=3, qkv=4,
                     o_proj=5, sampler=6, router=8, qkv_finalize=9, attn_combine=10,
                     residual_norm=11, router_topk=12, route=13, gather=14, combine_norm=15,
-                    embed=16)
+                    embed=16, quant_h=17)
 
 
 class Config(C.Structure):
@@ -31,7 +31,8 @@ class Config(C.Structure):
 
 class LayerWeights(C.Structure):
     _fields_ = [(n, C.c_void_p) for n in
-                ("attn_norm", "wqkv", "wo", "ffn_norm", "wr", "w_gu", "w_d", "ws_gu", "ws_d")]
+                ("attn_norm", "wqkv", "wo", "ffn_norm", "wr", "w_gu", "w_d", "ws_gu", "ws_d",
+                 "w_gu_scale", "w_d_scale", "ws_gu_scale", "ws_d_scale")]
 
 
 class Weights(C.Structure):
@@ -68,6 +69,9 @@ _PROTOS = {
     "dg_moe_workspace_bytes": (C.c_int, [_I, _I, _I, _I, _I, _I, C.POINTER(_SZ)]),
     "dg_moe_ffn": (C.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
                              _P, _SZ, _P]),
+    "dg_moe_ffn_e4m3": (C.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I,
+                                  _I, _I, _I, _I, _I, _P, _SZ, _P]),
+    "dg_quantize_e4m3": (C.c_int, [_P, _I, _I, C.c_int64, _P, C.c_int64, _P, _P]),
     "dg_debug_logits": (C.c_int, [_P, _P, _P]),
     "dg_debug_layer": (C.c_int, [_P, _I, _P, _P, _I, _I, _P]),
     "dg_debug_hidden": (C.c_int, [_P, C.POINTER(_P)]),

@@ -32,14 +32,23 @@ def _need_cuda(t, name, dtype=None):
 
 
 def make_config(shape, *, kv_capacity, fixed_steps=16, max_steps=48, tau=0.9, h_bound=0.005,
-                eps=1e-6, rope_theta=10000.0, prefill_chunk=0):
+                eps=1e-6, rope_theta=10000.0, prefill_chunk=0, experts="bf16"):
+    """Config of a model shape; experts="e4m3" selects the FP8 expert format (bf16 model)."""
     s = shape
+    if experts not in ("bf16", "e4m3"):
+        raise ValueError("experts must be 'bf16' or 'e4m3'")
+    if s["storage"] == "fp32":
+        if experts != "bf16":
+            raise ValueError("the all-fp32 model has no e4m3 expert format")
+        dtype = L.DTYPE_FP32
+    else:
+        dtype = L.DTYPE_BF16_E4M3 if experts == "e4m3" else L.DTYPE_BF16
     return L.Config(
         n_layers=s["n_layers"], d_model=s["d_model"], n_heads=s["n_heads"],
         n_kv_heads=s["n_kv_heads"], head_dim=s["head_dim"], n_experts=s["n_experts"],
         top_k=s["top_k"], expert_hidden=s["expert_hidden"], shared_hidden=s["shared_hidden"],
         vocab=s["vocab"], canvas=s["canvas"], kv_capacity=kv_capacity,
-        dtype=L.DTYPE_FP32 if s["storage"] == "fp32" else L.DTYPE_BF16, eps=eps,
+        dtype=dtype, eps=eps,
         rope_theta=rope_theta, tau=tau, h_bound=h_bound, max_steps=max_steps,
         fixed_steps=fixed_steps, prefill_chunk=prefill_chunk)
 
@@ -63,7 +72,8 @@ class DiffusionModel:
         self.scratch = torch.empty(sc_b, dtype=torch.uint8, device=self.device)
         layers = (L.LayerWeights * cfg.n_layers)()
         for i, lw in enumerate(weights["layers"]):
-            for name in ("attn_norm", "wqkv", "wo", "ffn_norm", "wr", "w_gu", "w_d", "ws_gu", "ws_d"):
+            for name in ("attn_norm", "wqkv", "wo", "ffn_norm", "wr", "w_gu", "w_d", "ws_gu", "ws_d",
+                         "w_gu_scale", "w_d_scale", "ws_gu_scale", "ws_d_scale"):
                 t = lw.get(name)
                 _need_cuda(t, name)
                 setattr(layers[i], name, None if t is None else t.data_ptr())
@@ -287,4 +297,74 @@ def moe_ffn(x, wr, w_gu, w_d, top_k, ws_gu=None, ws_d=None, residual=None, works
                            _ptr(ws_d), _ptr(out), _ptr(ids), _ptr(weights), _ptr(router_logits), t,
                            d, e, top_k, h, hs, _ptr(workspace), workspace.numel(), _stream(stream)),
           "dg_moe_ffn")
+    return out
+
+
+def e4m3_pitch(cols):
+    """Row pitch (bytes) of an e4m3 matrix with `cols` codes per row (DG_E4M3_PITCH)."""
+    return (cols + 127) // 128 * 128
+
+
+def quantize_e4m3(x, pitch=None, stream=None):
+    """Row-wise e4m3 quantisation of a bf16 tensor [..., cols] (cols % 16 == 0).
+
+    Returns (codes uint8 [..., pitch], scales fp32 [...]): scale = max|row| / 448 and
+    code = rn_satfinite(x / scale), the FP8 expert format of dg_quantize_e4m3; codes past `cols`
+    are zero.  The default pitch is the expert-weight pitch e4m3_pitch(cols).
+    """
+    _need_cuda(x, "x", torch.bfloat16)
+    cols = x.shape[-1]
+    pitch = e4m3_pitch(cols) if pitch is None else pitch
+    rows = x.numel() // max(cols, 1)
+    codes = torch.empty(x.shape[:-1] + (pitch,), dtype=torch.uint8, device=x.device)
+    scales = torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device)
+    check(lib().dg_quantize_e4m3(_ptr(x), rows, cols, cols, _ptr(codes), pitch, _ptr(scales),
+                                 _stream(stream)), "dg_quantize_e4m3")
+    return codes, scales
+
+
+def quantize_experts(weights, stream=None):
+    """A copy of a bf16 weight dict with every layer's expert matrices (routed and shared) in
+    the e4m3 format: w_gu, w_d, ws_gu, ws_d become codes (rows at e4m3_pitch) and *_scale their
+    row scales."""
+    out = dict(weights)
+    out["layers"] = []
+    for lw in weights["layers"]:
+        q = dict(lw)
+        for name in ("w_gu", "w_d", "ws_gu", "ws_d"):
+            if lw.get(name) is not None:
+                q[name], q[name + "_scale"] = quantize_e4m3(lw[name], stream)
+        out["layers"].append(q)
+    return out
+
+
+def moe_ffn_e4m3(x, wr, w_gu, w_gu_scale, w_d, w_d_scale, top_k, ws_gu=None, ws_gu_scale=None,
+                 ws_d=None, ws_d_scale=None, residual=None, workspace=None, out=None, ids=None,
+                 weights=None, router_logits=None, stream=None):
+    """moe_ffn with e4m3 experts (codes uint8 with rows at e4m3_pitch + fp32 row scales, as
+    quantize_e4m3 returns them)."""
+    for t, n in ((x, "x"), (wr, "wr")):
+        _need_cuda(t, n, torch.bfloat16)
+    for t, n in ((w_gu, "w_gu"), (w_d, "w_d"), (ws_gu, "ws_gu"), (ws_d, "ws_d")):
+        _need_cuda(t, n, torch.uint8)
+    for t, n in ((w_gu_scale, "w_gu_scale"), (w_d_scale, "w_d_scale"),
+                 (ws_gu_scale, "ws_gu_scale"), (ws_d_scale, "ws_d_scale")):
+        _need_cuda(t, n, torch.float32)
+    t, d = x.shape
+    e, two_h, _ = w_gu.shape
+    h = two_h // 2
+    hs = 0 if ws_gu is None else ws_gu.shape[0] // 2
+    for wt, n, rows, cols in ((w_gu, "w_gu", e * 2 * h, d), (w_d, "w_d", e * d, h),
+                              (ws_gu, "ws_gu", 2 * hs, d), (ws_d, "ws_d", d, hs)):
+        if wt is not None and (wt.shape[-1] != e4m3_pitch(cols) or wt.numel() != rows * e4m3_pitch(cols)):
+            raise ValueError(f"{n} must be [.., {rows} rows, e4m3_pitch({cols})] codes")
+    if workspace is None:
+        workspace = moe_workspace(t, d, e, top_k, h, hs, x.device)
+    if out is None:
+        out = torch.empty(t, d, dtype=torch.float32, device=x.device)
+    check(lib().dg_moe_ffn_e4m3(_ptr(x), _ptr(residual), _ptr(wr), _ptr(w_gu), _ptr(w_gu_scale),
+                                _ptr(w_d), _ptr(w_d_scale), _ptr(ws_gu), _ptr(ws_gu_scale),
+                                _ptr(ws_d), _ptr(ws_d_scale), _ptr(out), _ptr(ids), _ptr(weights),
+                                _ptr(router_logits), t, d, e, top_k, h, hs, _ptr(workspace),
+                                workspace.numel(), _stream(stream)), "dg_moe_ffn_e4m3")
     return out

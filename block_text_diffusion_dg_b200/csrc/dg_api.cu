@@ -18,6 +18,7 @@
 #include "attention.cuh"
 #include "dg_common.cuh"
 #include "fp32_path.cuh"
+#include "fp8.cuh"
 #include "gemm.cuh"
 #include "gemm_cluster.cuh"
 #include "layer.cuh"
@@ -86,6 +87,8 @@ inline void prof_after(int kind, cudaStream_t st) {
 inline cudaStream_t S(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 inline int cdiv(long long a, long long b) { return static_cast<int>((a + b - 1) / b); }
+// Row pitch (bytes) of an e4m3 matrix with `cols` codes per row (DG_E4M3_PITCH).
+inline int e4m3_pitch(int cols) { return (cols + 127) / 128 * 128; }
 
 // ---- TMA descriptor encoding through the driver entry point ---------------------------
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -107,20 +110,22 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// bf16 matrix [rows, cols] with row pitch `pitch` elements; box = 64 columns x box_rows,
-// 128-byte swizzle (the layout the UMMA descriptors expect).
+// Matrix [rows, cols] of bf16 (elem 2) or e4m3 codes (elem 1) with row pitch `pitch` elements;
+// box = one 128-byte row segment (64 bf16 or 128 codes) x box_rows, 128-byte swizzle (the
+// layout the UMMA descriptors expect).  Columns past `cols` read as zero.
 int make_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint64_t pitch,
-              uint32_t box_rows) {
+              uint32_t box_rows, int elem = 2) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
-  if (reinterpret_cast<uintptr_t>(base) % 16 != 0 || (pitch * 2) % 16 != 0)
+  if (reinterpret_cast<uintptr_t>(base) % 16 != 0 || (pitch * elem) % 16 != 0)
     return fail(DG_ERR_INVALID_ARG, "TMA operand not 16-byte aligned (base %p, pitch %llu)", base,
                 (unsigned long long)pitch);
   const cuuint64_t dims[2] = {cols, rows};
-  const cuuint64_t strides[1] = {pitch * 2};
-  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint64_t strides[1] = {pitch * elem};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / elem), box_rows};
   const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+  const CUresult r = fn(m, elem == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                        2, const_cast<void*>(base), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -207,11 +212,11 @@ constexpr int kRouterChunk = 64;  // tokens per router cluster
 constexpr int kPrefetchExperts = 4;  // routed chunks whose expert weights the gather prefetches
 
 // ta2/tb2 are read only by items of the alternate group (p.alt_group >= 0).
-template <int MAXN, int STAGES, int EPI>
+template <int MAXN, int STAGES, int EPI, bool F8 = false>
 int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, int grid,
                 cudaStream_t st, int kind = -1, const CUtensorMap* ta2 = nullptr,
                 const CUtensorMap* tb2 = nullptr) {
-  auto k = gemm_swapab_kernel<MAXN, STAGES, EPI>;
+  auto k = gemm_swapab_kernel<MAXN, STAGES, EPI, F8>;
   constexpr int smem = GemmCfg<MAXN, STAGES>::kSmemBytes;
   if (p.alt_group >= 0 && (!ta2 || !tb2))
     return fail(DG_ERR_INVALID_ARG, "alternate group without its tensor maps");
@@ -273,6 +278,179 @@ int clu_splits(int tiles, int kb_total, int sms) {
   return std::max(1, std::min({kCluMaxSplits, kb_total, sms / std::max(1, tiles)}));
 }
 
+// Grouped expert GEMM with the token-chunk width the pass needs (see group_wide).
+template <int EPI, bool F8>
+int launch_grouped(bool wide, const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
+                   int sms, cudaStream_t st, int kind, const CUtensorMap* ta2,
+                   const CUtensorMap* tb2) {
+  if (wide)
+    return launch_gemm<kGroupWideN, kGroupWideStages, EPI, F8>(ta, tb, p, sms, st, kind, ta2, tb2);
+  return launch_gemm<kGroupN, kGroupStages, EPI, F8>(ta, tb, p, sms, st, kind, ta2, tb2);
+}
+
+// The expert half of an MoE pass once the routing exists: gather the routed token rows (bf16),
+// or gather and quantise them (e4m3, together with the unpermuted tokens for the shared
+// expert); grouped gate/up GEMM with the SiLU-GLU epilogue; e4m3: quantise h per slot and the
+// shared h per token; grouped down GEMM with the weighted scatter.  The shared expert rides
+// along in both GEMMs as the alternate group.
+struct ExpertPass {
+  int n, d, k, E, hid, hs;
+  bool f8;
+  const int32_t* perm;
+  const float* topk_w;
+  const int4* chunks;
+  const int* n_chunks;
+  const __nv_bfloat16* xn;  // normed tokens [n, d]
+  void* x_perm;             // routed rows [n k, d]: bf16, or e4m3 codes
+  float* x_perm_scale;      // e4m3: [n k]
+  void* x_sh;               // e4m3: quantised tokens [n, d] for the shared expert
+  float* x_sh_scale;
+  __nv_bfloat16* h;         // SiLU-GLU output per slot [n k, hid]
+  __nv_bfloat16* h_sh;      // shared expert's [n, hs]
+  void* hq;                 // e4m3: codes of h, h_sh and their scales
+  float* hq_scale;
+  void* hsq;
+  float* hsq_scale;
+  float* y_slot;
+  float* y_shared;
+  const void* w_gu;  // routed gate/up weights: the first chunks' experts are hinted into L2
+  const void* ws_d;  // shared down weights: hinted into L2 by the gate/up GEMM's tail
+  const float *w_gu_scale, *w_d_scale, *ws_gu_scale, *ws_d_scale;
+  const CUtensorMap *tm_wgu, *tm_xperm, *tm_wsgu, *tm_xsh, *tm_wd, *tm_h, *tm_wsd, *tm_hs;
+  const void* pf0;  // hinted into L2 by the down GEMM's tail
+  long long pf0_bytes;
+  const void* pf1;
+  long long pf1_bytes;
+  int* err;
+  const int* done;
+  bool profile;  // record under the per-kernel profiling kinds
+};
+
+int launch_experts(const ExpertPass& e, int sms, cudaStream_t st) {
+  const int n_slots = e.n * e.k;
+  const bool shared = e.hs > 0;
+  const bool wide = group_wide(n_slots, e.E);
+  const int nch = wide ? kGroupWideN : kGroupN;
+  const int kel = e.f8 ? 128 : 64;  // elements per 128-byte K slab
+  // bytes per operand row: bf16 rows are packed, e4m3 rows padded to 128-byte multiples
+  const long long row_d = e.f8 ? e4m3_pitch(e.d) : 2ll * e.d;
+  const long long row_h = e.f8 ? e4m3_pitch(e.hid) : 2ll * e.hid;
+  const long long row_hs = e.f8 ? e4m3_pitch(e.hs) : 2ll * e.hs;
+  const int kind_g = e.profile ? DG_KERNEL_GATHER : -1;
+  const ExpertPrefetch epf{e.chunks, e.n_chunks, kPrefetchExperts, e.w_gu, 2ll * e.hid * row_d};
+  prof_before(kind_g, st);
+  if (e.f8) {
+    QuantJob j{};
+    j.seg[0] = QuantSeg{e.xn, e.d, e.perm, e.k, n_slots, e.d,
+                        static_cast<uint8_t*>(e.x_perm), row_d, e.x_perm_scale};
+    j.seg[1] = QuantSeg{e.xn, e.d, nullptr, 1, e.n, e.d, static_cast<uint8_t*>(e.x_sh), row_d,
+                        e.x_sh_scale};
+    j.n_seg = shared ? 2 : 1;
+    j.pf = epf;
+    DG_TRY(launch_pdl(quant_rows_kernel, dim3(cdiv(n_slots + (shared ? e.n : 0), 8)), dim3(256),
+                      0, st, j, e.done));
+  } else {
+    DG_TRY(launch_pdl(gather_rows_kernel, dim3(cdiv(n_slots, 4)), dim3(256), 0, st, e.xn, e.perm,
+                      e.k, e.d, n_slots, static_cast<__nv_bfloat16*>(e.x_perm), epf, e.done));
+  }
+  DG_LAUNCHED();
+  prof_after(kind_g, st);
+
+  GemmParams p{};
+  p.chunks = e.chunks;
+  p.chunk_count = e.n_chunks;
+  p.m_tiles = cdiv(2 * e.hid, 128);
+  p.n_chunk = nch;
+  p.alt_m_tiles = cdiv(2 * e.hs, 128);
+  p.alt_chunks = cdiv(e.n, nch);
+  p.alt_tokens = e.n;
+  p.a_rows_per_group = 2 * e.hid;
+  p.kb_total = cdiv(e.d, kel);
+  p.m_valid = 2 * e.hid;
+  p.out_bf16 = e.h;
+  p.ld_out = e.hid;
+  p.alt_group = shared ? e.E : -1;
+  p.alt_kb_total = cdiv(e.d, kel);
+  p.alt_m_valid = 2 * e.hs;
+  p.alt_out_bf16 = e.h_sh;
+  p.alt_ld_out = e.hs;
+  p.a_scale = e.w_gu_scale;
+  p.b_scale = e.x_perm_scale;
+  p.alt_a_scale = e.ws_gu_scale;
+  p.alt_b_scale = e.x_sh_scale;
+  if (shared) {  // the down GEMM starts with the shared expert's items
+    p.pf0 = e.ws_d;
+    p.pf0_bytes = static_cast<long long>(e.d) * row_hs;
+  }
+  p.err = e.err;
+  p.done = e.done;
+  const int kind_gu = e.profile ? DG_KERNEL_EXPERT_GATE_UP : -1;
+  const CUtensorMap* ta2 = shared ? e.tm_wsgu : nullptr;
+  const CUtensorMap* tb2 = shared ? e.tm_xsh : nullptr;
+  if (e.f8)
+    DG_TRY((launch_grouped<kEpiGluBf16, true>(wide, *e.tm_wgu, *e.tm_xperm, p, sms, st, kind_gu,
+                                              ta2, tb2)));
+  else
+    DG_TRY((launch_grouped<kEpiGluBf16, false>(wide, *e.tm_wgu, *e.tm_xperm, p, sms, st, kind_gu,
+                                               ta2, tb2)));
+
+  if (e.f8) {
+    const int kind_q = e.profile ? DG_KERNEL_QUANT_H : -1;
+    QuantJob j{};
+    j.seg[0] = QuantSeg{e.h, e.hid, nullptr, 1, n_slots, e.hid, static_cast<uint8_t*>(e.hq), row_h,
+                        e.hq_scale};
+    j.seg[1] = QuantSeg{e.h_sh, e.hs, nullptr, 1, e.n, e.hs, static_cast<uint8_t*>(e.hsq), row_hs,
+                        e.hsq_scale};
+    j.n_seg = shared ? 2 : 1;
+    prof_before(kind_q, st);
+    DG_TRY(launch_pdl(quant_rows_kernel, dim3(cdiv(n_slots + (shared ? e.n : 0), 8)), dim3(256),
+                      0, st, j, e.done));
+    DG_LAUNCHED();
+    prof_after(kind_q, st);
+  }
+
+  GemmParams q{};
+  q.chunks = e.chunks;
+  q.chunk_count = e.n_chunks;
+  q.m_tiles = cdiv(e.d, 128);
+  q.n_chunk = nch;
+  q.alt_m_tiles = cdiv(e.d, 128);
+  q.alt_chunks = cdiv(e.n, nch);
+  q.alt_tokens = e.n;
+  q.a_rows_per_group = e.d;
+  q.kb_total = cdiv(e.hid, kel);
+  q.m_valid = e.d;
+  q.out_f32 = e.y_slot;
+  q.ld_out = e.d;
+  q.perm = e.perm;
+  q.scale = e.topk_w;
+  q.alt_group = shared ? e.E : -1;
+  q.alt_kb_total = cdiv(e.hs, kel);
+  q.alt_m_valid = e.d;
+  q.alt_out_f32 = e.y_shared;
+  q.alt_ld_out = e.d;
+  q.a_scale = e.w_d_scale;
+  q.b_scale = e.hq_scale;
+  q.alt_a_scale = e.ws_d_scale;
+  q.alt_b_scale = e.hsq_scale;
+  q.pf0 = e.pf0;
+  q.pf0_bytes = e.pf0_bytes;
+  q.pf1 = e.pf1;
+  q.pf1_bytes = e.pf1_bytes;
+  q.err = e.err;
+  q.done = e.done;
+  const int kind_d = e.profile ? DG_KERNEL_EXPERT_DOWN : -1;
+  const CUtensorMap* ta3 = shared ? e.tm_wsd : nullptr;
+  const CUtensorMap* tb3 = shared ? e.tm_hs : nullptr;
+  if (e.f8)
+    DG_TRY((launch_grouped<kEpiScatterF32, true>(wide, *e.tm_wd, *e.tm_h, q, sms, st, kind_d, ta3,
+                                                 tb3)));
+  else
+    DG_TRY((launch_grouped<kEpiScatterF32, false>(wide, *e.tm_wd, *e.tm_h, q, sms, st, kind_d,
+                                                  ta3, tb3)));
+  return DG_OK;
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------------------------------
@@ -308,6 +486,9 @@ struct dg_ctx {
   float* topk_w;
   int4* chunks;  // routed token chunks of the grouped GEMMs
   void *x_perm, *h, *hs;
+  bool f8;  // e4m3 experts
+  void *x_sh, *hq, *hsq;  // e4m3 codes: shared-expert tokens, h per slot, shared h per token
+  float *x_perm_scale, *x_sh_scale, *hq_scale, *hsq_scale;
   float *y_slot, *y_shared;
   StatPartial* lm_part;
   float* logits;  // fp32 path
@@ -315,6 +496,7 @@ struct dg_ctx {
   void *kc, *vtc;
   // tensor maps (bf16)
   CUtensorMap tm_xn32, tm_xn128, tm_o32, tm_xperm, tm_h, tm_hs, tm_q, tm_k, tm_vt, tm_embed;
+  CUtensorMap tm_xsh;  // e4m3: B operand of the shared expert's gate/up
   std::vector<CUtensorMap> tm_wqkv, tm_wo, tm_wr, tm_wgu, tm_wd, tm_wsgu, tm_wsd;
   uint64_t seed;
   uint32_t block;
@@ -345,7 +527,7 @@ int check_config(const dg_config* c) {
     return fail(DG_ERR_INVALID_ARG, "max_steps must be >= 1 and fixed_steps >= 0");
   if (c->prefill_chunk < 0 || c->prefill_chunk % 128 != 0 || c->prefill_chunk > 4096)
     return fail(DG_ERR_INVALID_ARG, "prefill_chunk must be 0 or a multiple of 128, <= 4096");
-  if (c->dtype == DG_DTYPE_BF16) {
+  if (c->dtype == DG_DTYPE_BF16 || c->dtype == DG_DTYPE_BF16_E4M3) {
     if (c->head_dim != 128) return fail(DG_ERR_UNSUPPORTED, "bf16 path needs head_dim 128");
     if (c->d_model % 64 || c->expert_hidden % 64 || c->shared_hidden % 64)
       return fail(DG_ERR_UNSUPPORTED, "bf16 path needs d, h, hs multiples of 64");
@@ -363,7 +545,7 @@ int check_config(const dg_config* c) {
 
 // Workspace plan: every buffer at a 256-byte boundary, in this order.
 struct Plan {
-  size_t off[40];
+  size_t off[48];
   size_t total;
   size_t kv;
 };
@@ -371,7 +553,8 @@ struct Plan {
 enum Buf {
   B_CANVAS, B_ARGMAX, B_PREV, B_LOCKED, B_STATE, B_TICKET, B_ERR, B_ENT, B_CONF, B_ROWH, B_X,
   B_XN, B_PART, B_Q, B_OPART, B_ML, B_O, B_RLOG, B_IDS, B_W, B_OFF, B_PERM, B_CHUNKS,
-  B_NCHUNKS, B_RTICKET, B_XPERM, B_H, B_HS, B_YSLOT, B_YSH, B_LMPART, B_LOGITS, B_ROPE, B_END
+  B_NCHUNKS, B_RTICKET, B_XPERM, B_H, B_HS, B_YSLOT, B_YSH, B_LMPART, B_LOGITS, B_ROPE,
+  B_XPS, B_XSH, B_XSHS, B_HQ, B_HQS, B_HSQ, B_HSQS, B_END
 };
 
 struct Derived {
@@ -385,7 +568,7 @@ int tokens_max(const dg_config& c) { return std::max(c.canvas, c.prefill_chunk);
 
 Derived derive(const dg_config& c, int sms) {
   Derived d{};
-  const bool bf16 = c.dtype == DG_DTYPE_BF16;
+  const bool bf16 = c.dtype != DG_DTYPE_FP32;
   d.esz = bf16 ? 2 : 4;
   const long long T = tokens_max(c);
   d.tq = bf16 ? std::max(256, cdiv(static_cast<int>(T), 128) * 128) : static_cast<int>(T);
@@ -410,7 +593,8 @@ Derived derive(const dg_config& c, int sms) {
 Plan plan(const dg_config& c, int sms) {
   Plan p{};
   const Derived dv = derive(c, sms);
-  const bool bf16 = c.dtype == DG_DTYPE_BF16;
+  const bool bf16 = c.dtype != DG_DTYPE_FP32;
+  const bool f8 = c.dtype == DG_DTYPE_BF16_E4M3;
   const size_t Tc = c.canvas, T = tokens_max(c), d = c.d_model, E = c.n_experts, k = c.top_k,
                es = dv.esz;
   const size_t hd = c.head_dim, Hq = c.n_heads;
@@ -435,7 +619,9 @@ Plan plan(const dg_config& c, int sms) {
   sz[B_CHUNKS] = bf16 ? dv.max_chunks * 16 : 0;
   sz[B_NCHUNKS] = 4;
   sz[B_RTICKET] = 4;
-  sz[B_XPERM] = bf16 ? T * k * d * es : 0;
+  const size_t dp = e4m3_pitch(c.d_model), hp = e4m3_pitch(c.expert_hidden),
+               hsp = e4m3_pitch(std::max(1, c.shared_hidden));
+  sz[B_XPERM] = bf16 ? T * k * (f8 ? dp : d * es) : 0;
   sz[B_H] = bf16 ? T * k * c.expert_hidden * es : 0;
   sz[B_HS] = bf16 ? T * std::max<size_t>(1, c.shared_hidden) * es : 0;
   sz[B_YSLOT] = T * k * d * 4;
@@ -443,6 +629,14 @@ Plan plan(const dg_config& c, int sms) {
   sz[B_LMPART] = Tc * nv * sizeof(StatPartial);
   sz[B_LOGITS] = bf16 ? 0 : Tc * c.vocab * 4;
   sz[B_ROPE] = static_cast<size_t>(c.kv_capacity) * (hd / 2) * 8;
+  // e4m3 experts: slot-row scales of x_perm, quantised tokens for the shared expert, quantised h
+  sz[B_XPS] = f8 ? T * k * 4 : 0;
+  sz[B_XSH] = f8 ? T * dp : 0;
+  sz[B_XSHS] = f8 ? T * 4 : 0;
+  sz[B_HQ] = f8 ? T * k * hp : 0;
+  sz[B_HQS] = f8 ? T * k * 4 : 0;
+  sz[B_HSQ] = f8 ? T * hsp : 0;
+  sz[B_HSQS] = f8 ? T * 4 : 0;
   size_t o = 0;
   for (int b = 0; b < B_END; ++b) {
     p.off[b] = o;
@@ -609,7 +803,7 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     a.o = static_cast<__nv_bfloat16*>(c->o);
     if (parts & 2 && g.shared_hidden > 0) {  // the shared expert's weights of this layer
       a.pf0 = w.ws_gu;
-      a.pf0_bytes = 2ll * g.shared_hidden * d * 2;
+      a.pf0_bytes = 2ll * g.shared_hidden * (c->f8 ? e4m3_pitch(d) : 2ll * d);
     }
     a.err = c->err;
     a.done = done;
@@ -651,90 +845,62 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     p.ticket = c->route_ticket;
     DG_TRY(launch_cluster<kCluRouter>(c->tm_wr[l], c->tm_xn32, p, st, DG_KERNEL_ROUTER));
   }
-  // permutation gather and grouped expert GEMMs; the shared expert rides along as group E
+  // permutation gather (+ e4m3 quantisation) and grouped expert GEMMs; the shared expert rides
+  // along as group E
   {
-    prof_before(DG_KERNEL_GATHER, st);
-    const ExpertPrefetch epf{c->chunks, c->n_chunks, kPrefetchExperts, w.w_gu,
-                             2ll * g.expert_hidden * d * 2};
-    DG_TRY(launch_pdl(gather_rows_kernel, dim3(cdiv(n_slots, 4)), dim3(256), 0, st,
-                      static_cast<const __nv_bfloat16*>(c->xn), c->perm, k, d, n_slots,
-                      static_cast<__nv_bfloat16*>(c->x_perm), epf, done));
-    DG_LAUNCHED();
-    prof_after(DG_KERNEL_GATHER, st);
-    const bool wide = group_wide(n_slots, E);
-    const int nch = wide ? kGroupWideN : kGroupN;
-    GemmParams p{};
-    p.chunks = c->chunks;
-    p.chunk_count = c->n_chunks;
-    p.m_tiles = cdiv(2 * g.expert_hidden, 128);
-    p.n_chunk = nch;
-    p.alt_m_tiles = cdiv(2 * g.shared_hidden, 128);
-    p.alt_chunks = cdiv(n, nch);
-    p.alt_tokens = n;
-    p.a_rows_per_group = 2 * g.expert_hidden;
-    p.kb_total = d / 64;
-    p.m_valid = 2 * g.expert_hidden;
-    p.out_bf16 = static_cast<__nv_bfloat16*>(c->h);
-    p.ld_out = g.expert_hidden;
-    p.alt_group = shared ? E : -1;
-    p.alt_kb_total = d / 64;
-    p.alt_m_valid = 2 * g.shared_hidden;
-    p.alt_out_bf16 = static_cast<__nv_bfloat16*>(c->hs);
-    p.alt_ld_out = g.shared_hidden;
-    if (shared) {  // the down GEMM starts with the shared expert's items
-      p.pf0 = w.ws_d;
-      p.pf0_bytes = static_cast<long long>(d) * g.shared_hidden * 2;
-    }
-    p.err = c->err;
-    p.done = done;
-    if (wide)
-      DG_TRY((launch_gemm<kGroupWideN, kGroupWideStages, kEpiGluBf16>(
-          c->tm_wgu[l], c->tm_xperm, p, c->sms, st, DG_KERNEL_EXPERT_GATE_UP,
-          shared ? &c->tm_wsgu[l] : nullptr, shared ? &c->tm_xn32 : nullptr)));
-    else
-      DG_TRY((launch_gemm<kGroupN, kGroupStages, kEpiGluBf16>(
-          c->tm_wgu[l], c->tm_xperm, p, c->sms, st, DG_KERNEL_EXPERT_GATE_UP,
-          shared ? &c->tm_wsgu[l] : nullptr, shared ? &c->tm_xn32 : nullptr)));
-    GemmParams q{};
-    q.chunks = c->chunks;
-    q.chunk_count = c->n_chunks;
-    q.m_tiles = cdiv(d, 128);
-    q.n_chunk = nch;
-    q.alt_m_tiles = cdiv(d, 128);
-    q.alt_chunks = cdiv(n, nch);
-    q.alt_tokens = n;
-    q.a_rows_per_group = d;
-    q.kb_total = g.expert_hidden / 64;
-    q.m_valid = d;
-    q.out_f32 = c->y_slot;
-    q.ld_out = d;
-    q.perm = c->perm;
-    q.scale = c->topk_w;
-    q.alt_group = shared ? E : -1;
-    q.alt_kb_total = g.shared_hidden / 64;
-    q.alt_m_valid = d;
-    q.alt_out_f32 = c->y_shared;
-    q.alt_ld_out = d;
+    ExpertPass e{};
+    e.n = n;
+    e.d = d;
+    e.k = k;
+    e.E = E;
+    e.hid = g.expert_hidden;
+    e.hs = g.shared_hidden;
+    e.f8 = c->f8;
+    e.perm = c->perm;
+    e.topk_w = c->topk_w;
+    e.chunks = c->chunks;
+    e.n_chunks = c->n_chunks;
+    e.xn = static_cast<const __nv_bfloat16*>(c->xn);
+    e.x_perm = c->x_perm;
+    e.x_perm_scale = c->x_perm_scale;
+    e.x_sh = c->x_sh;
+    e.x_sh_scale = c->x_sh_scale;
+    e.h = static_cast<__nv_bfloat16*>(c->h);
+    e.h_sh = static_cast<__nv_bfloat16*>(c->hs);
+    e.hq = c->hq;
+    e.hq_scale = c->hq_scale;
+    e.hsq = c->hsq;
+    e.hsq_scale = c->hsq_scale;
+    e.y_slot = c->y_slot;
+    e.y_shared = c->y_shared;
+    e.w_gu = w.w_gu;
+    e.ws_d = w.ws_d;
+    e.w_gu_scale = w.w_gu_scale;
+    e.w_d_scale = w.w_d_scale;
+    e.ws_gu_scale = w.ws_gu_scale;
+    e.ws_d_scale = w.ws_d_scale;
+    e.tm_wgu = &c->tm_wgu[l];
+    e.tm_xperm = &c->tm_xperm;
+    e.tm_wsgu = &c->tm_wsgu[l];
+    e.tm_xsh = c->f8 ? &c->tm_xsh : &c->tm_xn32;
+    e.tm_wd = &c->tm_wd[l];
+    e.tm_h = &c->tm_h;
+    e.tm_wsd = &c->tm_wsd[l];
+    e.tm_hs = &c->tm_hs;
     if (l + 1 < g.n_layers) {  // the next layer's QKV and O projections
       const dg_layer_weights& wn = c->layers[l + 1];
-      q.pf0 = wn.wqkv;
-      q.pf0_bytes = static_cast<long long>(c->qkv_rows) * d * 2;
-      q.pf1 = wn.wo;
-      q.pf1_bytes = static_cast<long long>(d) * g.n_heads * hd * 2;
+      e.pf0 = wn.wqkv;
+      e.pf0_bytes = static_cast<long long>(c->qkv_rows) * d * 2;
+      e.pf1 = wn.wo;
+      e.pf1_bytes = static_cast<long long>(d) * g.n_heads * hd * 2;
     } else {  // the first vocabulary tiles of the LM head
-      q.pf0 = c->embed;
-      q.pf0_bytes = std::min<long long>(64ll << 20, static_cast<long long>(g.vocab) * d * 2);
+      e.pf0 = c->embed;
+      e.pf0_bytes = std::min<long long>(64ll << 20, static_cast<long long>(g.vocab) * d * 2);
     }
-    q.err = c->err;
-    q.done = done;
-    if (wide)
-      DG_TRY((launch_gemm<kGroupWideN, kGroupWideStages, kEpiScatterF32>(
-          c->tm_wd[l], c->tm_h, q, c->sms, st, DG_KERNEL_EXPERT_DOWN,
-          shared ? &c->tm_wsd[l] : nullptr, shared ? &c->tm_hs : nullptr)));
-    else
-      DG_TRY((launch_gemm<kGroupN, kGroupStages, kEpiScatterF32>(
-          c->tm_wd[l], c->tm_h, q, c->sms, st, DG_KERNEL_EXPERT_DOWN,
-          shared ? &c->tm_wsd[l] : nullptr, shared ? &c->tm_hs : nullptr)));
+    e.err = c->err;
+    e.done = done;
+    e.profile = true;
+    DG_TRY(launch_experts(e, c->sms, st));
   }
   const float* ysh = shared ? c->y_shared : nullptr;
   prof_before(DG_KERNEL_COMBINE_NORM, st);
@@ -790,10 +956,16 @@ int bind_tmaps(dg_ctx* c) {
   DG_TRY(make_tmap(&c->tm_xn32, c->xn, T, d, d, 32));
   DG_TRY(make_tmap(&c->tm_xn128, c->xn, T, d, d, 128));
   DG_TRY(make_tmap(&c->tm_o32, c->o, T, g.n_heads * hd, g.n_heads * hd, 32));
-  DG_TRY(make_tmap(&c->tm_xperm, c->x_perm, T * k, d, d, 32));
-  DG_TRY(make_tmap(&c->tm_h, c->h, T * k, g.expert_hidden, g.expert_hidden, 32));
+  // expert GEMM operands: bf16, or e4m3 with rows at the 128-byte pitch
+  const int eb = c->f8 ? 1 : 2;
+  const uint64_t pd = c->f8 ? e4m3_pitch(g.d_model) : d;
+  const uint64_t ph = c->f8 ? e4m3_pitch(g.expert_hidden) : g.expert_hidden;
+  const uint64_t phs = c->f8 ? e4m3_pitch(std::max(1, g.shared_hidden)) : g.shared_hidden;
+  DG_TRY(make_tmap(&c->tm_xperm, c->x_perm, T * k, d, pd, 32, eb));
+  DG_TRY(make_tmap(&c->tm_h, c->f8 ? c->hq : c->h, T * k, g.expert_hidden, ph, 32, eb));
   if (g.shared_hidden > 0)
-    DG_TRY(make_tmap(&c->tm_hs, c->hs, T, g.shared_hidden, g.shared_hidden, 32));
+    DG_TRY(make_tmap(&c->tm_hs, c->f8 ? c->hsq : c->hs, T, g.shared_hidden, phs, 32, eb));
+  if (c->f8) DG_TRY(make_tmap(&c->tm_xsh, c->x_sh, T, d, pd, 32, 1));
   DG_TRY(make_tmap(&c->tm_q, c->q, static_cast<uint64_t>(g.n_heads) * c->tq, hd, hd, 128));
   const uint64_t kv_rows = static_cast<uint64_t>(g.n_layers) * g.n_kv_heads * g.kv_capacity;
   DG_TRY(make_tmap(&c->tm_k, c->kc, kv_rows, hd, hd, 128));
@@ -814,12 +986,12 @@ int bind_tmaps(dg_ctx* c) {
     DG_TRY(make_tmap(&c->tm_wo[l], w.wo, d, g.n_heads * hd, g.n_heads * hd, 128));
     DG_TRY(make_tmap(&c->tm_wr[l], w.wr, g.n_experts, d, d, 128));
     DG_TRY(make_tmap(&c->tm_wgu[l], w.w_gu, static_cast<uint64_t>(g.n_experts) * 2 * g.expert_hidden,
-                     d, d, 128));
+                     d, pd, 128, eb));
     DG_TRY(make_tmap(&c->tm_wd[l], w.w_d, static_cast<uint64_t>(g.n_experts) * d, g.expert_hidden,
-                     g.expert_hidden, 128));
+                     ph, 128, eb));
     if (g.shared_hidden > 0) {
-      DG_TRY(make_tmap(&c->tm_wsgu[l], w.ws_gu, 2ull * g.shared_hidden, d, d, 128));
-      DG_TRY(make_tmap(&c->tm_wsd[l], w.ws_d, d, g.shared_hidden, g.shared_hidden, 128));
+      DG_TRY(make_tmap(&c->tm_wsgu[l], w.ws_gu, 2ull * g.shared_hidden, d, pd, 128, eb));
+      DG_TRY(make_tmap(&c->tm_wsd[l], w.ws_d, d, g.shared_hidden, phs, 128, eb));
     }
   }
   return DG_OK;
@@ -886,6 +1058,10 @@ int dg_create(const dg_config* cfg, const dg_weights* w, void* d_kv, void* d_scr
       return fail(DG_ERR_INVALID_ARG, "layer %d has a null weight", l);
     if (cfg->shared_hidden > 0 && (!lw.ws_gu || !lw.ws_d))
       return fail(DG_ERR_INVALID_ARG, "layer %d lacks shared expert weights", l);
+    if (cfg->dtype == DG_DTYPE_BF16_E4M3 &&
+        (!lw.w_gu_scale || !lw.w_d_scale ||
+         (cfg->shared_hidden > 0 && (!lw.ws_gu_scale || !lw.ws_d_scale))))
+      return fail(DG_ERR_INVALID_ARG, "layer %d lacks e4m3 expert scales", l);
   }
   dg_ctx* c = new dg_ctx();
   c->cfg = *cfg;
@@ -896,7 +1072,8 @@ int dg_create(const dg_config* cfg, const dg_weights* w, void* d_kv, void* d_scr
   c->scratch = static_cast<uint8_t*>(d_scratch);
   c->kv_len = 0;
   c->sms = num_sms();
-  c->bf16 = cfg->dtype == DG_DTYPE_BF16;
+  c->bf16 = cfg->dtype != DG_DTYPE_FP32;
+  c->f8 = cfg->dtype == DG_DTYPE_BF16_E4M3;
   const Derived dv = derive(*cfg, c->sms);
   c->esz = dv.esz;
   c->tq = dv.tq;
@@ -939,6 +1116,13 @@ int dg_create(const dg_config* cfg, const dg_weights* w, void* d_kv, void* d_scr
   c->lm_part = reinterpret_cast<StatPartial*>(s + p.off[B_LMPART]);
   c->logits = reinterpret_cast<float*>(s + p.off[B_LOGITS]);
   c->rope_tab = reinterpret_cast<float2*>(s + p.off[B_ROPE]);
+  c->x_perm_scale = reinterpret_cast<float*>(s + p.off[B_XPS]);
+  c->x_sh = s + p.off[B_XSH];
+  c->x_sh_scale = reinterpret_cast<float*>(s + p.off[B_XSHS]);
+  c->hq = s + p.off[B_HQ];
+  c->hq_scale = reinterpret_cast<float*>(s + p.off[B_HQS]);
+  c->hsq = s + p.off[B_HSQ];
+  c->hsq_scale = reinterpret_cast<float*>(s + p.off[B_HSQS]);
   const size_t kv_half = p.kv / 2;
   c->kc = c->kv;
   c->vtc = c->kv + kv_half;
@@ -1344,37 +1528,174 @@ int dg_canvas_attention(const void* d_q, const void* d_k, const void* d_vt, void
 
 // ---- standalone MoE --------------------------------------------------------------------
 namespace {
+enum MoeBuf {
+  M_RLOG, M_IDS, M_W, M_OFF, M_PERM, M_CHUNKS, M_WORDS, M_XPERM, M_H, M_HS, M_YSH, M_YSLOT,
+  M_XPS, M_XSH, M_XSHS, M_HQ, M_HQS, M_HSQ, M_HSQS, M_END
+};
 struct MoePlan {
-  size_t off[12];
+  size_t off[M_END];
   size_t total;
   int split_r;
   long long chunks;
 };
+// Buffers of both expert formats (the e4m3 ones are small next to the bf16 x_perm).
 MoePlan moe_plan(int t, int d, int E, int k, int hid, int hs) {
   MoePlan m{};
   m.split_r = std::min(kCluMaxSplits, d / 64);
   m.chunks = E + (static_cast<long long>(t) * k + kGroupN - 1) / kGroupN;
-  size_t sz[12];
-  sz[0] = static_cast<size_t>(t) * E * 4;              // router logits (internal)
-  sz[1] = static_cast<size_t>(t) * k * 4;              // ids (internal)
-  sz[2] = static_cast<size_t>(t) * k * 4;              // weights (internal)
-  sz[3] = (E + 1) * 4;                                 // offsets
-  sz[4] = static_cast<size_t>(t) * k * 4;              // perm
-  sz[5] = m.chunks * 16;                               // routed token chunks
-  sz[6] = 0;                                           // (unused)
-  sz[7] = 16;                                          // chunk count, -, error word, route ticket
-  sz[8] = static_cast<size_t>(t) * k * d * 2;          // x_perm
-  sz[9] = static_cast<size_t>(t) * k * hid * 2;        // h
-  sz[10] = align256(static_cast<size_t>(t) * std::max(hs, 1) * 2) +
-           static_cast<size_t>(t) * d * 4;  // hs, then y_shared at the next 256-byte boundary
-  sz[11] = static_cast<size_t>(t) * k * d * 4;         // y_slot
+  const size_t T = t, tk = static_cast<size_t>(t) * k, hs1 = std::max(hs, 1);
+  size_t sz[M_END];
+  sz[M_RLOG] = T * E * 4;     // router logits (internal)
+  sz[M_IDS] = tk * 4;         // ids (internal)
+  sz[M_W] = tk * 4;           // weights (internal)
+  sz[M_OFF] = (E + 1) * 4;    // offsets
+  sz[M_PERM] = tk * 4;        // perm
+  sz[M_CHUNKS] = m.chunks * 16;  // routed token chunks
+  sz[M_WORDS] = 16;           // chunk count, -, error word, route ticket
+  sz[M_XPERM] = tk * d * 2;   // x_perm (bf16; e4m3 rows at the 128-byte pitch fit: d >= 128)
+  sz[M_H] = tk * hid * 2;     // h
+  sz[M_HS] = T * hs1 * 2;     // shared h
+  sz[M_YSH] = T * d * 4;      // y_shared
+  sz[M_YSLOT] = tk * d * 4;   // y_slot
+  sz[M_XPS] = tk * 4;         // e4m3: x_perm row scales
+  sz[M_XSH] = T * e4m3_pitch(d);    // e4m3: quantised tokens for the shared expert
+  sz[M_XSHS] = T * 4;
+  sz[M_HQ] = tk * e4m3_pitch(hid);  // e4m3: quantised h and its scales
+  sz[M_HQS] = tk * 4;
+  sz[M_HSQ] = T * e4m3_pitch(static_cast<int>(hs1));  // e4m3: quantised shared h, scales
+  sz[M_HSQS] = T * 4;
   size_t o = 0;
-  for (int i = 0; i < 12; ++i) {
+  for (int i = 0; i < M_END; ++i) {
     m.off[i] = o;
     o += align256(std::max<size_t>(sz[i], 1));
   }
   m.total = o;
   return m;
+}
+
+struct MoeScales {
+  const float *w_gu, *w_d, *ws_gu, *ws_d;
+};
+
+int moe_ffn_impl(bool f8, const MoeScales& sc, const void* d_x, const float* d_residual,
+                 const void* d_wr, const void* d_w_gu, const void* d_w_d, const void* d_ws_gu,
+                 const void* d_ws_d, float* d_y, int32_t* d_ids, float* d_weights,
+                 float* d_router_logits, int32_t t, int32_t d, int32_t n_experts, int32_t top_k,
+                 int32_t hidden, int32_t shared_hidden, void* d_workspace, size_t workspace_bytes,
+                 void* stream) {
+  size_t need = 0;
+  DG_TRY(dg_moe_workspace_bytes(t, d, n_experts, top_k, hidden, shared_hidden, &need));
+  if (!d_x || !d_wr || !d_w_gu || !d_w_d || !d_y || !d_workspace)
+    return fail(DG_ERR_INVALID_ARG, "null pointer argument");
+  if (shared_hidden > 0 && (!d_ws_gu || !d_ws_d))
+    return fail(DG_ERR_INVALID_ARG, "shared expert weights missing");
+  if (f8 && (!sc.w_gu || !sc.w_d || (shared_hidden > 0 && (!sc.ws_gu || !sc.ws_d))))
+    return fail(DG_ERR_INVALID_ARG, "e4m3 expert scales missing");
+  if (workspace_bytes < need) return fail(DG_ERR_CAPACITY, "MoE workspace too small");
+  if (t > 4096) return fail(DG_ERR_UNSUPPORTED, "at most 4096 tokens per call");
+  const MoePlan m = moe_plan(t, d, n_experts, top_k, hidden, shared_hidden);
+  uint8_t* ws = static_cast<uint8_t*>(d_workspace);
+  auto at = [&](int b) { return static_cast<void*>(ws + m.off[b]); };
+  float* rlog = static_cast<float*>(at(M_RLOG));
+  int32_t* ids = static_cast<int32_t*>(at(M_IDS));
+  float* wts = static_cast<float*>(at(M_W));
+  int32_t* offs = static_cast<int32_t*>(at(M_OFF));
+  int32_t* perm = static_cast<int32_t*>(at(M_PERM));
+  int4* chunks = static_cast<int4*>(at(M_CHUNKS));
+  int32_t* icnt = static_cast<int32_t*>(at(M_WORDS));
+  int* err = icnt + 2;
+  int32_t* route_ticket = icnt + 3;
+  const int sms = num_sms();
+  cudaStream_t st = S(stream);
+  DG_CUDA(cudaMemsetAsync(err, 0, 8, st));  // error word and route ticket
+  const int eb = f8 ? 1 : 2;
+  // operand row pitches (elements): e4m3 rows at the 128-byte pitch
+  const uint64_t pd = f8 ? e4m3_pitch(d) : d, ph = f8 ? e4m3_pitch(hidden) : hidden,
+                 phs = f8 ? e4m3_pitch(std::max(1, shared_hidden)) : shared_hidden;
+  const uint64_t tk = static_cast<uint64_t>(t) * top_k;
+  CUtensorMap t_x32, t_wr, t_xp, t_wgu, t_h, t_wd, t_wsgu, t_hs, t_wsd, t_xsh;
+  DG_TRY(make_tmap(&t_x32, d_x, t, d, d, 32));
+  DG_TRY(make_tmap(&t_wr, d_wr, n_experts, d, d, 128));
+  DG_TRY(make_tmap(&t_xp, at(M_XPERM), tk, d, pd, 32, eb));
+  DG_TRY(make_tmap(&t_wgu, d_w_gu, static_cast<uint64_t>(n_experts) * 2 * hidden, d, pd, 128, eb));
+  DG_TRY(make_tmap(&t_h, at(f8 ? M_HQ : M_H), tk, hidden, ph, 32, eb));
+  DG_TRY(make_tmap(&t_wd, d_w_d, static_cast<uint64_t>(n_experts) * d, hidden, ph, 128, eb));
+  if (f8) DG_TRY(make_tmap(&t_xsh, at(M_XSH), t, d, pd, 32, 1));
+  if (shared_hidden > 0) {
+    DG_TRY(make_tmap(&t_wsgu, d_ws_gu, 2ull * shared_hidden, d, pd, 128, eb));
+    DG_TRY(make_tmap(&t_hs, at(f8 ? M_HSQ : M_HS), t, shared_hidden, phs, 32, eb));
+    DG_TRY(make_tmap(&t_wsd, d_ws_d, d, shared_hidden, phs, 128, eb));
+  }
+  // router
+  CluParams pr = clu_params(n_experts, t, d / 64, m.split_r, err, nullptr, kRouterChunk);
+  pr.router_logits = d_router_logits ? d_router_logits : rlog;
+  pr.ids = ids;
+  pr.wts = wts;
+  pr.top_k = top_k;
+  const bool wide = group_wide(static_cast<long long>(t) * top_k, n_experts);
+  pr.route = RouteArgs{ids, t, top_k, n_experts, wide ? kGroupWideN : kGroupN, offs, perm, chunks,
+                       icnt};
+  pr.ticket = route_ticket;
+  DG_TRY(launch_cluster<kCluRouter>(t_wr, t_x32, pr, st, -1));
+  ExpertPass e{};
+  e.n = t;
+  e.d = d;
+  e.k = top_k;
+  e.E = n_experts;
+  e.hid = hidden;
+  e.hs = shared_hidden;
+  e.f8 = f8;
+  e.perm = perm;
+  e.topk_w = wts;
+  e.chunks = chunks;
+  e.n_chunks = icnt;
+  e.xn = static_cast<const __nv_bfloat16*>(d_x);
+  e.x_perm = at(M_XPERM);
+  e.x_perm_scale = static_cast<float*>(at(M_XPS));
+  e.x_sh = at(M_XSH);
+  e.x_sh_scale = static_cast<float*>(at(M_XSHS));
+  e.h = static_cast<__nv_bfloat16*>(at(M_H));
+  e.h_sh = static_cast<__nv_bfloat16*>(at(M_HS));
+  e.hq = at(M_HQ);
+  e.hq_scale = static_cast<float*>(at(M_HQS));
+  e.hsq = at(M_HSQ);
+  e.hsq_scale = static_cast<float*>(at(M_HSQS));
+  e.y_slot = static_cast<float*>(at(M_YSLOT));
+  e.y_shared = static_cast<float*>(at(M_YSH));
+  e.w_gu = d_w_gu;
+  e.ws_d = d_ws_d;
+  e.w_gu_scale = sc.w_gu;
+  e.w_d_scale = sc.w_d;
+  e.ws_gu_scale = sc.ws_gu;
+  e.ws_d_scale = sc.ws_d;
+  e.tm_wgu = &t_wgu;
+  e.tm_xperm = &t_xp;
+  e.tm_wsgu = &t_wsgu;
+  e.tm_xsh = f8 ? &t_xsh : &t_x32;
+  e.tm_wd = &t_wd;
+  e.tm_h = &t_h;
+  e.tm_wsd = &t_wsd;
+  e.tm_hs = &t_hs;
+  e.err = err;
+  e.done = nullptr;
+  e.profile = false;
+  DG_TRY(launch_experts(e, sms, st));
+  const float* ysh_ptr = shared_hidden > 0 ? e.y_shared : nullptr;
+  if (d_residual)
+    DG_CUDA(cudaMemcpyAsync(d_y, d_residual, static_cast<size_t>(t) * d * 4,
+                            cudaMemcpyDeviceToDevice, st));
+  else
+    DG_CUDA(cudaMemsetAsync(d_y, 0, static_cast<size_t>(t) * d * 4, st));
+  DG_TRY(launch_pdl(moe_combine_norm_kernel<__nv_bfloat16>, dim3(t), dim3(256), 0, st, d_y,
+                    e.y_slot, top_k, ysh_ptr, d, nullptr, 0.f, nullptr, nullptr));
+  DG_LAUNCHED();
+  if (d_ids)
+    DG_CUDA(cudaMemcpyAsync(d_ids, ids, static_cast<size_t>(t) * top_k * 4,
+                            cudaMemcpyDeviceToDevice, st));
+  if (d_weights)
+    DG_CUDA(cudaMemcpyAsync(d_weights, wts, static_cast<size_t>(t) * top_k * 4,
+                            cudaMemcpyDeviceToDevice, st));
+  return DG_OK;
 }
 }  // namespace
 
@@ -1394,129 +1715,43 @@ int dg_moe_ffn(const void* d_x, const float* d_residual, const void* d_wr, const
                int32_t* d_ids, float* d_weights, float* d_router_logits, int32_t t, int32_t d,
                int32_t n_experts, int32_t top_k, int32_t hidden, int32_t shared_hidden,
                void* d_workspace, size_t workspace_bytes, void* stream) {
-  size_t need = 0;
-  DG_TRY(dg_moe_workspace_bytes(t, d, n_experts, top_k, hidden, shared_hidden, &need));
-  if (!d_x || !d_wr || !d_w_gu || !d_w_d || !d_y || !d_workspace)
-    return fail(DG_ERR_INVALID_ARG, "null pointer argument");
-  if (shared_hidden > 0 && (!d_ws_gu || !d_ws_d))
-    return fail(DG_ERR_INVALID_ARG, "shared expert weights missing");
-  if (workspace_bytes < need) return fail(DG_ERR_CAPACITY, "MoE workspace too small");
-  if (t > 4096) return fail(DG_ERR_UNSUPPORTED, "at most 4096 tokens per call");
-  const MoePlan m = moe_plan(t, d, n_experts, top_k, hidden, shared_hidden);
-  uint8_t* ws = static_cast<uint8_t*>(d_workspace);
-  float* rlog = reinterpret_cast<float*>(ws + m.off[0]);
-  int32_t* ids = reinterpret_cast<int32_t*>(ws + m.off[1]);
-  float* wts = reinterpret_cast<float*>(ws + m.off[2]);
-  int32_t* offs = reinterpret_cast<int32_t*>(ws + m.off[3]);
-  int32_t* perm = reinterpret_cast<int32_t*>(ws + m.off[4]);
-  int4* chunks = reinterpret_cast<int4*>(ws + m.off[5]);
-  int32_t* icnt = reinterpret_cast<int32_t*>(ws + m.off[7]);
-  int* err = icnt + 2;
-  int32_t* route_ticket = icnt + 3;
-  __nv_bfloat16* x_perm = reinterpret_cast<__nv_bfloat16*>(ws + m.off[8]);
-  __nv_bfloat16* hbuf = reinterpret_cast<__nv_bfloat16*>(ws + m.off[9]);
-  __nv_bfloat16* hsbuf = reinterpret_cast<__nv_bfloat16*>(ws + m.off[10]);
-  float* ysh = reinterpret_cast<float*>(ws + m.off[10] + align256(static_cast<size_t>(t) * std::max(shared_hidden, 1) * 2));
-  float* y_slot = reinterpret_cast<float*>(ws + m.off[11]);
-  const int sms = num_sms();
-  cudaStream_t st = S(stream);
-  DG_CUDA(cudaMemsetAsync(err, 0, 8, st));  // error word and route ticket
-  CUtensorMap t_x32, t_wr, t_xp, t_wgu, t_h, t_wd, t_wsgu, t_hs, t_wsd;
-  DG_TRY(make_tmap(&t_x32, d_x, t, d, d, 32));
-  DG_TRY(make_tmap(&t_wr, d_wr, n_experts, d, d, 128));
-  DG_TRY(make_tmap(&t_xp, x_perm, static_cast<uint64_t>(t) * top_k, d, d, 32));
-  DG_TRY(make_tmap(&t_wgu, d_w_gu, static_cast<uint64_t>(n_experts) * 2 * hidden, d, d, 128));
-  DG_TRY(make_tmap(&t_h, hbuf, static_cast<uint64_t>(t) * top_k, hidden, hidden, 32));
-  DG_TRY(make_tmap(&t_wd, d_w_d, static_cast<uint64_t>(n_experts) * d, hidden, hidden, 128));
-  if (shared_hidden > 0) {
-    DG_TRY(make_tmap(&t_wsgu, d_ws_gu, 2ull * shared_hidden, d, d, 128));
-    DG_TRY(make_tmap(&t_hs, hsbuf, t, shared_hidden, shared_hidden, 32));
-    DG_TRY(make_tmap(&t_wsd, d_ws_d, d, shared_hidden, shared_hidden, 128));
-  }
-  // router
-  const bool shared = shared_hidden > 0;
-  CluParams pr = clu_params(n_experts, t, d / 64, m.split_r, err, nullptr, kRouterChunk);
-  pr.router_logits = d_router_logits ? d_router_logits : rlog;
-  pr.ids = ids;
-  pr.wts = wts;
-  pr.top_k = top_k;
-  const bool wide = group_wide(static_cast<long long>(t) * top_k, n_experts);
-  const int nch = wide ? kGroupWideN : kGroupN;
-  pr.route = RouteArgs{ids, t, top_k, n_experts, nch, offs, perm, chunks, icnt};
-  pr.ticket = route_ticket;
-  DG_TRY(launch_cluster<kCluRouter>(t_wr, t_x32, pr, st, -1));
-  DG_TRY(launch_pdl(gather_rows_kernel, dim3(cdiv(t * top_k, 4)), dim3(256), 0, st,
-                    static_cast<const __nv_bfloat16*>(d_x), perm, top_k, d, t * top_k, x_perm,
-                    ExpertPrefetch{chunks, icnt, kPrefetchExperts, d_w_gu, 2ll * hidden * d * 2},
-                    nullptr));
+  return moe_ffn_impl(false, MoeScales{}, d_x, d_residual, d_wr, d_w_gu, d_w_d, d_ws_gu, d_ws_d,
+                      d_y, d_ids, d_weights, d_router_logits, t, d, n_experts, top_k, hidden,
+                      shared_hidden, d_workspace, workspace_bytes, stream);
+}
+
+int dg_moe_ffn_e4m3(const void* d_x, const float* d_residual, const void* d_wr,
+                    const void* d_w_gu, const float* d_w_gu_scale, const void* d_w_d,
+                    const float* d_w_d_scale, const void* d_ws_gu, const float* d_ws_gu_scale,
+                    const void* d_ws_d, const float* d_ws_d_scale, float* d_y, int32_t* d_ids,
+                    float* d_weights, float* d_router_logits, int32_t t, int32_t d,
+                    int32_t n_experts, int32_t top_k, int32_t hidden, int32_t shared_hidden,
+                    void* d_workspace, size_t workspace_bytes, void* stream) {
+  return moe_ffn_impl(true, MoeScales{d_w_gu_scale, d_w_d_scale, d_ws_gu_scale, d_ws_d_scale},
+                      d_x, d_residual, d_wr, d_w_gu, d_w_d, d_ws_gu, d_ws_d, d_y, d_ids,
+                      d_weights, d_router_logits, t, d, n_experts, top_k, hidden, shared_hidden,
+                      d_workspace, workspace_bytes, stream);
+}
+
+int dg_quantize_e4m3(const void* d_in, int32_t rows, int32_t cols, int64_t ld_in,
+                     uint8_t* d_codes, int64_t ld_codes, float* d_scales, void* stream) {
+  if (!d_in || !d_codes || !d_scales) return fail(DG_ERR_INVALID_ARG, "null pointer argument");
+  if (rows < 0 || cols < 16 || cols % 16 || ld_in < cols || ld_in % 8 || ld_codes < cols ||
+      ld_codes % 16 || ld_codes > (1 << 30))
+    return fail(DG_ERR_INVALID_ARG,
+                "need cols %% 16 == 0, ld_in >= cols, ld_in %% 8 == 0, ld_codes >= cols, "
+                "ld_codes %% 16 == 0");
+  if (reinterpret_cast<uintptr_t>(d_in) % 16 || reinterpret_cast<uintptr_t>(d_codes) % 16 ||
+      reinterpret_cast<uintptr_t>(d_scales) % 4)
+    return fail(DG_ERR_INVALID_ARG, "misaligned pointer");
+  if (rows == 0) return DG_OK;
+  QuantJob j{};
+  j.seg[0] = QuantSeg{static_cast<const __nv_bfloat16*>(d_in), ld_in, nullptr, 1, rows, cols,
+                      d_codes, ld_codes, d_scales};
+  j.n_seg = 1;
+  DG_TRY(launch_pdl(quant_rows_kernel, dim3(cdiv(rows, 8)), dim3(256), 0, S(stream), j,
+                    static_cast<const int*>(nullptr)));
   DG_LAUNCHED();
-  GemmParams pg{};
-  pg.chunks = chunks;
-  pg.chunk_count = icnt;
-  pg.m_tiles = cdiv(2 * hidden, 128);
-  pg.n_chunk = nch;
-  pg.alt_m_tiles = cdiv(2 * shared_hidden, 128);
-  pg.alt_chunks = cdiv(t, nch);
-  pg.alt_tokens = t;
-  pg.a_rows_per_group = 2 * hidden;
-  pg.kb_total = d / 64;
-  pg.m_valid = 2 * hidden;
-  pg.out_bf16 = hbuf;
-  pg.ld_out = hidden;
-  pg.alt_group = shared ? n_experts : -1;
-  pg.alt_kb_total = d / 64;
-  pg.alt_m_valid = 2 * shared_hidden;
-  pg.alt_out_bf16 = hsbuf;
-  pg.alt_ld_out = shared_hidden;
-  pg.err = err;
-  if (wide)
-    DG_TRY((launch_gemm<kGroupWideN, kGroupWideStages, kEpiGluBf16>(
-        t_wgu, t_xp, pg, sms, st, -1, shared ? &t_wsgu : nullptr, shared ? &t_x32 : nullptr)));
-  else
-    DG_TRY((launch_gemm<kGroupN, kGroupStages, kEpiGluBf16>(
-        t_wgu, t_xp, pg, sms, st, -1, shared ? &t_wsgu : nullptr, shared ? &t_x32 : nullptr)));
-  GemmParams pd{};
-  pd.chunks = chunks;
-  pd.chunk_count = icnt;
-  pd.m_tiles = cdiv(d, 128);
-  pd.n_chunk = nch;
-  pd.alt_m_tiles = cdiv(d, 128);
-  pd.alt_chunks = cdiv(t, nch);
-  pd.alt_tokens = t;
-  pd.a_rows_per_group = d;
-  pd.kb_total = hidden / 64;
-  pd.m_valid = d;
-  pd.out_f32 = y_slot;
-  pd.ld_out = d;
-  pd.perm = perm;
-  pd.scale = wts;
-  pd.alt_group = shared ? n_experts : -1;
-  pd.alt_kb_total = shared_hidden / 64;
-  pd.alt_m_valid = d;
-  pd.alt_out_f32 = ysh;
-  pd.alt_ld_out = d;
-  pd.err = err;
-  if (wide)
-    DG_TRY((launch_gemm<kGroupWideN, kGroupWideStages, kEpiScatterF32>(
-        t_wd, t_h, pd, sms, st, -1, shared ? &t_wsd : nullptr, shared ? &t_hs : nullptr)));
-  else
-    DG_TRY((launch_gemm<kGroupN, kGroupStages, kEpiScatterF32>(
-        t_wd, t_h, pd, sms, st, -1, shared ? &t_wsd : nullptr, shared ? &t_hs : nullptr)));
-  const float* ysh_ptr = shared ? ysh : nullptr;
-  if (d_residual)
-    DG_CUDA(cudaMemcpyAsync(d_y, d_residual, static_cast<size_t>(t) * d * 4,
-                            cudaMemcpyDeviceToDevice, st));
-  else
-    DG_CUDA(cudaMemsetAsync(d_y, 0, static_cast<size_t>(t) * d * 4, st));
-  DG_TRY(launch_pdl(moe_combine_norm_kernel<__nv_bfloat16>, dim3(t), dim3(256), 0, st, d_y, y_slot, top_k, ysh_ptr, d, nullptr,
-                                                            0.f, nullptr, nullptr));
-  DG_LAUNCHED();
-  if (d_ids)
-    DG_CUDA(cudaMemcpyAsync(d_ids, ids, static_cast<size_t>(t) * top_k * 4,
-                            cudaMemcpyDeviceToDevice, st));
-  if (d_weights)
-    DG_CUDA(cudaMemcpyAsync(d_weights, wts, static_cast<size_t>(t) * top_k * 4,
-                            cudaMemcpyDeviceToDevice, st));
   return DG_OK;
 }
 

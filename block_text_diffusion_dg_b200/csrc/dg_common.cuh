@@ -160,6 +160,16 @@ DG_DEV void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// D[tmem] (+)= A[smem] * B[smem]^T, e4m3 inputs, fp32 accumulate (kind::f8f6f4; K = 32 per
+// instruction, the same 32 bytes of a 128-byte swizzle row as 16 bf16).
+DG_DEV void umma_e4m3(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                      uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 // Arrive on `bar` once every previously issued UMMA of this thread has completed.
 DG_DEV void umma_commit(uint64_t* bar) {
   asm volatile(
@@ -173,6 +183,16 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n) {
   return (1u << 4)                              // D format: f32
          | (1u << 7)                            // A format: bf16
          | (1u << 10)                           // B format: bf16
+         | (static_cast<uint32_t>(n >> 3) << 17)  // N / 8
+         | (static_cast<uint32_t>(m >> 4) << 24); // M / 16
+}
+
+// Instruction descriptor for kind::f8f6f4 with e4m3 A and B (format code 0), fp32 D, both
+// operands K-major, dense.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int m, int n) {
+  return (1u << 4)                              // D format: f32
+         | (0u << 7)                            // A format: e4m3
+         | (0u << 10)                           // B format: e4m3
          | (static_cast<uint32_t>(n >> 3) << 17)  // N / 8
          | (static_cast<uint32_t>(m >> 4) << 24); // M / 16
 }

@@ -9,6 +9,9 @@
 //   warps 2-5: epilogue, TMEM lane quarter (warp % 4), one accumulator row per thread.
 // Work items are either arithmetic (dense layers, optional split-K) or a device-built list
 // (grouped experts, one item per (expert, 128-row tile, token chunk)).
+// With F8 the operands are e4m3 codes (kind::f8f6f4): a 128-byte K slab holds 128 elements
+// instead of 64, the ring and descriptors are unchanged, and the epilogue first scales each
+// accumulator by its weight row's scale and its token row's scale.
 //
 // lmhead_kernel: logits tile = X[256 tokens] * E[256 vocab rows]^T (two M=128 token tiles,
 // N = 256 vocab) with the epilogue reducing every row of the tile straight from TMEM to the
@@ -57,6 +60,12 @@ struct GemmParams {
   long long pf0_bytes;
   const void* pf1;
   long long pf1_bytes;
+  // e4m3 operands: one fp32 scale per weight row (indexed by global weight row) and per token
+  // row of B (indexed by B row); alt_* for the alternate group
+  const float* a_scale;
+  const float* b_scale;
+  const float* alt_a_scale;
+  const float* alt_b_scale;
   int* err;
   const int* done;
 };
@@ -187,7 +196,7 @@ DG_DEV void gemm_epilogue_chunk(const GemmParams& p, const GemmItem& w, const fl
   }
 }
 
-template <int MAXN, int STAGES, int EPI>
+template <int MAXN, int STAGES, int EPI, bool F8 = false>
 __global__ void __launch_bounds__(GemmCfg<MAXN, STAGES>::kThreads, 1)
     gemm_swapab_kernel(const __grid_constant__ CUtensorMap tm_a,
                        const __grid_constant__ CUtensorMap tm_b,
@@ -258,9 +267,10 @@ __global__ void __launch_bounds__(GemmCfg<MAXN, STAGES>::kThreads, 1)
           uint8_t* sa = smem + stage * C::kStageBytes;
           uint8_t* sb = sa + C::kABytes;
           mbar_arrive_expect_tx(&full[stage], bytes);
-          tma_load_2d(ta, &full[stage], sa, kb * 64, w.a_row, pol_a);
+          const int kx = kb * (F8 ? 128 : 64);  // elements per 128-byte slab
+          tma_load_2d(ta, &full[stage], sa, kx, w.a_row, pol_a);
           for (int bx = 0; bx < nbox; ++bx)
-            tma_load_2d(tb, &full[stage], sb + bx * 4096, kb * 64, w.b_row + bx * 32, pol_b);
+            tma_load_2d(tb, &full[stage], sb + bx * 4096, kx, w.b_row + bx * 32, pol_b);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
@@ -277,7 +287,8 @@ __global__ void __launch_bounds__(GemmCfg<MAXN, STAGES>::kThreads, 1)
       bool ok = true;
       for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
         const GemmItem w = gemm_item(p, it);
-        const uint32_t idesc = idesc_bf16_f32(128, (w.n + 15) & ~15);
+        const uint32_t idesc = F8 ? idesc_e4m3_f32(128, (w.n + 15) & ~15)
+                                  : idesc_bf16_f32(128, (w.n + 15) & ~15);
         if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, p.err)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * MAXN;
@@ -291,8 +302,12 @@ __global__ void __launch_bounds__(GemmCfg<MAXN, STAGES>::kThreads, 1)
           const uint64_t da = sdesc_sw128(sa);
           const uint64_t db = sdesc_sw128(sa + C::kABytes);
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            umma_bf16(d_tmem, da + 2 * k, db + 2 * k, idesc, (kb > w.kb0 || k > 0) ? 1u : 0u);
+          for (int k = 0; k < 4; ++k) {
+            if constexpr (F8)
+              umma_e4m3(d_tmem, da + 2 * k, db + 2 * k, idesc, (kb > w.kb0 || k > 0) ? 1u : 0u);
+            else
+              umma_bf16(d_tmem, da + 2 * k, db + 2 * k, idesc, (kb > w.kb0 || k > 0) ? 1u : 0u);
+          }
           umma_commit(&empty[stage]);
           if (++stage == STAGES) {
             stage = 0;
@@ -331,6 +346,20 @@ __global__ void __launch_bounds__(GemmCfg<MAXN, STAGES>::kThreads, 1)
           }
         }
       }
+      // e4m3: this lane's weight-row scale and token scales, loaded before the accumulator is ready
+      float row_scale = 1.0f;
+      float tok_scale[MAXN / 32];
+      if constexpr (F8) {
+        const float* as = w.alt ? p.alt_a_scale : p.a_scale;
+        const float* bs = w.alt ? p.alt_b_scale : p.b_scale;
+        const int m_valid = w.alt ? p.alt_m_valid : p.m_valid;
+        row_scale = (w.r_base + r < m_valid) ? as[w.a_row + r] : 0.0f;
+#pragma unroll
+        for (int cc = 0; cc < MAXN / 32; ++cc) {
+          const int j = cc * 32 + lane_id();
+          tok_scale[cc] = j < w.n ? bs[w.b_row + j] : 0.0f;
+        }
+      }
       if (!mbar_wait(&acc_full[acc], acc_phase, p.err)) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + acc * MAXN + (static_cast<uint32_t>(q * 32) << 16);
@@ -340,6 +369,11 @@ __global__ void __launch_bounds__(GemmCfg<MAXN, STAGES>::kThreads, 1)
         if (cc % kGroups == grp && c < w.n) {
           float v[32];
           tmem_ld32(t_row + c, v);
+          if constexpr (F8) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              v[i] *= row_scale * __shfl_sync(0xffffffffu, tok_scale[cc], i);
+          }
           if constexpr (EPI == kEpiScatterF32)
             gemm_epilogue_chunk<EPI>(p, w, v, c, r, dst_lane[cc], scale_lane[cc]);
           else

@@ -11,7 +11,8 @@ Recipes (the pages give no dataset; these stand in for their workloads, a
     RMSNorm weights are 1 unless `norm_jitter` > 0 (then 1 + N(0, jitter));
   * activations and attention inputs ~ N(0, 1);
   * prompt ids uniform over the vocabulary;
-  * sampler logits: row i is N(0,1) * s_i with s_i log-uniform in [0.5, 40].
+  * sampler logits: row i is N(0,1) * s_i with s_i log-uniform in [0.5, 40];
+  * quantiser inputs (scaled_rows): N(0,1) rows with per-row powers of two over 2^+-30.
 """
 import math
 
@@ -137,3 +138,17 @@ def moe_inputs(tokens=256, d_model=2816, n_experts=128, expert_hidden=704, share
         ws_gu = _normal((2 * shared_hidden, d_model), std, g, dtype, device)
         ws_d = _normal((d_model, shared_hidden), std, g, dtype, device)
     return dict(x=x, wr=wr, w_gu=w_gu, w_d=w_d, ws_gu=ws_gu, ws_d=ws_d)
+
+
+def scaled_rows(rows, cols, seed=0, device="cpu"):
+    """bf16 rows ~ N(0,1) x 2^j with j uniform in [-30, 30] per row; for rows >= 3, row 1 is
+    zero and every third element of row 2 is 2^-12 smaller than the rest (down to the e4m3
+    subnormal range once the row is scaled to 448)."""
+    g = _gen(seed, device)
+    x = torch.empty(rows, cols, dtype=torch.float32, device=device).normal_(0.0, 1.0, generator=g)
+    j = torch.randint(-30, 31, (rows, 1), generator=g, device=device).to(torch.float32)
+    x = x * torch.exp2(j)
+    if rows >= 3:
+        x[1] = 0.0
+        x[2, ::3] *= 2.0 ** -12
+    return x.to(torch.bfloat16)

@@ -59,7 +59,12 @@ enum {
   DG_ERR_UNSUPPORTED = -5  /* shape outside what the kernels implement */
 };
 
-enum { DG_DTYPE_BF16 = 0, DG_DTYPE_FP32 = 1 };
+/* Model storage types.  DG_DTYPE_BF16_E4M3 is the bf16 model with the FP8 expert format
+ * ([formats]: the model ships as BF16, FP8 or NVFP4 weights): the routed and shared expert
+ * weights are e4m3 codes with one fp32 scale per weight row, and the expert GEMMs take e4m3
+ * activations, quantised per row on the fly (scale = max|row| / 448, codes = rn_satfinite(x /
+ * scale)); attention, router, norms and the LM head stay bf16. */
+enum { DG_DTYPE_BF16 = 0, DG_DTYPE_FP32 = 1, DG_DTYPE_BF16_E4M3 = 2 };
 
 /* Model and decode configuration.  Shapes follow the pages' model ([course], [arch]). */
 typedef struct dg_config {
@@ -75,7 +80,7 @@ typedef struct dg_config {
   int32_t vocab;          /* V; bf16: multiple of 256 */
   int32_t canvas;         /* canvas length T; 256 in the pages ([canvas]); 1..256 */
   int32_t kv_capacity;    /* positions the caller's KV cache holds (multiple of 8) */
-  int32_t dtype;          /* DG_DTYPE_BF16 or DG_DTYPE_FP32 */
+  int32_t dtype;          /* DG_DTYPE_BF16, DG_DTYPE_FP32 or DG_DTYPE_BF16_E4M3 */
   float eps;              /* RMSNorm epsilon (1e-6) */
   float rope_theta;       /* RoPE base (10000) */
   double tau;             /* lock threshold on max-probability confidence (0.9) */
@@ -87,9 +92,14 @@ typedef struct dg_config {
                              times per prompt at the cost of scratch memory */
 } dg_config;
 
-/* Per-layer weights, all device pointers, dtype = config dtype unless noted.
+/* Per-layer weights, all device pointers, dtype = config dtype unless noted (bf16 for
+ * DG_DTYPE_BF16_E4M3, except the four expert matrices, which are then e4m3 codes).
  * Gate and up projections are stored row-interleaved: row 2j is gate unit j, row 2j+1 is
- * up unit j. */
+ * up unit j.  The *_scale arrays are read only with DG_DTYPE_BF16_E4M3 (dg_quantize_e4m3
+ * writes codes and scales in this layout).  An e4m3 matrix row of c codes is stored with a
+ * pitch of round_up(c, 128) bytes (DG_E4M3_PITCH), so that every 128-byte K slab of every row
+ * starts on a 128-byte boundary; the pad bytes are never read. */
+#define DG_E4M3_PITCH(cols) ((((cols) + 127) / 128) * 128)
 typedef struct dg_layer_weights {
   const float* attn_norm; /* fp32 [d] */
   const void* wqkv;       /* [(Hq + 2 Hkv) * hd, d]: q heads, then k heads, then v heads */
@@ -100,6 +110,10 @@ typedef struct dg_layer_weights {
   const void* w_d;        /* experts down [E, d, h] */
   const void* ws_gu;      /* shared expert gate/up [2hs, d], or NULL */
   const void* ws_d;       /* shared expert down [d, hs], or NULL */
+  const float* w_gu_scale;  /* fp32 [E, 2h], one per w_gu row */
+  const float* w_d_scale;   /* fp32 [E, d], one per w_d row */
+  const float* ws_gu_scale; /* fp32 [2hs], or NULL */
+  const float* ws_d_scale;  /* fp32 [d], or NULL */
 } dg_layer_weights;
 
 typedef struct dg_weights {
@@ -238,6 +252,29 @@ DG_API int dg_moe_ffn(const void* d_x, const float* d_residual, const void* d_wr
                int32_t n_experts, int32_t top_k, int32_t hidden, int32_t shared_hidden,
                void* d_workspace, size_t workspace_bytes, void* stream);
 
+/* The same MoE with e4m3 experts (the FP8 format of DG_DTYPE_BF16_E4M3): w_gu, w_d, ws_gu,
+ * ws_d are e4m3 codes in the layouts above, rows at DG_E4M3_PITCH, with fp32 row scales w_gu_scale [E, 2h],
+ * w_d_scale [E, d], ws_gu_scale [2hs], ws_d_scale [d] (the shared ones NULL when hs = 0).
+ * x and the router stay bf16; x is quantised per token and each expert's SiLU-GLU output
+ * per token-slot.  Same shapes, outputs, errors and workspace size as dg_moe_ffn. */
+DG_API int dg_moe_ffn_e4m3(const void* d_x, const float* d_residual, const void* d_wr,
+               const void* d_w_gu, const float* d_w_gu_scale, const void* d_w_d,
+               const float* d_w_d_scale, const void* d_ws_gu, const float* d_ws_gu_scale,
+               const void* d_ws_d, const float* d_ws_d_scale, float* d_y, int32_t* d_ids,
+               float* d_weights, float* d_router_logits, int32_t t, int32_t d, int32_t n_experts,
+               int32_t top_k, int32_t hidden, int32_t shared_hidden, void* d_workspace,
+               size_t workspace_bytes, void* stream);
+
+/* Row-wise e4m3 quantisation (the FP8 expert format): for each of `rows` bf16 rows of `cols`
+ * values (row pitch ld_in elements) writes `cols` codes (uint8) at a row pitch of ld_codes
+ * bytes, zero from cols to ld_codes, and one fp32 scale per row: scale = max|row| / 448 (IEEE
+ * division), code = rn_satfinite(x / scale), an all-zero row giving scale 0 and zero codes.
+ * Weights for the model and dg_moe_ffn_e4m3 take ld_codes = DG_E4M3_PITCH(cols).
+ * cols % 16 == 0, ld_in % 8 == 0, ld_codes % 16 == 0, ld_codes >= cols and 16-byte aligned
+ * pointers, else DG_ERR_INVALID_ARG before any launch.  Asynchronous on `stream`. */
+DG_API int dg_quantize_e4m3(const void* d_in, int32_t rows, int32_t cols, int64_t ld_in,
+                            uint8_t* d_codes, int64_t ld_codes, float* d_scales, void* stream);
+
 /* ---- tracing ------------------------------------------------------------------------- */
 
 /* Kernels that dg_profile_kernel can time. */
@@ -256,10 +293,11 @@ enum {
   DG_KERNEL_RESIDUAL_NORM = 11, /* residual add + RMSNorm */
   DG_KERNEL_ROUTER_TOPK = 12,   /* reserved: top-k selection (inside kind 8 on bf16) */
   DG_KERNEL_ROUTE = 13,         /* reserved: expert permutation (inside kind 8 on bf16) */
-  DG_KERNEL_GATHER = 14,        /* permuted token rows */
+  DG_KERNEL_GATHER = 14,        /* permuted token rows (e4m3 experts: quantised as well) */
   DG_KERNEL_COMBINE_NORM = 15,  /* weighted expert sum + RMSNorm */
   DG_KERNEL_EMBED = 16,         /* embedding gather + RMSNorm */
-  DG_KERNEL_KINDS = 17
+  DG_KERNEL_QUANT_H = 17,       /* e4m3 experts: per-row quantisation of the SiLU-GLU output */
+  DG_KERNEL_KINDS = 18
 };
 
 /* Number of kernels this library has launched in the calling process (all entry points). */
