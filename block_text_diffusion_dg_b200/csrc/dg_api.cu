@@ -298,6 +298,7 @@ struct ExpertPass {
   bool f8;
   const int32_t* perm;
   const float* topk_w;
+  float* w_perm;            // [n k]: topk_w in permuted order (written by the gather)
   const int4* chunks;
   const int* n_chunks;
   const __nv_bfloat16* xn;  // normed tokens [n, d]
@@ -341,17 +342,18 @@ int launch_experts(const ExpertPass& e, int sms, cudaStream_t st) {
   prof_before(kind_g, st);
   if (e.f8) {
     QuantJob j{};
-    j.seg[0] = QuantSeg{e.xn, e.d, e.perm, e.k, n_slots, e.d,
+    j.seg[0] = QuantSeg{e.xn, e.d, e.perm, e.k, e.topk_w, e.w_perm, n_slots, e.d,
                         static_cast<uint8_t*>(e.x_perm), row_d, e.x_perm_scale};
-    j.seg[1] = QuantSeg{e.xn, e.d, nullptr, 1, e.n, e.d, static_cast<uint8_t*>(e.x_sh), row_d,
-                        e.x_sh_scale};
+    j.seg[1] = QuantSeg{e.xn, e.d, nullptr, 1, nullptr, nullptr, e.n, e.d,
+                        static_cast<uint8_t*>(e.x_sh), row_d, e.x_sh_scale};
     j.n_seg = shared ? 2 : 1;
     j.pf = epf;
     DG_TRY(launch_pdl(quant_rows_kernel, dim3(cdiv(n_slots + (shared ? e.n : 0), 8)), dim3(256),
                       0, st, j, e.done));
   } else {
     DG_TRY(launch_pdl(gather_rows_kernel, dim3(cdiv(n_slots, 4)), dim3(256), 0, st, e.xn, e.perm,
-                      e.k, e.d, n_slots, static_cast<__nv_bfloat16*>(e.x_perm), epf, e.done));
+                      e.k, e.d, n_slots, static_cast<__nv_bfloat16*>(e.x_perm), e.topk_w,
+                      e.w_perm, epf, e.done));
   }
   DG_LAUNCHED();
   prof_after(kind_g, st);
@@ -397,10 +399,10 @@ int launch_experts(const ExpertPass& e, int sms, cudaStream_t st) {
   if (e.f8) {
     const int kind_q = e.profile ? DG_KERNEL_QUANT_H : -1;
     QuantJob j{};
-    j.seg[0] = QuantSeg{e.h, e.hid, nullptr, 1, n_slots, e.hid, static_cast<uint8_t*>(e.hq), row_h,
-                        e.hq_scale};
-    j.seg[1] = QuantSeg{e.h_sh, e.hs, nullptr, 1, e.n, e.hs, static_cast<uint8_t*>(e.hsq), row_hs,
-                        e.hsq_scale};
+    j.seg[0] = QuantSeg{e.h, e.hid, nullptr, 1, nullptr, nullptr, n_slots, e.hid,
+                        static_cast<uint8_t*>(e.hq), row_h, e.hq_scale};
+    j.seg[1] = QuantSeg{e.h_sh, e.hs, nullptr, 1, nullptr, nullptr, e.n, e.hs,
+                        static_cast<uint8_t*>(e.hsq), row_hs, e.hsq_scale};
     j.n_seg = shared ? 2 : 1;
     prof_before(kind_q, st);
     DG_TRY(launch_pdl(quant_rows_kernel, dim3(cdiv(n_slots + (shared ? e.n : 0), 8)), dim3(256),
@@ -423,7 +425,7 @@ int launch_experts(const ExpertPass& e, int sms, cudaStream_t st) {
   q.out_f32 = e.y_slot;
   q.ld_out = e.d;
   q.perm = e.perm;
-  q.scale = e.topk_w;
+  q.scale = e.w_perm;
   q.alt_group = shared ? e.E : -1;
   q.alt_kb_total = cdiv(e.hs, kel);
   q.alt_m_valid = e.d;
@@ -489,6 +491,7 @@ struct dg_ctx {
   bool f8;  // e4m3 experts
   void *x_sh, *hq, *hsq;  // e4m3 codes: shared-expert tokens, h per slot, shared h per token
   float *x_perm_scale, *x_sh_scale, *hq_scale, *hsq_scale;
+  float* w_perm;  // route weights in permuted order
   float *y_slot, *y_shared;
   StatPartial* lm_part;
   float* logits;  // fp32 path
@@ -554,7 +557,7 @@ enum Buf {
   B_CANVAS, B_ARGMAX, B_PREV, B_LOCKED, B_STATE, B_TICKET, B_ERR, B_ENT, B_CONF, B_ROWH, B_X,
   B_XN, B_PART, B_Q, B_OPART, B_ML, B_O, B_RLOG, B_IDS, B_W, B_OFF, B_PERM, B_CHUNKS,
   B_NCHUNKS, B_RTICKET, B_XPERM, B_H, B_HS, B_YSLOT, B_YSH, B_LMPART, B_LOGITS, B_ROPE,
-  B_XPS, B_XSH, B_XSHS, B_HQ, B_HQS, B_HSQ, B_HSQS, B_END
+  B_XPS, B_XSH, B_XSHS, B_HQ, B_HQS, B_HSQ, B_HSQS, B_WPERM, B_END
 };
 
 struct Derived {
@@ -637,6 +640,7 @@ Plan plan(const dg_config& c, int sms) {
   sz[B_HQS] = f8 ? T * k * 4 : 0;
   sz[B_HSQ] = f8 ? T * hsp : 0;
   sz[B_HSQS] = f8 ? T * 4 : 0;
+  sz[B_WPERM] = bf16 ? T * k * 4 : 0;
   size_t o = 0;
   for (int b = 0; b < B_END; ++b) {
     p.off[b] = o;
@@ -858,6 +862,7 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     e.f8 = c->f8;
     e.perm = c->perm;
     e.topk_w = c->topk_w;
+    e.w_perm = c->w_perm;
     e.chunks = c->chunks;
     e.n_chunks = c->n_chunks;
     e.xn = static_cast<const __nv_bfloat16*>(c->xn);
@@ -1123,6 +1128,7 @@ int dg_create(const dg_config* cfg, const dg_weights* w, void* d_kv, void* d_scr
   c->hq_scale = reinterpret_cast<float*>(s + p.off[B_HQS]);
   c->hsq = s + p.off[B_HSQ];
   c->hsq_scale = reinterpret_cast<float*>(s + p.off[B_HSQS]);
+  c->w_perm = reinterpret_cast<float*>(s + p.off[B_WPERM]);
   const size_t kv_half = p.kv / 2;
   c->kc = c->kv;
   c->vtc = c->kv + kv_half;
@@ -1530,7 +1536,7 @@ int dg_canvas_attention(const void* d_q, const void* d_k, const void* d_vt, void
 namespace {
 enum MoeBuf {
   M_RLOG, M_IDS, M_W, M_OFF, M_PERM, M_CHUNKS, M_WORDS, M_XPERM, M_H, M_HS, M_YSH, M_YSLOT,
-  M_XPS, M_XSH, M_XSHS, M_HQ, M_HQS, M_HSQ, M_HSQS, M_END
+  M_XPS, M_XSH, M_XSHS, M_HQ, M_HQS, M_HSQ, M_HSQS, M_WPERM, M_END
 };
 struct MoePlan {
   size_t off[M_END];
@@ -1564,6 +1570,7 @@ MoePlan moe_plan(int t, int d, int E, int k, int hid, int hs) {
   sz[M_HQS] = tk * 4;
   sz[M_HSQ] = T * e4m3_pitch(static_cast<int>(hs1));  // e4m3: quantised shared h, scales
   sz[M_HSQS] = T * 4;
+  sz[M_WPERM] = tk * 4;       // route weights in permuted order
   size_t o = 0;
   for (int i = 0; i < M_END; ++i) {
     m.off[i] = o;
@@ -1647,6 +1654,7 @@ int moe_ffn_impl(bool f8, const MoeScales& sc, const void* d_x, const float* d_r
   e.f8 = f8;
   e.perm = perm;
   e.topk_w = wts;
+  e.w_perm = static_cast<float*>(at(M_WPERM));
   e.chunks = chunks;
   e.n_chunks = icnt;
   e.xn = static_cast<const __nv_bfloat16*>(d_x);
@@ -1746,8 +1754,8 @@ int dg_quantize_e4m3(const void* d_in, int32_t rows, int32_t cols, int64_t ld_in
     return fail(DG_ERR_INVALID_ARG, "misaligned pointer");
   if (rows == 0) return DG_OK;
   QuantJob j{};
-  j.seg[0] = QuantSeg{static_cast<const __nv_bfloat16*>(d_in), ld_in, nullptr, 1, rows, cols,
-                      d_codes, ld_codes, d_scales};
+  j.seg[0] = QuantSeg{static_cast<const __nv_bfloat16*>(d_in), ld_in, nullptr, 1, nullptr,
+                      nullptr, rows, cols, d_codes, ld_codes, d_scales};
   j.n_seg = 1;
   DG_TRY(launch_pdl(quant_rows_kernel, dim3(cdiv(rows, 8)), dim3(256), 0, S(stream), j,
                     static_cast<const int*>(nullptr)));

@@ -27,6 +27,8 @@ struct QuantSeg {
   long long ld_src;     // elements between source rows
   const int32_t* perm;  // null: row p reads source row p; else source row perm[p] / top_k
   int top_k;
+  const float* wsrc;    // with perm: wdst[p] = wsrc[perm[p]] (route weights in permuted order)
+  float* wdst;
   int rows, cols;       // cols % 16 == 0
   uint8_t* dst;
   long long ld_dst;     // bytes between destination rows (multiple of 16); [cols, ld_dst) = 0
@@ -97,7 +99,12 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const QuantJob job, con
   for (int sg = 0; sg < job.n_seg; ++sg) {
     const QuantSeg& q = job.seg[sg];
     if (row < q.rows) {
-      const int sr = q.perm ? q.perm[row] / q.top_k : row;
+      int sr = row;
+      if (q.perm) {
+        const int slot = q.perm[row];
+        if (lane_id() == 0 && q.wdst) q.wdst[row] = q.wsrc[slot];
+        sr = slot / q.top_k;
+      }
       quant_row_warp(q.src + static_cast<long long>(sr) * q.ld_src, q.cols,
                      static_cast<int>(q.ld_dst), q.dst + static_cast<long long>(row) * q.ld_dst,
                      q.scale + row);

@@ -40,8 +40,8 @@ struct GemmParams {
   __nv_bfloat16* out_bf16;
   long long ld_out;
   long long split_stride;
-  const int* perm;
-  const float* scale;
+  const int* perm;     // scatter: destination (token * k + slot) of each permuted row
+  const float* scale;  // scatter: route weight of each permuted row (indexed like B's rows)
   // the shared expert folded into a grouped launch (alt_group >= 0): its items read tm_a2 /
   // tm_b2 (rows of the unpermuted tokens), run alt_kb_total K slabs, write alt_out_* with no
   // permutation and weight 1
@@ -253,8 +253,12 @@ __global__ void __launch_bounds__(GemmCfg<MAXN, STAGES>::kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
+      // each item's descriptor is read one item ahead, so its load latency overlaps the copies
+      GemmItem wn{};
+      if (static_cast<int>(blockIdx.x) < n_items) wn = gemm_item(p, blockIdx.x);
       for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-        const GemmItem w = gemm_item(p, it);
+        const GemmItem w = wn;
+        if (it + static_cast<int>(gridDim.x) < n_items) wn = gemm_item(p, it + gridDim.x);
         const int nbox = (w.n + 31) >> 5;
         const uint32_t bytes = C::kABytes + nbox * 32 * 128;
         const CUtensorMap* ta = w.alt ? &tm_a2 : &tm_a;
@@ -285,8 +289,11 @@ __global__ void __launch_bounds__(GemmCfg<MAXN, STAGES>::kThreads, 1)
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
+      GemmItem wn{};
+      if (static_cast<int>(blockIdx.x) < n_items) wn = gemm_item(p, blockIdx.x);
       for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-        const GemmItem w = gemm_item(p, it);
+        const GemmItem w = wn;
+        if (it + static_cast<int>(gridDim.x) < n_items) wn = gemm_item(p, it + gridDim.x);
         const uint32_t idesc = F8 ? idesc_e4m3_f32(128, (w.n + 15) & ~15)
                                   : idesc_bf16_f32(128, (w.n + 15) & ~15);
         if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, p.err)) break;
@@ -328,8 +335,13 @@ __global__ void __launch_bounds__(GemmCfg<MAXN, STAGES>::kThreads, 1)
     const int grp = (warp - 2) >> 2;
     int acc = 0;
     uint32_t acc_phase = 0;
+    // descriptor one item ahead; the item's row data below are independent loads indexed by its
+    // B rows, issued before the accumulator wait
+    GemmItem wn{};
+    if (static_cast<int>(blockIdx.x) < n_items) wn = gemm_item(p, blockIdx.x);
     for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
-      const GemmItem w = gemm_item(p, it);
+      const GemmItem w = wn;
+      if (it + static_cast<int>(gridDim.x) < n_items) wn = gemm_item(p, it + gridDim.x);
       // scatter: this lane's token of each 32-wide chunk, loaded before the accumulator is ready
       int dst_lane[MAXN / 32];
       float scale_lane[MAXN / 32];
@@ -340,9 +352,8 @@ __global__ void __launch_bounds__(GemmCfg<MAXN, STAGES>::kThreads, 1)
           dst_lane[cc] = 0;
           scale_lane[cc] = 1.0f;
           if (!w.alt && j < w.n) {
-            const int dst = p.perm ? p.perm[w.b_row + j] : w.b_row + j;
-            dst_lane[cc] = dst;
-            scale_lane[cc] = p.scale ? p.scale[dst] : 1.0f;
+            dst_lane[cc] = p.perm ? p.perm[w.b_row + j] : w.b_row + j;
+            scale_lane[cc] = p.scale ? p.scale[w.b_row + j] : 1.0f;
           }
         }
       }

@@ -394,11 +394,15 @@ struct ExpertPrefetch {
   long long expert_bytes;
 };
 
-// x_perm[p] = xn[perm[p] / k]; 64 threads per permuted row, 4 rows per CTA, 16-byte copies.
+// x_perm[p] = xn[perm[p] / k] and w_perm[p] = topk_w[perm[p]] (the route weight in permuted
+// order, which the down GEMM's scatter reads by permuted row); 64 threads per permuted row, 4
+// rows per CTA, 16-byte copies.
 __global__ void __launch_bounds__(256) gather_rows_kernel(const __nv_bfloat16* __restrict__ xn,
                                                           const int32_t* __restrict__ perm,
                                                           int top_k, int d, int n_rows,
                                                           __nv_bfloat16* __restrict__ x_perm,
+                                                          const float* __restrict__ topk_w,
+                                                          float* __restrict__ w_perm,
                                                           ExpertPrefetch pf, const int* done) {
   pdl_enter();
   if (block_done(done)) return;
@@ -413,7 +417,9 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const __nv_bfloat16* _
   }
   const int p = blockIdx.x * 4 + (threadIdx.x >> 6);
   if (p >= n_rows) return;
-  const int t = perm[p] / top_k;
+  const int slot = perm[p];
+  if ((threadIdx.x & 63) == 0) w_perm[p] = topk_w[slot];
+  const int t = slot / top_k;
   const uint4* src = reinterpret_cast<const uint4*>(xn + static_cast<long long>(t) * d);
   uint4* dst = reinterpret_cast<uint4*>(x_perm + static_cast<long long>(p) * d);
   for (int i = threadIdx.x & 63; i < d / 8; i += 64) dst[i] = src[i];
