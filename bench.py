@@ -394,7 +394,8 @@ def run_ours(args, rank, world, local_rank):
     }
     # DRAM bytes (read + write) of one launch from the ncu capture summarised in profiles/
     # (dram__bytes_read.sum + dram__bytes_write.sum); None where no capture of the current kernel
-    traffic = {} if f8 else {"expert_gate_up": 1051851000 + 4439808}
+    traffic = ({"expert_gate_up": 532844544 + 5702400, "expert_down": 286637312 + 9329920} if f8
+               else {"expert_gate_up": 1051851000 + 4439808})
     roof = None
     if args.roofline_kernel in algo and rec:
         achieved = algo[args.roofline_kernel] / (avg_ms / 1e3) / 1e9
