@@ -1,7 +1,7 @@
 // fp8.cuh -- e4m3 quantisation for the FP8 expert format.
 //
 // The model ships as BF16, FP8 or NVFP4 weights (jakiprompt.pl, "Diffusion Gemma – nowy model
-// Google", section "Wymagania sprzętowe"); the pages give no scheme, so the plainest symmetric
+// językowy Google", section "Wymagania sprzętowe"); the pages give no scheme, so the plainest symmetric
 // one is used.  A row v (an output row of an expert weight matrix, or one token's activation row
 // where it enters an expert GEMM) gets one fp32 scale s = max|v| / 448 and e4m3 codes
 // rn_satfinite(v / s) (IEEE division, round to nearest even, clamp to +-448); an all-zero row

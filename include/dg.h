@@ -60,7 +60,7 @@ enum {
 };
 
 /* Model storage types.  DG_DTYPE_BF16_E4M3 is the bf16 model with the FP8 expert format
- * ([formats]: the model ships as BF16, FP8 or NVFP4 weights): the routed and shared expert
+ * ([pl]: the model ships as BF16, FP8 or NVFP4 weights): the routed and shared expert
  * weights are e4m3 codes with one fp32 scale per weight row, and the expert GEMMs take e4m3
  * activations, quantised per row on the fly (scale = max|row| / 448, codes = rn_satfinite(x /
  * scale)); attention, router, norms and the LM head stay bf16. */

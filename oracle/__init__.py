@@ -40,8 +40,8 @@ Sources (the pages describe the method in prose only; no code, no equations):
           "Cách thức hoạt động của khuếch tán văn bản": canvas of random placeholder
           tokens, iterative refinement that locks correct tokens and uses them as
           context; a new "diffusion head" on the Gemma 4 base.
-[formats] jakiprompt.pl, "Diffusion Gemma – nowy model Google", section "Wymagania
-          sprzętowe" (hardware requirements): the model ships as BF16, FP8 and NVFP4
+[pl]      jakiprompt.pl, "Diffusion Gemma – nowy model językowy Google", section
+          "Wymagania sprzętowe" (hardware requirements): the model ships as BF16, FP8 and NVFP4
           weights (52 / 27 / 18 GB); [course] table 2.2 quotes fp8 on an H100.
 [philox]  Salmon, Moraes, Dror & Shaw, "Parallel random numbers: as easy as 1, 2, 3",
           SC'11: the Philox4x32-10 counter-based generator.

@@ -1,6 +1,6 @@
 """FP8 (e4m3) quantisation of expert weights and activations (oracle side, test infrastructure).
 
-[formats] lists the weight formats the model ships in (BF16, FP8 and NVFP4, with their memory
+[pl] lists the weight formats the model ships in (BF16, FP8 and NVFP4, with their memory
 footprints) and [course] table 2.2 quotes the fp8 speed on one H100; neither page gives the
 scheme, so the plainest symmetric one is read here:
 
