@@ -89,3 +89,63 @@ def test_standalone_shape_checks(L):
                                    None, 0, None) == -1
     assert lib.dg_sampler_step(None, 0, 256, 262144, 0, 0, 1, 0.9, 0.005, 48, 0, None, None, None,
                                None, None, None, None) == -1
+
+
+def test_e4m3_config_and_workspace(L):
+    from block_text_diffusion_dg_b200.api import make_config, workspace_bytes
+    from dg_synth import SHAPES
+    c16 = make_config(SHAPES["a4b"], kv_capacity=5376)
+    c8 = make_config(SHAPES["a4b"], kv_capacity=5376, experts="e4m3")
+    assert c8.dtype == L.DTYPE_BF16_E4M3 and c16.dtype == L.DTYPE_BF16
+    kv16, sc16 = workspace_bytes(c16)
+    kv8, sc8 = workspace_bytes(c8)
+    assert kv8 == kv16  # the KV cache stays bf16
+    # x_perm shrinks to one byte per code at the 128-byte pitch; the e4m3 buffers are added
+    assert sc8 != sc16 and sc8 % 256 == 0
+    with pytest.raises(ValueError):
+        make_config(SHAPES["tiny_fp32"], kv_capacity=512, experts="e4m3")
+    with pytest.raises(ValueError):
+        make_config(SHAPES["small_bf16"], kv_capacity=512, experts="int4")
+    from block_text_diffusion_dg_b200 import e4m3_pitch
+    assert [e4m3_pitch(c) for c in (16, 128, 129, 704, 2112, 2816)] == [128, 128, 256, 768, 2176,
+                                                                       2816]
+
+
+def test_quantiser_argument_checks(L):
+    lib = L.lib()
+    a = 1 << 20  # a 16-byte aligned address that is never dereferenced: checks run first
+    assert lib.dg_quantize_e4m3(None, 4, 64, 64, a, 64, a, None) == -1
+    assert lib.dg_quantize_e4m3(a, 4, 24, 24, a, 32, a, None) == -1      # cols % 16
+    assert lib.dg_quantize_e4m3(a, 4, 64, 60, a, 64, a, None) == -1      # ld_in < cols
+    assert lib.dg_quantize_e4m3(a, 4, 64, 64, a, 48, a, None) == -1      # ld_codes < cols
+    assert lib.dg_quantize_e4m3(a, 4, 64, 64, a, 72, a, None) == -1      # ld_codes % 16
+    assert lib.dg_quantize_e4m3(a + 8, 4, 64, 64, a, 64, a, None) == -1  # misaligned input
+    assert lib.dg_quantize_e4m3(a, 4, 64, 64, a + 4, 64, a, None) == -1  # misaligned codes
+    assert "ld_codes" in lib.dg_last_error().decode() or "misaligned" in lib.dg_last_error().decode()
+    assert lib.dg_quantize_e4m3(a, 0, 64, 64, a, 64, a, None) == 0       # nothing to do
+
+
+def test_e4m3_moe_requires_scales(L):
+    lib = L.lib()
+    n = C.c_size_t()
+    assert lib.dg_moe_workspace_bytes(256, 2816, 128, 8, 704, 2112, C.byref(n)) == 0
+    a = 1 << 20
+    rc = lib.dg_moe_ffn_e4m3(a, None, a, a, None, a, a, a, a, a, a, a, None, None, None, 256, 2816,
+                             128, 8, 704, 2112, a, n.value, None)
+    assert rc == -1 and "scales" in lib.dg_last_error().decode()
+
+
+def test_e4m3_create_requires_scales(L):
+    lib = L.lib()
+    cfg = _cfg(L, "small_bf16", experts="e4m3", kv_capacity=1024)
+    a = 1 << 20
+    layers = (L.LayerWeights * cfg.n_layers)()
+    for lw in layers:
+        for name in ("attn_norm", "wqkv", "wo", "ffn_norm", "wr", "w_gu", "w_d", "ws_gu", "ws_d",
+                     "w_gu_scale", "w_d_scale", "ws_gu_scale", "ws_d_scale"):
+            setattr(lw, name, a)
+    layers[1].ws_d_scale = None
+    w = L.Weights(embed=a, final_norm=a, layers=layers)
+    out = C.c_void_p()
+    assert lib.dg_create(C.byref(cfg), C.byref(w), a, a, None, C.byref(out)) == -1
+    assert "e4m3 expert scales" in lib.dg_last_error().decode()
