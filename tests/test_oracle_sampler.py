@@ -148,3 +148,83 @@ def test_mean_entropy_includes_every_position():
     res = smp.run_block(f, 1, 0, 2, 4)
     assert res["stop_step"] == 48
     assert math.isclose(res["steps"][0]["mean_entropy"], (math.log(2) + 3 * _hb(30.0)) / 4, rel_tol=1e-12)
+
+
+# ---- sampler variants: temperature, entropy-bound locking, sticky locks ------------------------
+
+@pytest.mark.parametrize("vocab,temp", [(2, 0.3), (5, 2.5), (1000, 0.7), (1000, 4.0)])
+def test_temperature_stats_against_scipy(vocab, temp):
+    from scipy.special import entr, softmax
+    rng = np.random.default_rng(vocab)
+    x = rng.standard_normal((16, vocab)) * 3
+    conf, ent, amax = smp.row_stats(x, temperature=temp)
+    p = softmax(x / temp, axis=1)
+    assert np.allclose(conf, p.max(axis=1), rtol=1e-12, atol=1e-15)
+    assert np.allclose(ent, entr(p).sum(axis=1), rtol=1e-10, atol=1e-13)
+    assert np.array_equal(amax, np.argmax(x, axis=1))
+
+
+def test_temperature_limits():
+    rng = np.random.default_rng(1)
+    x = rng.standard_normal((8, 64))
+    _, ent, _ = smp.row_stats(x, temperature=1e7)
+    assert np.allclose(ent, np.log(64), atol=1e-6)  # hot: uniform over the vocabulary
+    x[:, 7] = x.max(axis=1) + 0.5  # a unique maximum at index 7, 0.5 above the rest
+    conf, ent, amax = smp.row_stats(x, temperature=1e-3)
+    assert np.all(amax == 7) and np.all(conf >= 1 - 1e-15) and np.all(ent < 1e-100)
+    with pytest.raises(ValueError):
+        smp.row_stats(x, temperature=0.0)
+
+
+def test_entropy_bound_rule_hand_worked():
+    # row 0: one logit 20 above three others -> H ~ 3 * 21 e^-20 << 0.1: lock to 0
+    # row 1: uniform over 4 -> H = ln 4 > 0.1: re-noise
+    # row 2: two equal maxima -> H >= ln 2 > 0.1 although conf = 0.5: re-noise
+    # row 3: conf 0.95 (locks under the confidence rule) but entropy above a bound of 0.1
+    x = np.array([[20.0, 0, 0, 0], [1.0, 1, 1, 1], [3.0, 3, 0, 0],
+                  [np.log(0.95 / 0.05 * 3), 0, 0, 0]])
+    conf, ent, amax = smp.row_stats(x)
+    assert ent[3] > 0.1 and conf[3] > 0.9
+    nxt, lock = smp.sample_update(conf, amax, 9, 0, 1, 4, entropy=ent, rule="entropy_bound",
+                                  entropy_bound=0.1)
+    assert lock.tolist() == [True, False, False, False]
+    noise = smp.uniform_ids(9, 0, 1, np.arange(4), smp.TAG_RENOISE, 4)
+    assert nxt.tolist() == [0, noise[1], noise[2], noise[3]]
+    _, lock_c = smp.sample_update(conf, amax, 9, 0, 1, 4)
+    assert lock_c.tolist() == [True, False, False, True]
+    with pytest.raises(ValueError):
+        smp.sample_update(conf, amax, 9, 0, 1, 4, rule="entropy_bound")
+
+
+def test_sticky_lock_keeps_its_token():
+    v = 8
+    conf1, amax1 = np.array([0.95, 0.2]), np.array([3, 1])
+    nxt1, lock1 = smp.sample_update(conf1, amax1, 5, 0, 1, v)
+    assert nxt1[0] == 3 and lock1.tolist() == [True, False]
+    conf2, amax2 = np.array([0.3, 0.2]), np.array([6, 2])  # position 0 loses its confidence
+    sticky, lock_s = smp.sample_update(conf2, amax2, 5, 0, 2, v, sticky=True, prev_canvas=nxt1,
+                                       prev_locked=lock1)
+    plain, lock_p = smp.sample_update(conf2, amax2, 5, 0, 2, v)
+    noise2 = smp.uniform_ids(5, 0, 2, np.arange(2), smp.TAG_RENOISE, v)
+    assert sticky.tolist() == [3, noise2[1]] and lock_s.tolist() == [True, False]
+    assert plain.tolist() == [noise2[0], noise2[1]] and lock_p.tolist() == [False, False]
+
+
+def test_sticky_block_commits_locked_tokens():
+    # position 0 is confident on token 2 at step 1 only, then flat; position 1 is never confident
+    v, steps = 4, 3
+
+    def logits(t, canvas):
+        x = np.zeros((2, v))
+        if t == 1:
+            x[0, 2] = 10.0
+        else:
+            x[0, 1] = 0.01  # argmax moves to 1, confidence ~ 0.25
+        return x
+
+    plain = smp.run_block(logits, 3, 0, v, 2, fixed_steps=steps)
+    sticky = smp.run_block(logits, 3, 0, v, 2, fixed_steps=steps, sticky=True)
+    assert plain["committed"].tolist() == [1, 0]        # argmax vector of the last step
+    assert sticky["committed"].tolist() == [2, 0]       # the sticky lock keeps token 2
+    assert sticky["steps"][2]["canvas_in"][0] == 2      # and feeds it to every later step
+    assert plain["steps"][2]["canvas_in"][0] != 2 or plain["steps"][1]["canvas_out"][0] != 2
