@@ -56,7 +56,8 @@ renormalises the k probabilities; a shared expert is added with weight 1;
 RoPE is rotate-half with theta 10000 at absolute positions; RMSNorm is
 pre-norm with eps 1e-6; embeddings are tied with the LM head; commit re-encodes
 the final argmax block causally, exactly like the prompt; FP8 experts are e4m3 with
-one scale per weight row and per activation row (quant.py).
+one scale per weight row and per activation row (quant.py); NVFP4 is e2m1 with an e4m3
+scale per 16-element block and an fp32 row scale.
 
 Parity status: every function here is pinned by a CPU test against a closed
 form, a brute-force evaluation, a library routine, published known-answer

@@ -24,7 +24,7 @@ only and is undone here with strided views.
 import numpy as np
 
 from .numerics import round_f32, round_storage
-from .quant import quantize_matrix, quantize_rows
+from .quant import dequantize_nvfp4, quantize_matrix, quantize_nvfp4_rows, quantize_rows
 
 
 def silu(x):
@@ -131,3 +131,43 @@ def moe_ffn_fp8(xn, w_r, w_gu, w_d, top_k, shared=None):
         y = y + ys
     return y, dict(router_logits=logits, ids=ids, weights=w, y_slot=y_slot, y_shared=ys,
                    x_codes=xq, x_scales=xs)
+
+
+# ---- NVFP4 experts (e2m1 elements, e4m3 block scales, fp32 row scales; see quant.py) ---------
+
+def _nvfp4(v):
+    """Dequantised NVFP4 image of the rows of v (float64)."""
+    return dequantize_nvfp4(*quantize_nvfp4_rows(v))
+
+
+def gate_up_nvfp4(x, gu):
+    """SiLU-GLU hidden (bf16-stored) from NVFP4-quantised token rows x [n, d] and gate/up rows
+    gu [2hid, d] (row-interleaved): the sums of dequantised products, exact in float64."""
+    acc = _nvfp4(x) @ _nvfp4(gu).T
+    return round_storage(silu(acc[:, 0::2]) * acc[:, 1::2], "bf16")
+
+
+def down_nvfp4(h, w_d):
+    """Down projection of h [n, hid] (NVFP4-quantised per row here) with NVFP4 weights [d, hid]."""
+    return _nvfp4(h) @ _nvfp4(w_d).T
+
+
+def moe_ffn_nvfp4(xn, w_r, w_gu, w_d, top_k, shared=None):
+    """MoE output with NVFP4 experts: the router as in moe_ffn (bf16 weights); expert weights,
+    the token rows and each expert's h quantised to NVFP4 row by row."""
+    xn = np.asarray(xn, dtype=np.float64)
+    t, d = xn.shape
+    logits, ids, w = router(xn, w_r, top_k)
+    y_slot = np.zeros((t, top_k, d), dtype=np.float64)
+    for e in np.unique(ids):
+        rows, slots = np.nonzero(ids == e)
+        h = gate_up_nvfp4(xn[rows], w_gu[e])
+        y_slot[rows, slots] = down_nvfp4(h, w_d[e])
+    y = np.zeros((t, d), dtype=np.float64)
+    for s in range(top_k):  # slot order 0..k-1
+        y = y + w[:, s:s + 1] * y_slot[:, s]
+    ys = None
+    if shared is not None:
+        ys = down_nvfp4(gate_up_nvfp4(xn, shared[0]), shared[1])
+        y = y + ys
+    return y, dict(router_logits=logits, ids=ids, weights=w, y_slot=y_slot, y_shared=ys)

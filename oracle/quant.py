@@ -16,10 +16,12 @@ scheme, so the plainest symmetric one is read here:
   * Activations are quantised where they enter an expert GEMM: the stored (bf16) normed hidden
     state, once per token, and the stored (bf16) SiLU-GLU output h, once per token-slot.
 
-Pinned in tests/test_oracle_quant.py: the 256-code table against the format definition written
-independently as bit fields, rounding against torch's float8_e4m3fn conversion on every binary32
-neighbourhood of the grid, ties, saturation, the error bound of a row quantisation, and the fp8
-MoE against the bf16 MoE when every operand already lies on the e4m3 grid.
+Pinned in tests/test_oracle_quant.py: the 256-code table against torch's float8_e4m3fn bit
+patterns, rounding against torch's conversion on every binary32 neighbourhood of the grid, ties,
+saturation, the error bound of a row quantisation, and the fp8 MoE against the bf16 MoE when every
+operand already lies on the e4m3 grid.  The NVFP4 part at the end (e2m1 elements with e4m3 block
+scales) is pinned by brute-force nearest rounding, on-grid identity, a closed-form error bound
+and the bf16 expert on grid operands.
 """
 import numpy as np
 
@@ -106,3 +108,87 @@ def quantize_matrix(w):
     lead = w.shape[:-1]
     q, s = quantize_rows(w.reshape(-1, w.shape[-1]))
     return q.reshape(w.shape), s.reshape(lead)
+
+
+# ---- NVFP4: e2m1 elements with one e4m3 scale per 16-element block ----------------------------
+#
+# The pages name NVFP4 as the 4-bit weight format (18 GB, [pl]) that Blackwell kernels run
+# ([blog], "NVFP4 kernels"), without its arithmetic.  Read here as: elements e2m1 (a sign bit,
+# two exponent bits with bias 1, one mantissa bit: 0, 0.5, 1, 1.5, 2, 3, 4, 6); every 16
+# consecutive elements of a row along K share one e4m3 block scale; every row has one binary32
+# scale g = max|row| / (6 * 448), so that the block scales use the e4m3 range.  With a = max|block|:
+#     s_b  = e4m3(a / 6 / g)                  (binary32 divisions, RNE to e4m3, clamped)
+#     code = e2m1(x / (s_b * g))              (binary32 product and division, RNE, clamped to 6)
+# and the dequantised element is code * s_b * g.  A block whose scale rounds to 0 has zero codes.
+
+E2M1_MAX = 6.0
+NVFP4_BLOCK = 16
+
+
+def e2m1_table():
+    """The value of each of the 16 e2m1 codes (bit 3 sign, bits 2-1 exponent, bit 0 mantissa)."""
+    out = np.empty(16, dtype=np.float64)
+    for c in range(16):
+        sign = -1.0 if c & 0x8 else 1.0
+        e = (c >> 1) & 0x3
+        m = c & 0x1
+        out[c] = sign * (m * 0.5 if e == 0 else (1.0 + m / 2.0) * 2.0 ** (e - 1))
+    return out
+
+
+def round_e2m1(v):
+    """Nearest e2m1 value (ties to the even mantissa), clamped to +-6; float64 out."""
+    v = np.asarray(v, dtype=np.float64)
+    a = np.abs(v)
+    _, ex = np.frexp(np.maximum(a, 1.0))        # binades [1,2), [2,4), [4,8); below 1 as [1,2)
+    binade = np.minimum(ex - 1, 2)
+    quantum = np.ldexp(1.0, binade - 1)         # one mantissa bit: spacing 0.5, 1, 2
+    r = np.minimum(np.rint(a / quantum) * quantum, E2M1_MAX)
+    return np.copysign(r, v)
+
+
+def encode_e2m1(values):
+    """Codes (uint8, 0..15) of values on the e2m1 grid."""
+    values = np.asarray(values, dtype=np.float64)
+    mags = e2m1_table()[:8]
+    a = np.abs(values)
+    code = np.searchsorted(mags, a).astype(np.int64)
+    if np.any(code > 7) or not np.array_equal(mags[np.minimum(code, 7)], a):
+        raise ValueError("value not on the e2m1 grid")
+    return (code | np.where(np.signbit(values), 0x8, 0)).astype(np.uint8)
+
+
+def quantize_nvfp4_rows(v):
+    """NVFP4 quantisation of a 2-D array of binary32-representable values, k % 16 == 0.
+
+    Returns (element values on the e2m1 grid float64 [n, k], block scales on the e4m3 grid
+    float64 [n, k / 16], row scales float32 [n]); the dequantised row is
+    values * repeat(block scales, 16) * row scale.
+    """
+    v = np.ascontiguousarray(np.asarray(v, dtype=np.float64).astype(np.float32))
+    n, k = v.shape
+    if k % NVFP4_BLOCK:
+        raise ValueError("row length must be a multiple of 16")
+    amax = np.max(np.abs(v), axis=1) if k else np.zeros(n, np.float32)
+    g = (amax / np.float32(E2M1_MAX * E4M3_MAX)).astype(np.float32)
+    blocks = v.reshape(n, k // NVFP4_BLOCK, NVFP4_BLOCK)
+    bmax = np.max(np.abs(blocks), axis=2)
+    sb = np.zeros(bmax.shape, dtype=np.float64)
+    q = np.zeros(blocks.shape, dtype=np.float64)
+    rows = g > 0
+    t = (bmax[rows] / np.float32(E2M1_MAX)).astype(np.float32)
+    t = (t / g[rows, None]).astype(np.float32)
+    sb[rows] = round_e4m3(t.astype(np.float64))
+    step = (sb.astype(np.float32) * g[:, None]).astype(np.float32)   # binary32 product
+    live = step > 0
+    quo = (blocks[live] / step[live][:, None]).astype(np.float32)
+    q[live] = round_e2m1(quo.astype(np.float64))
+    return q.reshape(n, k), sb, g
+
+
+def dequantize_nvfp4(q, sb, g):
+    """code * block scale * row scale (float64)."""
+    q = np.asarray(q, dtype=np.float64)
+    n, k = q.shape
+    s = np.repeat(np.asarray(sb, dtype=np.float64), NVFP4_BLOCK, axis=1)
+    return q * s * np.asarray(g, dtype=np.float64)[:, None]

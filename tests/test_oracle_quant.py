@@ -166,3 +166,106 @@ def test_fp8_moe_within_the_quantisation_bound_of_the_bf16_moe():
     err = np.abs(y8 - y16)
     assert np.all(err <= bound * 1.001 + 1e-12)
     assert err.max() > 0  # h quantisation did change something
+
+
+# ---- NVFP4 ---------------------------------------------------------------------------------
+
+from oracle.quant import (dequantize_nvfp4, e2m1_table, encode_e2m1, quantize_nvfp4_rows,  # noqa: E402
+                          round_e2m1)
+
+
+def test_e2m1_code_table():
+    # the eight magnitudes the format admits: exponent field 0 holds 0 and 0.5, then 1, 1.5 /
+    # 2, 3 / 4, 6; bit 3 is the sign
+    tab = e2m1_table()
+    assert tab[:8].tolist() == [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    assert np.array_equal(tab[8:], -tab[:8]) and np.signbit(tab[8])
+    assert np.array_equal(encode_e2m1(tab), np.arange(16, dtype=np.uint8))
+
+
+def test_e2m1_rounding_brute_force():
+    rng = np.random.default_rng(5)
+    x = np.concatenate([rng.uniform(-8, 8, 20000), np.arange(-7, 7.01, 0.125)])
+    got = round_e2m1(x)
+    grid = e2m1_table()[:8]
+    for v, g in zip(x, got):
+        a = abs(v)
+        if a >= 6:
+            assert g == np.copysign(6.0, v)
+            continue
+        dist = np.abs(grid - a)
+        best = np.flatnonzero(dist == dist.min())
+        if len(best) == 2:  # a tie: the even code (mantissa bit 0) wins
+            pick = best[0] if best[0] % 2 == 0 else best[1]
+        else:
+            pick = best[0]
+        assert g == np.copysign(grid[pick], v), (v, g)
+
+
+def _nvfp4_on_grid(rng, rows, k, j_lo=-14, j_hi=-8):
+    """Rows code * block scale * 2^j where every 16-block holds a +-6 code and the row's largest
+    block scale is 448: NVFP4 quantisation returns them exactly."""
+    codes = e2m1_table()[rng.integers(0, 8, (rows, k // 16, 16))]
+    codes[:, :, rng.integers(0, 16)] = 6.0
+    codes *= np.where(rng.random(codes.shape) < 0.5, -1.0, 1.0)
+    sb = e4m3_table()[rng.integers(0x30, 0x7F, (rows, k // 16))]
+    sb[:, 0] = 448.0
+    g = np.exp2(rng.integers(j_lo, j_hi, rows)).astype(np.float64)
+    return (codes * sb[:, :, None] * g[:, None, None]).reshape(rows, k), codes.reshape(rows, k), sb, g
+
+
+def test_nvfp4_rows_on_grid_are_exact():
+    rng = np.random.default_rng(6)
+    x, codes, sb, g = _nvfp4_on_grid(rng, 12, 64)
+    q, sb2, g2 = quantize_nvfp4_rows(x)
+    assert np.array_equal(q, codes) and np.array_equal(sb2, sb)
+    assert np.array_equal(g2.astype(np.float64), g)
+    assert np.array_equal(dequantize_nvfp4(q, sb2, g2), x)
+
+
+def test_nvfp4_error_bound_and_max_block():
+    rng = np.random.default_rng(7)
+    x = (rng.standard_normal((32, 128)) * np.exp2(rng.uniform(-10, 10, (32, 1)))).astype(np.float32)
+    x[4] = 0.0
+    q, sb, g = quantize_nvfp4_rows(x)
+    assert g[4] == 0 and not q[4].any()
+    d = dequantize_nvfp4(q, sb, g)
+    blocks = np.abs(x.astype(np.float64)).reshape(32, 8, 16)
+    bmax = np.repeat(blocks.max(axis=2), 16, axis=1)
+    # half an e2m1 spacing (<= |x| / 4, or 1/4 of the block step below 1) with a block step of
+    # at most (block max / 6) * (1 + 1/16) after the e4m3 rounding of the block scale
+    bound = 0.25 * np.abs(x) + 0.25 * bmax / 6 * (17 / 16)
+    assert np.all(np.abs(d - x) <= bound * (1 + 1e-6))
+    nz = g > 0
+    amax_blk = blocks.max(axis=2).argmax(axis=1)
+    assert np.all(sb[nz, amax_blk[nz]] == 448.0)  # the block holding the row maximum
+    assert np.all(np.abs(q[nz]).max(axis=1) == 6.0)
+
+
+def test_nvfp4_stages_equal_the_bf16_expert_on_grid_operands():
+    rng = np.random.default_rng(8)
+    n, d, hid = 8, 64, 32
+    x, *_ = _nvfp4_on_grid(rng, n, d, -6, -4)
+    w_gu, *_ = _nvfp4_on_grid(rng, 2 * hid, d, -16, -12)
+    w_d, *_ = _nvfp4_on_grid(rng, d, hid, -16, -12)
+    y16, h16 = om.expert_glu(x, w_gu, w_d, "bf16")
+    assert np.array_equal(om.gate_up_nvfp4(x, w_gu), h16)
+    hg, *_ = _nvfp4_on_grid(rng, n, hid, -8, -6)
+    ref = hg @ w_d.T
+    assert np.allclose(om.down_nvfp4(hg, w_d), ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+
+
+def test_nvfp4_moe_runs_and_routes_like_bf16():
+    rng = np.random.default_rng(9)
+    t, d, e, k, hid, hs = 32, 64, 8, 2, 32, 48
+    x = rng.standard_normal((t, d))
+    wr = rng.standard_normal((e, d)) * 0.02
+    w_gu = rng.standard_normal((e, 2 * hid, d)) * 0.02
+    w_d = rng.standard_normal((e, d, hid)) * 0.02
+    sh = (rng.standard_normal((2 * hs, d)) * 0.02, rng.standard_normal((d, hs)) * 0.02)
+    y4, i4 = om.moe_ffn_nvfp4(x, wr, w_gu, w_d, k, sh)
+    y16, i16 = om.moe_ffn(x, wr, w_gu, w_d, k, "bf16", sh)
+    assert np.array_equal(i4["ids"], i16["ids"])
+    # 4-bit elements: the outputs agree to the format's precision, not to bf16's
+    rel = np.linalg.norm(y4 - y16) / np.linalg.norm(y16)
+    assert 1e-3 < rel < 0.25, rel
