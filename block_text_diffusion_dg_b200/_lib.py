@@ -26,6 +26,7 @@ class Config(C.Structure):
         ("dtype", C.c_int32), ("eps", C.c_float), ("rope_theta", C.c_float),
         ("tau", C.c_double), ("h_bound", C.c_double), ("max_steps", C.c_int32),
         ("fixed_steps", C.c_int32), ("prefill_chunk", C.c_int32),
+        ("lock_rule", C.c_int32), ("entropy_lock", C.c_double), ("sticky_locks", C.c_int32),
     ]
 
 

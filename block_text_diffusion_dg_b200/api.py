@@ -32,11 +32,17 @@ def _need_cuda(t, name, dtype=None):
 
 
 def make_config(shape, *, kv_capacity, fixed_steps=16, max_steps=48, tau=0.9, h_bound=0.005,
-                eps=1e-6, rope_theta=10000.0, prefill_chunk=0, experts="bf16"):
-    """Config of a model shape; experts="e4m3" selects the FP8 expert format (bf16 model)."""
+                eps=1e-6, rope_theta=10000.0, prefill_chunk=0, experts="bf16",
+                lock_rule="confidence", entropy_lock=0.1, sticky=False):
+    """Config of a model shape; experts="e4m3" selects the FP8 expert format (bf16 model);
+    lock_rule="entropy_bound" locks positions with entropy <= entropy_lock (nats) instead of
+    confidence >= tau; sticky=True keeps a locked position's token for the rest of the block."""
     s = shape
     if experts not in ("bf16", "e4m3"):
         raise ValueError("experts must be 'bf16' or 'e4m3'")
+    rules = {"confidence": 0, "entropy_bound": 1}
+    if lock_rule not in rules:
+        raise ValueError("lock_rule must be 'confidence' or 'entropy_bound'")
     if s["storage"] == "fp32":
         if experts != "bf16":
             raise ValueError("the all-fp32 model has no e4m3 expert format")
@@ -50,7 +56,8 @@ def make_config(shape, *, kv_capacity, fixed_steps=16, max_steps=48, tau=0.9, h_
         vocab=s["vocab"], canvas=s["canvas"], kv_capacity=kv_capacity,
         dtype=dtype, eps=eps,
         rope_theta=rope_theta, tau=tau, h_bound=h_bound, max_steps=max_steps,
-        fixed_steps=fixed_steps, prefill_chunk=prefill_chunk)
+        fixed_steps=fixed_steps, prefill_chunk=prefill_chunk, lock_rule=rules[lock_rule],
+        entropy_lock=entropy_lock, sticky_locks=int(bool(sticky)))
 
 
 def workspace_bytes(cfg):

@@ -492,6 +492,7 @@ struct dg_ctx {
   void *x_sh, *hq, *hsq;  // e4m3 codes: shared-expert tokens, h per slot, shared h per token
   float *x_perm_scale, *x_sh_scale, *hq_scale, *hsq_scale;
   float* w_perm;  // route weights in permuted order
+  int32_t* commit_ids;  // sticky locks: the ids a block commits
   float *y_slot, *y_shared;
   StatPartial* lm_part;
   float* logits;  // fp32 path
@@ -530,6 +531,9 @@ int check_config(const dg_config* c) {
     return fail(DG_ERR_INVALID_ARG, "max_steps must be >= 1 and fixed_steps >= 0");
   if (c->prefill_chunk < 0 || c->prefill_chunk % 128 != 0 || c->prefill_chunk > 4096)
     return fail(DG_ERR_INVALID_ARG, "prefill_chunk must be 0 or a multiple of 128, <= 4096");
+  if (c->lock_rule < 0 || c->lock_rule > 1 || !(c->entropy_lock >= 0.0) || c->sticky_locks < 0 ||
+      c->sticky_locks > 1)
+    return fail(DG_ERR_INVALID_ARG, "lock_rule must be 0 or 1, entropy_lock >= 0, sticky 0 or 1");
   if (c->dtype == DG_DTYPE_BF16 || c->dtype == DG_DTYPE_BF16_E4M3) {
     if (c->head_dim != 128) return fail(DG_ERR_UNSUPPORTED, "bf16 path needs head_dim 128");
     if (c->d_model % 64 || c->expert_hidden % 64 || c->shared_hidden % 64)
@@ -557,7 +561,7 @@ enum Buf {
   B_CANVAS, B_ARGMAX, B_PREV, B_LOCKED, B_STATE, B_TICKET, B_ERR, B_ENT, B_CONF, B_ROWH, B_X,
   B_XN, B_PART, B_Q, B_OPART, B_ML, B_O, B_RLOG, B_IDS, B_W, B_OFF, B_PERM, B_CHUNKS,
   B_NCHUNKS, B_RTICKET, B_XPERM, B_H, B_HS, B_YSLOT, B_YSH, B_LMPART, B_LOGITS, B_ROPE,
-  B_XPS, B_XSH, B_XSHS, B_HQ, B_HQS, B_HSQ, B_HSQS, B_WPERM, B_END
+  B_XPS, B_XSH, B_XSHS, B_HQ, B_HQS, B_HSQ, B_HSQS, B_WPERM, B_COMMIT, B_END
 };
 
 struct Derived {
@@ -641,6 +645,7 @@ Plan plan(const dg_config& c, int sms) {
   sz[B_HSQ] = f8 ? T * hsp : 0;
   sz[B_HSQS] = f8 ? T * 4 : 0;
   sz[B_WPERM] = bf16 ? T * k * 4 : 0;
+  sz[B_COMMIT] = Tc * 4;  // committed ids with sticky locks
   size_t o = 0;
   for (int b = 0; b < B_END; ++b) {
     p.off[b] = o;
@@ -1129,6 +1134,7 @@ int dg_create(const dg_config* cfg, const dg_weights* w, void* d_kv, void* d_scr
   c->hsq = s + p.off[B_HSQ];
   c->hsq_scale = reinterpret_cast<float*>(s + p.off[B_HSQS]);
   c->w_perm = reinterpret_cast<float*>(s + p.off[B_WPERM]);
+  c->commit_ids = reinterpret_cast<int32_t*>(s + p.off[B_COMMIT]);
   const size_t kv_half = p.kv / 2;
   c->kc = c->kv;
   c->vtc = c->kv + kv_half;
@@ -1194,7 +1200,8 @@ int dg_canvas_init(dg_ctx* ctx, uint64_t seed, uint32_t block, void* stream) {
   ctx->seed = seed;
   ctx->block = block;
   DG_TRY(launch_pdl(canvas_init_kernel, dim3(cdiv(ctx->cfg.canvas, 256)), dim3(256), 0, S(stream),
-      ctx->canvas, ctx->cfg.canvas, ctx->cfg.vocab, seed, block, ctx->state, ctx->ticket));
+      ctx->canvas, ctx->cfg.canvas, ctx->cfg.vocab, seed, block, ctx->state, ctx->ticket,
+      ctx->locked));
   DG_LAUNCHED();
   return DG_OK;
 }
@@ -1225,6 +1232,9 @@ int dg_sample_update(dg_ctx* ctx, uint32_t step, void* stream) {
   a.step = step;
   a.tau = g.tau;
   a.h_bound = g.h_bound;
+  a.lock_rule = g.lock_rule;
+  a.entropy_lock = static_cast<float>(g.entropy_lock);
+  a.sticky = g.sticky_locks;
   a.max_steps = g.max_steps;
   a.fixed_steps = g.fixed_steps;
   a.canvas = ctx->canvas;
@@ -1248,11 +1258,21 @@ int dg_commit_block(dg_ctx* ctx, int32_t* d_out_ids, int32_t* d_state, void* str
   const dg_config& g = ctx->cfg;
   if (ctx->kv_len + g.canvas > g.kv_capacity) return fail(DG_ERR_CAPACITY, "cache full");
   cudaStream_t st = S(stream);
+  // the committed ids: the argmax of the stop step, or with sticky locks the locked tokens
+  const int32_t* ids = ctx->argmax;
+  if (g.sticky_locks) {
+    DG_TRY(launch_pdl(commit_ids_kernel, dim3(cdiv(g.canvas, 256)), dim3(256), 0, st,
+                      static_cast<const int32_t*>(ctx->canvas),
+                      static_cast<const int32_t*>(ctx->argmax),
+                      static_cast<const int32_t*>(ctx->locked), ctx->commit_ids, g.canvas));
+    DG_LAUNCHED();
+    ids = ctx->commit_ids;
+  }
   if (d_out_ids)
-    DG_CUDA(cudaMemcpyAsync(d_out_ids, ctx->argmax, g.canvas * 4, cudaMemcpyDeviceToDevice, st));
+    DG_CUDA(cudaMemcpyAsync(d_out_ids, ids, g.canvas * 4, cudaMemcpyDeviceToDevice, st));
   if (d_state)
     DG_CUDA(cudaMemcpyAsync(d_state, ctx->state, kStWords * 4, cudaMemcpyDeviceToDevice, st));
-  DG_TRY(run_forward(ctx, ctx->argmax, g.canvas, ctx->kv_len, 1, nullptr, st));
+  DG_TRY(run_forward(ctx, ids, g.canvas, ctx->kv_len, 1, nullptr, st));
   ctx->kv_len += g.canvas;
   return DG_OK;
 }

@@ -8,7 +8,9 @@
 // entropy is H = ln S - U / S (nats).  The decision rules follow the canvas description:
 // lock when conf >= tau, otherwise re-noise with the Philox draw of (position, step,
 // block, tag 1); stop after step t >= 2 when mean H < h_bound and the argmax vector equals
-// the previous step's.
+// the previous step's.  Variants: lock when H <= entropy_lock instead (the recipe's
+// "entropy_bound" sampler), and sticky locks (a locked position keeps its token for the rest
+// of the block instead of being re-decided every step).
 #pragma once
 #include "dg_common.cuh"
 #include "philox.cuh"
@@ -54,11 +56,15 @@ DG_DEV StatD stat_merge(const StatD& x, const StatD& y) {
 }
 
 __global__ void canvas_init_kernel(int32_t* canvas, int32_t t, int32_t vocab, uint64_t seed,
-                                   uint32_t block, int32_t* state, int32_t* ticket) {
+                                   uint32_t block, int32_t* state, int32_t* ticket,
+                                   int32_t* locked) {
   pdl_enter();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < t) canvas[i] = canvas_uniform_id(seed, block, 0u, static_cast<uint32_t>(i), 0u,
-                                           static_cast<uint32_t>(vocab));
+  if (i < t) {
+    canvas[i] = canvas_uniform_id(seed, block, 0u, static_cast<uint32_t>(i), 0u,
+                                  static_cast<uint32_t>(vocab));
+    if (locked) locked[i] = 0;
+  }
   if (blockIdx.x == 0 && threadIdx.x < kStWords) {
     state[threadIdx.x] = 0;
     if (threadIdx.x == 0) *ticket = 0;
@@ -191,6 +197,9 @@ struct SamplerArgs {
   uint32_t step;
   float tau;
   float h_bound;
+  int32_t lock_rule;   // 0: lock when conf >= tau; 1: lock when H <= entropy_lock
+  float entropy_lock;
+  int32_t sticky;      // nonzero: a locked position keeps its token (locked[] persists)
   int32_t max_steps;
   int32_t fixed_steps;
   int32_t* canvas;
@@ -214,17 +223,28 @@ DG_DEV bool sampler_row_finish(const SamplerArgs& p, int row, const StatD& r) {
     p.conf[row] = static_cast<float>(conf);
     p.entropy[row] = static_cast<float>(h);
     p.row_h[row] = h;
-    const bool lock = conf >= static_cast<double>(p.tau);
+    const bool lock = p.lock_rule == 0 ? conf >= static_cast<double>(p.tau)
+                                        : h <= static_cast<double>(p.entropy_lock);
+    const bool kept = p.sticky != 0 && p.locked[row] != 0;
     p.argmax[row] = r.a;
-    p.locked[row] = lock ? 1 : 0;
-    p.canvas[row] = lock ? r.a
-                         : canvas_uniform_id(p.seed, p.block, p.step, static_cast<uint32_t>(row),
-                                             1u, static_cast<uint32_t>(p.vocab));
+    p.locked[row] = (lock || kept) ? 1 : 0;
+    if (!kept)
+      p.canvas[row] = lock ? r.a
+                           : canvas_uniform_id(p.seed, p.block, p.step, static_cast<uint32_t>(row),
+                                               1u, static_cast<uint32_t>(p.vocab));
     __threadfence();
     is_last = (atomicAdd(p.ticket, 1) == p.rows - 1);
   }
   __syncthreads();
   return is_last;
+}
+
+// Committed ids with sticky locks: a locked position's canvas token, otherwise the argmax.
+__global__ void commit_ids_kernel(const int32_t* canvas, const int32_t* argmax,
+                                  const int32_t* locked, int32_t* out, int n) {
+  pdl_enter();
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) out[i] = locked[i] ? canvas[i] : argmax[i];
 }
 
 // Merge one row's nsplit partials (block-wide, fp64 tree) and finish the row.

@@ -90,6 +90,12 @@ typedef struct dg_config {
   int32_t prefill_chunk;  /* tokens per causal-encode pass of dg_kv_append (0 = canvas); a
                              multiple of 128, <= 4096; larger chunks stream the weights fewer
                              times per prompt at the cost of scratch memory */
+  /* Sampler variants (zero = the plain rule above).  The recipe's "entropy_bound" sampler
+   * ([canvas], A/B commands: bound 0.1) has no definition on the pages; read as: */
+  int32_t lock_rule;      /* 0: lock when conf >= tau; 1: lock when entropy <= entropy_lock */
+  double entropy_lock;    /* nats, >= 0 (rule 1) */
+  int32_t sticky_locks;   /* 1: a locked position keeps its token for the rest of the block
+                             and the commit takes it (0: locks are re-decided every step) */
 } dg_config;
 
 /* Per-layer weights, all device pointers, dtype = config dtype unless noted (bf16 for

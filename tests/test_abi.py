@@ -149,3 +149,19 @@ def test_e4m3_create_requires_scales(L):
     out = C.c_void_p()
     assert lib.dg_create(C.byref(cfg), C.byref(w), a, a, None, C.byref(out)) == -1
     assert "e4m3 expert scales" in lib.dg_last_error().decode()
+
+
+def test_sampler_variant_config(L):
+    from block_text_diffusion_dg_b200.api import make_config, workspace_bytes
+    from dg_synth import SHAPES
+    cfg = make_config(SHAPES["small_bf16"], kv_capacity=1024, lock_rule="entropy_bound",
+                      entropy_lock=0.1, sticky=True)
+    assert (cfg.lock_rule, cfg.entropy_lock, cfg.sticky_locks) == (1, 0.1, 1)
+    workspace_bytes(cfg)
+    for field, value in (("entropy_lock", -1.0), ("lock_rule", 2), ("sticky_locks", 3)):
+        bad = make_config(SHAPES["small_bf16"], kv_capacity=1024)
+        setattr(bad, field, value)
+        with pytest.raises(RuntimeError, match="INVALID_ARG"):
+            workspace_bytes(bad)
+    with pytest.raises(ValueError):
+        make_config(SHAPES["small_bf16"], kv_capacity=1024, lock_rule="top_p")
