@@ -166,11 +166,7 @@ def denoise_logits(cfg, weights, canvas, cache, keep_info=False):
     return (logits, infos) if keep_info else logits
 
 
-def causal_encode(cfg, weights, ids, cache):
-    """Prefill / commit: encode ids causally at positions P.. and append their K/V."""
-    p = cache.length
-    pos = p + np.arange(len(ids))
-    _, kv_new, _ = forward_tokens(cfg, weights, ids, pos, cache, causal=True)
+def _append(cache, kv_new):
     for l, (k, v) in enumerate(kv_new):
         if len(cache.k) <= l:
             cache.k.append(k)
@@ -181,8 +177,32 @@ def causal_encode(cfg, weights, ids, cache):
     return cache
 
 
-def decode(cfg, weights, prompt_ids, n_blocks, seed, fixed_steps=None):
-    """Block-autoregressive diffusion decode; returns committed ids and per-block records."""
+def causal_encode(cfg, weights, ids, cache):
+    """Prefill / commit: encode ids causally at positions P.. and append their K/V."""
+    p = cache.length
+    pos = p + np.arange(len(ids))
+    _, kv_new, _ = forward_tokens(cfg, weights, ids, pos, cache, causal=True)
+    return _append(cache, kv_new)
+
+
+def commit_reusing_canvas_kv(cfg, weights, canvas_in, cache):
+    """The commit variant that keeps the K/V the last denoise forward computed for the canvas:
+    the bidirectional forward of that step's input canvas at positions P..P+T-1, appended as is
+    (no causal re-encode of the committed ids).  The pages only say the block is committed to the
+    cache ([canvas] step 4, [arch]); re-encoding is the default reading, this is its alternative."""
+    p = cache.length
+    pos = p + np.arange(len(canvas_in))
+    _, kv_new, _ = forward_tokens(cfg, weights, canvas_in, pos, cache, causal=False)
+    return _append(cache, kv_new)
+
+
+def decode(cfg, weights, prompt_ids, n_blocks, seed, fixed_steps=None, commit="reencode"):
+    """Block-autoregressive diffusion decode; returns committed ids and per-block records.
+
+    commit="reencode" encodes each committed block causally like the prompt; "reuse_kv" keeps
+    the canvas K/V of the block's last denoise step instead (commit_reusing_canvas_kv)."""
+    if commit not in ("reencode", "reuse_kv"):
+        raise ValueError(f"unknown commit mode {commit!r}")
     cache = KVCache()
     causal_encode(cfg, weights, prompt_ids, cache)
     blocks = []
@@ -190,7 +210,11 @@ def decode(cfg, weights, prompt_ids, n_blocks, seed, fixed_steps=None):
         res = smp.run_block(lambda t, canvas: denoise_logits(cfg, weights, canvas, cache),
                             seed, b, cfg.vocab, cfg.canvas, max_steps=cfg.max_steps,
                             fixed_steps=fixed_steps, tau=cfg.tau, h_bound=cfg.h_bound)
-        causal_encode(cfg, weights, res["committed"], cache)
+        if commit == "reencode":
+            causal_encode(cfg, weights, res["committed"], cache)
+        else:
+            last = res["steps"][res["stop_step"] - 1]
+            commit_reusing_canvas_kv(cfg, weights, last["canvas_in"], cache)
         blocks.append(res)
     out = np.concatenate([b["committed"] for b in blocks]) if blocks else np.zeros(0, np.int64)
     return out, blocks, cache

@@ -115,3 +115,38 @@ def test_bf16_storage_points_are_rounded():
         a = infos[0][key]
         assert np.array_equal(a, round_bf16(a)), key
     assert np.array_equal(cache.k[0], round_bf16(cache.k[0]))
+
+
+def test_reuse_kv_commit_equals_reencode_when_tokens_only_see_themselves():
+    # zero blocks: every layer's K/V of a token depend on its own embedding and position only, so
+    # the bidirectional K/V of a canvas equal the causal K/V of the same ids; with tau = 0 the
+    # canvas never moves (the committed ids are the last step's input canvas)
+    cfg = _cfg(tau=0.0)
+    w = _weights(cfg, zero_blocks=True)
+    w["embed"] = np.random.default_rng(3).standard_normal((cfg.vocab, cfg.d_model)) * 0.02
+    ids_a, _, cache_a = om.decode(cfg, w, np.arange(5), 2, seed=9, fixed_steps=3)
+    ids_b, _, cache_b = om.decode(cfg, w, np.arange(5), 2, seed=9, fixed_steps=3,
+                                  commit="reuse_kv")
+    assert np.array_equal(ids_a, ids_b) and cache_a.length == cache_b.length
+    for l in range(cfg.n_layers):
+        assert np.array_equal(cache_a.k[l], cache_b.k[l]) and np.array_equal(cache_a.v[l], cache_b.v[l])
+
+
+def test_reuse_kv_commit_keeps_the_last_step_canvas_kv():
+    cfg = _cfg()
+    w = _weights(cfg, std=0.2)
+    ids, blocks, cache = om.decode(cfg, w, np.arange(6), 1, seed=4, fixed_steps=2,
+                                   commit="reuse_kv")
+    canvas_in = blocks[0]["steps"][1]["canvas_in"]
+    assert not np.array_equal(canvas_in, ids)  # nothing locked: the canvas is not the block
+    prompt_cache = om.causal_encode(cfg, w, np.arange(6), om.KVCache())
+    _, kv_last, _ = om.forward_tokens(cfg, w, canvas_in, 6 + np.arange(cfg.canvas), prompt_cache,
+                                      causal=False)
+    reenc = om.causal_encode(cfg, w, ids, om.causal_encode(cfg, w, np.arange(6), om.KVCache()))
+    for l in range(cfg.n_layers):
+        assert np.array_equal(cache.k[l][:, :6], prompt_cache.k[l])
+        assert np.array_equal(cache.k[l][:, 6:], kv_last[l][0])
+        assert np.array_equal(cache.v[l][:, 6:], kv_last[l][1])
+        assert not np.allclose(cache.k[l][:, 6:], reenc.k[l][:, 6:])  # not the re-encode
+    with pytest.raises(ValueError):
+        om.decode(cfg, w, np.arange(6), 1, seed=4, fixed_steps=2, commit="other")
