@@ -27,6 +27,7 @@ class Config(C.Structure):
         ("tau", C.c_double), ("h_bound", C.c_double), ("max_steps", C.c_int32),
         ("fixed_steps", C.c_int32), ("prefill_chunk", C.c_int32),
         ("lock_rule", C.c_int32), ("entropy_lock", C.c_double), ("sticky_locks", C.c_int32),
+        ("temperature", C.c_float), ("commit_reuse_kv", C.c_int32),
     ]
 
 
@@ -52,6 +53,7 @@ _PROTOS = {
     "dg_kv_truncate": (C.c_int, [_P, _I]),
     "dg_kv_append": (C.c_int, [_P, _P, _I, _P]),
     "dg_canvas_init": (C.c_int, [_P, C.c_uint64, C.c_uint32, _P]),
+    "dg_reset_block": (C.c_int, [_P, _P]),
     "dg_denoise_step": (C.c_int, [_P, C.c_uint32, _P]),
     "dg_sample_update": (C.c_int, [_P, C.c_uint32, _P]),
     "dg_commit_block": (C.c_int, [_P, _P, _P, _P]),

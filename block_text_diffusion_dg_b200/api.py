@@ -33,10 +33,15 @@ def _need_cuda(t, name, dtype=None):
 
 def make_config(shape, *, kv_capacity, fixed_steps=16, max_steps=48, tau=0.9, h_bound=0.005,
                 eps=1e-6, rope_theta=10000.0, prefill_chunk=0, experts="bf16",
-                lock_rule="confidence", entropy_lock=0.1, sticky=False):
+                lock_rule="confidence", entropy_lock=0.1, sticky=False, temperature=1.0,
+                commit="reencode"):
     """Config of a model shape; experts="e4m3" selects the FP8 expert format (bf16 model);
     lock_rule="entropy_bound" locks positions with entropy <= entropy_lock (nats) instead of
-    confidence >= tau; sticky=True keeps a locked position's token for the rest of the block."""
+    confidence >= tau; sticky=True keeps a locked position's token for the rest of the block;
+    temperature sets T of the sampler's softmax(logits / T); commit="reuse_kv" commits a block
+    by keeping the canvas K/V of its last denoise step instead of re-encoding it causally."""
+    if commit not in ("reencode", "reuse_kv"):
+        raise ValueError("commit must be 'reencode' or 'reuse_kv'")
     s = shape
     if experts not in ("bf16", "e4m3"):
         raise ValueError("experts must be 'bf16' or 'e4m3'")
@@ -57,7 +62,8 @@ def make_config(shape, *, kv_capacity, fixed_steps=16, max_steps=48, tau=0.9, h_
         dtype=dtype, eps=eps,
         rope_theta=rope_theta, tau=tau, h_bound=h_bound, max_steps=max_steps,
         fixed_steps=fixed_steps, prefill_chunk=prefill_chunk, lock_rule=rules[lock_rule],
-        entropy_lock=entropy_lock, sticky_locks=int(bool(sticky)))
+        entropy_lock=entropy_lock, sticky_locks=int(bool(sticky)), temperature=temperature,
+        commit_reuse_kv=int(commit == "reuse_kv"))
 
 
 def workspace_bytes(cfg):
@@ -119,6 +125,9 @@ class DiffusionModel:
     def canvas_init(self, seed, block, stream=None):
         check(lib().dg_canvas_init(self.handle, C.c_uint64(seed), block, _stream(stream)),
               "dg_canvas_init")
+
+    def reset_block(self, stream=None):
+        check(lib().dg_reset_block(self.handle, _stream(stream)), "dg_reset_block")
 
     def denoise_step(self, step, stream=None):
         check(lib().dg_denoise_step(self.handle, step, _stream(stream)), "dg_denoise_step")

@@ -531,6 +531,10 @@ int check_config(const dg_config* c) {
     return fail(DG_ERR_INVALID_ARG, "max_steps must be >= 1 and fixed_steps >= 0");
   if (c->prefill_chunk < 0 || c->prefill_chunk % 128 != 0 || c->prefill_chunk > 4096)
     return fail(DG_ERR_INVALID_ARG, "prefill_chunk must be 0 or a multiple of 128, <= 4096");
+  if (c->commit_reuse_kv < 0 || c->commit_reuse_kv > 1)
+    return fail(DG_ERR_INVALID_ARG, "commit_reuse_kv must be 0 or 1");
+  if (!(c->temperature >= 0.0f) || c->temperature > 1e4f)
+    return fail(DG_ERR_INVALID_ARG, "temperature must be in (0, 1e4] (0 means 1)");
   if (c->lock_rule < 0 || c->lock_rule > 1 || !(c->entropy_lock >= 0.0) || c->sticky_locks < 0 ||
       c->sticky_locks > 1)
     return fail(DG_ERR_INVALID_ARG, "lock_rule must be 0 or 1, entropy_lock >= 0, sticky 0 or 1");
@@ -669,13 +673,13 @@ int run_forward(dg_ctx* c, const int32_t* ids, int n, int pos0, int causal, cons
   const dg_config& g = c->cfg;
   prof_before(DG_KERNEL_EMBED, st);
   if (c->bf16)
-    DG_TRY(launch_pdl(embed_norm_kernel<__nv_bfloat16, __nv_bfloat16>, dim3(n), dim3(256), 0, st, 
-        ids, static_cast<const __nv_bfloat16*>(c->embed), g.d_model, c->layers[0].attn_norm, g.eps,
-        c->x, static_cast<__nv_bfloat16*>(c->xn), done));
+    DG_TRY(launch_pdl(embed_norm_kernel<__nv_bfloat16, __nv_bfloat16>, dim3(n), dim3(256), 0, st,
+        ids, static_cast<const __nv_bfloat16*>(c->embed), g.d_model, g.vocab,
+        c->layers[0].attn_norm, g.eps, c->x, static_cast<__nv_bfloat16*>(c->xn), done, c->err));
   else
-    DG_TRY(launch_pdl(embed_norm_kernel<float, float>, dim3(n), dim3(256), 0, st, ids, static_cast<const float*>(c->embed),
-                                                       g.d_model, c->layers[0].attn_norm, g.eps,
-                                                       c->x, static_cast<float*>(c->xn), done));
+    DG_TRY(launch_pdl(embed_norm_kernel<float, float>, dim3(n), dim3(256), 0, st, ids,
+        static_cast<const float*>(c->embed), g.d_model, g.vocab, c->layers[0].attn_norm, g.eps,
+        c->x, static_cast<float*>(c->xn), done, c->err));
   DG_LAUNCHED();
   prof_after(DG_KERNEL_EMBED, st);
   for (int l = 0; l < g.n_layers; ++l) {
@@ -932,6 +936,7 @@ int run_lm_head(dg_ctx* c, float* logits_out, const int* done, cudaStream_t st) 
     p.partials = c->lm_part;
     p.logits = logits_out;
     p.vocab = g.vocab;
+    p.inv_t = g.temperature > 0.0f ? 1.0f / g.temperature : 1.0f;
     p.err = c->err;
     p.done = done;
     const int grid = std::min(p.n_vtiles, c->sms);
@@ -953,8 +958,9 @@ int run_lm_head(dg_ctx* c, float* logits_out, const int* done, cudaStream_t st) 
       dst, g.vocab, done));
   DG_LAUNCHED();
   if (!logits_out) {
-    DG_TRY(launch_pdl(logits_stats_kernel<float, 16>, dim3(cdiv(g.vocab, 4096), T), dim3(256), 0, st, 
-        c->logits, g.vocab, 4096, c->lm_part, done));
+    DG_TRY(launch_pdl(logits_stats_kernel<float, 16>, dim3(cdiv(g.vocab, 4096), T), dim3(256), 0, st,
+        c->logits, g.vocab, 4096, c->lm_part, done,
+        g.temperature > 0.0f ? 1.0f / g.temperature : 1.0f));
     DG_LAUNCHED();
   }
   return DG_OK;
@@ -1206,6 +1212,14 @@ int dg_canvas_init(dg_ctx* ctx, uint64_t seed, uint32_t block, void* stream) {
   return DG_OK;
 }
 
+int dg_reset_block(dg_ctx* ctx, void* stream) {
+  DG_TRY(check_ctx(ctx));
+  DG_TRY(launch_pdl(block_reset_kernel, dim3(cdiv(ctx->cfg.canvas, 256)), dim3(256), 0, S(stream),
+                    ctx->state, ctx->ticket, ctx->locked, ctx->cfg.canvas));
+  DG_LAUNCHED();
+  return DG_OK;
+}
+
 int dg_denoise_step(dg_ctx* ctx, uint32_t step, void* stream) {
   DG_TRY(check_ctx(ctx));
   if (step < 1) return fail(DG_ERR_INVALID_ARG, "steps are numbered from 1");
@@ -1272,7 +1286,8 @@ int dg_commit_block(dg_ctx* ctx, int32_t* d_out_ids, int32_t* d_state, void* str
     DG_CUDA(cudaMemcpyAsync(d_out_ids, ids, g.canvas * 4, cudaMemcpyDeviceToDevice, st));
   if (d_state)
     DG_CUDA(cudaMemcpyAsync(d_state, ctx->state, kStWords * 4, cudaMemcpyDeviceToDevice, st));
-  DG_TRY(run_forward(ctx, ids, g.canvas, ctx->kv_len, 1, nullptr, st));
+  // re-encode causally, or keep the canvas K/V the last denoise step left in slots P..P+T-1
+  if (!g.commit_reuse_kv) DG_TRY(run_forward(ctx, ids, g.canvas, ctx->kv_len, 1, nullptr, st));
   ctx->kv_len += g.canvas;
   return DG_OK;
 }
@@ -1293,6 +1308,9 @@ int dg_check_device_status(dg_ctx* ctx, void* stream) {
   DG_CUDA(cudaStreamSynchronize(S(stream)));
   int err = 0;
   DG_CUDA(cudaMemcpy(&err, ctx->err, 4, cudaMemcpyDeviceToHost));
+  if (err == kDevErrBadId)
+    return fail(DG_ERR_INVALID_ARG, "a token id outside [0, %d) reached the embedding",
+                ctx->cfg.vocab);
   if (err != 0) return fail(DG_ERR_TIMEOUT, "a device wait gave up (code %d)", err);
   return DG_OK;
 }
@@ -1806,24 +1824,53 @@ constexpr size_t kStaticBytes = kStaticTicketOff + 256;
 static __device__ __align__(256) uint8_t g_sampler_scratch[kStaticBytes];
 
 namespace {
-std::mutex g_static_mu;
-void* g_static_ptr[256] = {};  // device address of g_sampler_scratch, per device ordinal
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+CtxGetCurrentFn ctx_current_fn() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
 
-// First call on a device looks up the array's device address with that device current.
+std::mutex g_static_mu;
+struct StaticAddr {
+  CUcontext ctx;  // the context the address belongs to
+  void* ptr;      // device address of g_sampler_scratch in that context
+};
+StaticAddr g_static_addr[256] = {};  // per device ordinal
+
+// The first call on a device (and the first after that device's context was replaced, e.g. by
+// cudaDeviceReset, which reloads this module at a new address) looks up the array's device
+// address with that device current; later calls reuse it.
 int static_scratch(void** out) {
   int dev = 0;
   DG_CUDA(cudaGetDevice(&dev));
   if (dev < 0 || dev >= 256) return fail(DG_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  CtxGetCurrentFn cur = ctx_current_fn();
+  CUcontext ctx = nullptr;
+  if (!cur || cur(&ctx) != CUDA_SUCCESS)
+    return fail(DG_ERR_CUDA, "cannot query the current CUDA context");
   std::lock_guard<std::mutex> lock(g_static_mu);
-  if (!g_static_ptr[dev]) {
+  StaticAddr& a = g_static_addr[dev];
+  if (!ctx || !a.ptr || a.ctx != ctx) {
     void* p = nullptr;
+    // also makes the device's primary context current when no context was yet
     const cudaError_t e = cudaGetSymbolAddress(&p, g_sampler_scratch);
     if (e != cudaSuccess || !p)
       return fail(DG_ERR_CUDA, "cudaGetSymbolAddress(sampler scratch) failed: %s",
                   cudaGetErrorString(e));
-    g_static_ptr[dev] = p;
+    if (!ctx && (cur(&ctx) != CUDA_SUCCESS || !ctx))
+      return fail(DG_ERR_CUDA, "no current CUDA context after the symbol lookup");
+    a.ctx = ctx;
+    a.ptr = p;
   }
-  *out = g_static_ptr[dev];
+  *out = a.ptr;
   return DG_OK;
 }
 }  // namespace
@@ -1863,10 +1910,10 @@ extern "C" int dg_sampler_step_static(const void* d_logits, int32_t dtype, int32
   const int* done = d_state + kStDone;
   if (dtype == DG_DTYPE_BF16)
     DG_TRY(launch_pdl(logits_stats_kernel<__nv_bfloat16, 32>, dim3(nchunk, rows), dim3(256), 0, st, 
-        static_cast<const __nv_bfloat16*>(d_logits), vocab, chunk, part, done));
+        static_cast<const __nv_bfloat16*>(d_logits), vocab, chunk, part, done, 1.0f));
   else
-    DG_TRY(launch_pdl(logits_stats_kernel<float, 16>, dim3(nchunk, rows), dim3(256), 0, st, 
-        static_cast<const float*>(d_logits), vocab, chunk, part, done));
+    DG_TRY(launch_pdl(logits_stats_kernel<float, 16>, dim3(nchunk, rows), dim3(256), 0, st,
+        static_cast<const float*>(d_logits), vocab, chunk, part, done, 1.0f));
   DG_LAUNCHED();
   SamplerArgs a{};
   a.partials = part;

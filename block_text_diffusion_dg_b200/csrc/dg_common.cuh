@@ -14,6 +14,7 @@ namespace dg {
 
 // Status codes written into the device error word (mirrors DG_ERR_TIMEOUT).
 constexpr int kDevErrTimeout = 4;
+constexpr int kDevErrBadId = 5;  // a token id outside [0, V) reached the embedding gather
 // A device wait gives up after this many nanoseconds of %globaltimer.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 

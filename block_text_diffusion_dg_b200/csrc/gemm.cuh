@@ -415,6 +415,7 @@ struct LmHeadParams {
   StatPartial* partials;  // [n_tokens, n_vtiles]
   float* logits;          // debug: [n_tokens, vocab] when not null (statistics skipped)
   int vocab;
+  float inv_t;            // 1 / sampling temperature: statistics of logits / T
   int* err;
   const int* done;
 };
@@ -567,7 +568,7 @@ __global__ void __launch_bounds__(kLmThreads, 1)
             tmem_ld32(t_row + c, v);
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-              const float d = v[i] - m;
+              const float d = (v[i] - m) * p.inv_t;
               const float e = __expf(d);
               s4[i & 3] += e;
               u4[i & 3] = fmaf(e, d, u4[i & 3]);
@@ -577,7 +578,7 @@ __global__ void __launch_bounds__(kLmThreads, 1)
           const float u = (u4[0] + u4[1]) + (u4[2] + u4[3]);
           if (tok < p.n_tokens)
             p.partials[static_cast<long long>(tok) * p.n_vtiles + vt] =
-                StatPartial{m, s, u, vt * 256 + a};
+                StatPartial{m * p.inv_t, s, u, vt * 256 + a};
         } else {
           for (int c = 0; c < 256; c += 32) {
             float v[32];

@@ -35,14 +35,21 @@ DG_DEV float block_sum_256(float v, float* sm) {
 template <typename TW, typename TA>
 __global__ void __launch_bounds__(256) embed_norm_kernel(const int32_t* __restrict__ ids,
                                                          const TW* __restrict__ embed, int d,
+                                                         int vocab,
                                                          const float* __restrict__ w, float eps,
                                                          float* __restrict__ x,
-                                                         TA* __restrict__ xn, const int* done) {
+                                                         TA* __restrict__ xn, const int* done,
+                                                         int* err) {
   pdl_enter();
   if (block_done(done)) return;
   __shared__ float sm[8];
   const int t = blockIdx.x;
-  const TW* e = embed + static_cast<long long>(ids[t]) * d;
+  int id = ids[t];
+  if (id < 0 || id >= vocab) {  // never read outside the table: record the error, use row 0
+    if (threadIdx.x == 0) atomicExch(err, kDevErrBadId);
+    id = 0;
+  }
+  const TW* e = embed + static_cast<long long>(id) * d;
   float ss = 0.f;
   for (int i = threadIdx.x; i < d; i += 256) {
     const float v = load_as_f32<TW>(e, i);
@@ -191,6 +198,10 @@ __global__ void __launch_bounds__(256) residual_norm_kernel(float* __restrict__ 
 DG_DEV void router_topk_select(float (&v)[8], int n_experts, int top_k, int32_t* ids_t,
                                float* wts_t) {
   const int lane = lane_id();
+  // a NaN logit ranks as -inf, so every selection below names a valid expert (top_k <= E)
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    if (v[j] != v[j]) v[j] = -INFINITY;
   float sel_v[8];
   int sel_i[8];
   for (int kk = 0; kk < top_k; ++kk) {

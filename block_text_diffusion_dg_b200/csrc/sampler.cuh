@@ -71,14 +71,34 @@ __global__ void canvas_init_kernel(int32_t* canvas, int32_t t, int32_t vocab, ui
   }
 }
 
+// Floor of x - m in the exponent sums.  Logits may hold -inf (masked vocabulary entries) as long
+// as every row has a finite value: such an entry has x - m = -inf, and e^(x - m) (x - m) would be
+// 0 * -inf = NaN, which would make the row's entropy, the mean entropy and hence the stop test NaN.
+// Clamping x - m at -1e30 makes its term exactly 0 (2^(-1e30 log2 e) = 0, 0 * -1e30 = 0).
+constexpr float kMaskedDelta = -1e30f;
+
+// Fresh decode state for a block: state words and completion ticket zeroed, lock flags of the
+// t canvas positions cleared; the canvas itself is kept (dg_reset_block).
+__global__ void block_reset_kernel(int32_t* state, int32_t* ticket, int32_t* locked, int32_t t) {
+  pdl_enter();
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < t) locked[i] = 0;
+  if (blockIdx.x == 0 && threadIdx.x < kStWords) {
+    state[threadIdx.x] = 0;
+    if (threadIdx.x == 0) *ticket = 0;
+  }
+}
+
 // Statistics (m, S, U, argmax) of one row slice held in registers by a 256-thread CTA: pass 1
 // takes the maximum (only threads holding it then look for its lowest column), pass 2
 // accumulates e = 2^((x - m) log2 e), S += e, U += e (x - m).  Value i of a thread sits at column
 // c0 + ((i / kVec) * 256 + tid) * kVec + i % kVec; values past the row end are -inf (`full` = no
 // such padding in this slice, uniform over the CTA).
+// With a temperature T (inv_t = 1 / T) the statistics are those of x / T: d = (x - m) / T and
+// the slice maximum is returned as m / T; the argmax does not depend on T.
 template <int kPerThread, int kVec>
 DG_DEV StatPartial slice_stats(const float (&v)[kPerThread], int c0, bool full, float* sm_f,
-                               int* sm_i) {
+                               int* sm_i, float inv_t = 1.0f) {
   const int warp = threadIdx.x >> 5;
   float tm = v[0];
 #pragma unroll
@@ -104,7 +124,8 @@ DG_DEV StatPartial slice_stats(const float (&v)[kPerThread], int c0, bool full, 
   if (full) {
 #pragma unroll
     for (int i = 0; i < kPerThread; ++i) {
-      const float d = v[i] - bm;
+      // a -inf logit (masked vocabulary entry) gives d = -1e30: e = 0 and e * d = 0, not NaN
+      const float d = fmaxf((v[i] - bm) * inv_t, kMaskedDelta);
       const float e = fast_exp2(d * kLog2e);
       s4[i & 3] += e;
       u4[i & 3] = fmaf(e, d, u4[i & 3]);
@@ -113,7 +134,7 @@ DG_DEV StatPartial slice_stats(const float (&v)[kPerThread], int c0, bool full, 
 #pragma unroll
     for (int i = 0; i < kPerThread; ++i) {
       if (v[i] != -INFINITY) {
-        const float d = v[i] - bm;
+        const float d = (v[i] - bm) * inv_t;
         const float e = fast_exp2(d * kLog2e);
         s4[i & 3] += e;
         u4[i & 3] = fmaf(e, d, u4[i & 3]);
@@ -134,7 +155,7 @@ DG_DEV StatPartial slice_stats(const float (&v)[kPerThread], int c0, bool full, 
     sm_i[warp] = a;
   }
   __syncthreads();
-  StatPartial r{bm, 0.f, 0.f, 0x7fffffff};
+  StatPartial r{bm * inv_t, 0.f, 0.f, 0x7fffffff};
   if (threadIdx.x == 0) {
     for (int w = 0; w < 8; ++w) {
       r.s += sm_f[w];
@@ -173,7 +194,8 @@ template <typename T, int kPerThread>
 __global__ void __launch_bounds__(256) logits_stats_kernel(const T* __restrict__ logits,
                                                            int32_t vocab, int32_t chunk,
                                                            StatPartial* __restrict__ out,
-                                                           const int* done) {
+                                                           const int* done,
+                                                           float inv_t = 1.0f) {
   pdl_enter();
   if (block_done(done)) return;
   __shared__ float sm_f[16];
@@ -183,7 +205,7 @@ __global__ void __launch_bounds__(256) logits_stats_kernel(const T* __restrict__
   float v[kPerThread];
   const bool full = load_slice<T, kPerThread>(logits + static_cast<size_t>(row) * vocab, c0,
                                               min(c0 + chunk, vocab), v);
-  const StatPartial r = slice_stats<kPerThread, 16 / sizeof(T)>(v, c0, full, sm_f, sm_i);
+  const StatPartial r = slice_stats<kPerThread, 16 / sizeof(T)>(v, c0, full, sm_f, sm_i, inv_t);
   if (threadIdx.x == 0) out[static_cast<size_t>(row) * gridDim.x + blockIdx.x] = r;
 }
 
@@ -475,7 +497,10 @@ DG_DEV StatPartial stream_slice_stats(const T* base, int c0, int c1) {
         to_f32x8<T>(raw[l], v);
 #pragma unroll
         for (int j = 0; j < kVec; j += 2) {
-          const float2 t = fmul2(fadd2(make_float2(v[j], v[j + 1]), nm2), l2);
+          float2 t = fmul2(fadd2(make_float2(v[j], v[j + 1]), nm2), l2);
+          // -inf logits: t = -inf (or NaN while m is still -inf) becomes -1e30, so e = 0 and
+          // e * t = 0 instead of NaN
+          t = make_float2(fmaxf(t.x, kMaskedDelta), fmaxf(t.y, kMaskedDelta));
           const float2 e = make_float2(fast_exp2(t.x), fast_exp2(t.y));
           s2 = fadd2(s2, e);
           t2 = ffma2(e, t, t2);

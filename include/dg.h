@@ -96,6 +96,12 @@ typedef struct dg_config {
   double entropy_lock;    /* nats, >= 0 (rule 1) */
   int32_t sticky_locks;   /* 1: a locked position keeps its token for the rest of the block
                              and the commit takes it (0: locks are re-decided every step) */
+  float temperature;      /* sampler statistics of softmax(logits / T); 0 or 1 = plain */
+  /* Commit encoding ([canvas] step 4, [arch] only say the block is committed to the KV cache):
+   * 0: re-encode the committed ids causally, exactly like the prompt;
+   * 1: keep the K/V the last denoise step wrote for the canvas (the bidirectional forward of
+   *    that step's input canvas), so the commit launches nothing but a copy of the ids. */
+  int32_t commit_reuse_kv;
 } dg_config;
 
 /* Per-layer weights, all device pointers, dtype = config dtype unless noted (bf16 for
@@ -170,6 +176,15 @@ DG_API int dg_kv_append(dg_ctx* ctx, const int32_t* d_ids, int32_t n, void* stre
  * Resets the decode state words (done, steps, stop step). */
 DG_API int dg_canvas_init(dg_ctx* ctx, uint64_t seed, uint32_t block, void* stream);
 
+/* Start the current block's denoising over ([canvas] step 4: after a commit the next canvas starts
+ * with a fresh decode; the same holds for a block the caller abandons before committing it): zero
+ * the decode state words (done, stop step, would-stop step, steps run, locked count, error) and the
+ * per-position lock flags, keep the canvas ids and the committed cache.  Later dg_denoise_step and
+ * dg_sample_update calls run again (step numbering restarts at 1) even if the block had stopped.
+ * dg_canvas_init performs this reset itself before it fills the canvas, so a caller that starts
+ * every block with dg_canvas_init never needs this call.  Asynchronous on `stream`. */
+DG_API int dg_reset_block(dg_ctx* ctx, void* stream);
+
 /* One denoise forward ([uniform], [canvas] step 3): embed the canvas, run every layer with
  * bidirectional attention over [committed cache | canvas] (canvas K/V are written to the
  * cache slots P..P+T-1 but P does not advance), final RMSNorm, and the LM head fused with
@@ -186,7 +201,8 @@ DG_API int dg_sample_update(dg_ctx* ctx, uint32_t step, void* stream);
 
 /* Commit ([canvas] step 4, [arch]): copy the stop step's argmax block to d_out_ids (int32
  * [T], may be NULL), the decode state words to d_state (int32 [DG_STATE_WORDS], may be
- * NULL), then causally re-encode the block into the cache (P += T). */
+ * NULL), then causally re-encode the block into the cache (P += T), or with commit_reuse_kv
+ * keep the canvas K/V of the last denoise step in place (P += T). */
 DG_API int dg_commit_block(dg_ctx* ctx, int32_t* d_out_ids, int32_t* d_state, void* stream);
 
 /* Device buffers of the context (for inspection; owned by the caller's scratch):
@@ -194,13 +210,18 @@ DG_API int dg_commit_block(dg_ctx* ctx, int32_t* d_out_ids, int32_t* d_state, vo
 DG_API int dg_get_buffers(const dg_ctx* ctx, int32_t** canvas, int32_t** argmax, float** entropy,
                    float** conf, int32_t** state);
 
-/* Blocking: synchronise `stream` and return DG_ERR_TIMEOUT if a device wait gave up. */
+/* Blocking: synchronise `stream` and return DG_ERR_TIMEOUT if a device wait gave up, or
+ * DG_ERR_INVALID_ARG if a token id outside [0, V) reached the embedding gather (from the caller's
+ * ids, or an argmax over a row of NaN logits): such an id is never used as an address, row 0 of
+ * the table is read in its place and the results of that call are invalid.  The error word stays
+ * set for the life of the context; once it is set, later device waits give up early. */
 DG_API int dg_check_device_status(dg_ctx* ctx, void* stream);
 
 /* ---- standalone operators (the same kernels the context runs) -------------------- */
 
 /* Sampler over given logits ([canvas] step 3): d_logits [rows, V] (dtype), one call per
- * step.  d_state int32[DG_STATE_WORDS] and the workspace carry the stop test across
+ * step.  Logits are finite or -inf (a masked vocabulary entry: probability 0, no contribution to
+ * the entropy); every row needs at least one finite value.  d_state int32[DG_STATE_WORDS] and the workspace carry the stop test across
  * calls; zero both (dg_sampler_reset) before step 1.  Outputs: d_canvas (next ids),
  * d_argmax, d_entropy, d_conf, each [rows].  Requires V % 8 == 0, rows <= 1024. */
 DG_API int dg_sampler_workspace_bytes(int32_t rows, int32_t vocab, size_t* bytes);
@@ -221,7 +242,9 @@ DG_API int dg_sampler_step(const void* d_logits, int32_t dtype, int32_t rows, in
  * V % 8 == 0; larger requests return DG_ERR_CAPACITY.  Arguments and outputs are those of
  * dg_sampler_step; the caller zeroes d_state before step 1.  The first call on each device looks
  * up the array's device address (cudaGetSymbolAddress) with that device current, so make that
- * first call before any stream capture.  Every call on a device shares the one array, which keeps
+ * first call before any stream capture.  The address is kept per CUDA context: the first call
+ * after the device's context was replaced (cudaDeviceReset) looks it up again, under the same
+ * rule.  Every call on a device shares the one array, which keeps
  * the previous call's contents: calls that overlap on the GPU (other streams, other threads) race,
  * so serialise them.  Allocates no memory (no cudaMalloc, cudaFree or allocating library call). */
 DG_API int dg_sampler_step_static(const void* d_logits, int32_t dtype, int32_t rows,

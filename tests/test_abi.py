@@ -72,6 +72,15 @@ def test_create_rejects_null_buffers(L):
     assert lib.dg_create(C.byref(cfg), C.byref(w), None, None, None, C.byref(out)) == -1
 
 
+def test_loop_entry_points_reject_a_null_context(L):
+    lib = L.lib()
+    assert lib.dg_reset_block(None, None) == -1
+    assert lib.dg_canvas_init(None, 0, 0, None) == -1
+    assert lib.dg_denoise_step(None, 1, None) == -1
+    assert lib.dg_sample_update(None, 1, None) == -1
+    assert lib.dg_commit_block(None, None, None, None) == -1
+
+
 def test_standalone_shape_checks(L):
     lib = L.lib()
     n = C.c_size_t()

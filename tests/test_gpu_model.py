@@ -12,7 +12,8 @@ from dg_synth import SHAPES, model_weights, uniform_ids
 from oracle import model as om
 from oracle import sampler as osmp
 from oracle.numerics import round_bf16
-from tests._helpers import check_layer_parts, np64, rel_close, weights_to_np
+from tests._helpers import (check_layer_parts, kv_tokens_close, np64, rel_close, router_gaps,
+                            weights_to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -101,16 +102,6 @@ def _cache_prefix(cache, n):
     return c
 
 
-def _tokenwise_close(got, ref, rtol, min_frac):
-    """Per-token rel_close over [H, n, hd] K slices: the fraction of tokens that pass.  A token whose
-    MoE routing flipped at an earlier layer's near-tie legitimately differs."""
-    got = np.asarray(got)
-    ref = np.asarray(ref)
-    n = ref.shape[1]
-    good = [rel_close(got[:, j], ref[:, j], rtol)[0] for j in range(n)]
-    return float(np.mean(good)) >= min_frac, float(np.mean(good))
-
-
 def test_small_bf16_prefill_denoise_commit():
     from block_text_diffusion_dg_b200 import DiffusionModel, make_config
     shape = SHAPES["small_bf16"]
@@ -121,16 +112,17 @@ def test_small_bf16_prefill_denoise_commit():
     m = DiffusionModel(cfg, _to_cuda(w))
     ocfg, ow = _ocfg("small_bf16"), weights_to_np(w)
     ocache = om.causal_encode(ocfg, ow, prompt.numpy(), om.KVCache())
+    gaps = router_gaps(ocfg, ow, prompt.numpy(), np.arange(320), om.KVCache())
     m.kv_append(prompt.cuda())
     assert m.kv_length == 320
     k_gpu, vt_gpu = _kv_views(m, cfg)
     torch.cuda.synchronize()
     for l in range(cfg.n_layers):
-        ok, frac = _tokenwise_close(np64(k_gpu[l, :, :320]), ocache.k[l], 2e-2, 0.98 if l else 1.0)
-        assert ok, ("prefill K", l, frac)
-        ok, frac = _tokenwise_close(np64(vt_gpu[l, :, :, :320]).transpose(0, 2, 1), ocache.v[l], 2e-2,
-                                    0.98 if l else 1.0)
-        assert ok, ("prefill V", l, frac)
+        ok, bad, _ = kv_tokens_close(np64(k_gpu[l, :, :320]), ocache.k[l], gaps, l, 2e-2)
+        assert ok, ("prefill K", l, bad)
+        ok, bad, _ = kv_tokens_close(np64(vt_gpu[l, :, :, :320]).transpose(0, 2, 1), ocache.v[l],
+                                      gaps, l, 2e-2)
+        assert ok, ("prefill V", l, bad)
     # one denoise step
     m.canvas_init(11, 0)
     m.denoise_step(1)
@@ -170,12 +162,16 @@ def test_small_bf16_prefill_denoise_commit():
     ids_np = ids.cpu().numpy()
     assert st.cpu().tolist()[:2] == [1, 3]
     assert m.kv_length == 320 + 256
+    gaps = router_gaps(ocfg, ow, ids_np, 320 + np.arange(256), ocache)
     om.causal_encode(ocfg, ow, ids_np, ocache)
     k_gpu, vt_gpu = _kv_views(m, cfg)
     for l in range(cfg.n_layers):
-        ok, frac = _tokenwise_close(np64(k_gpu[l, :, 320:576]), ocache.k[l][:, 320:576], 2e-2,
-                                    0.98 if l else 1.0)
-        assert ok, ("commit K", l, frac)
+        ok, bad, _ = kv_tokens_close(np64(k_gpu[l, :, 320:576]), ocache.k[l][:, 320:576], gaps, l,
+                                      2e-2)
+        assert ok, ("commit K", l, bad)
+        ok, bad, _ = kv_tokens_close(np64(vt_gpu[l, :, :, 320:576]).transpose(0, 2, 1),
+                                      ocache.v[l][:, 320:576], gaps, l, 2e-2)
+        assert ok, ("commit V", l, bad)
     # second block runs against the longer history
     m.canvas_init(11, 1)
     for t in (1, 2, 3):
@@ -199,16 +195,17 @@ def test_small_bf16_prefill_in_large_chunks():
     m = DiffusionModel(cfg, _to_cuda(w))
     ocfg, ow = _ocfg("small_bf16"), weights_to_np(w)
     ocache = om.causal_encode(ocfg, ow, prompt.numpy(), om.KVCache())
+    gaps = router_gaps(ocfg, ow, prompt.numpy(), np.arange(640), om.KVCache())
     m.kv_append(prompt.cuda())
     assert m.kv_length == 640
     k_gpu, vt_gpu = _kv_views(m, cfg)
     torch.cuda.synchronize()
     for l in range(cfg.n_layers):
-        ok, frac = _tokenwise_close(np64(k_gpu[l, :, :640]), ocache.k[l], 2e-2, 0.98 if l else 1.0)
-        assert ok, ("prefill K", l, frac)
-        ok, frac = _tokenwise_close(np64(vt_gpu[l, :, :, :640]).transpose(0, 2, 1), ocache.v[l], 2e-2,
-                                    0.98 if l else 1.0)
-        assert ok, ("prefill V", l, frac)
+        ok, bad, _ = kv_tokens_close(np64(k_gpu[l, :, :640]), ocache.k[l], gaps, l, 2e-2)
+        assert ok, ("prefill K", l, bad)
+        ok, bad, _ = kv_tokens_close(np64(vt_gpu[l, :, :, :640]).transpose(0, 2, 1), ocache.v[l],
+                                      gaps, l, 2e-2)
+        assert ok, ("prefill V", l, bad)
     m.canvas_init(5, 0)
     m.denoise_step(1)
     m.sample_update(1)
