@@ -36,7 +36,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-PROMPT, BLOCKS, FIXED_STEPS, CANVAS = 4096, 4, 16, 256
+PROMPT, BLOCKS, FIXED_STEPS, CANVAS, MAX_STEPS = 4096, 4, 16, 256, 48
 PREFILL_CHUNK = 4096  # prompt tokens per causal-encode pass (the whole prompt)
 WORKLOAD = ("full block decode: 30-layer MoE decoder (d 2816, 16/8 heads x 128, 128 experts "
             "top-8 x 704 + shared 2112, vocab 262144, bf16, random init), 4096-token prompt "
@@ -279,11 +279,30 @@ def run_ops(dev, stream, hbm, tf_burst):
     return out
 
 
-def decode(model, seed, out_ids, out_states, stream):
+def step_bytes(shape, prefix, f8=False):
+    """Algorithmic HBM bytes of one denoise step at committed length `prefix`: every weight the
+    step reads once (QKV, O, router, all routed experts' gate/up and down, the shared expert; all
+    128 experts are routed at these shapes) per layer, the K/V cache read over prefix + canvas
+    keys and the canvas K/V written per layer, and the LM head's embedding table.  Activations
+    (a few MB per layer) are left out.  e4m3 experts: one byte per weight plus one fp32 scale per
+    weight row."""
+    d, hq, hkv, hd = shape["d_model"], shape["n_heads"], shape["n_kv_heads"], shape["head_dim"]
+    e, h, hs, v = shape["n_experts"], shape["expert_hidden"], shape["shared_hidden"], shape["vocab"]
+    dense = ((hq + 2 * hkv) * hd * d + d * hq * hd + e * d) * 2
+    if f8:
+        experts = (e * 2 * h + 2 * hs) * d + (e * h + hs) * d + (e * 2 * h + e * d + 2 * hs + d) * 4
+    else:
+        experts = (e * 3 * h * d + 3 * hs * d) * 2
+    kv = (prefix + CANVAS) * hkv * hd * 2 * 2 + CANVAS * hkv * hd * 2 * 2
+    return shape["n_layers"] * (dense + experts + kv) + v * d * 2
+
+
+def decode(model, seed, out_ids, out_states, stream, fixed=True):
     model.kv_truncate(PROMPT)
     for b in range(BLOCKS):
         model.canvas_init(seed, b, stream)
-        for t in range(1, FIXED_STEPS + 1):
+        # adaptive mode enqueues the 48-step cap; steps after the device-side stop are no-ops
+        for t in range(1, (FIXED_STEPS if fixed else MAX_STEPS) + 1):
             model.denoise_step(t, stream)
             model.sample_update(t, stream)
         model.commit_block(out_ids[b * CANVAS:(b + 1) * CANVAS], out_states[b], stream)
@@ -428,6 +447,36 @@ def run_ours(args, rank, world, local_rank):
     for v in table.values():
         v["share"] = round(v["us_per_step"] / step_us, 4)
 
+    # the whole denoise step against the HBM roofline (block 0: 4,096 committed positions)
+    sb = step_bytes(shape, PROMPT, f8)
+    step_gbs = sb / (us_step / 1e6) / 1e9
+    step_roof = dict(bound="hbm", achieved=round(step_gbs, 1), peak=hbm, unit="GB/s",
+                     frac=round(step_gbs / hbm, 4), algorithmic_bytes_per_step=sb,
+                     us_per_step=round(us_step, 1), floor_us=round(sb / hbm / 1e3, 1),
+                     peak_source=f"{src} (MEASURED_PEAKS.json hbm_gbs)")
+
+    # adaptive stop, 48-step cap ([canvas] step 3): random-init weights never reach the stop
+    # rule, so every block runs to the cap
+    cfg_a = make_config(shape, kv_capacity=cap, fixed_steps=0, max_steps=MAX_STEPS,
+                        prefill_chunk=PREFILL_CHUNK, experts=args.experts)
+    model_a = DiffusionModel(cfg_a, weights, device=dev)
+    model_a.kv_append(prompt_dev, stream)
+    decode(model_a, 300, out_ids, out_states, stream, fixed=False)  # warm-up
+    torch.cuda.synchronize()
+    barrier()
+    e0.record(stream)
+    decode(model_a, 301, out_ids, out_states, stream, fixed=False)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_a = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    st_a = out_states.cpu()
+    model_a.check_device_status(stream)
+    model_a.close()
+    adaptive = dict(value=round(replica_throughput(BLOCKS * CANVAS, world, ms_a), 2), unit="tok/s",
+                    max_steps=MAX_STEPS, ms_per_decode=round(ms_a, 2),
+                    steps_per_block=[int(x) for x in st_a[:, 1].tolist()],
+                    would_stop=[int(x) for x in st_a[:, 2].tolist()])
+
     ops = run_ops(dev, stream, hbm, tf_burst)
 
     # end to end through the public API, pinned host buffers in and out
@@ -465,7 +514,8 @@ def run_ours(args, rank, world, local_rank):
                                l2="inputs larger than L2: ~%d GB of weights streamed per denoise "
                                   "step" % (25 if f8 else 49)),
                    us_per_denoise_step=round(us_step, 1), prefill_ms=round(prefill_ms, 2),
-                   roofline=roof, cpu_baseline=cpu,
+                   roofline=roof, step_roofline=step_roof, adaptive_stop=adaptive,
+                   cpu_baseline=cpu,
                    e2e=dict(value=round(e2e_val, 2), unit="tok/s",
                             h2d_bytes_per_step=prompt.numel() * 4,
                             d2h_bytes_per_step=host_ids.numel() * 4 + host_states.numel() * 4,
