@@ -37,6 +37,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 PROMPT, BLOCKS, FIXED_STEPS, CANVAS, MAX_STEPS = 4096, 4, 16, 256, 48
+LONG_PROMPT = 32768  # the long-context measurement
 PREFILL_CHUNK = 4096  # prompt tokens per causal-encode pass (the whole prompt)
 WORKLOAD = ("full block decode: 30-layer MoE decoder (d 2816, 16/8 heads x 128, 128 experts "
             "top-8 x 704 + shared 2112, vocab 262144, bf16, random init), 4096-token prompt "
@@ -412,11 +413,10 @@ def run_ours(args, rank, world, local_rank):
                        + (slots + CANVAS) * d * 4 + (e * d + d + slots + CANVAS) * scale_b,
         "lm_head": shape["vocab"] * d * 2 + CANVAS * d * 2 + CANVAS * (shape["vocab"] // 256) * 16,
     }
-    # DRAM bytes (read + write) of one launch from the ncu capture summarised in profiles/
-    # (dram__bytes_read.sum + dram__bytes_write.sum); None where no capture of the current kernel
-    # (the bf16 grouped GEMMs changed after their last capture, 1,056,290,808 B for gate/up)
+    # DRAM bytes (read + write) of one launch from the ncu captures summarised in profiles/
+    # (dram__bytes_read.sum + dram__bytes_write.sum of the standalone MoE operator's launches)
     traffic = ({"expert_gate_up": 532844544 + 5702400, "expert_down": 286637312 + 9329920} if f8
-               else {})
+               else {"expert_gate_up": 1063746000 + 4687104, "expert_down": 523752000 + 6922496})
     roof = None
     if args.roofline_kernel in algo and rec:
         achieved = algo[args.roofline_kernel] / (avg_ms / 1e3) / 1e9
@@ -477,6 +477,34 @@ def run_ours(args, rank, world, local_rank):
                     steps_per_block=[int(x) for x in st_a[:, 1].tolist()],
                     would_stop=[int(x) for x in st_a[:, 2].tolist()])
 
+    # long context ([canvas] step 1 prefill; the pages' weak spot is the time to the first
+    # output): a 32,768-token prompt in 4,096-token passes, then the first block of 16 steps
+    cfg_l = make_config(shape, kv_capacity=LONG_PROMPT + 2 * CANVAS, fixed_steps=FIXED_STEPS,
+                        prefill_chunk=PREFILL_CHUNK, experts=args.experts)
+    model_l = DiffusionModel(cfg_l, weights, device=dev)
+    long_prompt = uniform_ids(LONG_PROMPT, shape["vocab"], seed=77 + rank).to(dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    torch.cuda.synchronize()
+    barrier()
+    ev[0].record(stream)
+    model_l.kv_append(long_prompt, stream)
+    ev[1].record(stream)
+    model_l.canvas_init(5, 0, stream)
+    for tt in range(1, FIXED_STEPS + 1):
+        model_l.denoise_step(tt, stream)
+        model_l.sample_update(tt, stream)
+    ev[2].record(stream)
+    model_l.commit_block(out_ids[:CANVAS], out_states[0], stream)
+    ev[3].record(stream)
+    torch.cuda.synchronize()
+    model_l.check_device_status(stream)
+    model_l.close()
+    del long_prompt
+    long_ctx = dict(prompt=LONG_PROMPT, prefill_ms=round(max_over_ranks(ev[0].elapsed_time(ev[1]), world, dev), 2),
+                    us_per_denoise_step=round(1e3 * ev[1].elapsed_time(ev[2]) / FIXED_STEPS, 1),
+                    first_block_ms=round(max_over_ranks(ev[0].elapsed_time(ev[3]), world, dev), 2),
+                    note="first_block_ms: prompt prefill + 16 denoise steps + commit of block 0")
+
     ops = run_ops(dev, stream, hbm, tf_burst)
 
     # end to end through the public API, pinned host buffers in and out
@@ -515,6 +543,7 @@ def run_ours(args, rank, world, local_rank):
                                   "step" % (25 if f8 else 49)),
                    us_per_denoise_step=round(us_step, 1), prefill_ms=round(prefill_ms, 2),
                    roofline=roof, step_roofline=step_roof, adaptive_stop=adaptive,
+                   long_context=long_ctx,
                    cpu_baseline=cpu,
                    e2e=dict(value=round(e2e_val, 2), unit="tok/s",
                             h2d_bytes_per_step=prompt.numel() * 4,
