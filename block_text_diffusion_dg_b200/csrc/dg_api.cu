@@ -521,6 +521,11 @@ int check_config(const dg_config* c) {
   if (c->canvas > 256) return fail(DG_ERR_UNSUPPORTED, "canvas must be <= 256");
   if (c->kv_capacity % 8 != 0 || c->kv_capacity < c->canvas)
     return fail(DG_ERR_INVALID_ARG, "kv_capacity must be a multiple of 8 and >= canvas");
+  // TMA row coordinates of the K cache ([L * Hkv * cap] rows) and the per-layer V^T offsets are
+  // 32-bit
+  if (static_cast<long long>(c->n_layers) * c->n_kv_heads * c->kv_capacity >= (1ll << 31) ||
+      static_cast<long long>(c->n_kv_heads) * c->head_dim * c->kv_capacity >= (1ll << 31))
+    return fail(DG_ERR_UNSUPPORTED, "kv_capacity too large for 32-bit cache coordinates");
   if (c->head_dim % 4 != 0) return fail(DG_ERR_INVALID_ARG, "head_dim must be a multiple of 4");
   if (c->d_model % 4 != 0 || c->d_model > 4096)
     return fail(DG_ERR_UNSUPPORTED, "d_model must be a multiple of 4 and at most 4096");

@@ -79,7 +79,8 @@ typedef struct dg_config {
   int32_t shared_hidden;  /* hs (0 = no shared expert); bf16: multiple of 64 */
   int32_t vocab;          /* V; bf16: multiple of 256 */
   int32_t canvas;         /* canvas length T; 256 in the pages ([canvas]); 1..256 */
-  int32_t kv_capacity;    /* positions the caller's KV cache holds (multiple of 8) */
+  int32_t kv_capacity;    /* positions the caller's KV cache holds (multiple of 8); L * Hkv * cap
+                             and Hkv * hd * cap below 2^31 (long contexts: 256K positions fit) */
   int32_t dtype;          /* DG_DTYPE_BF16, DG_DTYPE_FP32 or DG_DTYPE_BF16_E4M3 */
   float eps;              /* RMSNorm epsilon (1e-6) */
   float rope_theta;       /* RoPE base (10000) */

@@ -1,0 +1,143 @@
+"""Long contexts: causal prefill and canvas attention far beyond the 4,096-token prompt.
+
+The pages give the model a long context window (k7ail.com, use cases: a 256K window) and note that
+time-to-first-token is where the diffusion decoder is weakest (alphalab.site, "official
+benchmark"): the prompt goes through a causal prefill before the first canvas ([canvas] step 1).
+At these lengths the oracle cannot run the whole causal encode, so the checks sample outputs it
+can compute one by one:
+
+  * the attention operator on N(0, 1) inputs with 32K (causal, prefill-like) and 128K (no mask,
+    denoise at long context) committed keys: sampled (query, head) rows against the oracle's
+    attention over exactly the keys that row sees;
+  * a two-layer model after a 20,000-token prompt encoded in 4,096-token passes (the last one
+    ragged): every position's layer-0 K/V (functions of its own token only) against the oracle,
+    and sampled positions' layer-1 K/V, each recomputed by the oracle from that token's causal
+    layer-0 attention over the GPU-independent layer-0 cache and its MoE; then a denoise step over
+    the 20,256 keys, whose LM-head statistics are checked on the GPU's own logits and whose
+    first-layer attention half is compared teacher-forced.
+"""
+import numpy as np
+import pytest
+import torch
+
+from dg_synth import SHAPES, attention_inputs, model_weights, uniform_ids
+from oracle import model as om
+from oracle import sampler as osmp
+from oracle.attention import attention as o_attention
+from oracle.numerics import round_bf16, round_storage
+from tests._helpers import NEAR_TIE, check_layer_parts, np64, rel_close, weights_to_np
+
+pytestmark = pytest.mark.gpu
+RTOL = 2e-2
+
+
+@pytest.mark.parametrize("prefix,causal", [(32768, True), (131072, False)])
+def test_attention_long_context_sampled_rows(prefix, causal):
+    from block_text_diffusion_dg_b200 import canvas_attention
+    hq, hkv, t = 16, 8, 256
+    q, k, v = attention_inputs(hq, hkv, canvas=t, prefix=prefix, head_dim=128, seed=prefix % 97)
+    n_keys = prefix + t
+    vt = v.transpose(1, 2).contiguous()
+    o = canvas_attention(q.cuda(), k.cuda(), vt.cuda(), n_keys,
+                         causal_prefix=prefix if causal else -1, n_queries=t)
+    got = np64(o)
+    del vt
+    toks = np.array([0, 1, 63, 127, 128, 200, 254, 255])
+    q64 = np64(q)
+    for g in range(hkv):
+        kg, vg = np64(k[g:g + 1]), np64(v[g:g + 1])
+        heads = range(g * (hq // hkv), (g + 1) * (hq // hkv))
+        for tok in toks:
+            seen = prefix + tok + 1 if causal else n_keys  # keys this query row sees
+            ref = o_attention(q64[list(heads), tok:tok + 1], kg[:, :seen], vg[:, :seen],
+                              128 ** -0.5)
+            for j, h in enumerate(heads):
+                r = round_bf16(ref[j, 0])
+                ok, worst, nrel = rel_close(got[tok, h * 128:(h + 1) * 128], r, RTOL)
+                assert ok and nrel < 5e-3, (tok, h, worst, nrel)
+
+
+def _ocfg(shape):
+    return om.ModelConfig(**{k: shape[k] for k in (
+        "n_layers", "d_model", "n_heads", "n_kv_heads", "head_dim", "n_experts", "top_k",
+        "expert_hidden", "shared_hidden", "vocab", "canvas", "storage")})
+
+
+def _layer0_kv(ocfg, lw, ids, positions, embed):
+    """Layer-0 K/V of every position: each depends on its own token only (oracle pieces)."""
+    hq, hkv, hd = ocfg.n_heads, ocfg.n_kv_heads, ocfg.head_dim
+    x = np.asarray(embed, dtype=np.float64)[ids]
+    xn = round_storage(om.rmsnorm(x, lw["attn_norm"], ocfg.eps), ocfg.storage)
+    w = np.asarray(lw["wqkv"], dtype=np.float64)
+    k = (xn @ w[hq * hd:(hq + hkv) * hd].T).reshape(len(ids), hkv, hd).transpose(1, 0, 2)
+    v = (xn @ w[(hq + hkv) * hd:].T).reshape(len(ids), hkv, hd).transpose(1, 0, 2)
+    return (round_storage(om.rope(k, positions, ocfg.rope_theta), ocfg.storage),
+            round_storage(v, ocfg.storage))
+
+
+def test_model_long_prompt_prefill_and_denoise():
+    from block_text_diffusion_dg_b200 import DiffusionModel, make_config
+    shape = SHAPES["small_bf16"]
+    n_prompt = 20000
+    cap = ((n_prompt + 2 * 256 + 7) // 8) * 8
+    wt = model_weights("small_bf16", seed=51, norm_jitter=0.1)
+    cfg = make_config(shape, kv_capacity=cap, fixed_steps=1, prefill_chunk=4096)
+    wc = dict(embed=wt["embed"].cuda(), final_norm=wt["final_norm"].cuda(),
+              layers=[{k: (None if v is None else v.cuda()) for k, v in lw.items()}
+                      for lw in wt["layers"]])
+    m = DiffusionModel(cfg, wc)
+    prompt = uniform_ids(n_prompt, shape["vocab"], seed=52)
+    m.kv_append(prompt.cuda())
+    assert m.kv_length == n_prompt
+    kv = m.kv.view(torch.bfloat16)
+    half = kv.numel() // 2
+    k_gpu = kv[:half].view(cfg.n_layers, cfg.n_kv_heads, cap, cfg.head_dim)
+    vt_gpu = kv[half:].view(cfg.n_layers, cfg.n_kv_heads, cfg.head_dim, cap)
+    torch.cuda.synchronize()
+    ocfg, ow = _ocfg(shape), weights_to_np(wt)
+    ids = prompt.numpy()
+    pos = np.arange(n_prompt)
+    k0, v0 = _layer0_kv(ocfg, ow["layers"][0], ids, pos, ow["embed"])
+    ok, worst, _ = rel_close(np64(k_gpu[0, :, :n_prompt]), k0, RTOL)
+    assert ok, ("layer-0 K", worst)
+    ok, worst, _ = rel_close(np64(vt_gpu[0, :, :, :n_prompt]).transpose(0, 2, 1), v0, RTOL)
+    assert ok, ("layer-0 V", worst)
+    # sampled positions' layer-1 K/V: chunk seams, the ragged last pass, far positions
+    sample = [0, 1, 4095, 4096, 4097, 8191, 8192, 12288, 16383, 16384, 17000, 19998, 19999]
+    x_emb = np.asarray(ow["embed"], dtype=np.float64)[ids]
+    lw0, lw1 = ow["layers"][0], ow["layers"][1]
+    excused = 0
+    for i in sample:
+        x1, _, _, _ = om.attention_block(ocfg, lw0, x_emb[i:i + 1], pos[i:i + 1], k0[:, :i], v0[:, :i],
+                                         causal=False)  # one token: sees keys 0..i
+        x2, info = om.moe_block(ocfg, lw0, x1)
+        srt = -np.sort(-info["moe"]["router_logits"][0])
+        gap = srt[ocfg.top_k - 1] - srt[ocfg.top_k]
+        empty = np.zeros((ocfg.n_kv_heads, 0, ocfg.head_dim))
+        _, k1, v1, _ = om.attention_block(ocfg, lw1, x2, pos[i:i + 1], empty, empty, causal=False)
+        ok_k = rel_close(np64(k_gpu[1, :, i]), k1[:, 0], RTOL)[0]
+        ok_v = rel_close(np64(vt_gpu[1, :, :, i]), v1[:, 0], RTOL)[0]
+        if not (ok_k and ok_v):
+            assert gap < NEAR_TIE, ("layer-1 K/V at position", i, gap)
+            excused += 1
+    assert excused <= 2
+    # one denoise step over the 20,000 + 256 keys
+    m.canvas_init(53, 0)
+    m.denoise_step(1)
+    logits = np64(m.debug_logits())
+    m.sample_update(1)
+    bufs = m.buffers()
+    torch.cuda.synchronize()
+    conf, ent, amax = osmp.row_stats(logits)
+    assert np.array_equal(bufs["argmax"].cpu().numpy(), amax)
+    assert np.max(np.abs(bufs["entropy"].cpu().numpy() - ent)) < 1e-5
+    # the first layer's attention half, teacher-forced on the canvas, against the oracle's
+    # layer-0 cache (the GPU's own cache matches it to bf16 rounding, checked above)
+    canvas0 = osmp.canvas_init(53, 0, 256, shape["vocab"])
+    x = np.asarray(ow["embed"], dtype=np.float64)[canvas0]
+    att, moe, frac = check_layer_parts(m, ocfg, lw0, x, n_prompt + np.arange(256), k0, v0, 0,
+                                       shape["top_k"])
+    assert att[0] and att[2] < 5e-3, ("attention half", att)
+    assert moe[0] and moe[2] < 5e-3, ("moe half", moe)
+    m.check_device_status()
+    m.close()
