@@ -38,6 +38,7 @@ sys.path.insert(0, ROOT)
 
 PROMPT, BLOCKS, FIXED_STEPS, CANVAS, MAX_STEPS = 4096, 4, 16, 256, 48
 LONG_PROMPT = 32768  # the long-context measurement
+BATCH = 4  # sequences of the small-batch measurement
 PREFILL_CHUNK = 4096  # prompt tokens per causal-encode pass (the whole prompt)
 WORKLOAD = ("full block decode: 30-layer MoE decoder (d 2816, 16/8 heads x 128, 128 experts "
             "top-8 x 704 + shared 2112, vocab 262144, bf16, random init), 4096-token prompt "
@@ -298,6 +299,31 @@ def step_bytes(shape, prefix, f8=False):
     return shape["n_layers"] * (dense + experts + kv) + v * d * 2
 
 
+def live_kernel_table(model, stream, L):
+    """Live per-kernel table: for each kernel kind, one denoise step with CUDA events around that
+    kind's launches (on their stream); microseconds per launch and per step, and share."""
+    import ctypes as C
+    table = {}
+    for kname, kk in L.KERNEL_KINDS.items():
+        L.check(L.lib().dg_profile_kernel(kk, 64), "dg_profile_kernel")
+        model.kv_truncate(PROMPT)
+        model.canvas_init(9, 0, stream)
+        model.denoise_step(1, stream)
+        model.sample_update(1, stream)
+        torch.cuda.synchronize()
+        buf2 = (C.c_float * 64)()
+        nrec = L.lib().dg_profile_read(buf2, 64)
+        L.check(L.lib().dg_profile_kernel(0, 0), "dg_profile_kernel")
+        if nrec > 0:
+            tot = sum(buf2[:nrec]) * 1e3
+            table[kname] = dict(launches=nrec, us_per_launch=round(tot / nrec, 2),
+                                us_per_step=round(tot, 1))
+    step_us = sum(v["us_per_step"] for v in table.values())
+    for v in table.values():
+        v["share"] = round(v["us_per_step"] / step_us, 4)
+    return table
+
+
 def decode(model, seed, out_ids, out_states, stream, fixed=True):
     model.kv_truncate(PROMPT)
     for b in range(BLOCKS):
@@ -427,25 +453,7 @@ def run_ours(args, rank, world, local_rank):
                     algorithmic_bytes_per_launch=algo[args.roofline_kernel],
                     peak_source=f"{src} (MEASURED_PEAKS.json hbm_gbs)")
 
-    # live per-kernel table: one profiled denoise step per kernel kind
-    table = {}
-    for kname, kk in L.KERNEL_KINDS.items():
-        L.check(L.lib().dg_profile_kernel(kk, 64), "dg_profile_kernel")
-        model.kv_truncate(PROMPT)
-        model.canvas_init(9, 0, stream)
-        model.denoise_step(1, stream)
-        model.sample_update(1, stream)
-        torch.cuda.synchronize()
-        buf2 = (C.c_float * 64)()
-        nrec = L.lib().dg_profile_read(buf2, 64)
-        L.check(L.lib().dg_profile_kernel(0, 0), "dg_profile_kernel")
-        if nrec > 0:
-            tot = sum(buf2[:nrec]) * 1e3
-            table[kname] = dict(launches=nrec, us_per_launch=round(tot / nrec, 2),
-                                us_per_step=round(tot, 1))
-    step_us = sum(v["us_per_step"] for v in table.values())
-    for v in table.values():
-        v["share"] = round(v["us_per_step"] / step_us, 4)
+    table = live_kernel_table(model, stream, L)
 
     # the whole denoise step against the HBM roofline (block 0: 4,096 committed positions)
     sb = step_bytes(shape, PROMPT, f8)
@@ -505,6 +513,52 @@ def run_ours(args, rank, world, local_rank):
                     first_block_ms=round(max_over_ranks(ev[0].elapsed_time(ev[3]), world, dev), 2),
                     note="first_block_ms: prompt prefill + 16 denoise steps + commit of block 0")
 
+    # small-batch canvases: BATCH sequences (own prompts and caches) decoded in lockstep, every
+    # denoise step carrying BATCH x 256 canvas tokens through one weight stream
+    cfg_b = make_config(shape, kv_capacity=cap, fixed_steps=FIXED_STEPS,
+                        prefill_chunk=PREFILL_CHUNK, experts=args.experts, batch=BATCH)
+    model_b = DiffusionModel(cfg_b, weights, device=dev)
+    prompts_b = torch.stack([uniform_ids(PROMPT, shape["vocab"], seed=90 + BATCH * rank + b)
+                             for b in range(BATCH)]).to(dev)
+    model_b.kv_append(prompts_b, stream)
+    ids_b = torch.empty(BATCH * CANVAS, dtype=torch.int32, device=dev)
+    st_b = torch.empty(BATCH, L.STATE_WORDS, dtype=torch.int32, device=dev)
+
+    def decode_b(seed):
+        model_b.kv_truncate(PROMPT)
+        for blk in range(BLOCKS):
+            model_b.canvas_init(seed, blk, stream)
+            for tt in range(1, FIXED_STEPS + 1):
+                model_b.denoise_step(tt, stream)
+                model_b.sample_update(tt, stream)
+            model_b.commit_block(ids_b, st_b, stream)
+
+    decode_b(400)  # warm-up
+    torch.cuda.synchronize()
+    barrier()
+    e0.record(stream)
+    decode_b(401)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_b = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    model_b.kv_truncate(PROMPT)
+    model_b.canvas_init(402, 0, stream)
+    e0.record(stream)
+    for tt in range(1, FIXED_STEPS + 1):
+        model_b.denoise_step(tt, stream)
+        model_b.sample_update(tt, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    us_step_b = 1e3 * e0.elapsed_time(e1) / FIXED_STEPS
+    table_b = live_kernel_table(model_b, stream, L)
+    model_b.check_device_status(stream)
+    model_b.close()
+    del prompts_b
+    batched = dict(batch=BATCH, value=round(replica_throughput(BATCH * BLOCKS * CANVAS, world, ms_b), 2),
+                   unit="tok/s", ms_per_decode=round(ms_b, 2), us_per_denoise_step=round(us_step_b, 1),
+                   note=f"{BATCH} sequences x 4 blocks x 256 tokens, 16 fixed steps, lockstep",
+                   kernels_live=table_b)
+
     ops = run_ops(dev, stream, hbm, tf_burst)
 
     # end to end through the public API, pinned host buffers in and out
@@ -543,7 +597,7 @@ def run_ours(args, rank, world, local_rank):
                                   "step" % (25 if f8 else 49)),
                    us_per_denoise_step=round(us_step, 1), prefill_ms=round(prefill_ms, 2),
                    roofline=roof, step_roofline=step_roof, adaptive_stop=adaptive,
-                   long_context=long_ctx,
+                   long_context=long_ctx, small_batch=batched,
                    cpu_baseline=cpu,
                    e2e=dict(value=round(e2e_val, 2), unit="tok/s",
                             h2d_bytes_per_step=prompt.numel() * 4,

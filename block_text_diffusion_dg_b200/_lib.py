@@ -27,7 +27,7 @@ class Config(C.Structure):
         ("tau", C.c_double), ("h_bound", C.c_double), ("max_steps", C.c_int32),
         ("fixed_steps", C.c_int32), ("prefill_chunk", C.c_int32),
         ("lock_rule", C.c_int32), ("entropy_lock", C.c_double), ("sticky_locks", C.c_int32),
-        ("temperature", C.c_float), ("commit_reuse_kv", C.c_int32),
+        ("temperature", C.c_float), ("commit_reuse_kv", C.c_int32), ("batch", C.c_int32),
     ]
 
 

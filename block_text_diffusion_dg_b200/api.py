@@ -34,12 +34,13 @@ def _need_cuda(t, name, dtype=None):
 def make_config(shape, *, kv_capacity, fixed_steps=16, max_steps=48, tau=0.9, h_bound=0.005,
                 eps=1e-6, rope_theta=10000.0, prefill_chunk=0, experts="bf16",
                 lock_rule="confidence", entropy_lock=0.1, sticky=False, temperature=1.0,
-                commit="reencode"):
+                commit="reencode", batch=1):
     """Config of a model shape; experts="e4m3" selects the FP8 expert format (bf16 model);
     lock_rule="entropy_bound" locks positions with entropy <= entropy_lock (nats) instead of
     confidence >= tau; sticky=True keeps a locked position's token for the rest of the block;
     temperature sets T of the sampler's softmax(logits / T); commit="reuse_kv" commits a block
-    by keeping the canvas K/V of its last denoise step instead of re-encoding it causally."""
+    by keeping the canvas K/V of its last denoise step instead of re-encoding it causally;
+    batch=B decodes B sequences in lockstep (sequence b's Philox key is seed + b)."""
     if commit not in ("reencode", "reuse_kv"):
         raise ValueError("commit must be 'reencode' or 'reuse_kv'")
     s = shape
@@ -63,7 +64,7 @@ def make_config(shape, *, kv_capacity, fixed_steps=16, max_steps=48, tau=0.9, h_
         rope_theta=rope_theta, tau=tau, h_bound=h_bound, max_steps=max_steps,
         fixed_steps=fixed_steps, prefill_chunk=prefill_chunk, lock_rule=rules[lock_rule],
         entropy_lock=entropy_lock, sticky_locks=int(bool(sticky)), temperature=temperature,
-        commit_reuse_kv=int(commit == "reuse_kv"))
+        commit_reuse_kv=int(commit == "reuse_kv"), batch=int(batch))
 
 
 def workspace_bytes(cfg):
@@ -78,6 +79,8 @@ class DiffusionModel:
 
     def __init__(self, cfg, weights, device="cuda", stream=None):
         self.cfg = cfg
+        self.batch = max(1, cfg.batch)
+        self.n_tok = self.batch * cfg.canvas  # canvas positions of all sequences
         self.weights = weights  # keep the tensors alive
         self.device = torch.device(device)
         kv_b, sc_b = workspace_bytes(cfg)
@@ -102,8 +105,9 @@ class DiffusionModel:
         bufs = [C.c_void_p() for _ in range(5)]
         check(lib().dg_get_buffers(h, *[C.byref(b) for b in bufs]), "dg_get_buffers")
         self._bufs = [b.value for b in bufs]
-        self.out_ids = torch.empty(cfg.canvas, dtype=torch.int32, device=self.device)
-        self.out_state = torch.empty(L.STATE_WORDS, dtype=torch.int32, device=self.device)
+        self.out_ids = torch.empty(self.n_tok, dtype=torch.int32, device=self.device)
+        self.out_state = torch.empty(self.batch, L.STATE_WORDS, dtype=torch.int32,
+                                     device=self.device).squeeze(0)
 
     def close(self):
         if getattr(self, "handle", None):
@@ -118,9 +122,12 @@ class DiffusionModel:
 
     # --- the five entry points of the decode loop ---
     def kv_append(self, ids, stream=None):
+        """ids [n] (one sequence) or [batch, n] (row b: sequence b's next n tokens)."""
         _need_cuda(ids, "ids", torch.int32)
-        check(lib().dg_kv_append(self.handle, _ptr(ids), ids.numel(), _stream(stream)),
-              "dg_kv_append")
+        if ids.numel() % self.batch:
+            raise ValueError("ids must hold the same number of tokens for every sequence")
+        check(lib().dg_kv_append(self.handle, _ptr(ids), ids.numel() // self.batch,
+                                 _stream(stream)), "dg_kv_append")
 
     def canvas_init(self, seed, block, stream=None):
         check(lib().dg_canvas_init(self.handle, C.c_uint64(seed), block, _stream(stream)),
@@ -157,30 +164,33 @@ class DiffusionModel:
         return self.scratch[off:off + nbytes].view(dtype)
 
     def buffers(self):
-        t = self.cfg.canvas
+        """Views of the canvas, argmax, entropy and confidence ([batch * canvas], sequence-major)
+        and of the state words ([STATE_WORDS], or [batch, STATE_WORDS] when batched)."""
+        t = self.n_tok
+        st = self._view(self._bufs[4], self.batch * L.STATE_WORDS, torch.int32)
         return dict(canvas=self._view(self._bufs[0], t, torch.int32),
                     argmax=self._view(self._bufs[1], t, torch.int32),
                     entropy=self._view(self._bufs[2], t, torch.float32),
                     conf=self._view(self._bufs[3], t, torch.float32),
-                    state=self._view(self._bufs[4], L.STATE_WORDS, torch.int32))
+                    state=st if self.batch == 1 else st.view(self.batch, L.STATE_WORDS))
 
     def check_device_status(self, stream=None):
         check(lib().dg_check_device_status(self.handle, _stream(stream)), "dg_check_device_status")
 
     def debug_logits(self, stream=None):
-        out = torch.empty(self.cfg.canvas, self.cfg.vocab, dtype=torch.float32, device=self.device)
+        out = torch.empty(self.n_tok, self.cfg.vocab, dtype=torch.float32, device=self.device)
         check(lib().dg_debug_logits(self.handle, _ptr(out), _stream(stream)), "dg_debug_logits")
         return out
 
     def debug_hidden(self):
         p = C.c_void_p()
         check(lib().dg_debug_hidden(self.handle, C.byref(p)), "dg_debug_hidden")
-        return self._view(p.value, self.cfg.canvas * self.cfg.d_model, torch.float32).view(
-            self.cfg.canvas, self.cfg.d_model)
+        return self._view(p.value, self.n_tok * self.cfg.d_model, torch.float32).view(
+            self.n_tok, self.cfg.d_model)
 
     def debug_routing(self, n=None):
         """(ids [n, k], weights [n, k], router logits [n, E]) of the last layer run."""
-        n = self.cfg.canvas if n is None else n
+        n = self.n_tok if n is None else n
         ps = [C.c_void_p() for _ in range(3)]
         check(lib().dg_debug_routing(self.handle, *[C.byref(x) for x in ps]), "dg_debug_routing")
         k, e = self.cfg.top_k, self.cfg.n_experts
@@ -219,20 +229,27 @@ class DiffusionModel:
 
 
 def generate(model, prompt_ids, n_blocks, seed, stream=None):
-    """Block-autoregressive decode through the C ABI; returns (ids [n_blocks*T], states)."""
+    """Block-autoregressive decode through the C ABI.
+
+    One sequence: returns (ids [n_blocks * T], states [n_blocks, STATE_WORDS]).  A batched model
+    takes prompt_ids [batch, n] and returns (ids [batch, n_blocks * T], states [n_blocks, batch,
+    STATE_WORDS]); sequence b's canvases draw from the Philox key seed + b."""
     cfg = model.cfg
     if prompt_ids is not None and prompt_ids.numel():
         model.kv_append(prompt_ids, stream)
     steps = cfg.fixed_steps if cfg.fixed_steps > 0 else cfg.max_steps
-    out = torch.empty(n_blocks * cfg.canvas, dtype=torch.int32, device=model.device)
-    states = torch.empty(n_blocks, L.STATE_WORDS, dtype=torch.int32, device=model.device)
+    nb, t = model.batch, cfg.canvas
+    out = torch.empty(n_blocks, nb * t, dtype=torch.int32, device=model.device)
+    states = torch.empty(n_blocks, nb, L.STATE_WORDS, dtype=torch.int32, device=model.device)
     for b in range(n_blocks):
         model.canvas_init(seed, b, stream)
-        for t in range(1, steps + 1):
-            model.denoise_step(t, stream)
-            model.sample_update(t, stream)
-        model.commit_block(out[b * cfg.canvas:(b + 1) * cfg.canvas], states[b], stream)
-    return out, states
+        for s in range(1, steps + 1):
+            model.denoise_step(s, stream)
+            model.sample_update(s, stream)
+        model.commit_block(out[b], states[b], stream)
+    if nb == 1:
+        return out.view(n_blocks * t), states.view(n_blocks, L.STATE_WORDS)
+    return (out.view(n_blocks, nb, t).transpose(0, 1).reshape(nb, n_blocks * t), states)
 
 
 # ---------------------------------------------------------------------------------------

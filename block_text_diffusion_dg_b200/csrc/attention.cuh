@@ -37,6 +37,12 @@ struct AttnParams {
   int ldk;            // keys per kv head in tm_k rows
   int vt_row_base;    // tm_vt row of kv head 0, dim 0
   int n_heads;
+  // Batched canvases: queries come in runs of seq_len tokens (a multiple of 128; 0 = one
+  // sequence), run b attending to sequence b's cache, k_seq_rows / vt_seq_rows further down tm_k /
+  // tm_vt; key counts, positions and the causal prefix are relative to the run
+  int seq_len;
+  long long k_seq_rows;
+  int vt_seq_rows;
   float* o_part;      // [splits, Hq, tq, 128]
   float2* ml_part;    // [splits, Hq, tq] (max in log2 units, denominator)
   __nv_bfloat16* o;   // [T, Hq * 128] merged output
@@ -127,9 +133,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int split = blockIdx.z;
   const int head = g * p.group + mt / p.tiles_per_head;
   const int tok0 = (mt % p.tiles_per_head) * 128;
+  // the sequence this query tile belongs to, and the tile's first token within it
+  const int seq = p.seq_len > 0 ? tok0 / p.seq_len : 0;
+  const int rel0 = tok0 - seq * p.seq_len;
   const int n_kv_tiles = (p.n_keys + 127) >> 7;
   int tile_end = n_kv_tiles;
-  if (p.causal_prefix >= 0) tile_end = min(tile_end, (p.causal_prefix + tok0 + 127) / 128 + 1);
+  if (p.causal_prefix >= 0) tile_end = min(tile_end, (p.causal_prefix + rel0 + 127) / 128 + 1);
   const int tile0 = split * p.tiles_per_split;
   const int n_tiles = max(0, min(tile0 + p.tiles_per_split, tile_end) - tile0);
 
@@ -172,12 +181,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_arrive_expect_tx(q_full, 2 * kAttnTile);
       tma_load_2d(&tm_q, q_full, s_q, 0, q_row, pol);
       tma_load_2d(&tm_q, q_full, s_q + kAttnTile, 64, q_row, pol);
-      const int vt_row = p.vt_row_base + g * 128;
+      const int vt_row = p.vt_row_base + seq * p.vt_seq_rows + g * 128;
+      const long long k_base = p.k_row_base + seq * p.k_seq_rows + static_cast<long long>(g) * p.ldk;
       auto load_k = [&](int j) -> bool {
         const int st = j & 1;
         if (!mbar_wait(&k_empty[st], ((j >> 1) & 1) ^ 1u, p.err)) return false;
         const int key0 = (tile0 + j) * 128;
-        const int k_row = static_cast<int>(p.k_row_base + static_cast<long long>(g) * p.ldk + key0);
+        const int k_row = static_cast<int>(k_base + key0);
         uint8_t* sk = s_k + st * 2 * kAttnTile;
         mbar_arrive_expect_tx(&k_full[st], 2 * kAttnTile);
         tma_load_2d(&tm_k, &k_full[st], sk, 0, k_row, pol);
@@ -256,7 +266,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t xchg = tmem_base + 384 + lane_off;  // partner exchange columns
     const int bar_id = 1 + q4;                         // the two warps of this lane quarter
     const int key_lim =
-        p.causal_prefix >= 0 ? min(p.n_keys, p.causal_prefix + tok + 1) : p.n_keys;
+        p.causal_prefix >= 0 ? min(p.n_keys, p.causal_prefix + rel0 + r + 1) : p.n_keys;
     // Every thread passes the same named barriers whatever happens (one per tile and one at
     // the end), so a failed wait only turns the remaining work off: `ok` is warp-uniform.
     float m_run = -INFINITY, l_run = 0.f;

@@ -89,6 +89,7 @@ inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255);
 inline int cdiv(long long a, long long b) { return static_cast<int>((a + b - 1) / b); }
 // Row pitch (bytes) of an e4m3 matrix with `cols` codes per row (DG_E4M3_PITCH).
 inline int e4m3_pitch(int cols) { return (cols + 127) / 128 * 128; }
+constexpr int kMaxBatch = 16;  // sequences of a batched context
 
 // ---- TMA descriptor encoding through the driver entry point ---------------------------
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -204,10 +205,12 @@ int launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 
 // ---- GEMM launch helpers -----------------------------------------------------------------
 constexpr int kGroupN = 64, kGroupStages = 8;
-// Long passes (a prompt encoded at once) give each expert hundreds of tokens: there the grouped
-// GEMMs take 256-token chunks, so each expert weight tile streams once per 256 tokens, not 64.
+// Long passes (a prompt encoded at once, or a batch of canvases) give each expert many tokens:
+// there the grouped GEMMs take 256-token chunks, so each expert weight tile streams once per 256
+// tokens, not once per 64.  From 48 slots per expert on average, a good part of the experts would
+// need a second 64-token chunk (a second pass over their weights).
 constexpr int kGroupWideN = 256, kGroupWideStages = 4;
-bool group_wide(long long n_slots, int n_experts) { return n_slots > 64ll * n_experts; }
+bool group_wide(long long n_slots, int n_experts) { return n_slots >= 48ll * n_experts; }
 constexpr int kRouterChunk = 64;  // tokens per router cluster
 constexpr int kPrefetchExperts = 4;  // routed chunks whose expert weights the gather prefetches
 
@@ -465,6 +468,7 @@ struct dg_ctx {
   uint8_t* scratch;
   int32_t kv_len;
   int sms;
+  int batch;        // sequences decoded together (>= 1)
   bool bf16;
   int esz;          // bytes per stored element (2 or 4)
   int tq;           // query rows per head in the Q buffer
@@ -474,6 +478,7 @@ struct dg_ctx {
   size_t part_elems;
   // scratch views
   int32_t *canvas, *argmax, *prev_argmax, *locked, *state, *ticket, *err;
+  int32_t* all_done;  // [0] every canvas stopped, [1] stopped canvases (after the state words)
   float *entropy, *conf;
   double* row_h;
   float* x;
@@ -523,7 +528,8 @@ int check_config(const dg_config* c) {
     return fail(DG_ERR_INVALID_ARG, "kv_capacity must be a multiple of 8 and >= canvas");
   // TMA row coordinates of the K cache ([L * Hkv * cap] rows) and the per-layer V^T offsets are
   // 32-bit
-  if (static_cast<long long>(c->n_layers) * c->n_kv_heads * c->kv_capacity >= (1ll << 31) ||
+  if (static_cast<long long>(std::max(1, c->batch)) * c->n_layers * c->n_kv_heads *
+              c->kv_capacity >= (1ll << 31) ||
       static_cast<long long>(c->n_kv_heads) * c->head_dim * c->kv_capacity >= (1ll << 31))
     return fail(DG_ERR_UNSUPPORTED, "kv_capacity too large for 32-bit cache coordinates");
   if (c->head_dim % 4 != 0) return fail(DG_ERR_INVALID_ARG, "head_dim must be a multiple of 4");
@@ -536,6 +542,12 @@ int check_config(const dg_config* c) {
     return fail(DG_ERR_INVALID_ARG, "max_steps must be >= 1 and fixed_steps >= 0");
   if (c->prefill_chunk < 0 || c->prefill_chunk % 128 != 0 || c->prefill_chunk > 4096)
     return fail(DG_ERR_INVALID_ARG, "prefill_chunk must be 0 or a multiple of 128, <= 4096");
+  if (c->batch < 0 || c->batch > kMaxBatch)
+    return fail(DG_ERR_INVALID_ARG, "batch must be in [0, %d]", kMaxBatch);
+  if (c->batch > 1 && (c->dtype == DG_DTYPE_FP32 || c->canvas % 128 != 0 ||
+                       c->batch * c->canvas > 4096))
+    return fail(DG_ERR_UNSUPPORTED,
+                "batch > 1 needs a bf16 dtype, canvas %% 128 == 0 and batch * canvas <= 4096");
   if (c->commit_reuse_kv < 0 || c->commit_reuse_kv > 1)
     return fail(DG_ERR_INVALID_ARG, "commit_reuse_kv must be 0 or 1");
   if (!(c->temperature >= 0.0f) || c->temperature > 1e4f)
@@ -579,8 +591,10 @@ struct Derived {
   long long max_chunks;
 };
 
-// Most tokens one forward pass carries: a canvas, or a prefill chunk of the prompt.
-int tokens_max(const dg_config& c) { return std::max(c.canvas, c.prefill_chunk); }
+// Sequences decoded together (batched canvases).
+int n_seq(const dg_config& c) { return std::max(1, c.batch); }
+// Most tokens one forward pass carries: the batch's canvases, or a prefill chunk of one prompt.
+int tokens_max(const dg_config& c) { return std::max(n_seq(c) * c.canvas, c.prefill_chunk); }
 
 Derived derive(const dg_config& c, int sms) {
   Derived d{};
@@ -600,7 +614,7 @@ Derived derive(const dg_config& c, int sms) {
                              static_cast<size_t>(T) * c.n_experts});
   }
   const int group = c.n_heads / c.n_kv_heads;
-  const int m_tiles = group * cdiv(c.canvas, 128);  // the most splits are taken by a canvas
+  const int m_tiles = group * cdiv(c.canvas, 128) * n_seq(c);  // a denoise pass takes the most splits
   d.att_splits = std::max(1, std::min(kMaxAttnSplits, sms / std::max(1, m_tiles * c.n_kv_heads)));
   d.max_chunks = c.n_experts + (T * c.top_k + kGroupN - 1) / kGroupN;
   return d;
@@ -611,14 +625,17 @@ Plan plan(const dg_config& c, int sms) {
   const Derived dv = derive(c, sms);
   const bool bf16 = c.dtype != DG_DTYPE_FP32;
   const bool f8 = c.dtype == DG_DTYPE_BF16_E4M3;
-  const size_t Tc = c.canvas, T = tokens_max(c), d = c.d_model, E = c.n_experts, k = c.top_k,
-               es = dv.esz;
+  // Tc: canvas positions of all sequences; per-canvas arrays are [batch][canvas]
+  const size_t Tc = static_cast<size_t>(c.canvas) * n_seq(c), T = tokens_max(c), d = c.d_model,
+               E = c.n_experts, k = c.top_k, es = dv.esz;
   const size_t hd = c.head_dim, Hq = c.n_heads;
   const size_t nv = bf16 ? c.vocab / 256 : cdiv(c.vocab, 4096);
   size_t sz[B_END];
   sz[B_CANVAS] = sz[B_ARGMAX] = sz[B_PREV] = sz[B_LOCKED] = Tc * 4;
-  sz[B_STATE] = kStWords * 4;
-  sz[B_TICKET] = sz[B_ERR] = 4;
+  // state words per sequence, then the all-done flag and count
+  sz[B_STATE] = (static_cast<size_t>(n_seq(c)) * kStWords + 2) * 4;
+  sz[B_TICKET] = static_cast<size_t>(n_seq(c)) * 4;
+  sz[B_ERR] = 4;
   sz[B_ENT] = sz[B_CONF] = Tc * 4;
   sz[B_ROWH] = Tc * 8;
   sz[B_X] = T * d * 4;
@@ -661,7 +678,8 @@ Plan plan(const dg_config& c, int sms) {
     o += align256(std::max<size_t>(sz[b], 1));
   }
   p.total = o;
-  p.kv = 2 * static_cast<size_t>(c.n_layers) * c.n_kv_heads * c.kv_capacity * hd * es;
+  // K of every (sequence, layer), then V^T of every (sequence, layer)
+  p.kv = 2 * static_cast<size_t>(n_seq(c)) * c.n_layers * c.n_kv_heads * c.kv_capacity * hd * es;
   return p;
 }
 
@@ -670,11 +688,14 @@ Plan plan(const dg_config& c, int sms) {
 // K/V into cache slots pos0..pos0+n-1 and leaves the final-normed hidden state in xn.
 // parts: bit 0 = attention sub-block (QKV .. O projection, residual, ffn norm), bit 1 = MoE
 // sub-block (router .. weighted combine, residual, next norm).
+// seq0: the sequence whose cache the pass uses (a prefill pass of one prompt); seq_len > 0: the n
+// tokens are consecutive runs of seq_len tokens of sequences 0, 1, ... (a denoise or commit pass
+// over a batch of canvases), each at positions pos0.. of its own cache.
 int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_norm,
-              const int* done, cudaStream_t st, int parts = 3);
+              const int* done, cudaStream_t st, int parts = 3, int seq0 = 0, int seq_len = 0);
 
 int run_forward(dg_ctx* c, const int32_t* ids, int n, int pos0, int causal, const int* done,
-                cudaStream_t st) {
+                cudaStream_t st, int seq0 = 0, int seq_len = 0) {
   const dg_config& g = c->cfg;
   prof_before(DG_KERNEL_EMBED, st);
   if (c->bf16)
@@ -689,7 +710,7 @@ int run_forward(dg_ctx* c, const int32_t* ids, int n, int pos0, int causal, cons
   prof_after(DG_KERNEL_EMBED, st);
   for (int l = 0; l < g.n_layers; ++l) {
     const float* nn = (l + 1 < g.n_layers) ? c->layers[l + 1].attn_norm : c->final_norm;
-    DG_TRY(run_layer(c, l, n, pos0, causal, nn, done, st));
+    DG_TRY(run_layer(c, l, n, pos0, causal, nn, done, st, 3, seq0, seq_len));
   }
   return DG_OK;
 }
@@ -712,11 +733,15 @@ int layer_tail_common(dg_ctx* c, int l, int n, int pos0, const int* done, cudaSt
 }
 
 int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_norm,
-              const int* done, cudaStream_t st, int parts) {
+              const int* done, cudaStream_t st, int parts, int seq0, int seq_len) {
   const dg_config& g = c->cfg;
+  // cache layer block of (sequence seq0, layer l); sequences are L layer blocks apart
+  const long long lb = static_cast<long long>(seq0) * g.n_layers + l;
+  const long long seq_blocks = seq_len > 0 ? g.n_layers : 0;
   const dg_layer_weights& w = c->layers[l];
   const int d = g.d_model, hd = g.head_dim, k = g.top_k, E = g.n_experts;
-  const int n_keys = pos0 + n;
+  // keys each query sees: the committed history plus its own sequence's new tokens
+  const int n_keys = pos0 + (seq_len > 0 ? seq_len : n);
   const int n_slots = n * k;
   if (!c->bf16) {
     // ---------------- all-fp32 path ----------------
@@ -788,8 +813,10 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     p.ldk = g.kv_capacity;
     p.rope_tab = c->rope_tab;
     p.q = static_cast<__nv_bfloat16*>(c->q);
-    p.k_cache = static_cast<__nv_bfloat16*>(c->kc) + static_cast<size_t>(l) * g.n_kv_heads * kv_head_elems;
-    p.vt_cache = static_cast<__nv_bfloat16*>(c->vtc) + static_cast<size_t>(l) * g.n_kv_heads * kv_head_elems;
+    p.k_cache = static_cast<__nv_bfloat16*>(c->kc) + static_cast<size_t>(lb) * g.n_kv_heads * kv_head_elems;
+    p.vt_cache = static_cast<__nv_bfloat16*>(c->vtc) + static_cast<size_t>(lb) * g.n_kv_heads * kv_head_elems;
+    p.seq_len = seq_len;
+    p.seq_kv_stride = seq_blocks * g.n_kv_heads * static_cast<long long>(kv_head_elems);
     DG_TRY(launch_cluster<kCluQkv>(c->tm_wqkv[l], c->tm_xn32, p, st, DG_KERNEL_QKV));
   }
   // attention over [cache 0..pos0 | new tokens], split over keys
@@ -812,9 +839,12 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(hd)));
     a.tiles_per_split = tps;
     a.q_row_base = 0;
-    a.k_row_base = static_cast<long long>(l) * g.n_kv_heads * g.kv_capacity;
+    a.k_row_base = lb * g.n_kv_heads * g.kv_capacity;
     a.ldk = g.kv_capacity;
-    a.vt_row_base = l * g.n_kv_heads * hd;
+    a.vt_row_base = static_cast<int>(lb * g.n_kv_heads * hd);
+    a.seq_len = seq_len;
+    a.k_seq_rows = seq_blocks * g.n_kv_heads * g.kv_capacity;
+    a.vt_seq_rows = static_cast<int>(seq_blocks * g.n_kv_heads * hd);
     a.n_heads = g.n_heads;
     a.o_part = c->o_part;
     a.ml_part = c->ml_part;
@@ -934,27 +964,34 @@ int run_lm_head(dg_ctx* c, float* logits_out, const int* done, cudaStream_t st) 
   const dg_config& g = c->cfg;
   const int T = g.canvas;
   if (c->bf16) {
-    LmHeadParams p{};
-    p.n_tokens = T;
-    p.n_vtiles = g.vocab / 256;
-    p.kb_total = g.d_model / 64;
-    p.partials = c->lm_part;
-    p.logits = logits_out;
-    p.vocab = g.vocab;
-    p.inv_t = g.temperature > 0.0f ? 1.0f / g.temperature : 1.0f;
-    p.err = c->err;
-    p.done = done;
-    const int grid = std::min(p.n_vtiles, c->sms);
-    prof_before(DG_KERNEL_LM_HEAD, st);
-    if (logits_out) {
-      DG_TRY(set_smem(lmhead_kernel<false>, kLmSmemBytes));
-      DG_TRY(launch_pdl(lmhead_kernel<false>, dim3(grid), dim3(kLmThreads), kLmSmemBytes, st, c->tm_xn128, c->tm_embed, p));
-    } else {
-      DG_TRY(set_smem(lmhead_kernel<true>, kLmSmemBytes));
-      DG_TRY(launch_pdl(lmhead_kernel<true>, dim3(grid), dim3(kLmThreads), kLmSmemBytes, st, c->tm_xn128, c->tm_embed, p));
+    // one launch per 256 canvas tokens (each launch holds two 128-token accumulators in TMEM)
+    const int n_tok = T * c->batch;
+    for (int t0 = 0; t0 < n_tok; t0 += 256) {
+      LmHeadParams p{};
+      p.n_tokens = std::min(256, n_tok - t0);
+      p.tok_base = t0;
+      p.n_vtiles = g.vocab / 256;
+      p.kb_total = g.d_model / 64;
+      p.partials = c->lm_part;
+      p.logits = logits_out;
+      p.vocab = g.vocab;
+      p.inv_t = g.temperature > 0.0f ? 1.0f / g.temperature : 1.0f;
+      p.err = c->err;
+      p.done = done;
+      const int grid = std::min(p.n_vtiles, c->sms);
+      prof_before(DG_KERNEL_LM_HEAD, st);
+      if (logits_out) {
+        DG_TRY(set_smem(lmhead_kernel<false>, kLmSmemBytes));
+        DG_TRY(launch_pdl(lmhead_kernel<false>, dim3(grid), dim3(kLmThreads), kLmSmemBytes, st,
+                          c->tm_xn128, c->tm_embed, p));
+      } else {
+        DG_TRY(set_smem(lmhead_kernel<true>, kLmSmemBytes));
+        DG_TRY(launch_pdl(lmhead_kernel<true>, dim3(grid), dim3(kLmThreads), kLmSmemBytes, st,
+                          c->tm_xn128, c->tm_embed, p));
+      }
+      DG_LAUNCHED();
+      prof_after(DG_KERNEL_LM_HEAD, st);
     }
-    DG_LAUNCHED();
-    prof_after(DG_KERNEL_LM_HEAD, st);
     return DG_OK;
   }
   float* dst = logits_out ? logits_out : c->logits;
@@ -988,9 +1025,11 @@ int bind_tmaps(dg_ctx* c) {
     DG_TRY(make_tmap(&c->tm_hs, c->f8 ? c->hsq : c->hs, T, g.shared_hidden, phs, 32, eb));
   if (c->f8) DG_TRY(make_tmap(&c->tm_xsh, c->x_sh, T, d, pd, 32, 1));
   DG_TRY(make_tmap(&c->tm_q, c->q, static_cast<uint64_t>(g.n_heads) * c->tq, hd, hd, 128));
-  const uint64_t kv_rows = static_cast<uint64_t>(g.n_layers) * g.n_kv_heads * g.kv_capacity;
+  // every (sequence, layer) pair of a batched context is one more layer block of the cache
+  const uint64_t kv_rows =
+      static_cast<uint64_t>(c->batch) * g.n_layers * g.n_kv_heads * g.kv_capacity;
   DG_TRY(make_tmap(&c->tm_k, c->kc, kv_rows, hd, hd, 128));
-  const uint64_t vt_rows = static_cast<uint64_t>(g.n_layers) * g.n_kv_heads * hd;
+  const uint64_t vt_rows = static_cast<uint64_t>(c->batch) * g.n_layers * g.n_kv_heads * hd;
   DG_TRY(make_tmap(&c->tm_vt, c->vtc, vt_rows, g.kv_capacity, g.kv_capacity, 128));
   DG_TRY(make_tmap(&c->tm_embed, c->embed, g.vocab, d, d, 256));
   const int L = g.n_layers;
@@ -1093,6 +1132,7 @@ int dg_create(const dg_config* cfg, const dg_weights* w, void* d_kv, void* d_scr
   c->scratch = static_cast<uint8_t*>(d_scratch);
   c->kv_len = 0;
   c->sms = num_sms();
+  c->batch = n_seq(*cfg);
   c->bf16 = cfg->dtype != DG_DTYPE_FP32;
   c->f8 = cfg->dtype == DG_DTYPE_BF16_E4M3;
   const Derived dv = derive(*cfg, c->sms);
@@ -1109,6 +1149,7 @@ int dg_create(const dg_config* cfg, const dg_weights* w, void* d_kv, void* d_scr
   c->prev_argmax = reinterpret_cast<int32_t*>(s + p.off[B_PREV]);
   c->locked = reinterpret_cast<int32_t*>(s + p.off[B_LOCKED]);
   c->state = reinterpret_cast<int32_t*>(s + p.off[B_STATE]);
+  c->all_done = c->state + static_cast<size_t>(c->batch) * kStWords;
   c->ticket = reinterpret_cast<int32_t*>(s + p.off[B_TICKET]);
   c->err = reinterpret_cast<int32_t*>(s + p.off[B_ERR]);
   c->entropy = reinterpret_cast<float*>(s + p.off[B_ENT]);
@@ -1196,11 +1237,14 @@ int dg_kv_append(dg_ctx* ctx, const int32_t* d_ids, int32_t n, void* stream) {
                 ctx->cfg.kv_capacity, ctx->kv_len + n, ctx->cfg.canvas);
   cudaStream_t st = S(stream);
   const int chunk = ctx->cfg.prefill_chunk > 0 ? ctx->cfg.prefill_chunk : ctx->cfg.canvas;
-  for (int off = 0; off < n; off += chunk) {
-    const int m = std::min(chunk, n - off);
-    DG_TRY(run_forward(ctx, d_ids + off, m, ctx->kv_len, 1, nullptr, st));
-    ctx->kv_len += m;
-  }
+  // every sequence's prompt (row b of d_ids) into its own cache, in passes of `chunk` tokens
+  for (int b = 0; b < ctx->batch; ++b)
+    for (int off = 0; off < n; off += chunk) {
+      const int m = std::min(chunk, n - off);
+      DG_TRY(run_forward(ctx, d_ids + static_cast<size_t>(b) * n + off, m, ctx->kv_len + off, 1,
+                         nullptr, st, b, 0));
+    }
+  ctx->kv_len += n;
   return DG_OK;
 }
 
@@ -1210,17 +1254,18 @@ int dg_canvas_init(dg_ctx* ctx, uint64_t seed, uint32_t block, void* stream) {
     return fail(DG_ERR_CAPACITY, "no room for a canvas after %d committed positions", ctx->kv_len);
   ctx->seed = seed;
   ctx->block = block;
-  DG_TRY(launch_pdl(canvas_init_kernel, dim3(cdiv(ctx->cfg.canvas, 256)), dim3(256), 0, S(stream),
-      ctx->canvas, ctx->cfg.canvas, ctx->cfg.vocab, seed, block, ctx->state, ctx->ticket,
-      ctx->locked));
+  DG_TRY(launch_pdl(canvas_init_kernel, dim3(cdiv(ctx->cfg.canvas * ctx->batch, 256)), dim3(256),
+      0, S(stream), ctx->canvas, ctx->cfg.canvas, ctx->batch, ctx->cfg.vocab, seed, block,
+      ctx->state, ctx->ticket, ctx->locked, ctx->all_done));
   DG_LAUNCHED();
   return DG_OK;
 }
 
 int dg_reset_block(dg_ctx* ctx, void* stream) {
   DG_TRY(check_ctx(ctx));
-  DG_TRY(launch_pdl(block_reset_kernel, dim3(cdiv(ctx->cfg.canvas, 256)), dim3(256), 0, S(stream),
-                    ctx->state, ctx->ticket, ctx->locked, ctx->cfg.canvas));
+  DG_TRY(launch_pdl(block_reset_kernel, dim3(cdiv(ctx->cfg.canvas * ctx->batch, 256)), dim3(256),
+                    0, S(stream), ctx->state, ctx->ticket, ctx->locked, ctx->cfg.canvas,
+                    ctx->batch, ctx->all_done));
   DG_LAUNCHED();
   return DG_OK;
 }
@@ -1231,8 +1276,10 @@ int dg_denoise_step(dg_ctx* ctx, uint32_t step, void* stream) {
   if (ctx->kv_len + ctx->cfg.canvas > ctx->cfg.kv_capacity)
     return fail(DG_ERR_CAPACITY, "no room for the canvas");
   cudaStream_t st = S(stream);
-  const int* done = ctx->state + kStDone;
-  DG_TRY(run_forward(ctx, ctx->canvas, ctx->cfg.canvas, ctx->kv_len, 0, done, st));
+  // a no-op on the device once every canvas has stopped
+  const int* done = ctx->all_done;
+  DG_TRY(run_forward(ctx, ctx->canvas, ctx->cfg.canvas * ctx->batch, ctx->kv_len, 0, done, st, 0,
+                     ctx->cfg.canvas));
   DG_TRY(run_lm_head(ctx, nullptr, done, st));
   return DG_OK;
 }
@@ -1265,8 +1312,10 @@ int dg_sample_update(dg_ctx* ctx, uint32_t step, void* stream) {
   a.locked = ctx->locked;
   a.state = ctx->state;
   a.ticket = ctx->ticket;
+  a.n_seq = ctx->batch;
+  a.all_done = ctx->all_done;
   prof_before(DG_KERNEL_SAMPLER, S(stream));
-  DG_TRY(launch_pdl(sampler_merge_kernel, dim3(g.canvas), dim3(256), 0, S(stream), a));
+  DG_TRY(launch_pdl(sampler_merge_kernel, dim3(g.canvas * ctx->batch), dim3(256), 0, S(stream), a));
   DG_LAUNCHED();
   prof_after(DG_KERNEL_SAMPLER, S(stream));
   return DG_OK;
@@ -1278,21 +1327,26 @@ int dg_commit_block(dg_ctx* ctx, int32_t* d_out_ids, int32_t* d_state, void* str
   if (ctx->kv_len + g.canvas > g.kv_capacity) return fail(DG_ERR_CAPACITY, "cache full");
   cudaStream_t st = S(stream);
   // the committed ids: the argmax of the stop step, or with sticky locks the locked tokens
+  const int n_tok = g.canvas * ctx->batch;
   const int32_t* ids = ctx->argmax;
   if (g.sticky_locks) {
-    DG_TRY(launch_pdl(commit_ids_kernel, dim3(cdiv(g.canvas, 256)), dim3(256), 0, st,
+    DG_TRY(launch_pdl(commit_ids_kernel, dim3(cdiv(n_tok, 256)), dim3(256), 0, st,
                       static_cast<const int32_t*>(ctx->canvas),
                       static_cast<const int32_t*>(ctx->argmax),
-                      static_cast<const int32_t*>(ctx->locked), ctx->commit_ids, g.canvas));
+                      static_cast<const int32_t*>(ctx->locked), ctx->commit_ids, n_tok));
     DG_LAUNCHED();
     ids = ctx->commit_ids;
   }
   if (d_out_ids)
-    DG_CUDA(cudaMemcpyAsync(d_out_ids, ids, g.canvas * 4, cudaMemcpyDeviceToDevice, st));
+    DG_CUDA(cudaMemcpyAsync(d_out_ids, ids, static_cast<size_t>(n_tok) * 4,
+                            cudaMemcpyDeviceToDevice, st));
   if (d_state)
-    DG_CUDA(cudaMemcpyAsync(d_state, ctx->state, kStWords * 4, cudaMemcpyDeviceToDevice, st));
-  // re-encode causally, or keep the canvas K/V the last denoise step left in slots P..P+T-1
-  if (!g.commit_reuse_kv) DG_TRY(run_forward(ctx, ids, g.canvas, ctx->kv_len, 1, nullptr, st));
+    DG_CUDA(cudaMemcpyAsync(d_state, ctx->state, static_cast<size_t>(ctx->batch) * kStWords * 4,
+                            cudaMemcpyDeviceToDevice, st));
+  // re-encode causally (every sequence's block into its own cache), or keep the canvas K/V the
+  // last denoise step left in slots P..P+T-1
+  if (!g.commit_reuse_kv)
+    DG_TRY(run_forward(ctx, ids, n_tok, ctx->kv_len, 1, nullptr, st, 0, g.canvas));
   ctx->kv_len += g.canvas;
   return DG_OK;
 }
@@ -1341,9 +1395,13 @@ int dg_debug_layer_part(dg_ctx* ctx, int32_t layer, int32_t part, const float* d
   const dg_config& g = ctx->cfg;
   if (layer < 0 || layer >= g.n_layers) return fail(DG_ERR_INVALID_ARG, "bad layer %d", layer);
   if (part != 0 && part != 1) return fail(DG_ERR_INVALID_ARG, "part must be 0 or 1");
-  if (!d_x_in || !d_x_out || n < 1 || n > g.canvas)
-    return fail(DG_ERR_INVALID_ARG, "need x_in, x_out and 1 <= n <= canvas");
-  if (ctx->kv_len + n > g.kv_capacity) return fail(DG_ERR_CAPACITY, "cache full");
+  // a batched context runs the layer over all its canvases' tokens (n = batch * canvas)
+  const int seq_len = ctx->batch > 1 ? g.canvas : 0;
+  if (!d_x_in || !d_x_out || n < 1 || (seq_len ? n != g.canvas * ctx->batch : n > g.canvas))
+    return fail(DG_ERR_INVALID_ARG, "need x_in, x_out and 1 <= n <= canvas (batch * canvas)");
+  // every sequence writes its own tokens' K/V at positions P.. of its own cache
+  if (ctx->kv_len + (seq_len ? seq_len : n) > g.kv_capacity)
+    return fail(DG_ERR_CAPACITY, "cache full");
   cudaStream_t st = S(stream);
   DG_CUDA(cudaMemcpyAsync(ctx->x, d_x_in, static_cast<size_t>(n) * g.d_model * 4,
                           cudaMemcpyDeviceToDevice, st));
@@ -1356,7 +1414,8 @@ int dg_debug_layer_part(dg_ctx* ctx, int32_t layer, int32_t part, const float* d
                                                    static_cast<float*>(ctx->xn), nullptr));
   DG_LAUNCHED();
   const float* nn = (layer + 1 < g.n_layers) ? ctx->layers[layer + 1].attn_norm : ctx->final_norm;
-  DG_TRY(run_layer(ctx, layer, n, ctx->kv_len, causal, nn, nullptr, st, part == 0 ? 1 : 2));
+  DG_TRY(run_layer(ctx, layer, n, ctx->kv_len, causal, nn, nullptr, st, part == 0 ? 1 : 2, 0,
+                   seq_len));
   DG_CUDA(cudaMemcpyAsync(d_x_out, ctx->x, static_cast<size_t>(n) * g.d_model * 4,
                           cudaMemcpyDeviceToDevice, st));
   return DG_OK;
@@ -1382,9 +1441,13 @@ int dg_debug_layer(dg_ctx* ctx, int32_t layer, const float* d_x_in, float* d_x_o
   DG_TRY(check_ctx(ctx));
   const dg_config& g = ctx->cfg;
   if (layer < 0 || layer >= g.n_layers) return fail(DG_ERR_INVALID_ARG, "bad layer %d", layer);
-  if (!d_x_in || !d_x_out || n < 1 || n > g.canvas)
-    return fail(DG_ERR_INVALID_ARG, "need x_in, x_out and 1 <= n <= canvas");
-  if (ctx->kv_len + n > g.kv_capacity) return fail(DG_ERR_CAPACITY, "cache full");
+  // a batched context runs the layer over all its canvases' tokens (n = batch * canvas)
+  const int seq_len = ctx->batch > 1 ? g.canvas : 0;
+  if (!d_x_in || !d_x_out || n < 1 || (seq_len ? n != g.canvas * ctx->batch : n > g.canvas))
+    return fail(DG_ERR_INVALID_ARG, "need x_in, x_out and 1 <= n <= canvas (batch * canvas)");
+  // every sequence writes its own tokens' K/V at positions P.. of its own cache
+  if (ctx->kv_len + (seq_len ? seq_len : n) > g.kv_capacity)
+    return fail(DG_ERR_CAPACITY, "cache full");
   cudaStream_t st = S(stream);
   DG_CUDA(cudaMemcpyAsync(ctx->x, d_x_in, static_cast<size_t>(n) * g.d_model * 4,
                           cudaMemcpyDeviceToDevice, st));
@@ -1397,7 +1460,7 @@ int dg_debug_layer(dg_ctx* ctx, int32_t layer, const float* d_x_in, float* d_x_o
                                                    static_cast<float*>(ctx->xn), nullptr));
   DG_LAUNCHED();
   const float* nn = (layer + 1 < g.n_layers) ? ctx->layers[layer + 1].attn_norm : ctx->final_norm;
-  DG_TRY(run_layer(ctx, layer, n, ctx->kv_len, causal, nn, nullptr, st));
+  DG_TRY(run_layer(ctx, layer, n, ctx->kv_len, causal, nn, nullptr, st, 3, 0, seq_len));
   DG_CUDA(cudaMemcpyAsync(d_x_out, ctx->x, static_cast<size_t>(n) * g.d_model * 4,
                           cudaMemcpyDeviceToDevice, st));
   return DG_OK;
@@ -1489,6 +1552,7 @@ int dg_sampler_step(const void* d_logits, int32_t dtype, int32_t rows, int32_t v
   a.locked = locked;
   a.state = d_state;
   a.ticket = ticket;
+  a.n_seq = 1;
   // one wave of resident CTAs, each streaming an equal run of segments
   static const int grid_bf16 = resident_ctas(sampler_stream_kernel<__nv_bfloat16, 4>);
   static const int grid_f32 = resident_ctas(sampler_stream_kernel<float, 8>);
@@ -1941,6 +2005,7 @@ extern "C" int dg_sampler_step_static(const void* d_logits, int32_t dtype, int32
   a.locked = locked;
   a.state = d_state;
   a.ticket = ticket;
+  a.n_seq = 1;
   DG_TRY(launch_pdl(sampler_merge_kernel, dim3(rows), dim3(256), 0, st, a));
   DG_LAUNCHED();
   return DG_OK;

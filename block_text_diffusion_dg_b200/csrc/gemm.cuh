@@ -409,7 +409,8 @@ __global__ void __launch_bounds__(GemmCfg<MAXN, STAGES>::kThreads, 1)
 
 // ---------------------------------------------------------------------------------------
 struct LmHeadParams {
-  int n_tokens;   // valid token rows (<= 256)
+  int n_tokens;   // valid token rows of this launch (<= 256), starting at token row tok_base
+  int tok_base;   // first token row (tm_x row, partial / logits row) of this launch
   int n_vtiles;   // vocab / 256
   int kb_total;   // d / 64
   StatPartial* partials;  // [n_tokens, n_vtiles]
@@ -483,7 +484,8 @@ __global__ void __launch_bounds__(kLmThreads, 1)
           uint8_t* s0 = smem + stage * kLmStageBytes;
           mbar_arrive_expect_tx(&full[stage], n_ttiles * 16384 + 32768);
           for (int tt = 0; tt < n_ttiles; ++tt)
-            tma_load_2d(&tm_x, &full[stage], s0 + tt * 16384, kb * 64, tt * 128, pol_x);
+            tma_load_2d(&tm_x, &full[stage], s0 + tt * 16384, kb * 64, p.tok_base + tt * 128,
+                        pol_x);
           tma_load_2d(&tm_e, &full[stage], s0 + 32768, kb * 64, vt * 256, pol_e);
           if (++stage == kLmStages) {
             stage = 0;
@@ -577,7 +579,7 @@ __global__ void __launch_bounds__(kLmThreads, 1)
           const float s = (s4[0] + s4[1]) + (s4[2] + s4[3]);
           const float u = (u4[0] + u4[1]) + (u4[2] + u4[3]);
           if (tok < p.n_tokens)
-            p.partials[static_cast<long long>(tok) * p.n_vtiles + vt] =
+            p.partials[static_cast<long long>(p.tok_base + tok) * p.n_vtiles + vt] =
                 StatPartial{m * p.inv_t, s, u, vt * 256 + a};
         } else {
           for (int c = 0; c < 256; c += 32) {
@@ -585,7 +587,7 @@ __global__ void __launch_bounds__(kLmThreads, 1)
             tmem_ld32(t_row + c, v);
             if (tok < p.n_tokens) {
               float4* dst = reinterpret_cast<float4*>(
-                  p.logits + static_cast<long long>(tok) * p.vocab + vt * 256 + c);
+                  p.logits + static_cast<long long>(p.tok_base + tok) * p.vocab + vt * 256 + c);
 #pragma unroll
               for (int i = 0; i < 8; ++i)
                 dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);

@@ -54,6 +54,10 @@ struct CluParams {
   __nv_bfloat16* q;
   __nv_bfloat16* k_cache;   // [Hkv, ldk, hd] of this layer
   __nv_bfloat16* vt_cache;  // [Hkv, hd, ldk] of this layer
+  // batched canvases: token t belongs to sequence t / seq_len at position pos0 + t % seq_len,
+  // whose cache lies seq_kv_stride elements after sequence 0's (seq_len 0: one sequence)
+  int seq_len;
+  long long seq_kv_stride;
   // kCluResidual
   float* x;                 // [tokens, m_rows] fp32
   // kCluRouter
@@ -297,7 +301,9 @@ __global__ void __launch_bounds__(kCluThreads, 1)
             tt[2 * k] = tt[2 * k + 1] = t;
             rr[2 * k] = r4;
             rr[2 * k + 1] = r4 + 16;
-            const float2* tab = p.rope_tab + static_cast<long long>(p.pos0 + t0 + t) * 64 + 4 * r4;
+            const int tg = t0 + t;
+            const int rel = p.seq_len > 0 ? tg % p.seq_len : tg;
+            const float2* tab = p.rope_tab + static_cast<long long>(p.pos0 + rel) * 64 + 4 * r4;
 #pragma unroll
             for (int i = 0; i < 4; ++i) cs[k][i] = tab[i];
           }
@@ -307,12 +313,14 @@ __global__ void __launch_bounds__(kCluThreads, 1)
           for (int k = 0; k < 2; ++k) {
             if (u0 + k * kCluThreads >= nt * 16) break;
             const int tg = t0 + tt[2 * k], r4 = rr[2 * k];
+            const int sq = p.seq_len > 0 ? tg / p.seq_len : 0;
+            const int rel = tg - sq * p.seq_len;
             const float4 a = sum[2 * k], b = sum[2 * k + 1];
             __nv_bfloat16* dst =
                 head < p.n_heads
                     ? p.q + (static_cast<long long>(head) * p.tq + tg) * 128
-                    : p.k_cache +
-                          (static_cast<long long>(head - p.n_heads) * p.ldk + p.pos0 + tg) * 128;
+                    : p.k_cache + sq * p.seq_kv_stride +
+                          (static_cast<long long>(head - p.n_heads) * p.ldk + p.pos0 + rel) * 128;
             const float2 c0 = cs[k][0], c1 = cs[k][1], c2 = cs[k][2], c3 = cs[k][3];
             const float lo[4] = {a.x * c0.x - b.x * c0.y, a.y * c1.x - b.y * c1.y,
                                  a.z * c2.x - b.z * c2.y, a.w * c3.x - b.w * c3.y};
@@ -340,8 +348,10 @@ __global__ void __launch_bounds__(kCluThreads, 1)
         const int g = head - p.n_heads - p.n_kv_heads;
         for (int u = tid; u < 128 * nt; u += kCluThreads) {
           const int dd = u / nt, tl = u % nt;
-          p.vt_cache[(static_cast<long long>(g) * 128 + dd) * p.ldk + p.pos0 + t0 + t_lo + tl] =
-              vt_s[dd * vp + tl];
+          const int tg = t0 + t_lo + tl;
+          const int sq = p.seq_len > 0 ? tg / p.seq_len : 0;
+          p.vt_cache[sq * p.seq_kv_stride + (static_cast<long long>(g) * 128 + dd) * p.ldk +
+                     p.pos0 + tg - sq * p.seq_len] = vt_s[dd * vp + tl];
         }
       }
     }

@@ -55,19 +55,26 @@ DG_DEV StatD stat_merge(const StatD& x, const StatD& y) {
   return r;
 }
 
-__global__ void canvas_init_kernel(int32_t* canvas, int32_t t, int32_t vocab, uint64_t seed,
-                                   uint32_t block, int32_t* state, int32_t* ticket,
-                                   int32_t* locked) {
+// Canvas fill of n_seq canvases of t positions: canvas b takes the Philox stream keyed by seed + b
+// ([canvas] step 2: ids uniform over the vocabulary), with counter (position, 0, block, 0).  The
+// decode state of every canvas is reset (state words [n_seq][kStWords], completion tickets
+// [n_seq], lock flags) and so are the all-canvases-done words (all_done[0] flag, all_done[1]
+// count; may be null).
+__global__ void canvas_init_kernel(int32_t* canvas, int32_t t, int32_t n_seq, int32_t vocab,
+                                   uint64_t seed, uint32_t block, int32_t* state, int32_t* ticket,
+                                   int32_t* locked, int32_t* all_done) {
   pdl_enter();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < t) {
-    canvas[i] = canvas_uniform_id(seed, block, 0u, static_cast<uint32_t>(i), 0u,
-                                  static_cast<uint32_t>(vocab));
+  if (i < t * n_seq) {
+    const int b = i / t;
+    canvas[i] = canvas_uniform_id(seed + static_cast<uint64_t>(b), block, 0u,
+                                  static_cast<uint32_t>(i - b * t), 0u, static_cast<uint32_t>(vocab));
     if (locked) locked[i] = 0;
   }
-  if (blockIdx.x == 0 && threadIdx.x < kStWords) {
-    state[threadIdx.x] = 0;
-    if (threadIdx.x == 0) *ticket = 0;
+  if (blockIdx.x == 0) {
+    for (int w = threadIdx.x; w < n_seq * kStWords; w += blockDim.x) state[w] = 0;
+    if (threadIdx.x < n_seq) ticket[threadIdx.x] = 0;
+    if (all_done && threadIdx.x < 2) all_done[threadIdx.x] = 0;
   }
 }
 
@@ -77,15 +84,18 @@ __global__ void canvas_init_kernel(int32_t* canvas, int32_t t, int32_t vocab, ui
 // Clamping x - m at -1e30 makes its term exactly 0 (2^(-1e30 log2 e) = 0, 0 * -1e30 = 0).
 constexpr float kMaskedDelta = -1e30f;
 
-// Fresh decode state for a block: state words and completion ticket zeroed, lock flags of the
-// t canvas positions cleared; the canvas itself is kept (dg_reset_block).
-__global__ void block_reset_kernel(int32_t* state, int32_t* ticket, int32_t* locked, int32_t t) {
+// Fresh decode state for a block: state words, completion tickets and all-done words zeroed, lock
+// flags of the n_seq * t canvas positions cleared; the canvases themselves are kept
+// (dg_reset_block).
+__global__ void block_reset_kernel(int32_t* state, int32_t* ticket, int32_t* locked, int32_t t,
+                                   int32_t n_seq, int32_t* all_done) {
   pdl_enter();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < t) locked[i] = 0;
-  if (blockIdx.x == 0 && threadIdx.x < kStWords) {
-    state[threadIdx.x] = 0;
-    if (threadIdx.x == 0) *ticket = 0;
+  if (i < t * n_seq) locked[i] = 0;
+  if (blockIdx.x == 0) {
+    for (int w = threadIdx.x; w < n_seq * kStWords; w += blockDim.x) state[w] = 0;
+    if (threadIdx.x < n_seq) ticket[threadIdx.x] = 0;
+    if (all_done && threadIdx.x < 2) all_done[threadIdx.x] = 0;
   }
 }
 
@@ -233,7 +243,31 @@ struct SamplerArgs {
   int32_t* locked;
   int32_t* state;
   int32_t* ticket;
+  // Batched canvases: n_seq canvases of `rows` positions each, stored one after another in every
+  // per-row array (partials too); canvas b keys its Philox stream with seed + b and has its own
+  // state words (state + b * kStWords) and ticket (ticket + b).  all_done (may be null): [0] is
+  // set once every canvas has stopped, [1] counts the stopped canvases.
+  int32_t n_seq;
+  int32_t* all_done;
 };
+
+// The arguments of canvas b alone.
+DG_DEV SamplerArgs seq_view(const SamplerArgs& p, int b) {
+  SamplerArgs q = p;
+  const long long r0 = static_cast<long long>(b) * p.rows;
+  q.partials = p.partials + r0 * p.nsplit;
+  q.seed = p.seed + static_cast<uint64_t>(b);
+  q.canvas = p.canvas + r0;
+  q.argmax = p.argmax + r0;
+  q.prev_argmax = p.prev_argmax + r0;
+  q.entropy = p.entropy + r0;
+  q.conf = p.conf + r0;
+  q.row_h = p.row_h + r0;
+  q.locked = p.locked + r0;
+  q.state = p.state + b * kStWords;
+  q.ticket = p.ticket + b;
+  return q;
+}
 
 // Decide lock / re-noise for one row from its merged statistics and write the row's outputs;
 // returns (in every thread) whether this CTA is the last row to finish the step.
@@ -364,6 +398,7 @@ DG_DEV void sampler_stop_test(const SamplerArgs& p) {
     if (done) {
       st[kStStopStep] = step;
       st[kStDone] = 1;
+      if (p.all_done && atomicAdd(p.all_done + 1, 1) == p.n_seq - 1) p.all_done[0] = 1;
     }
     *p.ticket = 0;
   }
@@ -371,12 +406,15 @@ DG_DEV void sampler_stop_test(const SamplerArgs& p) {
   for (int i = threadIdx.x; i < p.rows; i += blockDim.x) p.prev_argmax[i] = __ldcg(p.argmax + i);
 }
 
-// One CTA per row: merge the row's partials, decide lock / re-noise; the last CTA to finish
-// evaluates the stop rule for the whole canvas (no CTA ever waits on another).
+// One CTA per row of the n_seq canvases: merge the row's partials, decide lock / re-noise; the
+// last CTA of a canvas to finish evaluates the stop rule for that canvas (no CTA ever waits on
+// another).  A canvas that has stopped is left as it is while the others go on.
 __global__ void __launch_bounds__(256) sampler_merge_kernel(SamplerArgs p) {
   pdl_enter();
-  if (block_done(p.state + kStDone)) return;
-  if (sampler_row(p, blockIdx.x)) sampler_stop_test(p);
+  const int b = blockIdx.x / p.rows;
+  const SamplerArgs q = seq_view(p, b);
+  if (block_done(q.state + kStDone)) return;
+  if (sampler_row(q, blockIdx.x - b * p.rows)) sampler_stop_test(q);
 }
 
 // (m, S, U, a) <- merge with (m2, S2, U2, a2) in fp32 (2^x on the special-function unit); an

@@ -103,6 +103,14 @@ typedef struct dg_config {
    * 1: keep the K/V the last denoise step wrote for the canvas (the bidirectional forward of
    *    that step's input canvas), so the commit launches nothing but a copy of the ids. */
   int32_t commit_reuse_kv;
+  /* Small-batch canvases (the pages: the advantage is strongest at small-to-medium batch on one
+   * accelerator): B independent sequences decoded in lockstep, each with its own KV cache, canvas,
+   * sampler state and stop test, sharing every weight stream of a denoise step (B * T tokens per
+   * forward).  0 or 1: one sequence.  B > 1 needs a bf16 dtype, canvas % 128 == 0 and
+   * B * canvas <= 4096; all sequences hold the same committed length (equal-length prompts, blocks
+   * committed together once every canvas has stopped; a stopped canvas is frozen meanwhile), and
+   * sequence b draws its Philox stream with key seed + b. */
+  int32_t batch;
 } dg_config;
 
 /* Per-layer weights, all device pointers, dtype = config dtype unless noted (bf16 for
@@ -168,13 +176,14 @@ DG_API int dg_kv_truncate(dg_ctx* ctx, int32_t length);
 
 /* Causal encode ([canvas] step 1, [arch] prefill): run every layer over ids[0..n) at
  * positions P..P+n-1 with a causal mask and append their K/V to the cache (P += n).
- * d_ids: int32 [n], each in [0, V).  Processed in chunks of `canvas` tokens.
+ * d_ids: int32 [n], each in [0, V); a batched context takes [batch, n], row b into sequence b's
+ * cache.  Processed in passes of prefill_chunk (else canvas) tokens.
  * DG_ERR_CAPACITY if P + n + canvas > kv_capacity (room for the next canvas is kept). */
 DG_API int dg_kv_append(dg_ctx* ctx, const int32_t* d_ids, int32_t n, void* stream);
 
 /* Fill the canvas with ids uniform over [0, V) ([canvas] step 2): Philox4x32-10 with
  * counter (position, 0, block, 0) and key (seed lo32, seed hi32); id = floor(r0 V / 2^32).
- * Resets the decode state words (done, steps, stop step). */
+ * Resets the decode state words (done, steps, stop step).  Batched: canvas b uses key seed + b. */
 DG_API int dg_canvas_init(dg_ctx* ctx, uint64_t seed, uint32_t block, void* stream);
 
 /* Start the current block's denoising over ([canvas] step 4: after a commit the next canvas starts
@@ -201,13 +210,14 @@ DG_API int dg_denoise_step(dg_ctx* ctx, uint32_t step, void* stream);
 DG_API int dg_sample_update(dg_ctx* ctx, uint32_t step, void* stream);
 
 /* Commit ([canvas] step 4, [arch]): copy the stop step's argmax block to d_out_ids (int32
- * [T], may be NULL), the decode state words to d_state (int32 [DG_STATE_WORDS], may be
- * NULL), then causally re-encode the block into the cache (P += T), or with commit_reuse_kv
+ * [T], batched [batch * T], may be NULL), the decode state words to d_state (int32
+ * [DG_STATE_WORDS], batched [batch, DG_STATE_WORDS], may be NULL), then causally re-encode the block into the cache (P += T), or with commit_reuse_kv
  * keep the canvas K/V of the last denoise step in place (P += T). */
 DG_API int dg_commit_block(dg_ctx* ctx, int32_t* d_out_ids, int32_t* d_state, void* stream);
 
 /* Device buffers of the context (for inspection; owned by the caller's scratch):
- * canvas int32 [T], argmax int32 [T], entropy fp32 [T], conf fp32 [T], state int32 [16]. */
+ * canvas int32 [T], argmax int32 [T], entropy fp32 [T], conf fp32 [T], state int32 [16]; a
+ * batched context has [batch * T] (sequence-major) and state [batch, 16]. */
 DG_API int dg_get_buffers(const dg_ctx* ctx, int32_t** canvas, int32_t** argmax, float** entropy,
                    float** conf, int32_t** state);
 

@@ -218,3 +218,16 @@ def decode(cfg, weights, prompt_ids, n_blocks, seed, fixed_steps=None, commit="r
         blocks.append(res)
     out = np.concatenate([b["committed"] for b in blocks]) if blocks else np.zeros(0, np.int64)
     return out, blocks, cache
+
+
+def decode_batch(cfg, weights, prompts, n_blocks, seed, fixed_steps=None, commit="reencode"):
+    """Small-batch canvases: B sequences decoded in lockstep, one canvas each per denoise step.
+
+    The pages only say the method's advantage is strongest at small-to-medium batch on one
+    accelerator; the plainest reading keeps the sequences independent: sequence b is the
+    single-sequence decode of prompts[b] whose Philox stream has key seed + b.  Lockstep (every
+    canvas commits once all have stopped; a stopped canvas is frozen meanwhile) changes no
+    sequence's result, because a stopped canvas's committed block is fixed at its stop step.
+    Returns a list of decode() results."""
+    return [decode(cfg, weights, np.asarray(p), n_blocks, seed + b, fixed_steps, commit)
+            for b, p in enumerate(prompts)]

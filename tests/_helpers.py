@@ -80,23 +80,31 @@ def router_gaps(ocfg, ow, ids, pos, cache, causal=True):
     return np.array(out)
 
 
+# Router near-ties.  Teacher-forced (the GPU's own attention output feeds both sides' MoE half):
+# the two sides' router inputs differ only by the re-rounding of the RMSNorm output, margins
+# below 1e-3 may flip.  Untethered forward passes (prefill, commit, denoise over the GPU's own
+# activations): the bf16 storage of the attention output and of the normed hidden state lets the
+# router input differ by up to half a bf16 step per element, i.e. a router-logit change of
+# standard deviation 2^-9 / sqrt(3) * ||w_r|| ~ 5e-4 for the test models (||w_r|| = 0.02 sqrt(512));
+# margins below ten of those, 5e-3, may flip.
 NEAR_TIE = 1e-3
+NEAR_TIE_FORWARD = 5e-3
 
 
-def kv_tokens_close(got, ref, gaps, layer, rtol):
+def kv_tokens_close(got, ref, gaps, layer, rtol, near_tie=NEAR_TIE_FORWARD):
     """Per-token parity of a K (or V) slice [H, n, hd] of `layer`.
 
     In these two-layer models a token's layer-1 K/V depend on the layer-0 K/V of the tokens it
-    attends to (functions of their embeddings only) and on its own layer-0 MoE routing.  bf16
-    storage moves router logits by about 1e-4, so where the oracle's top-k margin of that token
-    at an earlier layer is below NEAR_TIE the GPU may legitimately route it to another expert and
-    its K/V differ.  Every other token must be within rtol.  Returns (ok, the offending tokens
-    with their smallest earlier margin, count of excused tokens that differ)."""
+    attends to (functions of their embeddings only) and on its own layer-0 MoE routing.  Where the
+    oracle's top-k margin of that token at an earlier layer is below `near_tie` the GPU may
+    legitimately route it to another expert and its K/V differ.  Every other token must be within
+    rtol.  Returns (ok, the offending tokens with their smallest earlier margin, count of excused
+    tokens that differ)."""
     got = np.asarray(got)
     ref = np.asarray(ref)
     n = ref.shape[1]
     good = np.array([rel_close(got[:, j], ref[:, j], rtol)[0] for j in range(n)])
     earlier = gaps[:layer].min(axis=0) if layer else np.full(n, np.inf)
-    excused = earlier < NEAR_TIE
+    excused = earlier < near_tie
     bad = np.nonzero(~good & ~excused)[0]
     return bad.size == 0, [(int(j), float(earlier[j])) for j in bad[:8]], int((~good & excused).sum())

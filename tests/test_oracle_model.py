@@ -150,3 +150,18 @@ def test_reuse_kv_commit_keeps_the_last_step_canvas_kv():
         assert not np.allclose(cache.k[l][:, 6:], reenc.k[l][:, 6:])  # not the re-encode
     with pytest.raises(ValueError):
         om.decode(cfg, w, np.arange(6), 1, seed=4, fixed_steps=2, commit="other")
+
+
+def test_decode_batch_is_independent_sequences():
+    cfg = _cfg()
+    w = _weights(cfg, std=0.2)
+    prompts = np.random.default_rng(7).integers(0, cfg.vocab, (3, 6))
+    res = om.decode_batch(cfg, w, prompts, 1, seed=40, fixed_steps=2)
+    assert len(res) == 3
+    for b in range(3):
+        ids, blocks, _ = om.decode(cfg, w, prompts[b], 1, seed=40 + b, fixed_steps=2)
+        assert np.array_equal(res[b][0], ids)
+        assert np.array_equal(blocks[0]["steps"][0]["canvas_in"],
+                              smp.canvas_init(40 + b, 0, cfg.canvas, cfg.vocab))
+    # different keys give different canvases
+    assert not np.array_equal(res[0][1][0]["steps"][0]["canvas_in"], res[1][1][0]["steps"][0]["canvas_in"])
