@@ -384,12 +384,13 @@ def run_ours(args, rank, world, local_rank):
     # shapes) and the shared expert's, which rides in the same launch, plus tokens in and out;
     # e4m3: one byte per weight and per quantised activation, plus the fp32 row scales
     wb = 1 if f8 else 2
+    scale_b = 4 if f8 else 0  # one fp32 scale per weight row and per quantised token row
     algo = {
         "expert_gate_up": (e * 2 * h + 2 * hs) * d * wb + (slots + CANVAS) * d * wb
                           + slots * h * 2 + CANVAS * hs * 2
-                          + (f8 and (e * 2 * h + 2 * hs + slots + CANVAS) * 4),
+                          + (e * 2 * h + 2 * hs + slots + CANVAS) * scale_b,
         "expert_down": (e * h + hs) * d * wb + slots * h * wb + CANVAS * hs * wb
-                       + (slots + CANVAS) * d * 4 + (f8 and (e * d + d + slots + CANVAS) * 4),
+                       + (slots + CANVAS) * d * 4 + (e * d + d + slots + CANVAS) * scale_b,
         "lm_head": shape["vocab"] * d * 2 + CANVAS * d * 2 + CANVAS * (shape["vocab"] // 256) * 16,
     }
     # DRAM bytes (read + write) of one launch from the ncu capture summarised in profiles/
