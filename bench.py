@@ -44,6 +44,7 @@ WORKLOAD = ("full block decode: 30-layer MoE decoder (d 2816, 16/8 heads x 128, 
             "top-8 x 704 + shared 2112, vocab 262144, bf16, random init), 4096-token prompt "
             "prefilled in one pass, 4 canvases x 256 tokens x 16 fixed denoise steps")
 WORKLOAD_E4M3 = WORKLOAD.replace("bf16, random init", "bf16 with e4m3 experts, random init")
+WORKLOAD_NVFP4 = WORKLOAD.replace("bf16, random init", "bf16 with NVFP4 experts, random init")
 
 
 def parse():
@@ -55,7 +56,7 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--roofline-kernel", default="expert_gate_up")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--experts", choices=["bf16", "e4m3"], default="bf16",
+    ap.add_argument("--experts", choices=["bf16", "e4m3", "nvfp4"], default="bf16",
                     help="expert weight format of the decode model")
     ap.add_argument("--profile", choices=["decode_step", "decode_step_small", "decode_step_e4m3",
                                           "moe", "moe_e4m3", "attention", "sampler"],
@@ -345,12 +346,13 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     shape = SHAPES["a4b"]
     cap = PROMPT + BLOCKS * CANVAS + CANVAS
-    f8 = args.experts == "e4m3"
-    cfg = make_config(shape, kv_capacity=cap, fixed_steps=FIXED_STEPS, prefill_chunk=PREFILL_CHUNK,
-                      experts=args.experts)
+    f8 = args.experts != "bf16"  # quantised experts (e4m3 or NVFP4)
+    f4 = args.experts == "nvfp4"
+    cfg = make_config(shape, kv_capacity=cap, fixed_steps=FIXED_STEPS,
+                      prefill_chunk=1024 if f4 else PREFILL_CHUNK, experts=args.experts)
     weights = model_weights("a4b", seed=1000 + rank, device=dev)
     if f8:  # the bf16 expert matrices are dropped once quantised
-        weights = quantize_experts(weights)
+        weights = quantize_experts(weights, fmt=args.experts)
         torch.cuda.synchronize()
         torch.cuda.empty_cache()
     model = DiffusionModel(cfg, weights, device=dev)
@@ -429,19 +431,21 @@ def run_ours(args, rank, world, local_rank):
     # algorithmic bytes per launch: every routed expert's weights (all 128 are routed at these
     # shapes) and the shared expert's, which rides in the same launch, plus tokens in and out;
     # e4m3: one byte per weight and per quantised activation, plus the fp32 row scales
-    wb = 1 if f8 else 2
+    wb = 0.5625 if f4 else 1 if f8 else 2  # NVFP4: half a byte + one e4m3 scale per 16
     scale_b = 4 if f8 else 0  # one fp32 scale per weight row and per quantised token row
     algo = {
-        "expert_gate_up": (e * 2 * h + 2 * hs) * d * wb + (slots + CANVAS) * d * wb
+        "expert_gate_up": int((e * 2 * h + 2 * hs) * d * wb + (slots + CANVAS) * d * wb)
                           + slots * h * 2 + CANVAS * hs * 2
                           + (e * 2 * h + 2 * hs + slots + CANVAS) * scale_b,
-        "expert_down": (e * h + hs) * d * wb + slots * h * wb + CANVAS * hs * wb
+        "expert_down": int((e * h + hs) * d * wb + slots * h * wb + CANVAS * hs * wb)
                        + (slots + CANVAS) * d * 4 + (e * d + d + slots + CANVAS) * scale_b,
         "lm_head": shape["vocab"] * d * 2 + CANVAS * d * 2 + CANVAS * (shape["vocab"] // 256) * 16,
     }
     # DRAM bytes (read + write) of one launch from the ncu captures summarised in profiles/
-    # (dram__bytes_read.sum + dram__bytes_write.sum of the standalone MoE operator's launches)
-    traffic = ({"expert_gate_up": 532844544 + 5702400, "expert_down": 286637312 + 9329920} if f8
+    # (dram__bytes_read.sum + dram__bytes_write.sum of the standalone MoE operator's launches);
+    # None for the NVFP4 kernels until they are captured
+    traffic = ({} if f4 else
+               {"expert_gate_up": 532844544 + 5702400, "expert_down": 286637312 + 9329920} if f8
                else {"expert_gate_up": 1063746000 + 4687104, "expert_down": 523752000 + 6922496})
     roof = None
     if args.roofline_kernel in algo and rec:
@@ -588,13 +592,15 @@ def run_ours(args, rank, world, local_rank):
         out = dict(metric="committed canvas tokens/s", value=round(value, 2), unit="tok/s",
                    n_gpus=world, steps=args.steps, warmup=args.warmup,
                    ms_per_step=round(ms_max / args.steps, 3), higher_is_better=True,
-                   scaling="weak", vs_baseline=None, dtype="bf16+e4m3" if f8 else "bf16",
+                   scaling="weak", vs_baseline=None,
+                   dtype={"bf16": "bf16", "e4m3": "bf16+e4m3", "nvfp4": "bf16+nvfp4"}[args.experts],
                    data="synthetic",
-                   config=dict(workload=WORKLOAD_E4M3 if f8 else WORKLOAD, global_batch=world,
+                   config=dict(workload={"bf16": WORKLOAD, "e4m3": WORKLOAD_E4M3,
+                                         "nvfp4": WORKLOAD_NVFP4}[args.experts], global_batch=world,
                                seq_len=PROMPT + BLOCKS * CANVAS,
                                parallelism=f"replicas x{world}",
                                l2="inputs larger than L2: ~%d GB of weights streamed per denoise "
-                                  "step" % (25 if f8 else 49)),
+                                  "step" % (15 if f4 else 25 if f8 else 49)),
                    us_per_denoise_step=round(us_step, 1), prefill_ms=round(prefill_ms, 2),
                    roofline=roof, step_roofline=step_roof, adaptive_stop=adaptive,
                    long_context=long_ctx, small_batch=batched,

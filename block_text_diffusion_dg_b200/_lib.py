@@ -8,7 +8,7 @@ LIB_PATH = os.path.join(_HERE, "libdg.so")
 DG_OK = 0
 DG_ERR = {-1: "DG_ERR_INVALID_ARG", -2: "DG_ERR_CAPACITY", -3: "DG_ERR_CUDA",
           -4: "DG_ERR_TIMEOUT", -5: "DG_ERR_UNSUPPORTED"}
-DTYPE_BF16, DTYPE_FP32, DTYPE_BF16_E4M3 = 0, 1, 2
+DTYPE_BF16, DTYPE_FP32, DTYPE_BF16_E4M3, DTYPE_BF16_NVFP4 = 0, 1, 2, 3
 STATE_DONE, STATE_STOP_STEP, STATE_WOULD_STOP, STATE_STEPS_RUN, STATE_LOCKED, STATE_ERROR = range(6)
 STATE_WORDS = 16
 KERNEL_KINDS = dict(expert_gate_up=0, expert_down=1, attention=2, lm_head=3, qkv=4,
@@ -34,7 +34,8 @@ class Config(C.Structure):
 class LayerWeights(C.Structure):
     _fields_ = [(n, C.c_void_p) for n in
                 ("attn_norm", "wqkv", "wo", "ffn_norm", "wr", "w_gu", "w_d", "ws_gu", "ws_d",
-                 "w_gu_scale", "w_d_scale", "ws_gu_scale", "ws_d_scale")]
+                 "w_gu_scale", "w_d_scale", "ws_gu_scale", "ws_d_scale",
+                 "w_gu_sf", "w_d_sf", "ws_gu_sf", "ws_d_sf")]
 
 
 class Weights(C.Structure):
@@ -75,6 +76,8 @@ _PROTOS = {
     "dg_moe_ffn_e4m3": (C.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I,
                                   _I, _I, _I, _I, _I, _P, _SZ, _P]),
     "dg_quantize_e4m3": (C.c_int, [_P, _I, _I, C.c_int64, _P, C.c_int64, _P, _P]),
+    "dg_quantize_nvfp4": (C.c_int, [_P, _I, _I, C.c_int64, _P, C.c_int64, _P, _P, _P]),
+    "dg_moe_ffn_nvfp4": (C.c_int, [_P] * 19 + [_I] * 6 + [_P, _SZ, _P]),
     "dg_debug_logits": (C.c_int, [_P, _P, _P]),
     "dg_debug_layer": (C.c_int, [_P, _I, _P, _P, _I, _I, _P]),
     "dg_debug_hidden": (C.c_int, [_P, C.POINTER(_P)]),

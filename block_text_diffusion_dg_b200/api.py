@@ -44,8 +44,8 @@ def make_config(shape, *, kv_capacity, fixed_steps=16, max_steps=48, tau=0.9, h_
     if commit not in ("reencode", "reuse_kv"):
         raise ValueError("commit must be 'reencode' or 'reuse_kv'")
     s = shape
-    if experts not in ("bf16", "e4m3"):
-        raise ValueError("experts must be 'bf16' or 'e4m3'")
+    if experts not in ("bf16", "e4m3", "nvfp4"):
+        raise ValueError("experts must be 'bf16', 'e4m3' or 'nvfp4'")
     rules = {"confidence": 0, "entropy_bound": 1}
     if lock_rule not in rules:
         raise ValueError("lock_rule must be 'confidence' or 'entropy_bound'")
@@ -54,7 +54,8 @@ def make_config(shape, *, kv_capacity, fixed_steps=16, max_steps=48, tau=0.9, h_
             raise ValueError("the all-fp32 model has no e4m3 expert format")
         dtype = L.DTYPE_FP32
     else:
-        dtype = L.DTYPE_BF16_E4M3 if experts == "e4m3" else L.DTYPE_BF16
+        dtype = {"bf16": L.DTYPE_BF16, "e4m3": L.DTYPE_BF16_E4M3,
+                 "nvfp4": L.DTYPE_BF16_NVFP4}[experts]
     return L.Config(
         n_layers=s["n_layers"], d_model=s["d_model"], n_heads=s["n_heads"],
         n_kv_heads=s["n_kv_heads"], head_dim=s["head_dim"], n_experts=s["n_experts"],
@@ -89,7 +90,8 @@ class DiffusionModel:
         layers = (L.LayerWeights * cfg.n_layers)()
         for i, lw in enumerate(weights["layers"]):
             for name in ("attn_norm", "wqkv", "wo", "ffn_norm", "wr", "w_gu", "w_d", "ws_gu", "ws_d",
-                         "w_gu_scale", "w_d_scale", "ws_gu_scale", "ws_d_scale"):
+                         "w_gu_scale", "w_d_scale", "ws_gu_scale", "ws_d_scale",
+                         "w_gu_sf", "w_d_sf", "ws_gu_sf", "ws_d_sf"):
                 t = lw.get(name)
                 _need_cuda(t, name)
                 setattr(layers[i], name, None if t is None else t.data_ptr())
@@ -356,17 +358,43 @@ def quantize_e4m3(x, pitch=None, stream=None):
     return codes, scales
 
 
-def quantize_experts(weights, stream=None):
-    """A copy of a bf16 weight dict with every layer's expert matrices (routed and shared) in
-    the e4m3 format: w_gu, w_d, ws_gu, ws_d become codes (rows at e4m3_pitch) and *_scale their
-    row scales."""
+def quantize_nvfp4(x, stream=None):
+    """NVFP4 quantisation of a bf16 tensor [..., cols] (cols % 64 == 0), rows flattened.
+
+    Returns (codes uint8 [..., e4m3_pitch(cols / 2)] with two e2m1 codes per byte, block-scale
+    atoms uint8 [ceil(rows / 128), 4 * ceil(cols / 256), 512], row scales fp32 [...]) as
+    dg_quantize_nvfp4 lays them out.
+    """
+    _need_cuda(x, "x", torch.bfloat16)
+    cols = x.shape[-1]
+    rows = x.numel() // max(cols, 1)
+    pitch = e4m3_pitch(cols // 2)
+    codes = torch.empty(x.shape[:-1] + (pitch,), dtype=torch.uint8, device=x.device)
+    sf = torch.empty(((rows + 127) // 128, 4 * ((cols + 255) // 256), 512), dtype=torch.uint8,
+                     device=x.device)
+    scales = torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device)
+    check(lib().dg_quantize_nvfp4(_ptr(x), rows, cols, cols, _ptr(codes), pitch, _ptr(sf),
+                                  _ptr(scales), _stream(stream)), "dg_quantize_nvfp4")
+    return codes, sf, scales
+
+
+def quantize_experts(weights, fmt="e4m3", stream=None):
+    """A copy of a bf16 weight dict with every layer's expert matrices (routed and shared) in the
+    e4m3 format (w_gu, w_d, ws_gu, ws_d become codes at e4m3_pitch, *_scale their row scales) or
+    the NVFP4 format (codes, *_scale row scales and *_sf block-scale atoms)."""
+    if fmt not in ("e4m3", "nvfp4"):
+        raise ValueError("fmt must be 'e4m3' or 'nvfp4'")
     out = dict(weights)
     out["layers"] = []
     for lw in weights["layers"]:
         q = dict(lw)
         for name in ("w_gu", "w_d", "ws_gu", "ws_d"):
-            if lw.get(name) is not None:
+            if lw.get(name) is None:
+                continue
+            if fmt == "e4m3":
                 q[name], q[name + "_scale"] = quantize_e4m3(lw[name], stream)
+            else:
+                q[name], q[name + "_sf"], q[name + "_scale"] = quantize_nvfp4(lw[name], stream)
         out["layers"].append(q)
     return out
 
@@ -400,4 +428,33 @@ def moe_ffn_e4m3(x, wr, w_gu, w_gu_scale, w_d, w_d_scale, top_k, ws_gu=None, ws_
                                 _ptr(ws_d), _ptr(ws_d_scale), _ptr(out), _ptr(ids), _ptr(weights),
                                 _ptr(router_logits), t, d, e, top_k, h, hs, _ptr(workspace),
                                 workspace.numel(), _stream(stream)), "dg_moe_ffn_e4m3")
+    return out
+
+
+def moe_ffn_nvfp4(x, wr, w_gu, w_d, top_k, ws_gu=None, ws_d=None, residual=None, workspace=None,
+                  out=None, ids=None, weights=None, router_logits=None, stream=None):
+    """moe_ffn with NVFP4 experts: each of w_gu, w_d, ws_gu, ws_d is the (codes, atoms, row
+    scales) triple quantize_nvfp4 returns for the stacked matrix."""
+    _need_cuda(x, "x", torch.bfloat16)
+    _need_cuda(wr, "wr", torch.bfloat16)
+    t, d = x.shape
+    e = wr.shape[0]
+    h = w_gu[0].shape[-2] // 2
+    hs = 0 if ws_gu is None else ws_gu[0].shape[-2] // 2
+    trip = [w_gu, w_d, ws_gu, ws_d]
+    ptrs = []
+    for tr in trip:
+        if tr is None:
+            ptrs += [None, None, None]
+        else:
+            codes, sf, scales = tr
+            ptrs += [codes, scales, sf]
+    if workspace is None:
+        workspace = moe_workspace(t, d, e, top_k, h, hs, x.device)
+    if out is None:
+        out = torch.empty(t, d, dtype=torch.float32, device=x.device)
+    check(lib().dg_moe_ffn_nvfp4(_ptr(x), _ptr(residual), _ptr(wr), *[_ptr(p) for p in ptrs],
+                                 _ptr(out), _ptr(ids), _ptr(weights), _ptr(router_logits), t, d, e,
+                                 top_k, h, hs, _ptr(workspace), workspace.numel(), _stream(stream)),
+          "dg_moe_ffn_nvfp4")
     return out

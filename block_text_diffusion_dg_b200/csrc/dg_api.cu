@@ -18,6 +18,7 @@
 #include "attention.cuh"
 #include "dg_common.cuh"
 #include "fp32_path.cuh"
+#include "fp4.cuh"
 #include "fp8.cuh"
 #include "gemm.cuh"
 #include "gemm_cluster.cuh"
@@ -215,17 +216,18 @@ constexpr int kRouterChunk = 64;  // tokens per router cluster
 constexpr int kPrefetchExperts = 4;  // routed chunks whose expert weights the gather prefetches
 
 // ta2/tb2 are read only by items of the alternate group (p.alt_group >= 0).
-template <int MAXN, int STAGES, int EPI, bool F8 = false>
+template <int MAXN, int STAGES, int EPI, int FMT = 0>
 int launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, int grid,
                 cudaStream_t st, int kind = -1, const CUtensorMap* ta2 = nullptr,
                 const CUtensorMap* tb2 = nullptr) {
-  auto k = gemm_swapab_kernel<MAXN, STAGES, EPI, F8>;
-  constexpr int smem = GemmCfg<MAXN, STAGES>::kSmemBytes;
+  auto k = gemm_swapab_kernel<MAXN, STAGES, EPI, FMT>;
+  constexpr int smem = GemmCfg<MAXN, STAGES, FMT>::kSmemBytes;
   if (p.alt_group >= 0 && (!ta2 || !tb2))
     return fail(DG_ERR_INVALID_ARG, "alternate group without its tensor maps");
   DG_TRY(set_smem(k, smem));
   prof_before(kind, st);
-  DG_TRY(launch_pdl(k, dim3(grid), dim3(GemmCfg<MAXN, STAGES>::kThreads), smem, st, ta, tb, ta2 ? *ta2 : ta, tb2 ? *tb2 : tb, p));
+  DG_TRY(launch_pdl(k, dim3(grid), dim3(GemmCfg<MAXN, STAGES, FMT>::kThreads), smem, st, ta, tb,
+                    ta2 ? *ta2 : ta, tb2 ? *tb2 : tb, p));
   DG_LAUNCHED();
   prof_after(kind, st);
   return DG_OK;
@@ -281,14 +283,21 @@ int clu_splits(int tiles, int kb_total, int sms) {
   return std::max(1, std::min({kCluMaxSplits, kb_total, sms / std::max(1, tiles)}));
 }
 
-// Grouped expert GEMM with the token-chunk width the pass needs (see group_wide).
-template <int EPI, bool F8>
+// Grouped expert GEMM with the token-chunk width the pass needs (see group_wide).  NVFP4 runs
+// the 64-token instance only (its scale atoms are laid out per chunk of at most 128 rows).
+constexpr int kGroupFp4Stages = 7;
+template <int EPI, int FMT>
 int launch_grouped(bool wide, const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
                    int sms, cudaStream_t st, int kind, const CUtensorMap* ta2,
                    const CUtensorMap* tb2) {
-  if (wide)
-    return launch_gemm<kGroupWideN, kGroupWideStages, EPI, F8>(ta, tb, p, sms, st, kind, ta2, tb2);
-  return launch_gemm<kGroupN, kGroupStages, EPI, F8>(ta, tb, p, sms, st, kind, ta2, tb2);
+  if constexpr (FMT == 2) {
+    return launch_gemm<kGroupN, kGroupFp4Stages, EPI, FMT>(ta, tb, p, sms, st, kind, ta2, tb2);
+  } else {
+    if (wide)
+      return launch_gemm<kGroupWideN, kGroupWideStages, EPI, FMT>(ta, tb, p, sms, st, kind, ta2,
+                                                                 tb2);
+    return launch_gemm<kGroupN, kGroupStages, EPI, FMT>(ta, tb, p, sms, st, kind, ta2, tb2);
+  }
 }
 
 // The expert half of an MoE pass once the routing exists: gather the routed token rows (bf16),
@@ -298,28 +307,30 @@ int launch_grouped(bool wide, const CUtensorMap& ta, const CUtensorMap& tb, cons
 // along in both GEMMs as the alternate group.
 struct ExpertPass {
   int n, d, k, E, hid, hs;
-  bool f8;
+  int fmt;                  // expert operands: 0 bf16, 1 e4m3, 2 NVFP4
   const int32_t* perm;
   const float* topk_w;
   float* w_perm;            // [n k]: topk_w in permuted order (written by the gather)
   const int4* chunks;
   const int* n_chunks;
   const __nv_bfloat16* xn;  // normed tokens [n, d]
-  void* x_perm;             // routed rows [n k, d]: bf16, or e4m3 codes
-  float* x_perm_scale;      // e4m3: [n k]
-  void* x_sh;               // e4m3: quantised tokens [n, d] for the shared expert
+  void* x_perm;             // routed rows [n k, d]: bf16, or e4m3 / e2m1 codes
+  float* x_perm_scale;      // e4m3 / NVFP4: row scales [n k]
+  void* x_sh;               // e4m3 / NVFP4: quantised tokens [n, d] for the shared expert
   float* x_sh_scale;
   __nv_bfloat16* h;         // SiLU-GLU output per slot [n k, hid]
   __nv_bfloat16* h_sh;      // shared expert's [n, hs]
-  void* hq;                 // e4m3: codes of h, h_sh and their scales
+  void* hq;                 // e4m3 / NVFP4: codes of h, h_sh and their row scales
   float* hq_scale;
   void* hsq;
   float* hsq_scale;
+  uint8_t *x_sf, *x_sh_sf, *h_sf, *hs_sf;  // NVFP4: block-scale atoms of the token operands
   float* y_slot;
   float* y_shared;
   const void* w_gu;  // routed gate/up weights: the first chunks' experts are hinted into L2
   const void* ws_d;  // shared down weights: hinted into L2 by the gate/up GEMM's tail
   const float *w_gu_scale, *w_d_scale, *ws_gu_scale, *ws_d_scale;
+  const uint8_t *w_gu_sf, *w_d_sf, *ws_gu_sf, *ws_d_sf;  // NVFP4: weight block-scale atoms
   const CUtensorMap *tm_wgu, *tm_xperm, *tm_wsgu, *tm_xsh, *tm_wd, *tm_h, *tm_wsd, *tm_hs;
   const void* pf0;  // hinted into L2 by the down GEMM's tail
   long long pf0_bytes;
@@ -330,35 +341,79 @@ struct ExpertPass {
   bool profile;  // record under the per-kernel profiling kinds
 };
 
+// Bytes of one operand row of `cols` values in expert format fmt: bf16 rows are packed, e4m3 and
+// NVFP4 code rows are padded to 128-byte multiples.
+long long operand_row_bytes(int fmt, int cols) {
+  return fmt == 2 ? e4m3_pitch(cols / 2) : fmt == 1 ? e4m3_pitch(cols) : 2ll * cols;
+}
+
+// The routed chunk width of a pass: 256-token chunks for long passes, except NVFP4 (64 always).
+int route_chunk(int fmt, long long n_slots, int n_experts) {
+  return fmt != 2 && group_wide(n_slots, n_experts) ? kGroupWideN : kGroupN;
+}
+
+template <int EPI>
+int launch_grouped_fmt(int fmt, bool wide, const CUtensorMap& ta, const CUtensorMap& tb,
+                       const GemmParams& p, int sms, cudaStream_t st, int kind,
+                       const CUtensorMap* ta2, const CUtensorMap* tb2) {
+  if (fmt == 2) return launch_grouped<EPI, 2>(wide, ta, tb, p, sms, st, kind, ta2, tb2);
+  if (fmt == 1) return launch_grouped<EPI, 1>(wide, ta, tb, p, sms, st, kind, ta2, tb2);
+  return launch_grouped<EPI, 0>(wide, ta, tb, p, sms, st, kind, ta2, tb2);
+}
+
+// Quantise (e4m3 or NVFP4) up to two row segments: routed rows (optionally gathered by perm,
+// NVFP4 scale atoms per routed chunk) and the shared expert's token rows (atoms per token chunk).
+int launch_quant(const ExpertPass& e, const __nv_bfloat16* src0, long long ld0, const int32_t* perm,
+                 int rows0, void* dst0, float* scale0, uint8_t* sf0, const __nv_bfloat16* src1,
+                 long long ld1, int rows1, void* dst1, float* scale1, uint8_t* sf1, int cols0,
+                 int cols1, int tok_chunk, const ExpertPrefetch& pf, cudaStream_t st) {
+  const int rows = rows0 + rows1;
+  if (e.fmt == 2) {
+    QuantFp4Job j{};
+    j.seg[0] = QuantFp4Seg{src0, ld0, perm, e.k, perm ? e.topk_w : nullptr, perm ? e.w_perm : nullptr,
+                           rows0, cols0, static_cast<uint8_t*>(dst0), operand_row_bytes(2, cols0),
+                           sf0, scale0, e.chunks, e.n_chunks, 0};
+    j.seg[1] = QuantFp4Seg{src1, ld1, nullptr, 1, nullptr, nullptr, rows1, cols1,
+                           static_cast<uint8_t*>(dst1), operand_row_bytes(2, cols1), sf1, scale1,
+                           nullptr, nullptr, tok_chunk};
+    j.n_seg = rows1 > 0 ? 2 : 1;
+    j.pf = pf;
+    DG_TRY(launch_pdl(quant_fp4_rows_kernel, dim3(cdiv(rows, 8)), dim3(256), 0, st, j, e.done));
+  } else {
+    QuantJob j{};
+    j.seg[0] = QuantSeg{src0, ld0, perm, e.k, perm ? e.topk_w : nullptr, perm ? e.w_perm : nullptr,
+                        rows0, cols0, static_cast<uint8_t*>(dst0), operand_row_bytes(1, cols0),
+                        scale0};
+    j.seg[1] = QuantSeg{src1, ld1, nullptr, 1, nullptr, nullptr, rows1, cols1,
+                        static_cast<uint8_t*>(dst1), operand_row_bytes(1, cols1), scale1};
+    j.n_seg = rows1 > 0 ? 2 : 1;
+    j.pf = pf;
+    DG_TRY(launch_pdl(quant_rows_kernel, dim3(cdiv(rows, 8)), dim3(256), 0, st, j, e.done));
+  }
+  DG_LAUNCHED();
+  return DG_OK;
+}
+
 int launch_experts(const ExpertPass& e, int sms, cudaStream_t st) {
   const int n_slots = e.n * e.k;
   const bool shared = e.hs > 0;
-  const bool wide = group_wide(n_slots, e.E);
-  const int nch = wide ? kGroupWideN : kGroupN;
-  const int kel = e.f8 ? 128 : 64;  // elements per 128-byte K slab
-  // bytes per operand row: bf16 rows are packed, e4m3 rows padded to 128-byte multiples
-  const long long row_d = e.f8 ? e4m3_pitch(e.d) : 2ll * e.d;
-  const long long row_h = e.f8 ? e4m3_pitch(e.hid) : 2ll * e.hid;
-  const long long row_hs = e.f8 ? e4m3_pitch(e.hs) : 2ll * e.hs;
+  const int nch = route_chunk(e.fmt, n_slots, e.E);
+  const bool wide = nch == kGroupWideN;
+  const int slab = 64 << e.fmt;  // K elements per 128-byte slab: 64 bf16, 128 e4m3, 256 e2m1
+  const long long row_d = operand_row_bytes(e.fmt, e.d);
+  const long long row_hs = operand_row_bytes(e.fmt, e.hs);
   const int kind_g = e.profile ? DG_KERNEL_GATHER : -1;
   const ExpertPrefetch epf{e.chunks, e.n_chunks, kPrefetchExperts, e.w_gu, 2ll * e.hid * row_d};
   prof_before(kind_g, st);
-  if (e.f8) {
-    QuantJob j{};
-    j.seg[0] = QuantSeg{e.xn, e.d, e.perm, e.k, e.topk_w, e.w_perm, n_slots, e.d,
-                        static_cast<uint8_t*>(e.x_perm), row_d, e.x_perm_scale};
-    j.seg[1] = QuantSeg{e.xn, e.d, nullptr, 1, nullptr, nullptr, e.n, e.d,
-                        static_cast<uint8_t*>(e.x_sh), row_d, e.x_sh_scale};
-    j.n_seg = shared ? 2 : 1;
-    j.pf = epf;
-    DG_TRY(launch_pdl(quant_rows_kernel, dim3(cdiv(n_slots + (shared ? e.n : 0), 8)), dim3(256),
-                      0, st, j, e.done));
+  if (e.fmt != 0) {
+    DG_TRY(launch_quant(e, e.xn, e.d, e.perm, n_slots, e.x_perm, e.x_perm_scale, e.x_sf, e.xn, e.d,
+                        shared ? e.n : 0, e.x_sh, e.x_sh_scale, e.x_sh_sf, e.d, e.d, nch, epf, st));
   } else {
     DG_TRY(launch_pdl(gather_rows_kernel, dim3(cdiv(n_slots, 4)), dim3(256), 0, st, e.xn, e.perm,
                       e.k, e.d, n_slots, static_cast<__nv_bfloat16*>(e.x_perm), e.topk_w,
                       e.w_perm, epf, e.done));
+    DG_LAUNCHED();
   }
-  DG_LAUNCHED();
   prof_after(kind_g, st);
 
   GemmParams p{};
@@ -370,12 +425,12 @@ int launch_experts(const ExpertPass& e, int sms, cudaStream_t st) {
   p.alt_chunks = cdiv(e.n, nch);
   p.alt_tokens = e.n;
   p.a_rows_per_group = 2 * e.hid;
-  p.kb_total = cdiv(e.d, kel);
+  p.kb_total = cdiv(e.d, slab);
   p.m_valid = 2 * e.hid;
   p.out_bf16 = e.h;
   p.ld_out = e.hid;
   p.alt_group = shared ? e.E : -1;
-  p.alt_kb_total = cdiv(e.d, kel);
+  p.alt_kb_total = cdiv(e.d, slab);
   p.alt_m_valid = 2 * e.hs;
   p.alt_out_bf16 = e.h_sh;
   p.alt_ld_out = e.hs;
@@ -383,6 +438,10 @@ int launch_experts(const ExpertPass& e, int sms, cudaStream_t st) {
   p.b_scale = e.x_perm_scale;
   p.alt_a_scale = e.ws_gu_scale;
   p.alt_b_scale = e.x_sh_scale;
+  p.a_sf = e.w_gu_sf;
+  p.b_sf = e.x_sf;
+  p.alt_a_sf = e.ws_gu_sf;
+  p.alt_b_sf = e.x_sh_sf;
   if (shared) {  // the down GEMM starts with the shared expert's items
     p.pf0 = e.ws_d;
     p.pf0_bytes = static_cast<long long>(e.d) * row_hs;
@@ -390,27 +449,16 @@ int launch_experts(const ExpertPass& e, int sms, cudaStream_t st) {
   p.err = e.err;
   p.done = e.done;
   const int kind_gu = e.profile ? DG_KERNEL_EXPERT_GATE_UP : -1;
-  const CUtensorMap* ta2 = shared ? e.tm_wsgu : nullptr;
-  const CUtensorMap* tb2 = shared ? e.tm_xsh : nullptr;
-  if (e.f8)
-    DG_TRY((launch_grouped<kEpiGluBf16, true>(wide, *e.tm_wgu, *e.tm_xperm, p, sms, st, kind_gu,
-                                              ta2, tb2)));
-  else
-    DG_TRY((launch_grouped<kEpiGluBf16, false>(wide, *e.tm_wgu, *e.tm_xperm, p, sms, st, kind_gu,
-                                               ta2, tb2)));
+  DG_TRY(launch_grouped_fmt<kEpiGluBf16>(e.fmt, wide, *e.tm_wgu, *e.tm_xperm, p, sms, st, kind_gu,
+                                         shared ? e.tm_wsgu : nullptr,
+                                         shared ? e.tm_xsh : nullptr));
 
-  if (e.f8) {
+  if (e.fmt != 0) {
     const int kind_q = e.profile ? DG_KERNEL_QUANT_H : -1;
-    QuantJob j{};
-    j.seg[0] = QuantSeg{e.h, e.hid, nullptr, 1, nullptr, nullptr, n_slots, e.hid,
-                        static_cast<uint8_t*>(e.hq), row_h, e.hq_scale};
-    j.seg[1] = QuantSeg{e.h_sh, e.hs, nullptr, 1, nullptr, nullptr, e.n, e.hs,
-                        static_cast<uint8_t*>(e.hsq), row_hs, e.hsq_scale};
-    j.n_seg = shared ? 2 : 1;
     prof_before(kind_q, st);
-    DG_TRY(launch_pdl(quant_rows_kernel, dim3(cdiv(n_slots + (shared ? e.n : 0), 8)), dim3(256),
-                      0, st, j, e.done));
-    DG_LAUNCHED();
+    DG_TRY(launch_quant(e, e.h, e.hid, nullptr, n_slots, e.hq, e.hq_scale, e.h_sf, e.h_sh, e.hs,
+                        shared ? e.n : 0, e.hsq, e.hsq_scale, e.hs_sf, e.hid, e.hs, nch,
+                        ExpertPrefetch{}, st));
     prof_after(kind_q, st);
   }
 
@@ -423,14 +471,14 @@ int launch_experts(const ExpertPass& e, int sms, cudaStream_t st) {
   q.alt_chunks = cdiv(e.n, nch);
   q.alt_tokens = e.n;
   q.a_rows_per_group = e.d;
-  q.kb_total = cdiv(e.hid, kel);
+  q.kb_total = cdiv(e.hid, slab);
   q.m_valid = e.d;
   q.out_f32 = e.y_slot;
   q.ld_out = e.d;
   q.perm = e.perm;
   q.scale = e.w_perm;
   q.alt_group = shared ? e.E : -1;
-  q.alt_kb_total = cdiv(e.hs, kel);
+  q.alt_kb_total = cdiv(e.hs, slab);
   q.alt_m_valid = e.d;
   q.alt_out_f32 = e.y_shared;
   q.alt_ld_out = e.d;
@@ -438,6 +486,10 @@ int launch_experts(const ExpertPass& e, int sms, cudaStream_t st) {
   q.b_scale = e.hq_scale;
   q.alt_a_scale = e.ws_d_scale;
   q.alt_b_scale = e.hsq_scale;
+  q.a_sf = e.w_d_sf;
+  q.b_sf = e.h_sf;
+  q.alt_a_sf = e.ws_d_sf;
+  q.alt_b_sf = e.hs_sf;
   q.pf0 = e.pf0;
   q.pf0_bytes = e.pf0_bytes;
   q.pf1 = e.pf1;
@@ -445,14 +497,9 @@ int launch_experts(const ExpertPass& e, int sms, cudaStream_t st) {
   q.err = e.err;
   q.done = e.done;
   const int kind_d = e.profile ? DG_KERNEL_EXPERT_DOWN : -1;
-  const CUtensorMap* ta3 = shared ? e.tm_wsd : nullptr;
-  const CUtensorMap* tb3 = shared ? e.tm_hs : nullptr;
-  if (e.f8)
-    DG_TRY((launch_grouped<kEpiScatterF32, true>(wide, *e.tm_wd, *e.tm_h, q, sms, st, kind_d, ta3,
-                                                 tb3)));
-  else
-    DG_TRY((launch_grouped<kEpiScatterF32, false>(wide, *e.tm_wd, *e.tm_h, q, sms, st, kind_d,
-                                                  ta3, tb3)));
+  DG_TRY(launch_grouped_fmt<kEpiScatterF32>(e.fmt, wide, *e.tm_wd, *e.tm_h, q, sms, st, kind_d,
+                                            shared ? e.tm_wsd : nullptr,
+                                            shared ? e.tm_hs : nullptr));
   return DG_OK;
 }
 
@@ -493,7 +540,8 @@ struct dg_ctx {
   float* topk_w;
   int4* chunks;  // routed token chunks of the grouped GEMMs
   void *x_perm, *h, *hs;
-  bool f8;  // e4m3 experts
+  int fmt;  // expert operands: 0 bf16, 1 e4m3, 2 NVFP4
+  uint8_t *x_sf, *x_sh_sf, *h_sf, *hs_sf;  // NVFP4 token-side scale atoms
   void *x_sh, *hq, *hsq;  // e4m3 codes: shared-expert tokens, h per slot, shared h per token
   float *x_perm_scale, *x_sh_scale, *hq_scale, *hsq_scale;
   float* w_perm;  // route weights in permuted order
@@ -555,7 +603,10 @@ int check_config(const dg_config* c) {
   if (c->lock_rule < 0 || c->lock_rule > 1 || !(c->entropy_lock >= 0.0) || c->sticky_locks < 0 ||
       c->sticky_locks > 1)
     return fail(DG_ERR_INVALID_ARG, "lock_rule must be 0 or 1, entropy_lock >= 0, sticky 0 or 1");
-  if (c->dtype == DG_DTYPE_BF16 || c->dtype == DG_DTYPE_BF16_E4M3) {
+  if (c->dtype == DG_DTYPE_BF16_NVFP4 && c->d_model % 128)
+    return fail(DG_ERR_UNSUPPORTED, "NVFP4 experts need d a multiple of 128");
+  if (c->dtype == DG_DTYPE_BF16 || c->dtype == DG_DTYPE_BF16_E4M3 ||
+      c->dtype == DG_DTYPE_BF16_NVFP4) {
     if (c->head_dim != 128) return fail(DG_ERR_UNSUPPORTED, "bf16 path needs head_dim 128");
     if (c->d_model % 64 || c->expert_hidden % 64 || c->shared_hidden % 64)
       return fail(DG_ERR_UNSUPPORTED, "bf16 path needs d, h, hs multiples of 64");
@@ -573,7 +624,7 @@ int check_config(const dg_config* c) {
 
 // Workspace plan: every buffer at a 256-byte boundary, in this order.
 struct Plan {
-  size_t off[48];
+  size_t off[56];
   size_t total;
   size_t kv;
 };
@@ -582,7 +633,8 @@ enum Buf {
   B_CANVAS, B_ARGMAX, B_PREV, B_LOCKED, B_STATE, B_TICKET, B_ERR, B_ENT, B_CONF, B_ROWH, B_X,
   B_XN, B_PART, B_Q, B_OPART, B_ML, B_O, B_RLOG, B_IDS, B_W, B_OFF, B_PERM, B_CHUNKS,
   B_NCHUNKS, B_RTICKET, B_XPERM, B_H, B_HS, B_YSLOT, B_YSH, B_LMPART, B_LOGITS, B_ROPE,
-  B_XPS, B_XSH, B_XSHS, B_HQ, B_HQS, B_HSQ, B_HSQS, B_WPERM, B_COMMIT, B_END
+  B_XPS, B_XSH, B_XSHS, B_HQ, B_HQS, B_HSQ, B_HSQS, B_WPERM, B_COMMIT, B_XSF, B_XSHSF, B_HSF,
+  B_HSSF, B_END
 };
 
 struct Derived {
@@ -624,7 +676,8 @@ Plan plan(const dg_config& c, int sms) {
   Plan p{};
   const Derived dv = derive(c, sms);
   const bool bf16 = c.dtype != DG_DTYPE_FP32;
-  const bool f8 = c.dtype == DG_DTYPE_BF16_E4M3;
+  const int fmt = c.dtype == DG_DTYPE_BF16_E4M3 ? 1 : c.dtype == DG_DTYPE_BF16_NVFP4 ? 2 : 0;
+  const bool f8 = fmt != 0;  // quantised expert operands
   // Tc: canvas positions of all sequences; per-canvas arrays are [batch][canvas]
   const size_t Tc = static_cast<size_t>(c.canvas) * n_seq(c), T = tokens_max(c), d = c.d_model,
                E = c.n_experts, k = c.top_k, es = dv.esz;
@@ -652,8 +705,9 @@ Plan plan(const dg_config& c, int sms) {
   sz[B_CHUNKS] = bf16 ? dv.max_chunks * 16 : 0;
   sz[B_NCHUNKS] = 4;
   sz[B_RTICKET] = 4;
-  const size_t dp = e4m3_pitch(c.d_model), hp = e4m3_pitch(c.expert_hidden),
-               hsp = e4m3_pitch(std::max(1, c.shared_hidden));
+  const size_t dp = operand_row_bytes(fmt, c.d_model),
+               hp = operand_row_bytes(fmt, c.expert_hidden),
+               hsp = operand_row_bytes(fmt, std::max(64, c.shared_hidden));
   sz[B_XPERM] = bf16 ? T * k * (f8 ? dp : d * es) : 0;
   sz[B_H] = bf16 ? T * k * c.expert_hidden * es : 0;
   sz[B_HS] = bf16 ? T * std::max<size_t>(1, c.shared_hidden) * es : 0;
@@ -672,6 +726,15 @@ Plan plan(const dg_config& c, int sms) {
   sz[B_HSQS] = f8 ? T * 4 : 0;
   sz[B_WPERM] = bf16 ? T * k * 4 : 0;
   sz[B_COMMIT] = Tc * 4;  // committed ids with sticky locks
+  // NVFP4: token-side scale atoms, per routed chunk (routed rows) and per 64-token chunk
+  // (the shared expert's rows), 4 * ceil(K / 256) atoms of 512 B each
+  const size_t tok_chunks = cdiv(static_cast<long long>(T), kGroupN);
+  const size_t atoms_d = 4 * cdiv(c.d_model, 256), atoms_h = 4 * cdiv(c.expert_hidden, 256),
+               atoms_hs = 4 * cdiv(std::max(64, c.shared_hidden), 256);
+  sz[B_XSF] = fmt == 2 ? dv.max_chunks * atoms_d * 512 : 0;
+  sz[B_XSHSF] = fmt == 2 ? tok_chunks * atoms_d * 512 : 0;
+  sz[B_HSF] = fmt == 2 ? dv.max_chunks * atoms_h * 512 : 0;
+  sz[B_HSSF] = fmt == 2 ? tok_chunks * atoms_hs * 512 : 0;
   size_t o = 0;
   for (int b = 0; b < B_END; ++b) {
     p.off[b] = o;
@@ -851,7 +914,7 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     a.o = static_cast<__nv_bfloat16*>(c->o);
     if (parts & 2 && g.shared_hidden > 0) {  // the shared expert's weights of this layer
       a.pf0 = w.ws_gu;
-      a.pf0_bytes = 2ll * g.shared_hidden * (c->f8 ? e4m3_pitch(d) : 2ll * d);
+      a.pf0_bytes = 2ll * g.shared_hidden * operand_row_bytes(c->fmt, d);
     }
     a.err = c->err;
     a.done = done;
@@ -888,8 +951,8 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     p.ids = c->topk_ids;
     p.wts = c->topk_w;
     p.top_k = k;
-    p.route = RouteArgs{c->topk_ids, n, k, E, group_wide(n_slots, E) ? kGroupWideN : kGroupN,
-                        c->offsets, c->perm, c->chunks, c->n_chunks};
+    p.route = RouteArgs{c->topk_ids, n, k, E, route_chunk(c->fmt, n_slots, E), c->offsets,
+                        c->perm, c->chunks, c->n_chunks};
     p.ticket = c->route_ticket;
     DG_TRY(launch_cluster<kCluRouter>(c->tm_wr[l], c->tm_xn32, p, st, DG_KERNEL_ROUTER));
   }
@@ -903,7 +966,7 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     e.E = E;
     e.hid = g.expert_hidden;
     e.hs = g.shared_hidden;
-    e.f8 = c->f8;
+    e.fmt = c->fmt;
     e.perm = c->perm;
     e.topk_w = c->topk_w;
     e.w_perm = c->w_perm;
@@ -920,6 +983,10 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     e.hq_scale = c->hq_scale;
     e.hsq = c->hsq;
     e.hsq_scale = c->hsq_scale;
+    e.x_sf = c->x_sf;
+    e.x_sh_sf = c->x_sh_sf;
+    e.h_sf = c->h_sf;
+    e.hs_sf = c->hs_sf;
     e.y_slot = c->y_slot;
     e.y_shared = c->y_shared;
     e.w_gu = w.w_gu;
@@ -928,10 +995,14 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     e.w_d_scale = w.w_d_scale;
     e.ws_gu_scale = w.ws_gu_scale;
     e.ws_d_scale = w.ws_d_scale;
+    e.w_gu_sf = static_cast<const uint8_t*>(w.w_gu_sf);
+    e.w_d_sf = static_cast<const uint8_t*>(w.w_d_sf);
+    e.ws_gu_sf = static_cast<const uint8_t*>(w.ws_gu_sf);
+    e.ws_d_sf = static_cast<const uint8_t*>(w.ws_d_sf);
     e.tm_wgu = &c->tm_wgu[l];
     e.tm_xperm = &c->tm_xperm;
     e.tm_wsgu = &c->tm_wsgu[l];
-    e.tm_xsh = c->f8 ? &c->tm_xsh : &c->tm_xn32;
+    e.tm_xsh = c->fmt != 0 ? &c->tm_xsh : &c->tm_xn32;
     e.tm_wd = &c->tm_wd[l];
     e.tm_h = &c->tm_h;
     e.tm_wsd = &c->tm_wsd[l];
@@ -1014,16 +1085,21 @@ int bind_tmaps(dg_ctx* c) {
   DG_TRY(make_tmap(&c->tm_xn32, c->xn, T, d, d, 32));
   DG_TRY(make_tmap(&c->tm_xn128, c->xn, T, d, d, 128));
   DG_TRY(make_tmap(&c->tm_o32, c->o, T, g.n_heads * hd, g.n_heads * hd, 32));
-  // expert GEMM operands: bf16, or e4m3 with rows at the 128-byte pitch
-  const int eb = c->f8 ? 1 : 2;
-  const uint64_t pd = c->f8 ? e4m3_pitch(g.d_model) : d;
-  const uint64_t ph = c->f8 ? e4m3_pitch(g.expert_hidden) : g.expert_hidden;
-  const uint64_t phs = c->f8 ? e4m3_pitch(std::max(1, g.shared_hidden)) : g.shared_hidden;
-  DG_TRY(make_tmap(&c->tm_xperm, c->x_perm, T * k, d, pd, 32, eb));
-  DG_TRY(make_tmap(&c->tm_h, c->f8 ? c->hq : c->h, T * k, g.expert_hidden, ph, 32, eb));
+  // expert GEMM operands: bf16, or e4m3 / e2m1 codes (maps over bytes: K or K / 2 columns)
+  // with rows at the 128-byte pitch
+  const bool q8 = c->fmt != 0;
+  const int eb = q8 ? 1 : 2;
+  auto mcols = [&](int kk) { return static_cast<uint64_t>(c->fmt == 2 ? kk / 2 : kk); };
+  auto mpitch = [&](int kk) {
+    return static_cast<uint64_t>(q8 ? operand_row_bytes(c->fmt, kk) : kk);
+  };
+  DG_TRY(make_tmap(&c->tm_xperm, c->x_perm, T * k, mcols(d), mpitch(d), 32, eb));
+  DG_TRY(make_tmap(&c->tm_h, q8 ? c->hq : c->h, T * k, mcols(g.expert_hidden),
+                   mpitch(g.expert_hidden), 32, eb));
   if (g.shared_hidden > 0)
-    DG_TRY(make_tmap(&c->tm_hs, c->f8 ? c->hsq : c->hs, T, g.shared_hidden, phs, 32, eb));
-  if (c->f8) DG_TRY(make_tmap(&c->tm_xsh, c->x_sh, T, d, pd, 32, 1));
+    DG_TRY(make_tmap(&c->tm_hs, q8 ? c->hsq : c->hs, T, mcols(g.shared_hidden),
+                     mpitch(g.shared_hidden), 32, eb));
+  if (q8) DG_TRY(make_tmap(&c->tm_xsh, c->x_sh, T, mcols(d), mpitch(d), 32, 1));
   DG_TRY(make_tmap(&c->tm_q, c->q, static_cast<uint64_t>(g.n_heads) * c->tq, hd, hd, 128));
   // every (sequence, layer) pair of a batched context is one more layer block of the cache
   const uint64_t kv_rows =
@@ -1046,12 +1122,14 @@ int bind_tmaps(dg_ctx* c) {
     DG_TRY(make_tmap(&c->tm_wo[l], w.wo, d, g.n_heads * hd, g.n_heads * hd, 128));
     DG_TRY(make_tmap(&c->tm_wr[l], w.wr, g.n_experts, d, d, 128));
     DG_TRY(make_tmap(&c->tm_wgu[l], w.w_gu, static_cast<uint64_t>(g.n_experts) * 2 * g.expert_hidden,
-                     d, pd, 128, eb));
-    DG_TRY(make_tmap(&c->tm_wd[l], w.w_d, static_cast<uint64_t>(g.n_experts) * d, g.expert_hidden,
-                     ph, 128, eb));
+                     mcols(d), mpitch(d), 128, eb));
+    DG_TRY(make_tmap(&c->tm_wd[l], w.w_d, static_cast<uint64_t>(g.n_experts) * d,
+                     mcols(g.expert_hidden), mpitch(g.expert_hidden), 128, eb));
     if (g.shared_hidden > 0) {
-      DG_TRY(make_tmap(&c->tm_wsgu[l], w.ws_gu, 2ull * g.shared_hidden, d, pd, 128, eb));
-      DG_TRY(make_tmap(&c->tm_wsd[l], w.ws_d, d, g.shared_hidden, phs, 128, eb));
+      DG_TRY(make_tmap(&c->tm_wsgu[l], w.ws_gu, 2ull * g.shared_hidden, mcols(d), mpitch(d), 128,
+                       eb));
+      DG_TRY(make_tmap(&c->tm_wsd[l], w.ws_d, d, mcols(g.shared_hidden), mpitch(g.shared_hidden),
+                       128, eb));
     }
   }
   return DG_OK;
@@ -1118,10 +1196,13 @@ int dg_create(const dg_config* cfg, const dg_weights* w, void* d_kv, void* d_scr
       return fail(DG_ERR_INVALID_ARG, "layer %d has a null weight", l);
     if (cfg->shared_hidden > 0 && (!lw.ws_gu || !lw.ws_d))
       return fail(DG_ERR_INVALID_ARG, "layer %d lacks shared expert weights", l);
-    if (cfg->dtype == DG_DTYPE_BF16_E4M3 &&
+    if ((cfg->dtype == DG_DTYPE_BF16_E4M3 || cfg->dtype == DG_DTYPE_BF16_NVFP4) &&
         (!lw.w_gu_scale || !lw.w_d_scale ||
          (cfg->shared_hidden > 0 && (!lw.ws_gu_scale || !lw.ws_d_scale))))
       return fail(DG_ERR_INVALID_ARG, "layer %d lacks e4m3 expert scales", l);
+    if (cfg->dtype == DG_DTYPE_BF16_NVFP4 &&
+        (!lw.w_gu_sf || !lw.w_d_sf || (cfg->shared_hidden > 0 && (!lw.ws_gu_sf || !lw.ws_d_sf))))
+      return fail(DG_ERR_INVALID_ARG, "layer %d lacks NVFP4 block-scale atoms", l);
   }
   dg_ctx* c = new dg_ctx();
   c->cfg = *cfg;
@@ -1134,7 +1215,7 @@ int dg_create(const dg_config* cfg, const dg_weights* w, void* d_kv, void* d_scr
   c->sms = num_sms();
   c->batch = n_seq(*cfg);
   c->bf16 = cfg->dtype != DG_DTYPE_FP32;
-  c->f8 = cfg->dtype == DG_DTYPE_BF16_E4M3;
+  c->fmt = cfg->dtype == DG_DTYPE_BF16_E4M3 ? 1 : cfg->dtype == DG_DTYPE_BF16_NVFP4 ? 2 : 0;
   const Derived dv = derive(*cfg, c->sms);
   c->esz = dv.esz;
   c->tq = dv.tq;
@@ -1187,6 +1268,10 @@ int dg_create(const dg_config* cfg, const dg_weights* w, void* d_kv, void* d_scr
   c->hsq_scale = reinterpret_cast<float*>(s + p.off[B_HSQS]);
   c->w_perm = reinterpret_cast<float*>(s + p.off[B_WPERM]);
   c->commit_ids = reinterpret_cast<int32_t*>(s + p.off[B_COMMIT]);
+  c->x_sf = s + p.off[B_XSF];
+  c->x_sh_sf = s + p.off[B_XSHSF];
+  c->h_sf = s + p.off[B_HSF];
+  c->hs_sf = s + p.off[B_HSSF];
   const size_t kv_half = p.kv / 2;
   c->kc = c->kv;
   c->vtc = c->kv + kv_half;
@@ -1643,7 +1728,8 @@ int dg_canvas_attention(const void* d_q, const void* d_k, const void* d_vt, void
 namespace {
 enum MoeBuf {
   M_RLOG, M_IDS, M_W, M_OFF, M_PERM, M_CHUNKS, M_WORDS, M_XPERM, M_H, M_HS, M_YSH, M_YSLOT,
-  M_XPS, M_XSH, M_XSHS, M_HQ, M_HQS, M_HSQ, M_HSQS, M_WPERM, M_END
+  M_XPS, M_XSH, M_XSHS, M_HQ, M_HQS, M_HSQ, M_HSQS, M_WPERM, M_XSF, M_XSHSF, M_HSF, M_HSSF,
+  M_END
 };
 struct MoePlan {
   size_t off[M_END];
@@ -1678,6 +1764,12 @@ MoePlan moe_plan(int t, int d, int E, int k, int hid, int hs) {
   sz[M_HSQ] = T * e4m3_pitch(static_cast<int>(hs1));  // e4m3: quantised shared h, scales
   sz[M_HSQS] = T * 4;
   sz[M_WPERM] = tk * 4;       // route weights in permuted order
+  // NVFP4 token-side scale atoms (per routed chunk, per 64-token chunk of the shared expert)
+  const size_t tok_chunks = (T + kGroupN - 1) / kGroupN;
+  sz[M_XSF] = m.chunks * 4 * cdiv(d, 256) * 512;
+  sz[M_XSHSF] = tok_chunks * 4 * cdiv(d, 256) * 512;
+  sz[M_HSF] = m.chunks * 4 * cdiv(hid, 256) * 512;
+  sz[M_HSSF] = tok_chunks * 4 * cdiv(static_cast<int>(hs1), 256) * 512;
   size_t o = 0;
   for (int i = 0; i < M_END; ++i) {
     m.off[i] = o;
@@ -1689,9 +1781,10 @@ MoePlan moe_plan(int t, int d, int E, int k, int hid, int hs) {
 
 struct MoeScales {
   const float *w_gu, *w_d, *ws_gu, *ws_d;
+  const void *w_gu_sf, *w_d_sf, *ws_gu_sf, *ws_d_sf;  // NVFP4 block-scale atoms
 };
 
-int moe_ffn_impl(bool f8, const MoeScales& sc, const void* d_x, const float* d_residual,
+int moe_ffn_impl(int fmt, const MoeScales& sc, const void* d_x, const float* d_residual,
                  const void* d_wr, const void* d_w_gu, const void* d_w_d, const void* d_ws_gu,
                  const void* d_ws_d, float* d_y, int32_t* d_ids, float* d_weights,
                  float* d_router_logits, int32_t t, int32_t d, int32_t n_experts, int32_t top_k,
@@ -1703,8 +1796,13 @@ int moe_ffn_impl(bool f8, const MoeScales& sc, const void* d_x, const float* d_r
     return fail(DG_ERR_INVALID_ARG, "null pointer argument");
   if (shared_hidden > 0 && (!d_ws_gu || !d_ws_d))
     return fail(DG_ERR_INVALID_ARG, "shared expert weights missing");
+  const bool f8 = fmt != 0;  // quantised expert operands
   if (f8 && (!sc.w_gu || !sc.w_d || (shared_hidden > 0 && (!sc.ws_gu || !sc.ws_d))))
     return fail(DG_ERR_INVALID_ARG, "e4m3 expert scales missing");
+  if (fmt == 2 && (!sc.w_gu_sf || !sc.w_d_sf ||
+                   (shared_hidden > 0 && (!sc.ws_gu_sf || !sc.ws_d_sf))))
+    return fail(DG_ERR_INVALID_ARG, "NVFP4 block-scale atoms missing");
+  if (fmt == 2 && d % 128) return fail(DG_ERR_UNSUPPORTED, "NVFP4 experts need d % 128 == 0");
   if (workspace_bytes < need) return fail(DG_ERR_CAPACITY, "MoE workspace too small");
   if (t > 4096) return fail(DG_ERR_UNSUPPORTED, "at most 4096 tokens per call");
   const MoePlan m = moe_plan(t, d, n_experts, top_k, hidden, shared_hidden);
@@ -1723,32 +1821,37 @@ int moe_ffn_impl(bool f8, const MoeScales& sc, const void* d_x, const float* d_r
   cudaStream_t st = S(stream);
   DG_CUDA(cudaMemsetAsync(err, 0, 8, st));  // error word and route ticket
   const int eb = f8 ? 1 : 2;
-  // operand row pitches (elements): e4m3 rows at the 128-byte pitch
-  const uint64_t pd = f8 ? e4m3_pitch(d) : d, ph = f8 ? e4m3_pitch(hidden) : hidden,
-                 phs = f8 ? e4m3_pitch(std::max(1, shared_hidden)) : shared_hidden;
+  // operand maps: bf16, or e4m3 / e2m1 codes over bytes (K or K / 2 columns) at 128-byte pitches
+  auto mc = [&](int kk) { return static_cast<uint64_t>(fmt == 2 ? kk / 2 : kk); };
+  auto mp = [&](int kk) { return static_cast<uint64_t>(f8 ? operand_row_bytes(fmt, kk) : kk); };
   const uint64_t tk = static_cast<uint64_t>(t) * top_k;
   CUtensorMap t_x32, t_wr, t_xp, t_wgu, t_h, t_wd, t_wsgu, t_hs, t_wsd, t_xsh;
   DG_TRY(make_tmap(&t_x32, d_x, t, d, d, 32));
   DG_TRY(make_tmap(&t_wr, d_wr, n_experts, d, d, 128));
-  DG_TRY(make_tmap(&t_xp, at(M_XPERM), tk, d, pd, 32, eb));
-  DG_TRY(make_tmap(&t_wgu, d_w_gu, static_cast<uint64_t>(n_experts) * 2 * hidden, d, pd, 128, eb));
-  DG_TRY(make_tmap(&t_h, at(f8 ? M_HQ : M_H), tk, hidden, ph, 32, eb));
-  DG_TRY(make_tmap(&t_wd, d_w_d, static_cast<uint64_t>(n_experts) * d, hidden, ph, 128, eb));
-  if (f8) DG_TRY(make_tmap(&t_xsh, at(M_XSH), t, d, pd, 32, 1));
+  DG_TRY(make_tmap(&t_xp, at(M_XPERM), tk, mc(d), mp(d), 32, eb));
+  DG_TRY(make_tmap(&t_wgu, d_w_gu, static_cast<uint64_t>(n_experts) * 2 * hidden, mc(d), mp(d),
+                   128, eb));
+  DG_TRY(make_tmap(&t_h, at(f8 ? M_HQ : M_H), tk, mc(hidden), mp(hidden), 32, eb));
+  DG_TRY(make_tmap(&t_wd, d_w_d, static_cast<uint64_t>(n_experts) * d, mc(hidden), mp(hidden),
+                   128, eb));
+  if (f8) DG_TRY(make_tmap(&t_xsh, at(M_XSH), t, mc(d), mp(d), 32, 1));
   if (shared_hidden > 0) {
-    DG_TRY(make_tmap(&t_wsgu, d_ws_gu, 2ull * shared_hidden, d, pd, 128, eb));
-    DG_TRY(make_tmap(&t_hs, at(f8 ? M_HSQ : M_HS), t, shared_hidden, phs, 32, eb));
-    DG_TRY(make_tmap(&t_wsd, d_ws_d, d, shared_hidden, phs, 128, eb));
+    DG_TRY(make_tmap(&t_wsgu, d_ws_gu, 2ull * shared_hidden, mc(d), mp(d), 128, eb));
+    DG_TRY(make_tmap(&t_hs, at(f8 ? M_HSQ : M_HS), t, mc(shared_hidden), mp(shared_hidden), 32,
+                     eb));
+    DG_TRY(make_tmap(&t_wsd, d_ws_d, d, mc(shared_hidden), mp(shared_hidden), 128, eb));
   }
+  if (fmt == 2)  // pad atoms must read as zero scales
+    DG_CUDA(cudaMemsetAsync(at(M_XSF), 0, m.total - m.off[M_XSF], st));  // the last 4 buffers
   // router
   CluParams pr = clu_params(n_experts, t, d / 64, m.split_r, err, nullptr, kRouterChunk);
   pr.router_logits = d_router_logits ? d_router_logits : rlog;
   pr.ids = ids;
   pr.wts = wts;
   pr.top_k = top_k;
-  const bool wide = group_wide(static_cast<long long>(t) * top_k, n_experts);
-  pr.route = RouteArgs{ids, t, top_k, n_experts, wide ? kGroupWideN : kGroupN, offs, perm, chunks,
-                       icnt};
+  pr.route = RouteArgs{ids, t, top_k, n_experts,
+                       route_chunk(fmt, static_cast<long long>(t) * top_k, n_experts), offs,
+                       perm, chunks, icnt};
   pr.ticket = route_ticket;
   DG_TRY(launch_cluster<kCluRouter>(t_wr, t_x32, pr, st, -1));
   ExpertPass e{};
@@ -1758,7 +1861,7 @@ int moe_ffn_impl(bool f8, const MoeScales& sc, const void* d_x, const float* d_r
   e.E = n_experts;
   e.hid = hidden;
   e.hs = shared_hidden;
-  e.f8 = f8;
+  e.fmt = fmt;
   e.perm = perm;
   e.topk_w = wts;
   e.w_perm = static_cast<float*>(at(M_WPERM));
@@ -1775,6 +1878,10 @@ int moe_ffn_impl(bool f8, const MoeScales& sc, const void* d_x, const float* d_r
   e.hq_scale = static_cast<float*>(at(M_HQS));
   e.hsq = at(M_HSQ);
   e.hsq_scale = static_cast<float*>(at(M_HSQS));
+  e.x_sf = static_cast<uint8_t*>(at(M_XSF));
+  e.x_sh_sf = static_cast<uint8_t*>(at(M_XSHSF));
+  e.h_sf = static_cast<uint8_t*>(at(M_HSF));
+  e.hs_sf = static_cast<uint8_t*>(at(M_HSSF));
   e.y_slot = static_cast<float*>(at(M_YSLOT));
   e.y_shared = static_cast<float*>(at(M_YSH));
   e.w_gu = d_w_gu;
@@ -1783,6 +1890,10 @@ int moe_ffn_impl(bool f8, const MoeScales& sc, const void* d_x, const float* d_r
   e.w_d_scale = sc.w_d;
   e.ws_gu_scale = sc.ws_gu;
   e.ws_d_scale = sc.ws_d;
+  e.w_gu_sf = static_cast<const uint8_t*>(sc.w_gu_sf);
+  e.w_d_sf = static_cast<const uint8_t*>(sc.w_d_sf);
+  e.ws_gu_sf = static_cast<const uint8_t*>(sc.ws_gu_sf);
+  e.ws_d_sf = static_cast<const uint8_t*>(sc.ws_d_sf);
   e.tm_wgu = &t_wgu;
   e.tm_xperm = &t_xp;
   e.tm_wsgu = &t_wsgu;
@@ -1830,7 +1941,7 @@ int dg_moe_ffn(const void* d_x, const float* d_residual, const void* d_wr, const
                int32_t* d_ids, float* d_weights, float* d_router_logits, int32_t t, int32_t d,
                int32_t n_experts, int32_t top_k, int32_t hidden, int32_t shared_hidden,
                void* d_workspace, size_t workspace_bytes, void* stream) {
-  return moe_ffn_impl(false, MoeScales{}, d_x, d_residual, d_wr, d_w_gu, d_w_d, d_ws_gu, d_ws_d,
+  return moe_ffn_impl(0, MoeScales{}, d_x, d_residual, d_wr, d_w_gu, d_w_d, d_ws_gu, d_ws_d,
                       d_y, d_ids, d_weights, d_router_logits, t, d, n_experts, top_k, hidden,
                       shared_hidden, d_workspace, workspace_bytes, stream);
 }
@@ -1842,10 +1953,55 @@ int dg_moe_ffn_e4m3(const void* d_x, const float* d_residual, const void* d_wr,
                     float* d_weights, float* d_router_logits, int32_t t, int32_t d,
                     int32_t n_experts, int32_t top_k, int32_t hidden, int32_t shared_hidden,
                     void* d_workspace, size_t workspace_bytes, void* stream) {
-  return moe_ffn_impl(true, MoeScales{d_w_gu_scale, d_w_d_scale, d_ws_gu_scale, d_ws_d_scale},
+  return moe_ffn_impl(1, MoeScales{d_w_gu_scale, d_w_d_scale, d_ws_gu_scale, d_ws_d_scale,
+                                   nullptr, nullptr, nullptr, nullptr},
                       d_x, d_residual, d_wr, d_w_gu, d_w_d, d_ws_gu, d_ws_d, d_y, d_ids,
                       d_weights, d_router_logits, t, d, n_experts, top_k, hidden, shared_hidden,
                       d_workspace, workspace_bytes, stream);
+}
+
+int dg_moe_ffn_nvfp4(const void* d_x, const float* d_residual, const void* d_wr,
+                     const void* d_w_gu, const float* d_w_gu_scale, const void* d_w_gu_sf,
+                     const void* d_w_d, const float* d_w_d_scale, const void* d_w_d_sf,
+                     const void* d_ws_gu, const float* d_ws_gu_scale, const void* d_ws_gu_sf,
+                     const void* d_ws_d, const float* d_ws_d_scale, const void* d_ws_d_sf,
+                     float* d_y, int32_t* d_ids, float* d_weights, float* d_router_logits,
+                     int32_t t, int32_t d, int32_t n_experts, int32_t top_k, int32_t hidden,
+                     int32_t shared_hidden, void* d_workspace, size_t workspace_bytes,
+                     void* stream) {
+  return moe_ffn_impl(2, MoeScales{d_w_gu_scale, d_w_d_scale, d_ws_gu_scale, d_ws_d_scale,
+                                   d_w_gu_sf, d_w_d_sf, d_ws_gu_sf, d_ws_d_sf},
+                      d_x, d_residual, d_wr, d_w_gu, d_w_d, d_ws_gu, d_ws_d, d_y, d_ids,
+                      d_weights, d_router_logits, t, d, n_experts, top_k, hidden, shared_hidden,
+                      d_workspace, workspace_bytes, stream);
+}
+
+int dg_quantize_nvfp4(const void* d_in, int32_t rows, int32_t cols, int64_t ld_in,
+                      uint8_t* d_codes, int64_t ld_codes, uint8_t* d_sf, float* d_row_scales,
+                      void* stream) {
+  if (!d_in || !d_codes || !d_sf || !d_row_scales)
+    return fail(DG_ERR_INVALID_ARG, "null pointer argument");
+  if (rows < 0 || cols < 64 || cols % 64 || ld_in < cols || ld_in % 8 || ld_codes < cols / 2 ||
+      ld_codes % 16 || ld_codes > (1 << 30))
+    return fail(DG_ERR_INVALID_ARG,
+                "need cols %% 64 == 0, ld_in >= cols, ld_in %% 8 == 0, ld_codes >= cols / 2, "
+                "ld_codes %% 16 == 0");
+  if (reinterpret_cast<uintptr_t>(d_in) % 16 || reinterpret_cast<uintptr_t>(d_codes) % 16 ||
+      reinterpret_cast<uintptr_t>(d_sf) % 16 || reinterpret_cast<uintptr_t>(d_row_scales) % 4)
+    return fail(DG_ERR_INVALID_ARG, "misaligned pointer");
+  if (rows == 0) return DG_OK;
+  cudaStream_t st = S(stream);
+  const size_t sf_bytes = static_cast<size_t>(cdiv(rows, 128)) * 4 * cdiv(cols, 256) * 512;
+  DG_CUDA(cudaMemsetAsync(d_sf, 0, sf_bytes, st));  // pad atoms and rows past `rows` read as 0
+  QuantFp4Job j{};
+  j.seg[0] = QuantFp4Seg{static_cast<const __nv_bfloat16*>(d_in), ld_in, nullptr, 1, nullptr,
+                         nullptr, rows, cols, d_codes, ld_codes, d_sf, d_row_scales, nullptr,
+                         nullptr, 128};
+  j.n_seg = 1;
+  DG_TRY(launch_pdl(quant_fp4_rows_kernel, dim3(cdiv(rows, 8)), dim3(256), 0, st, j,
+                    static_cast<const int*>(nullptr)));
+  DG_LAUNCHED();
+  return DG_OK;
 }
 
 int dg_quantize_e4m3(const void* d_in, int32_t rows, int32_t cols, int64_t ld_in,

@@ -188,6 +188,55 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n) {
          | (static_cast<uint32_t>(m >> 4) << 24); // M / 16
 }
 
+// D[tmem] (+)= A[smem] * B[smem]^T with e2m1 A and B (two codes per byte) and one ue4m3 scale per
+// 16 elements of each row of A and B, read from TMEM at sfa / sfb (kind::mxf4nvf4, K = 64 per
+// instruction: the same 32 bytes of a 128-byte swizzle row).
+DG_DEV void umma_fp4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                     uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem),
+      "r"(sfb_tmem)
+      : "memory");
+}
+
+// Instruction descriptor of the block-scaled kind::mxf4nvf4: e2m1 A and B (format 1), ue4m3
+// scales (bit 23 = 0), scale ids 0, K = 64, dense; the accumulator is fp32.
+__host__ __device__ constexpr uint32_t idesc_fp4_f32(int m, int n) {
+  return (1u << 7)                              // A format: e2m1
+         | (1u << 10)                           // B format: e2m1
+         | (static_cast<uint32_t>(n >> 3) << 17)  // N / 8
+         | (static_cast<uint32_t>(m >> 4) << 24); // M / 16
+}
+
+// Copy a 32-row x 16-byte shared-memory matrix (one 512-byte scale atom) into TMEM columns
+// taddr .. taddr + 3 of every 32-lane quarter.
+DG_DEV void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+               : "memory");
+}
+
+// Shared-memory descriptor of an unswizzled K-major matrix of 16-byte rows stored back to back
+// (core matrices of 8 rows x 16 B, 128 B apart along the rows): the source of tmem_cp_32x128b_x4.
+DG_DEV uint64_t sdesc_rows16(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>(128 >> 4) << 16;     // leading byte offset (one core matrix along K)
+  d |= static_cast<uint64_t>(128 >> 4) << 32;     // stride byte offset: next 8 rows
+  d |= static_cast<uint64_t>(1) << 46;            // descriptor version
+  return d;                                       // layout type 0: no swizzle
+}
+
+// Bulk copy of `bytes` (multiple of 16, 16-byte aligned ends) from global to this CTA's shared
+// memory, completing on `bar` (counted in its expected transaction bytes).
+DG_DEV void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_u32(smem_dst)), "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // Instruction descriptor for kind::f8f6f4 with e4m3 A and B (format code 0), fp32 D, both
 // operands K-major, dense.
 __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int m, int n) {

@@ -9,8 +9,11 @@
 //   warps 2-5: epilogue, TMEM lane quarter (warp % 4), one accumulator row per thread.
 // Work items are either arithmetic (dense layers, optional split-K) or a device-built list
 // (grouped experts, one item per (expert, 128-row tile, token chunk)).
-// With F8 the operands are e4m3 codes (kind::f8f6f4): a 128-byte K slab holds 128 elements
-// instead of 64, the ring and descriptors are unchanged, and the epilogue first scales each
+// Operand formats (FMT): 0 bf16; 1 e4m3 codes (kind::f8f6f4: a 128-byte K slab holds 128
+// elements); 2 NVFP4 (kind::mxf4nvf4.block_scale.block16: a slab holds 256 e2m1 codes, and each
+// stage also brings the slab's 512-byte scale atoms for A and B, which the MMA thread moves into
+// TMEM with tcgen05.cp before the four MMAs that read them).  The ring and the operand
+// descriptors are the same for all three; with FMT != 0 the epilogue first scales each
 // accumulator by its weight row's scale and its token row's scale.
 //
 // lmhead_kernel: logits tile = X[256 tokens] * E[256 vocab rows]^T (two M=128 token tiles,
@@ -66,12 +69,19 @@ struct GemmParams {
   const float* b_scale;
   const float* alt_a_scale;
   const float* alt_b_scale;
+  // NVFP4 block-scale atoms (512 B each, 4 * kb_total per 128-row tile of A, per routed chunk
+  // of B, per token chunk of the alternate group's B)
+  const uint8_t* a_sf;
+  const uint8_t* b_sf;
+  const uint8_t* alt_a_sf;
+  const uint8_t* alt_b_sf;
   int* err;
   const int* done;
 };
 
 struct GemmItem {
   int a_row, b_row, n, kb0, kb1, r_base, aux;
+  int chunk;  // routed chunk, or token chunk of the alternate group (NVFP4 scale atoms of B)
   bool alt;
 };
 
@@ -79,6 +89,7 @@ DG_DEV GemmItem gemm_item(const GemmParams& p, int it) {
   GemmItem w;
   w.alt = false;
   w.kb0 = 0;
+  w.chunk = 0;
   if (p.chunks == nullptr) {
     const int mt = it % p.m_tiles;
     const int rest = it / p.m_tiles;
@@ -102,6 +113,7 @@ DG_DEV GemmItem gemm_item(const GemmParams& p, int it) {
       w.n = min(p.n_chunk, p.alt_tokens - ch * p.n_chunk);
       w.kb1 = p.alt_kb_total;
       w.aux = p.alt_group;
+      w.chunk = ch;
     } else {
       const int r = it - sh_items;
       const int ch = r / p.m_tiles, m = r % p.m_tiles;
@@ -112,6 +124,7 @@ DG_DEV GemmItem gemm_item(const GemmParams& p, int it) {
       w.n = c.z;
       w.kb1 = p.kb_total;
       w.aux = c.x;
+      w.chunk = ch;
     }
   }
   return w;
@@ -123,13 +136,21 @@ DG_DEV int gemm_item_count(const GemmParams& p) {
   return sh_items + *reinterpret_cast<const volatile int*>(p.chunk_count) * p.m_tiles;
 }
 
-template <int MAXN, int STAGES>
+template <int MAXN, int STAGES, int FMT = 0>
 struct GemmCfg {
-  static constexpr int kABytes = 128 * 128;   // 128 rows x 64 bf16
-  static constexpr int kBBytes = MAXN * 128;  // MAXN rows x 64 bf16
-  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kABytes = 128 * 128;   // 128 rows x 128 B (64 bf16 / 128 e4m3 / 256 e2m1)
+  static constexpr int kBBytes = MAXN * 128;  // MAXN rows x 128 B
+  // NVFP4: the slab's four scale atoms for A, then for B (one per 128 rows of B)
+  static constexpr int kSfaBytes = FMT == 2 ? 4 * 512 : 0;
+  static constexpr int kSfbBytes = FMT == 2 ? 4 * 512 * ((MAXN + 127) / 128) : 0;
+  static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
   static constexpr int kAccBufs = MAXN <= 128 ? 4 : 2;  // TMEM accumulators in flight
-  static constexpr int kTmemCols = kAccBufs * MAXN;
+  static constexpr int kAccCols = kAccBufs * MAXN;
+  // NVFP4: per stage 16 TMEM columns of A scales and 16 per 128 rows of B after the accumulators
+  static constexpr int kSfCols = FMT == 2 ? 16 + 16 * ((MAXN + 127) / 128) : 0;
+  static constexpr int kTmemUsed = kAccCols + STAGES * kSfCols;
+  static constexpr int kTmemCols = kTmemUsed <= 256 ? 256 : 512;
+  static_assert(kTmemUsed <= 512, "TMEM");
   // epilogue warps: two per TMEM lane quarter for wide token tiles (they split the columns)
   static constexpr int kEpiWarps = MAXN >= 128 ? 8 : 4;
   static constexpr int kThreads = 64 + 32 * kEpiWarps;
@@ -196,13 +217,14 @@ DG_DEV void gemm_epilogue_chunk(const GemmParams& p, const GemmItem& w, const fl
   }
 }
 
-template <int MAXN, int STAGES, int EPI, bool F8 = false>
-__global__ void __launch_bounds__(GemmCfg<MAXN, STAGES>::kThreads, 1)
+template <int MAXN, int STAGES, int EPI, int FMT = 0>
+__global__ void __launch_bounds__(GemmCfg<MAXN, STAGES, FMT>::kThreads, 1)
     gemm_swapab_kernel(const __grid_constant__ CUtensorMap tm_a,
                        const __grid_constant__ CUtensorMap tm_b,
                        const __grid_constant__ CUtensorMap tm_a2,
                        const __grid_constant__ CUtensorMap tm_b2, const GemmParams p) {
-  using C = GemmCfg<MAXN, STAGES>;
+  using C = GemmCfg<MAXN, STAGES, FMT>;
+  constexpr bool kScaled = FMT != 0;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -260,7 +282,7 @@ __global__ void __launch_bounds__(GemmCfg<MAXN, STAGES>::kThreads, 1)
         const GemmItem w = wn;
         if (it + static_cast<int>(gridDim.x) < n_items) wn = gemm_item(p, it + gridDim.x);
         const int nbox = (w.n + 31) >> 5;
-        const uint32_t bytes = C::kABytes + nbox * 32 * 128;
+        const uint32_t bytes = C::kABytes + nbox * 32 * 128 + C::kSfaBytes + C::kSfbBytes;
         const CUtensorMap* ta = w.alt ? &tm_a2 : &tm_a;
         const CUtensorMap* tb = w.alt ? &tm_b2 : &tm_b;
         for (int kb = w.kb0; kb < w.kb1; ++kb) {
@@ -271,10 +293,21 @@ __global__ void __launch_bounds__(GemmCfg<MAXN, STAGES>::kThreads, 1)
           uint8_t* sa = smem + stage * C::kStageBytes;
           uint8_t* sb = sa + C::kABytes;
           mbar_arrive_expect_tx(&full[stage], bytes);
-          const int kx = kb * (F8 ? 128 : 64);  // elements per 128-byte slab
+          const int kx = kb * (FMT != 0 ? 128 : 64);  // map columns per 128-byte slab
           tma_load_2d(ta, &full[stage], sa, kx, w.a_row, pol_a);
           for (int bx = 0; bx < nbox; ++bx)
             tma_load_2d(tb, &full[stage], sb + bx * 4096, kx, w.b_row + bx * 32, pol_b);
+          if constexpr (FMT == 2) {
+            // the slab's scale atoms: A by 128-row tile, B by chunk (4 per slab, padded)
+            const int kt = w.alt ? p.alt_kb_total : p.kb_total;
+            const uint8_t* fa = (w.alt ? p.alt_a_sf : p.a_sf) +
+                                (static_cast<long long>(w.a_row >> 7) * 4 * kt + 4 * kb) * 512;
+            const uint8_t* fb = (w.alt ? p.alt_b_sf : p.b_sf) +
+                                (static_cast<long long>(w.chunk) * 4 * kt + 4 * kb) * 512 *
+                                    ((MAXN + 127) / 128);
+            bulk_load(sb + C::kBBytes, fa, C::kSfaBytes, &full[stage]);
+            bulk_load(sb + C::kBBytes + C::kSfaBytes, fb, C::kSfbBytes, &full[stage]);
+          }
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
@@ -294,8 +327,9 @@ __global__ void __launch_bounds__(GemmCfg<MAXN, STAGES>::kThreads, 1)
       for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
         const GemmItem w = wn;
         if (it + static_cast<int>(gridDim.x) < n_items) wn = gemm_item(p, it + gridDim.x);
-        const uint32_t idesc = F8 ? idesc_e4m3_f32(128, (w.n + 15) & ~15)
-                                  : idesc_bf16_f32(128, (w.n + 15) & ~15);
+        const uint32_t idesc = FMT == 2   ? idesc_fp4_f32(128, (w.n + 15) & ~15)
+                               : FMT == 1 ? idesc_e4m3_f32(128, (w.n + 15) & ~15)
+                                          : idesc_bf16_f32(128, (w.n + 15) & ~15);
         if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, p.err)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * MAXN;
@@ -308,12 +342,27 @@ __global__ void __launch_bounds__(GemmCfg<MAXN, STAGES>::kThreads, 1)
           const uint32_t sa = smem_u32(smem + stage * C::kStageBytes);
           const uint64_t da = sdesc_sw128(sa);
           const uint64_t db = sdesc_sw128(sa + C::kABytes);
+          if constexpr (FMT == 2) {
+            // scale atoms into this stage's TMEM columns (in issue order before their MMAs)
+            const uint32_t sfa = sa + C::kABytes + C::kBBytes;
+            const uint32_t t_sf = tmem_base + C::kAccCols + stage * C::kSfCols;
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            if constexpr (F8)
-              umma_e4m3(d_tmem, da + 2 * k, db + 2 * k, idesc, (kb > w.kb0 || k > 0) ? 1u : 0u);
-            else
-              umma_bf16(d_tmem, da + 2 * k, db + 2 * k, idesc, (kb > w.kb0 || k > 0) ? 1u : 0u);
+            for (int k = 0; k < 4; ++k) {
+              tmem_cp_32x128b_x4(t_sf + 4 * k, sdesc_rows16(sfa + 512 * k));
+              tmem_cp_32x128b_x4(t_sf + 16 + 4 * k, sdesc_rows16(sfa + C::kSfaBytes + 512 * k));
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              umma_fp4(d_tmem, da + 2 * k, db + 2 * k, idesc, t_sf + 4 * k, t_sf + 16 + 4 * k,
+                       (kb > w.kb0 || k > 0) ? 1u : 0u);
+          } else {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              if constexpr (FMT == 1)
+                umma_e4m3(d_tmem, da + 2 * k, db + 2 * k, idesc, (kb > w.kb0 || k > 0) ? 1u : 0u);
+              else
+                umma_bf16(d_tmem, da + 2 * k, db + 2 * k, idesc, (kb > w.kb0 || k > 0) ? 1u : 0u);
+            }
           }
           umma_commit(&empty[stage]);
           if (++stage == STAGES) {
@@ -357,10 +406,11 @@ __global__ void __launch_bounds__(GemmCfg<MAXN, STAGES>::kThreads, 1)
           }
         }
       }
-      // e4m3: this lane's weight-row scale and token scales, loaded before the accumulator is ready
+      // e4m3 / NVFP4: this lane's weight-row scale and token scales, loaded before the
+      // accumulator is ready
       float row_scale = 1.0f;
       float tok_scale[MAXN / 32];
-      if constexpr (F8) {
+      if constexpr (kScaled) {
         const float* as = w.alt ? p.alt_a_scale : p.a_scale;
         const float* bs = w.alt ? p.alt_b_scale : p.b_scale;
         const int m_valid = w.alt ? p.alt_m_valid : p.m_valid;
@@ -380,7 +430,7 @@ __global__ void __launch_bounds__(GemmCfg<MAXN, STAGES>::kThreads, 1)
         if (cc % kGroups == grp && c < w.n) {
           float v[32];
           tmem_ld32(t_row + c, v);
-          if constexpr (F8) {
+          if constexpr (kScaled) {
 #pragma unroll
             for (int i = 0; i < 32; ++i)
               v[i] *= row_scale * __shfl_sync(0xffffffffu, tok_scale[cc], i);

@@ -64,7 +64,11 @@ enum {
  * weights are e4m3 codes with one fp32 scale per weight row, and the expert GEMMs take e4m3
  * activations, quantised per row on the fly (scale = max|row| / 448, codes = rn_satfinite(x /
  * scale)); attention, router, norms and the LM head stay bf16. */
-enum { DG_DTYPE_BF16 = 0, DG_DTYPE_FP32 = 1, DG_DTYPE_BF16_E4M3 = 2 };
+enum { DG_DTYPE_BF16 = 0, DG_DTYPE_FP32 = 1, DG_DTYPE_BF16_E4M3 = 2, DG_DTYPE_BF16_NVFP4 = 3 };
+/* DG_DTYPE_BF16_NVFP4 is the same with the NVFP4 expert format ([pl]: 18 GB; [blog]: NVFP4
+ * kernels on Blackwell): e2m1 codes (two per byte, low nibble first, rows at
+ * DG_E4M3_PITCH(K / 2) bytes), one e4m3 scale per 16 codes in 512-byte atoms (see
+ * dg_quantize_nvfp4) and one fp32 scale per row; the expert GEMMs take NVFP4 activations. */
 
 /* Model and decode configuration.  Shapes follow the pages' model ([course], [arch]). */
 typedef struct dg_config {
@@ -135,6 +139,10 @@ typedef struct dg_layer_weights {
   const float* w_d_scale;   /* fp32 [E, d], one per w_d row */
   const float* ws_gu_scale; /* fp32 [2hs], or NULL */
   const float* ws_d_scale;  /* fp32 [d], or NULL */
+  const void* w_gu_sf;      /* DG_DTYPE_BF16_NVFP4: block-scale atoms of w_gu (as written by */
+  const void* w_d_sf;       /*   dg_quantize_nvfp4 for the stacked [E * rows, K] matrix),    */
+  const void* ws_gu_sf;     /*   of w_d, ws_gu and ws_d; NULL otherwise                       */
+  const void* ws_d_sf;
 } dg_layer_weights;
 
 typedef struct dg_weights {
@@ -314,6 +322,32 @@ DG_API int dg_moe_ffn_e4m3(const void* d_x, const float* d_residual, const void*
  * pointers, else DG_ERR_INVALID_ARG before any launch.  Asynchronous on `stream`. */
 DG_API int dg_quantize_e4m3(const void* d_in, int32_t rows, int32_t cols, int64_t ld_in,
                             uint8_t* d_codes, int64_t ld_codes, float* d_scales, void* stream);
+
+/* NVFP4 quantisation of `rows` bf16 rows of `cols` values (row pitch ld_in elements), the
+ * 4-bit expert format: per row g = max|row| / 2688 (fp32, IEEE division); per 16 consecutive
+ * values s = e4m3_rn_satfinite(max|block| / 6 / g); codes e2m1_rn_satfinite(x / (s * g)), two
+ * per byte with the lower column in the low nibble, rows at ld_codes bytes (zero past cols / 2).
+ * Block scales go to 512-byte atoms, one per (128-row tile, 64 columns): tile t's atoms start
+ * at d_sf + t * 4 * ceil(cols / 256) * 512 (the ones past cols / 64 are zero); inside an atom
+ * the scale of tile row r and 16-wide block b is byte (r % 32) * 16 + (r / 32) * 4 + b.
+ * d_sf must hold ceil(rows / 128) * 4 * ceil(cols / 256) * 512 bytes.  cols % 64 == 0,
+ * ld_codes >= cols / 2 and a multiple of 16, ld_in % 8 == 0, 16-byte aligned pointers, else
+ * DG_ERR_INVALID_ARG before any launch.  Asynchronous on `stream`. */
+DG_API int dg_quantize_nvfp4(const void* d_in, int32_t rows, int32_t cols, int64_t ld_in,
+                             uint8_t* d_codes, int64_t ld_codes, uint8_t* d_sf,
+                             float* d_row_scales, void* stream);
+
+/* The MoE with NVFP4 experts: codes, row scales and scale atoms of w_gu, w_d (and ws_gu, ws_d
+ * when hs > 0) as dg_quantize_nvfp4 writes them for the stacked matrices.  Shapes as
+ * dg_moe_ffn, with d a multiple of 128; workspace size from dg_moe_workspace_bytes. */
+DG_API int dg_moe_ffn_nvfp4(const void* d_x, const float* d_residual, const void* d_wr,
+               const void* d_w_gu, const float* d_w_gu_scale, const void* d_w_gu_sf,
+               const void* d_w_d, const float* d_w_d_scale, const void* d_w_d_sf,
+               const void* d_ws_gu, const float* d_ws_gu_scale, const void* d_ws_gu_sf,
+               const void* d_ws_d, const float* d_ws_d_scale, const void* d_ws_d_sf, float* d_y,
+               int32_t* d_ids, float* d_weights, float* d_router_logits, int32_t t, int32_t d,
+               int32_t n_experts, int32_t top_k, int32_t hidden, int32_t shared_hidden,
+               void* d_workspace, size_t workspace_bytes, void* stream);
 
 /* ---- tracing ------------------------------------------------------------------------- */
 

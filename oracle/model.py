@@ -31,7 +31,7 @@ import numpy as np
 
 from . import sampler as smp
 from .attention import attention
-from .moe import moe_ffn, moe_ffn_fp8
+from .moe import moe_ffn, moe_ffn_fp8, moe_ffn_nvfp4
 from .numerics import round_f32, round_storage
 
 
@@ -49,7 +49,7 @@ class ModelConfig:
     vocab: int
     canvas: int = 256
     storage: str = "bf16"
-    experts: str = "bf16"  # "fp8": e4m3 expert weights and activations (oracle.quant)
+    experts: str = "bf16"  # "fp8" / "nvfp4": quantised expert weights and activations (quant.py)
     eps: float = 1e-6
     rope_theta: float = 10000.0
     tau: float = smp.TAU
@@ -117,6 +117,8 @@ def moe_block(cfg, lw, x1):
     shared = (lw["ws_gu"], lw["ws_d"]) if lw.get("ws_gu") is not None else None
     if cfg.experts == "fp8":
         y, minfo = moe_ffn_fp8(xn2, lw["wr"], lw["w_gu"], lw["w_d"], cfg.top_k, shared)
+    elif cfg.experts == "nvfp4":
+        y, minfo = moe_ffn_nvfp4(xn2, lw["wr"], lw["w_gu"], lw["w_d"], cfg.top_k, shared)
     else:
         y, minfo = moe_ffn(xn2, lw["wr"], lw["w_gu"], lw["w_d"], cfg.top_k, st, shared)
     x2 = round_f32(np.asarray(x1, dtype=np.float64) + y)
