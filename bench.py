@@ -56,6 +56,8 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--roofline-kernel", default="expert_gate_up")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--head", choices=["bf16", "e4m3"], default="bf16",
+                    help="LM head format (e4m3: the head on e4m3 operands)")
     ap.add_argument("--experts", choices=["bf16", "e4m3", "nvfp4"], default="bf16",
                     help="expert weight format of the decode model")
     ap.add_argument("--profile", choices=["decode_step", "decode_step_small", "decode_step_e4m3",
@@ -282,22 +284,23 @@ def run_ops(dev, stream, hbm, tf_burst):
     return out
 
 
-def step_bytes(shape, prefix, f8=False):
+def step_bytes(shape, prefix, experts="bf16", head="bf16"):
     """Algorithmic HBM bytes of one denoise step at committed length `prefix`: every weight the
     step reads once (QKV, O, router, all routed experts' gate/up and down, the shared expert; all
     128 experts are routed at these shapes) per layer, the K/V cache read over prefix + canvas
-    keys and the canvas K/V written per layer, and the LM head's embedding table.  Activations
-    (a few MB per layer) are left out.  e4m3 experts: one byte per weight plus one fp32 scale per
-    weight row."""
+    keys and the canvas K/V written per layer, and the LM head's table.  Activations (a few MB per
+    layer) are left out.  e4m3: one byte per weight plus one fp32 scale per weight row; NVFP4:
+    half a byte per weight, one e4m3 block scale per 16 weights, one fp32 scale per row."""
     d, hq, hkv, hd = shape["d_model"], shape["n_heads"], shape["n_kv_heads"], shape["head_dim"]
     e, h, hs, v = shape["n_experts"], shape["expert_hidden"], shape["shared_hidden"], shape["vocab"]
     dense = ((hq + 2 * hkv) * hd * d + d * hq * hd + e * d) * 2
-    if f8:
-        experts = (e * 2 * h + 2 * hs) * d + (e * h + hs) * d + (e * 2 * h + e * d + 2 * hs + d) * 4
-    else:
-        experts = (e * 3 * h * d + 3 * hs * d) * 2
+    n_w = e * 3 * h * d + 3 * hs * d                     # expert weights
+    n_rows = e * 2 * h + e * d + 2 * hs + d               # expert weight rows
+    per_w = {"bf16": 2.0, "e4m3": 1.0, "nvfp4": 0.5 + 1.0 / 16}[experts]
+    ex = int(n_w * per_w) + (0 if experts == "bf16" else n_rows * 4)
     kv = (prefix + CANVAS) * hkv * hd * 2 * 2 + CANVAS * hkv * hd * 2 * 2
-    return shape["n_layers"] * (dense + experts + kv) + v * d * 2
+    lm = v * d * 2 if head == "bf16" else v * d + v * 4
+    return shape["n_layers"] * (dense + ex + kv) + lm
 
 
 def live_kernel_table(model, stream, L):
@@ -337,7 +340,8 @@ def decode(model, seed, out_ids, out_states, stream, fixed=True):
 
 
 def run_ours(args, rank, world, local_rank):
-    from block_text_diffusion_dg_b200 import DiffusionModel, generate, make_config, quantize_experts
+    from block_text_diffusion_dg_b200 import (DiffusionModel, generate, make_config, quantize_experts,
+                                              quantize_head)
     from block_text_diffusion_dg_b200 import _lib as L
     from dg_synth import SHAPES, model_weights, uniform_ids
     import torch.distributed as dist
@@ -349,8 +353,10 @@ def run_ours(args, rank, world, local_rank):
     f8 = args.experts != "bf16"  # quantised experts (e4m3 or NVFP4)
     f4 = args.experts == "nvfp4"
     cfg = make_config(shape, kv_capacity=cap, fixed_steps=FIXED_STEPS,
-                      prefill_chunk=1024 if f4 else PREFILL_CHUNK, experts=args.experts)
+                      prefill_chunk=1024 if f4 else PREFILL_CHUNK, experts=args.experts, head=args.head)
     weights = model_weights("a4b", seed=1000 + rank, device=dev)
+    if args.head == "e4m3":
+        weights = quantize_head(weights)
     if f8:  # the bf16 expert matrices are dropped once quantised
         weights = quantize_experts(weights, fmt=args.experts)
         torch.cuda.synchronize()
@@ -460,7 +466,7 @@ def run_ours(args, rank, world, local_rank):
     table = live_kernel_table(model, stream, L)
 
     # the whole denoise step against the HBM roofline (block 0: 4,096 committed positions)
-    sb = step_bytes(shape, PROMPT, f8)
+    sb = step_bytes(shape, PROMPT, args.experts, args.head)
     step_gbs = sb / (us_step / 1e6) / 1e9
     step_roof = dict(bound="hbm", achieved=round(step_gbs, 1), peak=hbm, unit="GB/s",
                      frac=round(step_gbs / hbm, 4), algorithmic_bytes_per_step=sb,
@@ -470,7 +476,7 @@ def run_ours(args, rank, world, local_rank):
     # adaptive stop, 48-step cap ([canvas] step 3): random-init weights never reach the stop
     # rule, so every block runs to the cap
     cfg_a = make_config(shape, kv_capacity=cap, fixed_steps=0, max_steps=MAX_STEPS,
-                        prefill_chunk=PREFILL_CHUNK, experts=args.experts)
+                        prefill_chunk=PREFILL_CHUNK, experts=args.experts, head=args.head)
     model_a = DiffusionModel(cfg_a, weights, device=dev)
     model_a.kv_append(prompt_dev, stream)
     decode(model_a, 300, out_ids, out_states, stream, fixed=False)  # warm-up
@@ -492,7 +498,7 @@ def run_ours(args, rank, world, local_rank):
     # long context ([canvas] step 1 prefill; the pages' weak spot is the time to the first
     # output): a 32,768-token prompt in 4,096-token passes, then the first block of 16 steps
     cfg_l = make_config(shape, kv_capacity=LONG_PROMPT + 2 * CANVAS, fixed_steps=FIXED_STEPS,
-                        prefill_chunk=PREFILL_CHUNK, experts=args.experts)
+                        prefill_chunk=PREFILL_CHUNK, experts=args.experts, head=args.head)
     model_l = DiffusionModel(cfg_l, weights, device=dev)
     long_prompt = uniform_ids(LONG_PROMPT, shape["vocab"], seed=77 + rank).to(dev)
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
@@ -520,7 +526,7 @@ def run_ours(args, rank, world, local_rank):
     # small-batch canvases: BATCH sequences (own prompts and caches) decoded in lockstep, every
     # denoise step carrying BATCH x 256 canvas tokens through one weight stream
     cfg_b = make_config(shape, kv_capacity=cap, fixed_steps=FIXED_STEPS,
-                        prefill_chunk=PREFILL_CHUNK, experts=args.experts, batch=BATCH)
+                        prefill_chunk=PREFILL_CHUNK, experts=args.experts, head=args.head, batch=BATCH)
     model_b = DiffusionModel(cfg_b, weights, device=dev)
     prompts_b = torch.stack([uniform_ids(PROMPT, shape["vocab"], seed=90 + BATCH * rank + b)
                              for b in range(BATCH)]).to(dev)
@@ -593,10 +599,13 @@ def run_ours(args, rank, world, local_rank):
                    n_gpus=world, steps=args.steps, warmup=args.warmup,
                    ms_per_step=round(ms_max / args.steps, 3), higher_is_better=True,
                    scaling="weak", vs_baseline=None,
-                   dtype={"bf16": "bf16", "e4m3": "bf16+e4m3", "nvfp4": "bf16+nvfp4"}[args.experts],
+                   dtype={"bf16": "bf16", "e4m3": "bf16+e4m3", "nvfp4": "bf16+nvfp4"}[args.experts]
+                         + ("+e4m3 head" if args.head == "e4m3" else ""),
                    data="synthetic",
                    config=dict(workload={"bf16": WORKLOAD, "e4m3": WORKLOAD_E4M3,
-                                         "nvfp4": WORKLOAD_NVFP4}[args.experts], global_batch=world,
+                                         "nvfp4": WORKLOAD_NVFP4}[args.experts]
+                               + (", LM head on e4m3 operands" if args.head == "e4m3" else ""),
+                               global_batch=world,
                                seq_len=PROMPT + BLOCKS * CANVAS,
                                parallelism=f"replicas x{world}",
                                l2="inputs larger than L2: ~%d GB of weights streamed per denoise "

@@ -28,6 +28,7 @@ class Config(C.Structure):
         ("fixed_steps", C.c_int32), ("prefill_chunk", C.c_int32),
         ("lock_rule", C.c_int32), ("entropy_lock", C.c_double), ("sticky_locks", C.c_int32),
         ("temperature", C.c_float), ("commit_reuse_kv", C.c_int32), ("batch", C.c_int32),
+        ("lm_head_e4m3", C.c_int32),
     ]
 
 
@@ -40,7 +41,8 @@ class LayerWeights(C.Structure):
 
 class Weights(C.Structure):
     _fields_ = [("embed", C.c_void_p), ("final_norm", C.c_void_p),
-                ("layers", C.POINTER(LayerWeights))]
+                ("layers", C.POINTER(LayerWeights)), ("head_codes", C.c_void_p),
+                ("head_scale", C.c_void_p)]
 
 
 _P = C.c_void_p

@@ -34,13 +34,16 @@ def _need_cuda(t, name, dtype=None):
 def make_config(shape, *, kv_capacity, fixed_steps=16, max_steps=48, tau=0.9, h_bound=0.005,
                 eps=1e-6, rope_theta=10000.0, prefill_chunk=0, experts="bf16",
                 lock_rule="confidence", entropy_lock=0.1, sticky=False, temperature=1.0,
-                commit="reencode", batch=1):
+                commit="reencode", batch=1, head="bf16"):
     """Config of a model shape; experts="e4m3" selects the FP8 expert format (bf16 model);
     lock_rule="entropy_bound" locks positions with entropy <= entropy_lock (nats) instead of
     confidence >= tau; sticky=True keeps a locked position's token for the rest of the block;
     temperature sets T of the sampler's softmax(logits / T); commit="reuse_kv" commits a block
     by keeping the canvas K/V of its last denoise step instead of re-encoding it causally;
-    batch=B decodes B sequences in lockstep (sequence b's Philox key is seed + b)."""
+    batch=B decodes B sequences in lockstep (sequence b's Philox key is seed + b); head="e4m3"
+    runs the LM head on e4m3 operands (weights from quantize_head)."""
+    if head not in ("bf16", "e4m3"):
+        raise ValueError("head must be 'bf16' or 'e4m3'")
     if commit not in ("reencode", "reuse_kv"):
         raise ValueError("commit must be 'reencode' or 'reuse_kv'")
     s = shape
@@ -65,7 +68,8 @@ def make_config(shape, *, kv_capacity, fixed_steps=16, max_steps=48, tau=0.9, h_
         rope_theta=rope_theta, tau=tau, h_bound=h_bound, max_steps=max_steps,
         fixed_steps=fixed_steps, prefill_chunk=prefill_chunk, lock_rule=rules[lock_rule],
         entropy_lock=entropy_lock, sticky_locks=int(bool(sticky)), temperature=temperature,
-        commit_reuse_kv=int(commit == "reuse_kv"), batch=int(batch))
+        commit_reuse_kv=int(commit == "reuse_kv"), batch=int(batch),
+        lm_head_e4m3=int(head == "e4m3"))
 
 
 def workspace_bytes(cfg):
@@ -98,8 +102,12 @@ class DiffusionModel:
         _need_cuda(weights["embed"], "embed")
         _need_cuda(weights["final_norm"], "final_norm")
         self._layers = layers
+        hc, hs = weights.get("head_codes"), weights.get("head_scale")
+        _need_cuda(hc, "head_codes")
+        _need_cuda(hs, "head_scale")
         w = L.Weights(embed=weights["embed"].data_ptr(), final_norm=weights["final_norm"].data_ptr(),
-                      layers=layers)
+                      layers=layers, head_codes=None if hc is None else hc.data_ptr(),
+                      head_scale=None if hs is None else hs.data_ptr())
         h = C.c_void_p()
         check(lib().dg_create(C.byref(cfg), C.byref(w), _ptr(self.kv), _ptr(self.scratch),
                               _stream(stream), C.byref(h)), "dg_create")
@@ -376,6 +384,15 @@ def quantize_nvfp4(x, stream=None):
     check(lib().dg_quantize_nvfp4(_ptr(x), rows, cols, cols, _ptr(codes), pitch, _ptr(sf),
                                   _ptr(scales), _stream(stream)), "dg_quantize_nvfp4")
     return codes, sf, scales
+
+
+def quantize_head(weights, stream=None):
+    """A copy of a weight dict with the e4m3 head added: head_codes (codes of the embedding table
+    at e4m3_pitch) and head_scale (one fp32 scale per vocabulary row).  The bf16 embedding stays
+    for the canvas embedding gather."""
+    out = dict(weights)
+    out["head_codes"], out["head_scale"] = quantize_e4m3(weights["embed"], stream=stream)
+    return out
 
 
 def quantize_experts(weights, fmt="e4m3", stream=None):

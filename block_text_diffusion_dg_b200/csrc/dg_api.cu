@@ -511,6 +511,10 @@ struct dg_ctx {
   std::vector<dg_layer_weights> layers;
   const void* embed;
   const float* final_norm;
+  const void* head_codes;   // e4m3 head: embedding codes [V, pitch] and row scales [V]
+  const float* head_scale;
+  uint8_t* xhq;             // e4m3 head: codes [batch * T, pitch] and scales of the normed tokens
+  float* xhs;
   uint8_t* kv;
   uint8_t* scratch;
   int32_t kv_len;
@@ -554,6 +558,7 @@ struct dg_ctx {
   // tensor maps (bf16)
   CUtensorMap tm_xn32, tm_xn128, tm_o32, tm_xperm, tm_h, tm_hs, tm_q, tm_k, tm_vt, tm_embed;
   CUtensorMap tm_xsh;  // e4m3: B operand of the shared expert's gate/up
+  CUtensorMap tm_xhq, tm_ehq;  // e4m3 head: token codes (128-row boxes), vocabulary codes (256)
   std::vector<CUtensorMap> tm_wqkv, tm_wo, tm_wr, tm_wgu, tm_wd, tm_wsgu, tm_wsd;
   uint64_t seed;
   uint32_t block;
@@ -596,6 +601,9 @@ int check_config(const dg_config* c) {
                        c->batch * c->canvas > 4096))
     return fail(DG_ERR_UNSUPPORTED,
                 "batch > 1 needs a bf16 dtype, canvas %% 128 == 0 and batch * canvas <= 4096");
+  if (c->lm_head_e4m3 < 0 || c->lm_head_e4m3 > 1 ||
+      (c->lm_head_e4m3 && c->dtype == DG_DTYPE_FP32))
+    return fail(DG_ERR_INVALID_ARG, "lm_head_e4m3 must be 0 or 1 (1 needs a bf16 dtype)");
   if (c->commit_reuse_kv < 0 || c->commit_reuse_kv > 1)
     return fail(DG_ERR_INVALID_ARG, "commit_reuse_kv must be 0 or 1");
   if (!(c->temperature >= 0.0f) || c->temperature > 1e4f)
@@ -634,7 +642,7 @@ enum Buf {
   B_XN, B_PART, B_Q, B_OPART, B_ML, B_O, B_RLOG, B_IDS, B_W, B_OFF, B_PERM, B_CHUNKS,
   B_NCHUNKS, B_RTICKET, B_XPERM, B_H, B_HS, B_YSLOT, B_YSH, B_LMPART, B_LOGITS, B_ROPE,
   B_XPS, B_XSH, B_XSHS, B_HQ, B_HQS, B_HSQ, B_HSQS, B_WPERM, B_COMMIT, B_XSF, B_XSHSF, B_HSF,
-  B_HSSF, B_END
+  B_HSSF, B_XHQ, B_XHS, B_END
 };
 
 struct Derived {
@@ -735,6 +743,9 @@ Plan plan(const dg_config& c, int sms) {
   sz[B_XSHSF] = fmt == 2 ? tok_chunks * atoms_d * 512 : 0;
   sz[B_HSF] = fmt == 2 ? dv.max_chunks * atoms_h * 512 : 0;
   sz[B_HSSF] = fmt == 2 ? tok_chunks * atoms_hs * 512 : 0;
+  // e4m3 head: codes and scales of the final normed canvas tokens
+  sz[B_XHQ] = c.lm_head_e4m3 ? Tc * e4m3_pitch(c.d_model) : 0;
+  sz[B_XHS] = c.lm_head_e4m3 ? Tc * 4 : 0;
   size_t o = 0;
   for (int b = 0; b < B_END; ++b) {
     p.off[b] = o;
@@ -1037,12 +1048,23 @@ int run_lm_head(dg_ctx* c, float* logits_out, const int* done, cudaStream_t st) 
   if (c->bf16) {
     // one launch per 256 canvas tokens (each launch holds two 128-token accumulators in TMEM)
     const int n_tok = T * c->batch;
+    const bool f8h = g.lm_head_e4m3 != 0;
+    if (f8h) {  // e4m3 codes and scales of the final normed tokens
+      QuantJob j{};
+      j.seg[0] = QuantSeg{static_cast<const __nv_bfloat16*>(c->xn), g.d_model, nullptr, 1, nullptr,
+                          nullptr, n_tok, g.d_model, c->xhq, e4m3_pitch(g.d_model), c->xhs};
+      j.n_seg = 1;
+      DG_TRY(launch_pdl(quant_rows_kernel, dim3(cdiv(n_tok, 8)), dim3(256), 0, st, j, done));
+      DG_LAUNCHED();
+    }
     for (int t0 = 0; t0 < n_tok; t0 += 256) {
       LmHeadParams p{};
       p.n_tokens = std::min(256, n_tok - t0);
       p.tok_base = t0;
       p.n_vtiles = g.vocab / 256;
-      p.kb_total = g.d_model / 64;
+      p.kb_total = f8h ? cdiv(g.d_model, 128) : g.d_model / 64;
+      p.x_scale = c->xhs;
+      p.e_scale = c->head_scale;
       p.partials = c->lm_part;
       p.logits = logits_out;
       p.vocab = g.vocab;
@@ -1051,14 +1073,16 @@ int run_lm_head(dg_ctx* c, float* logits_out, const int* done, cudaStream_t st) 
       p.done = done;
       const int grid = std::min(p.n_vtiles, c->sms);
       prof_before(DG_KERNEL_LM_HEAD, st);
+      const CUtensorMap& tx = f8h ? c->tm_xhq : c->tm_xn128;
+      const CUtensorMap& te = f8h ? c->tm_ehq : c->tm_embed;
       if (logits_out) {
-        DG_TRY(set_smem(lmhead_kernel<false>, kLmSmemBytes));
-        DG_TRY(launch_pdl(lmhead_kernel<false>, dim3(grid), dim3(kLmThreads), kLmSmemBytes, st,
-                          c->tm_xn128, c->tm_embed, p));
+        auto k = f8h ? lmhead_kernel<false, true> : lmhead_kernel<false, false>;
+        DG_TRY(set_smem(k, kLmSmemBytes));
+        DG_TRY(launch_pdl(k, dim3(grid), dim3(kLmThreads), kLmSmemBytes, st, tx, te, p));
       } else {
-        DG_TRY(set_smem(lmhead_kernel<true>, kLmSmemBytes));
-        DG_TRY(launch_pdl(lmhead_kernel<true>, dim3(grid), dim3(kLmThreads), kLmSmemBytes, st,
-                          c->tm_xn128, c->tm_embed, p));
+        auto k = f8h ? lmhead_kernel<true, true> : lmhead_kernel<true, false>;
+        DG_TRY(set_smem(k, kLmSmemBytes));
+        DG_TRY(launch_pdl(k, dim3(grid), dim3(kLmThreads), kLmSmemBytes, st, tx, te, p));
       }
       DG_LAUNCHED();
       prof_after(DG_KERNEL_LM_HEAD, st);
@@ -1108,6 +1132,11 @@ int bind_tmaps(dg_ctx* c) {
   const uint64_t vt_rows = static_cast<uint64_t>(c->batch) * g.n_layers * g.n_kv_heads * hd;
   DG_TRY(make_tmap(&c->tm_vt, c->vtc, vt_rows, g.kv_capacity, g.kv_capacity, 128));
   DG_TRY(make_tmap(&c->tm_embed, c->embed, g.vocab, d, d, 256));
+  if (g.lm_head_e4m3) {
+    const uint64_t hp = e4m3_pitch(g.d_model);
+    DG_TRY(make_tmap(&c->tm_xhq, c->xhq, static_cast<uint64_t>(g.canvas) * c->batch, d, hp, 128, 1));
+    DG_TRY(make_tmap(&c->tm_ehq, c->head_codes, g.vocab, d, hp, 256, 1));
+  }
   const int L = g.n_layers;
   c->tm_wqkv.resize(L);
   c->tm_wo.resize(L);
@@ -1188,6 +1217,9 @@ int dg_create(const dg_config* cfg, const dg_weights* w, void* d_kv, void* d_scr
   DG_TRY(check_config(cfg));
   if (!w || !w->embed || !w->final_norm || !w->layers || !d_kv || !d_scratch || !out)
     return fail(DG_ERR_INVALID_ARG, "null weights or buffers");
+  if (cfg->lm_head_e4m3 && (!w->head_codes || !w->head_scale ||
+                            reinterpret_cast<uintptr_t>(w->head_codes) % 16))
+    return fail(DG_ERR_INVALID_ARG, "lm_head_e4m3 needs 16-byte aligned head codes and scales");
   if (reinterpret_cast<uintptr_t>(d_kv) % 256 || reinterpret_cast<uintptr_t>(d_scratch) % 256)
     return fail(DG_ERR_INVALID_ARG, "kv and scratch must be 256-byte aligned");
   for (int l = 0; l < cfg->n_layers; ++l) {
@@ -1209,6 +1241,8 @@ int dg_create(const dg_config* cfg, const dg_weights* w, void* d_kv, void* d_scr
   c->layers.assign(w->layers, w->layers + cfg->n_layers);
   c->embed = w->embed;
   c->final_norm = w->final_norm;
+  c->head_codes = w->head_codes;
+  c->head_scale = w->head_scale;
   c->kv = static_cast<uint8_t*>(d_kv);
   c->scratch = static_cast<uint8_t*>(d_scratch);
   c->kv_len = 0;
@@ -1268,6 +1302,8 @@ int dg_create(const dg_config* cfg, const dg_weights* w, void* d_kv, void* d_scr
   c->hsq_scale = reinterpret_cast<float*>(s + p.off[B_HSQS]);
   c->w_perm = reinterpret_cast<float*>(s + p.off[B_WPERM]);
   c->commit_ids = reinterpret_cast<int32_t*>(s + p.off[B_COMMIT]);
+  c->xhq = s + p.off[B_XHQ];
+  c->xhs = reinterpret_cast<float*>(s + p.off[B_XHS]);
   c->x_sf = s + p.off[B_XSF];
   c->x_sh_sf = s + p.off[B_XSHSF];
   c->h_sf = s + p.off[B_HSF];

@@ -467,6 +467,9 @@ struct LmHeadParams {
   float* logits;          // debug: [n_tokens, vocab] when not null (statistics skipped)
   int vocab;
   float inv_t;            // 1 / sampling temperature: statistics of logits / T
+  // e4m3 head (kF8): per-row scales of the token codes [n_tokens] and of the vocabulary rows [V]
+  const float* x_scale;
+  const float* e_scale;
   int* err;
   const int* done;
 };
@@ -477,7 +480,10 @@ constexpr int kLmSmemBytes = kLmStages * kLmStageBytes + 1024 + 256;
 
 constexpr int kLmThreads = 64 + 32 * 8;  // TMA, MMA, two epilogue warpgroups (one per token tile)
 
-template <bool kStats>
+// kF8: tokens and vocabulary rows are e4m3 codes (kind::f8f6f4; a 128-byte K slab holds 128
+// codes, so the ring and descriptors are unchanged) and every accumulator is scaled by its
+// token's and its vocabulary row's scale before the statistics (or the debug logits).
+template <bool kStats, bool kF8 = false>
 __global__ void __launch_bounds__(kLmThreads, 1)
     lmhead_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_e,
                   const LmHeadParams p) {
@@ -533,10 +539,10 @@ __global__ void __launch_bounds__(kLmThreads, 1)
           }
           uint8_t* s0 = smem + stage * kLmStageBytes;
           mbar_arrive_expect_tx(&full[stage], n_ttiles * 16384 + 32768);
+          const int kx = kb * (kF8 ? 128 : 64);  // elements per 128-byte K slab
           for (int tt = 0; tt < n_ttiles; ++tt)
-            tma_load_2d(&tm_x, &full[stage], s0 + tt * 16384, kb * 64, p.tok_base + tt * 128,
-                        pol_x);
-          tma_load_2d(&tm_e, &full[stage], s0 + 32768, kb * 64, vt * 256, pol_e);
+            tma_load_2d(&tm_x, &full[stage], s0 + tt * 16384, kx, p.tok_base + tt * 128, pol_x);
+          tma_load_2d(&tm_e, &full[stage], s0 + 32768, kx, vt * 256, pol_e);
           if (++stage == kLmStages) {
             stage = 0;
             phase ^= 1u;
@@ -548,7 +554,7 @@ __global__ void __launch_bounds__(kLmThreads, 1)
     if (elect_one()) {
       int stage = 0;
       uint32_t phase = 0, acc_phase = 0;
-      const uint32_t idesc = idesc_bf16_f32(128, 256);
+      const uint32_t idesc = kF8 ? idesc_e4m3_f32(128, 256) : idesc_bf16_f32(128, 256);
       bool ok = true;
       for (int vt = blockIdx.x; vt < p.n_vtiles && ok; vt += gridDim.x) {
         if (!mbar_wait(acc_empty, acc_phase ^ 1u, p.err)) break;
@@ -564,9 +570,14 @@ __global__ void __launch_bounds__(kLmThreads, 1)
           for (int tt = 0; tt < n_ttiles; ++tt) {
             const uint64_t dx = sdesc_sw128(s0 + tt * 16384);
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-              umma_bf16(tmem_base + tt * 256, dx + 2 * k, de + 2 * k, idesc,
-                        (kb > 0 || k > 0) ? 1u : 0u);
+            for (int k = 0; k < 4; ++k) {
+              if constexpr (kF8)
+                umma_e4m3(tmem_base + tt * 256, dx + 2 * k, de + 2 * k, idesc,
+                          (kb > 0 || k > 0) ? 1u : 0u);
+              else
+                umma_bf16(tmem_base + tt * 256, dx + 2 * k, de + 2 * k, idesc,
+                          (kb > 0 || k > 0) ? 1u : 0u);
+            }
           }
           umma_commit(&empty[stage]);
           if (++stage == kLmStages) {
@@ -589,6 +600,21 @@ __global__ void __launch_bounds__(kLmThreads, 1)
       if (tt < n_ttiles) {
         const int tok = tt * 128 + r;
         const uint32_t t_row = tmem_base + tt * 256 + (static_cast<uint32_t>(q * 32) << 16);
+        // e4m3: accumulator (tok, column c) x x_scale[tok] x e_scale[vocab row of c]
+        const float xs = kF8 ? (tok < p.n_tokens ? p.x_scale[p.tok_base + tok] : 0.f) : 1.f;
+        const float* es = kF8 ? p.e_scale + vt * 256 : nullptr;
+        auto scale32 = [&](float (&v)[32], int c) {
+          if constexpr (kF8) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+              const float4 e4 = __ldg(reinterpret_cast<const float4*>(es + c + i));
+              v[i] *= xs * e4.x;
+              v[i + 1] *= xs * e4.y;
+              v[i + 2] *= xs * e4.z;
+              v[i + 3] *= xs * e4.w;
+            }
+          }
+        };
         if constexpr (kStats) {
           float m = -INFINITY;
           int a = 0;
@@ -596,6 +622,7 @@ __global__ void __launch_bounds__(kLmThreads, 1)
           for (int c = 0; c < 256; c += 32) {
             float v[32];
             tmem_ld32(t_row + c, v);
+            scale32(v, c);
             // tree argmax of the chunk, lowest index on equal values
             int idx[32];
 #pragma unroll
@@ -618,6 +645,7 @@ __global__ void __launch_bounds__(kLmThreads, 1)
           for (int c = 0; c < 256; c += 32) {
             float v[32];
             tmem_ld32(t_row + c, v);
+            scale32(v, c);
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
               const float d = (v[i] - m) * p.inv_t;
@@ -635,6 +663,7 @@ __global__ void __launch_bounds__(kLmThreads, 1)
           for (int c = 0; c < 256; c += 32) {
             float v[32];
             tmem_ld32(t_row + c, v);
+            scale32(v, c);
             if (tok < p.n_tokens) {
               float4* dst = reinterpret_cast<float4*>(
                   p.logits + static_cast<long long>(p.tok_base + tok) * p.vocab + vt * 256 + c);

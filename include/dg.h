@@ -115,6 +115,12 @@ typedef struct dg_config {
    * committed together once every canvas has stopped; a stopped canvas is frozen meanwhile), and
    * sequence b draws its Philox stream with key seed + b. */
   int32_t batch;
+  /* FP8 LM head (the FP8 weight format of [pl] applied to the tied head; bf16 dtypes only): the
+   * head multiplies e4m3 codes of the final normed tokens (quantised per row on the fly,
+   * scale = max|row| / 448) by an e4m3 copy of the embedding table with one fp32 scale per
+   * vocabulary row (dg_weights.head_codes / head_scale, written by dg_quantize_e4m3 at a pitch of
+   * DG_E4M3_PITCH(d)); the canvas embedding gather keeps the bf16 table.  0: bf16 head. */
+  int32_t lm_head_e4m3;
 } dg_config;
 
 /* Per-layer weights, all device pointers, dtype = config dtype unless noted (bf16 for
@@ -149,6 +155,8 @@ typedef struct dg_weights {
   const void* embed;              /* tied embedding / LM head [V, d] */
   const float* final_norm;        /* fp32 [d] */
   const dg_layer_weights* layers; /* HOST array of n_layers entries (copied by dg_create) */
+  const void* head_codes;         /* lm_head_e4m3: e4m3 codes of embed [V, DG_E4M3_PITCH(d)] */
+  const float* head_scale;        /* lm_head_e4m3: fp32 [V], one per vocabulary row */
 } dg_weights;
 
 /* Device-side decode state words (int32), readable by the caller after a block. */

@@ -33,6 +33,7 @@ from . import sampler as smp
 from .attention import attention
 from .moe import moe_ffn, moe_ffn_fp8, moe_ffn_nvfp4
 from .numerics import round_f32, round_storage
+from .quant import quantize_rows
 
 
 @dataclass
@@ -50,6 +51,7 @@ class ModelConfig:
     canvas: int = 256
     storage: str = "bf16"
     experts: str = "bf16"  # "fp8" / "nvfp4": quantised expert weights and activations (quant.py)
+    head: str = "bf16"     # "fp8": the LM head on e4m3 operands (lm_head_fp8)
     eps: float = 1e-6
     rope_theta: float = 10000.0
     tau: float = smp.TAU
@@ -156,7 +158,22 @@ def forward_tokens(cfg, weights, ids, positions, cache, causal, keep_info=False)
 def lm_head(cfg, weights, x):
     """Final norm then the tied LM head; logits rounded to fp32 like the GPU's accumulators."""
     xf = round_storage(rmsnorm(x, weights["final_norm"], cfg.eps), cfg.storage)
+    if cfg.head == "fp8":
+        return lm_head_fp8(xf, weights["embed"])
     return round_f32(xf @ np.asarray(weights["embed"], dtype=np.float64).T)
+
+
+def lm_head_fp8(xf, embed):
+    """The tied LM head with e4m3 operands (the FP8 weight format applied to the head; [pl] lists
+    FP8 weights, the pages give no scheme): the stored normed rows xf [T, d] and the embedding
+    rows [V, d] are each quantised per row (quant.quantize_rows: scale = max|row| / 448, codes
+    rounded to nearest even); the code products are summed and scaled by (token scale) x
+    (vocabulary-row scale); logits rounded to fp32."""
+    xq, xs = quantize_rows(xf)
+    eq, es = quantize_rows(embed)
+    acc = xq @ eq.T
+    return round_f32(acc * np.asarray(xs, dtype=np.float64)[:, None]
+                     * np.asarray(es, dtype=np.float64)[None, :])
 
 
 def denoise_logits(cfg, weights, canvas, cache, keep_info=False):

@@ -168,3 +168,90 @@ def test_e4m3_model_rejects_missing_scales():
     cfg = make_config(shape, kv_capacity=512, experts="e4m3")
     with pytest.raises(RuntimeError, match="scales"):
         DiffusionModel(cfg, w)
+
+
+# ---- the LM head on e4m3 operands (dg_config.lm_head_e4m3) ----------------------------------------
+
+@pytest.mark.parametrize("batch", [1, 2])
+def test_e4m3_lm_head_small_model(batch):
+    """The e4m3 head's logits (dg_debug_logits: the same MMA core and scaling as the fused
+    statistics) against the oracle's lm_head_fp8 on the GPU's own final hidden state; the fused
+    statistics and the sampler on the GPU's logits; one and two sequences."""
+    from block_text_diffusion_dg_b200 import DiffusionModel, make_config, quantize_head
+    shape = SHAPES["small_bf16"]
+    v, t = shape["vocab"], shape["canvas"]
+    w = model_weights("small_bf16", seed=31, norm_jitter=0.1)
+    wc = quantize_head(_to_cuda(w))
+    cfg = make_config(shape, kv_capacity=1024, fixed_steps=2, head="e4m3", batch=batch)
+    m = DiffusionModel(cfg, wc)
+    prompts = torch.stack([uniform_ids(96, v, seed=32 + b) for b in range(batch)])
+    m.kv_append(prompts.cuda())
+    m.canvas_init(7, 0)
+    m.denoise_step(1)
+    logits = np64(m.debug_logits())
+    m.sample_update(1)
+    bufs = m.buffers()
+    torch.cuda.synchronize()
+    x_final = np64(m.debug_hidden())
+    ocfg = om.ModelConfig(**{k: shape[k] for k in (
+        "n_layers", "d_model", "n_heads", "n_kv_heads", "head_dim", "n_experts", "top_k",
+        "expert_hidden", "shared_hidden", "vocab", "canvas", "storage")}, head="fp8")
+    ow = weights_to_np(w)
+    ref = om.lm_head(ocfg, ow, x_final)
+    err = np.max(np.abs(logits - ref))
+    assert err < 3e-2, err
+    # the quantisation acts: the bf16 head differs by more than the comparison's noise
+    ref16 = om.lm_head(om.ModelConfig(**{**ocfg.__dict__, "head": "bf16"}), ow, x_final)
+    assert np.max(np.abs(ref16 - ref)) > 5 * err
+    conf, ent, amax = osmp.row_stats(logits)
+    assert np.array_equal(bufs["argmax"].cpu().numpy(), amax)
+    assert np.max(np.abs(bufs["entropy"].cpu().numpy() - ent)) < 1e-5
+    g_canvas = bufs["canvas"].cpu().numpy().reshape(batch, t)
+    for b in range(batch):
+        rows = slice(b * t, (b + 1) * t)
+        nxt, _ = osmp.sample_update(conf[rows], amax[rows], 7 + b, 0, 1, v)
+        clear = np.abs(conf[rows] - 0.9) > 1e-4
+        assert np.array_equal(g_canvas[b][clear], nxt[clear])
+    m.commit_block()
+    m.check_device_status()
+    m.close()
+
+
+def test_e4m3_lm_head_full_vocabulary():
+    """One decoder layer of the full model's shapes with the 262,144-entry tied head in e4m3: the
+    head's codes bit-exact for sampled vocabulary rows, the logits of sampled (row, vocabulary)
+    entries against the oracle (tokens quantised from the GPU's own final hidden state), the
+    fused statistics of all 256 rows on the GPU's logits."""
+    from block_text_diffusion_dg_b200 import DiffusionModel, make_config, quantize_head
+    shape = dict(SHAPES["a4b"], n_layers=1)
+    v, d = shape["vocab"], shape["d_model"]
+    w = model_weights(shape, seed=41, device="cuda")
+    wc = quantize_head(w)
+    cfg = make_config(shape, kv_capacity=1024, fixed_steps=1, head="e4m3")
+    m = DiffusionModel(cfg, wc)
+    m.kv_append(uniform_ids(128, v, seed=42).cuda())
+    m.canvas_init(43, 0)
+    m.denoise_step(1)
+    logits = m.debug_logits()
+    m.sample_update(1)
+    bufs = m.buffers()
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(44)
+    vrows = np.sort(rng.choice(v, 2048, replace=False))
+    emb = npf32(w["embed"][torch.from_numpy(vrows).cuda()])
+    eq, es = quantize_rows(emb)
+    codes = wc["head_codes"][torch.from_numpy(vrows).cuda()].cpu().numpy()[:, :d]
+    assert _same_codes(codes, eq)
+    assert np.array_equal(wc["head_scale"][torch.from_numpy(vrows).cuda()].cpu().numpy(), es)
+    x_final = np64(m.debug_hidden())
+    rows = np.arange(0, 256, 17)
+    xf = om.rmsnorm(x_final[rows], npf32(w["final_norm"]), 1e-6)
+    from oracle.numerics import round_bf16
+    ref = om.lm_head_fp8(round_bf16(xf).astype(np.float64), emb)
+    got = np64(logits[torch.from_numpy(rows).cuda()][:, torch.from_numpy(vrows).cuda()])
+    assert np.max(np.abs(got - ref)) < 3e-2
+    conf, ent, amax = osmp.row_stats(np64(logits))
+    assert np.array_equal(bufs["argmax"].cpu().numpy(), amax)
+    assert np.max(np.abs(bufs["entropy"].cpu().numpy() - ent)) < 1e-5
+    m.check_device_status()
+    m.close()

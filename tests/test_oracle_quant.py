@@ -269,3 +269,43 @@ def test_nvfp4_moe_runs_and_routes_like_bf16():
     # 4-bit elements: the outputs agree to the format's precision, not to bf16's
     rel = np.linalg.norm(y4 - y16) / np.linalg.norm(y16)
     assert 1e-3 < rel < 0.25, rel
+
+
+# ---- the LM head on e4m3 operands ---------------------------------------------------------------
+
+def test_lm_head_fp8_equals_bf16_head_on_grid_operands():
+    # rows already on the e4m3 grid whose maximum is 448: quantisation is the identity (scale 1),
+    # so the fp8 head equals the plain product exactly
+    from oracle import model as om
+    from oracle.quant import e4m3_table
+    rng = np.random.default_rng(5)
+    grid = e4m3_table()
+    grid = grid[np.isfinite(grid) & (np.abs(grid) <= 448)]
+    xf = rng.choice(grid, (6, 64))
+    emb = rng.choice(grid, (40, 64))
+    xf[:, 0] = 448.0
+    emb[:, 3] = -448.0
+    got = om.lm_head_fp8(xf, emb)
+    assert np.array_equal(got, (xf @ emb.T).astype(np.float32).astype(np.float64))
+
+
+def test_lm_head_fp8_error_bound_and_planted_mistake():
+    from oracle import model as om
+    from oracle.quant import quantize_rows
+    rng = np.random.default_rng(6)
+    xf = rng.standard_normal((8, 96))
+    emb = rng.standard_normal((50, 96)) * 0.02
+    got = om.lm_head_fp8(xf, emb)
+    exact = xf @ emb.T
+    # each element moves by at most half an e4m3 step: 2^-4 relative to a normal value, plus the
+    # subnormal quantum (2^-9 of the row scale, halved) near zero
+    ex = np.abs(xf) * 2.0 ** -4 + np.max(np.abs(xf), 1, keepdims=True) / 448 * 2.0 ** -10
+    ee = np.abs(emb) * 2.0 ** -4 + np.max(np.abs(emb), 1, keepdims=True) / 448 * 2.0 ** -10
+    bound = (np.abs(xf) + ex) @ ee.T + ex @ np.abs(emb).T + 1e-12
+    assert np.all(np.abs(got - exact) <= bound)
+    assert np.max(np.abs(got - exact)) > 0  # the quantisation does act
+    # a dropped vocabulary-row scale does not pass the bound
+    xq, xs = quantize_rows(xf)
+    eq, es = quantize_rows(emb)
+    wrong = (xq @ eq.T) * xs[:, None]
+    assert not np.all(np.abs(wrong - exact) <= bound)
