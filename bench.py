@@ -61,7 +61,7 @@ def parse():
     ap.add_argument("--experts", choices=["bf16", "e4m3", "nvfp4"], default="bf16",
                     help="expert weight format of the decode model")
     ap.add_argument("--profile", choices=["decode_step", "decode_step_small", "decode_step_e4m3",
-                                          "moe", "moe_e4m3", "attention", "sampler"],
+                                          "moe", "moe_e4m3", "moe_nvfp4", "attention", "sampler"],
                     help="run one profiled region between cudaProfilerStart/Stop and exit "
                          "(for ncu --profile-from-start off); prints no JSON")
     return ap.parse_args()
@@ -634,6 +634,7 @@ def run_profile(args):
     decode_step_e4m3: decode_step with e4m3 experts.
     moe:         the MoE operator at 256 tokens, d 2816, 128 experts top-8 + shared (1.5 GB).
     moe_e4m3:    the same operator with e4m3 experts (0.8 GB of expert weights).
+    moe_nvfp4:   the same operator with NVFP4 experts (0.45 GB of expert weights).
     attention:   canvas attention, 16/8 heads x 128, 4096 + 256 keys.
     sampler:     the sampler on bf16 logits [256, 262144].
     """
@@ -685,6 +686,15 @@ def run_profile(args):
         call = lambda: dg.moe_ffn_e4m3(m["x"], m["wr"], q["w_gu"], q["w_gu_scale"], q["w_d"],
                                        q["w_d_scale"], 8, q["ws_gu"], q["ws_gu_scale"], q["ws_d"],
                                        q["ws_d_scale"], workspace=ws)
+    elif args.profile == "moe_nvfp4":
+        m = {k: (None if v is None else v.to(dev)) for k, v in moe_inputs(seed=0).items()}
+        q = {}
+        for name in ("w_gu", "w_d", "ws_gu", "ws_d"):
+            q[name] = dg.quantize_nvfp4(m[name])
+            m[name] = None
+        ws = dg.moe_workspace(256, 2816, 128, 8, 704, 2112, dev)
+        call = lambda: dg.moe_ffn_nvfp4(m["x"], m["wr"], q["w_gu"], q["w_d"], 8, q["ws_gu"],
+                                        q["ws_d"], workspace=ws)
     elif args.profile == "attention":
         q, k, v = (t.to(dev) for t in attention_inputs(seed=0))
         vt = v.transpose(1, 2).contiguous()
