@@ -206,12 +206,17 @@ int launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 
 // ---- GEMM launch helpers -----------------------------------------------------------------
 constexpr int kGroupN = 64, kGroupStages = 8;
-// Long passes (a prompt encoded at once, or a batch of canvases) give each expert many tokens:
-// there the grouped GEMMs take 256-token chunks, so each expert weight tile streams once per 256
-// tokens, not once per 64.  From 48 slots per expert on average, a good part of the experts would
-// need a second 64-token chunk (a second pass over their weights).
+// Passes that give each expert many tokens (a batch of canvases, a prompt encoded at once) take
+// wider token chunks, so each expert weight tile streams once per 128 or 256 tokens instead of
+// once per 64: from 48 slots per expert on average a good part of the experts would otherwise
+// need a second 64-token chunk (a second pass over their weights).  The 128-token instance keeps
+// six stages in flight; the 256-token one, for prompt passes, four.
+constexpr int kGroupMidN = 128, kGroupMidStages = 6;
 constexpr int kGroupWideN = 256, kGroupWideStages = 4;
-bool group_wide(long long n_slots, int n_experts) { return n_slots >= 48ll * n_experts; }
+int group_chunk(long long n_slots, int n_experts) {
+  if (n_slots < 48ll * n_experts) return kGroupN;
+  return n_slots < 160ll * n_experts ? kGroupMidN : kGroupWideN;
+}
 constexpr int kRouterChunk = 64;  // tokens per router cluster
 constexpr int kPrefetchExperts = 4;  // routed chunks whose expert weights the gather prefetches
 
@@ -283,19 +288,22 @@ int clu_splits(int tiles, int kb_total, int sms) {
   return std::max(1, std::min({kCluMaxSplits, kb_total, sms / std::max(1, tiles)}));
 }
 
-// Grouped expert GEMM with the token-chunk width the pass needs (see group_wide).  NVFP4 runs
+// Grouped expert GEMM with the token-chunk width the pass needs (see group_chunk).  NVFP4 runs
 // the 64-token instance only (its scale atoms are laid out per chunk of at most 128 rows).
 constexpr int kGroupFp4Stages = 7;
 template <int EPI, int FMT>
-int launch_grouped(bool wide, const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
+int launch_grouped(int nch, const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
                    int sms, cudaStream_t st, int kind, const CUtensorMap* ta2,
                    const CUtensorMap* tb2) {
   if constexpr (FMT == 2) {
     return launch_gemm<kGroupN, kGroupFp4Stages, EPI, FMT>(ta, tb, p, sms, st, kind, ta2, tb2);
   } else {
-    if (wide)
+    if (nch == kGroupWideN)
       return launch_gemm<kGroupWideN, kGroupWideStages, EPI, FMT>(ta, tb, p, sms, st, kind, ta2,
                                                                  tb2);
+    if (nch == kGroupMidN)
+      return launch_gemm<kGroupMidN, kGroupMidStages, EPI, FMT>(ta, tb, p, sms, st, kind, ta2,
+                                                               tb2);
     return launch_gemm<kGroupN, kGroupStages, EPI, FMT>(ta, tb, p, sms, st, kind, ta2, tb2);
   }
 }
@@ -349,16 +357,16 @@ long long operand_row_bytes(int fmt, int cols) {
 
 // The routed chunk width of a pass: 256-token chunks for long passes, except NVFP4 (64 always).
 int route_chunk(int fmt, long long n_slots, int n_experts) {
-  return fmt != 2 && group_wide(n_slots, n_experts) ? kGroupWideN : kGroupN;
+  return fmt != 2 ? group_chunk(n_slots, n_experts) : kGroupN;
 }
 
 template <int EPI>
-int launch_grouped_fmt(int fmt, bool wide, const CUtensorMap& ta, const CUtensorMap& tb,
+int launch_grouped_fmt(int fmt, int nch, const CUtensorMap& ta, const CUtensorMap& tb,
                        const GemmParams& p, int sms, cudaStream_t st, int kind,
                        const CUtensorMap* ta2, const CUtensorMap* tb2) {
-  if (fmt == 2) return launch_grouped<EPI, 2>(wide, ta, tb, p, sms, st, kind, ta2, tb2);
-  if (fmt == 1) return launch_grouped<EPI, 1>(wide, ta, tb, p, sms, st, kind, ta2, tb2);
-  return launch_grouped<EPI, 0>(wide, ta, tb, p, sms, st, kind, ta2, tb2);
+  if (fmt == 2) return launch_grouped<EPI, 2>(nch, ta, tb, p, sms, st, kind, ta2, tb2);
+  if (fmt == 1) return launch_grouped<EPI, 1>(nch, ta, tb, p, sms, st, kind, ta2, tb2);
+  return launch_grouped<EPI, 0>(nch, ta, tb, p, sms, st, kind, ta2, tb2);
 }
 
 // Quantise (e4m3 or NVFP4) up to two row segments: routed rows (optionally gathered by perm,
@@ -398,7 +406,6 @@ int launch_experts(const ExpertPass& e, int sms, cudaStream_t st) {
   const int n_slots = e.n * e.k;
   const bool shared = e.hs > 0;
   const int nch = route_chunk(e.fmt, n_slots, e.E);
-  const bool wide = nch == kGroupWideN;
   const int slab = 64 << e.fmt;  // K elements per 128-byte slab: 64 bf16, 128 e4m3, 256 e2m1
   const long long row_d = operand_row_bytes(e.fmt, e.d);
   const long long row_hs = operand_row_bytes(e.fmt, e.hs);
@@ -449,7 +456,7 @@ int launch_experts(const ExpertPass& e, int sms, cudaStream_t st) {
   p.err = e.err;
   p.done = e.done;
   const int kind_gu = e.profile ? DG_KERNEL_EXPERT_GATE_UP : -1;
-  DG_TRY(launch_grouped_fmt<kEpiGluBf16>(e.fmt, wide, *e.tm_wgu, *e.tm_xperm, p, sms, st, kind_gu,
+  DG_TRY(launch_grouped_fmt<kEpiGluBf16>(e.fmt, nch, *e.tm_wgu, *e.tm_xperm, p, sms, st, kind_gu,
                                          shared ? e.tm_wsgu : nullptr,
                                          shared ? e.tm_xsh : nullptr));
 
@@ -497,7 +504,7 @@ int launch_experts(const ExpertPass& e, int sms, cudaStream_t st) {
   q.err = e.err;
   q.done = e.done;
   const int kind_d = e.profile ? DG_KERNEL_EXPERT_DOWN : -1;
-  DG_TRY(launch_grouped_fmt<kEpiScatterF32>(e.fmt, wide, *e.tm_wd, *e.tm_h, q, sms, st, kind_d,
+  DG_TRY(launch_grouped_fmt<kEpiScatterF32>(e.fmt, nch, *e.tm_wd, *e.tm_h, q, sms, st, kind_d,
                                             shared ? e.tm_wsd : nullptr,
                                             shared ? e.tm_hs : nullptr));
   return DG_OK;
