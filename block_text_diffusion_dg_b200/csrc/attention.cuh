@@ -285,15 +285,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (key0 + i >= key_lim) x[i] = -INFINITY;
       }
       float mp;
-      {
-        float t[32];
+      {  // three-input maxima: 64 -> 22 -> 8 -> 3 -> 1
+        float t[22];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) t[i] = fmaxf(x[i], x[i + 32]);
+        for (int i = 0; i < 21; ++i) t[i] = fmax3(x[3 * i], x[3 * i + 1], x[3 * i + 2]);
+        t[21] = x[63];
 #pragma unroll
-        for (int w = 16; w >= 1; w >>= 1)
-#pragma unroll
-          for (int i = 0; i < w; ++i) t[i] = fmaxf(t[i], t[i + w]);
-        mp = t[0];
+        for (int i = 0; i < 7; ++i) t[i] = fmax3(t[3 * i], t[3 * i + 1], t[3 * i + 2]);
+        t[7] = t[21];
+        t[0] = fmax3(t[0], t[1], t[2]);
+        t[1] = fmax3(t[3], t[4], t[5]);
+        t[2] = fmaxf(t[6], t[7]);
+        mp = fmax3(t[0], t[1], t[2]);
       }
       // row maximum of the tile: my half and my partner's (raw scores, scale applied after)
       tmem_st1(xchg + 2 * st + half, mp);
@@ -339,14 +342,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // probabilities (bf16) of my 64 keys = slab `half` of the P buffer; 16-byte unit u of
       // row r's 128-byte line lands at unit u ^ (r % 8)
       uint8_t* pb = s_p + b * 2 * kAttnTile + half * kAttnTile + (r >> 3) * 1024 + (r & 7) * 128;
+      // e = 2^(x scale log2e - m): a masked key holds x = -inf, so e = 2^-inf = 0 (also when the
+      // whole tile is masked and m is still -inf, m then taken as 0)
       const float mr = (m_run == -INFINITY) ? 0.f : m_run;
-      float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      const float2 sc2 = make_float2(p.scale_log2, p.scale_log2), nm2 = make_float2(-mr, -mr);
+      float2 part[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                        make_float2(0.f, 0.f)};
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        float e = fast_exp2(fmaf(x[i], p.scale_log2, -mr));
-        if ((!full_tile && key0 + i >= key_lim) || m_run == -INFINITY) e = 0.f;
-        x[i] = e;
-        part[i & 7] += e;
+      for (int i = 0; i < 64; i += 2) {
+        const float2 t = __ffma2_rn(make_float2(x[i], x[i + 1]), sc2, nm2);
+        const float2 e = make_float2(fast_exp2(t.x), fast_exp2(t.y));
+        x[i] = e.x;
+        x[i + 1] = e.y;
+        part[(i >> 1) & 3] = __fadd2_rn(part[(i >> 1) & 3], e);
       }
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
@@ -358,8 +366,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         *reinterpret_cast<uint4*>(pb + ((u ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
-      const float rowsum = ((part[0] + part[1]) + (part[2] + part[3])) +
-                           ((part[4] + part[5]) + (part[6] + part[7]));
+      const float2 ps = __fadd2_rn(__fadd2_rn(part[0], part[1]), __fadd2_rn(part[2], part[3]));
+      const float rowsum = ps.x + ps.y;
       l_run = l_run * alpha + rowsum;
       fence_proxy_async_smem();
       tc_fence_before();

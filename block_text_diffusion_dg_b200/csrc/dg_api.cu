@@ -1596,34 +1596,28 @@ int dg_debug_layer(dg_ctx* ctx, int32_t layer, const float* d_x_in, float* d_x_o
 
 // ---- standalone sampler ----------------------------------------------------------------
 
-// The streaming sampler cuts rows into segments of kSamplerSpan columns (both dtypes).
-constexpr int kSamplerSpan = 8192;
+// The streaming sampler cuts rows into segments of stream_span<T>() columns (2048 for bf16, 1024
+// for fp32); the workspace holds one partial per segment at the finer of the two.
+static size_t sampler_segs_max(int vocab) { return cdiv(vocab, stream_span<float>()); }
 
 int dg_sampler_workspace_bytes(int32_t rows, int32_t vocab, size_t* bytes) {
   if (rows < 1 || rows > 1024 || vocab < 2 || vocab % 8 || !bytes)
     return fail(DG_ERR_INVALID_ARG, "need 1 <= rows <= 1024, vocab % 8 == 0");
-  const size_t segs = cdiv(vocab, kSamplerSpan);
-  *bytes = align256(rows * segs * sizeof(StatPartial)) + align256(rows * segs * 4) +
-           4 * align256(rows * 8) + 256;
+  *bytes = align256(rows * sampler_segs_max(vocab) * sizeof(StatPartial)) + 3 * align256(rows * 8) +
+           256;
   return DG_OK;
 }
 
-static void sampler_views(void* ws, int rows, int vocab, StatPartial** part, int32_t** piece_len,
-                          int32_t** prev, double** row_h, int32_t** locked, int32_t** ticket,
-                          int32_t** row_units) {
+static void sampler_views(void* ws, int rows, int vocab, StatPartial** part, int32_t** prev,
+                          double** row_h, int32_t** locked, int32_t** ticket) {
   uint8_t* b = static_cast<uint8_t*>(ws);
-  const size_t segs = cdiv(vocab, kSamplerSpan);
   *part = reinterpret_cast<StatPartial*>(b);
-  b += align256(rows * segs * sizeof(StatPartial));
-  *piece_len = reinterpret_cast<int32_t*>(b);
-  b += align256(rows * segs * 4);
+  b += align256(rows * sampler_segs_max(vocab) * sizeof(StatPartial));
   *prev = reinterpret_cast<int32_t*>(b);
   b += align256(rows * 8);
   *row_h = reinterpret_cast<double*>(b);
   b += align256(rows * 8);
   *locked = reinterpret_cast<int32_t*>(b);
-  b += align256(rows * 8);
-  *row_units = reinterpret_cast<int32_t*>(b);
   b += align256(rows * 8);
   *ticket = reinterpret_cast<int32_t*>(b);
 }
@@ -1653,12 +1647,12 @@ int dg_sampler_step(const void* d_logits, int32_t dtype, int32_t rows, int32_t v
   if (dtype != DG_DTYPE_BF16 && dtype != DG_DTYPE_FP32)
     return fail(DG_ERR_INVALID_ARG, "dtype must be bf16 or fp32");
   StatPartial* part;
-  int32_t *piece_len, *prev, *locked, *ticket, *row_units;
+  int32_t *prev, *locked, *ticket;
   double* row_h;
-  sampler_views(d_workspace, rows, vocab, &part, &piece_len, &prev, &row_h, &locked, &ticket,
-                &row_units);
+  sampler_views(d_workspace, rows, vocab, &part, &prev, &row_h, &locked, &ticket);
   cudaStream_t st = S(stream);
-  const int segs = cdiv(vocab, kSamplerSpan);
+  const bool bf16 = dtype == DG_DTYPE_BF16;
+  const int segs = cdiv(vocab, bf16 ? stream_span<__nv_bfloat16>() : stream_span<float>());
   SamplerArgs a{};
   a.partials = part;
   a.nsplit = segs;
@@ -1681,18 +1675,27 @@ int dg_sampler_step(const void* d_logits, int32_t dtype, int32_t rows, int32_t v
   a.state = d_state;
   a.ticket = ticket;
   a.n_seq = 1;
-  // one wave of resident CTAs, each streaming an equal run of segments
-  static const int grid_bf16 = resident_ctas(sampler_stream_kernel<__nv_bfloat16, 4>);
-  static const int grid_f32 = resident_ctas(sampler_stream_kernel<float, 8>);
+  // one wave of resident CTAs; each of their warps streams an equal run of segments, then one
+  // warp per row merges the row
+  static const int grid_bf16 = resident_ctas(sampler_stream_kernel<__nv_bfloat16>);
+  static const int grid_f32 = resident_ctas(sampler_stream_kernel<float>);
   const long long units = static_cast<long long>(rows) * segs;
-  const int grid = static_cast<int>(std::min<long long>(units, dtype == DG_DTYPE_BF16 ? grid_bf16 : grid_f32));
+  const int grid = static_cast<int>(std::min<long long>(cdiv(units, 8), bf16 ? grid_bf16 : grid_f32));
+  const long long workers = static_cast<long long>(grid) * 8;
   prof_before(DG_KERNEL_SAMPLER, st);
-  if (dtype == DG_DTYPE_BF16)
-    DG_TRY(launch_pdl(sampler_stream_kernel<__nv_bfloat16, 4>, dim3(grid), dim3(256), 0, st,
-                      static_cast<const __nv_bfloat16*>(d_logits), segs, a, row_units, piece_len));
-  else
-    DG_TRY(launch_pdl(sampler_stream_kernel<float, 8>, dim3(grid), dim3(256), 0, st,
-                      static_cast<const float*>(d_logits), segs, a, row_units, piece_len));
+  if (bf16) {
+    const auto* x = static_cast<const __nv_bfloat16*>(d_logits);
+    DG_TRY(launch_pdl(sampler_stream_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, st, x, segs, a));
+    DG_LAUNCHED();
+    DG_TRY(launch_pdl(sampler_stream_rows_kernel<__nv_bfloat16>, dim3(cdiv(rows, 8)), dim3(256), 0,
+                      st, x, segs, a, workers));
+  } else {
+    const auto* x = static_cast<const float*>(d_logits);
+    DG_TRY(launch_pdl(sampler_stream_kernel<float>, dim3(grid), dim3(256), 0, st, x, segs, a));
+    DG_LAUNCHED();
+    DG_TRY(launch_pdl(sampler_stream_rows_kernel<float>, dim3(cdiv(rows, 8)), dim3(256), 0, st, x,
+                      segs, a, workers));
+  }
   DG_LAUNCHED();
   prof_after(DG_KERNEL_SAMPLER, st);
   return DG_OK;

@@ -355,6 +355,14 @@ DG_DEV void named_barrier(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// The largest of three floats in one instruction (three-input max.f32; a NaN input is ignored
+// as by fmaxf).
+DG_DEV float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // 2^x on the special-function unit (approximate, flushes denormals).
 DG_DEV float fast_exp2(float x) {
   float y;
@@ -432,6 +440,14 @@ DG_DEV void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_depend
 DG_DEV void pdl_enter() {
   pdl_wait();
   pdl_launch_dependents();
+}
+
+// atomicAdd with acquire-release semantics at GPU scope: this thread's earlier writes are visible
+// before the update, and its later reads see what the writers of earlier updates released.
+DG_DEV int atomic_add_acq_rel(int* ptr, int v) {
+  int old;
+  asm volatile("atom.add.acq_rel.gpu.global.s32 %0, [%1], %2;" : "=r"(old) : "l"(ptr), "r"(v) : "memory");
+  return old;
 }
 
 // Early-out used by every kernel of a denoise step once the block has stopped.

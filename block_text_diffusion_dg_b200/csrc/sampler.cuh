@@ -33,27 +33,11 @@ struct StatPartial {  // 16 bytes: m, S, U, argmax (int bits)
   int a;
 };
 
-// Merge two statistics; on equal maxima the lower argmax wins (lowest-index rule).
+// Merged statistics of a row in fp64 (relative to the row maximum m).
 struct StatD {
   double m, s, u;
   int a;
 };
-DG_DEV StatD stat_merge(const StatD& x, const StatD& y) {
-  if (y.s == 0.0) return x;
-  if (x.s == 0.0) return y;
-  StatD r;
-  if (x.m > y.m || (x.m == y.m && x.a < y.a)) {
-    r.m = x.m;
-    r.a = x.a;
-  } else {
-    r.m = y.m;
-    r.a = y.a;
-  }
-  const double ex = exp(x.m - r.m), ey = exp(y.m - r.m);
-  r.s = ex * x.s + ey * y.s;
-  r.u = ex * (x.u + (x.m - r.m) * x.s) + ey * (y.u + (y.m - r.m) * y.s);
-  return r;
-}
 
 // Canvas fill of n_seq canvases of t positions: canvas b takes the Philox stream keyed by seed + b
 // ([canvas] step 2: ids uniform over the vocabulary), with counter (position, 0, block, 0).  The
@@ -269,11 +253,20 @@ DG_DEV SamplerArgs seq_view(const SamplerArgs& p, int b) {
   return q;
 }
 
-// Decide lock / re-noise for one row from its merged statistics and write the row's outputs;
-// returns (in every thread) whether this CTA is the last row to finish the step.
-DG_DEV bool sampler_row_finish(const SamplerArgs& p, int row, const StatD& r) {
-  __shared__ int is_last;
-  if (threadIdx.x == 0) {
+// The id a re-noised position takes: the Philox draw of (position, step, block, tag 1).
+DG_DEV int32_t renoise_id(const SamplerArgs& p, int row) {
+  return canvas_uniform_id(p.seed, p.block, p.step, static_cast<uint32_t>(row), 1u,
+                           static_cast<uint32_t>(p.vocab));
+}
+
+// Decide lock / re-noise for one row from its merged statistics (valid in lane 0) and write the
+// row's outputs; returns (in every lane) whether this warp is the last row to finish the step.
+// `noise` is the row's re-noise id when the caller drew it already (negative: drawn here).  The
+// completion ticket is taken with one acquire-release atomic: this row's outputs are visible
+// before it, and the last row sees every other row's outputs after it.
+DG_DEV bool sampler_row_finish(const SamplerArgs& p, int row, const StatD& r, int32_t noise = -1) {
+  int is_last = 0;
+  if (lane_id() == 0) {
     const double conf = 1.0 / r.s;
     const double h = log(r.s) - r.u / r.s;
     p.conf[row] = static_cast<float>(conf);
@@ -284,15 +277,12 @@ DG_DEV bool sampler_row_finish(const SamplerArgs& p, int row, const StatD& r) {
     const bool kept = p.sticky != 0 && p.locked[row] != 0;
     p.argmax[row] = r.a;
     p.locked[row] = (lock || kept) ? 1 : 0;
-    if (!kept)
-      p.canvas[row] = lock ? r.a
-                           : canvas_uniform_id(p.seed, p.block, p.step, static_cast<uint32_t>(row),
-                                               1u, static_cast<uint32_t>(p.vocab));
-    __threadfence();
-    is_last = (atomicAdd(p.ticket, 1) == p.rows - 1);
+    if (!kept) p.canvas[row] = lock ? r.a : (noise >= 0 ? noise : renoise_id(p, row));
+    is_last = (atomic_add_acq_rel(p.ticket, 1) == p.rows - 1);
   }
-  __syncthreads();
-  return is_last;
+  is_last = __shfl_sync(0xffffffffu, is_last, 0);
+  __syncwarp();
+  return is_last != 0;
 }
 
 // Committed ids with sticky locks: a locked position's canvas token, otherwise the argmax.
@@ -303,90 +293,118 @@ __global__ void commit_ids_kernel(const int32_t* canvas, const int32_t* argmax,
   if (i < n) out[i] = locked[i] ? canvas[i] : argmax[i];
 }
 
-// Merge one row's nsplit partials (block-wide, fp64 tree) and finish the row.
-DG_DEV bool sampler_row(const SamplerArgs& p, int row) {
-  StatD acc{0.0, 0.0, 0.0, 0x7fffffff};
-  for (int i = threadIdx.x; i < p.nsplit; i += blockDim.x) {
-    const float4 q4 = __ldcg(reinterpret_cast<const float4*>(p.partials) +
-                             static_cast<size_t>(row) * p.nsplit + i);
-    acc = stat_merge(acc, StatD{q4.x, q4.y, q4.z, __float_as_int(q4.w)});
+// Merge one row's nsplit partials with a 256-thread CTA, the row maximum M first (so the fp64
+// exponentials are independent, with no dependent chain), then S = sum e^(m_i - M) S_i and
+// U = sum e^(m_i - M) (U_i + (m_i - M) S_i); the argmax is the lowest index among the partials
+// holding M.  Thread t takes partials t, t + 256, ...; the warps' maxima and then their sums
+// combine through shared memory in warp order.  Valid in thread 0.
+DG_DEV StatD sampler_row(const SamplerArgs& p, int row) {
+  __shared__ float s_max[8];
+  __shared__ double s_sum[2][8];
+  __shared__ int s_arg[8];
+  const float4* part = reinterpret_cast<const float4*>(p.partials) + static_cast<size_t>(row) * p.nsplit;
+  const int tid = static_cast<int>(threadIdx.x), warp = tid >> 5;
+  constexpr int kC = 4;  // partials per thread held in registers (nsplit <= 1024)
+  float4 q[kC];
+#pragma unroll
+  for (int k = 0; k < kC; ++k) {
+    const int i = tid + 256 * k;
+    q[k] = i < p.nsplit ? __ldcg(part + i) : make_float4(-INFINITY, 0.f, 0.f, 0.f);
   }
-  __shared__ StatD red[256];
-  red[threadIdx.x] = acc;
+  float m = -INFINITY;
+#pragma unroll
+  for (int k = 0; k < kC; ++k)
+    if (q[k].y > 0.f) m = fmaxf(m, q[k].x);
+  for (int i = tid + 256 * kC; i < p.nsplit; i += 256) {
+    const float4 q4 = __ldcg(part + i);
+    if (q4.y > 0.f) m = fmaxf(m, q4.x);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane_id() == 0) s_max[warp] = m;
   __syncthreads();
-  for (int o = blockDim.x / 2; o > 0; o >>= 1) {
-    if (threadIdx.x < o) red[threadIdx.x] = stat_merge(red[threadIdx.x], red[threadIdx.x + o]);
-    __syncthreads();
-  }
-  return sampler_row_finish(p, row, red[0]);
-}
-
-// Merge one row's pieces in column order: the piece starting at segment s keeps its partial at
-// slot row * segs + s and its length in segments at the same slot of piece_len.
-DG_DEV bool sampler_row_pieces(const SamplerArgs& p, int row, int segs,
-                               const int32_t* piece_len) {
-  // every slot of the row in one parallel round trip (slots that start no piece hold stale
-  // values and are never visited), then thread 0 follows the chain from segment 0
-  constexpr int kMaxSegs = 256;
-  __shared__ float4 sp[kMaxSegs];
-  __shared__ int sl[kMaxSegs];
-  __shared__ StatD merged;
-  for (int i = threadIdx.x; i < segs && i < kMaxSegs; i += blockDim.x) {
-    const size_t slot = static_cast<size_t>(row) * segs + i;
-    sp[i] = __ldcg(reinterpret_cast<const float4*>(p.partials) + slot);
-    sl[i] = __ldcg(piece_len + slot);
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    StatD acc{0.0, 0.0, 0.0, 0x7fffffff};
-    for (int s = 0; s < segs;) {
-      float4 q4;
-      int len;
-      if (s < kMaxSegs) {
-        q4 = sp[s];
-        len = sl[s];
-      } else {
-        const size_t slot = static_cast<size_t>(row) * segs + s;
-        q4 = __ldcg(reinterpret_cast<const float4*>(p.partials) + slot);
-        len = __ldcg(piece_len + slot);
+  m = s_max[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) m = fmaxf(m, s_max[w]);
+  double sum = 0.0, usum = 0.0;
+  int a = 0x7fffffff;
+  if (m != -INFINITY) {
+    auto add = [&](const float4& q4) {
+      if (q4.y > 0.f) {
+        const double d = static_cast<double>(q4.x) - static_cast<double>(m);
+        const double e = exp(d);
+        sum += e * q4.y;
+        usum += e * (static_cast<double>(q4.z) + d * q4.y);
+        if (q4.x == m) a = min(a, __float_as_int(q4.w));
       }
-      acc = stat_merge(acc, StatD{q4.x, q4.y, q4.z, __float_as_int(q4.w)});
-      s += max(1, len);
-    }
-    merged = acc;
+    };
+#pragma unroll
+    for (int k = 0; k < kC; ++k) add(q[k]);
+    for (int i = tid + 256 * kC; i < p.nsplit; i += 256) add(__ldcg(part + i));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    usum += __shfl_xor_sync(0xffffffffu, usum, o);
+    a = min(a, __shfl_xor_sync(0xffffffffu, a, o));
+  }
+  if (lane_id() == 0) {
+    s_sum[0][warp] = sum;
+    s_sum[1][warp] = usum;
+    s_arg[warp] = a;
   }
   __syncthreads();
-  return sampler_row_finish(p, row, merged);
+  StatD r{static_cast<double>(m), 0.0, 0.0, 0x7fffffff};
+  if (tid == 0)
+    for (int w = 0; w < 8; ++w) {
+      r.s += s_sum[0][w];
+      r.u += s_sum[1][w];
+      r.a = min(r.a, s_arg[w]);
+    }
+  return r;
 }
 
-// The stop test over the whole canvas, run by the last row's CTA (after a fence).  Rows written
-// by other CTAs are read through L2 (ld.global.cg); the mean entropy is a fixed-shape fp64 tree
-// over the rows, so it does not depend on timing.  rows <= 1024.
+// The stop test over one canvas, run by the warp that finished its last row (after a fence).
+// Rows written by other warps are read through L2 (ld.global.cg), eight rows per lane per batch so
+// that the loads of a batch are in flight together; the mean entropy is a fixed-shape fp64 sum
+// (per lane in row order, then a butterfly whose lane-0 result is used), so it does not depend on
+// timing.  Each lane then stores its rows' argmax as the previous argmax of the next step.
 DG_DEV void sampler_stop_test(const SamplerArgs& p) {
   __threadfence();
-  __shared__ double hs[256];
-  __shared__ int n_diff, n_locked;
-  if (threadIdx.x == 0) {
-    n_diff = 0;
-    n_locked = 0;
+  constexpr int kBatch = 8;
+  const int lane = static_cast<int>(lane_id());
+  double h = 0.0;
+  int n_diff = 0, n_locked = 0;
+  for (int base = 0; base < p.rows; base += 32 * kBatch) {
+    int am[kBatch], pv[kBatch], lk[kBatch];
+    double hh[kBatch];
+#pragma unroll
+    for (int k = 0; k < kBatch; ++k) {
+      const int i = base + lane + 32 * k;
+      if (i < p.rows) {
+        am[k] = __ldcg(p.argmax + i);
+        pv[k] = p.prev_argmax[i];
+        lk[k] = __ldcg(p.locked + i);
+        hh[k] = __ldcg(p.row_h + i);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kBatch; ++k) {
+      const int i = base + lane + 32 * k;
+      if (i < p.rows) {
+        n_diff += am[k] != pv[k];
+        n_locked += lk[k];
+        h += hh[k];
+        p.prev_argmax[i] = am[k];
+      }
+    }
   }
-  double h_part = 0.0;
-  int my_diff = 0, my_locked = 0;
-  for (int i = threadIdx.x; i < p.rows; i += blockDim.x) {
-    my_diff += (__ldcg(p.argmax + i) != p.prev_argmax[i]);
-    my_locked += __ldcg(p.locked + i);
-    h_part += __ldcg(p.row_h + i);
-  }
-  hs[threadIdx.x] = h_part;
-  __syncthreads();
-  atomicAdd(&n_diff, my_diff);
-  atomicAdd(&n_locked, my_locked);
-  for (int o = 128; o > 0; o >>= 1) {
-    if (threadIdx.x < o) hs[threadIdx.x] += hs[threadIdx.x + o];
-    __syncthreads();
-  }
-  if (threadIdx.x == 0) {
-    const double hbar = hs[0] / p.rows;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) h += __shfl_xor_sync(0xffffffffu, h, o);
+  n_diff = __reduce_add_sync(0xffffffffu, n_diff);
+  n_locked = __reduce_add_sync(0xffffffffu, n_locked);
+  if (lane == 0) {
+    const double hbar = h / p.rows;
     const int step = static_cast<int>(p.step);
     const bool stop_now = step >= 2 && hbar < static_cast<double>(p.h_bound) && n_diff == 0;
     int32_t* st = p.state;
@@ -402,259 +420,315 @@ DG_DEV void sampler_stop_test(const SamplerArgs& p) {
     }
     *p.ticket = 0;
   }
-  __syncthreads();
-  for (int i = threadIdx.x; i < p.rows; i += blockDim.x) p.prev_argmax[i] = __ldcg(p.argmax + i);
 }
 
-// One CTA per row of the n_seq canvases: merge the row's partials, decide lock / re-noise; the
-// last CTA of a canvas to finish evaluates the stop rule for that canvas (no CTA ever waits on
-// another).  A canvas that has stopped is left as it is while the others go on.
+// One CTA per row of the n_seq canvases: merge the row's partials, decide lock / re-noise (warp 0);
+// the last row of a canvas to finish evaluates the stop rule for that canvas (no CTA ever waits
+// on another).  A canvas that has stopped is left as it is while the others go on.
 __global__ void __launch_bounds__(256) sampler_merge_kernel(SamplerArgs p) {
   pdl_enter();
   const int b = blockIdx.x / p.rows;
   const SamplerArgs q = seq_view(p, b);
   if (block_done(q.state + kStDone)) return;
-  if (sampler_row(q, blockIdx.x - b * p.rows)) sampler_stop_test(q);
+  const int row = blockIdx.x - b * p.rows;
+  const StatD r = sampler_row(q, row);
+  if (threadIdx.x < 32 && sampler_row_finish(q, row, r)) sampler_stop_test(q);
 }
 
-// (m, S, U, a) <- merge with (m2, S2, U2, a2) in fp32 (2^x on the special-function unit); an
-// empty side (S = 0) is ignored; equal maxima keep the lower argmax.
-DG_DEV void stat_merge_f32(float& m, float& s, float& u, int& a, float m2, float s2, float u2,
-                           int a2) {
-  constexpr float kLog2e = 1.4426950408889634f;
-  if (s2 == 0.f) return;
-  if (s == 0.f) {
-    m = m2;
-    s = s2;
-    u = u2;
-    a = a2;
-    return;
-  }
-  const float mm = fmaxf(m, m2);
-  const int aa = (m > m2 || (m == m2 && a < a2)) ? a : a2;
-  const float d1 = m - mm, d2 = m2 - mm;
-  const float e1 = fast_exp2(d1 * kLog2e), e2 = fast_exp2(d2 * kLog2e);
-  u = e1 * (u + d1 * s) + e2 * (u2 + d2 * s2);
-  s = e1 * s + e2 * s2;
-  m = mm;
-  a = aa;
-}
+// ---- the standalone streaming sampler -------------------------------------------------------
+// One warp streams a row slice in groups of kLoads 16-byte vectors per lane: column
+// g + (l * 32 + lane) * kVec + j of the group starting at g (a group is a contiguous run of
+// columns).  Per group a lane takes the group maximum first; when it exceeds the lane's running
+// maximum m, the lane's S and U are rescaled to it and the group's start is remembered.  Then
+//   d = x - m,  e = 2^(d log2 e),  S += e,  U += e d      (pairs in f32x2 arithmetic).
+// The slice's maximum first occurs in the lowest of the remembered groups of the lanes holding
+// it; the slice reports that group's start in place of a column, and the row's merge looks for
+// the exact column in that one group.  A logit below -1e30 (a masked, -inf entry) is raised to
+// -1e30 first, so e = 0 and e d = 0 instead of NaN; a row needs some logit above -1e30.
+constexpr float kMaskedLogit = -1e30f;
 
-// Streaming statistics of one row slice for a 256-thread CTA.  Every thread walks its columns in
-// groups of kLoads 16-byte vectors (column c0 + ((g * kLoads + l) * 256 + tid) * kVec + j,
-// increasing in (g, l, j)) keeping running (m, S, T, a) with T = sum e t, t = (x - m) log2 e,
-// e = 2^t (so U = T / log2 e) and a the first column holding m; S and T are rescaled only when a
-// group raises the maximum, which is also the only time the group is searched for its first
-// maximal column.  The CTA merge rescales every thread's sums once to the CTA maximum and adds
-// them up; the argmax is the lowest column among the threads holding that maximum.  Thread 0
-// returns the result.
-template <typename T> DG_DEV void to_f32x8(const uint4& raw, float (&v)[16 / sizeof(T)]);
-template <> DG_DEV void to_f32x8<__nv_bfloat16>(const uint4& raw, float (&v)[8]) {
-  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+template <typename T, int kLoads>
+DG_DEV void warp_load_group(const T* base, int g, int c1, uint4 (&r)[kLoads]) {
+  constexpr int kVec = 16 / static_cast<int>(sizeof(T));
+  const int lane = static_cast<int>(lane_id());
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    v[2 * q] = __uint_as_float(w[q] << 16);
-    v[2 * q + 1] = __uint_as_float(w[q] & 0xffff0000u);
+  for (int l = 0; l < kLoads; ++l) {
+    const int c = g + (l * 32 + lane) * kVec;
+    if (c < c1)
+      r[l] = __ldcs(reinterpret_cast<const uint4*>(base + c));
+    else if constexpr (sizeof(T) == 2)
+      r[l] = make_uint4(0xff80ff80u, 0xff80ff80u, 0xff80ff80u, 0xff80ff80u);  // bf16 -inf
+    else
+      r[l] = make_uint4(0xff800000u, 0xff800000u, 0xff800000u, 0xff800000u);  // fp32 -inf
   }
 }
-template <> DG_DEV void to_f32x8<float>(const uint4& raw, float (&v)[4]) {
-  v[0] = __uint_as_float(raw.x);
-  v[1] = __uint_as_float(raw.y);
-  v[2] = __uint_as_float(raw.z);
-  v[3] = __uint_as_float(raw.w);
+
+// value j (0 .. kVec-1) of a 16-byte vector as f32
+template <typename T>
+DG_DEV float vec_value(const uint4& v, int j) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  if constexpr (sizeof(T) == 2)
+    return __uint_as_float((j & 1) ? (w[j >> 1] & 0xffff0000u) : (w[j >> 1] << 16));
+  else
+    return __uint_as_float(w[j]);
 }
 
 template <typename T, int kLoads>
-DG_DEV StatPartial stream_slice_stats(const T* base, int c0, int c1) {
-  constexpr int kVec = 16 / sizeof(T);
-  constexpr int kSpan = kLoads * 256 * kVec;  // columns per group over the CTA
-  constexpr float kLog2e = 1.4426950408889634f;
-  const int tid = threadIdx.x;
-  float m = -INFINITY;
-  float2 s2 = make_float2(0.f, 0.f), t2 = make_float2(0.f, 0.f);
-  int a = 0x7fffffff;
-  for (int g0 = c0; g0 < c1; g0 += kSpan) {
-    const bool full = g0 + kSpan <= c1;
-    uint4 raw[kLoads];
+DG_DEV float group_max(const uint4 (&r)[kLoads]) {
+  if constexpr (sizeof(T) == 2) {
+    __nv_bfloat162 ml[kLoads];
 #pragma unroll
     for (int l = 0; l < kLoads; ++l) {
-      const int c = g0 + (l * 256 + tid) * kVec;
-      if (full || c < c1) {
-        raw[l] = __ldcs(reinterpret_cast<const uint4*>(base + c));
-      } else if constexpr (sizeof(T) == 2) {
-        raw[l] = make_uint4(0xff80ff80u, 0xff80ff80u, 0xff80ff80u, 0xff80ff80u);  // bf16 -inf
-      } else {
-        raw[l] = make_uint4(0xff800000u, 0xff800000u, 0xff800000u, 0xff800000u);  // fp32 -inf
-      }
+      const __nv_bfloat162* w = reinterpret_cast<const __nv_bfloat162*>(&r[l]);
+      ml[l] = __hmax2(__hmax2(w[0], w[1]), __hmax2(w[2], w[3]));
     }
-    // group maximum (packed bf16 pairs for bf16 input); -inf padding never wins
-    float gm;
+#pragma unroll
+    for (int st = 1; st < kLoads; st *= 2)
+#pragma unroll
+      for (int l = 0; l + st < kLoads; l += 2 * st) ml[l] = __hmax2(ml[l], ml[l + st]);
+    return fmaxf(__low2float(ml[0]), __high2float(ml[0]));
+  } else {
+    float ml[kLoads];
+#pragma unroll
+    for (int l = 0; l < kLoads; ++l)
+      ml[l] = fmaxf(fmaxf(__uint_as_float(r[l].x), __uint_as_float(r[l].y)),
+                    fmaxf(__uint_as_float(r[l].z), __uint_as_float(r[l].w)));
+#pragma unroll
+    for (int st = 1; st < kLoads; st *= 2)
+#pragma unroll
+      for (int l = 0; l + st < kLoads; l += 2 * st) ml[l] = fmaxf(ml[l], ml[l + st]);
+    return ml[0];
+  }
+}
+
+template <typename T, int kLoads>
+DG_DEV void group_accumulate(const uint4 (&r)[kLoads], float m, float2& s2, float2& u2) {
+  constexpr float kLog2e = 1.4426950408889634f;
+  const float2 nm2 = make_float2(-m, -m), l2 = make_float2(kLog2e, kLog2e);
+#pragma unroll
+  for (int l = 0; l < kLoads; ++l) {
+    const uint32_t w4[4] = {r[l].x, r[l].y, r[l].z, r[l].w};
     if constexpr (sizeof(T) == 2) {
-      __nv_bfloat162 mx = *reinterpret_cast<const __nv_bfloat162*>(&raw[0].x);
+      const __nv_bfloat162 lo2 = __float2bfloat162_rn(kMaskedLogit);
 #pragma unroll
-      for (int l = 0; l < kLoads; ++l) {
-        const uint32_t w[4] = {raw[l].x, raw[l].y, raw[l].z, raw[l].w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) mx = __hmax2(mx, *reinterpret_cast<const __nv_bfloat162*>(&w[q]));
+      for (int q = 0; q < 4; ++q) {
+        const __nv_bfloat162 c = __hmax2(*reinterpret_cast<const __nv_bfloat162*>(&w4[q]), lo2);
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(&c);
+        const float2 x = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+        const float2 d = __fadd2_rn(x, nm2);
+        const float2 t = __fmul2_rn(d, l2);
+        const float2 e = make_float2(fast_exp2(t.x), fast_exp2(t.y));
+        s2 = __fadd2_rn(s2, e);
+        u2 = __ffma2_rn(e, d, u2);
       }
-      gm = fmaxf(__low2float(mx), __high2float(mx));
     } else {
-      gm = -INFINITY;
 #pragma unroll
-      for (int l = 0; l < kLoads; ++l)
-        gm = fmaxf(fmaxf(__uint_as_float(raw[l].x), __uint_as_float(raw[l].y)),
-                   fmaxf(fmaxf(__uint_as_float(raw[l].z), __uint_as_float(raw[l].w)), gm));
+      for (int q = 0; q < 4; q += 2) {
+        const float2 x = make_float2(fmaxf(__uint_as_float(w4[q]), kMaskedLogit),
+                                     fmaxf(__uint_as_float(w4[q + 1]), kMaskedLogit));
+        const float2 d = __fadd2_rn(x, nm2);
+        const float2 t = __fmul2_rn(d, l2);
+        const float2 e = make_float2(fast_exp2(t.x), fast_exp2(t.y));
+        s2 = __fadd2_rn(s2, e);
+        u2 = __ffma2_rn(e, d, u2);
+      }
     }
+  }
+}
+
+// Statistics (m, S, U, g) of columns [c0, c1) of one row for one warp, g the start of the lowest
+// group holding the maximum (every lane gets the same g; S and U are valid in lane 0).
+template <typename T, int kLoads>
+DG_DEV StatPartial warp_slice_stats(const T* base, int c0, int c1) {
+  constexpr int kVec = 16 / static_cast<int>(sizeof(T));
+  constexpr int kSpan = kLoads * 32 * kVec;
+  constexpr float kLog2e = 1.4426950408889634f;
+  float m = -INFINITY;
+  float2 s2 = make_float2(0.f, 0.f), u2 = make_float2(0.f, 0.f);
+  int gidx = c0;
+  for (int g = c0; g < c1; g += kSpan) {
+    uint4 r[kLoads];
+    warp_load_group<T, kLoads>(base, g, c1, r);
+    const float gm = group_max<T, kLoads>(r);
     if (gm > m) {  // strict: an earlier group keeps an equal maximum
+      gidx = g;
       if (m != -INFINITY) {
-        const float dt = (m - gm) * kLog2e;  // t shifts by dt for every earlier term
-        const float sc = fast_exp2(dt);
-        t2 = make_float2(sc * (t2.x + dt * s2.x), sc * (t2.y + dt * s2.y));
+        const float d = m - gm;
+        const float sc = fast_exp2(d * kLog2e);
+        u2 = make_float2(sc * (u2.x + d * s2.x), sc * (u2.y + d * s2.y));
         s2 = make_float2(sc * s2.x, sc * s2.y);
       }
       m = gm;
-      // first column of this group holding the new maximum (columns increase with l, then j)
-      int found = 0x7fffffff;
-#pragma unroll
-      for (int l = kLoads - 1; l >= 0; --l) {
-        float v[kVec];
-        to_f32x8<T>(raw[l], v);
-#pragma unroll
-        for (int j = kVec - 1; j >= 0; --j)
-          if (v[j] == gm) found = g0 + (l * 256 + tid) * kVec + j;
-      }
-      a = found;
     }
-    // t = (x - m) log2 e with the subtraction first, so the maximum's own term is exactly 2^0
-    const float2 l2 = make_float2(kLog2e, kLog2e);
-    const float2 nm2 = make_float2(-m, -m);
-    if (full) {
-#pragma unroll
-      for (int l = 0; l < kLoads; ++l) {
-        float v[kVec];
-        to_f32x8<T>(raw[l], v);
-#pragma unroll
-        for (int j = 0; j < kVec; j += 2) {
-          float2 t = fmul2(fadd2(make_float2(v[j], v[j + 1]), nm2), l2);
-          // -inf logits: t = -inf (or NaN while m is still -inf) becomes -1e30, so e = 0 and
-          // e * t = 0 instead of NaN
-          t = make_float2(fmaxf(t.x, kMaskedDelta), fmaxf(t.y, kMaskedDelta));
-          const float2 e = make_float2(fast_exp2(t.x), fast_exp2(t.y));
-          s2 = fadd2(s2, e);
-          t2 = ffma2(e, t, t2);
-        }
-      }
-    } else {  // ragged end of the row: -inf padding contributes nothing (and no 0 * -inf)
-#pragma unroll
-      for (int l = 0; l < kLoads; ++l) {
-        float v[kVec];
-        to_f32x8<T>(raw[l], v);
-#pragma unroll
-        for (int j = 0; j < kVec; ++j)
-          if (v[j] != -INFINITY) {
-            const float t = (v[j] - m) * kLog2e;
-            const float e = fast_exp2(t);
-            s2.x += e;
-            t2.x = fmaf(e, t, t2.x);
-          }
-      }
-    }
+    if (m != -INFINITY) group_accumulate<T, kLoads>(r, m, s2, u2);
   }
-  float s = s2.x + s2.y, tt = t2.x + t2.y;
-  // CTA maximum
-  const int warp = tid >> 5;
-  __shared__ float wmax[8];
-  __shared__ float wsum[2][8];
-  __shared__ int warg[8];
+  float s = s2.x + s2.y, u = u2.x + u2.y;
+  // the warp maximum, every lane's sums relative to it, then plain sums
   float bm = m;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
-  if (lane_id() == 0) wmax[warp] = bm;
-  __syncthreads();
-  bm = wmax[0];
-#pragma unroll
-  for (int w = 1; w < 8; ++w) bm = fmaxf(bm, wmax[w]);
-  // every thread's sums relative to the CTA maximum, then plain sums; argmax = lowest column
-  // among the threads that hold the maximum
   if (m == -INFINITY || bm == -INFINITY) {
     s = 0.f;
-    tt = 0.f;
+    u = 0.f;
   } else if (m != bm) {
-    const float dt = (m - bm) * kLog2e;
-    const float sc = fast_exp2(dt);
-    tt = sc * (tt + dt * s);
+    const float d = m - bm;
+    const float sc = fast_exp2(d * kLog2e);
+    u = sc * (u + d * s);
     s *= sc;
   }
-  int am = (m == bm) ? a : 0x7fffffff;
+  int ga = (m == bm && bm != -INFINITY) ? gidx : 0x7fffffff;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     s += __shfl_xor_sync(0xffffffffu, s, o);
-    tt += __shfl_xor_sync(0xffffffffu, tt, o);
-    am = min(am, __shfl_xor_sync(0xffffffffu, am, o));
+    u += __shfl_xor_sync(0xffffffffu, u, o);
+    ga = min(ga, __shfl_xor_sync(0xffffffffu, ga, o));
   }
-  if (lane_id() == 0) {
-    wsum[0][warp] = s;
-    wsum[1][warp] = tt;
-    warg[warp] = am;
-  }
-  __syncthreads();
-  StatPartial r{-INFINITY, 0.f, 0.f, 0x7fffffff};
-  if (tid == 0) {
-    float rs = 0.f, rt = 0.f;
-    int ra = 0x7fffffff;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) {
-      rs += wsum[0][w];
-      rt += wsum[1][w];
-      ra = min(ra, warg[w]);
-    }
-    r = StatPartial{bm, rs, rt * (1.0f / kLog2e), ra};
-  }
-  __syncthreads();  // the shared arrays are rewritten by the next slice
-  return r;
+  return StatPartial{bm, s, u, ga};
 }
 
-// Statistics, merge and stop test in one launch on a balanced persistent grid.  The rows x segs
-// units (one kSpan-column group each) are cut into gridDim.x contiguous runs of equal length; a
-// CTA streams its run and writes one partial per row piece (a run covers a few rows at most),
-// kept at the piece's first segment together with its length.  A per-row count of finished
-// segments finds the CTA completing the row, which merges the pieces in column order; the last
-// row runs the stop test.  No CTA waits on another; row_units [rows] starts and ends at zero.
-template <typename T, int kLoads>
-__global__ void __launch_bounds__(256, sizeof(T) == 2 ? 5 : 3)
-    sampler_stream_kernel(const T* __restrict__ logits, int32_t segs, SamplerArgs p,
-                          int32_t* __restrict__ row_units, int32_t* __restrict__ piece_len) {
+// Columns per row segment of the streaming sampler: 8 vectors per lane (2048 bf16, 1024 fp32).
+constexpr int kStreamLoads = 8;
+template <typename T>
+constexpr int stream_span() {
+  return kStreamLoads * 32 * (16 / static_cast<int>(sizeof(T)));
+}
+
+// The run of units [floor(w T / W), floor((w + 1) T / W)) belongs to worker w; unit u is worked
+// by the largest w whose run starts at or before u, w(u) = floor(((u + 1) W - 1) / T).  Both
+// floors are taken of an fp64 quotient, exact while the numerator is below 2^53: for a / b with
+// a mod b <= b - 1 the quotient's rounding error (a / b) 2^-53 stays below the gap 1 / b to the
+// next integer.
+DG_DEV long long stream_run_start(long long w, long long workers, long long total) {
+  return static_cast<long long>(floor(static_cast<double>(w * total) / static_cast<double>(workers)));
+}
+DG_DEV long long stream_worker(long long u, long long workers, long long total) {
+  return static_cast<long long>(
+      floor(static_cast<double>((u + 1) * workers - 1) / static_cast<double>(total)));
+}
+
+// Statistics of every row piece in one launch on a persistent grid of warps.  The rows x segs
+// units (one group each) are cut into one contiguous run per warp; a warp streams its run and
+// writes one partial per row piece (a run covers a few rows at most) at the piece's first
+// segment.  No warp waits on another; sampler_stream_rows_kernel merges the rows.
+template <typename T>
+__global__ void __launch_bounds__(256, sizeof(T) == 2 ? 4 : 3)
+    sampler_stream_kernel(const T* __restrict__ logits, int32_t segs, SamplerArgs p) {
   pdl_enter();
   if (block_done(p.state + kStDone)) return;
-  constexpr int kSpan = kLoads * 256 * (16 / static_cast<int>(sizeof(T)));
-  __shared__ int last_piece;
+  constexpr int kSpan = stream_span<T>();
+  const long long workers = static_cast<long long>(gridDim.x) * 8;
+  const long long w = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   const long long total = static_cast<long long>(p.rows) * segs;
-  long long u = blockIdx.x * total / gridDim.x;
-  const long long u_end = (blockIdx.x + 1) * total / gridDim.x;
+  long long u = w * total / workers;
+  const long long u_end = (w + 1) * total / workers;
   while (u < u_end) {
     const int row = static_cast<int>(u / segs);
     const int seg0 = static_cast<int>(u % segs);
     const int len = static_cast<int>(min(u_end, static_cast<long long>(row + 1) * segs) - u);
     const int c0 = seg0 * kSpan;
     const int c1 = min(p.vocab, (seg0 + len) * kSpan);
-    const StatPartial r =
-        stream_slice_stats<T, kLoads>(logits + static_cast<size_t>(row) * p.vocab, c0, c1);
-    const size_t slot = static_cast<size_t>(row) * segs + seg0;
-    if (threadIdx.x == 0) {
-      const_cast<StatPartial*>(p.partials)[slot] = r;
-      piece_len[slot] = len;
-      __threadfence();
-      last_piece = (atomicAdd(row_units + row, len) + len == segs);
-    }
-    __syncthreads();
-    if (last_piece) {
-      __threadfence();
-      if (threadIdx.x == 0) row_units[row] = 0;
-      if (sampler_row_pieces(p, row, segs, piece_len)) sampler_stop_test(p);
-    }
-    __syncthreads();  // last_piece is rewritten by the next piece
+    const StatPartial r = warp_slice_stats<T, kStreamLoads>(
+        logits + static_cast<size_t>(row) * p.vocab, c0, c1);
+    if (lane_id() == 0)
+      const_cast<StatPartial*>(p.partials)[static_cast<size_t>(row) * segs + seg0] = r;
     u += len;
   }
+}
+
+// One warp per row (8 rows per CTA), after sampler_stream_kernel ran with `workers` warps: merge
+// the row's pieces (piece k is the part of worker w_lo + k's run inside the row, k = 0 starting at
+// the row's first segment; an empty run has none), find the first column holding the row maximum
+// in the lowest group reported for it, decide lock / re-noise; the last row to finish runs the
+// stop test.  The loads that do not depend on one another are issued together: the stopped flag,
+// the pieces and the re-noise draw first, the group holding the maximum before the fp64 sums.
+template <typename T>
+__global__ void __launch_bounds__(256) sampler_stream_rows_kernel(const T* __restrict__ logits,
+                                                                  int32_t segs, SamplerArgs p,
+                                                                  long long workers) {
+  pdl_enter();
+  const int row = static_cast<int>(blockIdx.x) * 8 + static_cast<int>(threadIdx.x >> 5);
+  if (row >= p.rows) return;
+  constexpr int kC = 4;
+  constexpr int kVec = 16 / static_cast<int>(sizeof(T));
+  const int lane = static_cast<int>(lane_id());
+  const int stopped = *reinterpret_cast<const volatile int*>(p.state + kStDone);
+  const long long total = static_cast<long long>(p.rows) * segs;
+  const long long r0 = static_cast<long long>(row) * segs;
+  const long long w_lo = stream_worker(r0, workers, total);
+  const long long w_hi = stream_worker(r0 + segs - 1, workers, total);
+  const int n = static_cast<int>(w_hi - w_lo + 1);
+  const float4* part = reinterpret_cast<const float4*>(p.partials) + r0;
+  auto slot_of = [&](int k) -> long long {
+    if (k == 0) return 0;
+    const long long a = stream_run_start(w_lo + k, workers, total);
+    if (w_lo + k < w_hi && a == stream_run_start(w_lo + k + 1, workers, total)) return -1;
+    return a - r0;
+  };
+  float4 q[kC];
+  auto load = [&](int base) {
+#pragma unroll
+    for (int k = 0; k < kC; ++k) {
+      const int i = base + lane + 32 * k;
+      const long long sl = i < n ? slot_of(i) : -1;
+      q[k] = sl >= 0 ? __ldcg(part + sl) : make_float4(-INFINITY, 0.f, 0.f, 0.f);
+    }
+  };
+  const int32_t noise = lane == 0 ? renoise_id(p, row) : 0;
+  // the row maximum and the lowest group holding it
+  float m = -INFINITY;
+  for (int base = 0; base < n; base += 32 * kC) {
+    load(base);
+#pragma unroll
+    for (int k = 0; k < kC; ++k)
+      if (q[k].y > 0.f) m = fmaxf(m, q[k].x);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  int g = 0x7fffffff;
+  for (int base = 0; base < n; base += 32 * kC) {
+    if (n > 32 * kC) load(base);
+#pragma unroll
+    for (int k = 0; k < kC; ++k)
+      if (q[k].y > 0.f && q[k].x == m) g = min(g, __float_as_int(q[k].w));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) g = min(g, __shfl_xor_sync(0xffffffffu, g, o));
+  if (stopped) return;  // uniform over the grid
+  uint4 v[kStreamLoads];
+  if (g != 0x7fffffff)
+    warp_load_group<T, kStreamLoads>(logits + static_cast<size_t>(row) * p.vocab, g, p.vocab, v);
+  // S and U relative to the row maximum while the group is on its way
+  double sum = 0.0, usum = 0.0;
+  if (m != -INFINITY) {
+    for (int base = 0; base < n; base += 32 * kC) {
+      if (n > 32 * kC) load(base);
+#pragma unroll
+      for (int k = 0; k < kC; ++k)
+        if (q[k].y > 0.f) {
+          const double d = static_cast<double>(q[k].x) - static_cast<double>(m);
+          const double e = exp(d);
+          sum += e * q[k].y;
+          usum += e * (static_cast<double>(q[k].z) + d * q[k].y);
+        }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    usum += __shfl_xor_sync(0xffffffffu, usum, o);
+  }
+  int a = 0x7fffffff;
+  if (g != 0x7fffffff) {
+#pragma unroll
+    for (int l = kStreamLoads - 1; l >= 0; --l)
+#pragma unroll
+      for (int j = kVec - 1; j >= 0; --j)
+        if (vec_value<T>(v[l], j) == m) a = g + (l * 32 + lane) * kVec + j;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) a = min(a, __shfl_xor_sync(0xffffffffu, a, o));
+  if (sampler_row_finish(p, row, StatD{static_cast<double>(m), sum, usum, a}, noise))
+    sampler_stop_test(p);
 }
 
 }  // namespace dg

@@ -247,9 +247,11 @@ DG_API int dg_check_device_status(dg_ctx* ctx, void* stream);
 /* ---- standalone operators (the same kernels the context runs) -------------------- */
 
 /* Sampler over given logits ([canvas] step 3): d_logits [rows, V] (dtype), one call per
- * step.  Logits are finite or -inf (a masked vocabulary entry: probability 0, no contribution to
- * the entropy); every row needs at least one finite value.  d_state int32[DG_STATE_WORDS] and the workspace carry the stop test across
- * calls; zero both (dg_sampler_reset) before step 1.  Outputs: d_canvas (next ids),
+ * step, two launches (a streaming pass over the logits, then one warp per row to merge, lock /
+ * re-noise and run the stop test).  Logits are finite or -inf (a masked vocabulary entry:
+ * probability 0, no contribution to the entropy); a logit below -1e30 counts as masked, and every
+ * row needs a logit above -1e30.  d_state int32[DG_STATE_WORDS] and the workspace carry the stop
+ * test across calls; zero both (dg_sampler_reset) before step 1.  Outputs: d_canvas (next ids),
  * d_argmax, d_entropy, d_conf, each [rows].  Requires V % 8 == 0, rows <= 1024. */
 DG_API int dg_sampler_workspace_bytes(int32_t rows, int32_t vocab, size_t* bytes);
 DG_API int dg_sampler_reset(int32_t rows, int32_t vocab, void* d_workspace, int32_t* d_state,

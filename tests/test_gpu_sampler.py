@@ -68,6 +68,33 @@ def test_sampler_exact_ties_take_lowest_index():
     assert int(s.canvas[3]) == 16383  # conf ~ 1 locks
 
 
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_sampler_ties_and_masked_entries_at_lane_and_segment_edges(dtype):
+    """Each warp streams groups of 8 vectors per lane (2048 bf16 / 1024 fp32 columns, one row
+    segment) and finds a lane's first maximal column only at the end, in the group where the lane
+    met its maximum: ties between lanes, within a lane's vector, across a lane's groups and across
+    segment edges must all give the lowest column; -inf (masked) entries contribute nothing."""
+    rows, vocab = 8, 3 * 4096 + 8
+    x = sampler_logits(rows, vocab, seed=11).to(dtype)
+    top = float(x.float().max()) + 4.0
+    x[0, [100, 40]] = top               # two lanes of one group
+    x[1, [8 + 2048, 8]] = top           # one lane meets its maximum again two groups later
+    x[2, [17, 16]] = top                # two maxima in one lane's vector
+    x[3, [2048, 2047]] = top            # bf16 group / segment edge
+    x[4, [1024, 1023]] = top            # fp32 group / segment edge
+    x[5, ::3] = -math.inf               # masked entries around the maximum
+    x[5, 4000] = top
+    x[6, :] = -math.inf                 # only two entries unmasked
+    x[6, 5], x[6, vocab - 1] = 1.0, 2.0
+    x[7, vocab - 8:] = top              # the maximum in the ragged end of the row
+    s = _gpu_sampler(rows, vocab)
+    s.step(x.cuda(), seed=4, block=0, step=1)
+    _check_step(s, x, 4, 0, 1)
+    torch.cuda.synchronize()
+    assert s.argmax.cpu().tolist() == [40, 8, 16, 2047, 1023, 4000, vocab - 1, vocab - 8]
+    assert abs(float(s.conf[6]) - 1.0 / (1.0 + math.exp(-1.0))) < 1e-6
+
+
 def test_sampler_full_size_stats():
     logits = sampler_logits(256, 262144, seed=0)
     s = _gpu_sampler(256, 262144)
