@@ -61,40 +61,75 @@ constexpr int kAttnTile = 16384;  // one 128-row x 128-byte swizzled slab
 constexpr int kAttnSmemBytes = 14 * kAttnTile + 1024 + 256;
 
 constexpr int kAttnThreads = 64 + 32 * 8;
+
+// 2^t for a pair of exponents on the FMA pipe, taking load off the special-function unit (which
+// sets the softmax's pace with two softmax warps per scheduler).  t is clamped to >= -125, rounded
+// to n with the 1.5 * 2^23 addition (n lands in the low mantissa bits), f = t - n in [-1/2, 1/2],
+// 2^f = c0 + c1 f + c2 f^2 + c3 f^3 + c4 f^4, and n is added to the exponent field.  The quartic is
+// a least-squares fit of 2^f on [-1/2, 1/2] weighted towards its largest relative errors: at most
+// 2.7e-6 relative in this fp32 Horner form, so P's bf16 values almost never differ from those of
+// the special-function unit's 2^t.  Valid for t <= 8 (the lazy rescale keeps exponents there);
+// -inf gives 2^-125.
+DG_DEV float2 exp2_fma_pipe(float2 t) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  const float2 tc = make_float2(fmaxf(t.x, -125.0f), fmaxf(t.y, -125.0f));
+  const float2 r = __fadd2_rn(tc, make_float2(kRound, kRound));
+  const float2 n = __fadd2_rn(r, make_float2(-kRound, -kRound));
+  const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), tc);
+  float2 q = __ffma2_rn(make_float2(0.0095701320f, 0.0095701320f), f,
+                        make_float2(0.055918001f, 0.055918001f));
+  q = __ffma2_rn(q, f, make_float2(0.24024744f, 0.24024744f));
+  q = __ffma2_rn(q, f, make_float2(0.69312179f, 0.69312179f));
+  q = __ffma2_rn(q, f, make_float2(0.99999928f, 0.99999928f));
+  // the bits of r are those of 1.5 * 2^23 plus n, and 1.5 * 2^23 shifted by 23 vanishes mod 2^32
+  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(r.x) << 23)),
+                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(r.y) << 23)));
+}
+constexpr int kAttnPolyEvery = 3;  // every third pair of a thread's 64 scores takes exp2_fma_pipe
 constexpr int kMaxAttnSplits = 8;  // the key splits of a query tile form one cluster
 
 // Merge of the key splits of one (token, head) by one warp: O = sum_s 2^(m_s - M) O_s /
 // sum_s 2^(m_s - M) l_s, lane d4 owning dims 4 d4 .. 4 d4 + 3, stored as bf16 into o [T, Hq * 128]
 // (token-major, the O projection's token operand).  Lane s < n_splits reads split s's
-// (max, denominator); the partials of other CTAs are read through L2.
-DG_DEV void attn_merge_row(const AttnParams& p, int n_splits, int tok, int head) {
+// (max, denominator); the partials of other CTAs are read through L2.  In two phases, so that a
+// warp can have the loads of two rows in flight together.
+struct AttnMergeIn {
+  float2 ml;                    // lane s < n_splits: split s's (max, denominator)
+  float4 v[kMaxAttnSplits];     // split s's 4 dims of this lane
+};
+
+DG_DEV void attn_merge_load(const AttnParams& p, int n_splits, int tok, int head, AttnMergeIn& in) {
   const int lane = lane_id();
-  float2 ml = make_float2(-INFINITY, 0.f);
+  in.ml = make_float2(-INFINITY, 0.f);
   if (lane < n_splits)
-    ml = __ldcg(p.ml_part + (static_cast<long long>(lane) * p.n_heads + head) * p.tq + tok);
-  float mmax = ml.x;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mmax = fmaxf(mmax, __shfl_xor_sync(0xffffffffu, mmax, o));
-  const float w_mine = (lane < n_splits && ml.y != 0.f) ? exp2f(ml.x - mmax) : 0.f;
-  float4 v[kMaxAttnSplits];
+    in.ml = __ldcg(p.ml_part + (static_cast<long long>(lane) * p.n_heads + head) * p.tq + tok);
 #pragma unroll
   for (int s = 0; s < kMaxAttnSplits; ++s)
     if (s < n_splits) {
       const long long row = (static_cast<long long>(s) * p.n_heads + head) * p.tq + tok;
-      v[s] = __ldcg(reinterpret_cast<const float4*>(p.o_part + row * 128) + lane);
+      in.v[s] = __ldcg(reinterpret_cast<const float4*>(p.o_part + row * 128) + lane);
     }
+}
+
+DG_DEV void attn_merge_store(const AttnParams& p, int n_splits, int tok, int head,
+                             const AttnMergeIn& in) {
+  const int lane = lane_id();
+  float mmax = in.ml.x;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mmax = fmaxf(mmax, __shfl_xor_sync(0xffffffffu, mmax, o));
+  const float w_mine = (lane < n_splits && in.ml.y != 0.f) ? exp2f(in.ml.x - mmax) : 0.f;
   float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
   float den = 0.f;
 #pragma unroll
   for (int s = 0; s < kMaxAttnSplits; ++s)
     if (s < n_splits) {
       const float w = __shfl_sync(0xffffffffu, w_mine, s);
-      const float l = __shfl_sync(0xffffffffu, ml.y, s);
+      const float l = __shfl_sync(0xffffffffu, in.ml.y, s);
       if (w != 0.f) {
-        num.x += w * v[s].x;
-        num.y += w * v[s].y;
-        num.z += w * v[s].z;
-        num.w += w * v[s].w;
+        num.x += w * in.v[s].x;
+        num.y += w * in.v[s].y;
+        num.z += w * in.v[s].z;
+        num.w += w * in.v[s].w;
         den += w * l;
       }
     }
@@ -342,8 +377,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // probabilities (bf16) of my 64 keys = slab `half` of the P buffer; 16-byte unit u of
       // row r's 128-byte line lands at unit u ^ (r % 8)
       uint8_t* pb = s_p + b * 2 * kAttnTile + half * kAttnTile + (r >> 3) * 1024 + (r & 7) * 128;
-      // e = 2^(x scale log2e - m): a masked key holds x = -inf, so e = 2^-inf = 0 (also when the
-      // whole tile is masked and m is still -inf, m then taken as 0)
+      // e = 2^(x scale log2e - m): a masked key holds x = -inf, so e = 0 on the special-function
+      // unit and 2^-125 on the FMA pipe (also when the whole tile is masked and m is still -inf, m
+      // then taken as 0)
       const float mr = (m_run == -INFINITY) ? 0.f : m_run;
       const float2 sc2 = make_float2(p.scale_log2, p.scale_log2), nm2 = make_float2(-mr, -mr);
       float2 part[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
@@ -351,7 +387,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
       for (int i = 0; i < 64; i += 2) {
         const float2 t = __ffma2_rn(make_float2(x[i], x[i + 1]), sc2, nm2);
-        const float2 e = make_float2(fast_exp2(t.x), fast_exp2(t.y));
+        const float2 e = (i / 2) % kAttnPolyEvery == kAttnPolyEvery - 1
+                             ? exp2_fma_pipe(t)
+                             : make_float2(fast_exp2(t.x), fast_exp2(t.y));
         x[i] = e.x;
         x[i + 1] = e.y;
         part[(i >> 1) & 3] = __fadd2_rn(part[(i >> 1) & 3], e);
@@ -429,9 +467,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   cluster_sync_all();
   const int n_splits = gridDim.z;
   const int r0 = 128 * split / n_splits, r1 = 128 * (split + 1) / n_splits;
-  for (int rr = r0 + warp; rr < r1; rr += kAttnThreads / 32) {
-    const int tok = tok0 + rr;
-    if (tok < p.n_queries) attn_merge_row(p, n_splits, tok, head);
+  constexpr int kWarps = kAttnThreads / 32;
+  for (int rr = r0 + warp; rr < r1; rr += 2 * kWarps) {  // two rows per warp at a time
+    const int rr2 = rr + kWarps;
+    const bool a = tok0 + rr < p.n_queries, b = rr2 < r1 && tok0 + rr2 < p.n_queries;
+    AttnMergeIn in_a, in_b;
+    if (a) attn_merge_load(p, n_splits, tok0 + rr, head, in_a);
+    if (b) attn_merge_load(p, n_splits, tok0 + rr2, head, in_b);
+    if (a) attn_merge_store(p, n_splits, tok0 + rr, head, in_a);
+    if (b) attn_merge_store(p, n_splits, tok0 + rr2, head, in_b);
   }
 }
 
