@@ -451,8 +451,8 @@ def run_ours(args, rank, world, local_rank):
     # (dram__bytes_read.sum + dram__bytes_write.sum of the standalone MoE operator's launches);
     # None for the NVFP4 kernels until they are captured
     traffic = ({} if f4 else
-               {"expert_gate_up": 532844544 + 5702400, "expert_down": 286637312 + 9329920} if f8
-               else {"expert_gate_up": 1063746000 + 4687104, "expert_down": 523752000 + 6922496})
+               {"expert_gate_up": 527095808 + 4883712, "expert_down": 286693632 + 5061632} if f8
+               else {"expert_gate_up": 1052264192 + 5308672, "expert_down": 523554560 + 4555520})
     roof = None
     if args.roofline_kernel in algo and rec:
         achieved = algo[args.roofline_kernel] / (avg_ms / 1e3) / 1e9

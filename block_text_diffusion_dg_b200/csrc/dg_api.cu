@@ -347,6 +347,7 @@ struct ExpertPass {
   int* err;
   const int* done;
   bool profile;  // record under the per-kernel profiling kinds
+  bool x_sh_ready;  // e4m3: x_sh already holds the codes of xn (written by the ffn norm)
 };
 
 // Bytes of one operand row of `cols` values in expert format fmt: bf16 rows are packed, e4m3 and
@@ -409,17 +410,20 @@ int launch_experts(const ExpertPass& e, int sms, cudaStream_t st) {
   const int slab = 64 << e.fmt;  // K elements per 128-byte slab: 64 bf16, 128 e4m3, 256 e2m1
   const long long row_d = operand_row_bytes(e.fmt, e.d);
   const long long row_hs = operand_row_bytes(e.fmt, e.hs);
-  const int kind_g = e.profile ? DG_KERNEL_GATHER : -1;
-  const ExpertPrefetch epf{e.chunks, e.n_chunks, kPrefetchExperts, e.w_gu, 2ll * e.hid * row_d};
+  // bf16 and e4m3: the gate/up GEMM copies each routed row's token (normed bf16, or its e4m3
+  // codes quantised once per token here) straight into its operand tiles; NVFP4 quantises the
+  // routed rows in permuted order with their per-chunk scale atoms (and hints the first experts'
+  // weights into L2, which the router does for the others)
+  const bool quant_x = e.fmt == 2 || (e.fmt == 1 && !e.x_sh_ready);
+  const int kind_g = e.profile && quant_x ? DG_KERNEL_GATHER : -1;
   prof_before(kind_g, st);
-  if (e.fmt != 0) {
+  if (e.fmt == 2) {
+    const ExpertPrefetch epf{e.chunks, e.n_chunks, kPrefetchExperts, e.w_gu, 2ll * e.hid * row_d};
     DG_TRY(launch_quant(e, e.xn, e.d, e.perm, n_slots, e.x_perm, e.x_perm_scale, e.x_sf, e.xn, e.d,
                         shared ? e.n : 0, e.x_sh, e.x_sh_scale, e.x_sh_sf, e.d, e.d, nch, epf, st));
-  } else {
-    DG_TRY(launch_pdl(gather_rows_kernel, dim3(cdiv(n_slots, 4)), dim3(256), 0, st, e.xn, e.perm,
-                      e.k, e.d, n_slots, static_cast<__nv_bfloat16*>(e.x_perm), e.topk_w,
-                      e.w_perm, epf, e.done));
-    DG_LAUNCHED();
+  } else if (e.fmt == 1 && !e.x_sh_ready) {
+    DG_TRY(launch_quant(e, e.xn, e.d, nullptr, e.n, e.x_sh, e.x_sh_scale, nullptr, nullptr, 0, 0,
+                        nullptr, nullptr, nullptr, e.d, e.d, nch, ExpertPrefetch{}, st));
   }
   prof_after(kind_g, st);
 
@@ -442,7 +446,13 @@ int launch_experts(const ExpertPass& e, int sms, cudaStream_t st) {
   p.alt_out_bf16 = e.h_sh;
   p.alt_ld_out = e.hs;
   p.a_scale = e.w_gu_scale;
-  p.b_scale = e.x_perm_scale;
+  p.b_scale = e.fmt == 1 ? e.x_sh_scale : e.x_perm_scale;
+  if (e.fmt != 2) {
+    p.gather_src = static_cast<const uint8_t*>(e.fmt == 1 ? e.x_sh : static_cast<const void*>(e.xn));
+    p.gather_perm = e.perm;
+    p.gather_k = e.k;
+    p.gather_ld = static_cast<int>(row_d);
+  }
   p.alt_a_scale = e.ws_gu_scale;
   p.alt_b_scale = e.x_sh_scale;
   p.a_sf = e.w_gu_sf;
@@ -848,7 +858,7 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
         c->part, d, done));
     DG_LAUNCHED();
     DG_TRY(launch_pdl(residual_norm_kernel<float>, dim3(n), dim3(256), 0, st, c->x, c->part, 1, 0, d, w.ffn_norm, g.eps,
-                                                   static_cast<float*>(c->xn), done));
+                                                   static_cast<float*>(c->xn), nullptr, 0, nullptr, done));
     DG_LAUNCHED();
     }
     if (!(parts & 2)) return DG_OK;
@@ -952,9 +962,13 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     p.x = c->x;
     DG_TRY(launch_cluster<kCluResidual>(c->tm_wo[l], c->tm_o32, p, st, DG_KERNEL_O_PROJ));
     prof_before(DG_KERNEL_RESIDUAL_NORM, st);
+    // with e4m3 experts it also writes the e4m3 codes of its output, the experts' token operand
+    const bool q8 = c->fmt == 1;
     DG_TRY(launch_pdl(residual_norm_kernel<__nv_bfloat16>, dim3(n), dim3(256), 0, st,
                       c->x, c->part, 0, 0ll, d, w.ffn_norm, g.eps,
-                      static_cast<__nv_bfloat16*>(c->xn), done));
+                      static_cast<__nv_bfloat16*>(c->xn),
+                      q8 ? static_cast<uint8_t*>(c->x_sh) : nullptr,
+                      static_cast<int>(operand_row_bytes(1, d)), q8 ? c->x_sh_scale : nullptr, done));
     DG_LAUNCHED();
     prof_after(DG_KERNEL_RESIDUAL_NORM, st);
   }
@@ -970,7 +984,13 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     p.wts = c->topk_w;
     p.top_k = k;
     p.route = RouteArgs{c->topk_ids, n, k, E, route_chunk(c->fmt, n_slots, E), c->offsets,
-                        c->perm, c->chunks, c->n_chunks};
+                        c->perm, c->chunks, c->n_chunks, nullptr, nullptr};
+    if (c->fmt != 2) {  // the gate/up GEMM gathers the rows itself; the routing permutes the weights
+      p.route.wts = c->topk_w;
+      p.route.w_perm = c->w_perm;
+      p.pf_first = w.w_gu;  // the first routed experts' gate/up weights
+      p.pf_first_bytes = kPrefetchExperts * 2ll * g.expert_hidden * operand_row_bytes(c->fmt, d);
+    }
     p.ticket = c->route_ticket;
     DG_TRY(launch_cluster<kCluRouter>(c->tm_wr[l], c->tm_xn32, p, st, DG_KERNEL_ROUTER));
   }
@@ -995,6 +1015,7 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     e.x_perm_scale = c->x_perm_scale;
     e.x_sh = c->x_sh;
     e.x_sh_scale = c->x_sh_scale;
+    e.x_sh_ready = c->fmt == 1;  // the ffn norm wrote the codes
     e.h = static_cast<__nv_bfloat16*>(c->h);
     e.h_sh = static_cast<__nv_bfloat16*>(c->hs);
     e.hq = c->hq;
@@ -1534,12 +1555,15 @@ int dg_debug_layer_part(dg_ctx* ctx, int32_t layer, int32_t part, const float* d
   DG_CUDA(cudaMemcpyAsync(ctx->x, d_x_in, static_cast<size_t>(n) * g.d_model * 4,
                           cudaMemcpyDeviceToDevice, st));
   const float* w = part == 0 ? ctx->layers[layer].attn_norm : ctx->layers[layer].ffn_norm;
+  const bool q8 = part == 1 && ctx->fmt == 1;  // the MoE half's token operand, as in run_layer
   if (ctx->bf16)
-    DG_TRY(launch_pdl(residual_norm_kernel<__nv_bfloat16>, dim3(n), dim3(256), 0, st, 
-        ctx->x, ctx->part, 0, 0, g.d_model, w, g.eps, static_cast<__nv_bfloat16*>(ctx->xn), nullptr));
+    DG_TRY(launch_pdl(residual_norm_kernel<__nv_bfloat16>, dim3(n), dim3(256), 0, st,
+        ctx->x, ctx->part, 0, 0, g.d_model, w, g.eps, static_cast<__nv_bfloat16*>(ctx->xn),
+        q8 ? static_cast<uint8_t*>(ctx->x_sh) : nullptr,
+        static_cast<int>(operand_row_bytes(1, g.d_model)), q8 ? ctx->x_sh_scale : nullptr, nullptr));
   else
     DG_TRY(launch_pdl(residual_norm_kernel<float>, dim3(n), dim3(256), 0, st, ctx->x, ctx->part, 0, 0, g.d_model, w, g.eps,
-                                                   static_cast<float*>(ctx->xn), nullptr));
+                                                   static_cast<float*>(ctx->xn), nullptr, 0, nullptr, nullptr));
   DG_LAUNCHED();
   const float* nn = (layer + 1 < g.n_layers) ? ctx->layers[layer + 1].attn_norm : ctx->final_norm;
   DG_TRY(run_layer(ctx, layer, n, ctx->kv_len, causal, nn, nullptr, st, part == 0 ? 1 : 2, 0,
@@ -1581,11 +1605,12 @@ int dg_debug_layer(dg_ctx* ctx, int32_t layer, const float* d_x_in, float* d_x_o
                           cudaMemcpyDeviceToDevice, st));
   const float* w = ctx->layers[layer].attn_norm;
   if (ctx->bf16)
-    DG_TRY(launch_pdl(residual_norm_kernel<__nv_bfloat16>, dim3(n), dim3(256), 0, st, 
-        ctx->x, ctx->part, 0, 0, g.d_model, w, g.eps, static_cast<__nv_bfloat16*>(ctx->xn), nullptr));
+    DG_TRY(launch_pdl(residual_norm_kernel<__nv_bfloat16>, dim3(n), dim3(256), 0, st,
+        ctx->x, ctx->part, 0, 0, g.d_model, w, g.eps, static_cast<__nv_bfloat16*>(ctx->xn),
+        nullptr, 0, nullptr, nullptr));
   else
     DG_TRY(launch_pdl(residual_norm_kernel<float>, dim3(n), dim3(256), 0, st, ctx->x, ctx->part, 0, 0, g.d_model, w, g.eps,
-                                                   static_cast<float*>(ctx->xn), nullptr));
+                                                   static_cast<float*>(ctx->xn), nullptr, 0, nullptr, nullptr));
   DG_LAUNCHED();
   const float* nn = (layer + 1 < g.n_layers) ? ctx->layers[layer + 1].attn_norm : ctx->final_norm;
   DG_TRY(run_layer(ctx, layer, n, ctx->kv_len, causal, nn, nullptr, st, 3, 0, seq_len));
@@ -1897,7 +1922,13 @@ int moe_ffn_impl(int fmt, const MoeScales& sc, const void* d_x, const float* d_r
   pr.top_k = top_k;
   pr.route = RouteArgs{ids, t, top_k, n_experts,
                        route_chunk(fmt, static_cast<long long>(t) * top_k, n_experts), offs,
-                       perm, chunks, icnt};
+                       perm, chunks, icnt, nullptr, nullptr};
+  if (fmt != 2) {  // the gate/up GEMM gathers the rows itself; the routing permutes the weights
+    pr.route.wts = wts;
+    pr.route.w_perm = static_cast<float*>(at(M_WPERM));
+    pr.pf_first = d_w_gu;
+    pr.pf_first_bytes = kPrefetchExperts * 2ll * hidden * operand_row_bytes(fmt, d);
+  }
   pr.ticket = route_ticket;
   DG_TRY(launch_cluster<kCluRouter>(t_wr, t_x32, pr, st, -1));
   ExpertPass e{};

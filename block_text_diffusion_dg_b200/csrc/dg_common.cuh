@@ -5,6 +5,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -127,6 +128,20 @@ DG_DEV void prefetch_l2_slice(const void* base, long long bytes, int part, int p
   const uint8_t* b = static_cast<const uint8_t*>(base);
   for (long long o = lo; o < hi; o += 65536)
     prefetch_l2_bulk(b + o, static_cast<uint32_t>(min(65536ll, hi - o)));
+}
+
+// 16-byte asynchronous copy global -> shared, bypassing L1; src_bytes < 16 fills the rest of the
+// 16 bytes with zeros (0: no global read at all, src only has to be a valid address).
+DG_DEV void cp_async_16(uint32_t dst_smem, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst_smem), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+// An arrival on the mbarrier once every cp.async this thread issued so far has landed; it counts
+// as one of the barrier's expected arrivals (no increment of the pending count).
+DG_DEV void cp_async_mbar_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
 }
 
 // Order generic-proxy shared-memory writes before async-proxy (UMMA/TMA) reads.
@@ -361,6 +376,14 @@ DG_DEV float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
+}
+
+// e4m3: the largest finite magnitude, and two values converted (round to nearest even,
+// saturating to +-448) and packed little-endian, `a` in the low byte.
+constexpr float kE4m3Max = 448.0f;
+DG_DEV uint32_t e4m3x2(float a, float b) {
+  return static_cast<uint32_t>(
+      __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3));
 }
 
 // 2^x on the special-function unit (approximate, flushes denormals).

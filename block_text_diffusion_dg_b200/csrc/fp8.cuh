@@ -20,8 +20,6 @@
 
 namespace dg {
 
-constexpr float kE4m3Max = 448.0f;
-
 struct QuantSeg {
   const __nv_bfloat16* src;
   long long ld_src;     // elements between source rows
@@ -43,12 +41,6 @@ struct QuantJob {
 
 DG_DEV float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
 DG_DEV float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
-
-// Two codes packed little-endian: `a` in the low byte.
-DG_DEV uint32_t e4m3x2(float a, float b) {
-  return static_cast<uint32_t>(
-      __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3));
-}
 
 // One warp quantises one row of `cols` bf16 values (16-byte vectors, cols % 8 == 0) into a
 // destination row of `pitch` bytes (pitch % 8 == 0), zero past the codes.

@@ -75,6 +75,14 @@ struct GemmParams {
   const uint8_t* b_sf;
   const uint8_t* alt_a_sf;
   const uint8_t* alt_b_sf;
+  // routed items that read their token rows straight from the unpermuted tokens (gather_src
+  // non-null): B row j of a routed chunk is token gather_perm[b_row + j] / gather_k, its K slab
+  // kb the 128 bytes at gather_src + token * gather_ld + 128 kb; the producer warp copies them
+  // with cp.async (the alternate group keeps its TMA loads)
+  const uint8_t* gather_src;
+  const int* gather_perm;
+  int gather_k;
+  int gather_ld;
   int* err;
   const int* done;
 };
@@ -153,7 +161,11 @@ struct GemmCfg {
   static_assert(kTmemUsed <= 512, "TMEM");
   // epilogue warps: two per TMEM lane quarter for wide token tiles (they split the columns)
   static constexpr int kEpiWarps = MAXN >= 128 ? 8 : 4;
-  static constexpr int kThreads = 64 + 32 * kEpiWarps;
+  // + the gather warps after the epilogue warps (idle unless the launch gathers token rows):
+  // 16-byte units per gather thread and stage, at most MAXN rows x 8 units over their threads
+  static constexpr int kGatherWarps = 4;
+  static constexpr int kGatherPer = MAXN * 8 / (32 * kGatherWarps);
+  static constexpr int kThreads = 64 + 32 * kEpiWarps + 32 * kGatherWarps;
   static constexpr int kSmemBytes = STAGES * kStageBytes + 1024 + 256;
   static_assert(MAXN % 32 == 0 && MAXN >= 32 && MAXN <= 256, "MAXN");
 };
@@ -234,10 +246,12 @@ __global__ void __launch_bounds__(GemmCfg<MAXN, STAGES, FMT>::kThreads, 1)
   uint64_t* acc_empty = acc_full + C::kAccBufs;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_empty + C::kAccBufs);
   const int warp = threadIdx.x >> 5;
+  // gathered token rows: every producer lane signals its copies on the stage's full barrier
+  const bool gather = FMT != 2 && p.gather_src != nullptr;
 
   if (warp == 0 && lane_id() == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], gather ? 1 + 32 * C::kGatherWarps : 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < C::kAccBufs; ++b) {
@@ -281,8 +295,10 @@ __global__ void __launch_bounds__(GemmCfg<MAXN, STAGES, FMT>::kThreads, 1)
       for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
         const GemmItem w = wn;
         if (it + static_cast<int>(gridDim.x) < n_items) wn = gemm_item(p, it + gridDim.x);
+        const bool gat = gather && !w.alt;  // B rows come from the gather warp
         const int nbox = (w.n + 31) >> 5;
-        const uint32_t bytes = C::kABytes + nbox * 32 * 128 + C::kSfaBytes + C::kSfbBytes;
+        const uint32_t bytes =
+            C::kABytes + (gat ? 0 : nbox * 32 * 128) + C::kSfaBytes + C::kSfbBytes;
         const CUtensorMap* ta = w.alt ? &tm_a2 : &tm_a;
         const CUtensorMap* tb = w.alt ? &tm_b2 : &tm_b;
         for (int kb = w.kb0; kb < w.kb1; ++kb) {
@@ -295,8 +311,9 @@ __global__ void __launch_bounds__(GemmCfg<MAXN, STAGES, FMT>::kThreads, 1)
           mbar_arrive_expect_tx(&full[stage], bytes);
           const int kx = kb * (FMT != 0 ? 128 : 64);  // map columns per 128-byte slab
           tma_load_2d(ta, &full[stage], sa, kx, w.a_row, pol_a);
-          for (int bx = 0; bx < nbox; ++bx)
-            tma_load_2d(tb, &full[stage], sb + bx * 4096, kx, w.b_row + bx * 32, pol_b);
+          if (!gat)
+            for (int bx = 0; bx < nbox; ++bx)
+              tma_load_2d(tb, &full[stage], sb + bx * 4096, kx, w.b_row + bx * 32, pol_b);
           if constexpr (FMT == 2) {
             // the slab's scale atoms: A by 128-row tile, B by chunk (4 per slab, padded)
             const int kt = w.alt ? p.alt_kb_total : p.kb_total;
@@ -338,6 +355,9 @@ __global__ void __launch_bounds__(GemmCfg<MAXN, STAGES, FMT>::kThreads, 1)
             ok = false;
             break;
           }
+          // token rows written by the producer lanes' cp.async (generic proxy) before the UMMA
+          // reads them through the async proxy
+          if (gather) fence_proxy_async_smem();
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + stage * C::kStageBytes);
           const uint64_t da = sdesc_sw128(sa);
@@ -374,6 +394,66 @@ __global__ void __launch_bounds__(GemmCfg<MAXN, STAGES, FMT>::kThreads, 1)
         if (++acc == C::kAccBufs) {
           acc = 0;
           acc_phase ^= 1u;
+        }
+      }
+    }
+  } else if (warp >= 2 + C::kEpiWarps) {
+    // the gather warps: with gathered token rows they fill B of every routed item's stages.
+    // Gather thread g copies 16-byte units g, g + 128, ...: row j = unit / 8 of the item, its
+    // piece u = unit % 8 landing at the swizzled 128-byte line of row j (destinations fixed for
+    // the kernel, sources per item: token perm[b_row + j] / k, zero fill past the item's rows).
+    // Every thread signals its copies on the stage's full barrier, for the alternate group's
+    // stages too (none pending); like the TMA producer each warp first waits for the stage to
+    // be free, which keeps the arrivals in step with the stage's uses.
+    if (gather) {
+      constexpr int kPer = C::kGatherPer;
+      constexpr uint32_t kSkip = 0xffffffffu, kZero = 0xfffffffeu;
+      const int lane = static_cast<int>(lane_id());
+      const int gt = (warp - 2 - C::kEpiWarps) * 32 + lane;
+      uint32_t dst_off[kPer];
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) {
+        const int c = gt + 32 * C::kGatherWarps * i, row = c >> 3, u = c & 7;
+        dst_off[i] = (row >> 3) * 1024 + (row & 7) * 128 + ((u ^ (row & 7)) << 4);
+      }
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+        const GemmItem w = gemm_item(p, it);
+        const bool gat = !w.alt;
+        const int npad = (w.n + 15) & ~15;  // B rows the UMMA reads
+        uint32_t src_off[kPer];
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+          const int c = gt + 32 * C::kGatherWarps * i, row = c >> 3, u = c & 7;
+          src_off[i] = !gat || row >= npad ? kSkip
+                       : row >= w.n        ? kZero
+                                           : static_cast<uint32_t>(__ldg(p.gather_perm + w.b_row + row) /
+                                                                   p.gather_k) *
+                                                     static_cast<uint32_t>(p.gather_ld) +
+                                                 u * 16;
+        }
+        for (int kb = w.kb0; kb < w.kb1; ++kb) {
+          int ready = 1;
+          if (lane == 0) ready = mbar_wait(&empty[stage], phase ^ 1u, p.err) ? 1 : 0;
+          if (!__shfl_sync(0xffffffffu, ready, 0)) {
+            ok = false;
+            break;
+          }
+          const uint32_t sbase = smem_u32(smem + stage * C::kStageBytes + C::kABytes);
+          const uint8_t* src = p.gather_src + kb * 128;
+#pragma unroll
+          for (int i = 0; i < kPer; ++i)
+            if (src_off[i] != kSkip) {
+              const bool real = src_off[i] != kZero;
+              cp_async_16(sbase + dst_off[i], real ? src + src_off[i] : p.gather_src, real ? 16u : 0u);
+            }
+          cp_async_mbar_arrive(&full[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
         }
       }
     }
@@ -418,7 +498,9 @@ __global__ void __launch_bounds__(GemmCfg<MAXN, STAGES, FMT>::kThreads, 1)
 #pragma unroll
         for (int cc = 0; cc < MAXN / 32; ++cc) {
           const int j = cc * 32 + lane_id();
-          tok_scale[cc] = j < w.n ? bs[w.b_row + j] : 0.0f;
+          tok_scale[cc] = j < w.n ? bs[gather && !w.alt ? __ldcg(p.gather_perm + w.b_row + j) / p.gather_k
+                                                      : w.b_row + j]
+                                  : 0.0f;
         }
       }
       if (!mbar_wait(&acc_full[acc], acc_phase, p.err)) break;

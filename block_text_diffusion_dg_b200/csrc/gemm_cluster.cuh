@@ -67,6 +67,8 @@ struct CluParams {
   int top_k;
   RouteArgs route;
   int32_t* ticket;          // starts and ends at zero
+  const void* pf_first;     // hinted into L2 by the CTAs that do not route (null: none)
+  long long pf_first_bytes;
   int* err;
   const int* done;
 };
@@ -394,6 +396,10 @@ __global__ void __launch_bounds__(kCluThreads, 1)
       __threadfence();
       if (tid == 0) *p.ticket = 0;
       route_canvas(p.route, reinterpret_cast<int*>(smem));
+    } else if (tid == 0) {
+      // the others hint the weights the grouped GEMM streams first into L2 (its items go in
+      // expert order, and a canvas' 2,048 slots leave hardly any expert empty)
+      prefetch_l2_slice(p.pf_first, p.pf_first_bytes, blockIdx.x, gridDim.x);
     }
   }
   tc_fence_before();

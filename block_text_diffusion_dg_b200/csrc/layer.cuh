@@ -9,8 +9,9 @@
 //   router_topk_*     router logits -> top-k ids (lowest index on ties) and the softmax of
 //                     the selected logits (= renormalised full-softmax probabilities) (a6)
 //   route_canvas      per-expert token bitmasks -> offsets, stable slot order, the token-chunk
-//                     list of the grouped GEMMs (run by the router kernel's last CTA)  (a7)
-//   gather_rows       x_perm[p] = xn2[token of slot perm[p]]                   (a7)
+//                     list of the grouped GEMMs, the route weights in permuted order (run by
+//                     the router kernel's last CTA); the bf16 / e4m3 gate/up GEMM then copies
+//                     each routed row's token itself                                   (a7)
 //   moe_combine_norm  x += sum over slots in order of y_slot + y_shared; xn = rmsnorm(x) * w
 //                     for the next layer (or the final norm)                  (a9, a2)
 // RMSNorm is x / sqrt(mean(x^2) + eps) * w (pre-norm, the Gemma-style plain reading).
@@ -28,6 +29,18 @@ DG_DEV float block_sum_256(float v, float* sm) {
   float t = 0.f;
 #pragma unroll
   for (int w = 0; w < 8; ++w) t += sm[w];
+  __syncthreads();
+  return t;
+}
+
+DG_DEV float block_max_256(float v, float* sm) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  if (lane_id() == 0) sm[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float t = sm[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) t = fmaxf(t, sm[w]);
   __syncthreads();
   return t;
 }
@@ -154,6 +167,8 @@ __global__ void __launch_bounds__(256) residual_norm_kernel(float* __restrict__ 
                                                             int splits, long long split_stride,
                                                             int d, const float* __restrict__ w,
                                                             float eps, TA* __restrict__ xn,
+                                                            uint8_t* __restrict__ q_codes,
+                                                            int q_pitch, float* __restrict__ q_scale,
                                                             const int* done) {
   pdl_enter();
   if (block_done(done)) return;
@@ -179,16 +194,43 @@ __global__ void __launch_bounds__(256) residual_norm_kernel(float* __restrict__ 
     }
   }
   const float inv = rsqrtf(block_sum_256(ss, sm) / d + eps);
+  float amax = 0.f;
 #pragma unroll
   for (int j = 0; j < kNormVec; ++j) {
     const int i = threadIdx.x + j * 256;
     if (i < nv) {
       const float4 g = reinterpret_cast<const float4*>(w)[i];
-      store4<TA>(xn + static_cast<long long>(t) * d + 4 * i,
-                 make_float4(v[j].x * inv * g.x, v[j].y * inv * g.y, v[j].z * inv * g.z,
-                             v[j].w * inv * g.w));
+      float4 y = make_float4(v[j].x * inv * g.x, v[j].y * inv * g.y, v[j].z * inv * g.z,
+                             v[j].w * inv * g.w);
+      store4<TA>(xn + static_cast<long long>(t) * d + 4 * i, y);
+      if (q_codes) {  // the stored (bf16-rounded) values are the ones quantised
+        y = make_float4(__bfloat162float(__float2bfloat16_rn(y.x)),
+                        __bfloat162float(__float2bfloat16_rn(y.y)),
+                        __bfloat162float(__float2bfloat16_rn(y.z)),
+                        __bfloat162float(__float2bfloat16_rn(y.w)));
+        amax = fmaxf(fmaxf(amax, fmaxf(fabsf(y.x), fabsf(y.y))), fmaxf(fabsf(y.z), fabsf(y.w)));
+      }
+      v[j] = y;
     }
   }
+  if (q_codes == nullptr) return;
+  // e4m3 codes of the row as quant_rows_kernel makes them: scale = max|row| / 448 (IEEE division),
+  // codes = e4m3_rn_satfinite(x / scale), all zero for a zero row; the row's pitch padding zero
+  const float sc = __fdiv_rn(block_max_256(amax, sm), kE4m3Max);
+  if (threadIdx.x == 0) q_scale[t] = sc;
+  uint8_t* qr = q_codes + static_cast<long long>(t) * q_pitch;
+#pragma unroll
+  for (int j = 0; j < kNormVec; ++j) {
+    const int i = threadIdx.x + j * 256;
+    if (i < nv) {
+      const uint32_t c =
+          sc > 0.f ? e4m3x2(__fdiv_rn(v[j].x, sc), __fdiv_rn(v[j].y, sc)) |
+                         (e4m3x2(__fdiv_rn(v[j].z, sc), __fdiv_rn(v[j].w, sc)) << 16)
+                   : 0u;
+      reinterpret_cast<uint32_t*>(qr)[i] = c;
+    }
+  }
+  for (int i = nv + threadIdx.x; i < (q_pitch >> 2); i += 256) reinterpret_cast<uint32_t*>(qr)[i] = 0u;
 }
 
 // Top-k of one token's router logits held by one warp; E <= 256 and E % 4 == 0, k <= 8.  Lane
@@ -284,6 +326,8 @@ struct RouteArgs {
   int32_t* perm;       // [n_slots] permuted row -> slot
   int4* chunks;        // [max chunks] (expert, first permuted row, tokens, 0) in expert order
   int32_t* n_chunks;   // [1] chunks in use
+  const float* wts;    // optional: route weights by slot, written to w_perm by permuted row
+  float* w_perm;
 };
 
 constexpr int kRouteMaxTokens = 4096;
@@ -386,6 +430,7 @@ DG_DEV void route_canvas(const RouteArgs& a, int* sm) {
         const int rank = prefix[e[b] * words + w] +
                          __popc(mask[e[b] * words + w] & ((1u << (t & 31)) - 1u));
         a.perm[off_s[e[b]] + rank] = s;
+        if (a.w_perm) a.w_perm[off_s[e[b]] + rank] = __ldcg(a.wts + s);
       }
     }
   }
@@ -395,8 +440,9 @@ DG_DEV void route_canvas(const RouteArgs& a, int* sm) {
                                            min(a.n_chunk, count_s[e] - c * a.n_chunk), 0);
 }
 
-// Weights of the first routed chunks' experts, prefetched into L2 by the gather (the grouped
-// GEMM reads them first): chunk c < n_first of the chunk list, `expert_bytes` per expert at w.
+// Weights of the first routed chunks' experts, prefetched into L2 by the NVFP4 quantiser of the
+// routed rows (the grouped GEMM reads them first): chunk c < n_first of the chunk list,
+// `expert_bytes` per expert at w.
 struct ExpertPrefetch {
   const int4* chunks;
   const int* n_chunks;
@@ -404,37 +450,6 @@ struct ExpertPrefetch {
   const void* w;
   long long expert_bytes;
 };
-
-// x_perm[p] = xn[perm[p] / k] and w_perm[p] = topk_w[perm[p]] (the route weight in permuted
-// order, which the down GEMM's scatter reads by permuted row); 64 threads per permuted row, 4
-// rows per CTA, 16-byte copies.
-__global__ void __launch_bounds__(256) gather_rows_kernel(const __nv_bfloat16* __restrict__ xn,
-                                                          const int32_t* __restrict__ perm,
-                                                          int top_k, int d, int n_rows,
-                                                          __nv_bfloat16* __restrict__ x_perm,
-                                                          const float* __restrict__ topk_w,
-                                                          float* __restrict__ w_perm,
-                                                          ExpertPrefetch pf, const int* done) {
-  pdl_enter();
-  if (block_done(done)) return;
-  if (threadIdx.x == 0 && pf.w != nullptr && pf.n_first > 0) {
-    const int nf = min(pf.n_first, *pf.n_chunks);
-    if (nf > 0 && static_cast<int>(gridDim.x) >= nf) {
-      const int c = blockIdx.x % nf, parts = gridDim.x / nf, part = blockIdx.x / nf;
-      if (part < parts)
-        prefetch_l2_slice(static_cast<const uint8_t*>(pf.w) + pf.chunks[c].x * pf.expert_bytes,
-                          pf.expert_bytes, part, parts);
-    }
-  }
-  const int p = blockIdx.x * 4 + (threadIdx.x >> 6);
-  if (p >= n_rows) return;
-  const int slot = perm[p];
-  if ((threadIdx.x & 63) == 0) w_perm[p] = topk_w[slot];
-  const int t = slot / top_k;
-  const uint4* src = reinterpret_cast<const uint4*>(xn + static_cast<long long>(t) * d);
-  uint4* dst = reinterpret_cast<uint4*>(x_perm + static_cast<long long>(p) * d);
-  for (int i = threadIdx.x & 63; i < d / 8; i += 64) dst[i] = src[i];
-}
 
 // x += sum over slots s = 0..k-1 (in order) of y_slot[t*k + s] + y_shared[t]; then, when w is
 // given, xn = rmsnorm(x) * w for the next layer (or the final norm).  One CTA per token.
