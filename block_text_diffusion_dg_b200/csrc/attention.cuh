@@ -8,11 +8,13 @@
 // group's heads (row = head * Tq + token), so every K/V tile is used by all of them.
 // Roles: warp 0 TMA (Q once, then K and V^T tiles of 128 keys through separate 2-deep rings:
 // a K slot frees as soon as its S = Q K^T is done, so K runs one tile ahead of V),
-// warp 1 UMMA (S = Q K^T into one of two TMEM buffers, then O += P V), warps 2-9 softmax:
-// two threads per query row, each owning 64 of the tile's 128 keys (the partners sit in
-// different warps of the same TMEM lane quarter and trade their partial row maxima through a
-// spare TMEM column); exp2 with the scale folded in, P written to shared memory in the UMMA's
-// 128-byte swizzled K-major layout.  O lives in TMEM for the whole key range;
+// warp 1 UMMA (S = Q K^T into one of two TMEM buffers, then O += P V with P read from TMEM),
+// warps 2-9 softmax: two threads per query row, each owning 64 of the tile's 128 keys (the
+// partners sit in different warps of the same TMEM lane quarter and trade their partial row
+// maxima through a spare TMEM column); exp2 with the scale folded in, P (bf16 pairs) written
+// over the first 64 columns of the S buffer it came from (both partners have read their S by
+// the exchange barrier, and the next S into that buffer is issued after this tile's P V, the
+// UMMAs running in order).  O lives in TMEM for the whole key range;
 // its running maximum is only moved (and O rescaled) when a new tile raises the row max by
 // more than 2^8, otherwise exponents relative to the stale maximum stay below 256.
 // Each split writes its unnormalised O, its max and its denominator; the splits of a query tile
@@ -57,8 +59,8 @@ struct AttnParams {
 };
 
 constexpr int kAttnTile = 16384;  // one 128-row x 128-byte swizzled slab
-// Q (2 slabs) + K,V^T ring (2 stages x 4 slabs) + P (2 buffers x 2 slabs) + barriers
-constexpr int kAttnSmemBytes = 14 * kAttnTile + 1024 + 256;
+// Q (2 slabs) + K,V^T ring (2 stages x 4 slabs) + barriers
+constexpr int kAttnSmemBytes = 10 * kAttnTile + 1024 + 256;
 
 constexpr int kAttnThreads = 64 + 32 * 8;
 
@@ -150,16 +152,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint8_t* s_q = smem;                   // slabs: hd 0-63, hd 64-127
   uint8_t* s_k = smem + 2 * kAttnTile;   // K stage s: 2 slabs (hd 0-63, 64-127)
   uint8_t* s_v = s_k + 4 * kAttnTile;    // V^T stage s: 2 slabs (keys 0-63, 64-127)
-  uint8_t* s_p = s_v + 4 * kAttnTile;    // P buffer b: 2 slabs (keys 0-63, 64-127)
-  uint64_t* bars = reinterpret_cast<uint64_t*>(s_p + 4 * kAttnTile);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s_v + 4 * kAttnTile);
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;    // [2] per K stage
   uint64_t* k_empty = bars + 3;   // [2] (S = Q K^T of that stage completed)
   uint64_t* v_full = bars + 5;    // [2] per V stage
   uint64_t* v_empty = bars + 7;   // [2] (P V of that stage completed)
   uint64_t* s_full = bars + 9;    // [2] per S buffer
-  uint64_t* p_full = bars + 11;   // [2] per P buffer
-  uint64_t* pv_done = bars + 13;  // [2] per P buffer (P V of that buffer completed)
+  uint64_t* p_full = bars + 11;   // [2] per S buffer (its P written)
+  uint64_t* pv_done = bars + 13;  // [2] per S buffer (P V of its P completed)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 15);
 
   const int warp = threadIdx.x >> 5;
@@ -280,13 +281,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (!mbar_wait(&p_full[b], (j >> 1) & 1, p.err)) break;
         if (!mbar_wait(&v_full[b], (j >> 1) & 1, p.err)) break;
         tc_fence_after();
-        const uint32_t a_p = smem_u32(s_p + b * 2 * kAttnTile);
         const uint32_t a_v = smem_u32(s_v + b * 2 * kAttnTile);
+        const uint32_t p_tmem = tmem_base + 128 + b * 128;  // P over the S buffer's first columns
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const uint32_t off = (k >> 2) * kAttnTile;
-          umma_bf16(tmem_base, sdesc_sw128(a_p + off) + 2 * (k & 3),
-                    sdesc_sw128(a_v + off) + 2 * (k & 3), idesc, (j > 0 || k > 0) ? 1u : 0u);
+          umma_bf16_ts(tmem_base, p_tmem + 8 * k, sdesc_sw128(a_v + off) + 2 * (k & 3), idesc,
+                       (j > 0 || k > 0) ? 1u : 0u);
         }
         umma_commit(&pv_done[b]);
         umma_commit(&v_empty[b]);
@@ -368,15 +369,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           tmem_st32(oa, v);
         }
       }
-      // the P buffer of this tile was last read by P V of tile j - 2
       const int b = j & 1;
-      if (j >= 2)
-        ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[b], ((j - 2) >> 1) & 1, p.err));
-      if (!ok) continue;
-      tc_fence_after();
-      // probabilities (bf16) of my 64 keys = slab `half` of the P buffer; 16-byte unit u of
-      // row r's 128-byte line lands at unit u ^ (r % 8)
-      uint8_t* pb = s_p + b * 2 * kAttnTile + half * kAttnTile + (r >> 3) * 1024 + (r & 7) * 128;
       // e = 2^(x scale log2e - m): a masked key holds x = -inf, so e = 0 on the special-function
       // unit and 2^-125 on the FMA pipe (also when the whole tile is masked and m is still -inf, m
       // then taken as 0)
@@ -394,20 +387,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         x[i + 1] = e.y;
         part[(i >> 1) & 3] = __fadd2_rn(part[(i >> 1) & 3], e);
       }
+      // probabilities (bf16 pairs) of my 64 keys into TMEM columns 32 half .. 32 half + 31 of
+      // the S buffer (keys 2c, 2c + 1 of my half in column c)
+      {
+        float pk[32];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        uint32_t pk[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const __nv_bfloat162 h2 = __floats2bfloat162_rn(x[u * 8 + 2 * q], x[u * 8 + 2 * q + 1]);
-          pk[q] = *reinterpret_cast<const uint32_t*>(&h2);
+        for (int c = 0; c < 32; ++c) {
+          const __nv_bfloat162 h2 = __floats2bfloat162_rn(x[2 * c], x[2 * c + 1]);
+          pk[c] = __uint_as_float(*reinterpret_cast<const uint32_t*>(&h2));
         }
-        *reinterpret_cast<uint4*>(pb + ((u ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        tmem_st32(tmem_base + 128 + b * 128 + 32 * half + lane_off, pk);
       }
       const float2 ps = __fadd2_rn(__fadd2_rn(part[0], part[1]), __fadd2_rn(part[2], part[3]));
       const float rowsum = ps.x + ps.y;
       l_run = l_run * alpha + rowsum;
-      fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&p_full[b]);
     }
