@@ -964,8 +964,9 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
     prof_before(DG_KERNEL_RESIDUAL_NORM, st);
     // with e4m3 experts it also writes the e4m3 codes of its output, the experts' token operand
     const bool q8 = c->fmt == 1;
-    DG_TRY(launch_pdl(residual_norm_kernel<__nv_bfloat16>, dim3(n), dim3(256), 0, st,
-                      c->x, c->part, 0, 0ll, d, w.ffn_norm, g.eps,
+    DG_TRY(launch_pdl(q8 ? residual_norm_kernel<__nv_bfloat16, true>
+                         : residual_norm_kernel<__nv_bfloat16, false>,
+                      dim3(n), dim3(256), 0, st, c->x, c->part, 0, 0ll, d, w.ffn_norm, g.eps,
                       static_cast<__nv_bfloat16*>(c->xn),
                       q8 ? static_cast<uint8_t*>(c->x_sh) : nullptr,
                       static_cast<int>(operand_row_bytes(1, d)), q8 ? c->x_sh_scale : nullptr, done));
@@ -1557,7 +1558,8 @@ int dg_debug_layer_part(dg_ctx* ctx, int32_t layer, int32_t part, const float* d
   const float* w = part == 0 ? ctx->layers[layer].attn_norm : ctx->layers[layer].ffn_norm;
   const bool q8 = part == 1 && ctx->fmt == 1;  // the MoE half's token operand, as in run_layer
   if (ctx->bf16)
-    DG_TRY(launch_pdl(residual_norm_kernel<__nv_bfloat16>, dim3(n), dim3(256), 0, st,
+    DG_TRY(launch_pdl(q8 ? residual_norm_kernel<__nv_bfloat16, true>
+                         : residual_norm_kernel<__nv_bfloat16, false>, dim3(n), dim3(256), 0, st,
         ctx->x, ctx->part, 0, 0, g.d_model, w, g.eps, static_cast<__nv_bfloat16*>(ctx->xn),
         q8 ? static_cast<uint8_t*>(ctx->x_sh) : nullptr,
         static_cast<int>(operand_row_bytes(1, g.d_model)), q8 ? ctx->x_sh_scale : nullptr, nullptr));

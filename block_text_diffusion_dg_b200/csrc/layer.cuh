@@ -161,7 +161,7 @@ __global__ void __launch_bounds__(128) qkv_finalize_kernel(
 // x += sum of split partials (0 splits: x unchanged); xn = rmsnorm(x) * w.  One CTA per token,
 // float4 columns, d % 4 == 0 and d <= 4 * 256 * kNormVec.
 constexpr int kNormVec = 4;
-template <typename TA>
+template <typename TA, bool kQ8 = false>
 __global__ void __launch_bounds__(256) residual_norm_kernel(float* __restrict__ x,
                                                             const float* __restrict__ part,
                                                             int splits, long long split_stride,
@@ -203,7 +203,7 @@ __global__ void __launch_bounds__(256) residual_norm_kernel(float* __restrict__ 
       float4 y = make_float4(v[j].x * inv * g.x, v[j].y * inv * g.y, v[j].z * inv * g.z,
                              v[j].w * inv * g.w);
       store4<TA>(xn + static_cast<long long>(t) * d + 4 * i, y);
-      if (q_codes) {  // the stored (bf16-rounded) values are the ones quantised
+      if constexpr (kQ8) {  // the stored (bf16-rounded) values are the ones quantised
         y = make_float4(__bfloat162float(__float2bfloat16_rn(y.x)),
                         __bfloat162float(__float2bfloat16_rn(y.y)),
                         __bfloat162float(__float2bfloat16_rn(y.z)),
@@ -213,7 +213,7 @@ __global__ void __launch_bounds__(256) residual_norm_kernel(float* __restrict__ 
       v[j] = y;
     }
   }
-  if (q_codes == nullptr) return;
+  if constexpr (!kQ8) return;
   // e4m3 codes of the row as quant_rows_kernel makes them: scale = max|row| / 448 (IEEE division),
   // codes = e4m3_rn_satfinite(x / scale), all zero for a zero row; the row's pitch padding zero
   const float sc = __fdiv_rn(block_max_256(amax, sm), kE4m3Max);
