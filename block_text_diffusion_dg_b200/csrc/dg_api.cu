@@ -410,20 +410,32 @@ int launch_experts(const ExpertPass& e, int sms, cudaStream_t st) {
   const int slab = 64 << e.fmt;  // K elements per 128-byte slab: 64 bf16, 128 e4m3, 256 e2m1
   const long long row_d = operand_row_bytes(e.fmt, e.d);
   const long long row_hs = operand_row_bytes(e.fmt, e.hs);
-  // bf16 and e4m3: the gate/up GEMM copies each routed row's token (normed bf16, or its e4m3
-  // codes quantised once per token here) straight into its operand tiles; NVFP4 quantises the
-  // routed rows in permuted order with their per-chunk scale atoms (and hints the first experts'
-  // weights into L2, which the router does for the others)
-  const bool quant_x = e.fmt == 2 || (e.fmt == 1 && !e.x_sh_ready);
-  const int kind_g = e.profile && quant_x ? DG_KERNEL_GATHER : -1;
+  // bf16 and e4m3 with 64-token chunks (decode): the gate/up GEMM copies each routed row's token
+  // (normed bf16, or its e4m3 codes quantised once per token) straight into its operand tiles.
+  // Wider chunks (prefill, batched canvases) read a permuted copy by TMA boxes instead: there a
+  // gather thread would issue 8-16 copies per stage.  NVFP4 quantises the routed rows in
+  // permuted order with their per-chunk scale atoms (and hints the first experts' weights into
+  // L2, which the router does for the others).
+  const bool gemm_gather = e.fmt != 2 && nch == kGroupN;
+  const int sh_rows = shared && !e.x_sh_ready ? e.n : 0;  // e4m3 tokens for the shared expert
+  const bool launch_g = e.fmt == 2 || !gemm_gather || (e.fmt == 1 && !e.x_sh_ready);
+  const int kind_g = e.profile && launch_g ? DG_KERNEL_GATHER : -1;
   prof_before(kind_g, st);
   if (e.fmt == 2) {
     const ExpertPrefetch epf{e.chunks, e.n_chunks, kPrefetchExperts, e.w_gu, 2ll * e.hid * row_d};
     DG_TRY(launch_quant(e, e.xn, e.d, e.perm, n_slots, e.x_perm, e.x_perm_scale, e.x_sf, e.xn, e.d,
                         shared ? e.n : 0, e.x_sh, e.x_sh_scale, e.x_sh_sf, e.d, e.d, nch, epf, st));
-  } else if (e.fmt == 1 && !e.x_sh_ready) {
-    DG_TRY(launch_quant(e, e.xn, e.d, nullptr, e.n, e.x_sh, e.x_sh_scale, nullptr, nullptr, 0, 0,
-                        nullptr, nullptr, nullptr, e.d, e.d, nch, ExpertPrefetch{}, st));
+  } else if (e.fmt == 1 && gemm_gather) {
+    if (!e.x_sh_ready)
+      DG_TRY(launch_quant(e, e.xn, e.d, nullptr, e.n, e.x_sh, e.x_sh_scale, nullptr, nullptr, 0, 0,
+                          nullptr, nullptr, nullptr, e.d, e.d, nch, ExpertPrefetch{}, st));
+  } else if (e.fmt == 1) {
+    DG_TRY(launch_quant(e, e.xn, e.d, e.perm, n_slots, e.x_perm, e.x_perm_scale, nullptr, e.xn, e.d,
+                        sh_rows, e.x_sh, e.x_sh_scale, nullptr, e.d, e.d, nch, ExpertPrefetch{}, st));
+  } else if (!gemm_gather) {
+    DG_TRY(launch_pdl(gather_rows_kernel, dim3(cdiv(n_slots, 4)), dim3(256), 0, st, e.xn, e.perm,
+                      e.k, e.d, n_slots, static_cast<__nv_bfloat16*>(e.x_perm), e.done));
+    DG_LAUNCHED();
   }
   prof_after(kind_g, st);
 
@@ -446,8 +458,8 @@ int launch_experts(const ExpertPass& e, int sms, cudaStream_t st) {
   p.alt_out_bf16 = e.h_sh;
   p.alt_ld_out = e.hs;
   p.a_scale = e.w_gu_scale;
-  p.b_scale = e.fmt == 1 ? e.x_sh_scale : e.x_perm_scale;
-  if (e.fmt != 2) {
+  p.b_scale = e.fmt == 1 && gemm_gather ? e.x_sh_scale : e.x_perm_scale;
+  if (gemm_gather) {
     p.gather_src = static_cast<const uint8_t*>(e.fmt == 1 ? e.x_sh : static_cast<const void*>(e.xn));
     p.gather_perm = e.perm;
     p.gather_k = e.k;

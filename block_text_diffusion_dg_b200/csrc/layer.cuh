@@ -11,7 +11,8 @@
 //   route_canvas      per-expert token bitmasks -> offsets, stable slot order, the token-chunk
 //                     list of the grouped GEMMs, the route weights in permuted order (run by
 //                     the router kernel's last CTA); the bf16 / e4m3 gate/up GEMM then copies
-//                     each routed row's token itself                                   (a7)
+//                     each routed row's token itself (64-token chunks)                  (a7)
+//   gather_rows       x_perm[p] = xn[perm[p] / k] for the wide-chunk passes           (a7)
 //   moe_combine_norm  x += sum over slots in order of y_slot + y_shared; xn = rmsnorm(x) * w
 //                     for the next layer (or the final norm)                  (a9, a2)
 // RMSNorm is x / sqrt(mean(x^2) + eps) * w (pre-norm, the Gemma-style plain reading).
@@ -450,6 +451,23 @@ struct ExpertPrefetch {
   const void* w;
   long long expert_bytes;
 };
+
+// x_perm[p] = xn[perm[p] / k]: the routed rows in permuted order for the passes whose grouped
+// GEMM reads them by TMA boxes (wide token chunks); 64 threads per row, 4 rows per CTA, 16-byte
+// copies.
+__global__ void __launch_bounds__(256) gather_rows_kernel(const __nv_bfloat16* __restrict__ xn,
+                                                          const int32_t* __restrict__ perm,
+                                                          int top_k, int d, int n_rows,
+                                                          __nv_bfloat16* __restrict__ x_perm,
+                                                          const int* done) {
+  pdl_enter();
+  if (block_done(done)) return;
+  const int row = blockIdx.x * 4 + (threadIdx.x >> 6);
+  if (row >= n_rows) return;
+  const uint4* src = reinterpret_cast<const uint4*>(xn + static_cast<long long>(perm[row] / top_k) * d);
+  uint4* dst = reinterpret_cast<uint4*>(x_perm + static_cast<long long>(row) * d);
+  for (int i = threadIdx.x & 63; i < d / 8; i += 64) dst[i] = src[i];
+}
 
 // x += sum over slots s = 0..k-1 (in order) of y_slot[t*k + s] + y_shared[t]; then, when w is
 // given, xn = rmsnorm(x) * w for the next layer (or the final norm).  One CTA per token.
