@@ -219,6 +219,9 @@ int group_chunk(long long n_slots, int n_experts) {
 }
 constexpr int kRouterChunk = 64;  // tokens per router cluster
 constexpr int kPrefetchExperts = 4;  // routed chunks whose expert weights the gather prefetches
+// Decode layers: routed experts whose gate/up weights the router's CTAs that do not route hint into
+// L2 (about 48 MB in bf16) while HBM is idle; 8 or 10 slowed the router more than they saved.
+constexpr int kRouterPrefetchExperts = 6;
 
 // ta2/tb2 are read only by items of the alternate group (p.alt_group >= 0).
 template <int MAXN, int STAGES, int EPI, int FMT = 0>
@@ -1002,7 +1005,7 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
       p.route.wts = c->topk_w;
       p.route.w_perm = c->w_perm;
       p.pf_first = w.w_gu;  // the first routed experts' gate/up weights
-      p.pf_first_bytes = kPrefetchExperts * 2ll * g.expert_hidden * operand_row_bytes(c->fmt, d);
+      p.pf_first_bytes = kRouterPrefetchExperts * 2ll * g.expert_hidden * operand_row_bytes(c->fmt, d);
     }
     p.ticket = c->route_ticket;
     DG_TRY(launch_cluster<kCluRouter>(c->tm_wr[l], c->tm_xn32, p, st, DG_KERNEL_ROUTER));
