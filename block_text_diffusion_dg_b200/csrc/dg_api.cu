@@ -1005,7 +1005,8 @@ int run_layer(dg_ctx* c, int l, int n, int pos0, int causal, const float* next_n
       p.route.wts = c->topk_w;
       p.route.w_perm = c->w_perm;
       p.pf_first = w.w_gu;  // the first routed experts' gate/up weights
-      p.pf_first_bytes = kRouterPrefetchExperts * 2ll * g.expert_hidden * operand_row_bytes(c->fmt, d);
+      p.pf_first_bytes = std::min(kRouterPrefetchExperts, E) * 2ll * g.expert_hidden *
+                         operand_row_bytes(c->fmt, d);
     }
     p.ticket = c->route_ticket;
     DG_TRY(launch_cluster<kCluRouter>(c->tm_wr[l], c->tm_xn32, p, st, DG_KERNEL_ROUTER));
@@ -1944,7 +1945,7 @@ int moe_ffn_impl(int fmt, const MoeScales& sc, const void* d_x, const float* d_r
     pr.route.wts = wts;
     pr.route.w_perm = static_cast<float*>(at(M_WPERM));
     pr.pf_first = d_w_gu;
-    pr.pf_first_bytes = kPrefetchExperts * 2ll * hidden * operand_row_bytes(fmt, d);
+    pr.pf_first_bytes = std::min(kPrefetchExperts, n_experts) * 2ll * hidden * operand_row_bytes(fmt, d);
   }
   pr.ticket = route_ticket;
   DG_TRY(launch_cluster<kCluRouter>(t_wr, t_x32, pr, st, -1));
