@@ -645,13 +645,16 @@ template <typename T>
 __global__ void __launch_bounds__(256) sampler_stream_rows_kernel(const T* __restrict__ logits,
                                                                   int32_t segs, SamplerArgs p,
                                                                   long long workers) {
-  pdl_enter();
   const int row = static_cast<int>(blockIdx.x) * 8 + static_cast<int>(threadIdx.x >> 5);
-  if (row >= p.rows) return;
+  if (row >= p.rows) {
+    pdl_enter();
+    return;
+  }
   constexpr int kC = 4;
   constexpr int kVec = 16 / static_cast<int>(sizeof(T));
   const int lane = static_cast<int>(lane_id());
-  const int stopped = *reinterpret_cast<const volatile int*>(p.state + kStDone);
+  // what depends on the arguments alone (the pieces' slots from the static split, the re-noise
+  // draw) is worked out while the streaming kernel finishes
   const long long total = static_cast<long long>(p.rows) * segs;
   const long long r0 = static_cast<long long>(row) * segs;
   const long long w_lo = stream_worker(r0, workers, total);
@@ -664,16 +667,24 @@ __global__ void __launch_bounds__(256) sampler_stream_rows_kernel(const T* __res
     if (w_lo + k < w_hi && a == stream_run_start(w_lo + k + 1, workers, total)) return -1;
     return a - r0;
   };
+  long long slot0[kC];  // the slots of the first pass
+#pragma unroll
+  for (int k = 0; k < kC; ++k) {
+    const int i = lane + 32 * k;
+    slot0[k] = i < n ? slot_of(i) : -1;
+  }
+  const int32_t noise = lane == 0 ? renoise_id(p, row) : 0;
+  pdl_enter();
+  const int stopped = *reinterpret_cast<const volatile int*>(p.state + kStDone);
   float4 q[kC];
   auto load = [&](int base) {
 #pragma unroll
     for (int k = 0; k < kC; ++k) {
       const int i = base + lane + 32 * k;
-      const long long sl = i < n ? slot_of(i) : -1;
+      const long long sl = base == 0 ? slot0[k] : (i < n ? slot_of(i) : -1);
       q[k] = sl >= 0 ? __ldcg(part + sl) : make_float4(-INFINITY, 0.f, 0.f, 0.f);
     }
   };
-  const int32_t noise = lane == 0 ? renoise_id(p, row) : 0;
   // the row maximum and the lowest group holding it
   float m = -INFINITY;
   for (int base = 0; base < n; base += 32 * kC) {
