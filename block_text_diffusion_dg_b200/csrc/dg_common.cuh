@@ -352,30 +352,6 @@ DG_DEV float tmem_ld1(uint32_t taddr) {
   return __uint_as_float(r);
 }
 
-// Packed fp32 pairs (sm_100 f32x2 arithmetic): a.x/a.y in one 64-bit register.
-DG_DEV float2 ffma2(float2 a, float2 b, float2 c) {
-  uint64_t r;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;"
-      : "=l"(r)
-      : "l"(*reinterpret_cast<const uint64_t*>(&a)), "l"(*reinterpret_cast<const uint64_t*>(&b)),
-        "l"(*reinterpret_cast<const uint64_t*>(&c)));
-  return *reinterpret_cast<const float2*>(&r);
-}
-DG_DEV float2 fmul2(float2 a, float2 b) {
-  uint64_t r;
-  asm("mul.rn.f32x2 %0, %1, %2;"
-      : "=l"(r)
-      : "l"(*reinterpret_cast<const uint64_t*>(&a)), "l"(*reinterpret_cast<const uint64_t*>(&b)));
-  return *reinterpret_cast<const float2*>(&r);
-}
-DG_DEV float2 fadd2(float2 a, float2 b) {
-  uint64_t r;
-  asm("add.rn.f32x2 %0, %1, %2;"
-      : "=l"(r)
-      : "l"(*reinterpret_cast<const uint64_t*>(&a)), "l"(*reinterpret_cast<const uint64_t*>(&b)));
-  return *reinterpret_cast<const float2*>(&r);
-}
-
 // Barrier over `count` threads (whole warps) on hardware barrier `id` (1..15).
 DG_DEV void named_barrier(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
@@ -426,8 +402,6 @@ DG_DEV void tmem_st32(uint32_t taddr, const float (&v)[32]) {
 
 // ---------------------------------------------------------------------------------------
 // small numeric helpers
-DG_DEV float bf16_to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
-DG_DEV __nv_bfloat16 f32_to_bf16(float x) { return __float2bfloat16_rn(x); }
 
 template <typename T>
 DG_DEV float load_as_f32(const T* p, size_t i);
